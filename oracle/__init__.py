@@ -1,0 +1,260 @@
+"""Python access to the CPU oracle (oracle.c) for the INT8 quantized-training
+Linear layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package; the CUDA library and its
+binding never do.  Every function takes and returns numpy arrays and does
+argument marshalling only; all arithmetic is in oracle.c, whose comments cite
+the passages each step follows.
+
+Status values are bit masks with the same bit positions as the library's
+device status word (``1 << code``): ARG 1<<1, SHAPE 1<<2, ZERO_ROW 1<<4,
+NONFINITE 1<<5, UNSUPPORTED 1<<6.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+BIT_ARG = 1 << 1
+BIT_SHAPE = 1 << 2
+BIT_ZERO_ROW = 1 << 4
+BIT_NONFINITE = 1 << 5
+BIT_UNSUPPORTED = 1 << 6
+REJECT_ZERO_ROWS = 1
+MAX_CONTRACTION = 131071
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(_build.build())
+        _declare(_lib)
+    return _lib
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_U32 = ctypes.c_uint32
+_U64 = ctypes.c_uint64
+_F = ctypes.c_float
+
+
+def _declare(L):
+    sigs = {
+        "ref_hadamard_scale": (_F, [ctypes.c_int]),
+        "ref_hadamard_rows": (_U32, [_P, _I64, _P, _I64, _I64, _I64, ctypes.c_int]),
+        "ref_hadamard_matrix_f64": (None, [ctypes.c_int, _P]),
+        "ref_quantize_rows": (_U32, [_P, _I64, _I64, _I64, _P, ctypes.c_int, _U32, _P, _I64, _P]),
+        "ref_gemm_nt": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
+        "ref_gemm_nn": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
+        "ref_gemm_tn": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
+        "ref_fwd": (_U32, [_P, _I64, _I64, _P, _P, _I64, _P, ctypes.c_int, _P, _P, _P]),
+        "ref_bwd_prep_rows": (_U32, [_P, _I64, _I64, _P, _P, _P]),
+        "ref_bwd_prep_cols": (_U32, [_P, _I64, _I64, _P, _P, _P, _P]),
+        "ref_bwd_dx": (_U32, [_P, _I64, _I64, _P, _P, _I64, ctypes.c_int, _P, _P, _P]),
+        "ref_bwd_dw": (_U32, [_P, _I64, _I64, _P, _P, _I64, _P, _P, _P, _P]),
+        "ref_philox4x32_10": (None, [_P, _P, _P]),
+        "ref_sr_u24": (_U32, [_U64, _U64, _U64]),
+        "ref_update_sr": (_U32, [_P, _P, _P, _I64, _I64, ctypes.c_int, _F, _F, _F, _F, _F,
+                                 _P, _P, _U64, _U64, _P, _P, _P]),
+        "ref_update_float": (_U32, [_P, _P, _P, _I64, _I64, ctypes.c_int, _F, _F, _F, _F, _F,
+                                    _P, _P, _U64, _P, _P, _P, _P]),
+        "ref_sr_expectation_enum": (ctypes.c_double, [_F]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _i8(a):
+    return np.ascontiguousarray(a, dtype=np.int8)
+
+
+# ---------------------------------------------------------------- rotation
+def hadamard_scale(B: int) -> float:
+    return float(lib().ref_hadamard_scale(B))
+
+
+def hadamard_rows(x: np.ndarray, B: int):
+    x = _f32(x)
+    rows, cols = x.shape
+    y = np.empty_like(x)
+    st = lib().ref_hadamard_rows(_p(x), cols, _p(y), cols, rows, cols, B)
+    return y, st
+
+
+def hadamard_matrix(B: int) -> np.ndarray:
+    R = np.empty((B, B), np.float64)
+    lib().ref_hadamard_matrix_f64(B, _p(R))
+    return R
+
+
+# ---------------------------------------------------------------- quantize
+def quantize_rows(x: np.ndarray, B: int = 0, col_scale=None, flags: int = 0):
+    x = _f32(x)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), np.int8)
+    s = np.empty((rows,), np.float32)
+    cs = None if col_scale is None else _f32(col_scale)
+    st = lib().ref_quantize_rows(_p(x), rows, cols, cols, _p(cs), B, flags, _p(q), cols, _p(s))
+    return q, s, st
+
+
+# ---------------------------------------------------------------- GEMMs
+def gemm_nt(A: np.ndarray, B: np.ndarray):
+    """out[m,n] = sum_c A[m,c] B[n,c] (int32), status."""
+    A, B = _i8(A), _i8(B)
+    M, C = A.shape
+    N = B.shape[0]
+    out = np.empty((M, N), np.int32)
+    st = lib().ref_gemm_nt(_p(A), C, _p(B), C, M, N, C, _p(out), N)
+    return out, st
+
+
+def gemm_nn(A: np.ndarray, B: np.ndarray):
+    """out[m,n] = sum_c A[m,c] B[c,n] (int32), status."""
+    A, B = _i8(A), _i8(B)
+    M, C = A.shape
+    N = B.shape[1]
+    out = np.empty((M, N), np.int32)
+    st = lib().ref_gemm_nn(_p(A), C, _p(B), N, M, N, C, _p(out), N)
+    return out, st
+
+
+def gemm_tn(A: np.ndarray, B: np.ndarray):
+    """out[m,n] = sum_c A[c,m] B[c,n] (int32), status."""
+    A, B = _i8(A), _i8(B)
+    C, M = A.shape
+    N = B.shape[1]
+    out = np.empty((M, N), np.int32)
+    st = lib().ref_gemm_tn(_p(A), M, _p(B), N, M, N, C, _p(out), N)
+    return out, st
+
+
+# ---------------------------------------------------------------- layer
+def fwd(x, wq, sw, bias=None, B: int = 0):
+    """Returns y (fp32 [M,N]), X_q, s_x, status."""
+    x, wq, sw = _f32(x), _i8(wq), _f32(sw)
+    M, K = x.shape
+    N = wq.shape[0]
+    b = None if bias is None else _f32(bias)
+    y = np.empty((M, N), np.float32)
+    xq = np.empty((M, K), np.int8)
+    sx = np.empty((M,), np.float32)
+    st = lib().ref_fwd(_p(x), M, K, _p(wq), _p(sw), N, _p(b), B, _p(y), _p(xq), _p(sx))
+    return y, xq, sx, st
+
+
+def bwd_prep_rows(dy, sw):
+    dy, sw = _f32(dy), _f32(sw)
+    M, N = dy.shape
+    q = np.empty((M, N), np.int8)
+    s1 = np.empty((M,), np.float32)
+    st = lib().ref_bwd_prep_rows(_p(dy), M, N, _p(sw), _p(q), _p(s1))
+    return q, s1, st
+
+
+def bwd_prep_cols(dy, sx):
+    dy, sx = _f32(dy), _f32(sx)
+    M, N = dy.shape
+    q = np.empty((M, N), np.int8)
+    s2 = np.empty((N,), np.float32)
+    db = np.empty((N,), np.float32)
+    st = lib().ref_bwd_prep_cols(_p(dy), M, N, _p(sx), _p(q), _p(s2), _p(db))
+    return q, s2, db, st
+
+
+def bwd_dx(dy, wq, sw, B: int = 0):
+    """Returns dX (fp32 [M,K]), dYq_r, s1, status."""
+    dy, wq, sw = _f32(dy), _i8(wq), _f32(sw)
+    M, N = dy.shape
+    K = wq.shape[1]
+    dx = np.empty((M, K), np.float32)
+    q = np.empty((M, N), np.int8)
+    s1 = np.empty((M,), np.float32)
+    st = lib().ref_bwd_dx(_p(dy), M, N, _p(wq), _p(sw), K, B, _p(dx), _p(q), _p(s1))
+    return dx, q, s1, st
+
+
+def bwd_dw(dy, xq, sx):
+    """Returns dW (fp32 [N,K]), db, dYq_c, s2, status."""
+    dy, xq, sx = _f32(dy), _i8(xq), _f32(sx)
+    M, N = dy.shape
+    K = xq.shape[1]
+    dw = np.empty((N, K), np.float32)
+    db = np.empty((N,), np.float32)
+    q = np.empty((M, N), np.int8)
+    s2 = np.empty((N,), np.float32)
+    st = lib().ref_bwd_dw(_p(dy), M, N, _p(xq), _p(sx), K, _p(dw), _p(db), _p(q), _p(s2))
+    return dw, db, q, s2, st
+
+
+# ---------------------------------------------------------------- RNG / update
+def philox4x32_10(ctr, key):
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.empty(4, np.uint32)
+    lib().ref_philox4x32_10(_p(c), _p(k), _p(out))
+    return out
+
+
+def sr_u24(seed: int, step: int, e: int) -> int:
+    return int(lib().ref_sr_u24(seed, step, e))
+
+
+def sr_expectation_enum(v: float) -> float:
+    return float(lib().ref_sr_expectation_enum(v))
+
+
+SGD, ADAMW = 0, 1
+
+
+def update_sr(q, s, grad, kind: int, lr: float, seed: int, step: int,
+              m=None, v=None, b1=0.9, b2=0.999, eps=1e-8, wd=0.0,
+              g=None, g_m=None, g_v=None):
+    """One optimizer step with stochastic requantization; returns the new
+    (q, s, m, v, g, g_m, g_v, status) as copies (inputs are not modified)."""
+    q, s, grad = _i8(q).copy(), _f32(s).copy(), _f32(grad)
+    N, K = q.shape
+    m = None if m is None else _f32(m).copy()
+    v = None if v is None else _f32(v).copy()
+    g = None if g is None else _f32(g).copy()
+    g_m = None if g_m is None else _f32(g_m).copy()
+    g_v = None if g_v is None else _f32(g_v).copy()
+    st = lib().ref_update_sr(_p(q), _p(s), _p(grad), N, K, kind, lr, b1, b2, eps, wd,
+                             _p(m), _p(v), seed, step, _p(g), _p(g_m), _p(g_v))
+    return q, s, m, v, g, g_m, g_v, st
+
+
+def update_float(q, s, grad, kind: int, lr: float, step: int,
+                 m=None, v=None, b1=0.9, b2=0.999, eps=1e-8, wd=0.0,
+                 g=None, g_m=None, g_v=None):
+    """The optimizer step alone, without requantization; returns the updated
+    float weights (or directions) [N,K] and the new (m, v, g, g_m, g_v), status."""
+    q, s, grad = _i8(q), _f32(s), _f32(grad)
+    N, K = q.shape
+    m = None if m is None else _f32(m).copy()
+    v = None if v is None else _f32(v).copy()
+    g = None if g is None else _f32(g).copy()
+    g_m = None if g_m is None else _f32(g_m).copy()
+    g_v = None if g_v is None else _f32(g_v).copy()
+    w = np.empty((N, K), np.float32)
+    st = lib().ref_update_float(_p(q), _p(s), _p(grad), N, K, kind, lr, b1, b2, eps, wd,
+                                _p(m), _p(v), step, _p(g), _p(g_m), _p(g_v), _p(w))
+    return w, m, v, g, g_m, g_v, st

@@ -1,0 +1,532 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself:
+values printed on the pages, closed forms, library routines (scipy's
+Hadamard matrix, numpy integer matmul, numpy's round-half-even, cuRAND's
+host Philox4x32-10, torch.optim and torch autograd), brute force on tiny
+inputs, and invariants of the method.  CPU only.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_constants.txt")
+
+
+def golden() -> dict:
+    out = {}
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        name, value = line.split("|")[0].split()
+        out[name] = value
+    return out
+
+
+# --------------------------------------------------------------------------
+# Block-Hadamard rotation
+# --------------------------------------------------------------------------
+
+def _rotation_fp32(B: int) -> np.ndarray:
+    R, st = oracle.hadamard_rows(np.eye(B, dtype=np.float32), B)
+    assert st == 0
+    return R
+
+
+def test_orthogonality_matches_page_value():
+    """OneTrainer PR #1681 item 3 prints 5.96e-08 for the fp32 buffer; the
+    spec bound is 1e-7 for every block size."""
+    page = float(golden()["hadamard_orthogonality_fp32_B128"])
+    R = torch.from_numpy(_rotation_fp32(128))
+    err = (R @ R.T - torch.eye(128)).abs().max().item()
+    assert f"{err:.2e}" == f"{page:.2e}"
+    for B in (2, 4, 8, 16, 32, 64, 128, 256):
+        R = torch.from_numpy(_rotation_fp32(B)).double()
+        assert (R @ R.T - torch.eye(B, dtype=torch.float64)).abs().max().item() <= 1e-7
+
+
+@pytest.mark.parametrize("B", [2, 4, 8, 16, 32, 64, 128, 256])
+def test_fwht_equals_sylvester_matrix(B):
+    """The butterfly form equals x @ H_B / sqrt(B), H_B from scipy (Sylvester)."""
+    x = workloads.normal((5, 3 * B), 1.0, 100 + B)
+    y, st = oracle.hadamard_rows(x, B)
+    assert st == 0
+    H = scipy.linalg.hadamard(B).astype(np.float64) / math.sqrt(B)
+    ref = np.concatenate([x[:, i * B:(i + 1) * B].astype(np.float64) @ H for i in range(3)], 1)
+    assert np.abs(y - ref).max() <= 1e-5 * max(1.0, np.abs(ref).max())
+    Rd = oracle.hadamard_matrix(B)
+    assert np.array_equal(Rd, H)
+
+
+def test_fwht_is_an_involution():
+    """H_B / sqrt(B) is symmetric and orthogonal, so applying it twice is I."""
+    x = workloads.normal((7, 512), 1.0, 7)
+    for B in (2, 16, 128, 256):
+        y, _ = oracle.hadamard_rows(x, B)
+        z, _ = oracle.hadamard_rows(y, B)
+        assert np.abs(z - x).max() <= 1e-5
+
+
+def test_rotation_identity_rotating_x_not_unrotating_w():
+    """(xR)(WR)^T == x W^T  (OneTrainer PR #1681 item 2 / Summary b)."""
+    x = workloads.normal((16, 384), 1.0, 1)
+    W = workloads.normal((24, 384), 0.02, 2)
+    xr, _ = oracle.hadamard_rows(x, 128)
+    wr, _ = oracle.hadamard_rows(W, 128)
+    lhs = xr.astype(np.float64) @ wr.astype(np.float64).T
+    rhs = x.astype(np.float64) @ W.astype(np.float64).T
+    assert np.linalg.norm(lhs - rhs) / np.linalg.norm(rhs) <= 1e-6
+
+
+def test_hadamard_rejects_bad_blocks():
+    x = np.zeros((2, 96), np.float32)
+    assert oracle.hadamard_rows(x, 64)[1] == oracle.BIT_SHAPE  # 96 % 64 != 0
+    assert oracle.hadamard_rows(x, 3)[1] == oracle.BIT_SHAPE
+    assert oracle.quantize_rows(x, B=3)[2] == oracle.BIT_ARG
+    assert oracle.quantize_rows(x, B=512)[2] == oracle.BIT_ARG
+    assert oracle.quantize_rows(x, B=64)[2] == oracle.BIT_SHAPE
+
+
+# --------------------------------------------------------------------------
+# Per-row INT8 quantization
+# --------------------------------------------------------------------------
+
+def test_quant_exact_multiples_round_trip():
+    """Rows s0*q with s0 a power of two and max |q| = 127 quantize to q, s0."""
+    rng = np.random.Generator(np.random.PCG64(3))
+    q = rng.integers(-127, 128, size=(9, 64)).astype(np.int8)
+    q[:, 5] = np.where(np.arange(9) % 2 == 0, 127, -127)
+    s0 = (2.0 ** -rng.integers(0, 12, size=9)).astype(np.float32)
+    x = q.astype(np.float32) * s0[:, None]
+    qq, s, st = oracle.quantize_rows(x)
+    assert st == 0
+    assert np.array_equal(qq, q)
+    assert np.array_equal(s, s0)
+
+
+def test_quant_ties_round_to_even():
+    """With amax = 127 the codes are numpy's round-half-to-even of x."""
+    vals = np.array([127.0, -127.0, 2.5, 3.5, -2.5, -3.5, 0.5, -0.5, 1.5, 126.5,
+                     -126.5, 4.4999995, 0.0, 64.5, 65.5, -1.5], np.float32)
+    x = np.tile(vals, (2, 1))
+    q, s, st = oracle.quantize_rows(x)
+    assert st == 0 and np.all(s == np.float32(1.0))
+    assert np.array_equal(q[0], np.rint(vals).astype(np.int8))
+
+
+def test_quant_error_bound_and_extremes():
+    """|t - s q| <= s/2 (+1 ulp), the amax element maps to +-127, |q| <= 127,
+    signs agree, and s = amax / 127."""
+    d = workloads.tiny_layer()
+    for x in (d["x"], d["w"], workloads.normal((33, 512), 3.0, 9)):
+        q, s, st = oracle.quantize_rows(x)
+        assert st == 0
+        amax = np.abs(x).max(1)
+        assert np.array_equal(s, (amax / np.float32(127)).astype(np.float32))
+        err = np.abs(x.astype(np.float64) - q.astype(np.float64) * s[:, None])
+        assert np.all(err <= s[:, None].astype(np.float64) * (0.5 + 1e-6))
+        idx = np.abs(x).argmax(1)
+        assert np.array_equal(np.abs(q[np.arange(len(q)), idx]), np.full(len(q), 127, np.int8))
+        assert np.abs(q.astype(np.int32)).max() <= 127
+        assert np.all((np.sign(q) == np.sign(x)) | (q == 0))
+
+
+def test_quant_zero_rows():
+    """Zero rows: s = 0, codes 0; flagged only when the caller rejects them
+    (zero directions are rejected, masked rows are legal)."""
+    x = workloads.normal((4, 32), 1.0, 4)
+    x[2] = 0.0
+    q, s, st = oracle.quantize_rows(x)
+    assert st == 0 and s[2] == 0 and not q[2].any()
+    q2, s2, st2 = oracle.quantize_rows(x, flags=oracle.REJECT_ZERO_ROWS)
+    assert st2 == oracle.BIT_ZERO_ROW
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+def test_quant_nonfinite_flag():
+    x = workloads.normal((3, 32), 1.0, 5)
+    x[1, 7] = np.nan
+    assert oracle.quantize_rows(x)[2] & oracle.BIT_NONFINITE
+    x[1, 7] = np.inf
+    assert oracle.quantize_rows(x)[2] & oracle.BIT_NONFINITE
+
+
+def test_quant_composes_with_col_scale_and_rotation():
+    x = workloads.normal((6, 256), 1.0, 6)
+    c = workloads.uniform((256,), 0.1, 3.0, 7)
+    a = oracle.quantize_rows(x, col_scale=c)
+    b = oracle.quantize_rows(x * c)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    xr, _ = oracle.hadamard_rows(x, 64)
+    a = oracle.quantize_rows(x, B=64)
+    b = oracle.quantize_rows(xr)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# --------------------------------------------------------------------------
+# Integer GEMMs
+# --------------------------------------------------------------------------
+
+def _brute(A, B, M, N, C, a_at, b_at):
+    out = [[0] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            out[m][n] = sum(int(a_at(A, m, c)) * int(b_at(B, n, c)) for c in range(C))
+    return np.array(out, dtype=np.int64)
+
+
+def test_gemm_brute_force_tiny():
+    rng = np.random.Generator(np.random.PCG64(11))
+    M, N, C = 3, 5, 7
+    A = rng.integers(-127, 128, size=(M, C)).astype(np.int8)
+    Bt = rng.integers(-127, 128, size=(N, C)).astype(np.int8)
+    out, st = oracle.gemm_nt(A, Bt)
+    assert st == 0
+    assert np.array_equal(out, _brute(A, Bt, M, N, C, lambda a, m, c: a[m, c], lambda b, n, c: b[n, c]))
+    Bn = rng.integers(-127, 128, size=(C, N)).astype(np.int8)
+    out, st = oracle.gemm_nn(A, Bn)
+    assert np.array_equal(out, _brute(A, Bn, M, N, C, lambda a, m, c: a[m, c], lambda b, n, c: b[c, n]))
+    At = rng.integers(-127, 128, size=(C, M)).astype(np.int8)
+    out, st = oracle.gemm_tn(At, Bn)
+    assert np.array_equal(out, _brute(At, Bn, M, N, C, lambda a, m, c: a[c, m], lambda b, n, c: b[c, n]))
+
+
+def test_gemm_matches_numpy_int64():
+    rng = np.random.Generator(np.random.PCG64(12))
+    A = rng.integers(-127, 128, size=(37, 300)).astype(np.int8)
+    Bt = rng.integers(-127, 128, size=(45, 300)).astype(np.int8)
+    Bn = rng.integers(-127, 128, size=(300, 45)).astype(np.int8)
+    At = rng.integers(-127, 128, size=(300, 37)).astype(np.int8)
+    i64 = lambda a: a.astype(np.int64)
+    assert np.array_equal(oracle.gemm_nt(A, Bt)[0], i64(A) @ i64(Bt).T)
+    assert np.array_equal(oracle.gemm_nn(A, Bn)[0], i64(A) @ i64(Bn))
+    assert np.array_equal(oracle.gemm_tn(At, Bn)[0], i64(At).T @ i64(Bn))
+
+
+def test_gemm_closed_forms_and_int32_limit():
+    """All-127 operands give 16129*C.  The pages' limit C = 131,071
+    (mini_trainer, contraction paragraph) is floor((2^31-1) / 128^2): no int8
+    dot product of that length leaves int32; at it all-127 gives 2,114,044,159."""
+    limit = int(golden()["int32_contraction_limit"])
+    assert limit == oracle.MAX_CONTRACTION == (2 ** 31 - 1) // (128 * 128)
+    assert 128 * 128 * limit < 2 ** 31 <= 128 * 128 * (limit + 1)
+    A = np.full((1, limit), 127, np.int8)
+    out, st = oracle.gemm_nt(A, A)
+    assert st == 0 and out[0, 0] == 16129 * limit == 2114044159
+    out, st = oracle.gemm_nt(A, -A)
+    assert st == 0 and out[0, 0] == -2114044159
+    # beyond the limit the layer reports the contraction as unsupported
+    x = np.zeros((1, limit + 1), np.float32)
+    w = np.zeros((1, limit + 1), np.int8)
+    y, _, _, st = oracle.fwd(x, w, np.zeros(1, np.float32))
+    assert st == oracle.BIT_UNSUPPORTED
+
+
+# --------------------------------------------------------------------------
+# Layer forward and backward
+# --------------------------------------------------------------------------
+
+def test_fwd_exact_when_inputs_are_representable():
+    """x = s_x q_x and W = s_w q_w with power-of-two scales: the layer output
+    equals the float64 product up to the float32 epilogue rounding."""
+    rng = np.random.Generator(np.random.PCG64(13))
+    M, K, N = 17, 96, 40
+    qx = rng.integers(-127, 128, size=(M, K)).astype(np.int8); qx[:, 0] = 127
+    qw = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    sx = (2.0 ** -rng.integers(0, 8, size=M)).astype(np.float32)
+    sw = (2.0 ** -rng.integers(4, 10, size=N)).astype(np.float32)
+    b = workloads.normal((N,), 0.01, 14)
+    x = qx.astype(np.float32) * sx[:, None]
+    y, xq, sxo, st = oracle.fwd(x, qw, sw, b)
+    assert st == 0 and np.array_equal(xq, qx) and np.array_equal(sxo, sx)
+    ref = (x.astype(np.float64) @ (qw.astype(np.float64) * sw[:, None]).T) + b
+    assert np.abs(y - ref).max() <= 1e-6 * np.abs(ref).max()
+
+
+def _prep_weight(w, B):
+    q, s, st = oracle.quantize_rows(w, B=B, flags=oracle.REJECT_ZERO_ROWS)
+    assert st == 0
+    return q, s
+
+
+def test_fwd_rotation_reduces_error_with_outliers():
+    """The int8 route approximates x W^T + b; with outlier channels the
+    rotated route (both operands rotated) is closer than the plain one
+    (OneTrainer PR #1681: the benefit tracks the outlier ratio)."""
+    d = workloads.tiny_layer()
+    x, w, b = d["x"], d["w"], d["bias"]
+    ref = x.astype(np.float64) @ w.astype(np.float64).T + b
+    errs = {}
+    for B in (0, 256):
+        wq, sw = _prep_weight(w, B)
+        y, _, _, st = oracle.fwd(x, wq, sw, b, B)
+        assert st == 0
+        errs[B] = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert errs[256] < 0.5 * errs[0]
+    assert errs[256] < 0.03
+
+
+def test_bwd_dx_exact_case():
+    """s_w = 1 and integer dY rows containing +-127: dYq_r = dY, s' = 1, so dX
+    is the integer product dY W_q (numpy int64)."""
+    rng = np.random.Generator(np.random.PCG64(15))
+    M, N, K = 9, 48, 80
+    dyi = rng.integers(-127, 128, size=(M, N)); dyi[:, 3] = 127
+    wq = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    dx, q, s1, st = oracle.bwd_dx(dyi.astype(np.float32), wq, np.ones(N, np.float32))
+    assert st == 0 and np.array_equal(q, dyi) and np.all(s1 == 1)
+    assert np.array_equal(dx, (dyi @ wq.astype(np.int64)).astype(np.float32))
+
+
+def test_bwd_dx_rotated_returns_to_input_basis():
+    """For a rotated layer dL/dx = (dY W_rot) R^T = dY W: the oracle's dX
+    approximates dY W in the original basis and not dY W_rot."""
+    d = workloads.tiny_layer()
+    w, dy = d["w"], d["dy"]
+    wq, sw = _prep_weight(w, 256)
+    dx, _, _, st = oracle.bwd_dx(dy, wq, sw, 256)
+    assert st == 0
+    ref = dy.astype(np.float64) @ w.astype(np.float64)
+    rot = dy.astype(np.float64) @ (wq.astype(np.float64) * sw[:, None])
+    assert np.linalg.norm(dx - ref) / np.linalg.norm(ref) < 0.03
+    assert np.linalg.norm(dx - rot) / np.linalg.norm(rot) > 0.5
+
+
+def test_bwd_dw_exact_case_and_bias_grad():
+    """s_x = 1 and integer dY columns containing +-127: dYq_c = dY, s'' = 1,
+    dW = dY^T X_q (numpy int64); db = column sums of dY."""
+    rng = np.random.Generator(np.random.PCG64(16))
+    M, N, K = 23, 40, 64
+    dyi = rng.integers(-127, 128, size=(M, N)); dyi[4, :] = -127
+    xq = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    dw, db, q, s2, st = oracle.bwd_dw(dyi.astype(np.float32), xq, np.ones(M, np.float32))
+    assert st == 0 and np.array_equal(q, dyi) and np.all(s2 == 1)
+    assert np.array_equal(dw, (dyi.T @ xq.astype(np.int64)).astype(np.float32))
+    assert np.array_equal(db, dyi.sum(0).astype(np.float32))
+
+
+def test_bwd_dw_approximates_float_gradient():
+    d = workloads.tiny_layer()
+    xq, sx, _ = oracle.quantize_rows(d["x"], B=256)
+    dy = d["dy"]
+    dw, db, _, _, st = oracle.bwd_dw(dy, xq, sx)
+    assert st == 0
+    ref = dy.astype(np.float64).T @ (xq.astype(np.float64) * sx[:, None])
+    assert np.linalg.norm(dw - ref) / np.linalg.norm(ref) < 0.03
+    assert np.allclose(db, dy.astype(np.float64).sum(0), rtol=1e-6, atol=1e-6)
+
+
+def test_bwd_zero_columns_are_legal():
+    dy = workloads.normal((8, 32), 1.0, 17)
+    dy[:, 5] = 0.0
+    q, s2, db, st = oracle.bwd_prep_cols(dy, np.ones(8, np.float32))
+    assert st == 0 and s2[5] == 0 and not q[:, 5].any() and db[5] == 0
+
+
+# --------------------------------------------------------------------------
+# Philox4x32-10 and stochastic rounding
+# --------------------------------------------------------------------------
+
+CURAND = "/usr/local/cuda/lib64/libcurand.so"
+
+
+def _curand_host_philox(seed: int, n: int) -> np.ndarray:
+    lib = ctypes.CDLL(CURAND)
+    g = ctypes.c_void_p()
+    assert lib.curandCreateGeneratorHost(ctypes.byref(g), 161) == 0  # PHILOX4_32_10
+    assert lib.curandSetPseudoRandomGeneratorSeed(g, ctypes.c_ulonglong(seed)) == 0
+    out = np.zeros(n, dtype=np.uint32)
+    assert lib.curandGenerate(g, out.ctypes.data_as(ctypes.c_void_p), ctypes.c_size_t(n)) == 0
+    lib.curandDestroyGenerator(g)
+    return out
+
+
+@pytest.mark.skipif(not os.path.exists(CURAND), reason="cuRAND host library not present")
+def test_philox_matches_curand_host_generator():
+    """cuRAND's host Philox4x32-10 (seed = key) emits block j from counter
+    (j / 65536, 0, j % 65536, 0); the oracle must reproduce every word."""
+    rng = np.random.Generator(np.random.PCG64(18))
+    for seed in (0, 7, 0x123456789ABCDEF0):
+        out = _curand_host_philox(seed, 4 * 65536 * 2)
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        blocks = list(range(0, 40)) + list(rng.integers(0, 2 * 65536, size=300))
+        for j in blocks:
+            j = int(j)
+            ctr = [j // 65536, 0, j % 65536, 0]
+            assert np.array_equal(oracle.philox4x32_10(ctr, key), out[4 * j:4 * j + 4]), (seed, j)
+        # the stochastic-rounding uniform: element e at step z uses counter
+        # (e >> 2, 0, z, 0) and word e & 3, top 24 bits
+        for j in blocks[:64]:
+            j = int(j)
+            x, z = j // 65536, j % 65536
+            for w in range(4):
+                assert oracle.sr_u24(seed, z, 4 * x + w) == int(out[4 * j + w]) >> 8
+
+
+def test_u24_is_uniform():
+    """Chi-square over 256 bins of u24 >> 16 for 2^17 consecutive elements."""
+    n = 1 << 17
+    u = np.array([oracle.sr_u24(1234, 3, e) for e in range(n)], np.int64)
+    assert u.min() >= 0 and u.max() < (1 << 24)
+    counts = np.bincount(u >> 16, minlength=256)
+    exp = n / 256
+    chi2 = ((counts - exp) ** 2 / exp).sum()
+    # 255 degrees of freedom: mean 255, sd ~22.6; 6 sd bound
+    assert chi2 < 255 + 6 * 22.6
+
+
+@pytest.mark.parametrize("v", [0.25, -0.25, 3.7, -3.7, 126.9, -126.9, 0.0,
+                               5.0, -101.0, 1.0 / 3.0, 2.0 ** -25, -(2.0 ** -23)])
+def test_sr_expectation_by_enumeration(v):
+    """Over all 2^24 uniforms, E[q] = floor(v) + ceil(frac * 2^24) / 2^24, so
+    |E[q] - v| < 2^-24: stochastic rounding is unbiased to 24 bits."""
+    v32 = float(np.float32(v))
+    E = oracle.sr_expectation_enum(v32)
+    f = math.floor(v32)
+    frac = v32 - f
+    assert E == f + math.ceil(frac * 2 ** 24) / 2 ** 24
+    assert abs(E - v32) < 2.0 ** -24
+    if v32 == f:
+        assert E == v32
+
+
+def test_sr_identity_when_values_are_codes():
+    """SGD with lr = 0 on a row with a power-of-two scale leaves every code
+    an integer after scaling, so the stochastic requant is exact."""
+    rng = np.random.Generator(np.random.PCG64(19))
+    q = rng.integers(-127, 128, size=(6, 64)).astype(np.int8); q[:, 0] = -127
+    s = (2.0 ** -rng.integers(3, 9, size=6)).astype(np.float32)
+    g = workloads.normal((6, 64), 1.0, 20)
+    q2, s2, *_, st = oracle.update_sr(q, s, g, oracle.SGD, 0.0, seed=5, step=1)
+    assert st == 0 and np.array_equal(q2, q) and np.array_equal(s2, s)
+
+
+def test_sr_unbiased_over_seeds():
+    """The mean of the requantized weight over many seeds approaches the
+    float update (5 sigma)."""
+    d = workloads.update_state(4, 64, seed=2)
+    q, s, _ = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    w1, *_ = oracle.update_float(q, s, d["grad"], oracle.SGD, 0.05, step=1)
+    n = 400
+    acc = np.zeros_like(w1, np.float64)
+    for seed in range(n):
+        q2, s2, *_ = oracle.update_sr(q, s, d["grad"], oracle.SGD, 0.05, seed=seed, step=1)
+        acc += q2.astype(np.float64) * s2[:, None]
+    mean = acc / n
+    step = (np.abs(w1).max(1) / 127.0)[:, None]
+    sigma = 0.5 * step / math.sqrt(n)
+    assert np.all(np.abs(mean - w1) <= 5 * sigma + 1e-9)
+
+
+# --------------------------------------------------------------------------
+# Optimizer steps against torch.optim / torch autograd (float64)
+# --------------------------------------------------------------------------
+
+def _f32(v: float) -> float:
+    """The float32 value the C ABI receives for a hyper-parameter."""
+    return float(np.float32(v))
+
+
+def _dequant(q, s):
+    return q.astype(np.float64) * s.astype(np.float64)[:, None]
+
+
+def test_sgd_step_matches_torch():
+    d = workloads.update_state(8, 96, seed=3)
+    q, s, _ = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    w, *_, st = oracle.update_float(q, s, d["grad"], oracle.SGD, 1e-2, step=1)
+    assert st == 0
+    p = torch.nn.Parameter(torch.from_numpy(q.astype(np.float32) * s[:, None]).double())
+    opt = torch.optim.SGD([p], lr=_f32(1e-2))
+    p.grad = torch.from_numpy(d["grad"]).double()
+    opt.step()
+    assert np.abs(w - p.detach().numpy()).max() <= 1e-8
+
+
+@pytest.mark.parametrize("warm", [False, True])
+def test_adamw_step_matches_torch(warm):
+    d = workloads.update_state(8, 96, seed=4, warm=warm)
+    q, s, _ = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    lr, wd, t = 1e-3, 0.01, d["step"]
+    w, m, v, *_, st = oracle.update_float(q, s, d["grad"], oracle.ADAMW, lr, step=t,
+                                          m=d["m"], v=d["v"], wd=wd)
+    assert st == 0
+    p = torch.nn.Parameter(torch.from_numpy(q.astype(np.float32) * s[:, None]).double())
+    opt = torch.optim.AdamW([p], lr=_f32(lr), betas=(_f32(0.9), _f32(0.999)), eps=_f32(1e-8),
+                            weight_decay=_f32(wd))
+    p.grad = torch.from_numpy(d["grad"]).double()
+    opt.state[p] = {"step": torch.tensor(float(t - 1)),
+                    "exp_avg": torch.from_numpy(d["m"]).double(),
+                    "exp_avg_sq": torch.from_numpy(d["v"]).double()}
+    opt.step()
+    st_t = opt.state[p]
+    assert np.allclose(m, st_t["exp_avg"].numpy(), rtol=1e-5, atol=1e-12)
+    assert np.allclose(v, st_t["exp_avg_sq"].numpy(), rtol=1e-5, atol=1e-16)
+    assert np.abs(w - p.detach().numpy()).max() <= 1e-6 * np.abs(w).max()
+
+
+def test_weight_norm_step_matches_torch_autograd():
+    """Row-wise weight norm (dim=0): w = g * v / ||v||.  torch autograd gives
+    dL/dg and dL/dv for dL/dw = grad; torch AdamW then steps g and v."""
+    d = workloads.update_state(6, 128, seed=5, weight_norm=True)
+    q, s, _ = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    lr, wd = 1e-3, 0.01
+    wv, m, v, g, gm, gv, st = oracle.update_float(
+        q, s, d["grad"], oracle.ADAMW, lr, step=1, m=d["m"], v=d["v"], wd=wd,
+        g=d["g"], g_m=d["g_m"], g_v=d["g_v"])
+    assert st == 0
+    vp = torch.nn.Parameter(torch.from_numpy(_dequant(q, s)))
+    gp = torch.nn.Parameter(torch.from_numpy(d["g"].astype(np.float64)))
+    w_eff = gp[:, None] * vp / vp.norm(dim=1, keepdim=True)
+    (w_eff * torch.from_numpy(d["grad"]).double()).sum().backward()
+    # direction gradient is orthogonal to the direction
+    assert (vp.grad * vp.detach()).sum(1).abs().max().item() <= 1e-12
+    opt = torch.optim.AdamW([vp, gp], lr=_f32(lr), betas=(_f32(0.9), _f32(0.999)),
+                            eps=_f32(1e-8), weight_decay=_f32(wd))
+    opt.step()
+    assert np.abs(wv - vp.detach().numpy()).max() <= 1e-6 * np.abs(wv).max()
+    assert np.allclose(g, gp.detach().numpy(), rtol=1e-6)
+    assert np.allclose(m, opt.state[vp]["exp_avg"].numpy(), rtol=1e-4, atol=1e-12)
+    assert np.allclose(gm, opt.state[gp]["exp_avg"].numpy(), rtol=1e-4, atol=1e-12)
+
+
+def test_weight_norm_effective_rows_have_norm_g():
+    d = workloads.update_state(5, 64, seed=6, weight_norm=True)
+    q, s, _ = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    q2, s2, m, v, g2, gm, gv, st = oracle.update_sr(
+        q, s, d["grad"], oracle.ADAMW, 1e-3, seed=1, step=1, m=d["m"], v=d["v"],
+        g=d["g"], g_m=d["g_m"], g_v=d["g_v"])
+    assert st == 0
+    w_eff = g2[:, None] * q2.astype(np.float64) / np.linalg.norm(q2.astype(np.float64), axis=1)[:, None]
+    assert np.allclose(np.linalg.norm(w_eff, axis=1), g2, rtol=1e-12)
+
+
+def test_weight_norm_rejects_zero_direction():
+    d = workloads.update_state(3, 32, seed=7, weight_norm=True)
+    q, s, _ = oracle.quantize_rows(d["w"])
+    q[1] = 0
+    s[1] = 0
+    q2, s2, m, v, g2, *_, st = oracle.update_sr(
+        q, s, d["grad"], oracle.ADAMW, 1e-3, seed=1, step=1, m=d["m"], v=d["v"],
+        g=d["g"], g_m=d["g_m"], g_v=d["g_v"])
+    assert st == oracle.BIT_ZERO_ROW
+    assert not q2[1].any() and g2[1] == d["g"][1] and not m[1].any()
+    assert q2[0].any() and q2[2].any()
+
+
+def test_update_argument_checks():
+    q = np.ones((2, 16), np.int8)
+    s = np.ones(2, np.float32)
+    g = np.zeros((2, 16), np.float32)
+    assert oracle.update_sr(q, s, g, oracle.SGD, 0.1, seed=0, step=0)[-1] == oracle.BIT_ARG
+    assert oracle.update_sr(q, s, g, oracle.SGD, 0.1, seed=0, step=1, wd=0.1)[-1] == oracle.BIT_ARG
+    assert oracle.update_sr(q, s, g, 7, 0.1, seed=0, step=1)[-1] == oracle.BIT_ARG
