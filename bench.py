@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the INT8 quantized-training Linear layer on B200.
+
+One step = one pass of the whole hot path over one batch: the 5376 -> 7168
+layer of OneTrainer PR #1681 "Int8 conv rot" at 12000 tokens with Hadamard
+block 128, bf16 X and dY:
+    qlinear_fwd       per-row rotate + quantize X (saved int8), int8 GEMM, scale + bias -> bf16 y
+    qlinear_bwd_dx    row-quantize dY*s_w, int8 GEMM (dY_q W_q), scale, fused rotation -> bf16 dX
+    qlinear_bwd_dw    column-quantize dY*s_x, int8 GEMM (dY_q^T X_q), scale -> fp32 dW, db
+    qweight_update_sr AdamW on the int8 weight + Philox stochastic requantization
+Metric: int8 tensor operations of the three GEMMs (3 x 2*M*N*K) per second,
+in TOPS, whole job (all ranks).  Inputs stay resident in HBM; the step's
+working set (about 1 GB) is far larger than the 126 MB L2.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+With N > 1 it runs under torchrun, one independent replica per GPU (the
+layer's path has no exchange step), and reports the max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+M_TOK, K_IN, N_OUT, BLOCK = 12000, 5376, 7168, 128
+GEMM_OPS = 2 * M_TOK * N_OUT * K_IN          # one GEMM launch
+STEP_OPS = 3 * GEMM_OPS                       # fwd + dX + dW
+UPDATE_BYTES = 22 * N_OUT * K_IN              # AdamW SR update: 1+4+4+4 in, 1+4+4 out
+METRIC = "INT8 qlinear fwd+bwd TOPS (3 int8 GEMMs per train step of the 5376->7168 layer, 12000 tokens)"
+WORKLOAD = ("qlinear train step: M=12000 K=5376 N=7168, Hadamard block 128, bf16 X/dY/y/dX, "
+            "fwd + dX + dW + AdamW stochastic requant")
+NOMINAL_INT8_OVER_BF16 = 2.0   # dense int8 4.5 POPS / dense bf16 2.25 PFLOPS
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- peaks / clocks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our path
+class Layer:
+    """Device state of one replica: the prepared int8 weight, AdamW moments,
+    bf16 X / dY of one batch, outputs and the backward workspace."""
+
+    def __init__(self):
+        import torch
+        import int8_quantized_act_b200 as ql
+        import workloads
+        self.ql, self.torch = ql, torch
+        d = workloads.rotated_layer(M=M_TOK, seed=1)
+        dev = "cuda"
+        self.x_host = d["x_bf16"].pin_memory()
+        self.dy_host = d["dy_bf16"].pin_memory()
+        self.x = self.x_host.to(dev)
+        self.dy = self.dy_host.to(dev)
+        self.bias = torch.from_numpy(d["bias"]).to(dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.wq = torch.empty((N_OUT, K_IN), dtype=torch.int8, device=dev)
+        self.sw = torch.empty(N_OUT, dtype=torch.float32, device=dev)
+        ql.qlinear_quantize_rows(torch.from_numpy(d["w"]).to(dev), self.wq, self.sw, self.status,
+                                 hadamard_block=BLOCK, flags=ql.QL_REJECT_ZERO_ROWS)
+        self.m = torch.zeros((N_OUT, K_IN), dtype=torch.float32, device=dev)
+        self.v = torch.zeros((N_OUT, K_IN), dtype=torch.float32, device=dev)
+        self.y = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=dev)
+        self.xq = torch.empty((M_TOK, K_IN), dtype=torch.int8, device=dev)
+        self.sx = torch.empty(M_TOK, dtype=torch.float32, device=dev)
+        self.dx = torch.empty((M_TOK, K_IN), dtype=torch.bfloat16, device=dev)
+        self.dw = torch.empty((N_OUT, K_IN), dtype=torch.float32, device=dev)
+        self.db = torch.empty(N_OUT, dtype=torch.float32, device=dev)
+        self.ws = torch.empty(ql.qlinear_workspace_bytes(M_TOK, N_OUT, K_IN, BLOCK),
+                              dtype=torch.uint8, device=dev)
+        self.opt = ql.Optim(kind=ql.QL_ADAMW, lr=1e-3, weight_decay=0.01)
+        self.t = 0
+        self.y_host = torch.empty_like(self.y, device="cpu").pin_memory()
+        self.dx_host = torch.empty_like(self.dx, device="cpu").pin_memory()
+        torch.cuda.synchronize()
+
+    def step(self, gemm_events=None, update_events=None):
+        ql = self.ql
+        self.t += 1
+        ev = gemm_events or [None] * 6
+        ql.ql_set_gemm_timing_events(ev[0], ev[1])
+        ql.qlinear_fwd(self.x, self.wq, self.sw, self.bias, BLOCK, self.y, self.xq, self.sx,
+                       self.status)
+        ql.ql_set_gemm_timing_events(ev[2], ev[3])
+        ql.qlinear_bwd_dx(self.dy, self.wq, self.sw, BLOCK, self.dx, self.ws, self.status)
+        ql.ql_set_gemm_timing_events(ev[4], ev[5])
+        ql.qlinear_bwd_dw(self.dy, self.xq, self.sx, self.dw, self.db, self.ws, self.status)
+        ql.ql_set_gemm_timing_events(None, None)
+        if update_events:
+            update_events[0].record()
+        ql.qweight_update_sr(self.wq, self.sw, self.dw, self.opt, self.m, self.v, 1234, self.t,
+                             self.status)
+        if update_events:
+            update_events[1].record()
+
+    def step_e2e(self):
+        """The same step through the public API with host buffers: X and dY
+        copied in from pinned host memory, y and dX copied back."""
+        self.x.copy_(self.x_host, non_blocking=True)
+        self.dy.copy_(self.dy_host, non_blocking=True)
+        self.step()
+        self.y_host.copy_(self.y, non_blocking=True)
+        self.dx_host.copy_(self.dx, non_blocking=True)
+
+
+def new_events(n):
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()  # materialise the CUDA event before the library records it
+    return evs
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import int8_quantized_act_b200 as ql
+
+    layer = Layer()
+    for _ in range(args.warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    gemm_ev = [new_events(6) for _ in range(args.steps)]
+    upd_ev = [new_events(2) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = ql.ql_kernel_launches()
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.start()
+    time.sleep(0.2)  # let the sampler start before the timed region
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(args.steps):
+        layer.step(gemm_ev[i], upd_ev[i])
+    stop.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    launches = ql.ql_kernel_launches() - launches0
+    ms = start.elapsed_time(stop)
+    ms_max = max_over_ranks(ms, world)
+    word = int(layer.status.item())
+    if word:
+        raise RuntimeError(f"device status {ql.status_flags(word)}")
+
+    gemm_ms = [e[2 * j].elapsed_time(e[2 * j + 1]) for e in gemm_ev for j in range(3)]
+    per_kind = {name: statistics.mean(gemm_ms[j::3]) for j, name in enumerate(("fwd", "dx", "dw"))}
+    gemm_avg = statistics.mean(gemm_ms)
+    upd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in upd_ev)
+
+    # end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    layer.step_e2e()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(e2e_steps):
+        layer.step_e2e()
+    t1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / e2e_steps
+
+    peaks = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    gemm_tops = GEMM_OPS / (gemm_avg * 1e-3) / 1e12
+    value = world * STEP_OPS * args.steps / (ms_max * 1e-3) / 1e12
+    h2d = layer.x.numel() * 2 + layer.dy.numel() * 2
+    d2h = layer.y.numel() * 2 + layer.dx.numel() * 2
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "i8",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT,
+                   "hadamard_block": BLOCK, "x_dtype": "bf16", "dy_dtype": "bf16",
+                   "y_dtype": "bf16", "dx_dtype": "bf16", "dw_dtype": "f32",
+                   "optimizer": "AdamW lr=1e-3 wd=0.01, fp32 moments",
+                   "l2": "no flush: step working set ~1.1 GB > 126 MB L2",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_i8 (tcgen05 kind::i8, fwd/dX/dW launches)",
+                     "achieved": round(gemm_tops, 1),
+                     "peak": round(int8_peak, 1), "unit": "TOPS",
+                     "frac": round(gemm_tops / int8_peak, 4),
+                     "peak_source": f"{peaks['source']}: bf16 dense burst x {NOMINAL_INT8_OVER_BF16} (int8/bf16 nominal ratio)",
+                     "ms_per_launch": {k: round(v, 4) for k, v in per_kind.items()},
+                     "traffic": None},
+        "row_kernel": {"kernel": "update_sr (AdamW + stochastic requant)", "bound": "hbm",
+                       "achieved": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9, 1),
+                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                       "ms_per_launch": round(upd_ms, 4)},
+        "e2e": {"value": round(world * STEP_OPS / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(seconds=12.0)
+    return out
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_sample_step(d, xq_all, sx_all, wq, sw, rows, wcols, urows, t):
+    """One bounded sample of the step on the oracle: forward and dX of `rows`
+    tokens, dW of `wcols` output rows over all tokens, AdamW requant of
+    `urows` weight rows.  Returns the int8 GEMM ops done."""
+    import numpy as np
+    import oracle
+    x = d["x"][:rows]
+    oracle.fwd(x, wq, sw, d["bias"], BLOCK)
+    oracle.bwd_dx(d["dy"][:rows], wq, sw, BLOCK)
+    dw, *_ = oracle.bwd_dw(d["dy"][:, :wcols], xq_all, sx_all)
+    g = np.ascontiguousarray(dw[:urows]) if urows <= wcols else np.zeros((urows, K_IN), np.float32)
+    zeros = np.zeros((urows, K_IN), np.float32)
+    oracle.update_sr(wq[:urows], sw[:urows], g, oracle.ADAMW, 1e-3, 1234, t, m=zeros, v=zeros,
+                     wd=0.01)
+    return 2 * rows * N_OUT * K_IN * 2 + 2 * wcols * K_IN * M_TOK
+
+
+def cpu_prepare():
+    import oracle
+    import workloads
+    d = workloads.rotated_layer(M=M_TOK, seed=1)
+    wq, sw, _ = oracle.quantize_rows(d["w"], B=BLOCK, flags=oracle.REJECT_ZERO_ROWS)
+    xq, sx, _ = oracle.quantize_rows(d["x"], B=BLOCK)
+    return d, xq, sx, wq, sw
+
+
+def cpu_baseline(seconds=12.0, prepared=None):
+    """The oracle as it stands (single-threaded C) on a bounded sample of the
+    workload, scaled to the metric's unit."""
+    d, xq, sx, wq, sw = prepared or cpu_prepare()
+    rows, wcols, urows = 4, 2, 8
+    ops, t0, t = 0, time.perf_counter(), 0
+    while time.perf_counter() - t0 < seconds:
+        t += 1
+        ops += cpu_sample_step(d, xq, sx, wq, sw, rows, wcols, urows, t)
+    el = time.perf_counter() - t0
+    return {"value": round(ops / el / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": (f"{t} samples of the step: fwd + dX of {rows} of 12000 tokens, dW of "
+                       f"{wcols} of 7168 output rows over all tokens, AdamW requant of {urows} "
+                       f"weight rows; {el:.1f} s single-threaded; ops = int8 GEMM ops done")}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    prepared = cpu_prepare()
+    for _ in range(args.warmup):
+        cpu_sample_step(*prepared, 4, 2, 8, 1)
+    ops, t0 = 0, time.perf_counter()
+    for i in range(args.steps):
+        ops += cpu_sample_step(*prepared, 4, 2, 8, i + 1)
+    el = time.perf_counter() - t0
+    value = ops / el / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT,
+                   "hadamard_block": BLOCK, "parallelism": "cpu oracle, rank 0"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+                         "sample": "each step: fwd + dX of 4 of 12000 tokens, dW of 2 of 7168 "
+                                   "output rows over all tokens, AdamW requant of 8 weight rows"},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    world_env = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, rank, world_env)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        out = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,220 @@
+/*
+ * qlinear.h - C ABI of the INT8 quantized-training Linear layer for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The layer keeps its weight as int8 codes with one float32 scale per output
+ * row and no floating master copy; it quantizes its input per row on every
+ * call, saves the int8 input for backward, runs int8 x int8 -> int32 GEMMs on
+ * the tensor cores for the forward and both backward products, and updates
+ * the weight with a stochastic requantization after each optimizer step.  An
+ * optional block-Hadamard rotation R along the contraction dimension spreads
+ * channel outliers before quantization.  Sources, cited by page title and part:
+ *
+ *   [QT] mini_trainer "docs/quantized-training.md": intro paragraph (INT8
+ *        weights and saved Linear inputs, integer forward/backward products,
+ *        no floating master weight, biases/gradients/optimizer state stay
+ *        float), feature table (row-wise weight norm with int8 direction and
+ *        float magnitude, zero directions rejected; bias, batched,
+ *        single-sample inputs; SGD and AdamW), the paragraph after the table
+ *        (updates requantize stochastically, fused row kernels), and the
+ *        paragraph on contractions above 131,071.
+ *   [CR] OneTrainer PR #1681 "Int8 conv rot": opening summary (block-Hadamard
+ *        rotation), commit note item 1 (activations quantized per row every
+ *        call; int8 route vs bf16 route), item 2 ((xR)(WR)^T = xW^T: rotate x,
+ *        never un-rotate W), item 3 (the torch._int_mm row floor, which this
+ *        library does not have), closing Summary.
+ *
+ * Conventions for every entry point
+ *   - Matrices are row-major.  M = tokens (rows of x), K = in_features,
+ *     N = out_features.  All pointers are DEVICE pointers unless stated.
+ *   - The caller owns every buffer.  The library never allocates device
+ *     memory; its only global state is a per-device, thread-safe, one-time
+ *     kernel attribute set-up on first use.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on `stream` and never
+ *     synchronizes.
+ *   - Argument, shape and alignment errors are detected on the host before
+ *     any launch and returned; no output is touched then.  Conditions found
+ *     on the device (zero rows, non-finite values, a wait that timed out)
+ *     are OR-ed as bits (1u << code) into *d_status, a caller-owned device
+ *     int32 that the caller zeroes and reads after its own synchronization.
+ *   - int8 operands and outputs need 16-byte aligned pointers and row pitches
+ *     that are multiples of 16 bytes (the tensor-memory-access engine reads
+ *     them); this is why K and N must be multiples of 16.  M has no floor:
+ *     M = 1 is valid, unlike torch._int_mm's "more than 16 rows" ([CR] item 3).
+ *   - Float inputs (x, dY) are float32 or bf16 (ql_dtype), 16-byte aligned.
+ *   - The float arithmetic that decides an integer code is IEEE binary32
+ *     with round-to-nearest-even and no fused multiply-add, so int8 codes,
+ *     scales and stochastic-rounding results are reproducible bit for bit.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QL_API __attribute__((visibility("default")))
+#else
+#define QL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes.  Device-side conditions use the bit (1u << code). */
+typedef enum {
+    QL_OK = 0,
+    QL_ERR_ARG = 1,         /* null pointer, bad enum, bad hyper-parameter      */
+    QL_ERR_SHAPE = 2,       /* negative size, K or N not a multiple of 16,
+                               bad Hadamard block, too-small workspace          */
+    QL_ERR_ALIGN = 3,       /* pointer or row pitch not 16-byte aligned        */
+    QL_ERR_ZERO_ROW = 4,    /* device: a rejected all-zero row / direction      */
+    QL_ERR_NONFINITE = 5,   /* device: inf or NaN met; affected outputs are
+                               unspecified                                       */
+    QL_ERR_UNSUPPORTED = 6, /* contraction above 131,071 ([QT]), row too long   */
+    QL_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed              */
+    QL_ERR_TIMEOUT = 8      /* device: a pipeline wait gave up (bounded waits;
+                               the kernel returns instead of hanging)            */
+} ql_status;
+
+typedef enum { QL_F32 = 0, QL_BF16 = 1 } ql_dtype;
+
+typedef enum { QL_SGD = 0, QL_ADAMW = 1 } ql_optim_kind;
+
+/* Optimizer hyper-parameters.  SGD: w' = w - lr*g (no momentum; weight_decay
+ * must be 0).  AdamW (decoupled weight decay): w1 = w*(1-lr*wd);
+ * m' = b1*m + (1-b1)*g; v' = b2*v + (1-b2)*g*g;
+ * w' = w1 - (lr/(1-b1^t)) * m' / (sqrt(v'/(1-b2^t)) + eps). */
+typedef struct {
+    int kind; /* ql_optim_kind */
+    float lr, beta1, beta2, eps, weight_decay;
+} ql_optim;
+
+/* Row-wise weight normalization (dim=0, [QT] feature table): the stored int8
+ * row is the direction v = s*q; the effective weight row is g[n]*q/||q||.
+ * g is float32 [N]; g_m, g_v are its AdamW moments (may be NULL for SGD). */
+typedef struct {
+    float *g;
+    float *g_m;
+    float *g_v;
+} ql_weightnorm;
+
+/* qlinear_quantize_rows flag: report all-zero rows as QL_ERR_ZERO_ROW (used
+ * when preparing weights: a zero direction cannot be represented). */
+#define QL_REJECT_ZERO_ROWS 1u
+
+/* Largest contraction length accepted by the GEMMs: no int8 dot product of
+ * this length can leave int32, floor((2^31-1)/128^2) ([QT], contraction
+ * paragraph). */
+#define QL_MAX_CONTRACTION 131071
+
+/* Human-readable name of a status code (static string). */
+QL_API const char *ql_status_string(int status);
+
+/* Bytes of device workspace that qlinear_bwd_dx / qlinear_bwd_dw need for
+ * a layer of these sizes and Hadamard block (0 = no rotation).  The buffer is
+ * scratch: its contents on entry do not matter and on exit are unspecified. */
+QL_API size_t qlinear_workspace_bytes(int64_t M, int64_t N, int64_t K, int hadamard_block);
+
+/* Per-row symmetric int8 quantization, optionally rotated ([CR] item 1 and
+ * summary).  For each row r of x [rows, cols] (pitch ldx elements, dtype xt):
+ *   t = x[r,:] * col_scale (elementwise, if col_scale != NULL)
+ *   t = t R                (if hadamard_block = B > 0; R = blockdiag(H_B)/sqrt(B),
+ *                           Sylvester order, butterflies h = 1..B/2 then one
+ *                           multiply by fl32(1/sqrt(B)))
+ *   amax = max|t|; row_scale[r] = amax/127; q[r,:] = clamp(rne(t*(127/amax)), +-127)
+ * amax = 0 gives scale 0 and zero codes, and sets QL_ERR_ZERO_ROW in
+ * *d_status when flags has QL_REJECT_ZERO_ROWS.  This is also the weight
+ * preparation step: quantize W [N,K] with the layer's block and the flag.
+ * Requirements: cols % 16 == 0; B in {0, 2, 4, ..., 256} with cols % B == 0;
+ * ldx >= cols, ldq >= cols, ldq % 16 == 0; x, q 16-byte aligned and
+ * ldx * sizeof(xt) % 16 == 0; col_scale (optional) 16-byte aligned. */
+QL_API int qlinear_quantize_rows(const void *x, int xt, int64_t rows, int64_t cols, int64_t ldx,
+                          const float *col_scale, int hadamard_block, unsigned flags,
+                          int8_t *q, int64_t ldq, float *row_scale,
+                          int32_t *d_status, void *stream);
+
+/* y = x R row by row (R as above), x [rows, cols] of dtype xt with pitch ldx,
+ * y of dtype yt with pitch ldy; y == x (same dtype and pitch) is allowed.
+ * R is its own inverse, so this also un-rotates (the "unquantized weight"
+ * of [CR] item 2: dequantize the codes, then call this). */
+QL_API int qlinear_hadamard(const void *x, int xt, int64_t ldx, void *y, int yt, int64_t ldy,
+                     int64_t rows, int64_t cols, int hadamard_block, void *stream);
+
+/* Forward ([CR] item 1 and summary; [QT] intro):
+ *   X_q, s_x = quantize_rows(x, B)                     (saved for backward)
+ *   y[m,n] = ((float)(sum_k X_q[m,k] W_q[n,k]) * s_x[m]) * s_w[n] + bias[n]
+ * x [M,K] (xt), W_q [N,K] int8 prepared in the same rotated basis, s_w [N],
+ * bias [N] float32 or NULL, y [M,N] of dtype yt, xq_saved [M,K] int8,
+ * sx_saved [M] float32.  K, N multiples of 16; K <= QL_MAX_CONTRACTION. */
+QL_API int qlinear_fwd(const void *x, int xt, int64_t M, int64_t K,
+                const int8_t *wq, const float *sw, int64_t N, const float *bias,
+                int hadamard_block, void *y, int yt,
+                int8_t *xq_saved, float *sx_saved, int32_t *d_status, void *stream);
+
+/* Input gradient:
+ *   dYq, s' = quantize_rows(dY, col_scale = s_w)       (row quantization of dY*s_w)
+ *   dX[m,k] = (float)(sum_n dYq[m,n] W_q[n,k]) * s'[m], then dX R if B > 0
+ * (the layer saw xR, and R is symmetric, so dL/dx = dL/d(xR) R^T = (...) R).
+ * dY [M,N] (dyt), W_q [N,K], s_w [N], dX [M,K] (dxt).  ws: device workspace of
+ * at least qlinear_workspace_bytes(M,N,K,B) bytes, 256-byte aligned.
+ * N <= QL_MAX_CONTRACTION. */
+QL_API int qlinear_bwd_dx(const void *dy, int dyt, int64_t M, int64_t N,
+                   const int8_t *wq, const float *sw, int64_t K, int hadamard_block,
+                   void *dx, int dxt, void *ws, size_t ws_bytes,
+                   int32_t *d_status, void *stream);
+
+/* Weight (and bias) gradient from the int8-saved input:
+ *   t''[m,n] = dY[m,n]*s_x[m]; per column n: s''[n] = max_m|t''|/127,
+ *   dYq_c[m,n] = clamp(rne(t''*(127/max_m|t''|)), +-127)
+ *   dW[n,k] = (float)(sum_m dYq_c[m,n] X_q[m,k]) * s''[n]   (float32 [N,K],
+ *             in the rotated basis when the layer is rotated)
+ *   db[n]   = sum_m dY[m,n] (float64 sum rounded to float32), if db != NULL.
+ * dY [M,N] (dyt), X_q [M,K] int8 and s_x [M] as saved by qlinear_fwd.
+ * M <= QL_MAX_CONTRACTION.  ws as for qlinear_bwd_dx. */
+QL_API int qlinear_bwd_dw(const void *dy, int dyt, int64_t M, int64_t N,
+                   const int8_t *xq, const float *sx, int64_t K,
+                   float *dw, float *db, void *ws, size_t ws_bytes,
+                   int32_t *d_status, void *stream);
+
+/* One optimizer step of an int8 weight [N,K] with stochastic requantization,
+ * in place ([QT] paragraph after the feature table; rows "Optimizers",
+ * "Row-wise weight normalization"):
+ *   w = s_w[n]*q[n,k]; w' = step(w, grad) (SGD or AdamW, moments m, v float32
+ *   [N,K] updated in place; NULL for SGD); per row: s' = max|w'|/127 and
+ *   q'[n,k] = floor(w'*127/max|w'|) + 1 with probability equal to the
+ *   fractional part, decided by u24 < frac*2^24 where u24 is the top 24 bits
+ *   of word (e & 3) of Philox4x32-10 with key = seed and counter =
+ *   (e>>2 low, e>>2 high, step low, step high), e = n*K + k.
+ * With wn != NULL the rows are weight-norm directions: grad is the gradient
+ * of the effective row g*q/||q||; the direction gradient
+ *   dv = (g/(s*||q||)) * (grad - dg*q/||q||),  dg = sum_k grad*q/||q||
+ * (dg summed in a fixed order: groups of 16 consecutive elements dealt
+ * round-robin to 256 lanes, each lane in increasing k, then an xor butterfly
+ * over the lanes with offsets 128..1) steps v = s*q, dg steps g; a zero
+ * direction sets QL_ERR_ZERO_ROW and leaves its row and state unchanged.
+ * opt and wn are HOST pointers (wn's members are device pointers).
+ * step >= 1.  K % 16 == 0, K <= 32768. */
+QL_API int qweight_update_sr(int8_t *wq, float *sw, const float *grad, int64_t N, int64_t K,
+                      const ql_optim *opt, float *m, float *v,
+                      uint64_t seed, uint64_t step, const ql_weightnorm *wn,
+                      int32_t *d_status, void *stream);
+
+/* Instrumentation (no effect on results).
+ * ql_set_gemm_timing_events: while set (non-NULL), every int8 GEMM kernel that
+ * the calling host thread launches records the cudaEvent_t `before` on its
+ * stream right before the launch and `after` right after it, so a caller can
+ * time the GEMM alone inside a layer call.  Pass NULL, NULL to stop.  The
+ * events are the caller's; the library only records them.
+ * ql_kernel_launches: number of CUDA kernels this library has launched in the
+ * process so far (all threads). */
+QL_API void ql_set_gemm_timing_events(void *before, void *after);
+QL_API uint64_t ql_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLINEAR_H */

@@ -1,0 +1,273 @@
+"""int8_quantized_act_b200 - INT8 quantized-training Linear layer for B200.
+
+Thin Python binding of the C-ABI library ``libqlinear.so`` (declared in
+``include/qlinear.h``).  Each function has the name of the C entry point,
+takes torch CUDA tensors, checks that they are CUDA tensors of the expected
+dtype and layout, passes their device pointers and sizes, and raises
+``QLError`` on a non-zero return code.  Every step of the layer runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and importing
+this package fails loudly if the library has not been built.
+
+Build the library with ``python -m int8_quantized_act_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "QL_OK", "QL_ERR_ARG", "QL_ERR_SHAPE", "QL_ERR_ALIGN", "QL_ERR_ZERO_ROW",
+    "QL_ERR_NONFINITE", "QL_ERR_UNSUPPORTED", "QL_ERR_CUDA", "QL_ERR_TIMEOUT",
+    "QL_F32", "QL_BF16", "QL_SGD", "QL_ADAMW", "QL_REJECT_ZERO_ROWS",
+    "QL_MAX_CONTRACTION", "QLError", "Optim", "lib", "library_path",
+    "ql_status_string", "qlinear_workspace_bytes", "qlinear_quantize_rows",
+    "qlinear_hadamard", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
+    "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
+]
+
+QL_OK, QL_ERR_ARG, QL_ERR_SHAPE, QL_ERR_ALIGN = 0, 1, 2, 3
+QL_ERR_ZERO_ROW, QL_ERR_NONFINITE, QL_ERR_UNSUPPORTED = 4, 5, 6
+QL_ERR_CUDA, QL_ERR_TIMEOUT = 7, 8
+QL_F32, QL_BF16 = 0, 1
+QL_SGD, QL_ADAMW = 0, 1
+QL_REJECT_ZERO_ROWS = 1
+QL_MAX_CONTRACTION = 131071
+
+_NAMES = {
+    QL_OK: "OK", QL_ERR_ARG: "ARG", QL_ERR_SHAPE: "SHAPE", QL_ERR_ALIGN: "ALIGN",
+    QL_ERR_ZERO_ROW: "ZERO_ROW", QL_ERR_NONFINITE: "NONFINITE",
+    QL_ERR_UNSUPPORTED: "UNSUPPORTED", QL_ERR_CUDA: "CUDA", QL_ERR_TIMEOUT: "TIMEOUT",
+}
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqlinear.so")
+
+
+class QLError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {ql_status_string(code)}")
+
+
+class _Optim(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("lr", ctypes.c_float), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float)]
+
+
+class _WeightNorm(ctypes.Structure):
+    _fields_ = [("g", ctypes.c_void_p), ("g_m", ctypes.c_void_p), ("g_v", ctypes.c_void_p)]
+
+
+@dataclass
+class Optim:
+    """Optimizer hyper-parameters of qweight_update_sr (see include/qlinear.h)."""
+    kind: int = QL_ADAMW
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.01
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqlinear.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(
+            f"{library_path} is missing: build it with "
+            "`python -m int8_quantized_act_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(library_path)
+    P, I64, I, U, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint, ctypes.c_float
+    L.ql_status_string.restype = ctypes.c_char_p
+    L.ql_status_string.argtypes = [I]
+    L.qlinear_workspace_bytes.restype = ctypes.c_size_t
+    L.qlinear_workspace_bytes.argtypes = [I64, I64, I64, I]
+    L.qlinear_quantize_rows.restype = I
+    L.qlinear_quantize_rows.argtypes = [P, I, I64, I64, I64, P, I, U, P, I64, P, P, P]
+    L.qlinear_hadamard.restype = I
+    L.qlinear_hadamard.argtypes = [P, I, I64, P, I, I64, I64, I64, I, P]
+    L.qlinear_fwd.restype = I
+    L.qlinear_fwd.argtypes = [P, I, I64, I64, P, P, I64, P, I, P, I, P, P, P, P]
+    L.qlinear_bwd_dx.restype = I
+    L.qlinear_bwd_dx.argtypes = [P, I, I64, I64, P, P, I64, I, P, I, P, ctypes.c_size_t, P, P]
+    L.qlinear_bwd_dw.restype = I
+    L.qlinear_bwd_dw.argtypes = [P, I, I64, I64, P, P, I64, P, P, P, ctypes.c_size_t, P, P]
+    L.ql_set_gemm_timing_events.restype = None
+    L.ql_set_gemm_timing_events.argtypes = [P, P]
+    L.ql_kernel_launches.restype = ctypes.c_uint64
+    L.ql_kernel_launches.argtypes = []
+    L.qweight_update_sr.restype = I
+    L.qweight_update_sr.argtypes = [P, P, P, I64, I64, ctypes.POINTER(_Optim), P, P,
+                                    ctypes.c_uint64, ctypes.c_uint64,
+                                    ctypes.POINTER(_WeightNorm), P, P]
+    _lib = L
+    return L
+
+
+# ------------------------------------------------------------------ helpers
+def _dtype_code(t: torch.Tensor, what: str) -> int:
+    if t.dtype == torch.float32:
+        return QL_F32
+    if t.dtype == torch.bfloat16:
+        return QL_BF16
+    raise TypeError(f"{what}: expected float32 or bfloat16, got {t.dtype}")
+
+
+def _dev(t: Optional[torch.Tensor], what: str, dtype=None):
+    """Device pointer of a CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{what}: expected a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what}: expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _rowmajor(t: torch.Tensor, what: str) -> int:
+    """Leading dimension of a 2-D tensor whose rows are contiguous."""
+    if t.dim() != 2 or (t.size(1) > 1 and t.stride(1) != 1):
+        raise ValueError(f"{what}: expected a 2-D tensor with contiguous rows")
+    return t.stride(0) if t.size(0) > 1 else max(t.stride(0), t.size(1))
+
+
+def _contig(t: Optional[torch.Tensor], what: str):
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{what}: expected a contiguous tensor")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(code: int, where: str):
+    if code != QL_OK:
+        raise QLError(code, where)
+
+
+def ql_status_string(code: int) -> str:
+    return lib().ql_status_string(int(code)).decode()
+
+
+def status_flags(word: int) -> list:
+    """Names of the status bits set in a device status word."""
+    return [name for code, name in _NAMES.items() if code and (int(word) >> code) & 1]
+
+
+def qlinear_workspace_bytes(M: int, N: int, K: int, hadamard_block: int = 0) -> int:
+    return int(lib().qlinear_workspace_bytes(M, N, K, hadamard_block))
+
+
+# ------------------------------------------------------------------ entry points
+def qlinear_quantize_rows(x, q, row_scale, status, col_scale=None, hadamard_block: int = 0,
+                          flags: int = 0, stream=None):
+    """q, row_scale <- per-row int8 quantization of x (optionally x*col_scale,
+    rotated by the block-Hadamard of width hadamard_block)."""
+    rows, cols = x.shape
+    code = lib().qlinear_quantize_rows(
+        _dev(x, "x"), _dtype_code(x, "x"), rows, cols, _rowmajor(x, "x"),
+        _dev(col_scale, "col_scale", torch.float32), hadamard_block, flags,
+        _dev(q, "q", torch.int8), _rowmajor(q, "q"), _dev(row_scale, "row_scale", torch.float32),
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qlinear_quantize_rows")
+
+
+def qlinear_hadamard(x, y, hadamard_block: int, stream=None):
+    """y <- x R (R = block-Hadamard / sqrt(block)); y may be x."""
+    rows, cols = x.shape
+    if tuple(y.shape) != (rows, cols):
+        raise ValueError("qlinear_hadamard: x and y shapes differ")
+    code = lib().qlinear_hadamard(
+        _dev(x, "x"), _dtype_code(x, "x"), _rowmajor(x, "x"), _dev(y, "y"), _dtype_code(y, "y"),
+        _rowmajor(y, "y"), rows, cols, hadamard_block, _stream(stream))
+    _check(code, "qlinear_hadamard")
+
+
+def qlinear_fwd(x, wq, sw, bias, hadamard_block: int, y, xq_saved, sx_saved, status,
+                stream=None):
+    """y <- forward of the layer; xq_saved, sx_saved <- the int8 input for backward."""
+    M, K = x.shape
+    N = wq.shape[0]
+    for t, n in ((x, "x"), (wq, "wq"), (sw, "sw"), (bias, "bias"), (y, "y"),
+                 (xq_saved, "xq_saved"), (sx_saved, "sx_saved")):
+        _contig(t, n)
+    code = lib().qlinear_fwd(
+        _dev(x, "x"), _dtype_code(x, "x"), M, K, _dev(wq, "wq", torch.int8),
+        _dev(sw, "sw", torch.float32), N, _dev(bias, "bias", torch.float32), hadamard_block,
+        _dev(y, "y"), _dtype_code(y, "y"), _dev(xq_saved, "xq_saved", torch.int8),
+        _dev(sx_saved, "sx_saved", torch.float32), _dev(status, "status", torch.int32),
+        _stream(stream))
+    _check(code, "qlinear_fwd")
+
+
+def qlinear_bwd_dx(dy, wq, sw, hadamard_block: int, dx, ws, status, stream=None):
+    """dx <- input gradient from dY and the int8 weight."""
+    M, N = dy.shape
+    K = wq.shape[1]
+    for t, n in ((dy, "dy"), (wq, "wq"), (sw, "sw"), (dx, "dx")):
+        _contig(t, n)
+    code = lib().qlinear_bwd_dx(
+        _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(wq, "wq", torch.int8),
+        _dev(sw, "sw", torch.float32), K, hadamard_block, _dev(dx, "dx"), _dtype_code(dx, "dx"),
+        _dev(ws, "ws", torch.uint8), ws.numel(), _dev(status, "status", torch.int32),
+        _stream(stream))
+    _check(code, "qlinear_bwd_dx")
+
+
+def qlinear_bwd_dw(dy, xq, sx, dw, db, ws, status, stream=None):
+    """dw (float32 [N,K]), db (float32 [N] or None) <- weight/bias gradients."""
+    M, N = dy.shape
+    K = xq.shape[1]
+    for t, n in ((dy, "dy"), (xq, "xq"), (sx, "sx"), (dw, "dw"), (db, "db")):
+        _contig(t, n)
+    code = lib().qlinear_bwd_dw(
+        _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(xq, "xq", torch.int8),
+        _dev(sx, "sx", torch.float32), K, _dev(dw, "dw", torch.float32),
+        _dev(db, "db", torch.float32), _dev(ws, "ws", torch.uint8), ws.numel(),
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qlinear_bwd_dw")
+
+
+def qweight_update_sr(wq, sw, grad, opt: Optim, m, v, seed: int, step: int, status,
+                      g=None, g_m=None, g_v=None, stream=None):
+    """One optimizer step of the int8 weight with stochastic requantization,
+    in place (wq, sw, m, v and, for weight norm, g, g_m, g_v)."""
+    N, K = wq.shape
+    for t, n in ((wq, "wq"), (sw, "sw"), (grad, "grad"), (m, "m"), (v, "v")):
+        _contig(t, n)
+    o = _Optim(int(opt.kind), float(opt.lr), float(opt.beta1), float(opt.beta2),
+               float(opt.eps), float(opt.weight_decay))
+    wn = None
+    if g is not None:
+        wn = ctypes.pointer(_WeightNorm(_dev(g, "g", torch.float32), _dev(g_m, "g_m", torch.float32),
+                                        _dev(g_v, "g_v", torch.float32)))
+    code = lib().qweight_update_sr(
+        _dev(wq, "wq", torch.int8), _dev(sw, "sw", torch.float32), _dev(grad, "grad", torch.float32),
+        N, K, ctypes.byref(o), _dev(m, "m", torch.float32), _dev(v, "v", torch.float32),
+        int(seed), int(step), wn, _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qweight_update_sr")
+
+
+def ql_set_gemm_timing_events(before=None, after=None):
+    """Record these torch.cuda.Event objects around every int8 GEMM launch of
+    this thread (None, None to stop).  Each event must have been recorded once
+    before (torch creates the underlying CUDA event lazily)."""
+    b = None if before is None else before.cuda_event
+    a = None if after is None else after.cuda_event
+    lib().ql_set_gemm_timing_events(b, a)
+
+
+def ql_kernel_launches() -> int:
+    """CUDA kernels launched by the library in this process so far."""
+    return int(lib().ql_kernel_launches())

@@ -1,0 +1,435 @@
+// gemm_i8.cu - int8 x int8 -> int32 GEMM on the sm_100a tensor cores
+// (tcgen05.mma.kind::i8) with the layer's scale/bias epilogues.
+//
+// One kernel serves the three products of the layer (the north-star
+// formulas; OneTrainer PR #1681 uses torch._int_mm for the forward one):
+//   forward  y  = X_q W_q^T      A = X_q   [M,K] K-major,  B = W_q [N,K] K-major
+//   input    dX = dYq_r W_q      A = dYq_r [M,N] K-major,  B = W_q [N,K] MN-major
+//   weight   dW = dYq_c^T X_q    A = dYq_c [M,N] MN-major, B = X_q [M,K] MN-major
+// tcgen05 reads 8-bit operands in either major-ness, so no transposed copy
+// of any operand is ever written.
+//
+// Structure (persistent, one CTA per SM, 6 warps):
+//   warp 0      TMA producer: 128x128-byte A tile + 256x128-byte B tile per
+//               stage into a 4-stage ring of 128B-swizzled shared memory.
+//   warp 1      allocates 512 TMEM columns (two 128x256 int32 accumulators),
+//               one elected thread issues tcgen05.mma (M=128, N=256, K=32)
+//               and tcgen05.commit to release ring stages / hand accumulators
+//               to the epilogue.
+//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, scale, bias,
+//               optional in-register block-Hadamard, 128-bit global stores;
+//               they drain one accumulator while the MMA fills the other.
+// Tiles whose rows / columns / contraction run past the matrix are zero-
+// filled by TMA, so M has no floor and tails need no special path.
+// No TMA multicast is used anywhere.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "launch.h"
+#include "sm100.cuh"
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+namespace {
+
+constexpr int BM = 128;                // tile rows (TMEM lanes)
+constexpr int BN = 256;                // tile columns (TMEM columns per accumulator)
+constexpr int BK = 128;                // contraction bytes per stage (4 MMAs of K=32)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK;       // 16 KiB
+constexpr int B_BYTES = BN * BK;       // 32 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 2 * BN;      // 512: the whole TMEM of the SM
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+
+struct Epi {
+  void* out;
+  int64_t ldo;
+  int rows, cols;
+  const float* row_scale;
+  const float* col_scale;
+  const float* bias;
+  float hc;
+};
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N % 32 == 0, "chunks of 32 columns");
+#pragma unroll
+  for (int j = 0; j < N / 32; ++j)
+    tmem_ld32(taddr + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * j]));
+}
+
+// In-register block-Hadamard along one thread's row segment: blocks of HB
+// consecutive values, butterflies h = 1..HB/2 in order, then times hc.
+template <int N, int HB>
+__device__ __forceinline__ void fwht_regs(float (&v)[N], float hc) {
+#pragma unroll
+  for (int h = 1; h < HB; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < N; ++i) v[i] = v[i] * hc;
+}
+
+__device__ __forceinline__ void store16(float* p, const float* v) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    reinterpret_cast<float4*>(p)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+}
+
+__device__ __forceinline__ void store16(__nv_bfloat16* p, const float* v) {
+  reinterpret_cast<uint4*>(p)[0] =
+      make_uint4(bf16x2(v[0], v[1]), bf16x2(v[2], v[3]), bf16x2(v[4], v[5]), bf16x2(v[6], v[7]));
+  reinterpret_cast<uint4*>(p)[1] = make_uint4(bf16x2(v[8], v[9]), bf16x2(v[10], v[11]),
+                                              bf16x2(v[12], v[13]), bf16x2(v[14], v[15]));
+}
+
+template <bool A_MN, bool B_MN, typename OutT, int HB>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   int tiles_m, int tiles_n, int kblocks, Epi ep, int32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = tiles_m * tiles_n;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, issued = 0, issued_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int tm = t / tiles_n, tn = t % tiles_n;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
+          if (A_MN) tma_load_2d(a_dst, &tmA, fb, tm * BM, kb * BK);
+          else tma_load_2d(a_dst, &tmA, fb, kb * BK, tm * BM);
+          if (B_MN) {
+            tma_load_2d(b_dst, &tmB, fb, tn * BN, kb * BK);
+            tma_load_2d(b_dst + B_BYTES / 2, &tmB, fb, tn * BN + 128, kb * BK);
+          } else {
+            tma_load_2d(b_dst, &tmB, fb, kb * BK, tn * BN);
+          }
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Every copy issued must have landed before the CTA may exit.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) mbar_wait_drain(full0 + 8 * s, (issued_phase >> s) & 1u);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            // K-major: advance 32 bytes inside the 128-byte swizzle row.
+            // MN-major: advance 32 contraction rows of 128 bytes.
+            const uint64_t a_desc = A_MN ? smem_desc_sw128(a_base + kk * 4096, 16384, 1024)
+                                         : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t b_desc = B_MN ? smem_desc_sw128(b_base + kk * 4096, 16384, 1024)
+                                         : smem_desc_sw128(b_base + kk * 32, 16, 1024);
+            mma_i8(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(tfull0 + 8 * acc);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // All issued MMAs must be complete before TMEM is released.
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    constexpr int CH = HB > 32 ? HB : 32;  // columns per register chunk
+    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
+    const int row_local = quarter * 32 + lane;
+    uint32_t acc = 0, acc_phase = 0;
+    OutT* out = reinterpret_cast<OutT*>(ep.out);
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int tm = t / tiles_n, tn = t % tiles_n;
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int gr = tm * BM + row_local;
+      const bool row_ok = gr < ep.rows;
+      const float rs = (row_ok && ep.row_scale) ? ep.row_scale[gr] : 1.0f;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += CH) {
+        uint32_t r[CH];
+        tmem_ld_cols<CH>(taddr + c0, r);
+        tmem_wait_ld();
+        const int gc0 = tn * BN + c0;
+        if (row_ok && gc0 < ep.cols) {
+          float v[CH];
+#pragma unroll
+          for (int i = 0; i < CH; ++i) v[i] = __int2float_rn(static_cast<int>(r[i])) * rs;
+          if (ep.col_scale || ep.bias) {
+#pragma unroll
+            for (int g = 0; g < CH / 16; ++g) {
+              if (gc0 + 16 * g < ep.cols) {
+                if (ep.col_scale) {
+#pragma unroll
+                  for (int i = 0; i < 16; i += 4) {
+                    const float4 c4 = __ldg(reinterpret_cast<const float4*>(ep.col_scale + gc0 + 16 * g + i));
+                    v[16 * g + i] = v[16 * g + i] * c4.x;
+                    v[16 * g + i + 1] = v[16 * g + i + 1] * c4.y;
+                    v[16 * g + i + 2] = v[16 * g + i + 2] * c4.z;
+                    v[16 * g + i + 3] = v[16 * g + i + 3] * c4.w;
+                  }
+                }
+                if (ep.bias) {
+#pragma unroll
+                  for (int i = 0; i < 16; i += 4) {
+                    const float4 b4 = __ldg(reinterpret_cast<const float4*>(ep.bias + gc0 + 16 * g + i));
+                    v[16 * g + i] = v[16 * g + i] + b4.x;
+                    v[16 * g + i + 1] = v[16 * g + i + 1] + b4.y;
+                    v[16 * g + i + 2] = v[16 * g + i + 2] + b4.z;
+                    v[16 * g + i + 3] = v[16 * g + i + 3] + b4.w;
+                  }
+                }
+              }
+            }
+          }
+          if constexpr (HB > 0) fwht_regs<CH, HB>(v, ep.hc);
+          OutT* orow = out + static_cast<int64_t>(gr) * ep.ldo + gc0;
+#pragma unroll
+          for (int g = 0; g < CH / 16; ++g)
+            if (gc0 + 16 * g < ep.cols) store16(orow + 16 * g, v + 16 * g);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(status, 1 << QL_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ host
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D int8 tensor [outer][inner] with the given row pitch; boxes of
+// box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+               uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool A_MN, bool B_MN, typename OutT, int HB>
+cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
+                int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
+  auto kern = gemm_i8_kernel<A_MN, B_MN, OutT, HB>;
+  // Opt in to the large dynamic shared memory once per device.
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !__atomic_load_n(&configured[dev], __ATOMIC_ACQUIRE)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    __atomic_store_n(&configured[dev], 1, __ATOMIC_RELEASE);
+  }
+  const int tiles = tiles_m * tiles_n;
+  const int sms = device_info().sms;
+  const int grid = tiles < sms ? tiles : sms;
+  cudaEvent_t before = nullptr, after = nullptr;
+  gemm_timing_events(&before, &after);
+  if (before) cudaEventRecord(before, s);
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, ep, status);
+  cudaError_t e = cudaGetLastError();
+  if (after) cudaEventRecord(after, s);
+  count_launches(1);
+  return e;
+}
+
+cudaError_t dispatch_dx(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
+                        int kblocks, const Epi& ep, bool bf16, int hb, int32_t* status,
+                        cudaStream_t s) {
+#define QL_RUN(T, H) return run<false, true, T, H>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s)
+  if (bf16) {
+    switch (hb) {
+      case 0: QL_RUN(__nv_bfloat16, 0);
+      case 2: QL_RUN(__nv_bfloat16, 2);
+      case 4: QL_RUN(__nv_bfloat16, 4);
+      case 8: QL_RUN(__nv_bfloat16, 8);
+      case 16: QL_RUN(__nv_bfloat16, 16);
+      case 32: QL_RUN(__nv_bfloat16, 32);
+      case 64: QL_RUN(__nv_bfloat16, 64);
+      case 128: QL_RUN(__nv_bfloat16, 128);
+    }
+  } else {
+    switch (hb) {
+      case 0: QL_RUN(float, 0);
+      case 2: QL_RUN(float, 2);
+      case 4: QL_RUN(float, 4);
+      case 8: QL_RUN(float, 8);
+      case 16: QL_RUN(float, 16);
+      case 32: QL_RUN(float, 32);
+      case 64: QL_RUN(float, 64);
+      case 128: QL_RUN(float, 128);
+    }
+  }
+#undef QL_RUN
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
+                           int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
+                           const GemmEpilogue& e, int32_t* status, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  const bool ok_a = a_mn ? make_tmap(&ta, A, rows, kc, lda, 128, BK)
+                         : make_tmap(&ta, A, kc, rows, lda, BK, BM);
+  const bool ok_b = b_mn ? make_tmap(&tb, B, cols, kc, ldb, 128, BK)
+                         : make_tmap(&tb, B, kc, cols, ldb, BK, BN);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+  Epi ep;
+  ep.out = e.out;
+  ep.ldo = e.ldo;
+  ep.rows = static_cast<int>(rows);
+  ep.cols = static_cast<int>(cols);
+  ep.row_scale = e.row_scale;
+  ep.col_scale = e.col_scale;
+  ep.bias = e.bias;
+  ep.hc = e.hc;
+  const int tiles_m = static_cast<int>((rows + BM - 1) / BM);
+  const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
+  const int kblocks = static_cast<int>((kc + BK - 1) / BK);
+  const bool bf16 = e.out_bf16 != 0;
+  // The layer's three products: forward (K-major x K-major), input gradient
+  // (K-major x MN-major, optional fused rotation), weight gradient
+  // (MN-major x MN-major, float32 out).
+  if (!a_mn && !b_mn && e.hb == 0) {
+    if (bf16) return run<false, false, __nv_bfloat16, 0>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+    return run<false, false, float, 0>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+  }
+  if (!a_mn && b_mn) return dispatch_dx(ta, tb, tiles_m, tiles_n, kblocks, ep, bf16, e.hb, status, s);
+  if (a_mn && b_mn && e.hb == 0 && !bf16)
+    return run<true, true, float, 0>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ql

@@ -1,0 +1,83 @@
+// launch.h - host-side launchers of the CUDA kernels, called by the C ABI
+// (qlinear_api.cu) after it has validated every argument.  Each returns the
+// launch's cudaError_t; none allocates, none synchronizes.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace ql {
+
+struct DeviceInfo {
+  int sms = 0;
+};
+const DeviceInfo& device_info();  // current device, cached
+
+// Launch accounting (ql_kernel_launches) and the GEMM timing events
+// (ql_set_gemm_timing_events) of the calling thread.
+void count_launches(int n);
+void gemm_timing_events(cudaEvent_t* before, cudaEvent_t* after);
+
+// -------------------------------------------------------------- row kernels
+// Per-row quantization (optionally scaled per column and rotated); see
+// qlinear_quantize_rows.  xt: 0 = float32, 1 = bf16.
+cudaError_t launch_quant_rows(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,
+                              const float* col_scale, int B, float hc, unsigned flags,
+                              int8_t* q, int64_t ldq, float* row_scale, int32_t* status,
+                              cudaStream_t s);
+
+// y = x R per row (x may equal y).  xt / yt: 0 = float32, 1 = bf16.
+cudaError_t launch_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt, int64_t ldy,
+                            int64_t rows, int64_t cols, int B, float hc, cudaStream_t s);
+
+// Column statistics of t = dY[m,n]*s_x[m]: colmax[n] = bits of max|t|
+// (atomicMax; caller zeroes), colsum[n] += sum_m dY[m,n] in float64.
+cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
+                            uint32_t* colmax, double* colsum, int32_t* status, cudaStream_t s);
+
+// s2[n] = amax/127, inv2[n] = 127/amax (0 for a zero column), db[n] = colsum.
+cudaError_t launch_colfinalize(const uint32_t* colmax, const double* colsum, int64_t N,
+                               float* s2, float* inv2, float* db, cudaStream_t s);
+
+// dYq_c[m,n] = clamp(rne((dY[m,n]*s_x[m]) * inv2[n]), +-127).
+cudaError_t launch_colquant(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
+                            const float* inv2, int8_t* q, cudaStream_t s);
+
+// out[r, :] = bias (or 0), dtype ot; used when the contraction is empty.
+cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, const float* bias,
+                             cudaStream_t s);
+
+// -------------------------------------------------------------- GEMM
+// out[r, c] = ((float)acc[r,c] * row_scale[r]) * col_scale[c] + bias[c]
+// (each factor optional), then an optional in-register block-Hadamard of
+// width hb (0 or 2..128) along c; acc = int8 x int8 -> int32 on tcgen05.
+struct GemmEpilogue {
+  void* out = nullptr;
+  int out_bf16 = 0;
+  int64_t ldo = 0;
+  const float* row_scale = nullptr;
+  const float* col_scale = nullptr;
+  const float* bias = nullptr;
+  int hb = 0;
+  float hc = 1.0f;
+};
+
+// A: rows x contraction, K-major ([rows][kc], pitch lda bytes) or MN-major
+// ([kc][rows], pitch lda).  B likewise with `cols`.  rows, cols >= 1, kc >= 1.
+cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
+                           int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
+                           const GemmEpilogue& ep, int32_t* status, cudaStream_t s);
+
+// -------------------------------------------------------------- update
+struct UpdateConsts {
+  int kind = 0;  // 0 SGD, 1 AdamW
+  float lr = 0, a = 1, st = 0, bc2 = 1, b1 = 0, b2 = 0, omb1 = 0, omb2 = 0, eps = 0;
+};
+
+cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,
+                             const UpdateConsts& c, float* m, float* v, uint64_t seed,
+                             uint64_t step, float* g, float* g_m, float* g_v, int32_t* status,
+                             cudaStream_t s);
+
+}  // namespace ql

@@ -1,0 +1,315 @@
+// qlinear_api.cu - the extern "C" entry points declared in include/qlinear.h.
+// Each validates its arguments on the host (returning before any launch, so
+// no output is touched on error) and then launches the kernels of
+// rowops.cu, gemm_i8.cu and update_sr.cu on the caller's stream.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "launch.h"
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+const DeviceInfo& device_info() {
+  static DeviceInfo infos[64];
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  std::call_once(once[dev], [dev] {
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    infos[dev].sms = sms > 0 ? sms : 1;
+  });
+  return infos[dev];
+}
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+thread_local cudaEvent_t t_before = nullptr;
+thread_local cudaEvent_t t_after = nullptr;
+}  // namespace
+
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+void gemm_timing_events(cudaEvent_t* before, cudaEvent_t* after) {
+  *before = t_before;
+  *after = t_after;
+}
+
+}  // namespace ql
+
+namespace {
+
+using ql::GemmEpilogue;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool valid_dtype(int t) { return t == QL_F32 || t == QL_BF16; }
+
+inline int64_t elem_size(int t) { return t == QL_BF16 ? 2 : 4; }
+
+inline bool valid_block(int B) { return B == 0 || (B >= 2 && B <= 256 && (B & (B - 1)) == 0); }
+
+// c = 1/sqrt(B) computed in float64 and rounded once to float32.
+inline float hadamard_c(int B) { return B > 0 ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(B))) : 1.0f; }
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? QL_OK : QL_ERR_CUDA; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace carve-up shared by the two backward calls.
+struct WsLayout {
+  size_t dyq, s1, colmax, s2, inv2, colsum, dxtmp, total;
+};
+
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int B) {
+  WsLayout L;
+  size_t off = 0;
+  L.dyq = off;    off += align256(static_cast<size_t>(M) * static_cast<size_t>(N));
+  L.s1 = off;     off += align256(4 * static_cast<size_t>(M > 0 ? M : 1));
+  L.colmax = off; off += align256(4 * static_cast<size_t>(N > 0 ? N : 1));
+  L.s2 = off;     off += align256(4 * static_cast<size_t>(N > 0 ? N : 1));
+  L.inv2 = off;   off += align256(4 * static_cast<size_t>(N > 0 ? N : 1));
+  L.colsum = off; off += align256(8 * static_cast<size_t>(N > 0 ? N : 1));
+  L.dxtmp = off;
+  if (B > 128) off += align256(4 * static_cast<size_t>(M) * static_cast<size_t>(K));
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(base) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+void ql_set_gemm_timing_events(void* before, void* after) {
+  ql::t_before = reinterpret_cast<cudaEvent_t>(before);
+  ql::t_after = reinterpret_cast<cudaEvent_t>(after);
+}
+
+uint64_t ql_kernel_launches(void) { return ql::g_launches.load(std::memory_order_relaxed); }
+
+const char* ql_status_string(int status) {
+  switch (status) {
+    case QL_OK: return "QL_OK";
+    case QL_ERR_ARG: return "QL_ERR_ARG: invalid argument";
+    case QL_ERR_SHAPE: return "QL_ERR_SHAPE: invalid shape, block size or workspace size";
+    case QL_ERR_ALIGN: return "QL_ERR_ALIGN: pointer or pitch not 16-byte aligned";
+    case QL_ERR_ZERO_ROW: return "QL_ERR_ZERO_ROW: rejected all-zero row";
+    case QL_ERR_NONFINITE: return "QL_ERR_NONFINITE: inf or NaN in the input";
+    case QL_ERR_UNSUPPORTED: return "QL_ERR_UNSUPPORTED: size beyond the supported range";
+    case QL_ERR_CUDA: return "QL_ERR_CUDA: CUDA runtime error";
+    case QL_ERR_TIMEOUT: return "QL_ERR_TIMEOUT: device wait timed out";
+    default: return "unknown ql_status";
+  }
+}
+
+size_t qlinear_workspace_bytes(int64_t M, int64_t N, int64_t K, int hadamard_block) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return ws_layout(M, N, K, hadamard_block).total;
+}
+
+int qlinear_quantize_rows(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,
+                          const float* col_scale, int hadamard_block, unsigned flags, int8_t* q,
+                          int64_t ldq, float* row_scale, int32_t* d_status, void* stream) {
+  if (!valid_dtype(xt) || !valid_block(hadamard_block) || (flags & ~QL_REJECT_ZERO_ROWS))
+    return QL_ERR_ARG;
+  if (rows < 0 || cols < 0 || cols % 16 != 0 || ldx < cols || ldq < cols || ldq % 16 != 0 ||
+      cols > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (hadamard_block > 0 && cols % hadamard_block != 0) return QL_ERR_SHAPE;
+  if (rows == 0) return QL_OK;
+  if (!x || !q || !row_scale || !d_status) return QL_ERR_ARG;
+  if (!aligned16(x) || !aligned16(q) || (ldx * elem_size(xt)) % 16 != 0 ||
+      (col_scale && !aligned16(col_scale)))
+    return QL_ERR_ALIGN;
+  return cuda_status(ql::launch_quant_rows(x, xt, rows, cols, ldx, col_scale, hadamard_block,
+                                           hadamard_c(hadamard_block), flags, q, ldq, row_scale,
+                                           d_status, as_stream(stream)));
+}
+
+int qlinear_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt, int64_t ldy,
+                     int64_t rows, int64_t cols, int hadamard_block, void* stream) {
+  if (!valid_dtype(xt) || !valid_dtype(yt) || !valid_block(hadamard_block) || hadamard_block == 0)
+    return QL_ERR_ARG;
+  if (rows < 0 || cols < 0 || cols % 16 != 0 || cols % hadamard_block != 0 || ldx < cols ||
+      ldy < cols || cols > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return QL_OK;
+  if (!x || !y) return QL_ERR_ARG;
+  if (x == y && (xt != yt || ldx != ldy)) return QL_ERR_ARG;
+  if (!aligned16(x) || !aligned16(y) || (ldx * elem_size(xt)) % 16 != 0 ||
+      (ldy * elem_size(yt)) % 16 != 0)
+    return QL_ERR_ALIGN;
+  return cuda_status(ql::launch_hadamard(x, xt, ldx, y, yt, ldy, rows, cols, hadamard_block,
+                                         hadamard_c(hadamard_block), as_stream(stream)));
+}
+
+int qlinear_fwd(const void* x, int xt, int64_t M, int64_t K, const int8_t* wq, const float* sw,
+                int64_t N, const float* bias, int hadamard_block, void* y, int yt,
+                int8_t* xq_saved, float* sx_saved, int32_t* d_status, void* stream) {
+  if (!valid_dtype(xt) || !valid_dtype(yt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || M > INT32_MAX ||
+      N > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
+  if (K > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
+  if (M == 0) return QL_OK;
+  // With K == 0 the input, codes and weight are empty (possibly NULL).
+  if (!sx_saved || !d_status || (K > 0 && (!x || !xq_saved)) ||
+      (N > 0 && (!y || (K > 0 && (!wq || !sw)))))
+    return QL_ERR_ARG;
+  if ((K > 0 && (!aligned16(x) || !aligned16(xq_saved))) ||
+      (N > 0 && (!aligned16(y) || (K > 0 && (!aligned16(wq) || !aligned16(sw))))) ||
+      (bias && !aligned16(bias)))
+    return QL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = ql::launch_quant_rows(x, xt, M, K, K, nullptr, hadamard_block,
+                                        hadamard_c(hadamard_block), 0u, xq_saved, K, sx_saved,
+                                        d_status, s);
+  if (e != cudaSuccess || N == 0) return cuda_status(e);
+  if (K == 0) return cuda_status(ql::launch_fill_rows(y, yt, M, N, bias, s));
+  GemmEpilogue ep;
+  ep.out = y;
+  ep.out_bf16 = yt == QL_BF16;
+  ep.ldo = N;
+  ep.row_scale = sx_saved;
+  ep.col_scale = sw;
+  ep.bias = bias;
+  return cuda_status(ql::launch_gemm_i8(xq_saved, false, K, wq, false, K, M, N, K, ep, d_status, s));
+}
+
+int qlinear_bwd_dx(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
+                   const float* sw, int64_t K, int hadamard_block, void* dx, int dxt, void* ws,
+                   size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (!valid_dtype(dyt) || !valid_dtype(dxt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || M > INT32_MAX ||
+      K > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
+  if (N > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
+  if (M == 0 || K == 0) return QL_OK;
+  const WsLayout L = ws_layout(M, N, K, hadamard_block);
+  if (!dx || !d_status || !ws || (N > 0 && (!dy || !wq || !sw))) return QL_ERR_ARG;
+  if (ws_bytes < L.total) return QL_ERR_SHAPE;
+  if (!aligned16(dx) || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
+      (N > 0 && (!aligned16(dy) || !aligned16(wq) || !aligned16(sw))))
+    return QL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  if (N == 0) {  // empty contraction: dX = 0
+    return cuda_status(cudaMemsetAsync(dx, 0, static_cast<size_t>(M * K * elem_size(dxt)), s));
+  }
+  int8_t* dyq = at<int8_t>(ws, L.dyq);
+  float* s1 = at<float>(ws, L.s1);
+  cudaError_t e = ql::launch_quant_rows(dy, dyt, M, N, N, sw, 0, 1.0f, 0u, dyq, N, s1, d_status, s);
+  if (e != cudaSuccess) return QL_ERR_CUDA;
+  GemmEpilogue ep;
+  ep.row_scale = s1;
+  ep.ldo = K;
+  if (hadamard_block > 128) {
+    // Blocks wider than a thread's register chunk: write the float32 product
+    // (to dx itself when it is float32) and rotate it in a second pass.
+    float* tmp = dxt == QL_F32 ? reinterpret_cast<float*>(dx) : at<float>(ws, L.dxtmp);
+    ep.out = tmp;
+    ep.out_bf16 = 0;
+    e = ql::launch_gemm_i8(dyq, false, N, wq, true, K, M, K, N, ep, d_status, s);
+    if (e != cudaSuccess) return QL_ERR_CUDA;
+    return cuda_status(ql::launch_hadamard(tmp, QL_F32, K, dx, dxt, K, M, K, hadamard_block,
+                                           hadamard_c(hadamard_block), s));
+  }
+  ep.out = dx;
+  ep.out_bf16 = dxt == QL_BF16;
+  ep.hb = hadamard_block;
+  ep.hc = hadamard_c(hadamard_block);
+  return cuda_status(ql::launch_gemm_i8(dyq, false, N, wq, true, K, M, K, N, ep, d_status, s));
+}
+
+int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* xq,
+                   const float* sx, int64_t K, float* dw, float* db, void* ws, size_t ws_bytes,
+                   int32_t* d_status, void* stream) {
+  if (!valid_dtype(dyt)) return QL_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || N > INT32_MAX || K > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (M > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
+  if (N == 0) return QL_OK;
+  const WsLayout L = ws_layout(M, N, K, 0);
+  if (!d_status || !ws || (K > 0 && !dw) || (M > 0 && (!dy || !xq || !sx))) return QL_ERR_ARG;
+  if (ws_bytes < L.total) return QL_ERR_SHAPE;
+  if ((dw && !aligned16(dw)) || (db && !aligned16(db)) || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
+      (M > 0 && (!aligned16(dy) || !aligned16(xq) || !aligned16(sx))))
+    return QL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  if (M == 0) {  // empty contraction: dW = 0, db = 0
+    if (K > 0 && cudaMemsetAsync(dw, 0, static_cast<size_t>(N * K) * 4, s) != cudaSuccess)
+      return QL_ERR_CUDA;
+    if (db && cudaMemsetAsync(db, 0, static_cast<size_t>(N) * 4, s) != cudaSuccess)
+      return QL_ERR_CUDA;
+    return QL_OK;
+  }
+  uint32_t* colmax = at<uint32_t>(ws, L.colmax);
+  double* colsum = at<double>(ws, L.colsum);
+  float* s2 = at<float>(ws, L.s2);
+  float* inv2 = at<float>(ws, L.inv2);
+  int8_t* dyq = at<int8_t>(ws, L.dyq);
+  if (cudaMemsetAsync(colmax, 0, static_cast<size_t>(N) * 4, s) != cudaSuccess ||
+      cudaMemsetAsync(colsum, 0, static_cast<size_t>(N) * 8, s) != cudaSuccess)
+    return QL_ERR_CUDA;
+  cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, d_status, s);
+  if (e == cudaSuccess) e = ql::launch_colfinalize(colmax, colsum, N, s2, inv2, db, s);
+  if (e == cudaSuccess) e = ql::launch_colquant(dy, dyt, M, N, sx, inv2, dyq, s);
+  if (e != cudaSuccess || K == 0) return cuda_status(e);
+  GemmEpilogue ep;
+  ep.out = dw;
+  ep.ldo = K;
+  ep.row_scale = s2;
+  return cuda_status(ql::launch_gemm_i8(dyq, true, N, xq, true, K, N, K, M, ep, d_status, s));
+}
+
+int qweight_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,
+                      const ql_optim* opt, float* m, float* v, uint64_t seed, uint64_t step,
+                      const ql_weightnorm* wn, int32_t* d_status, void* stream) {
+  if (!opt || (opt->kind != QL_SGD && opt->kind != QL_ADAMW) || step < 1) return QL_ERR_ARG;
+  if (opt->kind == QL_SGD && opt->weight_decay != 0.0f) return QL_ERR_ARG;
+  if (!std::isfinite(opt->lr) || (opt->kind == QL_ADAMW &&
+                                  (!(opt->beta1 >= 0.0f && opt->beta1 < 1.0f) ||
+                                   !(opt->beta2 >= 0.0f && opt->beta2 < 1.0f) ||
+                                   !std::isfinite(opt->eps) || !std::isfinite(opt->weight_decay))))
+    return QL_ERR_ARG;
+  if (N < 0 || K < 0 || K % 16 != 0 || N > INT32_MAX) return QL_ERR_SHAPE;
+  if (K > 32768) return QL_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return QL_OK;
+  if (!wq || !sw || !grad || !d_status) return QL_ERR_ARG;
+  if (opt->kind == QL_ADAMW && (!m || !v)) return QL_ERR_ARG;
+  if (wn && (!wn->g || (opt->kind == QL_ADAMW && (!wn->g_m || !wn->g_v)))) return QL_ERR_ARG;
+  if (!aligned16(wq) || !aligned16(grad) || (m && !aligned16(m)) || (v && !aligned16(v)))
+    return QL_ERR_ALIGN;
+  ql::UpdateConsts c;
+  c.kind = opt->kind;
+  c.lr = opt->lr;
+  if (opt->kind == QL_ADAMW) {
+    // Host constants, each computed in float64 and rounded once.
+    const double t = static_cast<double>(step);
+    c.a = static_cast<float>(1.0 - static_cast<double>(opt->lr) * static_cast<double>(opt->weight_decay));
+    c.st = static_cast<float>(static_cast<double>(opt->lr) / (1.0 - std::pow(static_cast<double>(opt->beta1), t)));
+    c.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(opt->beta2), t));
+    c.b1 = opt->beta1;
+    c.b2 = opt->beta2;
+    c.omb1 = static_cast<float>(1.0 - static_cast<double>(opt->beta1));
+    c.omb2 = static_cast<float>(1.0 - static_cast<double>(opt->beta2));
+    c.eps = opt->eps;
+  }
+  return cuda_status(ql::launch_update_sr(wq, sw, grad, N, K, c, m, v, seed, step,
+                                          wn ? wn->g : nullptr, wn ? wn->g_m : nullptr,
+                                          wn ? wn->g_v : nullptr, d_status, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+// rowops.cuh - device helpers shared by the row kernels: 8-wide vector loads
+// and stores of float32 / bf16, the block-Hadamard butterflies of one
+// 256-element chunk held by a warp, and warp reductions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace ql {
+
+// -------------------------------------------------------------- 8-wide I/O
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// bf16 -> float32 is exact: the bf16 bits are the top half of the float.
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return a | (b << 16);
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+// -------------------------------------------------------------- int8 codes
+// Round to nearest even, clamp to [-127, 127].
+__device__ __forceinline__ int code_rne(float t) {
+  float r = rintf(t);
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return static_cast<int>(r);
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+}
+
+// -------------------------------------------------------------- Hadamard
+// Block-Hadamard rotation of one 256-element chunk spread across a warp,
+// lane l holding elements 8l..8l+7 in v.  For blocks of B elements (B a power
+// of two, 2..256) the Sylvester butterflies run for h = 1, 2, ..., B/2 in that
+// order, pair (j, j+h) -> (v_j + v_{j+h}, v_j - v_{j+h}); stages with h < 8
+// stay inside a lane, larger h exchange with lane ^ (h/8).  Then every value
+// is multiplied by c = fl32(1/sqrt(B)).  All 32 lanes must call this.
+__device__ __forceinline__ void fwht_chunk(float (&v)[8], int B, int lane, float c) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+    if (h < B) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if ((i & h) == 0) {
+          const float a = v[i], b = v[i + h];
+          v[i] = a + b;
+          v[i + h] = a - b;
+        }
+      }
+    }
+  }
+  for (int h = 8; h < B; h <<= 1) {
+    const int d = h >> 3;
+    const bool upper = (lane & d) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float p = __shfl_xor_sync(0xFFFFFFFFu, v[i], d);
+      v[i] = upper ? (p - v[i]) : (v[i] + p);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = v[i] * c;
+}
+
+// -------------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
+  return x;
+}
+
+__device__ __forceinline__ int warp_or(int x) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) x |= __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ int warp_sum_i(int x) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ bool finite(float x) { return isfinite(x); }
+
+}  // namespace ql

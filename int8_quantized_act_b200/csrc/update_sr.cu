@@ -1,0 +1,274 @@
+// update_sr.cu - fused optimizer step + stochastic requantization of int8
+// weight rows (mini_trainer "docs/quantized-training.md": the paragraph after
+// the feature table - updates requantize the represented weights
+// stochastically in CUDA row kernels, with no floating master weight; feature
+// table rows "Optimizers" and "Row-wise weight normalization").
+//
+// One CTA owns one weight row.  Thread t holds the 16-element groups
+// t, t+T, t+2T, ... (T = threads, a power of two <= 256) in registers, so the
+// row is read from HBM once: codes, gradient and moments in, new moments out
+// while the updated float row stays in registers; a CTA max-reduction gives
+// the new scale; then each group draws 16 24-bit uniforms from 4 Philox4x32-10
+// blocks and writes 16 stochastically rounded codes with one 128-bit store.
+// Bytes per element: AdamW 22 (1+4+4+4 in, 1+4+4 out), SGD 6.
+#include <cuda_runtime.h>
+
+#include "launch.h"
+#include "rowops.cuh"
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+namespace {
+
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of two
+// 32x32->64 multiplies, key bumped by the Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+__device__ __forceinline__ float adamw(const UpdateConsts& c, float w, float g, float& m,
+                                       float& v) {
+  const float w1 = w * c.a;
+  const float mn = c.b1 * m + c.omb1 * g;
+  const float vn = c.b2 * v + c.omb2 * (g * g);
+  const float den = sqrtf(vn / c.bc2) + c.eps;
+  m = mn;
+  v = vn;
+  return w1 - c.st * (mn / den);
+}
+
+// floor(v) + 1 with probability frac(v), decided by u24 < frac * 2^24.
+__device__ __forceinline__ int sr_code(float val, uint32_t u24) {
+  const float f = floorf(val);
+  const float frac = val - f;
+  float r = (__uint2float_rn(u24) < frac * 16777216.0f) ? f + 1.0f : f;
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return static_cast<int>(r);
+}
+
+__device__ __forceinline__ void load16f(const float* p, float (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 a = reinterpret_cast<const float4*>(p)[i];
+    v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
+  }
+}
+
+__device__ __forceinline__ void store16f(float* p, const float (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    reinterpret_cast<float4*>(p)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+__device__ __forceinline__ int code_at(const uint4& q, int i) {
+  const uint32_t w = (&q.x)[i >> 2];
+  return static_cast<int>(static_cast<int8_t>((w >> (8 * (i & 3))) & 0xFFu));
+}
+
+template <int GPT, bool WN>
+__global__ void __launch_bounds__(256) update_sr_kernel(
+    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
+    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, uint32_t seed_lo,
+    uint32_t seed_hi, uint32_t step_lo, uint32_t step_hi, float* __restrict__ gmag,
+    float* __restrict__ g_m, float* __restrict__ g_v, int32_t* __restrict__ status) {
+  __shared__ float s_red[256];
+  __shared__ int s_ired[8];
+  const int n = blockIdx.x;
+  const int t = threadIdx.x;
+  const int T = blockDim.x;  // power of two, <= 256
+  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
+  const int ngroups = K >> 4;
+  const int64_t row = static_cast<int64_t>(n) * K;
+  const bool adam = c.kind == QL_ADAMW;
+
+  const float s = sw[n];
+  uint4 qv[GPT];
+  float w[GPT][16];
+#pragma unroll
+  for (int i = 0; i < GPT; ++i) {
+    const int j = t + T * i;
+    qv[i] = j < ngroups ? *reinterpret_cast<const uint4*>(wq + row + 16 * j) : make_uint4(0, 0, 0, 0);
+  }
+
+  float dg = 0.0f, nq = 0.0f, coef = 0.0f;
+  if constexpr (WN) {
+    // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31).
+    int ss = 0;
+#pragma unroll
+    for (int i = 0; i < GPT; ++i)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int qc = code_at(qv[i], e);
+        ss += qc * qc;
+      }
+    ss = warp_sum_i(ss);
+    if (lane == 0) s_ired[warp] = ss;
+    __syncthreads();
+    ss = 0;
+    for (int k = 0; k < nwarps; ++k) ss += s_ired[k];
+    if (ss == 0) {  // a zero direction cannot be normalized: reject the row
+      if (t == 0) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+      return;
+    }
+    nq = static_cast<float>(sqrt(static_cast<double>(ss)));
+    // dg in the fixed order: thread t is lane t of 256 virtual lanes, adding
+    // its groups' products in increasing k; lanes >= T hold +0.
+    float p = 0.0f;
+#pragma unroll
+    for (int i = 0; i < GPT; ++i) {
+      const int j = t + T * i;
+      if (j < ngroups) {
+        float gr[16];
+        load16f(grad + row + 16 * j, gr);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) p = p + gr[e] * (static_cast<float>(code_at(qv[i], e)) / nq);
+      }
+    }
+    for (int off = 128; off >= 1; off >>= 1) {
+      if (off >= T) {
+        p = p + 0.0f;
+      } else if (off >= 32) {
+        s_red[t] = p;
+        __syncthreads();
+        const float o = s_red[t ^ off];
+        __syncthreads();
+        p = p + o;
+      } else {
+        p = p + __shfl_xor_sync(0xFFFFFFFFu, p, off);
+      }
+    }
+    dg = p;
+    coef = gmag[n] / (s * nq);
+  }
+
+  // Optimizer step of every element; moments written back immediately.
+  float amax = 0.0f;
+  int bad = 0;
+#pragma unroll
+  for (int i = 0; i < GPT; ++i) {
+    const int j = t + T * i;
+    if (j < ngroups) {
+      const int64_t off = row + 16 * j;
+      float gr[16], m1[16], m2[16];
+      load16f(grad + off, gr);
+      if (adam) {
+        load16f(mom1 + off, m1);
+        load16f(mom2 + off, m2);
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float qf = static_cast<float>(code_at(qv[i], e));
+        float gg = gr[e];
+        if constexpr (WN) gg = coef * (gr[e] - dg * (qf / nq));
+        const float wv = s * qf;
+        w[i][e] = adam ? adamw(c, wv, gg, m1[e], m2[e]) : wv - c.lr * gg;
+        bad |= !finite(w[i][e]);
+        amax = fmaxf(amax, fabsf(w[i][e]));
+      }
+      if (adam) {
+        store16f(mom1 + off, m1);
+        store16f(mom2 + off, m2);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) w[i][e] = 0.0f;
+    }
+  }
+  if constexpr (WN) {
+    if (t == 0) {
+      float gm = gmag[n];
+      if (adam) {
+        float a1 = g_m[n], a2 = g_v[n];
+        gm = adamw(c, gm, dg, a1, a2);
+        g_m[n] = a1;
+        g_v[n] = a2;
+      } else {
+        gm = gm - c.lr * dg;
+      }
+      gmag[n] = gm;
+    }
+  }
+
+  // Row max (also the barrier before the scale is overwritten).
+  amax = warp_max(amax);
+  bad = warp_or(bad);
+  __syncthreads();
+  if (lane == 0) {
+    s_red[warp] = amax;
+    s_ired[warp] = bad;
+  }
+  __syncthreads();
+  amax = 0.0f;
+  bad = 0;
+  for (int k = 0; k < nwarps; ++k) {
+    amax = fmaxf(amax, s_red[k]);
+    bad |= s_ired[k];
+  }
+  const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
+  if (t == 0) {
+    sw[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
+    if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  }
+
+  // Stochastic requantization: element e = n*K + k uses word e&3 of
+  // Philox(counter = (e>>2 lo, e>>2 hi, step lo, step hi), key = seed).
+#pragma unroll
+  for (int i = 0; i < GPT; ++i) {
+    const int j = t + T * i;
+    if (j < ngroups) {
+      const uint64_t blk0 = static_cast<uint64_t>(row + 16 * j) >> 2;
+      int cd[16];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint64_t blk = blk0 + b;
+        const uint4 r = philox10(make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32),
+                                            step_lo, step_hi),
+                                 seed_lo, seed_hi);
+        const uint32_t words[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cd[4 * b + e] = amax == 0.0f ? 0 : sr_code(w[i][4 * b + e] * inv, words[e] >> 8);
+      }
+      *reinterpret_cast<uint4*>(wq + row + 16 * j) =
+          make_uint4(pack4(cd[0], cd[1], cd[2], cd[3]), pack4(cd[4], cd[5], cd[6], cd[7]),
+                     pack4(cd[8], cd[9], cd[10], cd[11]), pack4(cd[12], cd[13], cd[14], cd[15]));
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,
+                             const UpdateConsts& c, float* m, float* v, uint64_t seed,
+                             uint64_t step, float* g, float* g_m, float* g_v, int32_t* status,
+                             cudaStream_t s) {
+  const int ngroups = static_cast<int>(K / 16);
+  int T = 32;
+  while (T < ngroups && T < 256) T <<= 1;
+  const int gpt = (ngroups + T - 1) / T;  // 1..8
+  const uint32_t sl = static_cast<uint32_t>(seed), sh = static_cast<uint32_t>(seed >> 32);
+  const uint32_t tl = static_cast<uint32_t>(step), th = static_cast<uint32_t>(step >> 32);
+  const int k = static_cast<int>(K);
+  const unsigned grid = static_cast<unsigned>(N);
+#define QL_UPD(G, W)                                                                          \
+  update_sr_kernel<G, W><<<grid, T, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, g, g_m, \
+                                            g_v, status)
+  const bool wn = g != nullptr;
+  if (gpt <= 1) { if (wn) QL_UPD(1, true); else QL_UPD(1, false); }
+  else if (gpt <= 2) { if (wn) QL_UPD(2, true); else QL_UPD(2, false); }
+  else if (gpt <= 4) { if (wn) QL_UPD(4, true); else QL_UPD(4, false); }
+  else { if (wn) QL_UPD(8, true); else QL_UPD(8, false); }
+#undef QL_UPD
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace ql

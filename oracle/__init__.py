@@ -63,7 +63,7 @@ def _declare(L):
         "ref_philox4x32_10": (None, [_P, _P, _P]),
         "ref_sr_u24": (_U32, [_U64, _U64, _U64]),
         "ref_update_sr": (_U32, [_P, _P, _P, _I64, _I64, ctypes.c_int, _F, _F, _F, _F, _F,
-                                 _P, _P, _U64, _U64, _P, _P, _P]),
+                                 _P, _P, _U64, _U64, _P, _P, _P, _I64]),
         "ref_update_float": (_U32, [_P, _P, _P, _I64, _I64, ctypes.c_int, _F, _F, _F, _F, _F,
                                     _P, _P, _U64, _P, _P, _P, _P]),
         "ref_sr_expectation_enum": (ctypes.c_double, [_F]),
@@ -227,9 +227,10 @@ SGD, ADAMW = 0, 1
 
 def update_sr(q, s, grad, kind: int, lr: float, seed: int, step: int,
               m=None, v=None, b1=0.9, b2=0.999, eps=1e-8, wd=0.0,
-              g=None, g_m=None, g_v=None):
+              g=None, g_m=None, g_v=None, row0: int = 0):
     """One optimizer step with stochastic requantization; returns the new
-    (q, s, m, v, g, g_m, g_v, status) as copies (inputs are not modified)."""
+    (q, s, m, v, g, g_m, g_v, status) as copies (inputs are not modified).
+    The arrays hold rows row0.. of the weight (row0 keys the random stream)."""
     q, s, grad = _i8(q).copy(), _f32(s).copy(), _f32(grad)
     N, K = q.shape
     m = None if m is None else _f32(m).copy()
@@ -238,7 +239,7 @@ def update_sr(q, s, grad, kind: int, lr: float, seed: int, step: int,
     g_m = None if g_m is None else _f32(g_m).copy()
     g_v = None if g_v is None else _f32(g_v).copy()
     st = lib().ref_update_sr(_p(q), _p(s), _p(grad), N, K, kind, lr, b1, b2, eps, wd,
-                             _p(m), _p(v), seed, step, _p(g), _p(g_m), _p(g_v))
+                             _p(m), _p(v), seed, step, _p(g), _p(g_m), _p(g_v), row0)
     return q, s, m, v, g, g_m, g_v, st
 
 

@@ -559,11 +559,13 @@ uint32_t ref_update_float(const int8_t *q, const float *s, const float *grad, in
 
 /* One optimizer step with stochastic requantization of an int8 [N,K] weight,
  * in place: row_step, then sr_requant_row of the updated row (seed, step).
- * Rows with a zero initial direction are left untouched.  step >= 1. */
+ * Rows with a zero initial direction are left untouched.  step >= 1.
+ * The arrays hold rows n0 .. n0+N-1 of the weight: the row index that keys
+ * the random stream is n0 + n (so a slice of rows can be checked alone). */
 uint32_t ref_update_sr(int8_t *q, float *s, const float *grad, int64_t N, int64_t K,
                        int kind, float lr, float b1, float b2, float eps, float wd,
                        float *m, float *v, uint64_t seed, uint64_t step,
-                       float *g, float *g_m, float *g_v) {
+                       float *g, float *g_m, float *g_v, int64_t n0) {
     uint32_t st = check_update_args(kind, wd, step);
     if (st) return st;
     adamw_consts c = adamw_setup(lr, b1, b2, eps, wd, step);
@@ -574,7 +576,7 @@ uint32_t ref_update_sr(int8_t *q, float *s, const float *grad, int64_t N, int64_
                               m ? m + n * K : NULL, v ? v + n * K : NULL,
                               g, g_m, g_v, w, qhat);
         if (r) { st |= r; continue; }
-        st |= sr_requant_row(w, K, n, seed, step, q + n * K, &s[n]);
+        st |= sr_requant_row(w, K, n0 + n, seed, step, q + n * K, &s[n]);
     }
     free(w);
     free(qhat);

@@ -1,0 +1,115 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads, exports
+every entry point that include/qlinear.h declares, and rejects bad
+arguments on the host before touching the GPU (no launch happens in these
+calls, so they run without a device)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import int8_quantized_act_b200 as ql
+from int8_quantized_act_b200 import build as cuda_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "qlinear.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    cuda_build.build()
+    return ql.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"QL_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert set(names) >= {"qlinear_quantize_rows", "qlinear_hadamard", "qlinear_fwd",
+                          "qlinear_bwd_dx", "qlinear_bwd_dw", "qweight_update_sr",
+                          "ql_status_string", "qlinear_workspace_bytes"}
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(9):
+        assert ql.ql_status_string(code).startswith("QL_")
+    assert ql.status_flags((1 << ql.QL_ERR_ZERO_ROW) | (1 << ql.QL_ERR_TIMEOUT)) == ["ZERO_ROW", "TIMEOUT"]
+
+
+def test_workspace_formula(L):
+    def a(x):
+        return (x + 255) // 256 * 256
+    M, N, K = 12000, 7168, 5376
+    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    assert ql.qlinear_workspace_bytes(M, N, K, 128) == base
+    assert ql.qlinear_workspace_bytes(M, N, K, 256) == base + a(4 * M * K)
+    assert ql.qlinear_workspace_bytes(-1, N, K, 0) == 0
+
+
+P = ctypes.c_void_p
+
+
+def fake(addr):
+    """A pointer value that is never dereferenced: these calls fail validation."""
+    return P(addr)
+
+
+def test_host_validation_returns_before_any_launch(L):
+    A = 0x10000  # 16-byte aligned fake address
+    # bad dtype / block / flags
+    assert L.qlinear_quantize_rows(fake(A), 7, 4, 32, 32, None, 0, 0, fake(A), 32, fake(A), fake(A), None) == ql.QL_ERR_ARG
+    assert L.qlinear_quantize_rows(fake(A), 0, 4, 32, 32, None, 3, 0, fake(A), 32, fake(A), fake(A), None) == ql.QL_ERR_ARG
+    assert L.qlinear_quantize_rows(fake(A), 0, 4, 32, 32, None, 0, 4, fake(A), 32, fake(A), fake(A), None) == ql.QL_ERR_ARG
+    # shapes: cols % 16, cols % block, ldq % 16
+    assert L.qlinear_quantize_rows(fake(A), 0, 4, 40, 40, None, 0, 0, fake(A), 48, fake(A), fake(A), None) == ql.QL_ERR_SHAPE
+    assert L.qlinear_quantize_rows(fake(A), 0, 4, 48, 48, None, 32, 0, fake(A), 48, fake(A), fake(A), None) == ql.QL_ERR_SHAPE
+    assert L.qlinear_quantize_rows(fake(A), 0, 4, 32, 32, None, 0, 0, fake(A), 40, fake(A), fake(A), None) == ql.QL_ERR_SHAPE
+    # null and misaligned pointers
+    assert L.qlinear_quantize_rows(None, 0, 4, 32, 32, None, 0, 0, fake(A), 32, fake(A), fake(A), None) == ql.QL_ERR_ARG
+    assert L.qlinear_quantize_rows(fake(A + 4), 0, 4, 32, 32, None, 0, 0, fake(A), 32, fake(A), fake(A), None) == ql.QL_ERR_ALIGN
+    # zero rows: nothing to do
+    assert L.qlinear_quantize_rows(None, 0, 0, 32, 32, None, 0, 0, None, 32, None, None, None) == ql.QL_OK
+    # forward: contraction limit of the pages, K and N multiples of 16
+    big = 131072
+    assert L.qlinear_fwd(fake(A), 0, 2, big, fake(A), fake(A), 32, None, 0, fake(A), 0, fake(A), fake(A), fake(A), None) == ql.QL_ERR_UNSUPPORTED
+    assert L.qlinear_fwd(fake(A), 0, 2, 40, fake(A), fake(A), 32, None, 0, fake(A), 0, fake(A), fake(A), fake(A), None) == ql.QL_ERR_SHAPE
+    assert L.qlinear_fwd(fake(A), 0, 2, 32, fake(A), fake(A), 24, None, 0, fake(A), 0, fake(A), fake(A), fake(A), None) == ql.QL_ERR_SHAPE
+    assert L.qlinear_fwd(fake(A), 0, 2, 32, fake(A), fake(A), 32, fake(A + 8), 0, fake(A), 0, fake(A), fake(A), fake(A), None) == ql.QL_ERR_ALIGN
+    # backward: workspace too small, contraction limit
+    assert L.qlinear_bwd_dx(fake(A), 0, 4, 32, fake(A), fake(A), 32, 0, fake(A), 0, fake(0x100000), 16, fake(A), None) == ql.QL_ERR_SHAPE
+    assert L.qlinear_bwd_dx(fake(A), 0, 4, big, fake(A), fake(A), 32, 0, fake(A), 0, fake(A), 1 << 30, fake(A), None) == ql.QL_ERR_UNSUPPORTED
+    assert L.qlinear_bwd_dw(fake(A), 0, big, 32, fake(A), fake(A), 32, fake(A), None, fake(A), 1 << 30, fake(A), None) == ql.QL_ERR_UNSUPPORTED
+    assert L.qlinear_bwd_dw(fake(A), 0, 4, 32, fake(A), fake(A), 32, fake(A), None, fake(A + 16), 1 << 30, fake(A), None) == ql.QL_ERR_ALIGN
+    # hadamard: in place needs the same dtype and pitch
+    assert L.qlinear_hadamard(fake(A), 0, 32, fake(A), 1, 32, 4, 32, 16, None) == ql.QL_ERR_ARG
+    assert L.qlinear_hadamard(fake(A), 0, 32, fake(A), 0, 32, 4, 32, 0, None) == ql.QL_ERR_ARG
+
+
+def test_update_validation(L):
+    A = 0x10000
+    opt = ql._Optim(ql.QL_SGD, 0.1, 0.9, 0.999, 1e-8, 0.5)
+    f = L.qweight_update_sr
+    assert f(fake(A), fake(A), fake(A), 4, 32, ctypes.byref(opt), None, None, 0, 1, None, fake(A), None) == ql.QL_ERR_ARG
+    opt = ql._Optim(ql.QL_ADAMW, 1e-3, 0.9, 1.5, 1e-8, 0.0)
+    assert f(fake(A), fake(A), fake(A), 4, 32, ctypes.byref(opt), fake(A), fake(A), 0, 1, None, fake(A), None) == ql.QL_ERR_ARG
+    opt = ql._Optim(ql.QL_ADAMW, 1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert f(fake(A), fake(A), fake(A), 4, 32, ctypes.byref(opt), fake(A), fake(A), 0, 0, None, fake(A), None) == ql.QL_ERR_ARG
+    assert f(fake(A), fake(A), fake(A), 4, 40, ctypes.byref(opt), fake(A), fake(A), 0, 1, None, fake(A), None) == ql.QL_ERR_SHAPE
+    assert f(fake(A), fake(A), fake(A), 4, 32784, ctypes.byref(opt), fake(A), fake(A), 0, 1, None, fake(A), None) == ql.QL_ERR_UNSUPPORTED
+    assert f(fake(A), fake(A), fake(A), 4, 32, ctypes.byref(opt), None, fake(A), 0, 1, None, fake(A), None) == ql.QL_ERR_ARG
+    assert f(fake(A + 8), fake(A), fake(A), 4, 32, ctypes.byref(opt), fake(A), fake(A), 0, 1, None, fake(A), None) == ql.QL_ERR_ALIGN
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros((4, 32))
+    with pytest.raises(TypeError):
+        ql.qlinear_quantize_rows(x, torch.zeros((4, 32), dtype=torch.int8), torch.zeros(4),
+                                 torch.zeros(1, dtype=torch.int32))

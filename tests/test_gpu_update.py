@@ -1,0 +1,149 @@
+"""GPU parity of the fused optimizer step + stochastic requantization against
+the oracle, through the C ABI.  New codes, scales, moments and (for weight
+norm) magnitudes must be bit-exact: both sides evaluate the same float32
+operations in the same order and draw the same Philox4x32-10 words."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import int8_quantized_act_b200 as ql
+from parity_util import dev, host, new_status, status_word
+
+pytestmark = pytest.mark.gpu
+
+
+def prepared(d):
+    q, s, st = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    assert st == 0
+    return q, s
+
+
+def run_gpu(q, s, grad, kind, lr, seed, step, m=None, v=None, wd=0.0, g=None, g_m=None,
+            g_v=None):
+    tq, ts, tg = dev(q), dev(s), dev(grad)
+    tm = dev(m) if m is not None else None
+    tv = dev(v) if v is not None else None
+    tgm = [dev(a) if a is not None else None for a in (g, g_m, g_v)]
+    st = new_status()
+    opt = ql.Optim(kind=kind, lr=lr, weight_decay=wd)
+    ql.qweight_update_sr(tq, ts, tg, opt, tm, tv, seed, step, st, g=tgm[0], g_m=tgm[1], g_v=tgm[2])
+    word = status_word(st)
+    out = [host(tq), host(ts), host(tm) if tm is not None else None,
+           host(tv) if tv is not None else None] + [host(a) if a is not None else None for a in tgm]
+    return out, word
+
+
+def check_equal(gpu, ref, names):
+    for a, b, n in zip(gpu, ref, names):
+        if b is None:
+            continue
+        assert a.shape == b.shape, n
+        bad = a.view(np.uint8) != b.view(np.uint8) if a.dtype != np.int8 else a != b
+        assert not bad.any(), f"{n}: {int(bad.sum())} elements differ"
+
+
+NAMES = ["codes", "scales", "m", "v", "g", "g_m", "g_v"]
+
+
+@pytest.mark.parametrize("N,K", [(128, 256), (64, 1024), (33, 5376), (16, 16384), (8, 32768),
+                                 (40, 400), (5, 16)])
+def test_sgd_update_bit_exact(N, K):
+    d = workloads.update_state(N, K, seed=N)
+    q, s = prepared(d)
+    gpu, st = run_gpu(q, s, d["grad"], ql.QL_SGD, 1e-2, seed=0, step=1)
+    ref = oracle.update_sr(q, s, d["grad"], oracle.SGD, 1e-2, seed=0, step=1)
+    assert st == 0 and ref[-1] == 0
+    check_equal(gpu[:2], ref[:2], NAMES)
+
+
+@pytest.mark.parametrize("warm", [False, True])
+@pytest.mark.parametrize("N,K", [(64, 1024), (48, 4096), (24, 14336), (16, 16384), (100, 272)])
+def test_adamw_update_bit_exact(N, K, warm):
+    d = workloads.update_state(N, K, seed=K + warm, warm=warm)
+    q, s = prepared(d)
+    seed = 0x1234_5678_9ABC
+    gpu, st = run_gpu(q, s, d["grad"], ql.QL_ADAMW, 1e-3, seed, d["step"], m=d["m"], v=d["v"],
+                      wd=0.01)
+    ref = oracle.update_sr(q, s, d["grad"], oracle.ADAMW, 1e-3, seed, d["step"], m=d["m"],
+                           v=d["v"], wd=0.01)
+    assert st == 0 and ref[-1] == 0
+    check_equal(gpu[:4], ref[:4], NAMES)
+
+
+@pytest.mark.parametrize("kind", [ql.QL_ADAMW, ql.QL_SGD])
+@pytest.mark.parametrize("N,K", [(32, 1024), (12, 4096), (6, 16384), (20, 80)])
+def test_weight_norm_update_bit_exact(N, K, kind):
+    d = workloads.update_state(N, K, seed=3 * K, weight_norm=True)
+    q, s = prepared(d)
+    adam = kind == ql.QL_ADAMW
+    kw = dict(m=d["m"], v=d["v"], wd=0.01) if adam else {}
+    gpu, st = run_gpu(q, s, d["grad"], kind, 1e-3, 99, 1, g=d["g"],
+                      g_m=d["g_m"] if adam else None, g_v=d["g_v"] if adam else None, **kw)
+    ref = oracle.update_sr(q, s, d["grad"], kind, 1e-3, 99, 1, g=d["g"],
+                           g_m=d["g_m"] if adam else None, g_v=d["g_v"] if adam else None, **kw)
+    assert st == 0 and ref[-1] == 0
+    check_equal(gpu, ref[:7], NAMES)
+
+
+def test_weight_norm_zero_direction_flagged_and_untouched():
+    d = workloads.update_state(6, 512, seed=5, weight_norm=True)
+    q, s = prepared(d)
+    q[2] = 0
+    s[2] = 0
+    gpu, st = run_gpu(q, s, d["grad"], ql.QL_ADAMW, 1e-3, 1, 1, m=d["m"], v=d["v"], g=d["g"],
+                      g_m=d["g_m"], g_v=d["g_v"])
+    ref = oracle.update_sr(q, s, d["grad"], oracle.ADAMW, 1e-3, 1, 1, m=d["m"], v=d["v"],
+                           g=d["g"], g_m=d["g_m"], g_v=d["g_v"])
+    assert st == (1 << ql.QL_ERR_ZERO_ROW) and ref[-1] == oracle.BIT_ZERO_ROW
+    check_equal(gpu, ref[:7], NAMES)
+
+
+@pytest.mark.parametrize("n", [4096, 16384])
+def test_adamw_full_size_sampled_rows(n):
+    """The [n, n] sweep sizes: the whole matrix updates on the GPU; sampled
+    rows are recomputed by the oracle (its random stream keyed by the
+    absolute row)."""
+    w = workloads.normal((n, n), 0.02, 71)
+    g = workloads.normal((n, n), 1e-3, 72)
+    tw = dev(w)
+    tq = torch.empty((n, n), dtype=torch.int8, device="cuda")
+    ts = torch.empty(n, dtype=torch.float32, device="cuda")
+    st = new_status()
+    ql.qlinear_quantize_rows(tw, tq, ts, st, flags=ql.QL_REJECT_ZERO_ROWS)
+    q0, s0 = host(tq), host(ts)
+    del tw
+    tm = torch.zeros((n, n), device="cuda")
+    tv = torch.zeros((n, n), device="cuda")
+    ql.qweight_update_sr(tq, ts, dev(g), ql.Optim(), tm, tv, 7, 1, st)
+    assert status_word(st) == 0
+    rows = np.array(sorted({0, 1, n // 2, n - 1} | set(
+        np.random.Generator(np.random.PCG64(n)).integers(0, n, 12).tolist())))
+    q1, s1 = host(tq), host(ts)
+    m1, v1 = host(tm[rows]), host(tv[rows])
+    for r in rows:
+        ref = oracle.update_sr(q0[r:r + 1], s0[r:r + 1], g[r:r + 1], oracle.ADAMW, 1e-3, 7, 1,
+                               m=np.zeros((1, n), np.float32), v=np.zeros((1, n), np.float32),
+                               wd=0.01, row0=int(r))
+        i = int(np.searchsorted(rows, r))
+        check_equal([q1[r:r + 1], s1[r:r + 1], m1[i:i + 1], v1[i:i + 1]], ref[:4], NAMES)
+
+
+def test_update_argument_errors():
+    q = torch.zeros((4, 32), dtype=torch.int8, device="cuda")
+    s = torch.ones(4, device="cuda")
+    g = torch.zeros((4, 32), device="cuda")
+    st = new_status()
+    with pytest.raises(ql.QLError) as e:
+        ql.qweight_update_sr(q, s, g, ql.Optim(kind=ql.QL_SGD, weight_decay=0.1), None, None, 0, 1, st)
+    assert e.value.code == ql.QL_ERR_ARG
+    with pytest.raises(ql.QLError) as e:
+        ql.qweight_update_sr(q, s, g, ql.Optim(kind=ql.QL_SGD, weight_decay=0.0), None, None, 0, 0, st)
+    assert e.value.code == ql.QL_ERR_ARG
+    with pytest.raises(ql.QLError) as e:
+        ql.qweight_update_sr(q, s, g, ql.Optim(), None, None, 0, 1, st)  # AdamW needs m, v
+    assert e.value.code == ql.QL_ERR_ARG
+    assert status_word(st) == 0
