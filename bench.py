@@ -39,6 +39,21 @@ WORKLOAD = ("qlinear train step: M=12000 K=5376 N=7168, Hadamard block 128, bf16
             "fwd + dX + dW + AdamW stochastic requant")
 NOMINAL_INT8_OVER_BF16 = 2.0   # dense int8 4.5 POPS / dense bf16 2.25 PFLOPS
 
+# DRAM bytes (read + write) per GEMM launch from the ncu capture summarised in
+# profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
+# weight-gradient launches), valid only for the GEMM source it was taken on.
+GEMM_TRAFFIC_BYTES = 409.6e6
+GEMM_TRAFFIC_SOURCE_SHA = "d50591545ba02a0c"
+
+
+def gemm_source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_i8.cu", "sm100.cuh"):
+        with open(os.path.join(ROOT, "int8_quantized_act_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
 
 def parse_args():
     p = argparse.ArgumentParser()
@@ -302,7 +317,9 @@ def run_ours(args, rank, world, local):
                      "frac": round(gemm_tops / int8_peak, 4),
                      "peak_source": f"{peaks['source']}: bf16 dense burst x {NOMINAL_INT8_OVER_BF16} (int8/bf16 nominal ratio)",
                      "ms_per_launch": {k: round(v, 4) for k, v in per_kind.items()},
-                     "traffic": None},
+                     "traffic": (GEMM_TRAFFIC_BYTES if gemm_source_sha() == GEMM_TRAFFIC_SOURCE_SHA
+                                 else None),
+                     "traffic_unit": "bytes per launch"},
         "row_kernel": {"kernel": "update_sr (AdamW + stochastic requant)", "bound": "hbm",
                        "achieved": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9, 1),
                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
