@@ -202,6 +202,39 @@ QL_API int qweight_update_sr(int8_t *wq, float *sw, const float *grad, int64_t N
                       uint64_t seed, uint64_t step, const ql_weightnorm *wn,
                       int32_t *d_status, void *stream);
 
+/* Capacity of the library-owned scratch used by qlinear_bwd_dx_noalloc:
+ * 32 MiB of device memory. */
+#define QL_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* qlinear_bwd_dx_noalloc - the input gradient of qlinear_bwd_dx, for callers
+ * that cannot allocate device memory and so cannot supply the `ws` buffer:
+ * code running inside a host framework that owns all device memory and
+ * forbids allocation while its kernels execute, or a process whose device
+ * memory is fully reserved by another allocator.  (This entry point is an
+ * interface convenience; the pages have no counterpart.)
+ *
+ * Arguments, results and errors are those of qlinear_bwd_dx without ws and
+ * ws_bytes.  Instead of a caller buffer it uses a scratch array of
+ * QL_NOALLOC_SCRATCH_BYTES that lives in the library's own device image: it
+ * is not allocated by any call, and every GPU that loads the library's
+ * device code holds it until the process exits.  Sizes whose workspace,
+ * qlinear_workspace_bytes(M, N, K, hadamard_block), exceeds that capacity are
+ * rejected with QL_ERR_UNSUPPORTED before anything runs (for example
+ * M = 2048, N = 7168 fits; M = 12000, N = 7168 does not).
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress, once per device, thread-safe); make that
+ * first call before any stream capture.  All calls in the process share the
+ * one array and it keeps whatever the last call left in it; nothing in it
+ * needs to start at zero, because every byte this call reads was written
+ * earlier in the same call.  Calls that may overlap on the GPU (different
+ * streams, or different host threads on one device) race on the array:
+ * order them, e.g. issue them on one stream.  The call allocates nothing. */
+QL_API int qlinear_bwd_dx_noalloc(const void *dy, int dyt, int64_t M, int64_t N,
+                                  const int8_t *wq, const float *sw, int64_t K,
+                                  int hadamard_block, void *dx, int dxt,
+                                  int32_t *d_status, void *stream);
+
 /* Instrumentation (no effect on results).
  * ql_set_gemm_timing_events: while set (non-NULL), every int8 GEMM kernel that
  * the calling host thread launches records the cudaEvent_t `before` on its

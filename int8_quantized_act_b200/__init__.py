@@ -27,6 +27,7 @@ __all__ = [
     "ql_status_string", "qlinear_workspace_bytes", "qlinear_quantize_rows",
     "qlinear_hadamard", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
     "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
+    "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES",
 ]
 
 QL_OK, QL_ERR_ARG, QL_ERR_SHAPE, QL_ERR_ALIGN = 0, 1, 2, 3
@@ -36,6 +37,7 @@ QL_F32, QL_BF16 = 0, 1
 QL_SGD, QL_ADAMW = 0, 1
 QL_REJECT_ZERO_ROWS = 1
 QL_MAX_CONTRACTION = 131071
+QL_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _NAMES = {
     QL_OK: "OK", QL_ERR_ARG: "ARG", QL_ERR_SHAPE: "SHAPE", QL_ERR_ALIGN: "ALIGN",
@@ -101,6 +103,8 @@ def lib() -> ctypes.CDLL:
     L.qlinear_bwd_dx.argtypes = [P, I, I64, I64, P, P, I64, I, P, I, P, ctypes.c_size_t, P, P]
     L.qlinear_bwd_dw.restype = I
     L.qlinear_bwd_dw.argtypes = [P, I, I64, I64, P, P, I64, P, P, P, ctypes.c_size_t, P, P]
+    L.qlinear_bwd_dx_noalloc.restype = I
+    L.qlinear_bwd_dx_noalloc.argtypes = [P, I, I64, I64, P, P, I64, I, P, I, P, P]
     L.ql_set_gemm_timing_events.restype = None
     L.ql_set_gemm_timing_events.argtypes = [P, P]
     L.ql_kernel_launches.restype = ctypes.c_uint64
@@ -223,6 +227,23 @@ def qlinear_bwd_dx(dy, wq, sw, hadamard_block: int, dx, ws, status, stream=None)
         _dev(ws, "ws", torch.uint8), ws.numel(), _dev(status, "status", torch.int32),
         _stream(stream))
     _check(code, "qlinear_bwd_dx")
+
+
+def qlinear_bwd_dx_noalloc(dy, wq, sw, hadamard_block: int, dx, status, stream=None):
+    """qlinear_bwd_dx for callers that cannot allocate device memory: no
+    workspace argument; the library's own fixed scratch (QL_NOALLOC_SCRATCH_BYTES)
+    is used instead, shared by all calls in the process (calls that may
+    overlap on the GPU race on it).  Sizes that need more scratch raise
+    QLError(QL_ERR_UNSUPPORTED)."""
+    M, N = dy.shape
+    K = wq.shape[1]
+    for t, n in ((dy, "dy"), (wq, "wq"), (sw, "sw"), (dx, "dx")):
+        _contig(t, n)
+    code = lib().qlinear_bwd_dx_noalloc(
+        _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(wq, "wq", torch.int8),
+        _dev(sw, "sw", torch.float32), K, hadamard_block, _dev(dx, "dx"), _dtype_code(dx, "dx"),
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qlinear_bwd_dx_noalloc")
 
 
 def qlinear_bwd_dw(dy, xq, sx, dw, db, ws, status, stream=None):
