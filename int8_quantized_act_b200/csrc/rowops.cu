@@ -10,6 +10,7 @@
 // warp shuffles.  Rows whose chunks fit in registers are read from HBM once.
 #include "launch.h"
 #include "rowops.cuh"
+#include "sm100.cuh"
 #include "../../include/qlinear.h"
 
 namespace ql {
@@ -24,6 +25,8 @@ __device__ __forceinline__ const T* row_ptr(const void* base, int64_t r, int64_t
 // ---------------------------------------------------------------------------
 // Quantize rows whose chunks fit in registers: WPR warps per row, CPW chunks
 // per warp (WPR * CPW * 256 >= cols).  CTA = 8 warps = 8/WPR rows at a time.
+// The row max is carried as |x| bit patterns (abs_bits), which also flags
+// inf/NaN; codes are rounded through the float adder (rne_bits).
 template <typename InT, int CPW, int WPR>
 __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
     const InT* __restrict__ x, int64_t rows, int cols, int64_t ldx,
@@ -31,8 +34,7 @@ __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
     int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
     int32_t* __restrict__ status) {
   constexpr int RPC = 8 / WPR;
-  __shared__ float s_max[8];
-  __shared__ int s_bad[8];
+  __shared__ uint32_t s_max[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp / WPR, wir = warp % WPR;
   for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * RPC; r0 < rows;
@@ -40,11 +42,11 @@ __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
     const int64_t r = r0 + slot;
     const bool rv = r < rows;
     float v[CPW][8];
-    float amax = 0.0f;
-    int bad = 0;
+    uint32_t mbits = 0;
 #pragma unroll
     for (int j = 0; j < CPW; ++j) {
-      const int col = (wir + j * WPR) * 256 + lane * 8;
+      const int chunk0 = (wir + j * WPR) * 256;  // same for the whole warp
+      const int col = chunk0 + lane * 8;
       if (rv && col < cols) {
         load8(x + r * ldx + col, v[j]);
         if (col_scale) {
@@ -57,56 +59,167 @@ __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[j][i] = 0.0f;
       }
-      if (B > 0) fwht_chunk(v[j], B, lane, hc);
+      if (B > 0 && rv && chunk0 < cols) fwht_chunk(v[j], B, lane, hc);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        bad |= !finite(v[j][i]);
-        amax = fmaxf(amax, fabsf(v[j][i]));
-      }
+      for (int i = 0; i < 8; ++i) mbits = max(mbits, abs_bits(v[j][i]));
     }
-    amax = warp_max(amax);
-    bad = warp_or(bad);
+    mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
     if (WPR > 1) {
-      if (lane == 0) {
-        s_max[warp] = amax;
-        s_bad[warp] = bad;
-      }
+      if (lane == 0) s_max[warp] = mbits;
       __syncthreads();
 #pragma unroll
-      for (int w = 0; w < WPR; ++w) {
-        amax = fmaxf(amax, s_max[slot * WPR + w]);
-        bad |= s_bad[slot * WPR + w];
-      }
+      for (int w = 0; w < WPR; ++w) mbits = max(mbits, s_max[slot * WPR + w]);
       __syncthreads();
     }
     if (rv) {
-      if (amax == 0.0f) {
+      const float amax = __uint_as_float(mbits);
+      const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
 #pragma unroll
-        for (int j = 0; j < CPW; ++j) {
-          const int col = (wir + j * WPR) * 256 + lane * 8;
-          if (col < cols) *reinterpret_cast<uint2*>(q + r * ldq + col) = make_uint2(0u, 0u);
+      for (int j = 0; j < CPW; ++j) {
+        const int col = (wir + j * WPR) * 256 + lane * 8;
+        if (col < cols) {
+          uint32_t b[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) b[i] = rne_bits(v[j][i] * inv);
+          *reinterpret_cast<uint2*>(q + r * ldq + col) =
+              make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
         }
-        if (wir == 0 && lane == 0) {
-          row_scale[r] = 0.0f;
-          if (flags & QL_REJECT_ZERO_ROWS) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
-        }
-      } else {
-        const float inv = 127.0f / amax;
+      }
+      if (wir == 0 && lane == 0) {
+        row_scale[r] = mbits == 0 ? 0.0f : amax / 127.0f;
+        if (mbits == 0 && (flags & QL_REJECT_ZERO_ROWS)) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+        if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Quantize rows staged in shared memory by the bulk-copy engine: a persistent
+// CTA (8 warps) walks rows r = blockIdx.x + i * gridDim.x through a ring of
+// `stages` row buffers, so several rows per CTA are in flight without holding
+// registers; each warp then takes chunks wir, wir + 8, ... (CPW of them) of the
+// staged row, exactly as the register kernel does.  Waits are bounded: on a
+// time-out the CTA reports QL_ERR_TIMEOUT, lets its copies land and returns.
+template <typename InT, int CPW>
+__global__ void __launch_bounds__(256) quant_rows_tma_kernel(
+    const InT* __restrict__ x, int64_t rows, int cols, int64_t ldx,
+    const float* __restrict__ col_scale, int B, float hc, unsigned flags,
+    int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
+    int32_t* __restrict__ status, int stages, int stage_bytes) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint32_t s_max[8];
+  __shared__ __align__(8) uint64_t s_full[8];
+  __shared__ volatile int s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t row_bytes = static_cast<uint32_t>(cols) * sizeof(InT);
+  const int64_t mine = rows > blockIdx.x ? (rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < stages; ++st) mbar_init(smem_u32(&s_full[st]), 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < stages && st < mine; ++st) {
+      const int64_t r = blockIdx.x + static_cast<int64_t>(st) * gridDim.x;
+      mbar_arrive_expect_tx(smem_u32(&s_full[st]), row_bytes);
+      bulk_load(smem_u32(smem + st * stage_bytes), x + r * ldx, row_bytes, smem_u32(&s_full[st]));
+    }
+  }
+  // A lane owns the same columns in every row: keep their scales in registers.
+  float cs[CPW][8];
 #pragma unroll
-        for (int j = 0; j < CPW; ++j) {
-          const int col = (wir + j * WPR) * 256 + lane * 8;
-          if (col < cols) {
-            int c[8];
+  for (int j = 0; j < CPW; ++j) {
+    const int col = (warp + 8 * j) * 256 + lane * 8;
+    if (col_scale && col < cols) {
+      load8(col_scale + col, cs[j]);
+    } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) c[i] = code_rne(v[j][i] * inv);
-            *reinterpret_cast<uint2*>(q + r * ldq + col) =
-                make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+      for (int e = 0; e < 8; ++e) cs[j][e] = 1.0f;
+    }
+  }
+  int64_t done = 0;
+  for (int64_t i = 0; i < mine; ++i) {
+    const int st = static_cast<int>(i % stages);
+    const uint32_t parity = static_cast<uint32_t>((i / stages) & 1);
+    const int64_t r = blockIdx.x + i * gridDim.x;
+    // A thread that gives up (mbar_wait raises s_abort) still takes part in
+    // both barriers below; the CTA leaves the loop together after the second.
+    const bool ok = mbar_wait(smem_u32(&s_full[st]), parity, &s_abort);
+    const InT* xs = reinterpret_cast<const InT*>(smem + st * stage_bytes);
+    float v[CPW][8];
+    uint32_t mbits = 0;
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) {
+      const int chunk0 = (warp + 8 * j) * 256;
+      const int col = chunk0 + lane * 8;
+      if (ok && col < cols) {
+        if constexpr (sizeof(InT) == 4) {
+          const float4 a = reinterpret_cast<const float4*>(xs + col)[0];
+          const float4 b = reinterpret_cast<const float4*>(xs + col)[1];
+          v[j][0] = a.x; v[j][1] = a.y; v[j][2] = a.z; v[j][3] = a.w;
+          v[j][4] = b.x; v[j][5] = b.y; v[j][6] = b.z; v[j][7] = b.w;
+        } else {
+          const uint4 u = *reinterpret_cast<const uint4*>(xs + col);
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[j][2 * e] = __uint_as_float(w4[e] << 16);
+            v[j][2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
           }
         }
-        if (wir == 0 && lane == 0) row_scale[r] = amax / 127.0f;
+        if (col_scale) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[j][e] = v[j][e] * cs[j][e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[j][e] = 0.0f;
       }
-      if (bad && wir == 0 && lane == 0) atomicOr(status, 1 << QL_ERR_NONFINITE);
+      if (B > 0 && chunk0 < cols) fwht_chunk(v[j], B, lane, hc);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mbits = max(mbits, abs_bits(v[j][e]));
     }
+    mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+    if (lane == 0) s_max[warp] = mbits;
+    __syncthreads();  // every thread is done reading stage st
+    if (threadIdx.x == 0 && i + stages < mine && !s_abort) {
+      fence_proxy_async_smem();
+      const int64_t rn = blockIdx.x + (i + stages) * gridDim.x;
+      mbar_arrive_expect_tx(smem_u32(&s_full[st]), row_bytes);
+      bulk_load(smem_u32(smem + st * stage_bytes), x + rn * ldx, row_bytes, smem_u32(&s_full[st]));
+    }
+#pragma unroll
+    for (int w = 0; w < 8; ++w) mbits = max(mbits, s_max[w]);
+    __syncthreads();  // s_max may be rewritten by the next row
+    if (s_abort) break;
+    const float amax = __uint_as_float(mbits);
+    const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) {
+      const int col = (warp + 8 * j) * 256 + lane * 8;
+      if (col < cols) {
+        uint32_t b[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) b[e] = rne_bits(v[j][e] * inv);
+        *reinterpret_cast<uint2*>(q + r * ldq + col) =
+            make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
+      }
+    }
+    if (threadIdx.x == 0) {
+      row_scale[r] = mbits == 0 ? 0.0f : amax / 127.0f;
+      if (mbits == 0 && (flags & QL_REJECT_ZERO_ROWS)) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+      if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    }
+    done = i + 1;
+  }
+  if (threadIdx.x == 0 && s_abort) {
+    // Timed out: let every copy already issued (rows done .. done+stages-1)
+    // land before the CTA exits.
+    atomicOr(status, 1 << QL_ERR_TIMEOUT);
+    for (int64_t i = done; i < mine && i < done + stages; ++i)
+      mbar_wait_drain(smem_u32(&s_full[i % stages]), static_cast<uint32_t>((i / stages) & 1));
   }
 }
 
@@ -114,82 +227,65 @@ __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
 // Quantize long rows (more chunks than fit in registers): one CTA per row,
 // two passes over the row (the second re-reads it, normally from L2).
 template <typename InT>
+__device__ __forceinline__ void load_chunk(const InT* xr, const float* cs, int col, int cols,
+                                           float (&v)[8]) {
+  if (col < cols) {
+    load8(xr + col, v);
+    if (cs) {
+      float c8[8];
+      load8(cs + col, c8);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = v[i] * c8[i];
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+  }
+}
+
+template <typename InT>
 __global__ void __launch_bounds__(256) quant_rows_stream_kernel(
     const InT* __restrict__ x, int64_t rows, int cols, int64_t ldx,
     const float* __restrict__ col_scale, int B, float hc, unsigned flags,
     int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
     int32_t* __restrict__ status) {
-  __shared__ float s_max[8];
-  __shared__ int s_bad[8];
+  __shared__ uint32_t s_max[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunks = (cols + 255) / 256;
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    float amax = 0.0f;
-    int bad = 0;
+    uint32_t mbits = 0;
+    for (int ch = warp; ch < nchunks; ch += 8) {
+      float v[8];
+      load_chunk(x + r * ldx, col_scale, ch * 256 + lane * 8, cols, v);
+      if (B > 0) fwht_chunk(v, B, lane, hc);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mbits = max(mbits, abs_bits(v[i]));
+    }
+    mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+    if (lane == 0) s_max[warp] = mbits;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < 8; ++w) mbits = max(mbits, s_max[w]);
+    __syncthreads();
+    const float amax = __uint_as_float(mbits);
+    const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
     for (int ch = warp; ch < nchunks; ch += 8) {
       const int col = ch * 256 + lane * 8;
       float v[8];
-      if (col < cols) {
-        load8(x + r * ldx + col, v);
-        if (col_scale) {
-          float c8[8];
-          load8(col_scale + col, c8);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = v[i] * c8[i];
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      }
-      if (B > 0) fwht_chunk(v, B, lane, hc);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        bad |= !finite(v[i]);
-        amax = fmaxf(amax, fabsf(v[i]));
-      }
-    }
-    amax = warp_max(amax);
-    bad = warp_or(bad);
-    if (lane == 0) {
-      s_max[warp] = amax;
-      s_bad[warp] = bad;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      amax = fmaxf(amax, s_max[w]);
-      bad |= s_bad[w];
-    }
-    __syncthreads();
-    const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
-    for (int ch = warp; ch < nchunks; ch += 8) {
-      const int col = ch * 256 + lane * 8;
-      float v[8];
-      if (col < cols) {
-        load8(x + r * ldx + col, v);
-        if (col_scale) {
-          float c8[8];
-          load8(col_scale + col, c8);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = v[i] * c8[i];
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      }
+      load_chunk(x + r * ldx, col_scale, col, cols, v);
       if (B > 0) fwht_chunk(v, B, lane, hc);
       if (col < cols) {
-        int c[8];
+        uint32_t b[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) c[i] = amax == 0.0f ? 0 : code_rne(v[i] * inv);
+        for (int i = 0; i < 8; ++i) b[i] = rne_bits(v[i] * inv);
         *reinterpret_cast<uint2*>(q + r * ldq + col) =
-            make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+            make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
       }
     }
     if (threadIdx.x == 0) {
-      row_scale[r] = amax == 0.0f ? 0.0f : amax / 127.0f;
-      if (amax == 0.0f && (flags & QL_REJECT_ZERO_ROWS)) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
-      if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
+      row_scale[r] = mbits == 0 ? 0.0f : amax / 127.0f;
+      if (mbits == 0 && (flags & QL_REJECT_ZERO_ROWS)) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+      if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
     }
   }
 }
@@ -246,53 +342,59 @@ __global__ void __launch_bounds__(256) colstats_kernel(const InT* __restrict__ d
                                                        uint32_t* __restrict__ colmax,
                                                        double* __restrict__ colsum,
                                                        int32_t* __restrict__ status) {
-  __shared__ float s_max[8][256];
+  __shared__ uint32_t s_max[8][256];
   __shared__ double s_sum[8][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int col = blockIdx.x * 256 + lane * 8;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kColSlab;
   const int64_t m1 = m0 + kColSlab < M ? m0 + kColSlab : M;
-  float mx[8];
-  double sm[8];
+  // Each thread sums at most kColSlab/8 = 16 values of a column in float32
+  // (relative error ~1e-6 of the column's sum of magnitudes); the slab
+  // partials are combined in float64.
+  uint32_t mx[8];
+  float smf[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    mx[i] = 0.0f;
-    sm[i] = 0.0;
+    mx[i] = 0;
+    smf[i] = 0.0f;
   }
-  int bad = 0;
   if (col < N) {
+#pragma unroll 4
     for (int64_t m = m0 + warp; m < m1; m += 8) {
       float d[8];
       load8(dy + m * N + col, d);
       const float s = __ldg(sx + m);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float t = d[i] * s;
-        bad |= !finite(t);
-        mx[i] = fmaxf(mx[i], fabsf(t));
-        sm[i] += static_cast<double>(d[i]);
+        mx[i] = max(mx[i], abs_bits(d[i] * s));
+        smf[i] += d[i];
       }
     }
   }
+  double sm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sm[i] = static_cast<double>(smf[i]);
+  // Transposed writes (column-major in the slab) keep the banks apart.
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    s_max[warp][lane * 8 + i] = mx[i];
-    s_sum[warp][lane * 8 + i] = sm[i];
+    s_max[warp][i * 32 + lane] = mx[i];
+    s_sum[warp][i * 32 + lane] = sm[i];
   }
-  bad = warp_or(bad);
-  if (bad && lane == 0) atomicOr(status, 1 << QL_ERR_NONFINITE);
   __syncthreads();
-  const int c = threadIdx.x;  // one column per thread
+  const int c = threadIdx.x;  // one column per thread: column c is lane c/8, element c%8
+  const int slotc = (c % 8) * 32 + c / 8;
   if (blockIdx.x * 256 + c < N) {
-    float a = 0.0f;
+    uint32_t a = 0;
     double t = 0.0;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
-      a = fmaxf(a, s_max[w][c]);
-      t += s_sum[w][c];
+      a = max(a, s_max[w][slotc]);
+      t += s_sum[w][slotc];
     }
-    // max of non-negative floats = max of their bit patterns
-    atomicMax(colmax + blockIdx.x * 256 + c, __float_as_uint(a));
+    // inf/NaN patterns sort above every finite value: report and let them
+    // through (the column's outputs are then unspecified).
+    if (a >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    atomicMax(colmax + blockIdx.x * 256 + c, a);
     atomicAdd(colsum + blockIdx.x * 256 + c, t);
   }
 }
@@ -308,33 +410,28 @@ __global__ void colfinalize_kernel(const uint32_t* __restrict__ colmax,
   if (db) db[n] = static_cast<float>(colsum[n]);
 }
 
-// One thread per 16 consecutive columns of one row.
+// Column quantization: block (x, y) owns the 2048-column segment y (8
+// columns per thread, their 127/amax factors kept in registers) and walks the
+// rows x, x + gridDim.x, ...
 template <typename InT>
 __global__ void __launch_bounds__(256) colquant_kernel(const InT* __restrict__ dy, int64_t M,
                                                        int N, const float* __restrict__ sx,
                                                        const float* __restrict__ inv2,
                                                        int8_t* __restrict__ q) {
-  const int per_row = N / 16;
-  const int64_t total = M * per_row;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
-       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t m = t / per_row;
-    const int col = static_cast<int>(t % per_row) * 16;
-    float d0[8], d1[8], i0[8], i1[8];
-    load8(dy + m * N + col, d0);
-    load8(dy + m * N + col + 8, d1);
-    load8(inv2 + col, i0);
-    load8(inv2 + col + 8, i1);
+  const int col = blockIdx.y * 2048 + threadIdx.x * 8;
+  if (col >= N) return;
+  float iv[8];
+  load8(inv2 + col, iv);
+#pragma unroll 4
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    float d[8];
+    load8(dy + m * N + col, d);
     const float s = __ldg(sx + m);
-    int c[16];
+    uint32_t b[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      c[i] = code_rne((d0[i] * s) * i0[i]);
-      c[8 + i] = code_rne((d1[i] * s) * i1[i]);
-    }
-    *reinterpret_cast<uint4*>(q + m * N + col) =
-        make_uint4(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]),
-                   pack4(c[8], c[9], c[10], c[11]), pack4(c[12], c[13], c[14], c[15]));
+    for (int i = 0; i < 8; ++i) b[i] = rne_bits((d[i] * s) * iv[i]);
+    *reinterpret_cast<uint2*>(q + m * N + col) =
+        make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
   }
 }
 
@@ -365,7 +462,35 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
   const InT* x = reinterpret_cast<const InT*>(xv);
   const int nch = static_cast<int>((cols + 255) / 256);
   const int c = static_cast<int>(cols);
-  if (nch <= 64) {
+  const int64_t row_bytes = cols * static_cast<int64_t>(sizeof(InT));
+  if (nch >= 9 && nch <= 32 && rows >= 2 * device_info().sms) {
+    // Rows of 2304..8192 columns, enough of them to fill the GPU: bulk-copy
+    // staged kernel, 2-4 rows per CTA in flight within ~96 KB.
+    const int stage_bytes = static_cast<int>((row_bytes + 127) / 128 * 128);
+    int stages = 98304 / stage_bytes;
+    stages = stages < 2 ? 2 : stages > 4 ? 4 : stages;
+    const int smem = stages * stage_bytes;
+    const int per_sm = 200000 / (smem + 2048) > 4 ? 4 : 200000 / (smem + 2048);
+    const int grid = grid_cap(rows, per_sm < 1 ? 1 : per_sm);
+    const int cpw = (nch + 7) / 8;
+#define QL_QT(CPW)                                                                             \
+  do {                                                                                         \
+    static bool attr_set[64] = {false};                                                        \
+    int dev = 0;                                                                               \
+    cudaGetDevice(&dev);                                                                       \
+    if (dev < 64 && !attr_set[dev]) {                                                          \
+      cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW>,                                    \
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, 100000);               \
+      attr_set[dev] = true;                                                                    \
+    }                                                                                          \
+    quant_rows_tma_kernel<InT, CPW><<<grid, 256, smem, s>>>(x, rows, c, ldx, cs, B, hc, flags, \
+                                                           q, ldq, rs, st, stages, stage_bytes); \
+  } while (0)
+    if (cpw <= 2) QL_QT(2);
+    else if (cpw <= 3) QL_QT(3);
+    else QL_QT(4);
+#undef QL_QT
+  } else if (nch <= 64) {
     const int wpr = nch <= 1 ? 1 : nch <= 2 ? 2 : nch <= 4 ? 4 : 8;
     const int cpw = (nch + wpr - 1) / wpr;  // 1..8
     const int rpc = 8 / wpr;
@@ -378,6 +503,7 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
     else if (wpr == 4) QL_QR(1, 4);
     else if (cpw <= 1) QL_QR(1, 8);
     else if (cpw <= 2) QL_QR(2, 8);
+    else if (cpw <= 3) QL_QR(3, 8);
     else if (cpw <= 4) QL_QR(4, 8);
     else QL_QR(8, 8);
 #undef QL_QR
@@ -445,8 +571,9 @@ cudaError_t launch_colfinalize(const uint32_t* colmax, const double* colsum, int
 
 cudaError_t launch_colquant(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
                             const float* inv2, int8_t* q, cudaStream_t s) {
-  const int64_t items = M * (N / 16);
-  const int grid = grid_cap((items + 255) / 256, 8);
+  const unsigned segs = static_cast<unsigned>((N + 2047) / 2048);
+  const int64_t want = (static_cast<int64_t>(device_info().sms) * 8 + segs - 1) / segs;
+  const dim3 grid(static_cast<unsigned>(want < M ? want : M), segs);
   if (dyt == QL_BF16)
     colquant_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         reinterpret_cast<const __nv_bfloat16*>(dy), M, static_cast<int>(N), sx, inv2, q);

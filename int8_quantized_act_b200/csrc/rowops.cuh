@@ -51,6 +51,30 @@ __device__ __forceinline__ int code_rne(float t) {
   return static_cast<int>(r);
 }
 
+// Round-to-nearest-even of v through the float adder, for |v| <= 127.5:
+// v + 1.5*2^23 lies in [2^23, 2^24), where adjacent floats are 1 apart, so
+// the IEEE addition itself rounds v to an integer, ties to even (exactly
+// rintf(v)).  The integer sits in the low mantissa bits of the sum: its low
+// byte is the int8 code.  Callers guarantee |v| <= 127(1 + 2^-22) (v = t *
+// 127/amax with |t| <= amax); for inf/NaN inputs the byte is unspecified,
+// like every output under QL_ERR_NONFINITE.
+constexpr float kRneMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t rne_bits(float v) { return __float_as_uint(v + kRneMagic); }
+
+// Low bytes of four rne_bits words, packed little-endian.
+__device__ __forceinline__ uint32_t pack_codes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Running max of |x| kept as the bit pattern of a non-negative float: for
+// finite values the integer order is the float order; inf and NaN patterns
+// (>= 0x7F800000) sort above every finite value, so one compare at the end
+// tells whether a non-finite value was met.
+__device__ __forceinline__ uint32_t abs_bits(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
+
+constexpr uint32_t kInfBits = 0x7F800000u;
+
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
          ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
@@ -79,11 +103,13 @@ __device__ __forceinline__ void fwht_chunk(float (&v)[8], int B, int lane, float
   }
   for (int h = 8; h < B; h <<= 1) {
     const int d = h >> 3;
-    const bool upper = (lane & d) != 0;
+    // The lane holding the higher index computes partner - own = partner +
+    // (-own): flip the sign bit instead of selecting between two sums.
+    const uint32_t flip = (lane & d) ? 0x80000000u : 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float p = __shfl_xor_sync(0xFFFFFFFFu, v[i], d);
-      v[i] = upper ? (p - v[i]) : (v[i] + p);
+      v[i] = p + __uint_as_float(__float_as_uint(v[i]) ^ flip);
     }
   }
 #pragma unroll

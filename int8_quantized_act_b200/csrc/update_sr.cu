@@ -26,9 +26,10 @@ namespace {
 __device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
-    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;  // one 32x32->64 multiply
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k0, static_cast<uint32_t>(p1),
+                   static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k1, static_cast<uint32_t>(p0));
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }
@@ -46,13 +47,37 @@ __device__ __forceinline__ float adamw(const UpdateConsts& c, float w, float g, 
   return w1 - c.st * (mn / den);
 }
 
-// floor(v) + 1 with probability frac(v), decided by u24 < frac * 2^24.
-__device__ __forceinline__ int sr_code(float val, uint32_t u24) {
+// floor(v) + 1 with probability frac(v), decided by u24 < frac * 2^24;
+// clamped to [-127, 127].  Returns rne_bits of the (integer-valued) result, so
+// its low byte is the int8 code (exact: adding 1.5*2^23 to an integer-valued
+// float below 2^22 in magnitude is exact).
+__device__ __forceinline__ uint32_t sr_code_bits(float val, uint32_t u24) {
   const float f = floorf(val);
   const float frac = val - f;
   float r = (__uint2float_rn(u24) < frac * 16777216.0f) ? f + 1.0f : f;
   r = fminf(fmaxf(r, -127.0f), 127.0f);
-  return static_cast<int>(r);
+  return rne_bits(r);
+}
+
+// Stochastic codes of 16 consecutive elements starting at element e0
+// (a multiple of 16): four Philox blocks, word e & 3 of block e >> 2.
+__device__ __forceinline__ uint4 sr_group(const float (&w)[16], float inv, bool zero_row,
+                                          uint64_t e0, uint32_t sl, uint32_t sh, uint32_t tl,
+                                          uint32_t th) {
+  uint32_t b[16];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint64_t blk = (e0 >> 2) + k;
+    const uint4 r = philox10(make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32),
+                                        tl, th),
+                             sl, sh);
+    const uint32_t words[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      b[4 * k + e] = zero_row ? 0u : sr_code_bits(w[4 * k + e] * inv, words[e] >> 8);
+  }
+  return make_uint4(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]),
+                    pack_codes(b[8], b[9], b[10], b[11]), pack_codes(b[12], b[13], b[14], b[15]));
 }
 
 __device__ __forceinline__ void load16f(const float* p, float (&v)[16]) {
@@ -224,23 +249,75 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
 #pragma unroll
   for (int i = 0; i < GPT; ++i) {
     const int j = t + T * i;
-    if (j < ngroups) {
-      const uint64_t blk0 = static_cast<uint64_t>(row + 16 * j) >> 2;
-      int cd[16];
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint64_t blk = blk0 + b;
-        const uint4 r = philox10(make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32),
-                                            step_lo, step_hi),
-                                 seed_lo, seed_hi);
-        const uint32_t words[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) cd[4 * b + e] = amax == 0.0f ? 0 : sr_code(w[i][4 * b + e] * inv, words[e] >> 8);
-      }
+    if (j < ngroups)
       *reinterpret_cast<uint4*>(wq + row + 16 * j) =
-          make_uint4(pack4(cd[0], cd[1], cd[2], cd[3]), pack4(cd[4], cd[5], cd[6], cd[7]),
-                     pack4(cd[8], cd[9], cd[10], cd[11]), pack4(cd[12], cd[13], cd[14], cd[15]));
+          sr_group(w[i], inv, amax == 0.0f, static_cast<uint64_t>(row + 16 * j), seed_lo, seed_hi,
+                   step_lo, step_hi);
+  }
+}
+
+// The plain (not weight-normalized) update with GPT = 1, 2 or 4 16-element
+// groups per thread and T = ceil(ngroups / GPT) threads rounded up to a warp
+// (<= 512), so threads finish their groups together at the row reduction.
+template <int GPT>
+__global__ void __launch_bounds__(512) update_sr_rows_kernel(
+    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
+    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, uint32_t seed_lo,
+    uint32_t seed_hi, uint32_t step_lo, uint32_t step_hi, int32_t* __restrict__ status) {
+  __shared__ uint32_t s_max[32];
+  const int n = blockIdx.x;
+  const int t = threadIdx.x;
+  const int T = blockDim.x;
+  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
+  const int ngroups = K >> 4;
+  const int64_t row = static_cast<int64_t>(n) * K;
+  const bool adam = c.kind == QL_ADAMW;
+  const float s = sw[n];
+
+  float w[GPT][16];
+  uint32_t mbits = 0;
+#pragma unroll
+  for (int i = 0; i < GPT; ++i) {
+    const int j = t + T * i;
+    if (j < ngroups) {
+      const int64_t off = row + 16 * j;
+      const uint4 qv = *reinterpret_cast<const uint4*>(wq + off);
+      float gr[16], m1[16], m2[16];
+      load16f(grad + off, gr);
+      if (adam) {
+        load16f(mom1 + off, m1);
+        load16f(mom2 + off, m2);
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float wv = s * static_cast<float>(code_at(qv, e));
+        w[i][e] = adam ? adamw(c, wv, gr[e], m1[e], m2[e]) : wv - c.lr * gr[e];
+        mbits = max(mbits, abs_bits(w[i][e]));
+      }
+      if (adam) {
+        store16f(mom1 + off, m1);
+        store16f(mom2 + off, m2);
+      }
     }
+  }
+  mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+  if (lane == 0) s_max[warp] = mbits;
+  __syncthreads();
+  mbits = 0;
+  for (int k = 0; k < nwarps; ++k) mbits = max(mbits, s_max[k]);
+  const float amax = __uint_as_float(mbits);
+  const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
+  if (t == 0) {
+    sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
+    if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  }
+#pragma unroll
+  for (int i = 0; i < GPT; ++i) {
+    const int j = t + T * i;
+    if (j < ngroups)
+      *reinterpret_cast<uint4*>(wq + row + 16 * j) =
+          sr_group(w[i], inv, mbits == 0, static_cast<uint64_t>(row + 16 * j), seed_lo, seed_hi,
+                   step_lo, step_hi);
   }
 }
 
@@ -261,11 +338,21 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
 #define QL_UPD(G, W)                                                                          \
   update_sr_kernel<G, W><<<grid, T, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, g, g_m, \
                                             g_v, status)
-  const bool wn = g != nullptr;
-  if (gpt <= 1) { if (wn) QL_UPD(1, true); else QL_UPD(1, false); }
-  else if (gpt <= 2) { if (wn) QL_UPD(2, true); else QL_UPD(2, false); }
-  else if (gpt <= 4) { if (wn) QL_UPD(4, true); else QL_UPD(4, false); }
-  else { if (wn) QL_UPD(8, true); else QL_UPD(8, false); }
+  if (g != nullptr) {  // weight norm: power-of-two thread count for the pinned reduction
+    if (gpt <= 1) QL_UPD(1, true);
+    else if (gpt <= 2) QL_UPD(2, true);
+    else if (gpt <= 4) QL_UPD(4, true);
+    else QL_UPD(8, true);
+  } else {
+    const int g1 = ngroups <= 512 ? 1 : ngroups <= 1024 ? 2 : 4;
+    const int tr = ((ngroups + g1 - 1) / g1 + 31) / 32 * 32;
+    if (g1 == 1)
+      update_sr_rows_kernel<1><<<grid, tr, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, status);
+    else if (g1 == 2)
+      update_sr_rows_kernel<2><<<grid, tr, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, status);
+    else
+      update_sr_rows_kernel<4><<<grid, tr, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, status);
+  }
 #undef QL_UPD
   count_launches(1);
   return cudaGetLastError();

@@ -39,6 +39,11 @@ CASES = [
     (5, 16384, 64, torch.float32),
     (3, 16, 2, torch.float32),
     (2, 4096, 4, torch.bfloat16),
+    # >= 2 rows per SM and 9..32 chunks: rows staged by the bulk-copy engine
+    (400, 2320, 16, torch.float32),    # 10 chunks, ragged last chunk
+    (500, 5376, 128, torch.bfloat16),  # 21 chunks
+    (320, 8192, 256, torch.bfloat16),  # 32 chunks
+    (2000, 4096, 0, torch.float32),    # several rows per CTA through the ring
 ]
 
 
@@ -55,10 +60,11 @@ def test_quantize_rows_bit_exact(rows, cols, B, dtype):
     assert np.array_equal(q, rq)
 
 
+@pytest.mark.parametrize("rows", [96, 700])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_quantize_rows_with_col_scale(dtype):
+def test_quantize_rows_with_col_scale(dtype, rows):
     """The row quantization of dY * s_w that precedes the input-gradient GEMM."""
-    x = workloads.normal((96, 7168), 1.0, 3)
+    x = workloads.normal((rows, 7168), 1.0, 3)
     cs = np.abs(workloads.normal((7168,), 1e-3, 4)) + np.float32(1e-5)
     xt = torch.from_numpy(x).to(dtype)
     q, s, st = _quant_gpu(dev(xt), 0, col_scale=dev(cs))
