@@ -100,6 +100,65 @@ __device__ __forceinline__ void store16(__nv_bfloat16* p, const float* v) {
                                               bf16x2(v[12], v[13]), bf16x2(v[14], v[15]));
 }
 
+// Epilogue of one 128-row slab of an accumulator tile: rows row0 + 32*quarter
+// + lane, columns col0 .. col0+255 of the output.  All 32 lanes of the warp
+// must call it (tcgen05.ld is warp-collective); rows/columns past the output
+// are computed but not stored.
+template <typename OutT, int HB>
+__device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, int quarter,
+                                              int lane, int row0, int col0) {
+  constexpr int CH = HB > 32 ? HB : 32;  // columns per register chunk
+  OutT* out = reinterpret_cast<OutT*>(ep.out);
+  const int gr = row0 + quarter * 32 + lane;
+  const bool row_ok = gr < ep.rows;
+  const float rs = (row_ok && ep.row_scale) ? ep.row_scale[gr] : 1.0f;
+  const uint32_t taddr = acc_tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += CH) {
+    uint32_t r[CH];
+    tmem_ld_cols<CH>(taddr + c0, r);
+    tmem_wait_ld();
+    const int gc0 = col0 + c0;
+    if (row_ok && gc0 < ep.cols) {
+      float v[CH];
+#pragma unroll
+      for (int i = 0; i < CH; ++i) v[i] = __int2float_rn(static_cast<int>(r[i])) * rs;
+      if (ep.col_scale || ep.bias) {
+#pragma unroll
+        for (int g = 0; g < CH / 16; ++g) {
+          if (gc0 + 16 * g < ep.cols) {
+            if (ep.col_scale) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4) {
+                const float4 c4 = __ldg(reinterpret_cast<const float4*>(ep.col_scale + gc0 + 16 * g + i));
+                v[16 * g + i] = v[16 * g + i] * c4.x;
+                v[16 * g + i + 1] = v[16 * g + i + 1] * c4.y;
+                v[16 * g + i + 2] = v[16 * g + i + 2] * c4.z;
+                v[16 * g + i + 3] = v[16 * g + i + 3] * c4.w;
+              }
+            }
+            if (ep.bias) {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4) {
+                const float4 b4 = __ldg(reinterpret_cast<const float4*>(ep.bias + gc0 + 16 * g + i));
+                v[16 * g + i] = v[16 * g + i] + b4.x;
+                v[16 * g + i + 1] = v[16 * g + i + 1] + b4.y;
+                v[16 * g + i + 2] = v[16 * g + i + 2] + b4.z;
+                v[16 * g + i + 3] = v[16 * g + i + 3] + b4.w;
+              }
+            }
+          }
+        }
+      }
+      if constexpr (HB > 0) fwht_regs<CH, HB>(v, ep.hc);
+      OutT* orow = out + static_cast<int64_t>(gr) * ep.ldo + gc0;
+#pragma unroll
+      for (int g = 0; g < CH / 16; ++g)
+        if (gc0 + 16 * g < ep.cols) store16(orow + 16 * g, v + 16 * g);
+    }
+  }
+}
+
 template <bool A_MN, bool B_MN, typename OutT, int HB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -230,63 +289,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    constexpr int CH = HB > 32 ? HB : 32;  // columns per register chunk
-    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
-    const int row_local = quarter * 32 + lane;
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     uint32_t acc = 0, acc_phase = 0;
-    OutT* out = reinterpret_cast<OutT*>(ep.out);
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       const int tm = t / tiles_n, tn = t % tiles_n;
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
       tc_fence_after();
-      const int gr = tm * BM + row_local;
-      const bool row_ok = gr < ep.rows;
-      const float rs = (row_ok && ep.row_scale) ? ep.row_scale[gr] : 1.0f;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += CH) {
-        uint32_t r[CH];
-        tmem_ld_cols<CH>(taddr + c0, r);
-        tmem_wait_ld();
-        const int gc0 = tn * BN + c0;
-        if (row_ok && gc0 < ep.cols) {
-          float v[CH];
-#pragma unroll
-          for (int i = 0; i < CH; ++i) v[i] = __int2float_rn(static_cast<int>(r[i])) * rs;
-          if (ep.col_scale || ep.bias) {
-#pragma unroll
-            for (int g = 0; g < CH / 16; ++g) {
-              if (gc0 + 16 * g < ep.cols) {
-                if (ep.col_scale) {
-#pragma unroll
-                  for (int i = 0; i < 16; i += 4) {
-                    const float4 c4 = __ldg(reinterpret_cast<const float4*>(ep.col_scale + gc0 + 16 * g + i));
-                    v[16 * g + i] = v[16 * g + i] * c4.x;
-                    v[16 * g + i + 1] = v[16 * g + i + 1] * c4.y;
-                    v[16 * g + i + 2] = v[16 * g + i + 2] * c4.z;
-                    v[16 * g + i + 3] = v[16 * g + i + 3] * c4.w;
-                  }
-                }
-                if (ep.bias) {
-#pragma unroll
-                  for (int i = 0; i < 16; i += 4) {
-                    const float4 b4 = __ldg(reinterpret_cast<const float4*>(ep.bias + gc0 + 16 * g + i));
-                    v[16 * g + i] = v[16 * g + i] + b4.x;
-                    v[16 * g + i + 1] = v[16 * g + i + 1] + b4.y;
-                    v[16 * g + i + 2] = v[16 * g + i + 2] + b4.z;
-                    v[16 * g + i + 3] = v[16 * g + i + 3] + b4.w;
-                  }
-                }
-              }
-            }
-          }
-          if constexpr (HB > 0) fwht_regs<CH, HB>(v, ep.hc);
-          OutT* orow = out + static_cast<int64_t>(gr) * ep.ldo + gc0;
-#pragma unroll
-          for (int g = 0; g < CH / 16; ++g)
-            if (gc0 + 16 * g < ep.cols) store16(orow + 16 * g, v + 16 * g);
-        }
-      }
+      epilogue_tile<OutT, HB>(ep, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -300,6 +309,184 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(status, 1 << QL_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ CTA pairs
+// The same GEMM on 256x256 tiles computed by a cluster of two CTAs on two
+// SMs (tcgen05 cta_group::2).  Each CTA loads 128 rows of A and 128 of the
+// 256 B columns per stage (32 KB; TMA loads without multicast, counted on the
+// even CTA's barrier), so per SM the operand traffic through shared memory
+// is 64 B/clk at full MMA rate instead of 96 for a 128x256 tile on one SM;
+// the even CTA issues the 256x256x32 MMAs and commits to both CTAs'
+// barriers; each CTA drains its own 128 accumulator rows.
+constexpr int PSTAGES = 6;
+constexpr int PA_BYTES = 128 * BK;                 // 16 KiB: this CTA's A rows
+constexpr int PB_BYTES = 128 * BK;                 // 16 KiB: this CTA's B columns
+constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;  // 32 KiB
+constexpr int PNUM_BARS = 2 * PSTAGES + 5;
+constexpr int PSMEM_BYTES = 1024 + PSTAGES * PSTAGE_BYTES + 8 * PNUM_BARS + 16;
+
+template <bool A_MN, bool B_MN, typename OutT, int HB>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, int tiles_m, int tiles_n,
+                        int kblocks, Epi ep, int32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + PSTAGES * PA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + PSTAGES * PB_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + PNUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + PSTAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * PSTAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * PSTAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * PSTAGES + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PSTAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);   // rank 0's: its expect_tx arrival + both CTAs' bytes
+      mbar_init(empty0 + 8 * s, 1);  // the pair's MMA commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);   // the pair's MMA commit
+      mbar_init(tempty0 + 8 * a, 8);  // rank 0's: 4 epilogue warps of each CTA
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = tiles_m * tiles_n;
+  const uint32_t lead_full0 = mapa_shared(full0, 0);
+  const uint32_t lead_tempty0 = mapa_shared(tempty0, 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, armed = 0, armed_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        const int tm = t / tiles_n, tn = t % tiles_n;
+        const int a_row = tm * 256 + static_cast<int>(rank) * 128;
+        const int b_col = tn * 256 + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) {
+            mbar_arrive_expect_tx(full0 + 8 * stage, 2 * PSTAGE_BYTES);
+            armed |= 1u << stage;
+            armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t fb = lead_full0 + 8 * stage;
+          const uint32_t a_dst = smem_u32(sA + stage * PA_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * PB_BYTES);
+          if (A_MN) tma_load_2d_pair(a_dst, &tmA, fb, a_row, kb * BK);
+          else tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
+          if (B_MN) tma_load_2d_pair(b_dst, &tmB, fb, b_col, kb * BK);
+          else tma_load_2d_pair(b_dst, &tmB, fb, kb * BK, b_col);
+          if (++stage == PSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (rank == 0) {
+        // Every stage armed here counts both CTAs' copies: wait for them.
+        for (int s = 0; s < PSTAGES; ++s)
+          if (armed & (1u << s)) mbar_wait_drain(full0 + 8 * s, (armed_phase >> s) & 1u);
+      } else if (!ok) {
+        __nanosleep(100000);  // give copies in flight time to land before exit
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (rank 0)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_i8(256, 256, A_MN ? 1 : 0, B_MN ? 1 : 0);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * PA_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * PB_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            const uint64_t a_desc = A_MN ? smem_desc_sw128(a_base + kk * 4096, 16384, 1024)
+                                         : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t b_desc = B_MN ? smem_desc_sw128(b_base + kk * 4096, 16384, 1024)
+                                         : smem_desc_sw128(b_base + kk * 32, 16, 1024);
+            mma_i8_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+          if (++stage == PSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(tfull0 + 8 * acc, 0x3);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      mma_commit_pair_mc(drain, 0x1);
+      mbar_wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int t = pair; t < num_tiles; t += npairs) {
+      const int tm = t / tiles_n, tn = t % tiles_n;
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
+      tc_fence_after();
+      epilogue_tile<OutT, HB>(ep, tmem_base + acc * BN, quarter, lane,
+                              tm * 256 + static_cast<int>(rank) * 128, tn * BN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead_tempty0 + 8 * acc);
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();  // neither CTA leaves while the pair may still touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
   if (threadIdx.x == 0 && *abort_flag) atomicOr(status, 1 << QL_ERR_TIMEOUT);
 }
@@ -338,6 +525,56 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Clusters of two that can be resident together (cached per device).
+template <typename K>
+int pair_slots(K kern) {
+  static int slots[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && slots[dev] > 0) return slots[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 74, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = PSMEM_BYTES;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1)
+    n = device_info().sms / 2;
+  if (dev < 64) slots[dev] = n;
+  return n;
+}
+
+template <bool A_MN, bool B_MN, typename OutT, int HB>
+cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
+                     int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
+  auto kern = gemm_i8_pair_kernel<A_MN, B_MN, OutT, HB>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !__atomic_load_n(&configured[dev], __ATOMIC_ACQUIRE)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    __atomic_store_n(&configured[dev], 1, __ATOMIC_RELEASE);
+  }
+  const int tiles = tiles_m * tiles_n;
+  const int slots = pair_slots(kern);
+  const int pairs = tiles < slots ? tiles : slots;
+  cudaEvent_t before = nullptr, after = nullptr;
+  gemm_timing_events(&before, &after);
+  if (before) cudaEventRecord(before, s);
+  kern<<<2 * pairs, NUM_THREADS, PSMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, ep, status);
+  cudaError_t e = cudaGetLastError();
+  if (after) cudaEventRecord(after, s);
+  count_launches(1);
+  return e;
+}
+
 template <bool A_MN, bool B_MN, typename OutT, int HB>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
                 int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
@@ -364,10 +601,17 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
   return e;
 }
 
-cudaError_t dispatch_dx(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
-                        int kblocks, const Epi& ep, bool bf16, int hb, int32_t* status,
-                        cudaStream_t s) {
-#define QL_RUN(T, H) return run<false, true, T, H>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s)
+template <bool A_MN, bool B_MN, typename OutT, int HB>
+cudaError_t go(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
+               int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
+  if (pair) return run_pair<A_MN, B_MN, OutT, HB>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+  return run<A_MN, B_MN, OutT, HB>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+}
+
+cudaError_t dispatch_dx(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m,
+                        int tiles_n, int kblocks, const Epi& ep, bool bf16, int hb,
+                        int32_t* status, cudaStream_t s) {
+#define QL_RUN(T, H) return go<false, true, T, H>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s)
   if (bf16) {
     switch (hb) {
       case 0: QL_RUN(__nv_bfloat16, 0);
@@ -400,11 +644,14 @@ cudaError_t dispatch_dx(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_
 cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
                            int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
                            const GemmEpilogue& e, int32_t* status, cudaStream_t s) {
+  // Outputs with more than one 128-row slab run on CTA pairs (256x256
+  // tiles); smaller ones on single CTAs (128x256 tiles).
+  const bool pair = rows > BM;
   CUtensorMap ta, tb;
   const bool ok_a = a_mn ? make_tmap(&ta, A, rows, kc, lda, 128, BK)
                          : make_tmap(&ta, A, kc, rows, lda, BK, BM);
   const bool ok_b = b_mn ? make_tmap(&tb, B, cols, kc, ldb, 128, BK)
-                         : make_tmap(&tb, B, kc, cols, ldb, BK, BN);
+                         : make_tmap(&tb, B, kc, cols, ldb, BK, pair ? 128 : BN);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   Epi ep;
   ep.out = e.out;
@@ -415,7 +662,8 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
   ep.col_scale = e.col_scale;
   ep.bias = e.bias;
   ep.hc = e.hc;
-  const int tiles_m = static_cast<int>((rows + BM - 1) / BM);
+  const int tile_rows = pair ? 2 * BM : BM;
+  const int tiles_m = static_cast<int>((rows + tile_rows - 1) / tile_rows);
   const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
   const int kblocks = static_cast<int>((kc + BK - 1) / BK);
   const bool bf16 = e.out_bf16 != 0;
@@ -423,12 +671,12 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
   // (K-major x MN-major, optional fused rotation), weight gradient
   // (MN-major x MN-major, float32 out).
   if (!a_mn && !b_mn && e.hb == 0) {
-    if (bf16) return run<false, false, __nv_bfloat16, 0>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
-    return run<false, false, float, 0>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+    if (bf16) return go<false, false, __nv_bfloat16, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+    return go<false, false, float, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
   }
-  if (!a_mn && b_mn) return dispatch_dx(ta, tb, tiles_m, tiles_n, kblocks, ep, bf16, e.hb, status, s);
+  if (!a_mn && b_mn) return dispatch_dx(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, bf16, e.hb, status, s);
   if (a_mn && b_mn && e.hb == 0 && !bf16)
-    return run<true, true, float, 0>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+    return go<true, true, float, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
   return cudaErrorInvalidValue;
 }
 
