@@ -5,8 +5,10 @@ One step = one pass of the whole hot path over one batch: the 5376 -> 7168
 layer of OneTrainer PR #1681 "Int8 conv rot" at 12000 tokens with Hadamard
 block 128, bf16 X and dY:
     qlinear_fwd       per-row rotate + quantize X (saved int8), int8 GEMM, scale + bias -> bf16 y
-    qlinear_bwd_dx    row-quantize dY*s_w, int8 GEMM (dY_q W_q), scale, fused rotation -> bf16 dX
-    qlinear_bwd_dw    column-quantize dY*s_x, int8 GEMM (dY_q^T X_q), scale -> fp32 dW, db
+    qlinear_bwd       from one shared preparation of dY (column statistics, then one pass
+                      writing the row-quantized dY*s_w and the column-quantized dY*s_x):
+                      int8 GEMM dY_q W_q, scale, fused rotation -> bf16 dX, and
+                      int8 GEMM dY_q^T X_q, scale -> fp32 dW; db
     qweight_update_sr AdamW on the int8 weight + Philox stochastic requantization
 Metric: int8 tensor operations of the three GEMMs (3 x 2*M*N*K) per second,
 in TOPS, whole job (all ranks).  Inputs stay resident in HBM; the step's
@@ -191,7 +193,7 @@ class Layer:
         self.dx = torch.empty((M_TOK, K_IN), dtype=torch.bfloat16, device=dev)
         self.dw = torch.empty((N_OUT, K_IN), dtype=torch.float32, device=dev)
         self.db = torch.empty(N_OUT, dtype=torch.float32, device=dev)
-        self.ws = torch.empty(ql.qlinear_workspace_bytes(M_TOK, N_OUT, K_IN, BLOCK),
+        self.ws = torch.empty(ql.qlinear_bwd_workspace_bytes(M_TOK, N_OUT, K_IN, BLOCK),
                               dtype=torch.uint8, device=dev)
         self.opt = ql.Optim(kind=ql.QL_ADAMW, lr=1e-3, weight_decay=0.01)
         self.t = 0
@@ -202,15 +204,13 @@ class Layer:
     def step(self, gemm_events=None, update_events=None):
         ql = self.ql
         self.t += 1
-        ev = gemm_events or [None] * 6
-        ql.ql_set_gemm_timing_events(ev[0], ev[1])
+        # events around the forward, input-gradient and weight-gradient GEMMs
+        ql.ql_set_gemm_timing_events(gemm_events or ())
         ql.qlinear_fwd(self.x, self.wq, self.sw, self.bias, BLOCK, self.y, self.xq, self.sx,
                        self.status)
-        ql.ql_set_gemm_timing_events(ev[2], ev[3])
-        ql.qlinear_bwd_dx(self.dy, self.wq, self.sw, BLOCK, self.dx, self.ws, self.status)
-        ql.ql_set_gemm_timing_events(ev[4], ev[5])
-        ql.qlinear_bwd_dw(self.dy, self.xq, self.sx, self.dw, self.db, self.ws, self.status)
-        ql.ql_set_gemm_timing_events(None, None)
+        ql.qlinear_bwd(self.dy, self.wq, self.sw, self.xq, self.sx, BLOCK, self.dx, self.dw,
+                       self.db, self.ws, self.status)
+        ql.ql_set_gemm_timing_events(())
         if update_events:
             update_events[0].record()
         ql.qweight_update_sr(self.wq, self.sw, self.dw, self.opt, self.m, self.v, 1234, self.t,
@@ -244,7 +244,7 @@ def run_ours(args, rank, world, local):
     for _ in range(args.warmup):
         layer.step()
     torch.cuda.synchronize()
-    gemm_ev = [new_events(6) for _ in range(args.steps)]
+    gemm_ev = [list(zip(*[iter(new_events(6))] * 2)) for _ in range(args.steps)]
     upd_ev = [new_events(2) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = ql.ql_kernel_launches()
@@ -268,7 +268,7 @@ def run_ours(args, rank, world, local):
     if word:
         raise RuntimeError(f"device status {ql.status_flags(word)}")
 
-    gemm_ms = [e[2 * j].elapsed_time(e[2 * j + 1]) for e in gemm_ev for j in range(3)]
+    gemm_ms = [b.elapsed_time(a) for pairs in gemm_ev for (b, a) in pairs]
     per_kind = {name: statistics.mean(gemm_ms[j::3]) for j, name in enumerate(("fwd", "dx", "dw"))}
     gemm_avg = statistics.mean(gemm_ms)
     upd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in upd_ev)

@@ -179,6 +179,22 @@ QL_API int qlinear_bwd_dw(const void *dy, int dyt, int64_t M, int64_t N,
                    float *dw, float *db, void *ws, size_t ws_bytes,
                    int32_t *d_status, void *stream);
 
+/* Bytes of device workspace that qlinear_bwd needs (qlinear_workspace_bytes
+ * plus room for the second int8 copy of the gradient, M*N bytes). */
+QL_API size_t qlinear_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int hadamard_block);
+
+/* Both backward products of the layer in one call: exactly the results of
+ * qlinear_bwd_dx (dX) followed by qlinear_bwd_dw (dW, db), but dY is read
+ * twice instead of three times: one pass gathers the column maxima and sums,
+ * a second pass writes both the row-quantized (dY*s_w) and the column-
+ * quantized (dY*s_x) int8 copies from the same read.  Arguments as for the
+ * two calls; ws holds qlinear_bwd_workspace_bytes(M, N, K, hadamard_block)
+ * bytes.  N, M <= QL_MAX_CONTRACTION. */
+QL_API int qlinear_bwd(const void *dy, int dyt, int64_t M, int64_t N,
+                       const int8_t *wq, const float *sw, const int8_t *xq, const float *sx,
+                       int64_t K, int hadamard_block, void *dx, int dxt, float *dw, float *db,
+                       void *ws, size_t ws_bytes, int32_t *d_status, void *stream);
+
 /* One optimizer step of an int8 weight [N,K] with stochastic requantization,
  * in place ([QT] paragraph after the feature table; rows "Optimizers",
  * "Row-wise weight normalization"):
@@ -236,14 +252,16 @@ QL_API int qlinear_bwd_dx_noalloc(const void *dy, int dyt, int64_t M, int64_t N,
                                   int32_t *d_status, void *stream);
 
 /* Instrumentation (no effect on results).
- * ql_set_gemm_timing_events: while set (non-NULL), every int8 GEMM kernel that
- * the calling host thread launches records the cudaEvent_t `before` on its
- * stream right before the launch and `after` right after it, so a caller can
- * time the GEMM alone inside a layer call.  Pass NULL, NULL to stop.  The
- * events are the caller's; the library only records them.
+ * ql_set_gemm_timing_events: the next n (<= 16) int8 GEMM kernels that the
+ * calling host thread launches record the cudaEvent_t before[i] on their
+ * stream right before the i-th launch and after[i] right after it, so a
+ * caller can time the GEMMs alone inside layer calls (qlinear_bwd launches
+ * two).  After n launches, or with n = 0, nothing is recorded.  The events
+ * (host arrays of cudaEvent_t passed as void*) are the caller's; the library
+ * copies the handles and only records them.
  * ql_kernel_launches: number of CUDA kernels this library has launched in the
  * process so far (all threads). */
-QL_API void ql_set_gemm_timing_events(void *before, void *after);
+QL_API void ql_set_gemm_timing_events(void *const *before, void *const *after, int n);
 QL_API uint64_t ql_kernel_launches(void);
 
 #ifdef __cplusplus

@@ -27,7 +27,8 @@ __all__ = [
     "ql_status_string", "qlinear_workspace_bytes", "qlinear_quantize_rows",
     "qlinear_hadamard", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
     "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
-    "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES",
+    "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES", "qlinear_bwd",
+    "qlinear_bwd_workspace_bytes",
 ]
 
 QL_OK, QL_ERR_ARG, QL_ERR_SHAPE, QL_ERR_ALIGN = 0, 1, 2, 3
@@ -103,10 +104,16 @@ def lib() -> ctypes.CDLL:
     L.qlinear_bwd_dx.argtypes = [P, I, I64, I64, P, P, I64, I, P, I, P, ctypes.c_size_t, P, P]
     L.qlinear_bwd_dw.restype = I
     L.qlinear_bwd_dw.argtypes = [P, I, I64, I64, P, P, I64, P, P, P, ctypes.c_size_t, P, P]
+    L.qlinear_bwd_workspace_bytes.restype = ctypes.c_size_t
+    L.qlinear_bwd_workspace_bytes.argtypes = [I64, I64, I64, I]
+    L.qlinear_bwd.restype = I
+    L.qlinear_bwd.argtypes = [P, I, I64, I64, P, P, P, P, I64, I, P, I, P, P, P,
+                              ctypes.c_size_t, P, P]
     L.qlinear_bwd_dx_noalloc.restype = I
     L.qlinear_bwd_dx_noalloc.argtypes = [P, I, I64, I64, P, P, I64, I, P, I, P, P]
     L.ql_set_gemm_timing_events.restype = None
-    L.ql_set_gemm_timing_events.argtypes = [P, P]
+    L.ql_set_gemm_timing_events.argtypes = [ctypes.POINTER(ctypes.c_void_p),
+                                            ctypes.POINTER(ctypes.c_void_p), I]
     L.ql_kernel_launches.restype = ctypes.c_uint64
     L.ql_kernel_launches.argtypes = []
     L.qweight_update_sr.restype = I
@@ -229,6 +236,27 @@ def qlinear_bwd_dx(dy, wq, sw, hadamard_block: int, dx, ws, status, stream=None)
     _check(code, "qlinear_bwd_dx")
 
 
+def qlinear_bwd_workspace_bytes(M: int, N: int, K: int, hadamard_block: int = 0) -> int:
+    return int(lib().qlinear_bwd_workspace_bytes(M, N, K, hadamard_block))
+
+
+def qlinear_bwd(dy, wq, sw, xq, sx, hadamard_block: int, dx, dw, db, ws, status, stream=None):
+    """dx, dw, db <- both backward products with one shared preparation of dY
+    (ws: qlinear_bwd_workspace_bytes bytes)."""
+    M, N = dy.shape
+    K = wq.shape[1]
+    for t, n in ((dy, "dy"), (wq, "wq"), (sw, "sw"), (xq, "xq"), (sx, "sx"), (dx, "dx"),
+                 (dw, "dw"), (db, "db")):
+        _contig(t, n)
+    code = lib().qlinear_bwd(
+        _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(wq, "wq", torch.int8),
+        _dev(sw, "sw", torch.float32), _dev(xq, "xq", torch.int8), _dev(sx, "sx", torch.float32),
+        K, hadamard_block, _dev(dx, "dx"), _dtype_code(dx, "dx"), _dev(dw, "dw", torch.float32),
+        _dev(db, "db", torch.float32), _dev(ws, "ws", torch.uint8), ws.numel(),
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qlinear_bwd")
+
+
 def qlinear_bwd_dx_noalloc(dy, wq, sw, hadamard_block: int, dx, status, stream=None):
     """qlinear_bwd_dx for callers that cannot allocate device memory: no
     workspace argument; the library's own fixed scratch (QL_NOALLOC_SCRATCH_BYTES)
@@ -280,13 +308,15 @@ def qweight_update_sr(wq, sw, grad, opt: Optim, m, v, seed: int, step: int, stat
     _check(code, "qweight_update_sr")
 
 
-def ql_set_gemm_timing_events(before=None, after=None):
-    """Record these torch.cuda.Event objects around every int8 GEMM launch of
-    this thread (None, None to stop).  Each event must have been recorded once
-    before (torch creates the underlying CUDA event lazily)."""
-    b = None if before is None else before.cuda_event
-    a = None if after is None else after.cuda_event
-    lib().ql_set_gemm_timing_events(b, a)
+def ql_set_gemm_timing_events(pairs=()):
+    """Record each (before, after) pair of torch.cuda.Event objects around the
+    next int8 GEMM launches of this thread, in order (empty: stop).  Each
+    event must have been recorded once before (torch creates the underlying
+    CUDA event lazily)."""
+    n = len(pairs)
+    b = (ctypes.c_void_p * max(n, 1))(*[p[0].cuda_event for p in pairs])
+    a = (ctypes.c_void_p * max(n, 1))(*[p[1].cuda_event for p in pairs])
+    lib().ql_set_gemm_timing_events(b, a, n)
 
 
 def ql_kernel_launches() -> int:

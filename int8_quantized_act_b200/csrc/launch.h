@@ -27,6 +27,15 @@ cudaError_t launch_quant_rows(const void* x, int xt, int64_t rows, int64_t cols,
                               int8_t* q, int64_t ldq, float* row_scale, int32_t* status,
                               cudaStream_t s);
 
+// Both gradient quantizations of the backward pass from one read of dY
+// [rows, cols] (contiguous, cols <= 8192): per row, q/row_scale as
+// launch_quant_rows with col_scale; per element, q2 = rne((x * rf2[row]) *
+// cf2[col]) (the column-wise codes, cf2 = 127/column amax).
+cudaError_t launch_quant_rows_cols(const void* x, int xt, int64_t rows, int64_t cols,
+                                   const float* col_scale, int8_t* q, float* row_scale,
+                                   const float* rf2, const float* cf2, int8_t* q2,
+                                   int32_t* status, cudaStream_t s);
+
 // y = x R per row (x may equal y).  xt / yt: 0 = float32, 1 = bf16.
 cudaError_t launch_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt, int64_t ldy,
                             int64_t rows, int64_t cols, int B, float hc, cudaStream_t s);

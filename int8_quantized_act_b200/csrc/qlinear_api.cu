@@ -28,15 +28,24 @@ const DeviceInfo& device_info() {
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
-thread_local cudaEvent_t t_before = nullptr;
-thread_local cudaEvent_t t_after = nullptr;
+constexpr int kMaxTimed = 16;
+thread_local cudaEvent_t t_before[kMaxTimed];
+thread_local cudaEvent_t t_after[kMaxTimed];
+thread_local int t_timed = 0;  // pairs set
+thread_local int t_next = 0;   // next pair to use
 }  // namespace
 
 void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 void gemm_timing_events(cudaEvent_t* before, cudaEvent_t* after) {
-  *before = t_before;
-  *after = t_after;
+  if (t_next < t_timed) {
+    *before = t_before[t_next];
+    *after = t_after[t_next];
+    ++t_next;
+  } else {
+    *before = nullptr;
+    *after = nullptr;
+  }
 }
 
 }  // namespace ql
@@ -91,9 +100,15 @@ T* at(void* base, size_t off) {
 
 extern "C" {
 
-void ql_set_gemm_timing_events(void* before, void* after) {
-  ql::t_before = reinterpret_cast<cudaEvent_t>(before);
-  ql::t_after = reinterpret_cast<cudaEvent_t>(after);
+void ql_set_gemm_timing_events(void* const* before, void* const* after, int n) {
+  if (n < 0 || !before || !after) n = 0;
+  if (n > ql::kMaxTimed) n = ql::kMaxTimed;
+  for (int i = 0; i < n; ++i) {
+    ql::t_before[i] = reinterpret_cast<cudaEvent_t>(before[i]);
+    ql::t_after[i] = reinterpret_cast<cudaEvent_t>(after[i]);
+  }
+  ql::t_timed = n;
+  ql::t_next = 0;
 }
 
 uint64_t ql_kernel_launches(void) { return ql::g_launches.load(std::memory_order_relaxed); }
@@ -272,6 +287,83 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   ep.ldo = K;
   ep.row_scale = s2;
   return cuda_status(ql::launch_gemm_i8(dyq, true, N, xq, true, K, N, K, M, ep, d_status, s));
+}
+
+size_t qlinear_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int hadamard_block) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return ws_layout(M, N, K, hadamard_block).total +
+         align256(static_cast<size_t>(M) * static_cast<size_t>(N));
+}
+
+int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq, const float* sw,
+                const int8_t* xq, const float* sx, int64_t K, int hadamard_block, void* dx,
+                int dxt, float* dw, float* db, void* ws, size_t ws_bytes, int32_t* d_status,
+                void* stream) {
+  if (!valid_dtype(dyt) || !valid_dtype(dxt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || M > INT32_MAX ||
+      N > INT32_MAX || K > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
+  if (N > QL_MAX_CONTRACTION || M > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
+  const WsLayout L = ws_layout(M, N, K, hadamard_block);
+  const size_t need = L.total + align256(static_cast<size_t>(M) * static_cast<size_t>(N));
+  if (!d_status || !ws) return QL_ERR_ARG;
+  if (ws_bytes < need) return QL_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return QL_ERR_ALIGN;
+  const bool fused = M > 0 && N > 0 && K > 0 && N <= 8192;
+  if (!fused) {
+    // Degenerate sizes and rows longer than the staged kernel holds: the two
+    // separate calls (stream-ordered, so they may share the workspace).
+    int r = qlinear_bwd_dx(dy, dyt, M, N, wq, sw, K, hadamard_block, dx, dxt, ws, ws_bytes,
+                           d_status, stream);
+    if (r != QL_OK) return r;
+    return qlinear_bwd_dw(dy, dyt, M, N, xq, sx, K, dw, db, ws, ws_bytes, d_status, stream);
+  }
+  if (!dy || !wq || !sw || !xq || !sx || !dx || !dw) return QL_ERR_ARG;
+  if (!aligned16(dy) || !aligned16(wq) || !aligned16(sw) || !aligned16(xq) || !aligned16(sx) ||
+      !aligned16(dx) || !aligned16(dw) || (db && !aligned16(db)))
+    return QL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  int8_t* dyq_r = at<int8_t>(ws, L.dyq);
+  int8_t* dyq_c = at<int8_t>(ws, L.total);
+  float* s1 = at<float>(ws, L.s1);
+  uint32_t* colmax = at<uint32_t>(ws, L.colmax);
+  double* colsum = at<double>(ws, L.colsum);
+  float* s2 = at<float>(ws, L.s2);
+  float* inv2 = at<float>(ws, L.inv2);
+  if (cudaMemsetAsync(colmax, 0, static_cast<size_t>(N) * 4, s) != cudaSuccess ||
+      cudaMemsetAsync(colsum, 0, static_cast<size_t>(N) * 8, s) != cudaSuccess)
+    return QL_ERR_CUDA;
+  cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, d_status, s);
+  if (e == cudaSuccess) e = ql::launch_colfinalize(colmax, colsum, N, s2, inv2, db, s);
+  if (e == cudaSuccess)
+    e = ql::launch_quant_rows_cols(dy, dyt, M, N, sw, dyq_r, s1, sx, inv2, dyq_c, d_status, s);
+  if (e != cudaSuccess) return QL_ERR_CUDA;
+  // Input gradient (as qlinear_bwd_dx after its quantization).
+  GemmEpilogue ex;
+  ex.row_scale = s1;
+  ex.ldo = K;
+  if (hadamard_block > 128) {
+    float* tmp = dxt == QL_F32 ? reinterpret_cast<float*>(dx) : at<float>(ws, L.dxtmp);
+    ex.out = tmp;
+    e = ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ex, d_status, s);
+    if (e == cudaSuccess)
+      e = ql::launch_hadamard(tmp, QL_F32, K, dx, dxt, K, M, K, hadamard_block,
+                              hadamard_c(hadamard_block), s);
+  } else {
+    ex.out = dx;
+    ex.out_bf16 = dxt == QL_BF16;
+    ex.hb = hadamard_block;
+    ex.hc = hadamard_c(hadamard_block);
+    e = ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ex, d_status, s);
+  }
+  if (e != cudaSuccess) return QL_ERR_CUDA;
+  // Weight gradient (as qlinear_bwd_dw after its quantization).
+  GemmEpilogue ew;
+  ew.out = dw;
+  ew.ldo = K;
+  ew.row_scale = s2;
+  return cuda_status(ql::launch_gemm_i8(dyq_c, true, N, xq, true, K, N, K, M, ew, d_status, s));
 }
 
 int qweight_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,

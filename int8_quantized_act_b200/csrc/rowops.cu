@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
         if (col < cols) {
           uint32_t b[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) b[i] = rne_bits(v[j][i] * inv);
+          for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(v[j][i], inv);
           *reinterpret_cast<uint2*>(q + r * ldq + col) =
               make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
         }
@@ -101,12 +101,18 @@ __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
 // registers; each warp then takes chunks wir, wir + 8, ... (CPW of them) of the
 // staged row, exactly as the register kernel does.  Waits are bounded: on a
 // time-out the CTA reports QL_ERR_TIMEOUT, lets its copies land and returns.
-template <typename InT, int CPW>
+// BT: 0 = no rotation, > 0 = block size fixed at compile time, < 0 = block
+// size B given at run time.
+// COLQ: also write q2[r, c] = rne((x[r,c] * rf2[r]) * cf2[c]) for every
+// element (the column-wise gradient codes of the weight-gradient product,
+// whose factors are known before the row pass), from the same staged row.
+template <typename InT, int CPW, int BT, bool COLQ>
 __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
     const InT* __restrict__ x, int64_t rows, int cols, int64_t ldx,
     const float* __restrict__ col_scale, int B, float hc, unsigned flags,
     int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
-    int32_t* __restrict__ status, int stages, int stage_bytes) {
+    int32_t* __restrict__ status, int stages, int stage_bytes, const float* __restrict__ rf2,
+    const float* __restrict__ cf2, int8_t* __restrict__ q2) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t s_max[8];
   __shared__ __align__(8) uint64_t s_full[8];
@@ -139,6 +145,19 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
       for (int e = 0; e < 8; ++e) cs[j][e] = 1.0f;
     }
   }
+  float cf[COLQ ? CPW : 1][8];
+  if constexpr (COLQ) {
+#pragma unroll
+    for (int j = 0; j < CPW; ++j) {
+      const int col = (warp + 8 * j) * 256 + lane * 8;
+      if (col < cols) {
+        load8(cf2 + col, cf[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cf[j][e] = 0.0f;
+      }
+    }
+  }
   int64_t done = 0;
   for (int64_t i = 0; i < mine; ++i) {
     const int st = static_cast<int>(i % stages);
@@ -169,6 +188,14 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
             v[j][2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
           }
         }
+        if constexpr (COLQ) {
+          const float f = __ldg(rf2 + r);
+          uint32_t b[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) b[e] = rne_bits_prod(__fmul_rn(v[j][e], f), cf[j][e]);
+          *reinterpret_cast<uint2*>(q2 + r * ldq + col) =
+              make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
+        }
         if (col_scale) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[j][e] = v[j][e] * cs[j][e];
@@ -177,7 +204,11 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[j][e] = 0.0f;
       }
-      if (B > 0 && chunk0 < cols) fwht_chunk(v[j], B, lane, hc);
+      if constexpr (BT > 0) {
+        if (chunk0 < cols) fwht_chunk_ct<BT>(v[j], lane, hc);
+      } else if constexpr (BT < 0) {
+        if (chunk0 < cols) fwht_chunk(v[j], B, lane, hc);
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e) mbits = max(mbits, abs_bits(v[j][e]));
     }
@@ -199,13 +230,7 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
 #pragma unroll
     for (int j = 0; j < CPW; ++j) {
       const int col = (warp + 8 * j) * 256 + lane * 8;
-      if (col < cols) {
-        uint32_t b[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) b[e] = rne_bits(v[j][e] * inv);
-        *reinterpret_cast<uint2*>(q + r * ldq + col) =
-            make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
-      }
+      if (col < cols) *reinterpret_cast<uint2*>(q + r * ldq + col) = codes8(v[j], inv);
     }
     if (threadIdx.x == 0) {
       row_scale[r] = mbits == 0 ? 0.0f : amax / 127.0f;
@@ -277,7 +302,7 @@ __global__ void __launch_bounds__(256) quant_rows_stream_kernel(
       if (col < cols) {
         uint32_t b[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = rne_bits(v[i] * inv);
+        for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(v[i], inv);
         *reinterpret_cast<uint2*>(q + r * ldq + col) =
             make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
       }
@@ -429,7 +454,7 @@ __global__ void __launch_bounds__(256) colquant_kernel(const InT* __restrict__ d
     const float s = __ldg(sx + m);
     uint32_t b[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = rne_bits((d[i] * s) * iv[i]);
+    for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], s), iv[i]);
     *reinterpret_cast<uint2*>(q + m * N + col) =
         make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
   }
@@ -473,22 +498,30 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
     const int per_sm = 200000 / (smem + 2048) > 4 ? 4 : 200000 / (smem + 2048);
     const int grid = grid_cap(rows, per_sm < 1 ? 1 : per_sm);
     const int cpw = (nch + 7) / 8;
-#define QL_QT(CPW)                                                                             \
+#define QL_QT(CPW, BT)                                                                         \
   do {                                                                                         \
     static bool attr_set[64] = {false};                                                        \
     int dev = 0;                                                                               \
     cudaGetDevice(&dev);                                                                       \
     if (dev < 64 && !attr_set[dev]) {                                                          \
-      cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW>,                                    \
+      cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW, BT, false>,                         \
                            cudaFuncAttributeMaxDynamicSharedMemorySize, 100000);               \
       attr_set[dev] = true;                                                                    \
     }                                                                                          \
-    quant_rows_tma_kernel<InT, CPW><<<grid, 256, smem, s>>>(x, rows, c, ldx, cs, B, hc, flags, \
-                                                           q, ldq, rs, st, stages, stage_bytes); \
+    quant_rows_tma_kernel<InT, CPW, BT, false><<<grid, 256, smem, s>>>(                        \
+        x, rows, c, ldx, cs, B, hc, flags, q, ldq, rs, st, stages, stage_bytes, nullptr,       \
+        nullptr, nullptr);                                                                     \
   } while (0)
-    if (cpw <= 2) QL_QT(2);
-    else if (cpw <= 3) QL_QT(3);
-    else QL_QT(4);
+#define QL_QT_B(CPW)                  \
+  do {                                \
+    if (B == 0) QL_QT(CPW, 0);        \
+    else if (B == 128) QL_QT(CPW, 128); \
+    else QL_QT(CPW, -1);              \
+  } while (0)
+    if (cpw <= 2) QL_QT_B(2);
+    else if (cpw <= 3) QL_QT_B(3);
+    else QL_QT_B(4);
+#undef QL_QT_B
 #undef QL_QT
   } else if (nch <= 64) {
     const int wpr = nch <= 1 ? 1 : nch <= 2 ? 2 : nch <= 4 ? 4 : 8;
@@ -516,7 +549,60 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
   return cudaGetLastError();
 }
 
+template <typename InT, int CPW>
+cudaError_t quant_rows_cols_t(const InT* x, int64_t rows, int c, const float* cs, int8_t* q,
+                              float* rs, const float* rf2, const float* cf2, int8_t* q2,
+                              int32_t* st, int grid, int smem, int stages, int stage_bytes,
+                              cudaStream_t s) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW, 0, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, 100000);
+    attr_set[dev] = true;
+  }
+  quant_rows_tma_kernel<InT, CPW, 0, true><<<grid, 256, smem, s>>>(
+      x, rows, c, c, cs, 0, 1.0f, 0u, q, c, rs, st, stages, stage_bytes, rf2, cf2, q2);
+  return cudaGetLastError();
+}
+
+template <typename InT>
+cudaError_t quant_rows_cols_dispatch(const void* xv, int64_t rows, int64_t cols, const float* cs,
+                                     int8_t* q, float* rs, const float* rf2, const float* cf2,
+                                     int8_t* q2, int32_t* st, cudaStream_t s) {
+  const InT* x = reinterpret_cast<const InT*>(xv);
+  const int nch = static_cast<int>((cols + 255) / 256);
+  const int64_t row_bytes = cols * static_cast<int64_t>(sizeof(InT));
+  const int stage_bytes = static_cast<int>((row_bytes + 127) / 128 * 128);
+  int stages = 98304 / stage_bytes;
+  stages = stages < 2 ? 2 : stages > 4 ? 4 : stages;
+  const int smem = stages * stage_bytes;
+  const int per_sm = 200000 / (smem + 2048) > 4 ? 4 : 200000 / (smem + 2048);
+  const int grid = grid_cap(rows, per_sm < 1 ? 1 : per_sm);
+  const int cpw = (nch + 7) / 8;
+  const int c = static_cast<int>(cols);
+  cudaError_t e;
+  if (cpw <= 1) e = quant_rows_cols_t<InT, 1>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
+  else if (cpw <= 2) e = quant_rows_cols_t<InT, 2>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
+  else if (cpw <= 3) e = quant_rows_cols_t<InT, 3>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
+  else e = quant_rows_cols_t<InT, 4>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
+  count_launches(1);
+  return e;
+}
+
 }  // namespace
+
+cudaError_t launch_quant_rows_cols(const void* x, int xt, int64_t rows, int64_t cols,
+                                   const float* col_scale, int8_t* q, float* row_scale,
+                                   const float* rf2, const float* cf2, int8_t* q2,
+                                   int32_t* status, cudaStream_t s) {
+  if (xt == QL_BF16)
+    return quant_rows_cols_dispatch<__nv_bfloat16>(x, rows, cols, col_scale, q, row_scale, rf2,
+                                                   cf2, q2, status, s);
+  return quant_rows_cols_dispatch<float>(x, rows, cols, col_scale, q, row_scale, rf2, cf2, q2,
+                                         status, s);
+}
 
 cudaError_t launch_quant_rows(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,
                               const float* col_scale, int B, float hc, unsigned flags,

@@ -60,7 +60,14 @@ __device__ __forceinline__ int code_rne(float t) {
 // like every output under QL_ERR_NONFINITE.
 constexpr float kRneMagic = 12582912.0f;  // 1.5 * 2^23
 
-__device__ __forceinline__ uint32_t rne_bits(float v) { return __float_as_uint(v + kRneMagic); }
+__device__ __forceinline__ uint32_t rne_bits(float v) { return __float_as_uint(__fadd_rn(v, kRneMagic)); }
+
+// rne_bits(t * f) with the product rounded first: __fmul_rn / __fadd_rn are
+// never merged into a fused multiply-add, which would skip the product's
+// rounding and break exact ties (t * f = k + 1/2) differently.
+__device__ __forceinline__ uint32_t rne_bits_prod(float t, float f) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(t, f), kRneMagic));
+}
 
 // Low bytes of four rne_bits words, packed little-endian.
 __device__ __forceinline__ uint32_t pack_codes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -80,7 +87,107 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
          ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
 }
 
+// -------------------------------------------------------------- packed pairs
+// sm_100a executes two float32 additions / multiplications per instruction
+// (add/sub/mul.rn.f32x2); each half is an ordinary IEEE round-to-nearest
+// operation, so results are bit-identical to the scalar forms.  A packed
+// multiply whose result feeds a packed add can be compiled into a fused
+// multiply-add (observed on this toolchain even with -fmad=false), so the
+// packed forms are used only where no product is added afterwards: the
+// butterflies (additions only) and the rotation's final scaling.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// v[i] = v[i] * c for 8 values, two per instruction.
+__device__ __forceinline__ void scale8(float (&v)[8], float c) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 r = mul2(make_float2(v[i], v[i + 1]), make_float2(c, c));
+    v[i] = r.x;
+    v[i + 1] = r.y;
+  }
+}
+
+// Codes of 8 values: rne(v[i] * inv) through the adder (see rne_bits_prod).
+__device__ __forceinline__ uint2 codes8(const float (&v)[8], float inv) {
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(v[i], inv);
+  return make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
+}
+
 // -------------------------------------------------------------- Hadamard
+// The butterflies of fwht_chunk with the block size fixed at compile time
+// (HB = 2..256) and the additions done two at a time.  Same operations in
+// the same order as fwht_chunk, so the same bits.
+template <int HB>
+__device__ __forceinline__ void fwht_chunk_ct(float (&v)[8], int lane, float c) {
+  if constexpr (HB >= 2) {  // h = 1: pairs (0,1) (2,3) (4,5) (6,7)
+    const float2 a0 = make_float2(v[0], v[2]), b0 = make_float2(v[1], v[3]);
+    const float2 a1 = make_float2(v[4], v[6]), b1 = make_float2(v[5], v[7]);
+    const float2 s0 = add2(a0, b0), d0 = sub2(a0, b0), s1 = add2(a1, b1), d1 = sub2(a1, b1);
+    v[0] = s0.x; v[1] = d0.x; v[2] = s0.y; v[3] = d0.y;
+    v[4] = s1.x; v[5] = d1.x; v[6] = s1.y; v[7] = d1.y;
+  }
+  if constexpr (HB >= 4) {  // h = 2: pairs (0,2) (1,3) (4,6) (5,7)
+    const float2 a0 = make_float2(v[0], v[1]), b0 = make_float2(v[2], v[3]);
+    const float2 a1 = make_float2(v[4], v[5]), b1 = make_float2(v[6], v[7]);
+    const float2 s0 = add2(a0, b0), d0 = sub2(a0, b0), s1 = add2(a1, b1), d1 = sub2(a1, b1);
+    v[0] = s0.x; v[1] = s0.y; v[2] = d0.x; v[3] = d0.y;
+    v[4] = s1.x; v[5] = s1.y; v[6] = d1.x; v[7] = d1.y;
+  }
+  if constexpr (HB >= 8) {  // h = 4: pairs (0,4) (1,5) (2,6) (3,7)
+    const float2 a0 = make_float2(v[0], v[1]), b0 = make_float2(v[4], v[5]);
+    const float2 a1 = make_float2(v[2], v[3]), b1 = make_float2(v[6], v[7]);
+    const float2 s0 = add2(a0, b0), d0 = sub2(a0, b0), s1 = add2(a1, b1), d1 = sub2(a1, b1);
+    v[0] = s0.x; v[1] = s0.y; v[4] = d0.x; v[5] = d0.y;
+    v[2] = s1.x; v[3] = s1.y; v[6] = d1.x; v[7] = d1.y;
+  }
+#pragma unroll
+  for (int h = 8; h < HB; h <<= 1) {
+    const int d = h >> 3;
+    const uint32_t flip = (lane & d) ? 0x80000000u : 0u;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const float p0 = __shfl_xor_sync(0xFFFFFFFFu, v[i], d);
+      const float p1 = __shfl_xor_sync(0xFFFFFFFFu, v[i + 1], d);
+      const float2 r = add2(make_float2(p0, p1),
+                            make_float2(__uint_as_float(__float_as_uint(v[i]) ^ flip),
+                                        __uint_as_float(__float_as_uint(v[i + 1]) ^ flip)));
+      v[i] = r.x;
+      v[i + 1] = r.y;
+    }
+  }
+  scale8(v, c);
+}
+
 // Block-Hadamard rotation of one 256-element chunk spread across a warp,
 // lane l holding elements 8l..8l+7 in v.  For blocks of B elements (B a power
 // of two, 2..256) the Sylvester butterflies run for h = 1, 2, ..., B/2 in that

@@ -61,6 +61,13 @@ def fake(addr):
     return P(addr)
 
 
+def test_bwd_workspace_formula(L):
+    def a(x):
+        return (x + 255) // 256 * 256
+    for (M, N, K, B) in ((12000, 7168, 5376, 128), (17, 144, 512, 256)):
+        assert ql.qlinear_bwd_workspace_bytes(M, N, K, B) == ql.qlinear_workspace_bytes(M, N, K, B) + a(M * N)
+
+
 def test_host_validation_returns_before_any_launch(L):
     A = 0x10000  # 16-byte aligned fake address
     # bad dtype / block / flags

@@ -237,6 +237,55 @@ def test_bwd_dw_int32_accumulator_bit_exact():
     assert np.array_equal(host(db), dyi.sum(0).astype(np.float32))
 
 
+# ------------------------------------------------------------------ combined backward
+def gpu_bwd(dy_t, wq, sw, xq, sx, B, dxt):
+    M, N = dy_t.shape
+    K = wq.shape[1]
+    ws = torch.empty(ql.qlinear_bwd_workspace_bytes(M, N, K, B), dtype=torch.uint8, device="cuda")
+    dx = torch.empty((M, K), dtype=dxt, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    db = torch.empty(N, dtype=torch.float32, device="cuda")
+    st = new_status()
+    ql.qlinear_bwd(dy_t, wq, sw, xq, sx, B, dx, dw, db, ws, st)
+    assert status_word(st) == 0
+    return dx, dw, db, ws
+
+
+BWD_CASES = [
+    # M, N, K, block, dy dtype, dx dtype
+    (32, 128, 256, 256, torch.float32, torch.float32),
+    (300, 272, 384, 128, torch.bfloat16, torch.bfloat16),
+    (129, 528, 1040, 16, torch.float32, torch.bfloat16),
+    (1000, 7168, 256, 0, torch.bfloat16, torch.float32),   # 28 chunks per dY row
+    (17, 144, 512, 64, torch.bfloat16, torch.float32),
+    (600, 8208, 128, 0, torch.float32, torch.float32),     # > 8192 columns: separate passes
+]
+
+
+@pytest.mark.parametrize("M,N,K,B,dyt,dxt", BWD_CASES)
+def test_bwd_combined_matches_oracle_and_separate_calls(M, N, K, B, dyt, dxt):
+    x_t, w, _, dy_t = layer_inputs(M, K, N, dyt, 400 + M + N)
+    wq, sw = prep_weight(w, B)
+    xq_np, sx_np, _ = oracle.quantize_rows(x_t.float().numpy(), B=B)
+    xq, sx = dev(xq_np), dev(sx_np)
+    dyd = dev(dy_t)
+    dx, dw, db, ws = gpu_bwd(dyd, wq, sw, xq, sx, B, dxt)
+    # the same results as the two separate calls, bit for bit
+    dx1, _ = gpu_dx(dyd, wq, sw, B, dxt)
+    dw1, db1, _ = gpu_dw(dyd, xq, sx)
+    assert torch.equal(dx, dx1) and torch.equal(dw, dw1) and torch.equal(db, db1)
+    dy32 = dy_t.float().numpy()
+    rdx, rq, rs1, _ = oracle.bwd_dx(dy32, host(wq), host(sw), B)
+    rdw, rdb, rqc, rs2, _ = oracle.bwd_dw(dy32, xq_np, sx_np)
+    acc, _ = oracle.gemm_nn(rq, host(wq))
+    pre = acc.astype(np.float64) * rs1[:, None]
+    assert_close(host(dx), rdx, rotated_magnitude(pre, B) if B else np.abs(pre),
+                 bf16=(dxt == torch.bfloat16), what="dX")
+    acc, _ = oracle.gemm_tn(rqc, xq_np)
+    assert_close(host(dw), rdw, np.abs(acc.astype(np.float64) * rs2[:, None]), what="dW")
+    assert_close(host(db), rdb, np.abs(dy32.astype(np.float64)).sum(0), what="db")
+
+
 # ------------------------------------------------------------------ full size
 def _sample_rows(M, n, seed):
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -274,6 +323,8 @@ def test_full_layer_sampled(M):
                  bf16=True, what="dX")
 
     dw, db, ws = gpu_dw(dy_t, xq, sx)
+    dx2, dw2, db2, _ = gpu_bwd(dy_t, wq, sw, xq, sx, B, torch.bfloat16)
+    assert torch.equal(dx2, dx) and torch.equal(dw2, dw) and torch.equal(db2, db)
     cols = _sample_rows(N, 12, M + 1)
     rdw, rdb, rqc, rs2, _ = oracle.bwd_dw(d["dy"][:, cols], xq_np, sx_np)
     gq = host(ws[: M * N]).view(np.int8).reshape(M, N)
