@@ -86,7 +86,9 @@ typedef enum { QL_SGD = 0, QL_ADAMW = 1 } ql_optim_kind;
 /* Optimizer hyper-parameters.  SGD: w' = w - lr*g (no momentum; weight_decay
  * must be 0).  AdamW (decoupled weight decay): w1 = w*(1-lr*wd);
  * m' = b1*m + (1-b1)*g; v' = b2*v + (1-b2)*g*g;
- * w' = w1 - (lr/(1-b1^t)) * m' / (sqrt(v'/(1-b2^t)) + eps). */
+ * w' = w1 - (lr/(1-b1^t)) * m' / (sqrt(v') * (1/sqrt(1-b2^t)) + eps), the
+ * factors lr/(1-b1^t), 1/sqrt(1-b2^t), 1-lr*wd, 1-b1, 1-b2 each computed in
+ * float64 on the host and rounded once to float32. */
 typedef struct {
     int kind; /* ql_optim_kind */
     float lr, beta1, beta2, eps, weight_decay;

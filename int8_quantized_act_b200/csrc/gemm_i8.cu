@@ -55,6 +55,23 @@ struct Epi {
   float hc;
 };
 
+// Tile t of a tiles_m x tiles_n grid in grouped order: runs of `group`
+// tile-rows are walked column by column, so the tiles in flight at any
+// moment form a compact block and share their operand stripes in L2.
+// group = 1 is plain row-major order (best when the B operand fits in L2 and
+// every tile-row reuses it); the weight gradient, whose operands are both
+// long stripes of the whole contraction, uses groups of 8.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int group, int& tm,
+                                            int& tn) {
+  const int per_group = group * tiles_n;
+  const int g = t / per_group;
+  const int first = g * group;
+  const int rows = tiles_m - first < group ? tiles_m - first : group;
+  const int r = t - g * per_group;
+  tm = first + r % rows;
+  tn = r / rows;
+}
+
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
   static_assert(N % 32 == 0, "chunks of 32 columns");
@@ -162,7 +179,7 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
 template <bool A_MN, bool B_MN, typename OutT, int HB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int tiles_m, int tiles_n, int kblocks, Epi ep, int32_t* status) {
+                   int tiles_m, int tiles_n, int kblocks, int group, Epi ep, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -212,7 +229,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0, issued = 0, issued_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int tm = t / tiles_n, tn = t % tiles_n;
+        int tm, tn;
+        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) {
             ok = false;
@@ -292,7 +310,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-      const int tm = t / tiles_n, tn = t % tiles_n;
+      int tm, tn;
+        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
       tc_fence_after();
       epilogue_tile<OutT, HB>(ep, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
@@ -332,7 +351,7 @@ template <bool A_MN, bool B_MN, typename OutT, int HB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int tiles_m, int tiles_n,
-                        int kblocks, Epi ep, int32_t* status) {
+                        int kblocks, int group, Epi ep, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -387,7 +406,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0, armed = 0, armed_phase = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs) {
-        const int tm = t / tiles_n, tn = t % tiles_n;
+        int tm, tn;
+        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
         const int a_row = tm * 256 + static_cast<int>(rank) * 128;
         const int b_col = tn * 256 + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -468,7 +488,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     uint32_t acc = 0, acc_phase = 0;
     for (int t = pair; t < num_tiles; t += npairs) {
-      const int tm = t / tiles_n, tn = t % tiles_n;
+      int tm, tn;
+        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
       tc_fence_after();
       epilogue_tile<OutT, HB>(ep, tmem_base + acc * BN, quarter, lane,
@@ -514,15 +535,7 @@ EncodeTiledFn encode_fn() {
 // box_inner x box_outer bytes, 128-byte swizzle, zero fill out of bounds.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
                uint32_t box_inner, uint32_t box_outer) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {pitch};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_tmap_2d(m, 1, base, inner, outer, pitch, box_inner, box_outer, true);
 }
 
 // Clusters of two that can be resident together (cached per device).
@@ -568,7 +581,8 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
-  kern<<<2 * pairs, NUM_THREADS, PSMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, ep, status);
+  kern<<<2 * pairs, NUM_THREADS, PSMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, A_MN ? 8 : 1,
+                                                    ep, status);
   cudaError_t e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
   count_launches(1);
@@ -594,7 +608,8 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, ep, status);
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, A_MN ? 8 : 1, ep,
+                                              status);
   cudaError_t e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
   count_launches(1);
@@ -640,6 +655,24 @@ cudaError_t dispatch_dx(bool pair, const CUtensorMap& ta, const CUtensorMap& tb,
 }
 
 }  // namespace
+
+bool encode_tmap_2d(CUtensorMap* m, int elem_bytes, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+                    bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
                            int64_t ldb, int64_t rows, int64_t cols, int64_t kc,

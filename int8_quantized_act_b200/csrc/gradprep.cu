@@ -1,0 +1,363 @@
+// gradprep.cu - the gradient quantizations of the backward pass, streamed
+// through shared memory by the tensor-memory-access (TMA) engine.
+//
+// The backward formulas (dX = s'[m] * quant_row(dY * s_w[n]) W_q and
+// dW = s''[n] * quant_col(dY * s_x[m])^T X_q) need, per column n, the max over
+// m of |dY * s_x| and, per row m, the max over n of |dY * s_w|, before any code
+// can be written.  Pass 1 (colstats) gathers the column maxima, the column
+// sums (the bias gradient) and, optionally, the row maxima; pass 2
+// (dualquant) writes one or both int8 code sets elementwise.
+//
+// Both passes stream dY in tiles of 256 columns x 32 rows (bf16) or 16 rows
+// (float32), 16 KB each, through a 4-stage ring: a producer warp issues one
+// TMA load per tile (rows / columns past the matrix read as zero) while 8
+// consumer warps work on earlier tiles, so ~64 KB per CTA are in flight
+// without tying up registers.  Block (x, y) owns column block x and a
+// contiguous run of row tiles, so per-column state stays in registers.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "launch.h"
+#include "rowops.cuh"
+#include "sm100.cuh"
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+namespace {
+
+constexpr int kCols = 256;        // columns per tile (8 per lane)
+constexpr int kStages = 4;
+constexpr int kTileBytes = 16384;
+constexpr int kThreads = 288;     // 8 consumer warps + 1 producer warp
+
+template <typename InT>
+struct Tile {
+  static constexpr int kRows = kTileBytes / (kCols * static_cast<int>(sizeof(InT)));  // 32 / 16
+  static constexpr int kRowsPerWarp = kRows / 8;
+};
+
+// 8 consecutive elements of a staged row as float32.
+template <typename InT>
+__device__ __forceinline__ void smem_load8(const uint8_t* p, float (&v)[8]) {
+  if constexpr (sizeof(InT) == 4) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = __uint_as_float(w[e] << 16);
+      v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  }
+}
+
+// The ring shared by both passes: tiles t0 .. t1-1 (row tiles) of column
+// block cb.  run() calls body(tile, stage_ptr) on the consumer warps for every
+// tile in order; the producer warp keeps up to kStages tiles in flight.
+struct Ring {
+  uint8_t* buf;
+  uint64_t* full;
+  uint64_t* empty;
+  volatile int* abort_flag;
+
+  __device__ void init(int tid) {
+    if (tid == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(smem_u32(&full[s]), 1);
+        mbar_init(smem_u32(&empty[s]), 8);
+      }
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+  }
+
+  // Producer (one thread): load tile t of column block cb into each free stage.
+  __device__ void produce(const CUtensorMap* tm, int cb, int t0, int t1, int rows_per_tile) {
+    uint32_t issued = 0, issued_phase = 0;
+    for (int t = t0, k = 0; t < t1; ++t, ++k) {
+      const int s = k % kStages;
+      const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
+      if (k >= kStages && !mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag)) break;
+      mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
+      tma_load_2d(smem_u32(buf + s * kTileBytes), tm, smem_u32(&full[s]), cb * kCols,
+                  t * rows_per_tile);
+      issued |= 1u << s;
+      issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
+    }
+    // Every copy issued must land before the CTA may exit.
+    for (int s = 0; s < kStages; ++s)
+      if (issued & (1u << s)) mbar_wait_drain(smem_u32(&full[s]), (issued_phase >> s) & 1u);
+  }
+
+  // Consumer warp: wait for tile k, run body, release the stage.
+  template <typename F>
+  __device__ void consume(int t0, int t1, int lane, F&& body) {
+    for (int t = t0, k = 0; t < t1; ++t, ++k) {
+      const int s = k % kStages;
+      const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
+      if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) break;
+      body(t, buf + s * kTileBytes);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+    }
+  }
+};
+
+// Pass 1: colmax[n] = bits of max |dY*sx[m]|, colsum[n] += sum dY (float32
+// within a block's rows, float64 across blocks), and with ROWMAX
+// rowmax[m] = bits of max |dY*sw[n]| (one atomic per row per column block).
+template <typename InT, bool ROWMAX>
+__global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
+    const __grid_constant__ CUtensorMap tm, int64_t M, int N, const float* __restrict__ sx,
+    uint32_t* __restrict__ colmax, double* __restrict__ colsum, const float* __restrict__ sw,
+    uint32_t* __restrict__ rowmax, int32_t* __restrict__ status, int tiles_per_cta) {
+  using T = Tile<InT>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* buf = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t s_full[kStages], s_empty[kStages];
+  __shared__ volatile int s_abort;
+  // The final per-column reduction reuses the (drained) ring buffer.
+  uint32_t(*s_max)[kCols] = reinterpret_cast<uint32_t(*)[kCols]>(buf);
+  float(*s_sum)[kCols] = reinterpret_cast<float(*)[kCols]>(buf + 8 * kCols * 4);
+  Ring ring{buf, s_full, s_empty, &s_abort};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  ring.init(tid);
+  __syncthreads();
+  const int cb = blockIdx.x;
+  const int tiles = static_cast<int>((M + T::kRows - 1) / T::kRows);
+  const int t0 = blockIdx.y * tiles_per_cta;
+  const int t1 = t0 + tiles_per_cta < tiles ? t0 + tiles_per_cta : tiles;
+  const int col = cb * kCols + lane * 8;
+  uint32_t mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  float sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  uint32_t rbad = 0;
+  if (warp == 8) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm);
+      ring.produce(&tm, cb, t0, t1, T::kRows);
+    }
+    __syncwarp();
+  } else {
+    float w8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (ROWMAX && col < N) load8(sw + col, w8);
+    ring.consume(t0, t1, lane, [&](int t, const uint8_t* tile) {
+#pragma unroll
+      for (int j = 0; j < T::kRowsPerWarp; ++j) {
+        const int r = warp * T::kRowsPerWarp + j;
+        const int64_t m = static_cast<int64_t>(t) * T::kRows + r;
+        if (m < M) {  // warp-uniform
+          float d[8];
+          smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
+          const float f = __ldg(sx + m);
+          uint32_t rb = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            mx[i] = max(mx[i], abs_bits(__fmul_rn(d[i], f)));
+            sm[i] += d[i];
+            if (ROWMAX) rb = max(rb, abs_bits(__fmul_rn(d[i], w8[i])));
+          }
+          if (ROWMAX) {
+            rb = __reduce_max_sync(0xFFFFFFFFu, rb);
+            if (lane == 0) atomicMax(rowmax + m, rb);
+            rbad = max(rbad, rb);
+          }
+        }
+      }
+    });
+  }
+  __syncthreads();  // ring drained (the producer waited for its copies): reuse it
+  if (warp < 8) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      s_max[warp][i * 32 + lane] = mx[i];  // column lane*8+i at slot i*32+lane
+      s_sum[warp][i * 32 + lane] = sm[i];
+    }
+  }
+  __syncthreads();
+  if (tid < kCols && cb * kCols + tid < N) {
+    const int slot = (tid % 8) * 32 + tid / 8;
+    uint32_t a = 0;
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      a = max(a, s_max[w][slot]);
+      t += static_cast<double>(s_sum[w][slot]);
+    }
+    // inf/NaN patterns sort above every finite value: report them (the
+    // affected outputs are unspecified).
+    if (a >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    atomicMax(colmax + cb * kCols + tid, a);
+    atomicAdd(colsum + cb * kCols + tid, t);
+  }
+  if (ROWMAX && rbad >= kInfBits && lane == 0) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  if (tid == 0 && s_abort) atomicOr(status, 1 << QL_ERR_TIMEOUT);
+}
+
+// Pass 2: q2[m,n] = rne((dY*rs2[m]) * cinv2[n]) and, with Q1,
+// q1[m,n] = rne((dY*cs1[n]) * rinv1[m]).
+template <typename InT, bool Q1>
+__global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
+    const __grid_constant__ CUtensorMap tm, int64_t M, int N, const float* __restrict__ cs1,
+    const float* __restrict__ rinv1, const float* __restrict__ rs2,
+    const float* __restrict__ cinv2, int8_t* __restrict__ q1, int8_t* __restrict__ q2,
+    int32_t* __restrict__ status, int tiles_per_cta) {
+  using T = Tile<InT>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* buf = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t s_full[kStages], s_empty[kStages];
+  __shared__ volatile int s_abort;
+  Ring ring{buf, s_full, s_empty, &s_abort};
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  ring.init(tid);
+  __syncthreads();
+  const int cb = blockIdx.x;
+  const int tiles = static_cast<int>((M + T::kRows - 1) / T::kRows);
+  const int t0 = blockIdx.y * tiles_per_cta;
+  const int t1 = t0 + tiles_per_cta < tiles ? t0 + tiles_per_cta : tiles;
+  const int col = cb * kCols + lane * 8;
+  const bool cv = col < N;
+  if (warp == 8) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm);
+      ring.produce(&tm, cb, t0, t1, T::kRows);
+    }
+    __syncwarp();
+  } else {
+    float w8[8] = {0, 0, 0, 0, 0, 0, 0, 0}, iv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (cv) {
+      load8(cinv2 + col, iv);
+      if (Q1) load8(cs1 + col, w8);
+    }
+    ring.consume(t0, t1, lane, [&](int t, const uint8_t* tile) {
+#pragma unroll
+      for (int j = 0; j < T::kRowsPerWarp; ++j) {
+        const int r = warp * T::kRowsPerWarp + j;
+        const int64_t m = static_cast<int64_t>(t) * T::kRows + r;
+        if (m < M && cv) {
+          float d[8];
+          smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
+          const float f2 = __ldg(rs2 + m);
+          uint32_t b[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], f2), iv[i]);
+          *reinterpret_cast<uint2*>(q2 + m * N + col) =
+              make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
+          if (Q1) {
+            const float r1 = __ldg(rinv1 + m);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], w8[i]), r1);
+            *reinterpret_cast<uint2*>(q1 + m * N + col) =
+                make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
+          }
+        }
+      }
+    });
+  }
+  __syncthreads();
+  if (tid == 0 && s_abort) atomicOr(status, 1 << QL_ERR_TIMEOUT);
+}
+
+constexpr int kSmemBytes = 1024 + kStages * kTileBytes;
+
+struct Grid {
+  dim3 grid;
+  int tiles_per_cta;
+};
+
+// Column blocks x row groups, about `per_sm` resident CTAs per SM in total.
+Grid plan(int64_t M, int64_t N, int rows_per_tile, int per_sm) {
+  const int cbs = static_cast<int>((N + kCols - 1) / kCols);
+  const int tiles = static_cast<int>((M + rows_per_tile - 1) / rows_per_tile);
+  int groups = device_info().sms * per_sm / cbs;  // round down: one wave of resident CTAs
+  if (groups > tiles) groups = tiles;
+  if (groups < 1) groups = 1;
+  const int per = (tiles + groups - 1) / groups;
+  groups = (tiles + per - 1) / per;
+  return {dim3(static_cast<unsigned>(cbs), static_cast<unsigned>(groups)), per};
+}
+
+// Opt kernel K in to kSmemBytes of dynamic shared memory, once per device
+// (one flag set per kernel: the template is keyed on the kernel itself).
+template <auto K>
+void allow_smem() {
+  static bool done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !done[dev]) {
+    cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    done[dev] = true;
+  }
+}
+
+template <typename InT>
+bool dy_map(CUtensorMap* tm, const void* dy, int64_t M, int64_t N) {
+  return encode_tmap_2d(tm, sizeof(InT), dy, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                        static_cast<uint64_t>(N) * sizeof(InT), kCols, Tile<InT>::kRows, false);
+}
+
+template <typename InT>
+cudaError_t colstats_t(const void* dy, int64_t M, int64_t N, const float* sx, uint32_t* colmax,
+                       double* colsum, const float* sw, uint32_t* rowmax, int32_t* status,
+                       cudaStream_t s) {
+  CUtensorMap tm;
+  if (!dy_map<InT>(&tm, dy, M, N)) return cudaErrorInvalidValue;
+  const Grid g = plan(M, N, Tile<InT>::kRows, 3);
+  if (rowmax) {
+    allow_smem<colstats_tma_kernel<InT, true>>();
+    colstats_tma_kernel<InT, true><<<g.grid, kThreads, kSmemBytes, s>>>(
+        tm, M, static_cast<int>(N), sx, colmax, colsum, sw, rowmax, status, g.tiles_per_cta);
+  } else {
+    allow_smem<colstats_tma_kernel<InT, false>>();
+    colstats_tma_kernel<InT, false><<<g.grid, kThreads, kSmemBytes, s>>>(
+        tm, M, static_cast<int>(N), sx, colmax, colsum, sw, rowmax, status, g.tiles_per_cta);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+template <typename InT>
+cudaError_t dualquant_t(const void* dy, int64_t M, int64_t N, const float* cs1,
+                        const float* rinv1, const float* rs2, const float* cinv2, int8_t* q1,
+                        int8_t* q2, int32_t* status, cudaStream_t s) {
+  CUtensorMap tm;
+  if (!dy_map<InT>(&tm, dy, M, N)) return cudaErrorInvalidValue;
+  const Grid g = plan(M, N, Tile<InT>::kRows, 3);
+  if (q1) {
+    allow_smem<dualquant_tma_kernel<InT, true>>();
+    dualquant_tma_kernel<InT, true><<<g.grid, kThreads, kSmemBytes, s>>>(
+        tm, M, static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
+  } else {
+    allow_smem<dualquant_tma_kernel<InT, false>>();
+    dualquant_tma_kernel<InT, false><<<g.grid, kThreads, kSmemBytes, s>>>(
+        tm, M, static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
+                            uint32_t* colmax, double* colsum, const float* sw, uint32_t* rowmax,
+                            int32_t* status, cudaStream_t s) {
+  if (dyt == QL_BF16)
+    return colstats_t<__nv_bfloat16>(dy, M, N, sx, colmax, colsum, sw, rowmax, status, s);
+  return colstats_t<float>(dy, M, N, sx, colmax, colsum, sw, rowmax, status, s);
+}
+
+cudaError_t launch_dualquant(const void* dy, int dyt, int64_t M, int64_t N, const float* cs1,
+                             const float* rinv1, const float* rs2, const float* cinv2,
+                             int8_t* q1, int8_t* q2, int32_t* status, cudaStream_t s) {
+  if (dyt == QL_BF16)
+    return dualquant_t<__nv_bfloat16>(dy, M, N, cs1, rinv1, rs2, cinv2, q1, q2, status, s);
+  return dualquant_t<float>(dy, M, N, cs1, rinv1, rs2, cinv2, q1, q2, status, s);
+}
+
+}  // namespace ql

@@ -19,6 +19,13 @@ const DeviceInfo& device_info();  // current device, cached
 void count_launches(int n);
 void gemm_timing_events(cudaEvent_t* before, cudaEvent_t* after);
 
+// 2-D tensor map over a row-major [outer][inner] array of elem_bytes-byte
+// elements (raw bits; the pitch in bytes), boxes of box_inner x box_outer
+// elements, out-of-range elements read as zero; 128-byte swizzle or none.
+bool encode_tmap_2d(CUtensorMap* m, int elem_bytes, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+                    bool swizzle128);
+
 // -------------------------------------------------------------- row kernels
 // Per-row quantization (optionally scaled per column and rotated); see
 // qlinear_quantize_rows.  xt: 0 = float32, 1 = bf16.
@@ -27,31 +34,30 @@ cudaError_t launch_quant_rows(const void* x, int xt, int64_t rows, int64_t cols,
                               int8_t* q, int64_t ldq, float* row_scale, int32_t* status,
                               cudaStream_t s);
 
-// Both gradient quantizations of the backward pass from one read of dY
-// [rows, cols] (contiguous, cols <= 8192): per row, q/row_scale as
-// launch_quant_rows with col_scale; per element, q2 = rne((x * rf2[row]) *
-// cf2[col]) (the column-wise codes, cf2 = 127/column amax).
-cudaError_t launch_quant_rows_cols(const void* x, int xt, int64_t rows, int64_t cols,
-                                   const float* col_scale, int8_t* q, float* row_scale,
-                                   const float* rf2, const float* cf2, int8_t* q2,
-                                   int32_t* status, cudaStream_t s);
-
 // y = x R per row (x may equal y).  xt / yt: 0 = float32, 1 = bf16.
 cudaError_t launch_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt, int64_t ldy,
                             int64_t rows, int64_t cols, int B, float hc, cudaStream_t s);
 
 // Column statistics of t = dY[m,n]*s_x[m]: colmax[n] = bits of max|t|
-// (atomicMax; caller zeroes), colsum[n] += sum_m dY[m,n] in float64.
+// (atomicMax; caller zeroes), colsum[n] += sum_m dY[m,n] in float64.  With
+// rowmax != NULL also rowmax[m] = bits of max_n |dY[m,n]*sw[n]| (caller zeroes).
 cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
-                            uint32_t* colmax, double* colsum, int32_t* status, cudaStream_t s);
+                            uint32_t* colmax, double* colsum, const float* sw, uint32_t* rowmax,
+                            int32_t* status, cudaStream_t s);
+
+// s1[m] = amax/127, inv1[m] = 127/amax of the row maxima (0 for a zero row).
+cudaError_t launch_rowfinalize(const uint32_t* rowmax, int64_t M, float* s1, float* inv1,
+                               cudaStream_t s);
+
+// q2 = rne((dY*rs2[m])*cinv2[n]) and, if q1 != NULL, q1 = rne((dY*cs1[n])*rinv1[m]),
+// both [M,N] (dY streamed through shared memory by TMA).
+cudaError_t launch_dualquant(const void* dy, int dyt, int64_t M, int64_t N, const float* cs1,
+                             const float* rinv1, const float* rs2, const float* cinv2,
+                             int8_t* q1, int8_t* q2, int32_t* status, cudaStream_t s);
 
 // s2[n] = amax/127, inv2[n] = 127/amax (0 for a zero column), db[n] = colsum.
 cudaError_t launch_colfinalize(const uint32_t* colmax, const double* colsum, int64_t N,
                                float* s2, float* inv2, float* db, cudaStream_t s);
-
-// dYq_c[m,n] = clamp(rne((dY[m,n]*s_x[m]) * inv2[n]), +-127).
-cudaError_t launch_colquant(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
-                            const float* inv2, int8_t* q, cudaStream_t s);
 
 // out[r, :] = bias (or 0), dtype ot; used when the contraction is empty.
 cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, const float* bias,
@@ -81,7 +87,7 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
 // -------------------------------------------------------------- update
 struct UpdateConsts {
   int kind = 0;  // 0 SGD, 1 AdamW
-  float lr = 0, a = 1, st = 0, bc2 = 1, b1 = 0, b2 = 0, omb1 = 0, omb2 = 0, eps = 0;
+  float lr = 0, a = 1, st = 0, rbc2 = 1, b1 = 0, b2 = 0, omb1 = 0, omb2 = 0, eps = 0;
 };
 
 cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,

@@ -278,9 +278,11 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   if (cudaMemsetAsync(colmax, 0, static_cast<size_t>(N) * 4, s) != cudaSuccess ||
       cudaMemsetAsync(colsum, 0, static_cast<size_t>(N) * 8, s) != cudaSuccess)
     return QL_ERR_CUDA;
-  cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, d_status, s);
+  cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, nullptr, nullptr,
+                                      d_status, s);
   if (e == cudaSuccess) e = ql::launch_colfinalize(colmax, colsum, N, s2, inv2, db, s);
-  if (e == cudaSuccess) e = ql::launch_colquant(dy, dyt, M, N, sx, inv2, dyq, s);
+  if (e == cudaSuccess)
+    e = ql::launch_dualquant(dy, dyt, M, N, nullptr, nullptr, sx, inv2, nullptr, dyq, d_status, s);
   if (e != cudaSuccess || K == 0) return cuda_status(e);
   GemmEpilogue ep;
   ep.out = dw;
@@ -289,10 +291,16 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   return cuda_status(ql::launch_gemm_i8(dyq, true, N, xq, true, K, N, K, M, ep, d_status, s));
 }
 
+// qlinear_bwd's workspace: the common layout, then the column-quantized
+// codes [M*N], the row maxima [M] and 127/row max [M].
+size_t bwd_extra(int64_t M, int64_t N) {
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(N)) +
+         2 * align256(4 * static_cast<size_t>(M > 0 ? M : 1));
+}
+
 size_t qlinear_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int hadamard_block) {
   if (M < 0 || N < 0 || K < 0) return 0;
-  return ws_layout(M, N, K, hadamard_block).total +
-         align256(static_cast<size_t>(M) * static_cast<size_t>(N));
+  return ws_layout(M, N, K, hadamard_block).total + bwd_extra(M, N);
 }
 
 int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq, const float* sw,
@@ -306,14 +314,14 @@ int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
   if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
   if (N > QL_MAX_CONTRACTION || M > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
   const WsLayout L = ws_layout(M, N, K, hadamard_block);
-  const size_t need = L.total + align256(static_cast<size_t>(M) * static_cast<size_t>(N));
+  const size_t need = L.total + bwd_extra(M, N);
   if (!d_status || !ws) return QL_ERR_ARG;
   if (ws_bytes < need) return QL_ERR_SHAPE;
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return QL_ERR_ALIGN;
-  const bool fused = M > 0 && N > 0 && K > 0 && N <= 8192;
+  const bool fused = M > 0 && N > 0 && K > 0;
   if (!fused) {
-    // Degenerate sizes and rows longer than the staged kernel holds: the two
-    // separate calls (stream-ordered, so they may share the workspace).
+    // Degenerate sizes: the two separate calls (stream-ordered, so they may
+    // share the workspace).
     int r = qlinear_bwd_dx(dy, dyt, M, N, wq, sw, K, hadamard_block, dx, dxt, ws, ws_bytes,
                            d_status, stream);
     if (r != QL_OK) return r;
@@ -326,18 +334,25 @@ int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
   cudaStream_t s = as_stream(stream);
   int8_t* dyq_r = at<int8_t>(ws, L.dyq);
   int8_t* dyq_c = at<int8_t>(ws, L.total);
+  const size_t rm_off = L.total + align256(static_cast<size_t>(M) * static_cast<size_t>(N));
+  uint32_t* rowmax = at<uint32_t>(ws, rm_off);
+  float* inv1 = at<float>(ws, rm_off + align256(4 * static_cast<size_t>(M)));
   float* s1 = at<float>(ws, L.s1);
   uint32_t* colmax = at<uint32_t>(ws, L.colmax);
   double* colsum = at<double>(ws, L.colsum);
   float* s2 = at<float>(ws, L.s2);
   float* inv2 = at<float>(ws, L.inv2);
+  // Pass 1 over dY: column maxima of |dY*s_x| and column sums, row maxima of
+  // |dY*s_w|; pass 2: both code sets, elementwise.
   if (cudaMemsetAsync(colmax, 0, static_cast<size_t>(N) * 4, s) != cudaSuccess ||
-      cudaMemsetAsync(colsum, 0, static_cast<size_t>(N) * 8, s) != cudaSuccess)
+      cudaMemsetAsync(colsum, 0, static_cast<size_t>(N) * 8, s) != cudaSuccess ||
+      cudaMemsetAsync(rowmax, 0, static_cast<size_t>(M) * 4, s) != cudaSuccess)
     return QL_ERR_CUDA;
-  cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, d_status, s);
+  cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, sw, rowmax, d_status, s);
   if (e == cudaSuccess) e = ql::launch_colfinalize(colmax, colsum, N, s2, inv2, db, s);
+  if (e == cudaSuccess) e = ql::launch_rowfinalize(rowmax, M, s1, inv1, s);
   if (e == cudaSuccess)
-    e = ql::launch_quant_rows_cols(dy, dyt, M, N, sw, dyq_r, s1, sx, inv2, dyq_c, d_status, s);
+    e = ql::launch_dualquant(dy, dyt, M, N, sw, inv1, sx, inv2, dyq_r, dyq_c, d_status, s);
   if (e != cudaSuccess) return QL_ERR_CUDA;
   // Input gradient (as qlinear_bwd_dx after its quantization).
   GemmEpilogue ex;
@@ -392,7 +407,7 @@ int qweight_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64
     const double t = static_cast<double>(step);
     c.a = static_cast<float>(1.0 - static_cast<double>(opt->lr) * static_cast<double>(opt->weight_decay));
     c.st = static_cast<float>(static_cast<double>(opt->lr) / (1.0 - std::pow(static_cast<double>(opt->beta1), t)));
-    c.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(opt->beta2), t));
+    c.rbc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(opt->beta2), t)));
     c.b1 = opt->beta1;
     c.b2 = opt->beta2;
     c.omb1 = static_cast<float>(1.0 - static_cast<double>(opt->beta1));

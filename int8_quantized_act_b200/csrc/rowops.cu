@@ -103,16 +103,12 @@ __global__ void __launch_bounds__(256) quant_rows_reg_kernel(
 // time-out the CTA reports QL_ERR_TIMEOUT, lets its copies land and returns.
 // BT: 0 = no rotation, > 0 = block size fixed at compile time, < 0 = block
 // size B given at run time.
-// COLQ: also write q2[r, c] = rne((x[r,c] * rf2[r]) * cf2[c]) for every
-// element (the column-wise gradient codes of the weight-gradient product,
-// whose factors are known before the row pass), from the same staged row.
-template <typename InT, int CPW, int BT, bool COLQ>
+template <typename InT, int CPW, int BT>
 __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
     const InT* __restrict__ x, int64_t rows, int cols, int64_t ldx,
     const float* __restrict__ col_scale, int B, float hc, unsigned flags,
     int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
-    int32_t* __restrict__ status, int stages, int stage_bytes, const float* __restrict__ rf2,
-    const float* __restrict__ cf2, int8_t* __restrict__ q2) {
+    int32_t* __restrict__ status, int stages, int stage_bytes) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t s_max[8];
   __shared__ __align__(8) uint64_t s_full[8];
@@ -145,19 +141,6 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
       for (int e = 0; e < 8; ++e) cs[j][e] = 1.0f;
     }
   }
-  float cf[COLQ ? CPW : 1][8];
-  if constexpr (COLQ) {
-#pragma unroll
-    for (int j = 0; j < CPW; ++j) {
-      const int col = (warp + 8 * j) * 256 + lane * 8;
-      if (col < cols) {
-        load8(cf2 + col, cf[j]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cf[j][e] = 0.0f;
-      }
-    }
-  }
   int64_t done = 0;
   for (int64_t i = 0; i < mine; ++i) {
     const int st = static_cast<int>(i % stages);
@@ -187,14 +170,6 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
             v[j][2 * e] = __uint_as_float(w4[e] << 16);
             v[j][2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
           }
-        }
-        if constexpr (COLQ) {
-          const float f = __ldg(rf2 + r);
-          uint32_t b[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) b[e] = rne_bits_prod(__fmul_rn(v[j][e], f), cf[j][e]);
-          *reinterpret_cast<uint2*>(q2 + r * ldq + col) =
-              make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
         }
         if (col_scale) {
 #pragma unroll
@@ -356,74 +331,6 @@ __global__ void __launch_bounds__(256) hadamard_kernel(const InT* x, int64_t ldx
   }
 }
 
-// ---------------------------------------------------------------------------
-// Column statistics for the weight-gradient quantization.  Block = 8 warps
-// over one 256-column chunk and a slab of rows; lane owns 8 columns.
-constexpr int kColSlab = 128;
-
-template <typename InT>
-__global__ void __launch_bounds__(256) colstats_kernel(const InT* __restrict__ dy, int64_t M,
-                                                       int N, const float* __restrict__ sx,
-                                                       uint32_t* __restrict__ colmax,
-                                                       double* __restrict__ colsum,
-                                                       int32_t* __restrict__ status) {
-  __shared__ uint32_t s_max[8][256];
-  __shared__ double s_sum[8][256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int col = blockIdx.x * 256 + lane * 8;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kColSlab;
-  const int64_t m1 = m0 + kColSlab < M ? m0 + kColSlab : M;
-  // Each thread sums at most kColSlab/8 = 16 values of a column in float32
-  // (relative error ~1e-6 of the column's sum of magnitudes); the slab
-  // partials are combined in float64.
-  uint32_t mx[8];
-  float smf[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    mx[i] = 0;
-    smf[i] = 0.0f;
-  }
-  if (col < N) {
-#pragma unroll 4
-    for (int64_t m = m0 + warp; m < m1; m += 8) {
-      float d[8];
-      load8(dy + m * N + col, d);
-      const float s = __ldg(sx + m);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        mx[i] = max(mx[i], abs_bits(d[i] * s));
-        smf[i] += d[i];
-      }
-    }
-  }
-  double sm[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) sm[i] = static_cast<double>(smf[i]);
-  // Transposed writes (column-major in the slab) keep the banks apart.
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    s_max[warp][i * 32 + lane] = mx[i];
-    s_sum[warp][i * 32 + lane] = sm[i];
-  }
-  __syncthreads();
-  const int c = threadIdx.x;  // one column per thread: column c is lane c/8, element c%8
-  const int slotc = (c % 8) * 32 + c / 8;
-  if (blockIdx.x * 256 + c < N) {
-    uint32_t a = 0;
-    double t = 0.0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      a = max(a, s_max[w][slotc]);
-      t += s_sum[w][slotc];
-    }
-    // inf/NaN patterns sort above every finite value: report and let them
-    // through (the column's outputs are then unspecified).
-    if (a >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
-    atomicMax(colmax + blockIdx.x * 256 + c, a);
-    atomicAdd(colsum + blockIdx.x * 256 + c, t);
-  }
-}
-
 __global__ void colfinalize_kernel(const uint32_t* __restrict__ colmax,
                                    const double* __restrict__ colsum, int N, float* s2,
                                    float* inv2, float* db) {
@@ -435,29 +342,14 @@ __global__ void colfinalize_kernel(const uint32_t* __restrict__ colmax,
   if (db) db[n] = static_cast<float>(colsum[n]);
 }
 
-// Column quantization: block (x, y) owns the 2048-column segment y (8
-// columns per thread, their 127/amax factors kept in registers) and walks the
-// rows x, x + gridDim.x, ...
-template <typename InT>
-__global__ void __launch_bounds__(256) colquant_kernel(const InT* __restrict__ dy, int64_t M,
-                                                       int N, const float* __restrict__ sx,
-                                                       const float* __restrict__ inv2,
-                                                       int8_t* __restrict__ q) {
-  const int col = blockIdx.y * 2048 + threadIdx.x * 8;
-  if (col >= N) return;
-  float iv[8];
-  load8(inv2 + col, iv);
-#pragma unroll 4
-  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
-    float d[8];
-    load8(dy + m * N + col, d);
-    const float s = __ldg(sx + m);
-    uint32_t b[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], s), iv[i]);
-    *reinterpret_cast<uint2*>(q + m * N + col) =
-        make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
-  }
+// s1[m] = amax/127 and inv1[m] = 127/amax of the row maxima (0 for a zero row).
+__global__ void rowfinalize_kernel(const uint32_t* __restrict__ rowmax, int64_t M, float* s1,
+                                   float* inv1) {
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (m >= M) return;
+  const float amax = __uint_as_float(rowmax[m]);
+  s1[m] = amax == 0.0f ? 0.0f : amax / 127.0f;
+  inv1[m] = amax == 0.0f ? 0.0f : 127.0f / amax;
 }
 
 template <typename OutT>
@@ -504,13 +396,12 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
     int dev = 0;                                                                               \
     cudaGetDevice(&dev);                                                                       \
     if (dev < 64 && !attr_set[dev]) {                                                          \
-      cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW, BT, false>,                         \
+      cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW, BT>,                                \
                            cudaFuncAttributeMaxDynamicSharedMemorySize, 100000);               \
       attr_set[dev] = true;                                                                    \
     }                                                                                          \
-    quant_rows_tma_kernel<InT, CPW, BT, false><<<grid, 256, smem, s>>>(                        \
-        x, rows, c, ldx, cs, B, hc, flags, q, ldq, rs, st, stages, stage_bytes, nullptr,       \
-        nullptr, nullptr);                                                                     \
+    quant_rows_tma_kernel<InT, CPW, BT><<<grid, 256, smem, s>>>(                               \
+        x, rows, c, ldx, cs, B, hc, flags, q, ldq, rs, st, stages, stage_bytes);               \
   } while (0)
 #define QL_QT_B(CPW)                  \
   do {                                \
@@ -549,60 +440,7 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
   return cudaGetLastError();
 }
 
-template <typename InT, int CPW>
-cudaError_t quant_rows_cols_t(const InT* x, int64_t rows, int c, const float* cs, int8_t* q,
-                              float* rs, const float* rf2, const float* cf2, int8_t* q2,
-                              int32_t* st, int grid, int smem, int stages, int stage_bytes,
-                              cudaStream_t s) {
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW, 0, true>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, 100000);
-    attr_set[dev] = true;
-  }
-  quant_rows_tma_kernel<InT, CPW, 0, true><<<grid, 256, smem, s>>>(
-      x, rows, c, c, cs, 0, 1.0f, 0u, q, c, rs, st, stages, stage_bytes, rf2, cf2, q2);
-  return cudaGetLastError();
-}
-
-template <typename InT>
-cudaError_t quant_rows_cols_dispatch(const void* xv, int64_t rows, int64_t cols, const float* cs,
-                                     int8_t* q, float* rs, const float* rf2, const float* cf2,
-                                     int8_t* q2, int32_t* st, cudaStream_t s) {
-  const InT* x = reinterpret_cast<const InT*>(xv);
-  const int nch = static_cast<int>((cols + 255) / 256);
-  const int64_t row_bytes = cols * static_cast<int64_t>(sizeof(InT));
-  const int stage_bytes = static_cast<int>((row_bytes + 127) / 128 * 128);
-  int stages = 98304 / stage_bytes;
-  stages = stages < 2 ? 2 : stages > 4 ? 4 : stages;
-  const int smem = stages * stage_bytes;
-  const int per_sm = 200000 / (smem + 2048) > 4 ? 4 : 200000 / (smem + 2048);
-  const int grid = grid_cap(rows, per_sm < 1 ? 1 : per_sm);
-  const int cpw = (nch + 7) / 8;
-  const int c = static_cast<int>(cols);
-  cudaError_t e;
-  if (cpw <= 1) e = quant_rows_cols_t<InT, 1>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
-  else if (cpw <= 2) e = quant_rows_cols_t<InT, 2>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
-  else if (cpw <= 3) e = quant_rows_cols_t<InT, 3>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
-  else e = quant_rows_cols_t<InT, 4>(x, rows, c, cs, q, rs, rf2, cf2, q2, st, grid, smem, stages, stage_bytes, s);
-  count_launches(1);
-  return e;
-}
-
 }  // namespace
-
-cudaError_t launch_quant_rows_cols(const void* x, int xt, int64_t rows, int64_t cols,
-                                   const float* col_scale, int8_t* q, float* row_scale,
-                                   const float* rf2, const float* cf2, int8_t* q2,
-                                   int32_t* status, cudaStream_t s) {
-  if (xt == QL_BF16)
-    return quant_rows_cols_dispatch<__nv_bfloat16>(x, rows, cols, col_scale, q, row_scale, rf2,
-                                                   cf2, q2, status, s);
-  return quant_rows_cols_dispatch<float>(x, rows, cols, col_scale, q, row_scale, rf2, cf2, q2,
-                                         status, s);
-}
 
 cudaError_t launch_quant_rows(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,
                               const float* col_scale, int B, float hc, unsigned flags,
@@ -632,17 +470,9 @@ cudaError_t launch_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt,
   return cudaGetLastError();
 }
 
-cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
-                            uint32_t* colmax, double* colsum, int32_t* status, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>((N + 255) / 256),
-                  static_cast<unsigned>((M + kColSlab - 1) / kColSlab));
-  if (dyt == QL_BF16)
-    colstats_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        reinterpret_cast<const __nv_bfloat16*>(dy), M, static_cast<int>(N), sx, colmax, colsum,
-        status);
-  else
-    colstats_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(dy), M,
-                                                static_cast<int>(N), sx, colmax, colsum, status);
+cudaError_t launch_rowfinalize(const uint32_t* rowmax, int64_t M, float* s1, float* inv1,
+                               cudaStream_t s) {
+  rowfinalize_kernel<<<static_cast<unsigned>((M + 255) / 256), 256, 0, s>>>(rowmax, M, s1, inv1);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -651,21 +481,6 @@ cudaError_t launch_colfinalize(const uint32_t* colmax, const double* colsum, int
                                float* s2, float* inv2, float* db, cudaStream_t s) {
   colfinalize_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, s>>>(
       colmax, colsum, static_cast<int>(N), s2, inv2, db);
-  count_launches(1);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_colquant(const void* dy, int dyt, int64_t M, int64_t N, const float* sx,
-                            const float* inv2, int8_t* q, cudaStream_t s) {
-  const unsigned segs = static_cast<unsigned>((N + 2047) / 2048);
-  const int64_t want = (static_cast<int64_t>(device_info().sms) * 8 + segs - 1) / segs;
-  const dim3 grid(static_cast<unsigned>(want < M ? want : M), segs);
-  if (dyt == QL_BF16)
-    colquant_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        reinterpret_cast<const __nv_bfloat16*>(dy), M, static_cast<int>(N), sx, inv2, q);
-  else
-    colquant_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(dy), M,
-                                                static_cast<int>(N), sx, inv2, q);
   count_launches(1);
   return cudaGetLastError();
 }

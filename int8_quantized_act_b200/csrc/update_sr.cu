@@ -41,7 +41,7 @@ __device__ __forceinline__ float adamw(const UpdateConsts& c, float w, float g, 
   const float w1 = w * c.a;
   const float mn = c.b1 * m + c.omb1 * g;
   const float vn = c.b2 * v + c.omb2 * (g * g);
-  const float den = sqrtf(vn / c.bc2) + c.eps;
+  const float den = sqrtf(vn) * c.rbc2 + c.eps;
   m = mn;
   v = vn;
   return w1 - c.st * (mn / den);
@@ -97,6 +97,12 @@ __device__ __forceinline__ void store16f(float* p, const float (&v)[16]) {
 __device__ __forceinline__ int code_at(const uint4& q, int i) {
   const uint32_t w = (&q.x)[i >> 2];
   return static_cast<int>(static_cast<int8_t>((w >> (8 * (i & 3))) & 0xFFu));
+}
+
+// The int8 code as a float without the conversion unit: 1.5*2^23 + q is
+// exact in float32 and its bit pattern is that of 1.5*2^23 plus q.
+__device__ __forceinline__ float code_f(const uint4& q, int i) {
+  return __fsub_rn(__int_as_float(0x4B400000 + code_at(q, i)), 12582912.0f);
 }
 
 template <int GPT, bool WN>
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
         float gr[16];
         load16f(grad + row + 16 * j, gr);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) p = p + gr[e] * (static_cast<float>(code_at(qv[i], e)) / nq);
+        for (int e = 0; e < 16; ++e) p = p + gr[e] * (code_f(qv[i], e) / nq);
       }
     }
     for (int off = 128; off >= 1; off >>= 1) {
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
       }
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float qf = static_cast<float>(code_at(qv[i], e));
+        const float qf = code_f(qv[i], e);
         float gg = gr[e];
         if constexpr (WN) gg = coef * (gr[e] - dg * (qf / nq));
         const float wv = s * qf;
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(512) update_sr_rows_kernel(
       }
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float wv = s * static_cast<float>(code_at(qv, e));
+        const float wv = s * code_f(qv, e);
         w[i][e] = adam ? adamw(c, wv, gr[e], m1[e], m2[e]) : wv - c.lr * gr[e];
         mbits = max(mbits, abs_bits(w[i][e]));
       }

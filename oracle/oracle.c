@@ -406,9 +406,9 @@ static float sr_round(float v, uint32_t u24) {
 
 /* Host-side AdamW constants, each computed in float64 and rounded once. */
 typedef struct {
-    float a;    /* 1 - lr*wd            (decoupled weight decay factor) */
-    float st;   /* lr / (1 - b1^t)      (bias-corrected step size)      */
-    float bc2;  /* 1 - b2^t                                             */
+    float a;     /* 1 - lr*wd             (decoupled weight decay factor) */
+    float st;    /* lr / (1 - b1^t)       (bias-corrected step size)      */
+    float rbc2;  /* 1 / sqrt(1 - b2^t)    (second-moment bias correction, on the root) */
     float b1, b2, omb1, omb2, eps, lr;
 } adamw_consts;
 
@@ -418,7 +418,7 @@ static adamw_consts adamw_setup(float lr, float b1, float b2, float eps, float w
     double t = (double)step;
     c.a = (float)(1.0 - (double)lr * (double)wd);
     c.st = (float)((double)lr / (1.0 - pow((double)b1, t)));
-    c.bc2 = (float)(1.0 - pow((double)b2, t));
+    c.rbc2 = (float)(1.0 / sqrt(1.0 - pow((double)b2, t)));
     c.b1 = b1;
     c.b2 = b2;
     c.omb1 = (float)(1.0 - (double)b1);
@@ -430,12 +430,14 @@ static adamw_consts adamw_setup(float lr, float b1, float b2, float eps, float w
 
 /* One AdamW step of one element (decoupled weight decay, Loshchilov & Hutter):
  * w1 = w*a; m' = b1*m + (1-b1)*g; v' = b2*v + (1-b2)*(g*g);
- * w' = w1 - st * (m' / (sqrt(v'/bc2) + eps)). */
+ * w' = w1 - st * (m' / (sqrt(v') * rbc2 + eps)),
+ * i.e. sqrt(v'/(1-b2^t)) taken as sqrt(v') / sqrt(1-b2^t) with the
+ * reciprocal root rounded once on the host. */
 static float adamw_elem(const adamw_consts *c, float w, float g, float *m, float *v) {
     float w1 = w * c->a;
     float mn = c->b1 * (*m) + c->omb1 * g;
     float vn = c->b2 * (*v) + c->omb2 * (g * g);
-    float den = sqrtf(vn / c->bc2) + c->eps;
+    float den = sqrtf(vn) * c->rbc2 + c->eps;
     *m = mn;
     *v = vn;
     return w1 - c->st * (mn / den);

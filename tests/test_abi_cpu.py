@@ -65,7 +65,8 @@ def test_bwd_workspace_formula(L):
     def a(x):
         return (x + 255) // 256 * 256
     for (M, N, K, B) in ((12000, 7168, 5376, 128), (17, 144, 512, 256)):
-        assert ql.qlinear_bwd_workspace_bytes(M, N, K, B) == ql.qlinear_workspace_bytes(M, N, K, B) + a(M * N)
+        assert (ql.qlinear_bwd_workspace_bytes(M, N, K, B)
+                == ql.qlinear_workspace_bytes(M, N, K, B) + a(M * N) + 2 * a(4 * M))
 
 
 def test_host_validation_returns_before_any_launch(L):
