@@ -44,8 +44,8 @@ NOMINAL_INT8_OVER_BF16 = 2.0   # dense int8 4.5 POPS / dense bf16 2.25 PFLOPS
 # DRAM bytes (read + write) per GEMM launch from the ncu capture summarised in
 # profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
-GEMM_TRAFFIC_BYTES = 409.6e6
-GEMM_TRAFFIC_SOURCE_SHA = "d50591545ba02a0c"
+GEMM_TRAFFIC_BYTES = 369.1e6
+GEMM_TRAFFIC_SOURCE_SHA = "76383a85d156eebd"
 
 
 def gemm_source_sha():
