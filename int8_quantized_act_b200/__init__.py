@@ -28,7 +28,7 @@ __all__ = [
     "qlinear_hadamard", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
     "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
     "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES", "qlinear_bwd",
-    "qlinear_bwd_workspace_bytes",
+    "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout",
 ]
 
 QL_OK, QL_ERR_ARG, QL_ERR_SHAPE, QL_ERR_ALIGN = 0, 1, 2, 3
@@ -104,6 +104,8 @@ def lib() -> ctypes.CDLL:
     L.qlinear_bwd_dx.argtypes = [P, I, I64, I64, P, P, I64, I, P, I, P, ctypes.c_size_t, P, P]
     L.qlinear_bwd_dw.restype = I
     L.qlinear_bwd_dw.argtypes = [P, I, I64, I64, P, P, I64, P, P, P, ctypes.c_size_t, P, P]
+    L.ql_test_wait_timeout.restype = I
+    L.ql_test_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
     L.qlinear_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.qlinear_bwd_workspace_bytes.argtypes = [I64, I64, I64, I]
     L.qlinear_bwd.restype = I
@@ -322,3 +324,11 @@ def ql_set_gemm_timing_events(pairs=()):
 def ql_kernel_launches() -> int:
     """CUDA kernels launched by the library in this process so far."""
     return int(lib().ql_kernel_launches())
+
+
+def ql_test_wait_timeout(status, limit_us: int, stream=None):
+    """Failure-detection check (include/qlinear_testing.h): a kernel waits on
+    a barrier that nothing completes; its bounded wait gives up after
+    limit_us and sets the QL_ERR_TIMEOUT bit in `status`."""
+    _check(lib().ql_test_wait_timeout(_dev(status, "status", torch.int32), int(limit_us),
+                                      _stream(stream)), "ql_test_wait_timeout")

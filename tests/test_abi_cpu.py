@@ -13,8 +13,7 @@ import pytest
 import int8_quantized_act_b200 as ql
 from int8_quantized_act_b200 import build as cuda_build
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
-                      "qlinear.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
 
 
 @pytest.fixture(scope="module")
@@ -24,15 +23,20 @@ def L():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    return re.findall(r"QL_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    names = []
+    for h in sorted(os.listdir(INCLUDE)):
+        if h.endswith(".h"):
+            text = open(os.path.join(INCLUDE, h)).read()
+            names += re.findall(r"QL_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
 
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_functions()
     assert set(names) >= {"qlinear_quantize_rows", "qlinear_hadamard", "qlinear_fwd",
                           "qlinear_bwd_dx", "qlinear_bwd_dw", "qweight_update_sr",
-                          "ql_status_string", "qlinear_workspace_bytes"}
+                          "ql_status_string", "qlinear_workspace_bytes", "qlinear_bwd",
+                          "qlinear_bwd_dx_noalloc", "ql_test_wait_timeout"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -121,3 +125,9 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(TypeError):
         ql.qlinear_quantize_rows(x, torch.zeros((4, 32), dtype=torch.int8), torch.zeros(4),
                                  torch.zeros(1, dtype=torch.int32))
+
+
+def test_timeout_hook_validation(L):
+    assert L.ql_test_wait_timeout(None, 1000, None) == ql.QL_ERR_ARG
+    assert L.ql_test_wait_timeout(fake(0x10000), 0, None) == ql.QL_ERR_ARG
+    assert L.ql_test_wait_timeout(fake(0x10000), 10000001, None) == ql.QL_ERR_ARG

@@ -102,34 +102,56 @@ def test_weight_norm_zero_direction_flagged_and_untouched():
     check_equal(gpu, ref[:7], NAMES)
 
 
-@pytest.mark.parametrize("n", [4096, 16384])
-def test_adamw_full_size_sampled_rows(n):
-    """The [n, n] sweep sizes: the whole matrix updates on the GPU; sampled
-    rows are recomputed by the oracle (its random stream keyed by the
-    absolute row)."""
-    w = workloads.normal((n, n), 0.02, 71)
-    g = workloads.normal((n, n), 1e-3, 72)
-    tw = dev(w)
-    tq = torch.empty((n, n), dtype=torch.int8, device="cuda")
-    ts = torch.empty(n, dtype=torch.float32, device="cuda")
+SAMPLED = [
+    # N, K, warm moments, weight norm
+    (1024, 1024, True, False),      # the [1024,1024] .. [16384,16384] sweep
+    (2048, 2048, False, True),
+    (4096, 4096, False, False),
+    (8192, 8192, True, False),
+    (8192, 8192, False, True),
+    (16384, 16384, False, False),
+    (16384, 16384, False, True),
+    (14336, 4096, True, False),     # SwiGLU w1 / w3
+    (28672, 4096, True, False),     # w1 and w3 stacked
+    (4096, 14336, True, False),     # SwiGLU w2
+]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("N,K,warm,wn", SAMPLED)
+def test_adamw_full_size_sampled_rows(N, K, warm, wn):
+    """Full-size AdamW updates (plain and row-wise weight norm): the whole
+    matrix updates on the GPU; sampled rows are recomputed by the oracle,
+    whose random stream is keyed by the absolute row."""
+    d = workloads.update_state(N, K, seed=N + K, warm=warm, weight_norm=wn)
+    q0, s0 = prepared(d)
+    del d["w"]
+    tq, ts, tg = dev(q0), dev(s0), dev(d["grad"])
+    if warm:
+        tm, tv = dev(d["m"]), dev(d["v"])
+    else:
+        tm = torch.zeros((N, K), device="cuda")
+        tv = torch.zeros((N, K), device="cuda")
+    wn_t = [dev(d[k]) for k in ("g", "g_m", "g_v")] if wn else [None] * 3
+    seed = 0xC0FFEE + N
     st = new_status()
-    ql.qlinear_quantize_rows(tw, tq, ts, st, flags=ql.QL_REJECT_ZERO_ROWS)
-    q0, s0 = host(tq), host(ts)
-    del tw
-    tm = torch.zeros((n, n), device="cuda")
-    tv = torch.zeros((n, n), device="cuda")
-    ql.qweight_update_sr(tq, ts, dev(g), ql.Optim(), tm, tv, 7, 1, st)
+    ql.qweight_update_sr(tq, ts, tg, ql.Optim(weight_decay=0.01), tm, tv, seed, d["step"], st,
+                         g=wn_t[0], g_m=wn_t[1], g_v=wn_t[2])
     assert status_word(st) == 0
-    rows = np.array(sorted({0, 1, n // 2, n - 1} | set(
-        np.random.Generator(np.random.PCG64(n)).integers(0, n, 12).tolist())))
-    q1, s1 = host(tq), host(ts)
-    m1, v1 = host(tm[rows]), host(tv[rows])
-    for r in rows:
-        ref = oracle.update_sr(q0[r:r + 1], s0[r:r + 1], g[r:r + 1], oracle.ADAMW, 1e-3, 7, 1,
-                               m=np.zeros((1, n), np.float32), v=np.zeros((1, n), np.float32),
-                               wd=0.01, row0=int(r))
-        i = int(np.searchsorted(rows, r))
-        check_equal([q1[r:r + 1], s1[r:r + 1], m1[i:i + 1], v1[i:i + 1]], ref[:4], NAMES)
+    del tg
+    rows = np.array(sorted({0, 1, N // 2, N - 1} | set(
+        np.random.Generator(np.random.PCG64(N * 3 + K)).integers(0, N, 10).tolist())))
+    ri = torch.from_numpy(rows).cuda()
+    got = [host(tq[ri]), host(ts[ri]), host(tm[ri]), host(tv[ri])]
+    got += [host(t[ri]) for t in wn_t] if wn else [None] * 3
+    for i, r in enumerate(rows):
+        r = int(r)
+        sl = slice(r, r + 1)
+        kw = dict(g=d["g"][sl], g_m=d["g_m"][sl], g_v=d["g_v"][sl]) if wn else {}
+        ref = oracle.update_sr(q0[sl], s0[sl], d["grad"][sl], oracle.ADAMW, 1e-3, seed,
+                               d["step"], m=d["m"][sl], v=d["v"][sl], wd=0.01, row0=r, **kw)
+        assert ref[-1] == 0
+        check_equal([None if a is None else a[i:i + 1] for a in got], ref[:7], NAMES)
 
 
 def test_update_argument_errors():
