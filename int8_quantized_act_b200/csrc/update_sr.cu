@@ -13,6 +13,8 @@
 // Bytes per element: AdamW 22 (1+4+4+4 in, 1+4+4 out), SGD 6.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "launch.h"
 #include "rowops.cuh"
 #include "../../include/qlinear.h"
@@ -262,49 +264,79 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
   }
 }
 
-// The plain (not weight-normalized) update with GPT = 1, 2 or 4 16-element
-// groups per thread and T = ceil(ngroups / GPT) threads rounded up to a warp
-// (<= 512), so threads finish their groups together at the row reduction.
-template <int GPT>
-__global__ void __launch_bounds__(512) update_sr_rows_kernel(
+// Philox round keys k_r = seed + r * (0x9E3779B9, 0xBB67AE85) mod 2^32,
+// computed once on the host so each round xors a kernel-parameter constant.
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+
+__device__ __forceinline__ uint4 philox10_keys(uint4 c, const PhiloxKeys& k) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k.k0[r], static_cast<uint32_t>(p1),
+                   static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k.k1[r], static_cast<uint32_t>(p0));
+  }
+  return c;
+}
+
+__device__ __forceinline__ float code_byte_f(uint32_t q4, int i) {
+  return __fsub_rn(__int_as_float(0x4B400000 + static_cast<int>(static_cast<int8_t>(q4 >> (8 * i)))),
+                   12582912.0f);
+}
+
+// The plain (not weight-normalized) update.  One CTA per weight row; the row
+// is cut into 4-element chunks (one Philox block each) dealt round-robin to
+// the threads, so every global access of a warp is one contiguous run.
+// Phase 1 streams codes, gradient and moments in, writes the new moments and
+// parks the updated float row in shared memory (4 K bytes) while keeping the
+// running max of |w'|; phase 2, after the CTA max reduction, draws the Philox
+// words and writes the stochastically rounded codes.  Parking the row in
+// shared memory instead of registers keeps the register count low, so
+// several rows are in flight per SM and their loads overlap the arithmetic.
+__global__ void __launch_bounds__(512, 2) update_sr_rows_kernel(
     int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
-    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, uint32_t seed_lo,
-    uint32_t seed_hi, uint32_t step_lo, uint32_t step_hi, int32_t* __restrict__ status) {
-  __shared__ uint32_t s_max[32];
+    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
+    uint32_t step_lo, uint32_t step_hi, int32_t* __restrict__ status) {
+  extern __shared__ float4 s_row[];
+  __shared__ uint32_t s_max[16];
   const int n = blockIdx.x;
   const int t = threadIdx.x;
   const int T = blockDim.x;
   const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
-  const int ngroups = K >> 4;
+  const int nch = K >> 2;
   const int64_t row = static_cast<int64_t>(n) * K;
   const bool adam = c.kind == QL_ADAMW;
   const float s = sw[n];
+  const uint32_t* q_in = reinterpret_cast<const uint32_t*>(wq + row);
+  const float4* g_in = reinterpret_cast<const float4*>(grad + row);
+  float4* m_io = reinterpret_cast<float4*>(mom1 + row);
+  float4* v_io = reinterpret_cast<float4*>(mom2 + row);
 
-  float w[GPT][16];
   uint32_t mbits = 0;
+#pragma unroll 2
+  for (int ch = t; ch < nch; ch += T) {
+    const uint32_t q4 = __ldcs(q_in + ch);
+    const float4 g4 = __ldcs(g_in + ch);
+    float gr[4] = {g4.x, g4.y, g4.z, g4.w};
+    float w[4];
+    if (adam) {
+      const float4 m4 = __ldcs(m_io + ch);
+      const float4 v4 = __ldcs(v_io + ch);
+      float m1[4] = {m4.x, m4.y, m4.z, m4.w};
+      float m2[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-  for (int i = 0; i < GPT; ++i) {
-    const int j = t + T * i;
-    if (j < ngroups) {
-      const int64_t off = row + 16 * j;
-      const uint4 qv = *reinterpret_cast<const uint4*>(wq + off);
-      float gr[16], m1[16], m2[16];
-      load16f(grad + off, gr);
-      if (adam) {
-        load16f(mom1 + off, m1);
-        load16f(mom2 + off, m2);
-      }
+      for (int e = 0; e < 4; ++e) w[e] = adamw(c, s * code_byte_f(q4, e), gr[e], m1[e], m2[e]);
+      __stcs(m_io + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
+      __stcs(v_io + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
+    } else {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float wv = s * code_f(qv, e);
-        w[i][e] = adam ? adamw(c, wv, gr[e], m1[e], m2[e]) : wv - c.lr * gr[e];
-        mbits = max(mbits, abs_bits(w[i][e]));
-      }
-      if (adam) {
-        store16f(mom1 + off, m1);
-        store16f(mom2 + off, m2);
-      }
+      for (int e = 0; e < 4; ++e) w[e] = s * code_byte_f(q4, e) - c.lr * gr[e];
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) mbits = max(mbits, abs_bits(w[e]));
+    s_row[ch] = make_float4(w[0], w[1], w[2], w[3]);
   }
   mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
   if (lane == 0) s_max[warp] = mbits;
@@ -317,15 +349,29 @@ __global__ void __launch_bounds__(512) update_sr_rows_kernel(
     sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
     if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
   }
-#pragma unroll
-  for (int i = 0; i < GPT; ++i) {
-    const int j = t + T * i;
-    if (j < ngroups)
-      *reinterpret_cast<uint4*>(wq + row + 16 * j) =
-          sr_group(w[i], inv, mbits == 0, static_cast<uint64_t>(row + 16 * j), seed_lo, seed_hi,
-                   step_lo, step_hi);
+
+  // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
+  // step lo, step hi), key = seed); chunk ch of this row is block row/4 + ch.
+  uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
+  const uint64_t blk0 = static_cast<uint64_t>(row) >> 2;
+#pragma unroll 2
+  for (int ch = t; ch < nch; ch += T) {
+    const uint64_t blk = blk0 + static_cast<uint64_t>(ch);
+    const uint4 r = philox10_keys(
+        make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32), step_lo, step_hi),
+        keys);
+    const float4 w = s_row[ch];
+    uint32_t out = 0;
+    if (mbits != 0)
+      out = pack_codes(sr_code_bits(w.x * inv, r.x >> 8), sr_code_bits(w.y * inv, r.y >> 8),
+                       sr_code_bits(w.z * inv, r.z >> 8), sr_code_bits(w.w * inv, r.w >> 8));
+    __stcs(q_out + ch, out);
   }
 }
+
+#ifndef QL_UPDATE_CHUNKS_PER_THREAD
+#define QL_UPDATE_CHUNKS_PER_THREAD 4
+#endif
 
 }  // namespace
 
@@ -350,14 +396,25 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     else if (gpt <= 4) QL_UPD(4, true);
     else QL_UPD(8, true);
   } else {
-    const int g1 = ngroups <= 512 ? 1 : ngroups <= 1024 ? 2 : 4;
-    const int tr = ((ngroups + g1 - 1) / g1 + 31) / 32 * 32;
-    if (g1 == 1)
-      update_sr_rows_kernel<1><<<grid, tr, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, status);
-    else if (g1 == 2)
-      update_sr_rows_kernel<2><<<grid, tr, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, status);
-    else
-      update_sr_rows_kernel<4><<<grid, tr, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, status);
+    // ~4 chunks per thread, a whole number of warps, at most 512 threads.
+    const int nch = static_cast<int>(K / 4);
+    int tr = (nch + QL_UPDATE_CHUNKS_PER_THREAD - 1) / QL_UPDATE_CHUNKS_PER_THREAD;
+    tr = std::min(512, std::max(32, (tr + 31) / 32 * 32));
+    static bool smem_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !smem_set[dev]) {
+      cudaFuncSetAttribute(update_sr_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           4 * 32768);
+      smem_set[dev] = true;
+    }
+    PhiloxKeys keys;
+    for (int r = 0; r < 10; ++r) {
+      keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
+      keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
+    }
+    update_sr_rows_kernel<<<grid, tr, static_cast<size_t>(4) * K, s>>>(
+        wq, sw, grad, k, c, m, v, keys, tl, th, status);
   }
 #undef QL_UPD
   count_launches(1);
