@@ -11,6 +11,7 @@ namespace ql {
 
 struct DeviceInfo {
   int sms = 0;
+  int smem_optin = 0;  // max dynamic shared memory per block (opt-in), bytes
 };
 const DeviceInfo& device_info();  // current device, cached
 

@@ -22,6 +22,9 @@ const DeviceInfo& device_info() {
     int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     infos[dev].sms = sms > 0 ? sms : 1;
+    int optin = 0;
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    infos[dev].smem_optin = optin > 0 ? optin : 48 * 1024;
   });
   return infos[dev];
 }

@@ -4,19 +4,23 @@
 // stochastically in CUDA row kernels, with no floating master weight; feature
 // table rows "Optimizers" and "Row-wise weight normalization").
 //
-// One CTA owns one weight row.  Thread t holds the 16-element groups
-// t, t+T, t+2T, ... (T = threads, a power of two <= 256) in registers, so the
-// row is read from HBM once: codes, gradient and moments in, new moments out
-// while the updated float row stays in registers; a CTA max-reduction gives
-// the new scale; then each group draws 16 24-bit uniforms from 4 Philox4x32-10
-// blocks and writes 16 stochastically rounded codes with one 128-bit store.
-// Bytes per element: AdamW 22 (1+4+4+4 in, 1+4+4 out), SGD 6.
+// One CTA owns one weight row and reads it from HBM once: codes, gradient
+// and moments in, new moments out, while the updated float row waits in
+// shared memory for the row max; the new scale follows from a CTA max
+// reduction; then every 4-element chunk draws one Philox4x32-10 block and
+// writes 4 stochastically rounded codes.  Rows up to ~8K elements are staged
+// whole by the bulk-copy engine (update_sr_staged_kernel); longer rows are
+// loaded through registers (update_sr_rows_kernel); the row-wise weight-norm
+// variant (update_sr_kernel) keeps 16-element groups for its pinned
+// reduction order.  Bytes per element: AdamW 22 (1+4+4+4 in, 1+4+4 out),
+// SGD 6.
 #include <cuda_runtime.h>
 
 #include <algorithm>
 
 #include "launch.h"
 #include "rowops.cuh"
+#include "sm100.cuh"
 #include "../../include/qlinear.h"
 
 namespace ql {
@@ -369,6 +373,118 @@ __global__ void __launch_bounds__(512, 2) update_sr_rows_kernel(
   }
 }
 
+// The same update with the row staged by the bulk-copy engine: one CTA per
+// row copies the row's codes, gradient and both moments into shared memory
+// with four bulk copies on one mbarrier (13 K bytes for AdamW), so every load
+// of the row is in flight at once without holding a register, and three such
+// CTAs share an SM; the updated float row is parked over the gradient.  Used
+// while a row fits twice in the shared memory of one CTA.
+__global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
+    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
+    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
+    uint32_t step_lo, uint32_t step_hi, int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint32_t s_max[16];
+  __shared__ __align__(8) uint64_t s_full;
+  __shared__ volatile int s_abort;
+  const int n = blockIdx.x;
+  const int t = threadIdx.x;
+  const int T = blockDim.x;
+  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
+  const int nch = K >> 2;
+  const bool adam = c.kind == QL_ADAMW;
+  const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
+  const int64_t row = static_cast<int64_t>(n) * K;
+  const uint32_t bar = smem_u32(&s_full);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    s_abort = 0;
+    fence_mbar_init();
+    const uint32_t dst = smem_u32(smem);
+    mbar_arrive_expect_tx(bar, qbytes + fbytes * (adam ? 3u : 1u));
+    bulk_load(dst, wq + row, qbytes, bar);
+    bulk_load(dst + qbytes, grad + row, fbytes, bar);
+    if (adam) {
+      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar);
+      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar);
+    }
+  }
+  const float s = sw[n];
+  __syncthreads();  // barrier initialised before anyone waits on it
+  const bool ok = mbar_wait(bar, 0, &s_abort);
+  const uint32_t* q_s = reinterpret_cast<const uint32_t*>(smem);
+  float4* g_s = reinterpret_cast<float4*>(smem + qbytes);  // then the updated row
+  const float4* m_s = reinterpret_cast<const float4*>(smem + qbytes + fbytes);
+  const float4* v_s = reinterpret_cast<const float4*>(smem + qbytes + 2 * fbytes);
+  float4* m_out = reinterpret_cast<float4*>(mom1 + row);
+  float4* v_out = reinterpret_cast<float4*>(mom2 + row);
+  uint32_t mbits = 0;
+  if (ok) {
+    for (int ch = t; ch < nch; ch += T) {
+      const uint32_t q4 = q_s[ch];
+      const float4 g4 = g_s[ch];
+      const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
+      float w[4];
+      if (adam) {
+        const float4 m4 = m_s[ch];
+        const float4 v4 = v_s[ch];
+        float m1[4] = {m4.x, m4.y, m4.z, m4.w};
+        float m2[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = adamw(c, s * code_byte_f(q4, e), gr[e], m1[e], m2[e]);
+        __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
+        __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = s * code_byte_f(q4, e) - c.lr * gr[e];
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mbits = max(mbits, abs_bits(w[e]));
+      g_s[ch] = make_float4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+  if (lane == 0) s_max[warp] = mbits;
+  __syncthreads();
+  if (s_abort) {
+    // Timed out: the copies may still be landing; wait for them (bounded)
+    // before the CTA's shared memory is released.
+    if (t == 0) {
+      atomicOr(status, 1 << QL_ERR_TIMEOUT);
+      mbar_wait_drain(bar, 0);
+    }
+    return;
+  }
+  mbits = 0;
+  for (int k = 0; k < nwarps; ++k) mbits = max(mbits, s_max[k]);
+  const float amax = __uint_as_float(mbits);
+  const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
+  if (t == 0) {
+    sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
+    if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  }
+  // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
+  // step lo, step hi), key = seed); chunk ch of this row is block row/4 + ch.
+  uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
+  const uint64_t blk0 = static_cast<uint64_t>(row) >> 2;
+  for (int ch = t; ch < nch; ch += T) {
+    const uint64_t blk = blk0 + static_cast<uint64_t>(ch);
+    const uint4 rn = philox10_keys(
+        make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32), step_lo, step_hi),
+        keys);
+    const float4 w = g_s[ch];
+    uint32_t out = 0;
+    if (mbits != 0)
+      out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
+                       sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+    __stcs(q_out + ch, out);
+  }
+}
+
+// Chunks of 4 elements per thread (sets the thread count of both kernels).
+#ifndef QL_UPDATE_STAGED_CHUNKS
+#define QL_UPDATE_STAGED_CHUNKS 6
+#endif
 #ifndef QL_UPDATE_CHUNKS_PER_THREAD
 #define QL_UPDATE_CHUNKS_PER_THREAD 4
 #endif
@@ -396,8 +512,30 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     else if (gpt <= 4) QL_UPD(4, true);
     else QL_UPD(8, true);
   } else {
-    // ~4 chunks per thread, a whole number of warps, at most 512 threads.
     const int nch = static_cast<int>(K / 4);
+    PhiloxKeys keys;
+    for (int r = 0; r < 10; ++r) {
+      keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
+      keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
+    }
+    const int64_t row_bytes = K * (c.kind == QL_ADAMW ? 13 : 5);
+    const int64_t budget = device_info().smem_optin - 1024;
+    if (2 * (row_bytes + 1024) <= budget) {
+      const int tr = std::min(512, std::max(32, (nch / QL_UPDATE_STAGED_CHUNKS + 31) / 32 * 32));
+      static bool staged_set[64] = {false};
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (dev < 64 && !staged_set[dev]) {
+        cudaFuncSetAttribute(update_sr_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(budget));
+        staged_set[dev] = true;
+      }
+      update_sr_staged_kernel<<<grid, tr, static_cast<size_t>(row_bytes), s>>>(
+          wq, sw, grad, k, c, m, v, keys, tl, th, status);
+      count_launches(1);
+      return cudaGetLastError();
+    }
+    // Longer rows: registers and a parked row of 4 K bytes.
     int tr = (nch + QL_UPDATE_CHUNKS_PER_THREAD - 1) / QL_UPDATE_CHUNKS_PER_THREAD;
     tr = std::min(512, std::max(32, (tr + 31) / 32 * 32));
     static bool smem_set[64] = {false};
@@ -407,11 +545,6 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
       cudaFuncSetAttribute(update_sr_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            4 * 32768);
       smem_set[dev] = true;
-    }
-    PhiloxKeys keys;
-    for (int r = 0; r < 10; ++r) {
-      keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
-      keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
     }
     update_sr_rows_kernel<<<grid, tr, static_cast<size_t>(4) * K, s>>>(
         wq, sw, grad, k, c, m, v, keys, tl, th, status);
