@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
 
 // Chunks of 4 elements per thread (sets the thread count of both kernels).
 #ifndef QL_UPDATE_STAGED_CHUNKS
-#define QL_UPDATE_STAGED_CHUNKS 6
+#define QL_UPDATE_STAGED_CHUNKS 4
 #endif
 #ifndef QL_UPDATE_CHUNKS_PER_THREAD
 #define QL_UPDATE_CHUNKS_PER_THREAD 4
