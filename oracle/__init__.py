@@ -52,6 +52,7 @@ def _declare(L):
         "ref_hadamard_rows": (_U32, [_P, _I64, _P, _I64, _I64, _I64, ctypes.c_int]),
         "ref_hadamard_matrix_f64": (None, [ctypes.c_int, _P]),
         "ref_quantize_rows": (_U32, [_P, _I64, _I64, _I64, _P, ctypes.c_int, _U32, _P, _I64, _P]),
+        "ref_dequantize": (_U32, [_P, _I64, _P, _I64, _I64, ctypes.c_int, _P, _I64]),
         "ref_gemm_nt": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
         "ref_gemm_nn": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
         "ref_gemm_tn": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
@@ -97,6 +98,16 @@ def hadamard_rows(x: np.ndarray, B: int):
     y = np.empty_like(x)
     st = lib().ref_hadamard_rows(_p(x), cols, _p(y), cols, rows, cols, B)
     return y, st
+
+
+def dequantize(q: np.ndarray, s: np.ndarray, B: int = 0):
+    """(s * q) R row by row: the weight back in floating point and in the
+    original basis.  Returns (w float32 [N,K], status)."""
+    q, s = _i8(q), _f32(s)
+    N, K = q.shape
+    w = np.empty((N, K), np.float32)
+    st = lib().ref_dequantize(_p(q), K, _p(s), N, K, B, _p(w), K)
+    return w, st
 
 
 def hadamard_matrix(B: int) -> np.ndarray:

@@ -173,6 +173,24 @@ uint32_t ref_quantize_rows(const float *x, int64_t rows, int64_t cols, int64_t l
 }
 
 /* ------------------------------------------------------------------ */
+/* Dequantization back to the original basis ([CR] third commit note,  */
+/* item 2: unquantized_weight un-rotates for LoRA and offload callers)  */
+/* ------------------------------------------------------------------ */
+
+/* w[n,k] = s[n] * (float)q[n,k] (one float32 product), then for B > 0 each
+ * row times R, which is its own inverse (H_B H_B = B I), so a weight that
+ * was rotated before quantization comes back in its original basis. */
+uint32_t ref_dequantize(const int8_t *q, int64_t ldq, const float *s, int64_t N, int64_t K,
+                        int B, float *w, int64_t ldw) {
+    if (!valid_block(B)) return ORC_BIT_ARG;
+    if (B > 0 && K % B != 0) return ORC_BIT_SHAPE;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) w[n * ldw + k] = (float)q[n * ldq + k] * s[n];
+    if (B > 0) return ref_hadamard_rows(w, ldw, w, ldw, N, K, B);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* Integer GEMMs ([CR] summary: int8 x int8 -> int32 as torch._int_mm; */
 /* [QT] intro: integer forward and backward matrix products)           */
 /* ------------------------------------------------------------------ */

@@ -173,6 +173,63 @@ def test_quant_composes_with_col_scale_and_rotation():
 
 
 # --------------------------------------------------------------------------
+# Dequantization back to the original basis
+# --------------------------------------------------------------------------
+
+def test_dequantize_exact_multiples_round_trip():
+    """Rows s0*q (s0 a power of two, max |q| = 127) quantize to (q, s0) and
+    dequantize back to exactly the same rows."""
+    rng = np.random.Generator(np.random.PCG64(21))
+    q = rng.integers(-127, 128, size=(7, 96)).astype(np.int8)
+    q[:, 3] = 127
+    s0 = (2.0 ** -rng.integers(0, 10, size=7)).astype(np.float32)
+    x = q.astype(np.float32) * s0[:, None]
+    qq, s, _ = oracle.quantize_rows(x)
+    w, st = oracle.dequantize(qq, s)
+    assert st == 0 and np.array_equal(w, x)
+
+
+@pytest.mark.parametrize("B", [2, 16, 128, 256])
+def test_dequantize_unrotates_against_scipy_hadamard(B):
+    """(s q) R against float64 (s q) @ blockdiag(scipy H_B)/sqrt(B): within a
+    few float32 ulps of the row's magnitude (log2 B butterfly roundings)."""
+    K = 2 * max(B, 64)
+    rng = np.random.Generator(np.random.PCG64(B))
+    q = rng.integers(-127, 128, size=(5, K)).astype(np.int8)
+    s = rng.uniform(1e-4, 1e-2, size=5).astype(np.float32)
+    w, st = oracle.dequantize(q, s, B)
+    assert st == 0
+    H = scipy.linalg.hadamard(B).astype(np.float64) / math.sqrt(B)
+    deq = q.astype(np.float64) * s.astype(np.float64)[:, None]
+    ref = (deq.reshape(5, K // B, B) @ H).reshape(5, K)
+    scale = np.abs(deq).reshape(5, K // B, B).sum(-1, keepdims=True) / math.sqrt(B)
+    bound = np.broadcast_to(scale, (5, K // B, B)).reshape(5, K) * (math.log2(B) + 2) * 2.0 ** -23
+    assert np.all(np.abs(w - ref) <= bound)
+
+
+def test_dequantize_inverts_rotated_quantization_within_error_bound():
+    """W -> rotate + quantize -> dequantize + un-rotate: per row the L2 error
+    is at most that of the rotated-basis codes, sqrt(K) * s / 2, because R is
+    orthogonal; without the un-rotation it would be of the order of |W|."""
+    d = workloads.rotated_layer(M=1, seed=2)
+    W = d["w"][:64]
+    q, s, _ = oracle.quantize_rows(W, B=128, flags=oracle.REJECT_ZERO_ROWS)
+    w, st = oracle.dequantize(q, s, 128)
+    assert st == 0
+    err = np.linalg.norm(W.astype(np.float64) - w, axis=1)
+    assert np.all(err <= math.sqrt(W.shape[1]) * s.astype(np.float64) / 2 * (1 + 1e-3))
+    w_plain, _ = oracle.dequantize(q, s, 0)
+    assert np.all(np.linalg.norm(W.astype(np.float64) - w_plain, axis=1) > 10 * err)
+
+
+def test_dequantize_argument_checks():
+    q = np.zeros((2, 48), np.int8)
+    s = np.ones(2, np.float32)
+    assert oracle.dequantize(q, s, 3)[1] == oracle.BIT_ARG
+    assert oracle.dequantize(q, s, 32)[1] == oracle.BIT_SHAPE
+
+
+# --------------------------------------------------------------------------
 # Integer GEMMs
 # --------------------------------------------------------------------------
 
