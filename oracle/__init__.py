@@ -57,6 +57,8 @@ def _declare(L):
         "ref_gemm_nn": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
         "ref_gemm_tn": (_U32, [_P, _I64, _P, _I64, _I64, _I64, _I64, _P, _I64]),
         "ref_fwd": (_U32, [_P, _I64, _I64, _P, _P, _I64, _P, ctypes.c_int, _P, _P, _P]),
+        "ref_round_bf16": (_F, [_F]),
+        "ref_fwd_bf16": (_U32, [_P, _I64, _I64, _P, _P, _I64, _P, ctypes.c_int, _P, _P]),
         "ref_bwd_prep_rows": (_U32, [_P, _I64, _I64, _P, _P, _P]),
         "ref_bwd_prep_cols": (_U32, [_P, _I64, _I64, _P, _P, _P, _P]),
         "ref_bwd_dx": (_U32, [_P, _I64, _I64, _P, _P, _I64, ctypes.c_int, _P, _P, _P]),
@@ -170,6 +172,22 @@ def fwd(x, wq, sw, bias=None, B: int = 0):
     sx = np.empty((M,), np.float32)
     st = lib().ref_fwd(_p(x), M, K, _p(wq), _p(sw), N, _p(b), B, _p(y), _p(xq), _p(sx))
     return y, xq, sx, st
+
+
+def round_bf16(v: float) -> float:
+    return float(lib().ref_round_bf16(float(v)))
+
+
+def fwd_bf16(x, wq, sw, bias=None, B: int = 0):
+    """The bf16 route: returns y (fp32 [M,N]), xr = bf16(x R) as fp32, status."""
+    x, wq, sw = _f32(x), _i8(wq), _f32(sw)
+    M, K = x.shape
+    N = wq.shape[0]
+    b = None if bias is None else _f32(bias)
+    y = np.empty((M, N), np.float32)
+    xr = np.empty((M, K), np.float32)
+    st = lib().ref_fwd_bf16(_p(x), M, K, _p(wq), _p(sw), N, _p(b), B, _p(y), _p(xr))
+    return y, xr, st
 
 
 def bwd_prep_rows(dy, sw):

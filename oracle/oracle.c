@@ -281,6 +281,55 @@ uint32_t ref_fwd(const float *x, int64_t M, int64_t K, const int8_t *wq, const f
 }
 
 /* ------------------------------------------------------------------ */
+/* The forward's bf16 route ([CR] third commit note, items 1 and 2: the  */
+/* activations are rotated instead of the weight being un-rotated, and   */
+/* they are not quantized)                                              */
+/* ------------------------------------------------------------------ */
+
+/* float32 -> bf16 (the upper 16 bits of a float32), rounding to nearest with
+ * ties to even; a NaN stays a (quiet) NaN.  Returned as the float32 it
+ * represents. */
+float ref_round_bf16(float v) {
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) {
+        u = (u | 0x00400000u) & 0xFFFF0000u;
+    } else {
+        uint32_t lsb = (u >> 16) & 1u;
+        u = (u + 0x7FFFu + lsb) & 0xFFFF0000u;
+    }
+    float r;
+    memcpy(&r, &u, 4);
+    return r;
+}
+
+/* xr = bf16(x R) (x itself, rounded, when B = 0); the weight enters as its
+ * codes q, exact in bf16; y[m,n] = ((float)(sum_k xr[m,k] q[n,k])) * s_w[n]
+ * + bias[n], with every product exact and the sum taken in float64.  The
+ * tensor cores accumulate in float32 in an order of their own, so a kernel
+ * matches this within a rounding bound, not bit for bit.  xr [M,K] is
+ * returned for the checks. */
+uint32_t ref_fwd_bf16(const float *x, int64_t M, int64_t K, const int8_t *wq, const float *sw,
+                      int64_t N, const float *bias, int B, float *y, float *xr) {
+    if (!valid_block(B)) return ORC_BIT_ARG;
+    if (B > 0 && K % B != 0) return ORC_BIT_SHAPE;
+    uint32_t st = 0;
+    if (B > 0) st = ref_hadamard_rows(x, K, xr, K, M, K, B);
+    else memcpy(xr, x, (size_t)(M * K) * sizeof(float));
+    for (int64_t i = 0; i < M * K; ++i) xr[i] = ref_round_bf16(xr[i]);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            const float *a = xr + m * K;
+            const int8_t *b = wq + n * K;
+            for (int64_t k = 0; k < K; ++k) acc += (double)a[k] * (double)b[k];
+            float v = (float)acc * sw[n];
+            y[m * N + n] = bias ? v + bias[n] : v;
+        }
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
 /* Backward preparation (the spec formulas for dX and dW)         */
 /* ------------------------------------------------------------------ */
 

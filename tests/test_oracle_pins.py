@@ -230,6 +230,57 @@ def test_dequantize_argument_checks():
 
 
 # --------------------------------------------------------------------------
+# The forward's bf16 route
+# --------------------------------------------------------------------------
+
+def test_round_bf16_matches_torch():
+    rng = np.random.Generator(np.random.PCG64(31))
+    vals = np.concatenate([
+        rng.standard_normal(2000).astype(np.float32) * np.float32(1e3),
+        (rng.standard_normal(200) * 1e-39).astype(np.float32),           # subnormals
+        np.array([0.0, -0.0, np.inf, -np.inf, 3.4e38, -3.4e38, 1.00390625, 1.01171875,
+                  1.0 + 2.0 ** -8 + 2.0 ** -20], np.float32),             # ties and near-ties
+    ])
+    ref = torch.from_numpy(vals).to(torch.bfloat16).float().numpy()
+    got = np.array([oracle.round_bf16(v) for v in vals], np.float32)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    assert math.isnan(oracle.round_bf16(float("nan")))
+
+
+def test_fwd_bf16_exact_when_inputs_are_representable():
+    """Small-integer x (exact in bf16), integer codes, power-of-two scales:
+    every step is exact, so y is the integer product times s_w plus bias."""
+    rng = np.random.Generator(np.random.PCG64(32))
+    x = rng.integers(-8, 9, size=(5, 96)).astype(np.float32)
+    q = rng.integers(-127, 128, size=(7, 96)).astype(np.int8)
+    sw = (2.0 ** -rng.integers(0, 8, size=7)).astype(np.float32)
+    b = rng.integers(-4, 5, size=7).astype(np.float32)
+    y, xr, st = oracle.fwd_bf16(x, q, sw, b, 0)
+    assert st == 0 and np.array_equal(xr, x)
+    ref = (x.astype(np.int64) @ q.astype(np.int64).T).astype(np.float64) * sw + b
+    assert np.array_equal(y, ref.astype(np.float32))
+
+
+def test_fwd_bf16_equals_x_times_dequantized_weight():
+    """(bf16(x R)) (s q)^T = x ((s q) R)^T = x W_hat^T up to the bf16 rounding
+    of x R (2^-9 relative per element): rotating the activations stands in
+    for un-rotating the weight ([CR] third commit note, item 2)."""
+    d = workloads.rotated_layer(M=1, seed=3)
+    x = workloads.normal((6, 5376), 1.0, 33)
+    W = d["w"][:40]
+    q, s, _ = oracle.quantize_rows(W, B=128, flags=oracle.REJECT_ZERO_ROWS)
+    y, xr, st = oracle.fwd_bf16(x, q, s, None, 128)
+    assert st == 0
+    w_hat, _ = oracle.dequantize(q, s, 128)
+    ref = x.astype(np.float64) @ w_hat.astype(np.float64).T
+    xR, _ = oracle.hadamard_rows(x, 128)
+    D = np.abs(xR.astype(np.float64)) @ np.abs(q.astype(np.float64) * s[:, None]).T
+    assert np.all(np.abs(y - ref) <= D * (2.0 ** -9 + 1e-5))
+    y0, _, _ = oracle.fwd_bf16(x, q, s, None, 0)     # the stored basis without rotating x
+    assert np.abs(y0 - ref).max() > 100 * np.abs(y - ref).max()
+
+
+# --------------------------------------------------------------------------
 # Integer GEMMs
 # --------------------------------------------------------------------------
 
