@@ -145,6 +145,52 @@ QL_API int qlinear_quantize_rows(const void *x, int xt, int64_t rows, int64_t co
 QL_API int qlinear_hadamard(const void *x, int xt, int64_t ldx, void *y, int yt, int64_t ldy,
                      int64_t rows, int64_t cols, int hadamard_block, void *stream);
 
+/* The weight back in floating point and in the original basis: the
+ * "unquantized weight" that LoRA decomposition and offload sizing read
+ * ([CR] third commit note, item 2: it un-rotates, only the forward uses the
+ * stored rotated basis).  For each row n of the codes wq [N, K] (pitch ldq):
+ *   w[n,:] = s_w[n] * wq[n,:]   (one float32 multiply per element)
+ *   w[n,:] = w[n,:] R           (if hadamard_block = B > 0; R as above, its
+ *                                own inverse, so this undoes the rotation
+ *                                the weight preparation applied)
+ * w [N, K] of dtype wt with pitch ldw (elements).  Requirements: K % 16 == 0,
+ * B in {0, 2, ..., 256} with K % B == 0, ldq >= K and ldq % 16 == 0, ldw >= K,
+ * wq and w 16-byte aligned, ldw * sizeof(wt) % 16 == 0.  Asynchronous on
+ * `stream`; argument errors are returned before any launch. */
+QL_API int qlinear_dequantize(const int8_t *wq, int64_t ldq, const float *sw, int64_t N,
+                              int64_t K, int hadamard_block, void *w, int wt, int64_t ldw,
+                              void *stream);
+
+/* The codes of an int8 weight as bf16, exactly (|q| <= 127 needs 7
+ * significant bits): the weight operand of qlinear_fwd_bf16, refreshed by
+ * the caller after each update.  out [N, K] bf16 with pitch ldo elements;
+ * same requirements as qlinear_dequantize. */
+QL_API int qlinear_codes_bf16(const int8_t *wq, int64_t ldq, int64_t N, int64_t K, void *out,
+                              int64_t ldo, void *stream);
+
+/* The forward's bf16 route ([CR] third commit note, items 1 and 2): the
+ * activations are rotated instead of the weight being un-rotated, and they
+ * are not quantized.
+ *   xr = bf16(x R)       (float32 butterflies as in qlinear_hadamard, one
+ *                         rounding to bf16; with B = 0 just bf16(x), and x
+ *                         itself when it is already bf16)
+ *   y[m,n] = (sum_k xr[m,k] * q[n,k]) * s_w[n] + bias[n]
+ * with the sum on the tensor cores (tcgen05 kind::f16, bf16 x bf16, float32
+ * accumulator): x times the dequantized weight, transposed, up to rounding.
+ * wq_bf16 [N, K]: the weight codes as bf16 (qlinear_codes_bf16), in the
+ * weight's stored (rotated) basis; sw, bias as in qlinear_fwd.  y [M, N] of
+ * dtype yt.  ws: qlinear_fwd_bf16_workspace_bytes(M, K, xt, B) bytes,
+ * 256-byte aligned (holds xr; 0 bytes and NULL allowed when x is bf16 and
+ * B = 0).  Requirements: K % 16 == 0, N % 16 == 0, B in {0, 2, ..., 256} with
+ * K % B == 0; x, wq_bf16, y 16-byte aligned; contiguous rows.  No
+ * contraction limit (float32 accumulation).  Device conditions (a bounded
+ * wait that timed out) are OR-ed into *d_status. */
+QL_API size_t qlinear_fwd_bf16_workspace_bytes(int64_t M, int64_t K, int xt, int hadamard_block);
+QL_API int qlinear_fwd_bf16(const void *x, int xt, int64_t M, int64_t K, const void *wq_bf16,
+                            const float *sw, int64_t N, const float *bias, int hadamard_block,
+                            void *y, int yt, void *ws, size_t ws_bytes, int32_t *d_status,
+                            void *stream);
+
 /* Forward ([CR] item 1 and summary; [QT] intro):
  *   X_q, s_x = quantize_rows(x, B)                     (saved for backward)
  *   y[m,n] = ((float)(sum_k X_q[m,k] W_q[n,k]) * s_x[m]) * s_w[n] + bias[n]

@@ -25,7 +25,8 @@ __all__ = [
     "QL_F32", "QL_BF16", "QL_SGD", "QL_ADAMW", "QL_REJECT_ZERO_ROWS",
     "QL_MAX_CONTRACTION", "QLError", "Optim", "lib", "library_path",
     "ql_status_string", "qlinear_workspace_bytes", "qlinear_quantize_rows",
-    "qlinear_hadamard", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
+    "qlinear_hadamard", "qlinear_dequantize", "qlinear_codes_bf16", "qlinear_fwd_bf16",
+    "qlinear_fwd_bf16_workspace_bytes", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
     "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
     "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES", "qlinear_bwd",
     "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout",
@@ -98,6 +99,14 @@ def lib() -> ctypes.CDLL:
     L.qlinear_quantize_rows.argtypes = [P, I, I64, I64, I64, P, I, U, P, I64, P, P, P]
     L.qlinear_hadamard.restype = I
     L.qlinear_hadamard.argtypes = [P, I, I64, P, I, I64, I64, I64, I, P]
+    L.qlinear_dequantize.restype = I
+    L.qlinear_dequantize.argtypes = [P, I64, P, I64, I64, I, P, I, I64, P]
+    L.qlinear_codes_bf16.restype = I
+    L.qlinear_codes_bf16.argtypes = [P, I64, I64, I64, P, I64, P]
+    L.qlinear_fwd_bf16_workspace_bytes.restype = ctypes.c_size_t
+    L.qlinear_fwd_bf16_workspace_bytes.argtypes = [I64, I64, I, I]
+    L.qlinear_fwd_bf16.restype = I
+    L.qlinear_fwd_bf16.argtypes = [P, I, I64, I64, P, P, I64, P, I, P, I, P, ctypes.c_size_t, P, P]
     L.qlinear_fwd.restype = I
     L.qlinear_fwd.argtypes = [P, I, I64, I64, P, P, I64, P, I, P, I, P, P, P, P]
     L.qlinear_bwd_dx.restype = I
@@ -205,6 +214,49 @@ def qlinear_hadamard(x, y, hadamard_block: int, stream=None):
         _dev(x, "x"), _dtype_code(x, "x"), _rowmajor(x, "x"), _dev(y, "y"), _dtype_code(y, "y"),
         _rowmajor(y, "y"), rows, cols, hadamard_block, _stream(stream))
     _check(code, "qlinear_hadamard")
+
+
+def qlinear_dequantize(wq, sw, hadamard_block: int, w, stream=None):
+    """w <- (s_w * wq) R: the weight in floating point, back in the original basis."""
+    N, K = wq.shape
+    if tuple(w.shape) != (N, K):
+        raise ValueError("qlinear_dequantize: wq and w shapes differ")
+    _contig(sw, "sw")
+    code = lib().qlinear_dequantize(
+        _dev(wq, "wq", torch.int8), _rowmajor(wq, "wq"), _dev(sw, "sw", torch.float32), N, K,
+        hadamard_block, _dev(w, "w"), _dtype_code(w, "w"), _rowmajor(w, "w"), _stream(stream))
+    _check(code, "qlinear_dequantize")
+
+
+def qlinear_codes_bf16(wq, out, stream=None):
+    """out <- the int8 codes of wq as bf16 (exact)."""
+    N, K = wq.shape
+    if tuple(out.shape) != (N, K) or out.dtype != torch.bfloat16:
+        raise ValueError("qlinear_codes_bf16: out must be a bf16 tensor shaped like wq")
+    code = lib().qlinear_codes_bf16(_dev(wq, "wq", torch.int8), _rowmajor(wq, "wq"), N, K,
+                                    _dev(out, "out"), _rowmajor(out, "out"), _stream(stream))
+    _check(code, "qlinear_codes_bf16")
+
+
+def qlinear_fwd_bf16_workspace_bytes(M: int, K: int, x_dtype, hadamard_block: int) -> int:
+    xt = QL_BF16 if x_dtype == torch.bfloat16 else QL_F32
+    return int(lib().qlinear_fwd_bf16_workspace_bytes(M, K, xt, hadamard_block))
+
+
+def qlinear_fwd_bf16(x, wq_bf16, sw, bias, hadamard_block: int, y, ws, status, stream=None):
+    """y <- the bf16 route of the forward: bf16(x R) times the bf16 codes on the
+    tensor cores, times s_w, plus bias (no activation quantization)."""
+    M, K = x.shape
+    N = wq_bf16.shape[0]
+    for t, n in ((x, "x"), (wq_bf16, "wq_bf16"), (sw, "sw"), (bias, "bias"), (y, "y")):
+        _contig(t, n)
+    code = lib().qlinear_fwd_bf16(
+        _dev(x, "x"), _dtype_code(x, "x"), M, K, _dev(wq_bf16, "wq_bf16", torch.bfloat16),
+        _dev(sw, "sw", torch.float32), N, _dev(bias, "bias", torch.float32), hadamard_block,
+        _dev(y, "y"), _dtype_code(y, "y"), _dev(ws, "ws"),
+        0 if ws is None else ws.numel() * ws.element_size(), _dev(status, "status", torch.int32),
+        _stream(stream))
+    _check(code, "qlinear_fwd_bf16")
 
 
 def qlinear_fwd(x, wq, sw, bias, hadamard_block: int, y, xq_saved, sx_saved, status,

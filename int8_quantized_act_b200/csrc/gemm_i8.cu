@@ -121,7 +121,7 @@ __device__ __forceinline__ void store16(__nv_bfloat16* p, const float* v) {
 // + lane, columns col0 .. col0+255 of the output.  All 32 lanes of the warp
 // must call it (tcgen05.ld is warp-collective); rows/columns past the output
 // are computed but not stored.
-template <typename OutT, int HB>
+template <typename OutT, int HB, bool F16>
 __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, int quarter,
                                               int lane, int row0, int col0) {
   constexpr int CH = HB > 32 ? HB : 32;  // columns per register chunk
@@ -139,7 +139,8 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
     if (row_ok && gc0 < ep.cols) {
       float v[CH];
 #pragma unroll
-      for (int i = 0; i < CH; ++i) v[i] = __int2float_rn(static_cast<int>(r[i])) * rs;
+      for (int i = 0; i < CH; ++i)
+        v[i] = (F16 ? __uint_as_float(r[i]) : __int2float_rn(static_cast<int>(r[i]))) * rs;
       if (ep.col_scale || ep.bias) {
 #pragma unroll
         for (int g = 0; g < CH / 16; ++g) {
@@ -176,7 +177,7 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
   }
 }
 
-template <bool A_MN, bool B_MN, typename OutT, int HB>
+template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int tiles_m, int tiles_n, int kblocks, int group, Epi ep, int32_t* status) {
@@ -196,6 +197,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Contraction elements per stage: the TMA coordinate counts elements,
+  // 128 for int8, 64 for bf16 (128 bytes either way).
+  static_assert(!F16 || (!A_MN && !B_MN), "bf16 operands are read K-major");
+  constexpr int KE = F16 ? BK / 2 : BK;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -241,12 +246,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
           if (A_MN) tma_load_2d(a_dst, &tmA, fb, tm * BM, kb * BK);
-          else tma_load_2d(a_dst, &tmA, fb, kb * BK, tm * BM);
+          else tma_load_2d(a_dst, &tmA, fb, kb * KE, tm * BM);
           if (B_MN) {
             tma_load_2d(b_dst, &tmB, fb, tn * BN, kb * BK);
             tma_load_2d(b_dst + B_BYTES / 2, &tmB, fb, tn * BN + 128, kb * BK);
           } else {
-            tma_load_2d(b_dst, &tmB, fb, kb * BK, tn * BN);
+            tma_load_2d(b_dst, &tmB, fb, kb * KE, tn * BN);
           }
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -264,7 +269,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+      constexpr uint32_t idesc = F16 ? idesc_bf16(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0)
+                                     : idesc_i8(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -287,7 +293,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                          : smem_desc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t b_desc = B_MN ? smem_desc_sw128(b_base + kk * 4096, 16384, 1024)
                                          : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            mma_i8(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (F16) mma_bf16(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else mma_i8(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           mma_commit(empty0 + 8 * stage);
           if (++stage == STAGES) {
@@ -314,7 +321,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tile_coords(t, tiles_m, tiles_n, group, tm, tn);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile<OutT, HB>(ep, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
+      epilogue_tile<OutT, HB, F16>(ep, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -347,7 +354,7 @@ constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;  // 32 KiB
 constexpr int PNUM_BARS = 2 * PSTAGES + 5;
 constexpr int PSMEM_BYTES = 1024 + PSTAGES * PSTAGE_BYTES + 8 * PNUM_BARS + 16;
 
-template <bool A_MN, bool B_MN, typename OutT, int HB>
+template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int tiles_m, int tiles_n,
@@ -368,6 +375,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain = smem_u32(bars + 2 * PSTAGES + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  static_assert(!F16 || (!A_MN && !B_MN), "bf16 operands are read K-major");
+  constexpr int KE = F16 ? BK / 2 : BK;  // contraction elements per stage
   const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   if (threadIdx.x == 0) {
@@ -424,9 +433,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_dst = smem_u32(sA + stage * PA_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * PB_BYTES);
           if (A_MN) tma_load_2d_pair(a_dst, &tmA, fb, a_row, kb * BK);
-          else tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
+          else tma_load_2d_pair(a_dst, &tmA, fb, kb * KE, a_row);
           if (B_MN) tma_load_2d_pair(b_dst, &tmB, fb, b_col, kb * BK);
-          else tma_load_2d_pair(b_dst, &tmB, fb, kb * BK, b_col);
+          else tma_load_2d_pair(b_dst, &tmB, fb, kb * KE, b_col);
           if (++stage == PSTAGES) {
             stage = 0;
             phase ^= 1u;
@@ -445,7 +454,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (rank 0)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_i8(256, 256, A_MN ? 1 : 0, B_MN ? 1 : 0);
+      constexpr uint32_t idesc = F16 ? idesc_bf16(256, 256, A_MN ? 1 : 0, B_MN ? 1 : 0)
+                                     : idesc_i8(256, 256, A_MN ? 1 : 0, B_MN ? 1 : 0);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs) {
@@ -466,7 +476,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                          : smem_desc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t b_desc = B_MN ? smem_desc_sw128(b_base + kk * 4096, 16384, 1024)
                                          : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            mma_i8_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (F16) mma_bf16_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else mma_i8_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           mma_commit_pair_mc(empty0 + 8 * stage, 0x3);
           if (++stage == PSTAGES) {
@@ -492,7 +503,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         tile_coords(t, tiles_m, tiles_n, group, tm, tn);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile<OutT, HB>(ep, tmem_base + acc * BN, quarter, lane,
+      epilogue_tile<OutT, HB, F16>(ep, tmem_base + acc * BN, quarter, lane,
                               tm * 256 + static_cast<int>(rank) * 128, tn * BN);
       tc_fence_before();
       __syncwarp();
@@ -563,10 +574,10 @@ int pair_slots(K kern) {
   return n;
 }
 
-template <bool A_MN, bool B_MN, typename OutT, int HB>
+template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
                      int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
-  auto kern = gemm_i8_pair_kernel<A_MN, B_MN, OutT, HB>;
+  auto kern = gemm_i8_pair_kernel<A_MN, B_MN, OutT, HB, F16>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -589,10 +600,10 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
   return e;
 }
 
-template <bool A_MN, bool B_MN, typename OutT, int HB>
+template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
                 int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
-  auto kern = gemm_i8_kernel<A_MN, B_MN, OutT, HB>;
+  auto kern = gemm_i8_kernel<A_MN, B_MN, OutT, HB, F16>;
   // Opt in to the large dynamic shared memory once per device.
   static int configured[64] = {0};
   int dev = 0;
@@ -616,11 +627,11 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
   return e;
 }
 
-template <bool A_MN, bool B_MN, typename OutT, int HB>
+template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t go(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
                int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
-  if (pair) return run_pair<A_MN, B_MN, OutT, HB>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
-  return run<A_MN, B_MN, OutT, HB>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+  if (pair) return run_pair<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+  return run<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
 }
 
 cudaError_t dispatch_dx(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m,
@@ -711,6 +722,38 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
   if (a_mn && b_mn && e.hb == 0 && !bf16)
     return go<true, true, float, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t rows,
+                             int64_t cols, int64_t kc, const GemmEpilogue& e, int32_t* status,
+                             cudaStream_t s) {
+  // Both operands K-major bf16: a 128-byte stage row holds 64 elements and
+  // each kind::f16 MMA consumes K = 16 (32 bytes), the same byte layout as
+  // the int8 path.
+  const bool pair = rows > BM;
+  CUtensorMap ta, tb;
+  const bool ok_a = encode_tmap_2d(&ta, 2, A, static_cast<uint64_t>(kc), static_cast<uint64_t>(rows),
+                                   static_cast<uint64_t>(lda) * 2, BK / 2, BM, true);
+  const bool ok_b = encode_tmap_2d(&tb, 2, B, static_cast<uint64_t>(kc), static_cast<uint64_t>(cols),
+                                   static_cast<uint64_t>(ldb) * 2, BK / 2, pair ? 128 : BN, true);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+  Epi ep;
+  ep.out = e.out;
+  ep.ldo = e.ldo;
+  ep.rows = static_cast<int>(rows);
+  ep.cols = static_cast<int>(cols);
+  ep.row_scale = e.row_scale;
+  ep.col_scale = e.col_scale;
+  ep.bias = e.bias;
+  ep.hc = e.hc;
+  const int tile_rows = pair ? 2 * BM : BM;
+  const int tiles_m = static_cast<int>((rows + tile_rows - 1) / tile_rows);
+  const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
+  const int kblocks = static_cast<int>((kc + BK / 2 - 1) / (BK / 2));
+  if (e.hb != 0) return cudaErrorInvalidValue;
+  if (e.out_bf16)
+    return go<false, false, __nv_bfloat16, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+  return go<false, false, float, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
 }
 
 }  // namespace ql

@@ -39,6 +39,11 @@ cudaError_t launch_quant_rows(const void* x, int xt, int64_t rows, int64_t cols,
 cudaError_t launch_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt, int64_t ldy,
                             int64_t rows, int64_t cols, int B, float hc, cudaStream_t s);
 
+// w[r,:] = s[r] * q[r,:] in float32, then times R for B > 0 (hc = fl32(1/sqrt(B))).
+cudaError_t launch_dequant_rows(const int8_t* q, int64_t ldq, const float* s, void* w, int wt,
+                                int64_t ldw, int64_t rows, int64_t cols, int B, float hc,
+                                cudaStream_t st);
+
 // Column statistics of t = dY[m,n]*s_x[m]: colmax[n] = bits of max|t|
 // (atomicMax; caller zeroes), colsum[n] += sum_m dY[m,n] in float64.  With
 // rowmax != NULL also rowmax[m] = bits of max_n |dY[m,n]*sw[n]| (caller zeroes).
@@ -84,6 +89,13 @@ struct GemmEpilogue {
 cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
                            int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
                            const GemmEpilogue& ep, int32_t* status, cudaStream_t s);
+
+// The same GEMM on bf16 operands (tcgen05 kind::f16, float32 accumulator):
+// A [rows][kc] and B [cols][kc] both K-major bf16 with pitches lda, ldb
+// elements; out = acc * row_scale * col_scale + bias as above, hb must be 0.
+cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t rows,
+                             int64_t cols, int64_t kc, const GemmEpilogue& ep, int32_t* status,
+                             cudaStream_t s);
 
 // -------------------------------------------------------------- update
 struct UpdateConsts {

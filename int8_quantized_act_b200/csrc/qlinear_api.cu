@@ -206,6 +206,72 @@ int qlinear_fwd(const void* x, int xt, int64_t M, int64_t K, const int8_t* wq, c
   return cuda_status(ql::launch_gemm_i8(xq_saved, false, K, wq, false, K, M, N, K, ep, d_status, s));
 }
 
+int qlinear_dequantize(const int8_t* wq, int64_t ldq, const float* sw, int64_t N, int64_t K,
+                       int hadamard_block, void* w, int wt, int64_t ldw, void* stream) {
+  if (!valid_dtype(wt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
+  if (N < 0 || K < 0 || K % 16 != 0 || N > INT32_MAX || K > INT32_MAX || ldq < K ||
+      ldq % 16 != 0 || ldw < K || (hadamard_block > 0 && K % hadamard_block != 0))
+    return QL_ERR_SHAPE;
+  if (N == 0 || K == 0) return QL_OK;
+  if (!wq || !sw || !w) return QL_ERR_ARG;
+  if (!aligned16(wq) || !aligned16(w) || (ldw * elem_size(wt)) % 16 != 0) return QL_ERR_ALIGN;
+  return cuda_status(ql::launch_dequant_rows(wq, ldq, sw, w, wt, ldw, N, K, hadamard_block,
+                                             hadamard_c(hadamard_block), as_stream(stream)));
+}
+
+int qlinear_codes_bf16(const int8_t* wq, int64_t ldq, int64_t N, int64_t K, void* out,
+                       int64_t ldo, void* stream) {
+  if (N < 0 || K < 0 || K % 16 != 0 || N > INT32_MAX || K > INT32_MAX || ldq < K ||
+      ldq % 16 != 0 || ldo < K)
+    return QL_ERR_SHAPE;
+  if (N == 0 || K == 0) return QL_OK;
+  if (!wq || !out) return QL_ERR_ARG;
+  if (!aligned16(wq) || !aligned16(out) || (ldo * 2) % 16 != 0) return QL_ERR_ALIGN;
+  // The codes times 1.0 (exact) stored as bf16 (exact).
+  return cuda_status(ql::launch_dequant_rows(wq, ldq, nullptr, out, QL_BF16, ldo, N, K, 0, 1.0f,
+                                             as_stream(stream)));
+}
+
+size_t qlinear_fwd_bf16_workspace_bytes(int64_t M, int64_t K, int xt, int hadamard_block) {
+  if (M < 0 || K < 0) return 0;
+  if (xt == QL_BF16 && hadamard_block == 0) return 0;
+  return align256(2 * static_cast<size_t>(M) * static_cast<size_t>(K));
+}
+
+int qlinear_fwd_bf16(const void* x, int xt, int64_t M, int64_t K, const void* wq_bf16,
+                     const float* sw, int64_t N, const float* bias, int hadamard_block, void* y,
+                     int yt, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (!valid_dtype(xt) || !valid_dtype(yt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX ||
+      K > INT32_MAX || (hadamard_block > 0 && K % hadamard_block != 0))
+    return QL_ERR_SHAPE;
+  if (M == 0 || N == 0) return QL_OK;
+  if (!y || !d_status || (K > 0 && (!x || !wq_bf16 || !sw))) return QL_ERR_ARG;
+  const bool need_xr = K > 0 && !(xt == QL_BF16 && hadamard_block == 0);
+  if (need_xr && (!ws || ws_bytes < qlinear_fwd_bf16_workspace_bytes(M, K, xt, hadamard_block)))
+    return QL_ERR_SHAPE;
+  if (!aligned16(y) || (bias && !aligned16(bias)) ||
+      (K > 0 && (!aligned16(x) || !aligned16(wq_bf16) || !aligned16(sw))) ||
+      (need_xr && (reinterpret_cast<uintptr_t>(ws) & 255u)))
+    return QL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  if (K == 0) return cuda_status(ql::launch_fill_rows(y, yt, M, N, bias, s));
+  const void* xr = x;
+  if (need_xr) {
+    cudaError_t e = ql::launch_hadamard(x, xt, K, ws, QL_BF16, K, M, K, hadamard_block,
+                                        hadamard_c(hadamard_block), s);
+    if (e != cudaSuccess) return QL_ERR_CUDA;
+    xr = ws;
+  }
+  GemmEpilogue ep;
+  ep.out = y;
+  ep.out_bf16 = yt == QL_BF16;
+  ep.ldo = N;
+  ep.col_scale = sw;
+  ep.bias = bias;
+  return cuda_status(ql::launch_gemm_bf16(xr, K, wq_bf16, K, M, N, K, ep, d_status, s));
+}
+
 int qlinear_bwd_dx(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
                    const float* sw, int64_t K, int hadamard_block, void* dx, int dxt, void* ws,
                    size_t ws_bytes, int32_t* d_status, void* stream) {

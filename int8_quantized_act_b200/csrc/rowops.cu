@@ -331,6 +331,41 @@ __global__ void __launch_bounds__(256) hadamard_kernel(const InT* x, int64_t ldx
   }
 }
 
+// w[r, :] = s[r] * q[r, :] (one float32 multiply), then for B > 0 the
+// block-Hadamard of fwht_chunk (R is its own inverse: back to the original
+// basis).  A warp converts one 256-column chunk, 8 codes per lane.
+template <typename OutT>
+__global__ void __launch_bounds__(256) dequant_rows_kernel(const int8_t* __restrict__ q,
+                                                           int64_t ldq, const float* __restrict__ s,
+                                                           OutT* __restrict__ w, int64_t ldw,
+                                                           int64_t rows, int cols, int B, float hc) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nchunks = (cols + 255) / 256;
+  const int64_t total = rows * nchunks;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); t < total;
+       t += wstride) {
+    const int64_t r = t / nchunks;
+    const int col = static_cast<int>(t % nchunks) * 256 + lane * 8;
+    float v[8];
+    if (col < cols) {
+      const float sr = s ? __ldg(s + r) : 1.0f;
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(q + r * ldq + col));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t word = i < 4 ? u.x : u.y;
+        const int code = static_cast<int8_t>((word >> (8 * (i & 3))) & 0xFFu);
+        v[i] = static_cast<float>(code) * sr;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+    if (B > 0) fwht_chunk(v, B, lane, hc);
+    if (col < cols) store8(w + r * ldw + col, v);
+  }
+}
+
 __global__ void colfinalize_kernel(const uint32_t* __restrict__ colmax,
                                    const double* __restrict__ colsum, int N, float* s2,
                                    float* inv2, float* db) {
@@ -466,6 +501,22 @@ cudaError_t launch_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt,
   else if (yt == QL_F32) QL_HD(__nv_bfloat16, float);
   else QL_HD(__nv_bfloat16, __nv_bfloat16);
 #undef QL_HD
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_rows(const int8_t* q, int64_t ldq, const float* s, void* w, int wt,
+                                int64_t ldw, int64_t rows, int64_t cols, int B, float hc,
+                                cudaStream_t st) {
+  const int64_t tasks = rows * ((cols + 255) / 256);
+  const int grid = grid_cap((tasks + 7) / 8, 8);
+  const int c = static_cast<int>(cols);
+  if (wt == QL_BF16)
+    dequant_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        q, ldq, s, reinterpret_cast<__nv_bfloat16*>(w), ldw, rows, c, B, hc);
+  else
+    dequant_rows_kernel<float><<<grid, 256, 0, st>>>(q, ldq, s, reinterpret_cast<float*>(w), ldw,
+                                                      rows, c, B, hc);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -36,7 +36,8 @@ def test_every_declared_symbol_is_exported(L):
     assert set(names) >= {"qlinear_quantize_rows", "qlinear_hadamard", "qlinear_fwd",
                           "qlinear_bwd_dx", "qlinear_bwd_dw", "qweight_update_sr",
                           "ql_status_string", "qlinear_workspace_bytes", "qlinear_bwd",
-                          "qlinear_bwd_dx_noalloc", "ql_test_wait_timeout"}
+                          "qlinear_bwd_dx_noalloc", "ql_test_wait_timeout", "qlinear_dequantize",
+                          "qlinear_codes_bf16", "qlinear_fwd_bf16", "qlinear_fwd_bf16_workspace_bytes"}
     for n in names:
         assert hasattr(L, n), n
 
@@ -131,3 +132,38 @@ def test_timeout_hook_validation(L):
     assert L.ql_test_wait_timeout(None, 1000, None) == ql.QL_ERR_ARG
     assert L.ql_test_wait_timeout(fake(0x10000), 0, None) == ql.QL_ERR_ARG
     assert L.ql_test_wait_timeout(fake(0x10000), 10000001, None) == ql.QL_ERR_ARG
+
+
+def test_dequantize_validation(L):
+    A = 0x10000
+    f = L.qlinear_dequantize
+    assert f(fake(A), 32, fake(A), 4, 32, 3, fake(A), 0, 32, None) == ql.QL_ERR_ARG      # block
+    assert f(fake(A), 32, fake(A), 4, 32, 0, fake(A), 7, 32, None) == ql.QL_ERR_ARG      # dtype
+    assert f(fake(A), 48, fake(A), 4, 48, 32, fake(A), 0, 48, None) == ql.QL_ERR_SHAPE   # K % B
+    assert f(fake(A), 40, fake(A), 4, 40, 0, fake(A), 0, 40, None) == ql.QL_ERR_SHAPE    # K % 16
+    assert f(fake(A), 24, fake(A), 4, 32, 0, fake(A), 0, 32, None) == ql.QL_ERR_SHAPE    # ldq < K
+    assert f(fake(A + 8), 32, fake(A), 4, 32, 0, fake(A), 0, 32, None) == ql.QL_ERR_ALIGN
+    assert f(fake(A), 32, fake(A), 4, 32, 0, fake(A), 1, 36, None) == ql.QL_ERR_ALIGN    # bf16 pitch
+    assert f(None, 32, None, 0, 32, 0, None, 0, 32, None) == ql.QL_OK                   # nothing to do
+
+
+def test_bf16_route_validation_and_workspace(L):
+    A = 0x10000
+    assert ql.lib().qlinear_fwd_bf16_workspace_bytes(100, 512, ql.QL_BF16, 0) == 0
+    assert ql.lib().qlinear_fwd_bf16_workspace_bytes(100, 512, ql.QL_BF16, 128) == 102400
+    assert ql.lib().qlinear_fwd_bf16_workspace_bytes(3, 32, ql.QL_F32, 0) == 256
+    f = L.qlinear_fwd_bf16
+    args = lambda **kw: [kw.get("x", fake(A)), kw.get("xt", 1), kw.get("M", 4), kw.get("K", 64),
+                         kw.get("w", fake(A)), fake(A), kw.get("N", 32), None, kw.get("B", 0),
+                         kw.get("y", fake(A)), 1, kw.get("ws", None), kw.get("wsb", 0), fake(A), None]
+    assert f(*args(B=3)) == ql.QL_ERR_ARG
+    assert f(*args(K=40)) == ql.QL_ERR_SHAPE
+    assert f(*args(N=24)) == ql.QL_ERR_SHAPE
+    assert f(*args(B=128)) == ql.QL_ERR_SHAPE                  # K % B
+    assert f(*args(B=32)) == ql.QL_ERR_SHAPE                   # needs a workspace
+    assert f(*args(B=32, ws=fake(A + 16), wsb=1 << 20)) == ql.QL_ERR_ALIGN
+    assert f(*args(x=fake(A + 8))) == ql.QL_ERR_ALIGN
+    assert f(*args(M=0)) == ql.QL_OK
+    g = L.qlinear_codes_bf16
+    assert g(fake(A), 32, 4, 40, fake(A), 40, None) == ql.QL_ERR_SHAPE
+    assert g(fake(A), 32, 4, 32, fake(A), 36, None) == ql.QL_ERR_ALIGN

@@ -145,3 +145,31 @@ def test_host_validation_errors():
         ql.qlinear_quantize_rows(flat[1:1 + 4 * 48].view(4, 48), q, s, st)  # misaligned
     assert e.value.code == ql.QL_ERR_ALIGN
     assert status_word(st) == 0
+
+
+@pytest.mark.parametrize("B", [0, 2, 16, 128, 256])
+@pytest.mark.parametrize("wt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("N,K", [(37, 768), (300, 5376), (5, 16)])
+def test_dequantize_matches_oracle(N, K, B, wt):
+    """(s_w q) R back to the original basis: the same float32 operations in
+    the same order as the oracle (bf16 output = the oracle's value rounded)."""
+    if B and K % B:
+        pytest.skip("block does not divide K")
+    w = workloads.normal((N, K), 0.02, N + K + B)
+    q, s, st = oracle.quantize_rows(w, B=B, flags=oracle.REJECT_ZERO_ROWS)
+    assert st == 0
+    out = torch.empty((N, K), dtype=wt, device="cuda")
+    ql.qlinear_dequantize(dev(q), dev(s), B, out)
+    ref, rst = oracle.dequantize(q, s, B)
+    assert rst == 0
+    ref_t = torch.from_numpy(ref).to(wt).float().numpy()
+    assert np.array_equal(host(out), ref_t)
+
+
+def test_dequantize_strided_output():
+    q = np.random.Generator(np.random.PCG64(5)).integers(-127, 128, (24, 512)).astype(np.int8)
+    s = workloads.uniform((24,), 1e-3, 1e-2, 6)
+    big = torch.zeros((24, 640), device="cuda")
+    ql.qlinear_dequantize(dev(q), dev(s), 64, big[:, :512])
+    ref, _ = oracle.dequantize(q, s, 64)
+    assert np.array_equal(host(big[:, :512]), ref) and not host(big[:, 512:]).any()
