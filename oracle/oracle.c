@@ -256,6 +256,39 @@ uint32_t ref_gemm_tn(const int8_t *A, int64_t lda, const int8_t *Bm, int64_t ldb
     return 0;
 }
 
+/* The same two products with int64 outputs and no range limit: contractions
+ * longer than 131,071 combine their bounded int32 partial dot products in
+ * int64 before scaling ([QT], contraction paragraph).  Integer addition is
+ * associative, so any chunking of the contraction gives this exact sum. */
+void ref_gemm_nn64(const int8_t *A, int64_t lda, const int8_t *Bm, int64_t ldb,
+                   int64_t M, int64_t N, int64_t C, int64_t *out, int64_t ldo) {
+    for (int64_t m = 0; m < M; ++m) {
+        int64_t *acc = out + m * ldo;
+        for (int64_t n = 0; n < N; ++n) acc[n] = 0;
+        for (int64_t c = 0; c < C; ++c) {
+            int64_t a = A[m * lda + c];
+            if (a == 0) continue;
+            const int8_t *b = Bm + c * ldb;
+            for (int64_t n = 0; n < N; ++n) acc[n] += a * (int64_t)b[n];
+        }
+    }
+}
+
+void ref_gemm_tn64(const int8_t *A, int64_t lda, const int8_t *Bm, int64_t ldb,
+                   int64_t M, int64_t N, int64_t C, int64_t *out, int64_t ldo) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) out[m * ldo + n] = 0;
+    for (int64_t c = 0; c < C; ++c) {
+        const int8_t *a = A + c * lda, *b = Bm + c * ldb;
+        for (int64_t m = 0; m < M; ++m) {
+            int64_t am = a[m];
+            if (am == 0) continue;
+            int64_t *row = out + m * ldo;
+            for (int64_t n = 0; n < N; ++n) row[n] += am * (int64_t)b[n];
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Layer forward ([CR] item 1 and Summary; [QT] intro and table row     */
 /* "Inputs and inference": bias, batched and single-sample inputs)      */
@@ -378,16 +411,18 @@ uint32_t ref_bwd_prep_cols(const float *dy, int64_t M, int64_t N, const float *s
 }
 
 /* dX[m,k] = (float)(sum_n dYq_r[m,n] W_q[n,k]) * s1[m]; then, for a rotated
- * layer (B > 0), each row of dX times R (R symmetric, so this is dX' R^T). */
+ * layer (B > 0), each row of dX times R (R symmetric, so this is dX' R^T).
+ * The sum is exact in int64 for any N: above 131,071 output classes it is
+ * the int64 combination of int32 chunk sums ([QT], contraction paragraph),
+ * converted to float32 once (round to nearest even). */
 uint32_t ref_bwd_dx(const float *dy, int64_t M, int64_t N, const int8_t *wq,
                     const float *sw, int64_t K, int B, float *dx,
                     int8_t *dyq_r, float *s1) {
-    if (N > ORC_MAX_CONTRACTION) return ORC_BIT_UNSUPP;
     if (!valid_block(B)) return ORC_BIT_ARG;
     if (B > 0 && K % B != 0) return ORC_BIT_SHAPE;
     uint32_t st = ref_bwd_prep_rows(dy, M, N, sw, dyq_r, s1);
-    int32_t *acc = (int32_t *)malloc((size_t)(M * K > 0 ? M * K : 1) * sizeof(int32_t));
-    st |= ref_gemm_nn(dyq_r, N, wq, K, M, K, N, acc, K);
+    int64_t *acc = (int64_t *)malloc((size_t)(M * K > 0 ? M * K : 1) * sizeof(int64_t));
+    ref_gemm_nn64(dyq_r, N, wq, K, M, K, N, acc, K);
     for (int64_t m = 0; m < M; ++m)
         for (int64_t k = 0; k < K; ++k) dx[m * K + k] = (float)acc[m * K + k] * s1[m];
     free(acc);
@@ -395,14 +430,15 @@ uint32_t ref_bwd_dx(const float *dy, int64_t M, int64_t N, const int8_t *wq,
     return st;
 }
 
-/* dW[n,k] = (float)(sum_m dYq_c[m,n] X_q[m,k]) * s2[n]; db as above. */
+/* dW[n,k] = (float)(sum_m dYq_c[m,n] X_q[m,k]) * s2[n]; db as above.  The
+ * sum over tokens is exact in int64 for any M (int64 combination of int32
+ * chunk sums above 131,071 tokens). */
 uint32_t ref_bwd_dw(const float *dy, int64_t M, int64_t N, const int8_t *xq,
                     const float *sx, int64_t K, float *dw, float *db,
                     int8_t *dyq_c, float *s2) {
-    if (M > ORC_MAX_CONTRACTION) return ORC_BIT_UNSUPP;
     uint32_t st = ref_bwd_prep_cols(dy, M, N, sx, dyq_c, s2, db);
-    int32_t *acc = (int32_t *)malloc((size_t)(N * K > 0 ? N * K : 1) * sizeof(int32_t));
-    st |= ref_gemm_tn(dyq_c, N, xq, K, N, K, M, acc, K);
+    int64_t *acc = (int64_t *)malloc((size_t)(N * K > 0 ? N * K : 1) * sizeof(int64_t));
+    ref_gemm_tn64(dyq_c, N, xq, K, N, K, M, acc, K);
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) dw[n * K + k] = (float)acc[n * K + k] * s2[n];
     free(acc);

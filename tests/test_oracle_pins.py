@@ -332,11 +332,51 @@ def test_gemm_closed_forms_and_int32_limit():
     assert st == 0 and out[0, 0] == 16129 * limit == 2114044159
     out, st = oracle.gemm_nt(A, -A)
     assert st == 0 and out[0, 0] == -2114044159
-    # beyond the limit the layer reports the contraction as unsupported
+    # beyond the limit the forward reports its contraction (in_features) as
+    # unsupported; the backward products combine chunks in int64 (below)
     x = np.zeros((1, limit + 1), np.float32)
     w = np.zeros((1, limit + 1), np.int8)
     y, _, _, st = oracle.fwd(x, w, np.zeros(1, np.float32))
     assert st == oracle.BIT_UNSUPPORTED
+
+
+def test_bwd_dx_beyond_int32_combines_in_int64():
+    """140,000 output classes of all-127 codes sum to 16129 * 140000 =
+    2,258,060,000 > 2^31 - 1: the input gradient's dot products leave int32,
+    and the page combines bounded int32 chunk sums in int64 before scaling,
+    which is the exact integer sum, converted to float32 once."""
+    N, M, K = 140000, 2, 32
+    dy = np.ones((M, N), np.float32)
+    dy[1] = -1.0
+    wq = np.full((N, K), 127, np.int8)
+    dx, rq, s1, st = oracle.bwd_dx(dy, wq, np.ones(N, np.float32), 0)
+    acc = 16129 * N
+    assert acc > 2 ** 31 - 1 and st == 0
+    assert np.all(rq[0] == 127) and np.all(rq[1] == -127)
+    assert np.array_equal(dx[0], np.full(K, np.float32(acc) * s1[0], np.float32))
+    assert np.array_equal(dx[1], np.full(K, np.float32(-acc) * s1[1], np.float32))
+
+
+def test_bwd_long_contractions_match_numpy_int64():
+    """dX over 150,000 output classes and dW over 140,000 tokens: the oracle's
+    sums against numpy's int64 matmul of the same codes."""
+    rng = np.random.Generator(np.random.PCG64(41))
+    N, M, K = 150000, 3, 16
+    dy = rng.standard_normal((M, N)).astype(np.float32)
+    wq = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    sw = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    dx, rq, s1, st = oracle.bwd_dx(dy, wq, sw, 0)
+    assert st == 0
+    acc = rq.astype(np.int64) @ wq.astype(np.int64)
+    assert np.array_equal(dx, acc.astype(np.float32) * s1[:, None])
+    M, N = 140000, 3
+    dy = rng.standard_normal((M, N)).astype(np.float32)
+    xq = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    sx = rng.uniform(1e-3, 1e-2, M).astype(np.float32)
+    dw, db, rqc, s2, st = oracle.bwd_dw(dy, xq, sx)
+    assert st == 0
+    acc = rqc.astype(np.int64).T @ xq.astype(np.int64)
+    assert np.array_equal(dw, acc.astype(np.float32) * s2[:, None])
 
 
 # --------------------------------------------------------------------------
