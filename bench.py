@@ -65,6 +65,9 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--routes", action="store_true",
+                   help="instead of the train step: time the forward's int8 and bf16 routes "
+                        "at 2048 and 12000 tokens (one JSON line)")
     return p.parse_args()
 
 
@@ -451,8 +454,90 @@ def run_reference(args, rank, world):
     }
 
 
+def run_routes(args):
+    """The page's forward-route comparison on this GPU: the int8 route
+    (rotate + quantize x, int8 GEMM) against the bf16 route (rotate x to
+    bf16, bf16 GEMM against the codes as bf16, converted once per weight
+    update and timed separately) at 2048 and 12000 tokens of the 5376 ->
+    7168 layer, block 128, bf16 x and y.  Whole-call and GEMM-only device
+    times (CUDA events), medians over `steps` calls."""
+    import torch
+    import int8_quantized_act_b200 as ql
+    import workloads
+    torch.cuda.set_device(0)
+    peaks = load_peaks()
+    out = {"metric": "forward route time (ms per call)", "unit": "ms", "higher_is_better": False,
+           "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic",
+           "config": {"workload": "5376 -> 7168 layer forward, Hadamard block 128, bf16 x and y",
+                      "K": K_IN, "N": N_OUT, "hadamard_block": BLOCK},
+           "routes": {}}
+    d = workloads.rotated_layer(M=12000, seed=1)
+    dev = "cuda"
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    wq = torch.empty((N_OUT, K_IN), dtype=torch.int8, device=dev)
+    sw = torch.empty(N_OUT, device=dev)
+    ql.qlinear_quantize_rows(torch.from_numpy(d["w"]).to(dev), wq, sw, st, hadamard_block=BLOCK,
+                             flags=ql.QL_REJECT_ZERO_ROWS)
+    wb = torch.empty((N_OUT, K_IN), dtype=torch.bfloat16, device=dev)
+    bias = torch.from_numpy(d["bias"]).to(dev)
+    x_all = d["x_bf16"].to(dev)
+
+    def timed(fn, gemm=False):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        gev = [tuple(new_events(2)) for _ in range(args.steps)] if gemm else None
+        for _ in range(args.warmup):
+            fn(None)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            ev[i][0].record()
+            fn(gev[i] if gemm else None)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        call = statistics.median(a.elapsed_time(b) for a, b in ev)
+        g = statistics.median(a.elapsed_time(b) for a, b in gev) if gemm else None
+        return call, g
+
+    ms_codes, _ = timed(lambda _e: ql.qlinear_codes_bf16(wq, wb))
+    out["codes_bf16_ms"] = round(ms_codes, 4)
+    for M in (2048, 12000):
+        x = x_all[:M].contiguous()
+        y = torch.empty((M, N_OUT), dtype=torch.bfloat16, device=dev)
+        xq = torch.empty((M, K_IN), dtype=torch.int8, device=dev)
+        sx = torch.empty(M, device=dev)
+        ws = torch.empty(ql.qlinear_fwd_bf16_workspace_bytes(M, K_IN, torch.bfloat16, BLOCK),
+                         dtype=torch.uint8, device=dev)
+
+        def int8_route(g):
+            ql.ql_set_gemm_timing_events([g] if g else ())
+            ql.qlinear_fwd(x, wq, sw, bias, BLOCK, y, xq, sx, st)
+            ql.ql_set_gemm_timing_events(())
+
+        def bf16_route(g):
+            ql.ql_set_gemm_timing_events([g] if g else ())
+            ql.qlinear_fwd_bf16(x, wb, sw, bias, BLOCK, y, ws, st)
+            ql.ql_set_gemm_timing_events(())
+
+        ops = 2.0 * M * N_OUT * K_IN
+        c8, g8 = timed(int8_route, gemm=True)
+        cb, gb = timed(bf16_route, gemm=True)
+        out["routes"][str(M)] = {
+            "int8_ms": round(c8, 4), "int8_gemm_ms": round(g8, 4),
+            "int8_gemm_tops": round(ops / (g8 * 1e-3) / 1e12, 1),
+            "bf16_ms": round(cb, 4), "bf16_gemm_ms": round(gb, 4),
+            "bf16_gemm_tflops": round(ops / (gb * 1e-3) / 1e12, 1),
+            "bf16_gemm_frac_of_measured_bf16_peak": round(ops / (gb * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+        }
+    if int(st.item()):
+        raise RuntimeError(f"device status {ql.status_flags(int(st.item()))}")
+    return out
+
+
 def main():
     args = parse_args()
+    if args.routes:
+        print(json.dumps(run_routes(args)), flush=True)
+        return
     world_env = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

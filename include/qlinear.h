@@ -73,7 +73,7 @@ typedef enum {
     QL_ERR_ZERO_ROW = 4,    /* device: a rejected all-zero row / direction      */
     QL_ERR_NONFINITE = 5,   /* device: inf or NaN met; affected outputs are
                                unspecified                                       */
-    QL_ERR_UNSUPPORTED = 6, /* contraction above 131,071 ([QT]), row too long   */
+    QL_ERR_UNSUPPORTED = 6, /* forward K above 131,071 ([QT]), row too long     */
     QL_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed              */
     QL_ERR_TIMEOUT = 8      /* device: a pipeline wait gave up (bounded waits;
                                the kernel returns instead of hanging)            */
@@ -107,9 +107,14 @@ typedef struct {
  * when preparing weights: a zero direction cannot be represented). */
 #define QL_REJECT_ZERO_ROWS 1u
 
-/* Largest contraction length accepted by the GEMMs: no int8 dot product of
- * this length can leave int32, floor((2^31-1)/128^2) ([QT], contraction
- * paragraph). */
+/* Longest int32-safe contraction: no int8 dot product of this length can
+ * leave int32, floor((2^31-1)/128^2) ([QT], contraction paragraph).  The
+ * forward accepts contractions (K) up to it.  The backward products go past
+ * it: the input gradient's sum over N output classes and the weight
+ * gradient's sum over M tokens then run in splits of at most 130,944 whose
+ * int32 partial sums are combined in int64 before scaling, exactly the int64
+ * sum ([QT]: this keeps input gradients at large output-class counts from
+ * saturating); the workspace grows by the partial sums. */
 #define QL_MAX_CONTRACTION 131071
 
 /* Human-readable name of a status code (static string). */
@@ -208,7 +213,7 @@ QL_API int qlinear_fwd(const void *x, int xt, int64_t M, int64_t K,
  * (the layer saw xR, and R is symmetric, so dL/dx = dL/d(xR) R^T = (...) R).
  * dY [M,N] (dyt), W_q [N,K], s_w [N], dX [M,K] (dxt).  ws: device workspace of
  * at least qlinear_workspace_bytes(M,N,K,B) bytes, 256-byte aligned.
- * N <= QL_MAX_CONTRACTION. */
+ * N above QL_MAX_CONTRACTION runs as int64-combined splits (see there). */
 QL_API int qlinear_bwd_dx(const void *dy, int dyt, int64_t M, int64_t N,
                    const int8_t *wq, const float *sw, int64_t K, int hadamard_block,
                    void *dx, int dxt, void *ws, size_t ws_bytes,
@@ -221,7 +226,8 @@ QL_API int qlinear_bwd_dx(const void *dy, int dyt, int64_t M, int64_t N,
  *             in the rotated basis when the layer is rotated)
  *   db[n]   = sum_m dY[m,n] (float64 sum rounded to float32), if db != NULL.
  * dY [M,N] (dyt), X_q [M,K] int8 and s_x [M] as saved by qlinear_fwd.
- * M <= QL_MAX_CONTRACTION.  ws as for qlinear_bwd_dx. */
+ * M above QL_MAX_CONTRACTION runs as int64-combined splits.  ws as for
+ * qlinear_bwd_dx. */
 QL_API int qlinear_bwd_dw(const void *dy, int dyt, int64_t M, int64_t N,
                    const int8_t *xq, const float *sx, int64_t K,
                    float *dw, float *db, void *ws, size_t ws_bytes,
@@ -237,7 +243,7 @@ QL_API size_t qlinear_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int h
  * a second pass writes both the row-quantized (dY*s_w) and the column-
  * quantized (dY*s_x) int8 copies from the same read.  Arguments as for the
  * two calls; ws holds qlinear_bwd_workspace_bytes(M, N, K, hadamard_block)
- * bytes.  N, M <= QL_MAX_CONTRACTION. */
+ * bytes.  Long contractions as for the two calls. */
 QL_API int qlinear_bwd(const void *dy, int dyt, int64_t M, int64_t N,
                        const int8_t *wq, const float *sw, const int8_t *xq, const float *sx,
                        int64_t K, int hadamard_block, void *dx, int dxt, float *dw, float *db,

@@ -23,6 +23,8 @@
 // filled by TMA, so M has no floor and tails need no special path.
 // No TMA multicast is used anywhere.
 #include <cuda.h>
+#include <algorithm>
+#include <type_traits>
 #include <cuda_bf16.h>
 
 #include "launch.h"
@@ -37,6 +39,9 @@ constexpr int BM = 128;                // tile rows (TMEM lanes)
 constexpr int BN = 256;                // tile columns (TMEM columns per accumulator)
 constexpr int BK = 128;                // contraction bytes per stage (4 MMAs of K=32)
 constexpr int STAGES = 4;
+// Longest int32-safe contraction split in 128-element blocks: 1023 * 128 =
+// 130,944 <= 131,071 = floor((2^31 - 1) / 128^2).
+constexpr int64_t kMaxSplitBlocks = 1023;
 constexpr int A_BYTES = BM * BK;       // 16 KiB
 constexpr int B_BYTES = BN * BK;       // 32 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -48,6 +53,7 @@ constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 8 *
 struct Epi {
   void* out;
   int64_t ldo;
+  int64_t split_stride;  // elements between the outputs of successive contraction splits
   int rows, cols;
   const float* row_scale;
   const float* col_scale;
@@ -128,6 +134,7 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
   OutT* out = reinterpret_cast<OutT*>(ep.out);
   const int gr = row0 + quarter * 32 + lane;
   const bool row_ok = gr < ep.rows;
+
   const float rs = (row_ok && ep.row_scale) ? ep.row_scale[gr] : 1.0f;
   const uint32_t taddr = acc_tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
@@ -177,10 +184,39 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
   }
 }
 
+// Raw int32 partial sums of one contraction split (no scaling), the same
+// slab as epilogue_tile.
+__device__ __forceinline__ void epilogue_tile_raw(const Epi& ep, uint32_t acc_tmem, int quarter,
+                                                  int lane, int row0, int col0) {
+  int32_t* out = reinterpret_cast<int32_t*>(ep.out);
+  const int gr = row0 + quarter * 32 + lane;
+  const bool row_ok = gr < ep.rows;
+  const uint32_t taddr = acc_tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld_cols<32>(taddr + c0, r);
+    tmem_wait_ld();
+    const int gc0 = col0 + c0;
+    if (row_ok && gc0 < ep.cols) {
+      int32_t* orow = out + static_cast<int64_t>(gr) * ep.ldo + gc0;
+#pragma unroll
+      for (int g = 0; g < 2; ++g)
+        if (gc0 + 16 * g < ep.cols)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            reinterpret_cast<uint4*>(orow + 16 * g)[i] =
+                make_uint4(r[16 * g + 4 * i], r[16 * g + 4 * i + 1], r[16 * g + 4 * i + 2],
+                           r[16 * g + 4 * i + 3]);
+    }
+  }
+}
+
 template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int tiles_m, int tiles_n, int kblocks, int group, Epi ep, int32_t* status) {
+                   int tiles_m, int tiles_n, int kblocks, int kps, int group, Epi ep,
+                   int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -226,7 +262,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = tiles_m * tiles_n;
+  // Contraction splits of kps k-blocks each (one split unless the
+  // contraction exceeds the int32-safe length); tile t is split t / per_split.
+  const int per_split = tiles_m * tiles_n;
+  const int num_tiles = per_split * ((kblocks + kps - 1) / kps);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -235,8 +274,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         int tm, tn;
-        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int sp = t / per_split;
+        tile_coords(t - sp * per_split, tiles_m, tiles_n, group, tm, tn);
+        const int kb1 = min(kblocks, (sp + 1) * kps);
+        for (int kb = sp * kps; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -277,7 +318,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int kb0 = (t / per_split) * kps;
+        const int kb1 = min(kblocks, kb0 + kps);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) {
             ok = false;
             break;
@@ -293,8 +336,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                          : smem_desc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t b_desc = B_MN ? smem_desc_sw128(b_base + kk * 4096, 16384, 1024)
                                          : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            if constexpr (F16) mma_bf16(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
-            else mma_i8(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (F16) mma_bf16(d_tmem, a_desc, b_desc, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+            else mma_i8(d_tmem, a_desc, b_desc, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
           }
           mma_commit(empty0 + 8 * stage);
           if (++stage == STAGES) {
@@ -318,10 +361,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       int tm, tn;
-        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
+      const int sp = t / per_split;
+      tile_coords(t - sp * per_split, tiles_m, tiles_n, group, tm, tn);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile<OutT, HB, F16>(ep, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
+      Epi eps = ep;
+      eps.out = reinterpret_cast<OutT*>(ep.out) + sp * ep.split_stride;
+      if constexpr (std::is_same<OutT, int32_t>::value)
+        epilogue_tile_raw(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
+      else
+        epilogue_tile<OutT, HB, F16>(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -358,7 +407,7 @@ template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int tiles_m, int tiles_n,
-                        int kblocks, int group, Epi ep, int32_t* status) {
+                        int kblocks, int kps, int group, Epi ep, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -405,7 +454,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = tiles_m * tiles_n;
+  // Contraction splits of kps k-blocks each (one split unless the
+  // contraction exceeds the int32-safe length); tile t is split t / per_split.
+  const int per_split = tiles_m * tiles_n;
+  const int num_tiles = per_split * ((kblocks + kps - 1) / kps);
   const uint32_t lead_full0 = mapa_shared(full0, 0);
   const uint32_t lead_tempty0 = mapa_shared(tempty0, 0);
 
@@ -416,10 +468,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += npairs) {
         int tm, tn;
-        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
+        const int sp = t / per_split;
+        tile_coords(t - sp * per_split, tiles_m, tiles_n, group, tm, tn);
         const int a_row = tm * 256 + static_cast<int>(rank) * 128;
         const int b_col = tn * 256 + static_cast<int>(rank) * 128;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int kb1 = min(kblocks, (sp + 1) * kps);
+        for (int kb = sp * kps; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -462,7 +516,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int kb0 = (t / per_split) * kps;
+        const int kb1 = min(kblocks, kb0 + kps);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag)) {
             ok = false;
             break;
@@ -476,8 +532,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                          : smem_desc_sw128(a_base + kk * 32, 16, 1024);
             const uint64_t b_desc = B_MN ? smem_desc_sw128(b_base + kk * 4096, 16384, 1024)
                                          : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            if constexpr (F16) mma_bf16_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
-            else mma_i8_pair(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (F16) mma_bf16_pair(d_tmem, a_desc, b_desc, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+            else mma_i8_pair(d_tmem, a_desc, b_desc, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
           }
           mma_commit_pair_mc(empty0 + 8 * stage, 0x3);
           if (++stage == PSTAGES) {
@@ -500,11 +556,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int t = pair; t < num_tiles; t += npairs) {
       int tm, tn;
-        tile_coords(t, tiles_m, tiles_n, group, tm, tn);
+      const int sp = t / per_split;
+      tile_coords(t - sp * per_split, tiles_m, tiles_n, group, tm, tn);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag)) break;
       tc_fence_after();
-      epilogue_tile<OutT, HB, F16>(ep, tmem_base + acc * BN, quarter, lane,
-                              tm * 256 + static_cast<int>(rank) * 128, tn * BN);
+      Epi eps = ep;
+      eps.out = reinterpret_cast<OutT*>(ep.out) + sp * ep.split_stride;
+      if constexpr (std::is_same<OutT, int32_t>::value)
+        epilogue_tile_raw(eps, tmem_base + acc * BN, quarter, lane,
+                          tm * 256 + static_cast<int>(rank) * 128, tn * BN);
+      else
+        epilogue_tile<OutT, HB, F16>(eps, tmem_base + acc * BN, quarter, lane,
+                                     tm * 256 + static_cast<int>(rank) * 128, tn * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead_tempty0 + 8 * acc);
@@ -576,7 +639,7 @@ int pair_slots(K kern) {
 
 template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
-                     int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
+                     int kblocks, int kps, const Epi& ep, int32_t* status, cudaStream_t s) {
   auto kern = gemm_i8_pair_kernel<A_MN, B_MN, OutT, HB, F16>;
   static int configured[64] = {0};
   int dev = 0;
@@ -586,13 +649,13 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
     if (e != cudaSuccess) return e;
     __atomic_store_n(&configured[dev], 1, __ATOMIC_RELEASE);
   }
-  const int tiles = tiles_m * tiles_n;
+  const int tiles = tiles_m * tiles_n * ((kblocks + kps - 1) / kps);
   const int slots = pair_slots(kern);
   const int pairs = tiles < slots ? tiles : slots;
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
-  kern<<<2 * pairs, NUM_THREADS, PSMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, A_MN ? 8 : 1,
+  kern<<<2 * pairs, NUM_THREADS, PSMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1,
                                                     ep, status);
   cudaError_t e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
@@ -602,7 +665,7 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
 
 template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
-                int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
+                int kblocks, int kps, const Epi& ep, int32_t* status, cudaStream_t s) {
   auto kern = gemm_i8_kernel<A_MN, B_MN, OutT, HB, F16>;
   // Opt in to the large dynamic shared memory once per device.
   static int configured[64] = {0};
@@ -613,13 +676,13 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
     if (e != cudaSuccess) return e;
     __atomic_store_n(&configured[dev], 1, __ATOMIC_RELEASE);
   }
-  const int tiles = tiles_m * tiles_n;
+  const int tiles = tiles_m * tiles_n * ((kblocks + kps - 1) / kps);
   const int sms = device_info().sms;
   const int grid = tiles < sms ? tiles : sms;
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, A_MN ? 8 : 1, ep,
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1, ep,
                                               status);
   cudaError_t e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
@@ -629,9 +692,10 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
 
 template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t go(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
-               int kblocks, const Epi& ep, int32_t* status, cudaStream_t s) {
-  if (pair) return run_pair<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
-  return run<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+               int kblocks, const Epi& ep, int32_t* status, cudaStream_t s, int kps = 0) {
+  if (kps <= 0) kps = kblocks;
+  if (pair) return run_pair<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, kps, ep, status, s);
+  return run<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, kps, ep, status, s);
 }
 
 cudaError_t dispatch_dx(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m,
@@ -700,6 +764,7 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
   Epi ep;
   ep.out = e.out;
   ep.ldo = e.ldo;
+  ep.split_stride = 0;
   ep.rows = static_cast<int>(rows);
   ep.cols = static_cast<int>(cols);
   ep.row_scale = e.row_scale;
@@ -740,6 +805,7 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
   Epi ep;
   ep.out = e.out;
   ep.ldo = e.ldo;
+  ep.split_stride = 0;
   ep.rows = static_cast<int>(rows);
   ep.cols = static_cast<int>(cols);
   ep.row_scale = e.row_scale;
@@ -754,6 +820,99 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
   if (e.out_bf16)
     return go<false, false, __nv_bfloat16, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
   return go<false, false, float, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+}
+
+// ------------------------------------------------------------------ long contractions
+// Sum of the int32 partial products of every split in int64, then the
+// epilogue of launch_gemm_i8: ((float)acc * row_scale) * col_scale + bias.
+// One thread per 4 consecutive outputs.
+template <typename OutT>
+__global__ void __launch_bounds__(256) combine_splits_kernel(
+    const int32_t* __restrict__ parts, int splits, int64_t split_stride, int64_t rows, int cols,
+    const float* __restrict__ row_scale, const float* __restrict__ col_scale,
+    const float* __restrict__ bias, OutT* __restrict__ out, int64_t ldo) {
+  const int64_t quads = rows * (cols / 4);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < quads;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / (cols / 4);
+    const int c = static_cast<int>(i - r * (cols / 4)) * 4;
+    long long acc[4] = {0, 0, 0, 0};
+    for (int sp = 0; sp < splits; ++sp) {
+      const int4 p = __ldcs(reinterpret_cast<const int4*>(parts + sp * split_stride + r * cols + c));
+      acc[0] += p.x;
+      acc[1] += p.y;
+      acc[2] += p.z;
+      acc[3] += p.w;
+    }
+    const float rs = row_scale ? row_scale[r] : 1.0f;
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[e] = __ll2float_rn(acc[e]) * rs;
+      if (col_scale) v[e] = v[e] * col_scale[c + e];
+      if (bias) v[e] = v[e] + bias[c + e];
+    }
+    OutT* o = out + r * ldo + c;
+    if constexpr (sizeof(OutT) == 4) {
+      *reinterpret_cast<float4*>(o) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+      *reinterpret_cast<uint2*>(o) = make_uint2(bf16x2(v[0], v[1]), bf16x2(v[2], v[3]));
+    }
+  }
+}
+
+int contraction_splits(int64_t kc) {
+  const int64_t kblocks = (kc + BK - 1) / BK;
+  return static_cast<int>((kblocks + kMaxSplitBlocks - 1) / kMaxSplitBlocks);
+}
+
+cudaError_t launch_gemm_i8_long(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
+                                int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
+                                int32_t* parts, const GemmEpilogue& e, int32_t* status,
+                                cudaStream_t s) {
+  // The contraction in splits of at most kMaxSplitBlocks * 128 = 130,944
+  // elements, each written as raw int32 partial sums [split][rows][cols];
+  // then one pass sums the splits in int64 and applies the epilogue.
+  if (e.hb != 0 || cols % 16 != 0) return cudaErrorInvalidValue;
+  const bool pair = rows > BM;
+  CUtensorMap ta, tb;
+  const bool ok_a = a_mn ? make_tmap(&ta, A, rows, kc, lda, 128, BK)
+                         : make_tmap(&ta, A, kc, rows, lda, BK, BM);
+  const bool ok_b = b_mn ? make_tmap(&tb, B, cols, kc, ldb, 128, BK)
+                         : make_tmap(&tb, B, kc, cols, ldb, BK, pair ? 128 : BN);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+  Epi ep{};
+  ep.out = parts;
+  ep.ldo = cols;
+  ep.split_stride = rows * cols;
+  ep.rows = static_cast<int>(rows);
+  ep.cols = static_cast<int>(cols);
+  const int tile_rows = pair ? 2 * BM : BM;
+  const int tiles_m = static_cast<int>((rows + tile_rows - 1) / tile_rows);
+  const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
+  const int kblocks = static_cast<int>((kc + BK - 1) / BK);
+  const int splits = contraction_splits(kc);
+  const int kps = (kblocks + splits - 1) / splits;
+  cudaError_t err;
+  if (!a_mn && b_mn)
+    err = go<false, true, int32_t, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s, kps);
+  else if (a_mn && b_mn)
+    err = go<true, true, int32_t, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s, kps);
+  else
+    return cudaErrorInvalidValue;
+  if (err != cudaSuccess) return err;
+  const int64_t quads = rows * (cols / 4);
+  const int grid = static_cast<int>(std::min<int64_t>((quads + 255) / 256, device_info().sms * 8));
+  if (e.out_bf16)
+    combine_splits_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        parts, splits, rows * cols, rows, static_cast<int>(cols), e.row_scale, e.col_scale, e.bias,
+        reinterpret_cast<__nv_bfloat16*>(e.out), e.ldo);
+  else
+    combine_splits_kernel<float><<<grid, 256, 0, s>>>(
+        parts, splits, rows * cols, rows, static_cast<int>(cols), e.row_scale, e.col_scale, e.bias,
+        reinterpret_cast<float*>(e.out), e.ldo);
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 }  // namespace ql

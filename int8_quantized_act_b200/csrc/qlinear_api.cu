@@ -7,6 +7,8 @@
 #include <cstdint>
 #include <mutex>
 
+#include <algorithm>
+
 #include "launch.h"
 #include "../../include/qlinear.h"
 
@@ -76,20 +78,28 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 // Workspace carve-up shared by the two backward calls.
 struct WsLayout {
-  size_t dyq, s1, colmax, s2, inv2, colsum, dxtmp, total;
+  size_t dyq, s1, colmax, s2, inv2, colsum, dxtmp, parts, total;
 };
 
+// Contractions longer than the int32-safe 131,071 (the input gradient's over
+// N output classes, the weight gradient's over M tokens) run in splits whose
+// int32 partial sums wait in `parts` to be combined in int64.
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int B) {
   WsLayout L;
+  const size_t m = static_cast<size_t>(M), n = static_cast<size_t>(N), k = static_cast<size_t>(K);
+  const size_t dx_splits = N > QL_MAX_CONTRACTION ? ql::contraction_splits(N) : 0;
+  const size_t dw_splits = M > QL_MAX_CONTRACTION ? ql::contraction_splits(M) : 0;
   size_t off = 0;
-  L.dyq = off;    off += align256(static_cast<size_t>(M) * static_cast<size_t>(N));
-  L.s1 = off;     off += align256(4 * static_cast<size_t>(M > 0 ? M : 1));
-  L.colmax = off; off += align256(4 * static_cast<size_t>(N > 0 ? N : 1));
-  L.s2 = off;     off += align256(4 * static_cast<size_t>(N > 0 ? N : 1));
-  L.inv2 = off;   off += align256(4 * static_cast<size_t>(N > 0 ? N : 1));
-  L.colsum = off; off += align256(8 * static_cast<size_t>(N > 0 ? N : 1));
+  L.dyq = off;    off += align256(m * n);
+  L.s1 = off;     off += align256(4 * (M > 0 ? m : 1));
+  L.colmax = off; off += align256(4 * (N > 0 ? n : 1));
+  L.s2 = off;     off += align256(4 * (N > 0 ? n : 1));
+  L.inv2 = off;   off += align256(4 * (N > 0 ? n : 1));
+  L.colsum = off; off += align256(8 * (N > 0 ? n : 1));
   L.dxtmp = off;
-  if (B > 128) off += align256(4 * static_cast<size_t>(M) * static_cast<size_t>(K));
+  if (B > 128 || (dx_splits > 0 && B > 0)) off += align256(4 * m * k);
+  L.parts = off;
+  off += align256(4 * std::max(dx_splits * m * k, dw_splits * n * k));
   L.total = off;
   return L;
 }
@@ -97,6 +107,49 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int B) {
 template <typename T>
 T* at(void* base, size_t off) {
   return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(base) + off);
+}
+
+// The input-gradient product from the row-quantized dY: dX = s1[m] *
+// (dyq_r W_q), times R when B > 0 (fused into the GEMM epilogue for B <= 128;
+// a second pass over a float32 product for B = 256 and for split contractions).
+int run_dx_product(const int8_t* dyq_r, const int8_t* wq, const float* s1, int64_t M, int64_t N,
+                   int64_t K, int B, void* dx, int dxt, void* ws, const WsLayout& L,
+                   int32_t* status, cudaStream_t s) {
+  GemmEpilogue ep;
+  ep.row_scale = s1;
+  ep.ldo = K;
+  const bool split = N > QL_MAX_CONTRACTION;
+  int32_t* parts = at<int32_t>(ws, L.parts);
+  if (B > 128 || (split && B > 0)) {
+    float* tmp = dxt == QL_F32 ? reinterpret_cast<float*>(dx) : at<float>(ws, L.dxtmp);
+    ep.out = tmp;
+    cudaError_t e = split ? ql::launch_gemm_i8_long(dyq_r, false, N, wq, true, K, M, K, N, parts, ep, status, s)
+                          : ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ep, status, s);
+    if (e != cudaSuccess) return QL_ERR_CUDA;
+    return cuda_status(ql::launch_hadamard(tmp, QL_F32, K, dx, dxt, K, M, K, B, hadamard_c(B), s));
+  }
+  ep.out = dx;
+  ep.out_bf16 = dxt == QL_BF16;
+  if (split)
+    return cuda_status(ql::launch_gemm_i8_long(dyq_r, false, N, wq, true, K, M, K, N, parts, ep, status, s));
+  ep.hb = B;
+  ep.hc = hadamard_c(B);
+  return cuda_status(ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ep, status, s));
+}
+
+// The weight-gradient product from the column-quantized dY: dW = s2[n] *
+// (dyq_c^T X_q), the contraction over the M tokens.
+int run_dw_product(const int8_t* dyq_c, const int8_t* xq, const float* s2, int64_t M, int64_t N,
+                   int64_t K, float* dw, void* ws, const WsLayout& L, int32_t* status,
+                   cudaStream_t s) {
+  GemmEpilogue ep;
+  ep.out = dw;
+  ep.ldo = K;
+  ep.row_scale = s2;
+  if (M > QL_MAX_CONTRACTION)
+    return cuda_status(ql::launch_gemm_i8_long(dyq_c, true, N, xq, true, K, N, K, M,
+                                               at<int32_t>(ws, L.parts), ep, status, s));
+  return cuda_status(ql::launch_gemm_i8(dyq_c, true, N, xq, true, K, N, K, M, ep, status, s));
 }
 
 }  // namespace
@@ -280,7 +333,6 @@ int qlinear_bwd_dx(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
       K > INT32_MAX)
     return QL_ERR_SHAPE;
   if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
-  if (N > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
   if (M == 0 || K == 0) return QL_OK;
   const WsLayout L = ws_layout(M, N, K, hadamard_block);
   if (!dx || !d_status || !ws || (N > 0 && (!dy || !wq || !sw))) return QL_ERR_ARG;
@@ -296,25 +348,7 @@ int qlinear_bwd_dx(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   float* s1 = at<float>(ws, L.s1);
   cudaError_t e = ql::launch_quant_rows(dy, dyt, M, N, N, sw, 0, 1.0f, 0u, dyq, N, s1, d_status, s);
   if (e != cudaSuccess) return QL_ERR_CUDA;
-  GemmEpilogue ep;
-  ep.row_scale = s1;
-  ep.ldo = K;
-  if (hadamard_block > 128) {
-    // Blocks wider than a thread's register chunk: write the float32 product
-    // (to dx itself when it is float32) and rotate it in a second pass.
-    float* tmp = dxt == QL_F32 ? reinterpret_cast<float*>(dx) : at<float>(ws, L.dxtmp);
-    ep.out = tmp;
-    ep.out_bf16 = 0;
-    e = ql::launch_gemm_i8(dyq, false, N, wq, true, K, M, K, N, ep, d_status, s);
-    if (e != cudaSuccess) return QL_ERR_CUDA;
-    return cuda_status(ql::launch_hadamard(tmp, QL_F32, K, dx, dxt, K, M, K, hadamard_block,
-                                           hadamard_c(hadamard_block), s));
-  }
-  ep.out = dx;
-  ep.out_bf16 = dxt == QL_BF16;
-  ep.hb = hadamard_block;
-  ep.hc = hadamard_c(hadamard_block);
-  return cuda_status(ql::launch_gemm_i8(dyq, false, N, wq, true, K, M, K, N, ep, d_status, s));
+  return run_dx_product(dyq, wq, s1, M, N, K, hadamard_block, dx, dxt, ws, L, d_status, s);
 }
 
 int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* xq,
@@ -323,7 +357,6 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   if (!valid_dtype(dyt)) return QL_ERR_ARG;
   if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || N > INT32_MAX || K > INT32_MAX)
     return QL_ERR_SHAPE;
-  if (M > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
   if (N == 0) return QL_OK;
   const WsLayout L = ws_layout(M, N, K, 0);
   if (!d_status || !ws || (K > 0 && !dw) || (M > 0 && (!dy || !xq || !sx))) return QL_ERR_ARG;
@@ -353,11 +386,7 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   if (e == cudaSuccess)
     e = ql::launch_dualquant(dy, dyt, M, N, nullptr, nullptr, sx, inv2, nullptr, dyq, d_status, s);
   if (e != cudaSuccess || K == 0) return cuda_status(e);
-  GemmEpilogue ep;
-  ep.out = dw;
-  ep.ldo = K;
-  ep.row_scale = s2;
-  return cuda_status(ql::launch_gemm_i8(dyq, true, N, xq, true, K, N, K, M, ep, d_status, s));
+  return run_dw_product(dyq, xq, s2, M, N, K, dw, ws, L, d_status, s);
 }
 
 // qlinear_bwd's workspace: the common layout, then the column-quantized
@@ -381,7 +410,6 @@ int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
       N > INT32_MAX || K > INT32_MAX)
     return QL_ERR_SHAPE;
   if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
-  if (N > QL_MAX_CONTRACTION || M > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
   const WsLayout L = ws_layout(M, N, K, hadamard_block);
   const size_t need = L.total + bwd_extra(M, N);
   if (!d_status || !ws) return QL_ERR_ARG;
@@ -423,31 +451,11 @@ int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
   if (e == cudaSuccess)
     e = ql::launch_dualquant(dy, dyt, M, N, sw, inv1, sx, inv2, dyq_r, dyq_c, d_status, s);
   if (e != cudaSuccess) return QL_ERR_CUDA;
-  // Input gradient (as qlinear_bwd_dx after its quantization).
-  GemmEpilogue ex;
-  ex.row_scale = s1;
-  ex.ldo = K;
-  if (hadamard_block > 128) {
-    float* tmp = dxt == QL_F32 ? reinterpret_cast<float*>(dx) : at<float>(ws, L.dxtmp);
-    ex.out = tmp;
-    e = ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ex, d_status, s);
-    if (e == cudaSuccess)
-      e = ql::launch_hadamard(tmp, QL_F32, K, dx, dxt, K, M, K, hadamard_block,
-                              hadamard_c(hadamard_block), s);
-  } else {
-    ex.out = dx;
-    ex.out_bf16 = dxt == QL_BF16;
-    ex.hb = hadamard_block;
-    ex.hc = hadamard_c(hadamard_block);
-    e = ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ex, d_status, s);
-  }
-  if (e != cudaSuccess) return QL_ERR_CUDA;
-  // Weight gradient (as qlinear_bwd_dw after its quantization).
-  GemmEpilogue ew;
-  ew.out = dw;
-  ew.ldo = K;
-  ew.row_scale = s2;
-  return cuda_status(ql::launch_gemm_i8(dyq_c, true, N, xq, true, K, N, K, M, ew, d_status, s));
+  // Input gradient (as qlinear_bwd_dx after its quantization), then weight
+  // gradient (as qlinear_bwd_dw after its quantization).
+  const int r = run_dx_product(dyq_r, wq, s1, M, N, K, hadamard_block, dx, dxt, ws, L, d_status, s);
+  if (r != QL_OK) return r;
+  return run_dw_product(dyq_c, xq, s2, M, N, K, dw, ws, L, d_status, s);
 }
 
 int qweight_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,

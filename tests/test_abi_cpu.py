@@ -66,6 +66,22 @@ def fake(addr):
     return P(addr)
 
 
+def test_workspace_grows_by_the_int32_partials_of_long_contractions(L):
+    def a(x):
+        return (x + 255) // 256 * 256
+    limit = ql.QL_MAX_CONTRACTION
+    # 1023 blocks of 128 per split: 131,072 -> 2 splits, 400,000 -> 4
+    M, K = 8, 256
+    for N, splits in ((limit + 1, 2), (400000, 4)):
+        base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+        assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * splits * M * K)
+        # rotated: the float32 product waits for its second pass
+        assert ql.qlinear_workspace_bytes(M, N, K, 128) == base + a(4 * M * K) + a(4 * splits * M * K)
+    M, N = 262144, 48          # 2048 blocks -> 3 splits over the tokens
+    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 3 * N * K)
+
+
 def test_bwd_workspace_formula(L):
     def a(x):
         return (x + 255) // 256 * 256
@@ -97,8 +113,11 @@ def test_host_validation_returns_before_any_launch(L):
     assert L.qlinear_fwd(fake(A), 0, 2, 32, fake(A), fake(A), 32, fake(A + 8), 0, fake(A), 0, fake(A), fake(A), fake(A), None) == ql.QL_ERR_ALIGN
     # backward: workspace too small, contraction limit
     assert L.qlinear_bwd_dx(fake(A), 0, 4, 32, fake(A), fake(A), 32, 0, fake(A), 0, fake(0x100000), 16, fake(A), None) == ql.QL_ERR_SHAPE
-    assert L.qlinear_bwd_dx(fake(A), 0, 4, big, fake(A), fake(A), 32, 0, fake(A), 0, fake(A), 1 << 30, fake(A), None) == ql.QL_ERR_UNSUPPORTED
-    assert L.qlinear_bwd_dw(fake(A), 0, big, 32, fake(A), fake(A), 32, fake(A), None, fake(A), 1 << 30, fake(A), None) == ql.QL_ERR_UNSUPPORTED
+    # long backward contractions need the larger workspace of their splits
+    need = ql.qlinear_workspace_bytes(4, big, 32, 0)
+    assert L.qlinear_bwd_dx(fake(A), 0, 4, big, fake(A), fake(A), 32, 0, fake(A), 0, fake(A), need - 256, fake(A), None) == ql.QL_ERR_SHAPE
+    need = ql.qlinear_workspace_bytes(big, 32, 32, 0)
+    assert L.qlinear_bwd_dw(fake(A), 0, big, 32, fake(A), fake(A), 32, fake(A), None, fake(A), need - 256, fake(A), None) == ql.QL_ERR_SHAPE
     assert L.qlinear_bwd_dw(fake(A), 0, 4, 32, fake(A), fake(A), 32, fake(A), None, fake(A + 16), 1 << 30, fake(A), None) == ql.QL_ERR_ALIGN
     # hadamard: in place needs the same dtype and pitch
     assert L.qlinear_hadamard(fake(A), 0, 32, fake(A), 1, 32, 4, 32, 16, None) == ql.QL_ERR_ARG
