@@ -44,17 +44,28 @@ NOMINAL_INT8_OVER_BF16 = 2.0   # dense int8 4.5 POPS / dense bf16 2.25 PFLOPS
 # DRAM bytes (read + write) per GEMM launch from the ncu capture summarised in
 # profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
-GEMM_TRAFFIC_BYTES = 369.1e6
-GEMM_TRAFFIC_SOURCE_SHA = "76383a85d156eebd"
+GEMM_TRAFFIC_BYTES = 368.8e6
+GEMM_TRAFFIC_SOURCE_SHA = "eac99f824e7968ac"
+# The same for the update kernel (profiles/update_sr_staged_N7168_K5376.md);
+# DRAM writes still held in L2 when the kernel ends are not counted.
+UPDATE_TRAFFIC_BYTES = 790.3e6
+UPDATE_TRAFFIC_SOURCE_SHA = "698dbcc8523edb2b"
 
 
-def gemm_source_sha():
+def source_sha(files=("gemm_i8.cu", "sm100.cuh")):
     import hashlib
     h = hashlib.sha256()
-    for f in ("gemm_i8.cu", "sm100.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "int8_quantized_act_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def gemm_source_sha():
+    return source_sha()
+
+
+UPDATE_SOURCES = ("update_sr.cu", "rowops.cuh", "sm100.cuh")
 
 
 def parse_args():
@@ -372,7 +383,10 @@ def run_ours(args, rank, world, local):
                        "achieved": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9, 1),
                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
                        "frac": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                       "ms_per_launch": round(upd_ms, 4)},
+                       "ms_per_launch": round(upd_ms, 4),
+                       "traffic": (UPDATE_TRAFFIC_BYTES if source_sha(UPDATE_SOURCES) == UPDATE_TRAFFIC_SOURCE_SHA
+                                   else None),
+                       "traffic_unit": "bytes per launch"},
         "e2e": {"value": round(job_tops(world, 1, e2e_ms), 2), "unit": "TOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
