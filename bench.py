@@ -79,6 +79,9 @@ def parse_args():
     p.add_argument("--routes", action="store_true",
                    help="instead of the train step: time the forward's int8 and bf16 routes "
                         "at 2048 and 12000 tokens (one JSON line)")
+    p.add_argument("--edge", action="store_true",
+                   help="instead of the train step: time the layer's calls at 1..128 tokens, "
+                        "where the weight stream bounds the forward (one JSON line)")
     return p.parse_args()
 
 
@@ -547,8 +550,114 @@ def run_routes(args):
     return out
 
 
+def run_edge(args):
+    """The 5376 -> 7168 layer (block 128, bf16) at 1, 4, 15, 16, 17, 64 and 128
+    tokens: forward, input gradient and weight gradient, whole call and GEMM
+    alone (CUDA events around single calls, medians; these include the host's
+    launch latency), and the device time per call with 20 calls captured in
+    a CUDA graph.  Below a GEMM's row floor the forward reads the 38.5 MB int8
+    weight once per call, so its bound is that read."""
+    import torch
+    import int8_quantized_act_b200 as ql
+    import workloads
+    torch.cuda.set_device(0)
+    peaks = load_peaks()
+    d = workloads.rotated_layer(M=128, seed=1)
+    dev = "cuda"
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    wq = torch.empty((N_OUT, K_IN), dtype=torch.int8, device=dev)
+    sw = torch.empty(N_OUT, device=dev)
+    ql.qlinear_quantize_rows(torch.from_numpy(d["w"]).to(dev), wq, sw, st, hadamard_block=BLOCK,
+                             flags=ql.QL_REJECT_ZERO_ROWS)
+    bias = torch.from_numpy(d["bias"]).to(dev)
+    x_all, dy_all = d["x_bf16"].to(dev), d["dy_bf16"].to(dev)
+    w_bytes = N_OUT * K_IN
+    out = {"metric": "layer call time at small token counts (us per call)", "unit": "us",
+           "higher_is_better": False, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+           "data": "synthetic",
+           "config": {"workload": "5376 -> 7168 layer, Hadamard block 128, bf16 x, dY, y, dX",
+                      "K": K_IN, "N": N_OUT, "weight_bytes": w_bytes,
+                      "hbm_peak_gbs": peaks["hbm_gbs"]},
+           "tokens": {}}
+
+    def timed(fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        gev = [tuple(new_events(2)) for _ in range(args.steps)]
+        for _ in range(args.warmup):
+            fn(None)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            ev[i][0].record()
+            fn(gev[i])
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return (statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3,
+                statistics.median(a.elapsed_time(b) for a, b in gev) * 1e3)
+
+    def graph_us(call, reps=20):
+        """Device time per call with the host out of the way: `reps` calls
+        captured in one CUDA graph, replayed after a warm-up."""
+        call()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                call()
+        for _ in range(args.warmup):
+            g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(args.steps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3 / (args.steps * reps)
+
+    for M in (1, 4, 15, 16, 17, 64, 128):
+        x, dy = x_all[:M].contiguous(), dy_all[:M].contiguous()
+        y = torch.empty((M, N_OUT), dtype=torch.bfloat16, device=dev)
+        xq = torch.empty((M, K_IN), dtype=torch.int8, device=dev)
+        sx = torch.empty(M, device=dev)
+        dx = torch.empty((M, K_IN), dtype=torch.bfloat16, device=dev)
+        dw = torch.empty((N_OUT, K_IN), device=dev)
+        db = torch.empty(N_OUT, device=dev)
+        ws = torch.empty(ql.qlinear_workspace_bytes(M, N_OUT, K_IN, BLOCK), dtype=torch.uint8,
+                         device=dev)
+
+        def with_events(call):
+            def f(g):
+                ql.ql_set_gemm_timing_events([g] if g else ())
+                call()
+                ql.ql_set_gemm_timing_events(())
+            return f
+
+        calls = {
+            "fwd": lambda: ql.qlinear_fwd(x, wq, sw, bias, BLOCK, y, xq, sx, st),
+            "dx": lambda: ql.qlinear_bwd_dx(dy, wq, sw, BLOCK, dx, ws, st),
+            "dw": lambda: ql.qlinear_bwd_dw(dy, xq, sx, dw, db, ws, st),
+        }
+        row = {}
+        for name, call in calls.items():
+            t_call, t_gemm = timed(with_events(call))
+            row[f"{name}_us"] = round(t_call, 2)
+            row[f"{name}_gemm_us"] = round(t_gemm, 2)
+            row[f"{name}_graph_us"] = round(graph_us(call), 2)
+        row["fwd_graph_weight_gbs"] = round(w_bytes / (row["fwd_graph_us"] * 1e-6) / 1e9, 1)
+        row["dx_graph_weight_gbs"] = round(w_bytes / (row["dx_graph_us"] * 1e-6) / 1e9, 1)
+        row["dw_graph_output_gbs"] = round(4 * w_bytes / (row["dw_graph_us"] * 1e-6) / 1e9, 1)
+        out["tokens"][str(M)] = row
+    if int(st.item()):
+        raise RuntimeError(f"device status {ql.status_flags(int(st.item()))}")
+    return out
+
+
 def main():
     args = parse_args()
+    if args.edge:
+        print(json.dumps(run_edge(args)), flush=True)
+        return
     if args.routes:
         print(json.dumps(run_routes(args)), flush=True)
         return

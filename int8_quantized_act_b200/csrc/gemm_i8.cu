@@ -42,6 +42,8 @@ constexpr int STAGES = 4;
 // Longest int32-safe contraction split in 128-element blocks: 1023 * 128 =
 // 130,944 <= 131,071 = floor((2^31 - 1) / 128^2).
 constexpr int64_t kMaxSplitBlocks = 1023;
+// Most contraction splits used to spread a small (<= 128-row) output.
+constexpr int64_t kMaxSmallSplits = QL_SMALL_OUTPUT_SPLITS;
 constexpr int A_BYTES = BM * BK;       // 16 KiB
 constexpr int B_BYTES = BN * BK;       // 32 KiB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -49,6 +51,21 @@ constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;      // 512: the whole TMEM of the SM
 constexpr int NUM_BARS = 2 * STAGES + 5;
 constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+
+// The single-CTA kernel's tile width: 256 columns, or 64 for outputs of one
+// 128-row slab whose 256-wide tiles would leave most SMs idle (the forward at
+// a few tokens streams the whole weight through few CTAs otherwise); the
+// narrower tile takes twice the stages to keep as many bytes in flight.
+template <int TBN>
+struct Single {
+  static constexpr int kBN = TBN;
+  static constexpr int kStages = TBN == 256 ? STAGES : 8;
+  static constexpr int kBBytes = TBN * BK;
+  static constexpr int kStageBytes = A_BYTES + kBBytes;
+  static constexpr int kTmemCols = 2 * TBN;  // two accumulators, a power of two >= 32
+  static constexpr int kNumBars = 2 * kStages + 5;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 8 * kNumBars + 16;
+};
 
 struct Epi {
   void* out;
@@ -127,7 +144,7 @@ __device__ __forceinline__ void store16(__nv_bfloat16* p, const float* v) {
 // + lane, columns col0 .. col0+255 of the output.  All 32 lanes of the warp
 // must call it (tcgen05.ld is warp-collective); rows/columns past the output
 // are computed but not stored.
-template <typename OutT, int HB, bool F16>
+template <typename OutT, int HB, bool F16, int TW = BN>
 __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, int quarter,
                                               int lane, int row0, int col0) {
   constexpr int CH = HB > 32 ? HB : 32;  // columns per register chunk
@@ -138,7 +155,7 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
   const float rs = (row_ok && ep.row_scale) ? ep.row_scale[gr] : 1.0f;
   const uint32_t taddr = acc_tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += CH) {
+  for (int c0 = 0; c0 < TW; c0 += CH) {
     uint32_t r[CH];
     tmem_ld_cols<CH>(taddr + c0, r);
     tmem_wait_ld();
@@ -186,6 +203,7 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
 
 // Raw int32 partial sums of one contraction split (no scaling), the same
 // slab as epilogue_tile.
+template <int TW = BN>
 __device__ __forceinline__ void epilogue_tile_raw(const Epi& ep, uint32_t acc_tmem, int quarter,
                                                   int lane, int row0, int col0) {
   int32_t* out = reinterpret_cast<int32_t*>(ep.out);
@@ -193,7 +211,7 @@ __device__ __forceinline__ void epilogue_tile_raw(const Epi& ep, uint32_t acc_tm
   const bool row_ok = gr < ep.rows;
   const uint32_t taddr = acc_tmem + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 32) {
+  for (int c0 = 0; c0 < TW; c0 += 32) {
     uint32_t r[32];
     tmem_ld_cols<32>(taddr + c0, r);
     tmem_wait_ld();
@@ -212,11 +230,15 @@ __device__ __forceinline__ void epilogue_tile_raw(const Epi& ep, uint32_t acc_tm
   }
 }
 
-template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16>
+template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16, int TBN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int tiles_m, int tiles_n, int kblocks, int kps, int group, Epi ep,
-                   int32_t* status) {
+                   int tiles_m, int tiles_n, int kblocks, int kps, int group, int a_box_rows,
+                   Epi ep, int32_t* status) {
+  using C = Single<TBN>;
+  static_assert(TBN == 256 || !B_MN, "narrow tiles read B K-major");
+  constexpr int BN = C::kBN, STAGES = C::kStages, B_BYTES = C::kBBytes;
+  constexpr int STAGE_BYTES = C::kStageBytes, TMEM_COLS = C::kTmemCols, NUM_BARS = C::kNumBars;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -283,7 +305,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          // A K-major output slab of fewer than 128 rows is loaded as a box of
+          // a_box_rows rows; the accumulator rows past it are never stored.
+          mbar_arrive_expect_tx(fb, STAGE_BYTES - (BM - a_box_rows) * BK);
           const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
           if (A_MN) tma_load_2d(a_dst, &tmA, fb, tm * BM, kb * BK);
@@ -368,9 +392,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       Epi eps = ep;
       eps.out = reinterpret_cast<OutT*>(ep.out) + sp * ep.split_stride;
       if constexpr (std::is_same<OutT, int32_t>::value)
-        epilogue_tile_raw(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
+        epilogue_tile_raw<BN>(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
       else
-        epilogue_tile<OutT, HB, F16>(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
+        epilogue_tile<OutT, HB, F16, BN>(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -586,6 +610,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   if (threadIdx.x == 0 && *abort_flag) atomicOr(status, 1 << QL_ERR_TIMEOUT);
 }
 
+// ------------------------------------------------------------------ a few rows
+// The forward at up to 4 tokens is a stream of the whole weight with at most
+// 4 multiply-adds per weight byte: a 128-row tensor-core tile would spend
+// its time on rows that do not exist.  One warp per weight row n: each lane
+// streams 16-byte pieces of the row (evict-first), multiplies them with the
+// same pieces of every token's codes (__dp4a: 4 int8 products into an int32
+// sum, exact), the warp adds its lanes' sums (redux.sync, exact), and lane m
+// writes y[m, n] = ((float)acc * row_scale[m]) * col_scale[n] + bias[n], the
+// epilogue of the tile kernel.
+template <int MT, typename OutT>
+__global__ void __launch_bounds__(256) gemv_i8_kernel(
+    const int8_t* __restrict__ xq, int64_t ldx, int M, const int8_t* __restrict__ wq,
+    int64_t ldw, int N, int K, const float* __restrict__ row_scale,
+    const float* __restrict__ col_scale, const float* __restrict__ bias, OutT* __restrict__ out,
+    int64_t ldo) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); n < N; n += nwarps) {
+    const int8_t* wrow = wq + n * ldw;
+    int acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0;
+#pragma unroll 4
+    for (int k0 = lane * 16; k0 < K; k0 += 512) {
+      const int4 w = __ldcs(reinterpret_cast<const int4*>(wrow + k0));
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        if (m < M) {
+          const int4 x = __ldg(reinterpret_cast<const int4*>(xq + m * ldx + k0));
+          acc[m] = __dp4a(w.x, x.x, acc[m]);
+          acc[m] = __dp4a(w.y, x.y, acc[m]);
+          acc[m] = __dp4a(w.z, x.z, acc[m]);
+          acc[m] = __dp4a(w.w, x.w, acc[m]);
+        }
+      }
+    }
+    int mine = 0;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const int t = __reduce_add_sync(0xFFFFFFFFu, acc[m]);
+      if (lane == m) mine = t;
+    }
+    if (lane < M) {
+      float v = __int2float_rn(mine) * (row_scale ? row_scale[lane] : 1.0f);
+      if (col_scale) v = v * col_scale[n];
+      if (bias) v = v + bias[n];
+      if constexpr (sizeof(OutT) == 4) out[lane * ldo + n] = v;
+      else out[lane * ldo + n] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+template <int MT>
+cudaError_t run_gemv(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, int64_t rows,
+                     int64_t cols, int64_t kc, const GemmEpilogue& e, cudaStream_t s) {
+  const int grid = static_cast<int>(std::min<int64_t>((cols + 7) / 8, device_info().sms * 8));
+  cudaEvent_t before = nullptr, after = nullptr;
+  gemm_timing_events(&before, &after);
+  if (before) cudaEventRecord(before, s);
+  if (e.out_bf16)
+    gemv_i8_kernel<MT, __nv_bfloat16><<<grid, 256, 0, s>>>(
+        A, lda, static_cast<int>(rows), B, ldb, static_cast<int>(cols), static_cast<int>(kc),
+        e.row_scale, e.col_scale, e.bias, reinterpret_cast<__nv_bfloat16*>(e.out), e.ldo);
+  else
+    gemv_i8_kernel<MT, float><<<grid, 256, 0, s>>>(
+        A, lda, static_cast<int>(rows), B, ldb, static_cast<int>(cols), static_cast<int>(kc),
+        e.row_scale, e.col_scale, e.bias, reinterpret_cast<float*>(e.out), e.ldo);
+  cudaError_t err = cudaGetLastError();
+  if (after) cudaEventRecord(after, s);
+  count_launches(1);
+  return err;
+}
+
 // ------------------------------------------------------------------ host
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -603,6 +700,12 @@ EncodeTiledFn encode_fn() {
     return reinterpret_cast<EncodeTiledFn>(p);
   }();
   return fn;
+}
+
+// Rows of the K-major A box: a slab of fewer than 128 output rows loads only
+// its rows (rounded up to 16) instead of a mostly zero-filled 128-row box.
+int a_box_rows(int64_t rows) {
+  return rows >= BM ? BM : static_cast<int>(std::max<int64_t>(16, (rows + 15) / 16 * 16));
 }
 
 // 2-D int8 tensor [outer][inner] with the given row pitch; boxes of
@@ -663,10 +766,11 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
   return e;
 }
 
-template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
+template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false, int TBN = 256>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
                 int kblocks, int kps, const Epi& ep, int32_t* status, cudaStream_t s) {
-  auto kern = gemm_i8_kernel<A_MN, B_MN, OutT, HB, F16>;
+  auto kern = gemm_i8_kernel<A_MN, B_MN, OutT, HB, F16, TBN>;
+  constexpr int SMEM_BYTES = Single<TBN>::kSmemBytes;
   // Opt in to the large dynamic shared memory once per device.
   static int configured[64] = {0};
   int dev = 0;
@@ -682,7 +786,8 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1, ep,
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1,
+                                              A_MN ? BM : a_box_rows(ep.rows), ep,
                                               status);
   cudaError_t e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
@@ -752,14 +857,27 @@ bool encode_tmap_2d(CUtensorMap* m, int elem_bytes, const void* base, uint64_t i
 cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
                            int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
                            const GemmEpilogue& e, int32_t* status, cudaStream_t s) {
+  // Up to 4 rows of K-major x K-major (the forward at a few tokens): one
+  // warp per output column on the CUDA cores, a single pass over B.  (Every
+  // row re-reads its piece of A per B row, so past a few rows the tensor-core
+  // tile is faster again.)
+  if (!a_mn && !b_mn && e.hb == 0 && rows <= 4 && kc % 16 == 0 && lda % 16 == 0 && ldb % 16 == 0) {
+    if (rows <= 1) return run_gemv<1>(A, lda, B, ldb, rows, cols, kc, e, s);
+    if (rows <= 2) return run_gemv<2>(A, lda, B, ldb, rows, cols, kc, e, s);
+    return run_gemv<4>(A, lda, B, ldb, rows, cols, kc, e, s);
+  }
   // Outputs with more than one 128-row slab run on CTA pairs (256x256
-  // tiles); smaller ones on single CTAs (128x256 tiles).
+  // tiles); smaller ones on single CTAs (128x256 tiles, or 128x64 when the
+  // wide tiles would occupy fewer than half the SMs: the forward at a few
+  // tokens is a stream of the whole weight and wants every SM on it).
   const bool pair = rows > BM;
+  const bool narrow = !pair && !a_mn && !b_mn && e.hb == 0 &&
+                      2 * ((cols + BN - 1) / BN) < device_info().sms;
   CUtensorMap ta, tb;
   const bool ok_a = a_mn ? make_tmap(&ta, A, rows, kc, lda, 128, BK)
-                         : make_tmap(&ta, A, kc, rows, lda, BK, BM);
+                         : make_tmap(&ta, A, kc, rows, lda, BK, pair ? BM : a_box_rows(rows));
   const bool ok_b = b_mn ? make_tmap(&tb, B, cols, kc, ldb, 128, BK)
-                         : make_tmap(&tb, B, kc, cols, ldb, BK, pair ? 128 : BN);
+                         : make_tmap(&tb, B, kc, cols, ldb, BK, pair ? 128 : narrow ? 64 : BN);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   Epi ep;
   ep.out = e.out;
@@ -779,6 +897,11 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
   // The layer's three products: forward (K-major x K-major), input gradient
   // (K-major x MN-major, optional fused rotation), weight gradient
   // (MN-major x MN-major, float32 out).
+  if (narrow) {
+    const int tn64 = static_cast<int>((cols + 63) / 64);
+    if (bf16) return run<false, false, __nv_bfloat16, 0, false, 64>(ta, tb, tiles_m, tn64, kblocks, kblocks, ep, status, s);
+    return run<false, false, float, 0, false, 64>(ta, tb, tiles_m, tn64, kblocks, kblocks, ep, status, s);
+  }
   if (!a_mn && !b_mn && e.hb == 0) {
     if (bf16) return go<false, false, __nv_bfloat16, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
     return go<false, false, float, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
@@ -796,11 +919,14 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
   // each kind::f16 MMA consumes K = 16 (32 bytes), the same byte layout as
   // the int8 path.
   const bool pair = rows > BM;
+  const bool narrow = !pair && 2 * ((cols + BN - 1) / BN) < device_info().sms;
   CUtensorMap ta, tb;
   const bool ok_a = encode_tmap_2d(&ta, 2, A, static_cast<uint64_t>(kc), static_cast<uint64_t>(rows),
-                                   static_cast<uint64_t>(lda) * 2, BK / 2, BM, true);
+                                   static_cast<uint64_t>(lda) * 2, BK / 2,
+                                   pair ? BM : a_box_rows(rows), true);
   const bool ok_b = encode_tmap_2d(&tb, 2, B, static_cast<uint64_t>(kc), static_cast<uint64_t>(cols),
-                                   static_cast<uint64_t>(ldb) * 2, BK / 2, pair ? 128 : BN, true);
+                                   static_cast<uint64_t>(ldb) * 2, BK / 2,
+                                   pair ? 128 : narrow ? 64 : BN, true);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   Epi ep;
   ep.out = e.out;
@@ -817,6 +943,12 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
   const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
   const int kblocks = static_cast<int>((kc + BK / 2 - 1) / (BK / 2));
   if (e.hb != 0) return cudaErrorInvalidValue;
+  if (narrow) {
+    const int tn64 = static_cast<int>((cols + 63) / 64);
+    if (e.out_bf16)
+      return run<false, false, __nv_bfloat16, 0, true, 64>(ta, tb, tiles_m, tn64, kblocks, kblocks, ep, status, s);
+    return run<false, false, float, 0, true, 64>(ta, tb, tiles_m, tn64, kblocks, kblocks, ep, status, s);
+  }
   if (e.out_bf16)
     return go<false, false, __nv_bfloat16, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
   return go<false, false, float, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
@@ -861,6 +993,16 @@ __global__ void __launch_bounds__(256) combine_splits_kernel(
   }
 }
 
+int small_output_splits(int64_t rows, int64_t cols, int64_t kc) {
+  // Splits that bring a one-slab output (rows <= 128) to about one wave.
+  if (rows > BM) return 1;
+  const int64_t tiles = (cols + BN - 1) / BN;
+  const int64_t kblocks = (kc + BK - 1) / BK;
+  int64_t sp = device_info().sms / tiles;
+  sp = std::min<int64_t>(std::min<int64_t>(sp, kMaxSmallSplits), kblocks / 4);
+  return static_cast<int>(std::max<int64_t>(sp, 1));
+}
+
 int contraction_splits(int64_t kc) {
   const int64_t kblocks = (kc + BK - 1) / BK;
   return static_cast<int>((kblocks + kMaxSplitBlocks - 1) / kMaxSplitBlocks);
@@ -868,16 +1010,17 @@ int contraction_splits(int64_t kc) {
 
 cudaError_t launch_gemm_i8_long(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
                                 int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
-                                int32_t* parts, const GemmEpilogue& e, int32_t* status,
-                                cudaStream_t s) {
+                                int32_t* parts, size_t parts_elems, const GemmEpilogue& e,
+                                int32_t* status, cudaStream_t s, int min_splits) {
   // The contraction in splits of at most kMaxSplitBlocks * 128 = 130,944
-  // elements, each written as raw int32 partial sums [split][rows][cols];
+  // elements (at least min_splits of them, to spread a small output over
+  // more SMs), each written as raw int32 partial sums [split][rows][cols];
   // then one pass sums the splits in int64 and applies the epilogue.
   if (e.hb != 0 || cols % 16 != 0) return cudaErrorInvalidValue;
   const bool pair = rows > BM;
   CUtensorMap ta, tb;
   const bool ok_a = a_mn ? make_tmap(&ta, A, rows, kc, lda, 128, BK)
-                         : make_tmap(&ta, A, kc, rows, lda, BK, BM);
+                         : make_tmap(&ta, A, kc, rows, lda, BK, pair ? BM : a_box_rows(rows));
   const bool ok_b = b_mn ? make_tmap(&tb, B, cols, kc, ldb, 128, BK)
                          : make_tmap(&tb, B, kc, cols, ldb, BK, pair ? 128 : BN);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
@@ -891,8 +1034,11 @@ cudaError_t launch_gemm_i8_long(const int8_t* A, bool a_mn, int64_t lda, const i
   const int tiles_m = static_cast<int>((rows + tile_rows - 1) / tile_rows);
   const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
   const int kblocks = static_cast<int>((kc + BK - 1) / BK);
-  const int splits = contraction_splits(kc);
+  const int splits = std::max(contraction_splits(kc), std::min(min_splits, kblocks));
   const int kps = (kblocks + splits - 1) / splits;
+  const int nsp = (kblocks + kps - 1) / kps;  // splits actually written
+  if (static_cast<size_t>(nsp) * static_cast<size_t>(rows) * static_cast<size_t>(cols) > parts_elems)
+    return cudaErrorInvalidValue;  // the partial sums would not fit
   cudaError_t err;
   if (!a_mn && b_mn)
     err = go<false, true, int32_t, 0>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s, kps);
@@ -905,11 +1051,11 @@ cudaError_t launch_gemm_i8_long(const int8_t* A, bool a_mn, int64_t lda, const i
   const int grid = static_cast<int>(std::min<int64_t>((quads + 255) / 256, device_info().sms * 8));
   if (e.out_bf16)
     combine_splits_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        parts, splits, rows * cols, rows, static_cast<int>(cols), e.row_scale, e.col_scale, e.bias,
+        parts, nsp, rows * cols, rows, static_cast<int>(cols), e.row_scale, e.col_scale, e.bias,
         reinterpret_cast<__nv_bfloat16*>(e.out), e.ldo);
   else
     combine_splits_kernel<float><<<grid, 256, 0, s>>>(
-        parts, splits, rows * cols, rows, static_cast<int>(cols), e.row_scale, e.col_scale, e.bias,
+        parts, nsp, rows * cols, rows, static_cast<int>(cols), e.row_scale, e.col_scale, e.bias,
         reinterpret_cast<float*>(e.out), e.ldo);
   count_launches(1);
   return cudaGetLastError();

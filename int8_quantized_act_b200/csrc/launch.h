@@ -92,14 +92,21 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
 
 // The same products for contractions longer than the int32-safe 131,071:
 // splits of at most 130,944 write raw int32 partial sums to `parts`
-// (contraction_splits(kc) * rows * cols int32, 16-byte aligned), then one pass
+// (splits * rows * cols int32, 16-byte aligned; parts_elems is its capacity,
+// checked before any launch), then one pass
 // sums them in int64 and applies ep (hb must be 0; cols % 16 == 0).  Input
 // gradient (K-major x MN-major) and weight gradient (MN-major x MN-major).
+// With min_splits > 1 the same path spreads an output of at most 128 rows
+// (one tile row) over more SMs: small_output_splits() gives the count, at
+// most QL_SMALL_OUTPUT_SPLITS, so the partial sums need at most that many
+// rows x cols int32 copies.
+#define QL_SMALL_OUTPUT_SPLITS 8
 int contraction_splits(int64_t kc);
+int small_output_splits(int64_t rows, int64_t cols, int64_t kc);
 cudaError_t launch_gemm_i8_long(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
                                 int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
-                                int32_t* parts, const GemmEpilogue& ep, int32_t* status,
-                                cudaStream_t s);
+                                int32_t* parts, size_t parts_elems, const GemmEpilogue& ep,
+                                int32_t* status, cudaStream_t s, int min_splits = 1);
 
 // The same GEMM on bf16 operands (tcgen05 kind::f16, float32 accumulator):
 // A [rows][kc] and B [cols][kc] both K-major bf16 with pitches lda, ldb

@@ -78,7 +78,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 // Workspace carve-up shared by the two backward calls.
 struct WsLayout {
-  size_t dyq, s1, colmax, s2, inv2, colsum, dxtmp, parts, total;
+  size_t dyq, s1, colmax, s2, inv2, colsum, dxtmp, parts, parts_elems, total;
 };
 
 // Contractions longer than the int32-safe 131,071 (the input gradient's over
@@ -87,8 +87,12 @@ struct WsLayout {
 WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int B) {
   WsLayout L;
   const size_t m = static_cast<size_t>(M), n = static_cast<size_t>(N), k = static_cast<size_t>(K);
-  const size_t dx_splits = N > QL_MAX_CONTRACTION ? ql::contraction_splits(N) : 0;
-  const size_t dw_splits = M > QL_MAX_CONTRACTION ? ql::contraction_splits(M) : 0;
+  // Outputs of at most 128 rows (few tokens for dX, few output features for
+  // dW) also run split, to spread over more SMs.
+  size_t dx_splits = N > QL_MAX_CONTRACTION ? ql::contraction_splits(N) : 0;
+  size_t dw_splits = M > QL_MAX_CONTRACTION ? ql::contraction_splits(M) : 0;
+  if (M <= 128) dx_splits = std::max<size_t>(dx_splits, QL_SMALL_OUTPUT_SPLITS);
+  if (N <= 128) dw_splits = std::max<size_t>(dw_splits, QL_SMALL_OUTPUT_SPLITS);
   size_t off = 0;
   L.dyq = off;    off += align256(m * n);
   L.s1 = off;     off += align256(4 * (M > 0 ? m : 1));
@@ -99,7 +103,8 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int B) {
   L.dxtmp = off;
   if (B > 128 || (dx_splits > 0 && B > 0)) off += align256(4 * m * k);
   L.parts = off;
-  off += align256(4 * std::max(dx_splits * m * k, dw_splits * n * k));
+  L.parts_elems = std::max(dx_splits * m * k, dw_splits * n * k);
+  off += align256(4 * L.parts_elems);
   L.total = off;
   return L;
 }
@@ -118,12 +123,13 @@ int run_dx_product(const int8_t* dyq_r, const int8_t* wq, const float* s1, int64
   GemmEpilogue ep;
   ep.row_scale = s1;
   ep.ldo = K;
-  const bool split = N > QL_MAX_CONTRACTION;
+  const int small = M <= 128 ? ql::small_output_splits(M, K, N) : 1;
+  const bool split = N > QL_MAX_CONTRACTION || small > 1;
   int32_t* parts = at<int32_t>(ws, L.parts);
   if (B > 128 || (split && B > 0)) {
     float* tmp = dxt == QL_F32 ? reinterpret_cast<float*>(dx) : at<float>(ws, L.dxtmp);
     ep.out = tmp;
-    cudaError_t e = split ? ql::launch_gemm_i8_long(dyq_r, false, N, wq, true, K, M, K, N, parts, ep, status, s)
+    cudaError_t e = split ? ql::launch_gemm_i8_long(dyq_r, false, N, wq, true, K, M, K, N, parts, L.parts_elems, ep, status, s, small)
                           : ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ep, status, s);
     if (e != cudaSuccess) return QL_ERR_CUDA;
     return cuda_status(ql::launch_hadamard(tmp, QL_F32, K, dx, dxt, K, M, K, B, hadamard_c(B), s));
@@ -131,7 +137,7 @@ int run_dx_product(const int8_t* dyq_r, const int8_t* wq, const float* s1, int64
   ep.out = dx;
   ep.out_bf16 = dxt == QL_BF16;
   if (split)
-    return cuda_status(ql::launch_gemm_i8_long(dyq_r, false, N, wq, true, K, M, K, N, parts, ep, status, s));
+    return cuda_status(ql::launch_gemm_i8_long(dyq_r, false, N, wq, true, K, M, K, N, parts, L.parts_elems, ep, status, s, small));
   ep.hb = B;
   ep.hc = hadamard_c(B);
   return cuda_status(ql::launch_gemm_i8(dyq_r, false, N, wq, true, K, M, K, N, ep, status, s));
@@ -146,9 +152,11 @@ int run_dw_product(const int8_t* dyq_c, const int8_t* xq, const float* s2, int64
   ep.out = dw;
   ep.ldo = K;
   ep.row_scale = s2;
-  if (M > QL_MAX_CONTRACTION)
+  const int small = N <= 128 ? ql::small_output_splits(N, K, M) : 1;
+  if (M > QL_MAX_CONTRACTION || small > 1)
     return cuda_status(ql::launch_gemm_i8_long(dyq_c, true, N, xq, true, K, N, K, M,
-                                               at<int32_t>(ws, L.parts), ep, status, s));
+                                               at<int32_t>(ws, L.parts), L.parts_elems, ep,
+                                               status, s, small));
   return cuda_status(ql::launch_gemm_i8(dyq_c, true, N, xq, true, K, N, K, M, ep, status, s));
 }
 

@@ -71,15 +71,37 @@ def test_workspace_grows_by_the_int32_partials_of_long_contractions(L):
         return (x + 255) // 256 * 256
     limit = ql.QL_MAX_CONTRACTION
     # 1023 blocks of 128 per split: 131,072 -> 2 splits, 400,000 -> 4
-    M, K = 8, 256
+    # (200 tokens: more than one 128-row slab, so no extra small-output splits)
+    M, K = 200, 256
     for N, splits in ((limit + 1, 2), (400000, 4)):
         base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
         assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * splits * M * K)
         # rotated: the float32 product waits for its second pass
         assert ql.qlinear_workspace_bytes(M, N, K, 128) == base + a(4 * M * K) + a(4 * splits * M * K)
-    M, N = 262144, 48          # 2048 blocks -> 3 splits over the tokens
+    M, N = 262144, 144         # 2048 blocks -> 3 splits over the tokens
     base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
     assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 3 * N * K)
+    # a small output takes the larger of the two split counts
+    M, N = 262144, 48
+    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 8 * N * K)
+    M, N = 8, 1100000          # 8594 blocks -> 9 splits > 8
+    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 9 * M * K)
+
+
+def test_workspace_small_outputs_reserve_split_partials(L):
+    """Outputs of at most 128 rows (dX for few tokens, dW for few output
+    features) run as up to 8 contraction splits: room for their partials."""
+    def a(x):
+        return (x + 255) // 256 * 256
+    M, N, K = 17, 7168, 5376
+    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 8 * M * K)
+    assert ql.qlinear_workspace_bytes(M, N, K, 128) == base + a(4 * M * K) + a(4 * 8 * M * K)
+    M, N = 4096, 64
+    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 8 * N * K)
 
 
 def test_bwd_workspace_formula(L):

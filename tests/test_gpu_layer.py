@@ -126,11 +126,14 @@ def test_fwd_edge_rows_full_layer(M):
     assert_close(host(y), ry, D, bf16=True, what="y")
 
 
-def test_fwd_int32_accumulator_bit_exact():
+@pytest.mark.parametrize("M,K,N", [(200, 1024, 384),   # CTA-pair tiles
+                                   (100, 1024, 384),   # one slab: 64-wide tiles
+                                   (1, 5376, 7168),    # up to 4 rows: warp per weight row
+                                   (3, 1040, 272), (4, 528, 4096), (16, 528, 4096)])
+def test_fwd_int32_accumulator_bit_exact(M, K, N):
     """Unit scales make y the int32 accumulator converted to float: integer
     rows with max |x| = 127 quantize to themselves with s_x = 1."""
-    rng = np.random.Generator(np.random.PCG64(7))
-    M, K, N = 200, 1024, 384
+    rng = np.random.Generator(np.random.PCG64(7 + M))
     xi = rng.integers(-127, 128, size=(M, K)).astype(np.float32)
     xi[:, 0] = 127.0
     wq_np = rng.integers(-127, 128, size=(N, K)).astype(np.int8)

@@ -110,3 +110,28 @@ def test_combined_backward_with_long_contractions_equals_separate_calls():
         ql.qlinear_bwd_dw(dy_t, xq, sx, dw1, db1, _ws(M, N, K, B), st)
         assert status_word(st) == 0
         assert torch.equal(dx, dx1) and torch.equal(dw, dw1) and torch.equal(db, db1)
+
+
+@pytest.mark.parametrize("M,N,K,B", [(1, 7168, 5376, 128), (17, 7168, 5376, 0), (128, 2048, 1024, 16)])
+def test_dx_small_output_splits_match_oracle(M, N, K, B):
+    """Outputs of at most 128 rows run as contraction splits (int32 partials
+    combined in int64) to spread over the SMs: still exact."""
+    dy = workloads.normal((M, N), 1.0, M + N + 3)
+    w = workloads.normal((N, K), 0.02, N + 4)
+    wq_np, sw_np, _ = oracle.quantize_rows(w, B=B, flags=oracle.REJECT_ZERO_ROWS)
+    dx = _dx(dev(dy), dev(wq_np), dev(sw_np), B, torch.float32)
+    rdx, _, _, st = oracle.bwd_dx(dy, wq_np, sw_np, B)
+    assert st == 0 and np.array_equal(host(dx), rdx)
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 64, 512), (12000, 128, 256)])
+def test_dw_small_output_splits_match_oracle(M, N, K):
+    x = workloads.normal((M, K), 1.0, M + 9)
+    xq_np, sx_np, _ = oracle.quantize_rows(x)
+    dy = workloads.normal((M, N), 1.0, M + 10)
+    dw = torch.empty((N, K), device="cuda")
+    st = new_status()
+    ql.qlinear_bwd_dw(dev(dy), dev(xq_np), dev(sx_np), dw, None, _ws(M, N, K, 0), st)
+    assert status_word(st) == 0
+    rdw, _, _, _, rst = oracle.bwd_dw(dy, xq_np, sx_np)
+    assert rst == 0 and np.array_equal(host(dw), rdw)
