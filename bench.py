@@ -231,8 +231,14 @@ class Layer:
         self.t += 1
         x, dy, y, dx = bufs or (self.x, self.dy, self.y, self.dx)
         # events around the forward, input-gradient and weight-gradient GEMMs
+        # and (update_events) around the forward call, the backward call and
+        # the update
         ql.ql_set_gemm_timing_events(gemm_events or ())
+        if update_events:
+            update_events[2].record()
         ql.qlinear_fwd(x, self.wq, self.sw, self.bias, BLOCK, y, self.xq, self.sx, self.status)
+        if update_events:
+            update_events[3].record()
         ql.qlinear_bwd(dy, self.wq, self.sw, self.xq, self.sx, BLOCK, dx, self.dw, self.db,
                        self.ws, self.status)
         ql.ql_set_gemm_timing_events(())
@@ -311,7 +317,7 @@ def run_ours(args, rank, world, local):
         layer.step()
     torch.cuda.synchronize()
     gemm_ev = [list(zip(*[iter(new_events(6))] * 2)) for _ in range(args.steps)]
-    upd_ev = [new_events(2) for _ in range(args.steps)]
+    upd_ev = [new_events(4) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = ql.ql_kernel_launches()
     clocks = ClockSampler(local)
@@ -338,6 +344,8 @@ def run_ours(args, rank, world, local):
     per_kind = {name: statistics.mean(gemm_ms[j::3]) for j, name in enumerate(("fwd", "dx", "dw"))}
     gemm_avg = statistics.mean(gemm_ms)
     upd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in upd_ev)
+    fwd_call_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in upd_ev)
+    bwd_call_ms = statistics.mean(e[3].elapsed_time(e[0]) for e in upd_ev)
 
     # end to end through the public API with host buffers
     e2e_steps = max(2, min(args.e2e_steps, args.steps))
@@ -390,6 +398,15 @@ def run_ours(args, rank, world, local):
                        "traffic": (UPDATE_TRAFFIC_BYTES if source_sha(UPDATE_SOURCES) == UPDATE_TRAFFIC_SOURCE_SHA
                                    else None),
                        "traffic_unit": "bytes per launch"},
+        "breakdown_ms": {
+            "fwd_call": round(fwd_call_ms, 4),
+            "fwd_quantize_x": round(fwd_call_ms - per_kind["fwd"], 4),
+            "bwd_call": round(bwd_call_ms, 4),
+            "bwd_gradient_prep": round(bwd_call_ms - per_kind["dx"] - per_kind["dw"], 4),
+            "update": round(upd_ms, 4),
+            "note": "CUDA events on the step's stream; fwd_quantize_x and bwd_gradient_prep are "
+                    "the call times minus their GEMM launches",
+        },
         "e2e": {"value": round(job_tops(world, 1, e2e_ms), 2), "unit": "TOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,

@@ -854,6 +854,25 @@ bool encode_tmap_2d(CUtensorMap* m, int elem_bytes, const void* base, uint64_t i
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_rows_128b(CUtensorMap* m, int elem_bytes, const void* base, uint64_t cols,
+                      uint64_t rows, uint64_t pitch, uint32_t box_rows) {
+  // [rows][cols / L][L] with L elements = 128 bytes per line; one box is
+  // box_rows whole rows, written to shared memory with the 128-byte swizzle.
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t L = 128 / static_cast<uint64_t>(elem_bytes);
+  if (cols % L != 0 || cols / L > 256) return false;
+  const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  const cuuint64_t dims[3] = {L, cols / L, rows};
+  const cuuint64_t strides[2] = {128, pitch};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(L), static_cast<cuuint32_t>(cols / L), box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t* B, bool b_mn,
                            int64_t ldb, int64_t rows, int64_t cols, int64_t kc,
                            const GemmEpilogue& e, int32_t* status, cudaStream_t s) {

@@ -23,6 +23,10 @@ void gemm_timing_events(cudaEvent_t* before, cudaEvent_t* after);
 // 2-D tensor map over a row-major [outer][inner] array of elem_bytes-byte
 // elements (raw bits; the pitch in bytes), boxes of box_inner x box_outer
 // elements, out-of-range elements read as zero; 128-byte swizzle or none.
+// Whole rows as [rows][cols / L][L] (L elements = one 128-byte line; cols a
+// multiple of L, at most 256 lines), boxes of box_rows rows, 128-byte swizzle.
+bool encode_rows_128b(CUtensorMap* m, int elem_bytes, const void* base, uint64_t cols,
+                      uint64_t rows, uint64_t pitch, uint32_t box_rows);
 bool encode_tmap_2d(CUtensorMap* m, int elem_bytes, const void* base, uint64_t inner,
                     uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
                     bool swizzle128);

@@ -8,6 +8,8 @@
 // read with 128-bit loads (fp32: two per lane).  A Hadamard block (<= 256)
 // never straddles chunks, so the rotation needs only in-lane butterflies and
 // warp shuffles.  Rows whose chunks fit in registers are read from HBM once.
+#include <algorithm>
+
 #include "launch.h"
 #include "rowops.cuh"
 #include "sm100.cuh"
@@ -224,6 +226,123 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// The block-128 rotation + quantization of bf16 rows (the forward's input):
+// a warp owns 1024 columns, 32 per lane, so five of the seven butterfly
+// stages stay inside a lane and two use shuffles (the 256-column layout
+// above needs four).  Pairs of rows arrive by one TMA load per stage from a
+// [rows][cols/64][64] view with the 128-byte swizzle, which puts each lane's
+// four 16-byte pieces in distinct banks; the rows of a pair are handled by
+// two groups of wpr = cols/1024 (rounded up) warps.
+constexpr int kWideStagesMax = 4;
+
+__global__ void __launch_bounds__(512) quant_b128_wide_kernel(
+    const __grid_constant__ CUtensorMap tm, int64_t rows, int cols, float hc, unsigned flags,
+    int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
+    int32_t* __restrict__ status, int stages, int stage_bytes) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ uint32_t s_max[16];
+  __shared__ __align__(8) uint64_t s_full[kWideStagesMax];
+  __shared__ volatile int s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpr = blockDim.x >> 6;  // warps per row
+  const int sub = warp >= wpr ? 1 : 0, cw = warp - sub * wpr;
+  const int lines = cols >> 6;      // 128-byte lines per row
+  const int64_t pairs = (rows + 1) >> 1;
+  const int64_t mine = pairs > blockIdx.x ? (pairs - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < stages; ++st) mbar_init(smem_u32(&s_full[st]), 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm);
+    for (int st = 0; st < stages && st < mine; ++st) {
+      const int64_t p = blockIdx.x + static_cast<int64_t>(st) * gridDim.x;
+      mbar_arrive_expect_tx(smem_u32(&s_full[st]), static_cast<uint32_t>(2 * lines * 128));
+      tma_load_3d(smem_u32(smem + st * stage_bytes), &tm, smem_u32(&s_full[st]), 0, 0,
+                  static_cast<int>(2 * p));
+    }
+  }
+  const int col0 = cw * 1024 + lane * 32;
+  const bool col_ok = col0 < cols;  // cols % 128 == 0: whole blocks are in or out
+  int64_t done = 0;
+  for (int64_t i = 0; i < mine; ++i) {
+    const int st = static_cast<int>(i % stages);
+    const uint32_t parity = static_cast<uint32_t>((i / stages) & 1);
+    const int64_t r = 2 * (blockIdx.x + i * gridDim.x) + sub;
+    // A thread that gives up (mbar_wait raises s_abort) still takes part in
+    // both barriers below; the CTA leaves the loop together after the second.
+    const bool ok = mbar_wait(smem_u32(&s_full[st]), parity, &s_abort);
+    float v[32];
+    if (ok && col_ok) {
+      // Lane l's 64 bytes are half of line gl = sub*lines + col0/64; piece j
+      // (16 bytes) sits at 16-byte slot (4*(l&1) + j) ^ (gl & 7) of the line.
+      const int gl = sub * lines + (col0 >> 6);
+      const uint8_t* line = smem + st * stage_bytes + gl * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 u = *reinterpret_cast<const uint4*>(line + ((((lane & 1) << 2) + j) ^ (gl & 7)) * 16);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[8 * j + 2 * e] = __uint_as_float(w4[e] << 16);
+          v[8 * j + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+    }
+    fwht128_wide(v, lane, hc);
+    uint32_t mbits = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mbits = max(mbits, abs_bits(v[e]));
+    mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+    if (lane == 0) s_max[warp] = mbits;
+    __syncthreads();  // every thread is done reading stage st
+    if (threadIdx.x == 0 && i + stages < mine && !s_abort) {
+      fence_proxy_async_smem();
+      const int64_t pn = blockIdx.x + (i + stages) * gridDim.x;
+      mbar_arrive_expect_tx(smem_u32(&s_full[st]), static_cast<uint32_t>(2 * lines * 128));
+      tma_load_3d(smem_u32(smem + st * stage_bytes), &tm, smem_u32(&s_full[st]), 0, 0,
+                  static_cast<int>(2 * pn));
+    }
+    mbits = 0;
+    for (int w = 0; w < wpr; ++w) mbits = max(mbits, s_max[sub * wpr + w]);
+    __syncthreads();  // s_max may be rewritten by the next pair
+    if (s_abort) break;
+    if (r < rows) {
+      const float amax = __uint_as_float(mbits);
+      const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
+      if (col_ok) {
+        uint32_t b[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) b[e] = rne_bits_prod(v[e], inv);
+        uint4* dst = reinterpret_cast<uint4*>(q + r * ldq + col0);
+        dst[0] = make_uint4(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]),
+                            pack_codes(b[8], b[9], b[10], b[11]), pack_codes(b[12], b[13], b[14], b[15]));
+        dst[1] = make_uint4(pack_codes(b[16], b[17], b[18], b[19]), pack_codes(b[20], b[21], b[22], b[23]),
+                            pack_codes(b[24], b[25], b[26], b[27]), pack_codes(b[28], b[29], b[30], b[31]));
+      }
+      if (cw == 0 && lane == 0) {
+        row_scale[r] = mbits == 0 ? 0.0f : amax / 127.0f;
+        if (mbits == 0 && (flags & QL_REJECT_ZERO_ROWS)) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+        if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+      }
+    }
+    done = i + 1;
+  }
+  if (threadIdx.x == 0 && s_abort) {
+    atomicOr(status, 1 << QL_ERR_TIMEOUT);
+    for (int64_t i = done; i < mine && i < done + stages; ++i)
+      mbar_wait_drain(smem_u32(&s_full[i % stages]), static_cast<uint32_t>((i / stages) & 1));
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Quantize long rows (more chunks than fit in registers): one CTA per row,
 // two passes over the row (the second re-reads it, normally from L2).
 template <typename InT>
@@ -415,6 +534,32 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
   const int nch = static_cast<int>((cols + 255) / 256);
   const int c = static_cast<int>(cols);
   const int64_t row_bytes = cols * static_cast<int64_t>(sizeof(InT));
+  if (sizeof(InT) == 2 && B == 128 && !cs && cols % 128 == 0 && cols >= 1024 && cols <= 8192 &&
+      (ldx * 2) % 16 == 0 && rows >= 4 * device_info().sms) {
+    CUtensorMap tm;
+    if (!encode_rows_128b(&tm, 2, x, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                          static_cast<uint64_t>(ldx) * 2, 2))
+      return cudaErrorInvalidValue;
+    const int wpr = static_cast<int>((cols + 1023) / 1024);
+    const int stage_bytes = static_cast<int>((2 * row_bytes + 1023) / 1024 * 1024);
+    int stages = 90000 / stage_bytes;
+    stages = stages < 2 ? 2 : stages > kWideStagesMax ? kWideStagesMax : stages;
+    const int smem = stages * stage_bytes + 1024;
+    const int per_sm = std::max(1, std::min(2048 / (64 * wpr), 220000 / (smem + 1024)));
+    const int64_t pairs = (rows + 1) / 2;
+    const int grid = static_cast<int>(std::min<int64_t>(pairs, static_cast<int64_t>(device_info().sms) * per_sm));
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+      cudaFuncSetAttribute(quant_b128_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 110000);
+      attr_set[dev] = true;
+    }
+    quant_b128_wide_kernel<<<grid, 64 * wpr, smem, s>>>(tm, rows, c, hc, flags, q, ldq, rs, st,
+                                                        stages, stage_bytes);
+    count_launches(1);
+    return cudaGetLastError();
+  }
   if (nch >= 9 && nch <= 32 && rows >= 2 * device_info().sms) {
     // Rows of 2304..8192 columns, enough of them to fill the GPU: bulk-copy
     // staged kernel, 2-4 rows per CTA in flight within ~96 KB.

@@ -125,6 +125,19 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return d;
 }
 
+// a * b + c for two pairs (fma.rn.f32x2), each rounded once.  Used only with
+// b = +-1, where the product is exact: fma(own, +-1, p) = p +- own rounded
+// once, the same bits as the butterfly's addition or subtraction.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 // v[i] = v[i] * c for 8 values, two per instruction.
 __device__ __forceinline__ void scale8(float (&v)[8], float c) {
 #pragma unroll
@@ -221,6 +234,50 @@ __device__ __forceinline__ void fwht_chunk(float (&v)[8], int B, int lane, float
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = v[i] * c;
+}
+
+// Block-128 rotation of a 1024-column chunk spread across a warp, lane l
+// holding columns 32l .. 32l+31 (lanes 4b .. 4b+3 hold block b): the
+// butterflies h = 1..16 stay inside the lane, h = 32 and 64 pair lanes l^1
+// and l^2 (the higher index takes partner - own), then every value is
+// multiplied by c.  The same operations in the same order as fwht_chunk with
+// B = 128, so the same bits, with half the shuffles.
+__device__ __forceinline__ void fwht128_wide(float (&v)[32], int lane, float c) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {  // h = 1: pairs (i, i+1), (i+2, i+3)
+    const float2 a = make_float2(v[i], v[i + 2]), b = make_float2(v[i + 1], v[i + 3]);
+    const float2 s2 = add2(a, b), d2 = sub2(a, b);
+    v[i] = s2.x; v[i + 1] = d2.x; v[i + 2] = s2.y; v[i + 3] = d2.y;
+  }
+#pragma unroll
+  for (int h = 2; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      if ((i & h) == 0) {  // pairs (i, i+h), (i+1, i+1+h)
+        const float2 a = make_float2(v[i], v[i + 1]), b = make_float2(v[i + h], v[i + h + 1]);
+        const float2 s2 = add2(a, b), d2 = sub2(a, b);
+        v[i] = s2.x; v[i + 1] = s2.y; v[i + h] = d2.x; v[i + h + 1] = d2.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int d = 1; d <= 2; d <<= 1) {
+    const float sg = (lane & d) ? -1.0f : 1.0f;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float p0 = __shfl_xor_sync(0xFFFFFFFFu, v[i], d);
+      const float p1 = __shfl_xor_sync(0xFFFFFFFFu, v[i + 1], d);
+      const float2 r = fma2(make_float2(v[i], v[i + 1]), make_float2(sg, sg), make_float2(p0, p1));
+      v[i] = r.x;
+      v[i + 1] = r.y;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 r = mul2(make_float2(v[i], v[i + 1]), make_float2(c, c));
+    v[i] = r.x;
+    v[i + 1] = r.y;
+  }
 }
 
 // -------------------------------------------------------------- reductions

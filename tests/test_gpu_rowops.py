@@ -44,6 +44,11 @@ CASES = [
     (500, 5376, 128, torch.bfloat16),  # 21 chunks
     (320, 8192, 256, torch.bfloat16),  # 32 chunks
     (2000, 4096, 0, torch.float32),    # several rows per CTA through the ring
+    # bf16, block 128, >= 4 rows per SM: 1024-column warps, pairs of rows per TMA load
+    (1200, 5376, 128, torch.bfloat16),
+    (601, 1024, 128, torch.bfloat16),  # odd row count: the last pair is half empty
+    (700, 8192, 128, torch.bfloat16),
+    (900, 2176, 128, torch.bfloat16),  # 2176 = 2 * 1024 + 128: a warp with one active block
 ]
 
 
