@@ -146,7 +146,18 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   } else {
     float w8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (ROWMAX && col < N) load8(sw + col, w8);
+    // The row scales of the next tile are loaded while this one is worked on.
+    float fcur[T::kRowsPerWarp], fnext[T::kRowsPerWarp];
+    auto load_scales = [&](int t, float (&f)[T::kRowsPerWarp]) {
+#pragma unroll
+      for (int j = 0; j < T::kRowsPerWarp; ++j) {
+        const int64_t m = static_cast<int64_t>(t) * T::kRows + warp * T::kRowsPerWarp + j;
+        f[j] = (t < t1 && m < M) ? __ldg(sx + m) : 0.0f;
+      }
+    };
+    load_scales(t0, fcur);
     ring.consume(t0, t1, lane, [&](int t, const uint8_t* tile) {
+      load_scales(t + 1, fnext);
 #pragma unroll
       for (int j = 0; j < T::kRowsPerWarp; ++j) {
         const int r = warp * T::kRowsPerWarp + j;
@@ -154,7 +165,7 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
         if (m < M) {  // warp-uniform
           float d[8];
           smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
-          const float f = __ldg(sx + m);
+          const float f = fcur[j];
           uint32_t rb = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -169,6 +180,8 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
           }
         }
       }
+#pragma unroll
+      for (int j = 0; j < T::kRowsPerWarp; ++j) fcur[j] = fnext[j];
     });
   }
   __syncthreads();  // ring drained (the producer waited for its copies): reuse it
@@ -235,7 +248,21 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
       load8(cinv2 + col, iv);
       if (Q1) load8(cs1 + col, w8);
     }
+    // The next tile's row factors are loaded while this one is worked on.
+    float f2cur[T::kRowsPerWarp], f2next[T::kRowsPerWarp];
+    float r1cur[T::kRowsPerWarp], r1next[T::kRowsPerWarp];
+    auto load_rows = [&](int t, float (&f2)[T::kRowsPerWarp], float (&r1)[T::kRowsPerWarp]) {
+#pragma unroll
+      for (int j = 0; j < T::kRowsPerWarp; ++j) {
+        const int64_t m = static_cast<int64_t>(t) * T::kRows + warp * T::kRowsPerWarp + j;
+        const bool in = t < t1 && m < M;
+        f2[j] = in ? __ldg(rs2 + m) : 0.0f;
+        r1[j] = (Q1 && in) ? __ldg(rinv1 + m) : 0.0f;
+      }
+    };
+    load_rows(t0, f2cur, r1cur);
     ring.consume(t0, t1, lane, [&](int t, const uint8_t* tile) {
+      load_rows(t + 1, f2next, r1next);
 #pragma unroll
       for (int j = 0; j < T::kRowsPerWarp; ++j) {
         const int r = warp * T::kRowsPerWarp + j;
@@ -243,20 +270,25 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
         if (m < M && cv) {
           float d[8];
           smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
-          const float f2 = __ldg(rs2 + m);
+          const float f2 = f2cur[j];
           uint32_t b[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], f2), iv[i]);
           *reinterpret_cast<uint2*>(q2 + m * N + col) =
               make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
           if (Q1) {
-            const float r1 = __ldg(rinv1 + m);
+            const float r1 = r1cur[j];
 #pragma unroll
             for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], w8[i]), r1);
             *reinterpret_cast<uint2*>(q1 + m * N + col) =
                 make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
           }
         }
+      }
+#pragma unroll
+      for (int j = 0; j < T::kRowsPerWarp; ++j) {
+        f2cur[j] = f2next[j];
+        r1cur[j] = r1next[j];
       }
     });
   }

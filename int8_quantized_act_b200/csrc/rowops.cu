@@ -235,18 +235,19 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
 // two groups of wpr = cols/1024 (rounded up) warps.
 constexpr int kWideStagesMax = 4;
 
-__global__ void __launch_bounds__(512) quant_b128_wide_kernel(
+template <int WPR>
+__global__ void __launch_bounds__(64 * WPR, WPR <= 6 ? 3 : 2) quant_b128_wide_kernel(
     const __grid_constant__ CUtensorMap tm, int64_t rows, int cols, float hc, unsigned flags,
     int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
     int32_t* __restrict__ status, int stages, int stage_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ uint32_t s_max[16];
+  __shared__ uint32_t s_max[2][2 * WPR];  // double-buffered by pair parity
   __shared__ __align__(8) uint64_t s_full[kWideStagesMax];
   __shared__ volatile int s_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wpr = blockDim.x >> 6;  // warps per row
+  constexpr int wpr = WPR;  // warps per row
   const int sub = warp >= wpr ? 1 : 0, cw = warp - sub * wpr;
   const int lines = cols >> 6;      // 128-byte lines per row
   const int64_t pairs = (rows + 1) >> 1;
@@ -301,8 +302,11 @@ __global__ void __launch_bounds__(512) quant_b128_wide_kernel(
 #pragma unroll
     for (int e = 0; e < 32; ++e) mbits = max(mbits, abs_bits(v[e]));
     mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
-    if (lane == 0) s_max[warp] = mbits;
-    __syncthreads();  // every thread is done reading stage st
+    uint32_t* smax = s_max[i & 1];
+    if (lane == 0) smax[warp] = mbits;
+    // Every thread is done reading stage st (and, one pair back, the other
+    // half of s_max, which the next pair rewrites).
+    __syncthreads();
     if (threadIdx.x == 0 && i + stages < mine && !s_abort) {
       fence_proxy_async_smem();
       const int64_t pn = blockIdx.x + (i + stages) * gridDim.x;
@@ -311,8 +315,8 @@ __global__ void __launch_bounds__(512) quant_b128_wide_kernel(
                   static_cast<int>(2 * pn));
     }
     mbits = 0;
-    for (int w = 0; w < wpr; ++w) mbits = max(mbits, s_max[sub * wpr + w]);
-    __syncthreads();  // s_max may be rewritten by the next pair
+#pragma unroll
+    for (int w = 0; w < wpr; ++w) mbits = max(mbits, smax[sub * wpr + w]);
     if (s_abort) break;
     if (r < rows) {
       const float amax = __uint_as_float(mbits);
@@ -542,21 +546,37 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
       return cudaErrorInvalidValue;
     const int wpr = static_cast<int>((cols + 1023) / 1024);
     const int stage_bytes = static_cast<int>((2 * row_bytes + 1023) / 1024 * 1024);
-    int stages = 90000 / stage_bytes;
+    // Three CTAs per SM up to 6 warps per row (two above), three stages each.
+    const int per_sm = wpr <= 6 ? 3 : 2;
+    int stages = (220000 / per_sm - 2048) / stage_bytes;
     stages = stages < 2 ? 2 : stages > kWideStagesMax ? kWideStagesMax : stages;
     const int smem = stages * stage_bytes + 1024;
-    const int per_sm = std::max(1, std::min(2048 / (64 * wpr), 220000 / (smem + 1024)));
     const int64_t pairs = (rows + 1) / 2;
     const int grid = static_cast<int>(std::min<int64_t>(pairs, static_cast<int64_t>(device_info().sms) * per_sm));
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-      cudaFuncSetAttribute(quant_b128_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 110000);
-      attr_set[dev] = true;
+#define QL_WIDE(W)                                                                              \
+  do {                                                                                          \
+    static bool attr_set[64] = {false};                                                         \
+    int dev = 0;                                                                                \
+    cudaGetDevice(&dev);                                                                        \
+    if (dev < 64 && !attr_set[dev]) {                                                           \
+      cudaFuncSetAttribute(quant_b128_wide_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           110000);                                                             \
+      attr_set[dev] = true;                                                                     \
+    }                                                                                           \
+    quant_b128_wide_kernel<W><<<grid, 64 * W, smem, s>>>(tm, rows, c, hc, flags, q, ldq, rs, st, \
+                                                         stages, stage_bytes);                  \
+  } while (0)
+    switch (wpr) {
+      case 1: QL_WIDE(1); break;
+      case 2: QL_WIDE(2); break;
+      case 3: QL_WIDE(3); break;
+      case 4: QL_WIDE(4); break;
+      case 5: QL_WIDE(5); break;
+      case 6: QL_WIDE(6); break;
+      case 7: QL_WIDE(7); break;
+      default: QL_WIDE(8); break;
     }
-    quant_b128_wide_kernel<<<grid, 64 * wpr, smem, s>>>(tm, rows, c, hc, flags, q, ldq, rs, st,
-                                                        stages, stage_bytes);
+#undef QL_WIDE
     count_launches(1);
     return cudaGetLastError();
   }

@@ -243,11 +243,14 @@ __device__ __forceinline__ void fwht_chunk(float (&v)[8], int B, int lane, float
 // multiplied by c.  The same operations in the same order as fwht_chunk with
 // B = 128, so the same bits, with half the shuffles.
 __device__ __forceinline__ void fwht128_wide(float (&v)[32], int lane, float c) {
+  // h = 1: pairs (i, i+1), one scalar add and subtract each (the pair's two
+  // halves would need to be regrouped for a packed operation); the later
+  // stages combine the register pairs (i, i+1) and (i+h, i+h+1) as they are.
 #pragma unroll
-  for (int i = 0; i < 32; i += 4) {  // h = 1: pairs (i, i+1), (i+2, i+3)
-    const float2 a = make_float2(v[i], v[i + 2]), b = make_float2(v[i + 1], v[i + 3]);
-    const float2 s2 = add2(a, b), d2 = sub2(a, b);
-    v[i] = s2.x; v[i + 1] = d2.x; v[i + 2] = s2.y; v[i + 3] = d2.y;
+  for (int i = 0; i < 32; i += 2) {
+    const float a = v[i], b = v[i + 1];
+    v[i] = a + b;
+    v[i + 1] = a - b;
   }
 #pragma unroll
   for (int h = 2; h < 32; h <<= 1) {
