@@ -79,6 +79,9 @@ def parse_args():
     p.add_argument("--routes", action="store_true",
                    help="instead of the train step: time the forward's int8 and bf16 routes "
                         "at 2048 and 12000 tokens (one JSON line)")
+    p.add_argument("--swiglu", action="store_true",
+                   help="instead of the train step: one SwiGLU MLP training step (d_model 4096, "
+                        "d_ff 14336, 8192 tokens; one JSON line)")
     p.add_argument("--edge", action="store_true",
                    help="instead of the train step: time the layer's calls at 1..128 tokens, "
                         "where the weight stream bounds the forward (one JSON line)")
@@ -670,8 +673,127 @@ def run_edge(args):
     return out
 
 
+def run_swiglu(args):
+    """A SwiGLU MLP training step through the layer calls: d_model 4096,
+    d_ff 14336, 8192 tokens, bf16 activations and gradients, no rotation,
+    AdamW (lr 1e-3, wd 0.01) with stochastic requantization of both weights.
+    w1 and w3 run stacked as one [28672, 4096] weight (one quantization of X
+    for both).  The gating silu(a) * b and its derivative are model glue in
+    torch (bf16 elementwise), timed separately.  Metric: the 9 int8 GEMMs' operations
+    (3 x 2 x 8192 x 4096 x 14336 x 3) per second of the whole step."""
+    import torch
+    import int8_quantized_act_b200 as ql
+    torch.cuda.set_device(0)
+    T, D, F = 8192, 4096, 14336
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    dev = "cuda"
+
+    def normal(shape, std, dtype=torch.float32):
+        return (torch.randn(shape, generator=gen, device=dev) * std).to(dtype)
+
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    class Weight:
+        def __init__(self, n, k):
+            self.q = torch.empty((n, k), dtype=torch.int8, device=dev)
+            self.s = torch.empty(n, device=dev)
+            ql.qlinear_quantize_rows(normal((n, k), 0.02), self.q, self.s, st,
+                                     flags=ql.QL_REJECT_ZERO_ROWS)
+            self.m = torch.zeros((n, k), device=dev)
+            self.v = torch.zeros((n, k), device=dev)
+            self.dw = torch.empty((n, k), device=dev)
+            self.db = torch.empty(n, device=dev)
+
+    w13, w2 = Weight(2 * F, D), Weight(D, F)
+    x = normal((T, D), 1.0, torch.bfloat16)
+    dy = normal((T, D), 1.0, torch.bfloat16)
+    h13 = torch.empty((T, 2 * F), dtype=torch.bfloat16, device=dev)
+    xq = torch.empty((T, D), dtype=torch.int8, device=dev)
+    sx = torch.empty(T, device=dev)
+    h = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
+    hq = torch.empty((T, F), dtype=torch.int8, device=dev)
+    sh = torch.empty(T, device=dev)
+    y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    dh = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
+    sl, sg, tmp = (torch.empty((T, F), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    d13 = torch.empty((T, 2 * F), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(ql.qlinear_bwd_workspace_bytes(T, D, F, 0),
+                         ql.qlinear_bwd_workspace_bytes(T, 2 * F, D, 0)), dtype=torch.uint8,
+                     device=dev)
+    opt = ql.Optim(kind=ql.QL_ADAMW, lr=1e-3, weight_decay=0.01)
+    t = [0]
+
+    def step(ev=None):
+        t[0] += 1
+        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+        rec(0)
+        ql.qlinear_fwd(x, w13.q, w13.s, None, 0, h13, xq, sx, st)
+        rec(1)
+        a, b = h13[:, :F], h13[:, F:]
+        torch.nn.functional.silu(a, out=sl)
+        torch.mul(sl, b, out=h)
+        rec(2)
+        ql.qlinear_fwd(h, w2.q, w2.s, None, 0, y, hq, sh, st)
+        ql.qlinear_bwd(dy, w2.q, w2.s, hq, sh, 0, dh, w2.dw, w2.db, ws, st)
+        rec(3)
+        # d/db = dh * silu(a); d/da = dh * b * silu'(a), silu' = s + silu * (1 - s)
+        torch.mul(dh, sl, out=d13[:, F:])
+        torch.sigmoid(a, out=sg)
+        torch.addcmul(sg, sl, 1 - sg, out=tmp)
+        torch.mul(dh, b, out=d13[:, :F])
+        d13[:, :F].mul_(tmp)
+        rec(4)
+        ql.qlinear_bwd(d13, w13.q, w13.s, xq, sx, 0, dx, w13.dw, w13.db, ws, st)
+        rec(5)
+        ql.qweight_update_sr(w13.q, w13.s, w13.dw, opt, w13.m, w13.v, 11, t[0], st)
+        ql.qweight_update_sr(w2.q, w2.s, w2.dw, opt, w2.m, w2.v, 12, t[0], st)
+        rec(6)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [new_events(7) for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.2)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if int(st.item()):
+        raise RuntimeError(f"device status {ql.status_flags(int(st.item()))}")
+    el = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
+    step_ms = el(0, 6)
+    glue_ms = el(1, 2) + el(3, 4)
+    upd_ms = el(5, 6)
+    ops = 9 * 2.0 * T * D * F
+    upd_bytes = 22 * (2 * F * D + D * F)
+    peaks = load_peaks()
+    return {
+        "metric": "SwiGLU MLP train step TOPS (9 int8 GEMMs per step, d_model 4096, d_ff 14336, 8192 tokens)",
+        "value": round(ops / (step_ms * 1e-3) / 1e12, 2), "unit": "TOPS", "higher_is_better": True,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic",
+        "dtype": "i8",
+        "config": {"workload": "SwiGLU MLP step: w1|w3 stacked [28672,4096], w2 [4096,14336], "
+                               "8192 tokens, bf16 x/dY, AdamW + stochastic requant of both weights",
+                   "tokens": T, "d_model": D, "d_ff": F},
+        "ms_per_step": round(step_ms, 4),
+        "breakdown_ms": {"layer_calls_and_updates": round(step_ms - glue_ms, 4),
+                         "gating_glue_torch": round(glue_ms, 4), "updates": round(upd_ms, 4)},
+        "tops_excluding_glue": round(ops / ((step_ms - glue_ms) * 1e-3) / 1e12, 2),
+        "update_gbs": round(upd_bytes / (upd_ms * 1e-3) / 1e9, 1),
+        "update_frac_of_hbm": round(upd_bytes / (upd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "clocks": clk,
+    }
+
+
 def main():
     args = parse_args()
+    if args.swiglu:
+        print(json.dumps(run_swiglu(args)), flush=True)
+        return
     if args.edge:
         print(json.dumps(run_edge(args)), flush=True)
         return
