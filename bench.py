@@ -731,7 +731,7 @@ def run_swiglu(args):
         ql.qlinear_fwd(x, w13.q, w13.s, None, 0, h13, xq, sx, st)
         rec(1)
         a, b = h13[:, :F], h13[:, F:]
-        torch.nn.functional.silu(a, out=sl)
+        torch.ops.aten.silu.out(a, out=sl)
         torch.mul(sl, b, out=h)
         rec(2)
         ql.qlinear_fwd(h, w2.q, w2.s, None, 0, y, hq, sh, st)

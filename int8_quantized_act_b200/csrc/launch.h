@@ -56,6 +56,13 @@ cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const
                             int32_t* status, cudaStream_t s);
 
 // s1[m] = amax/127, inv1[m] = 127/amax of the row maxima (0 for a zero row).
+// Zero colmax [N], colsum [N] and (if rowmax != NULL) rowmax [M] in one launch.
+cudaError_t launch_zero_stats(uint32_t* colmax, double* colsum, int64_t N, uint32_t* rowmax,
+                              int64_t M, cudaStream_t s);
+// launch_colfinalize and launch_rowfinalize in one launch.
+cudaError_t launch_finalize_both(const uint32_t* colmax, const double* colsum, int64_t N,
+                                 float* s2, float* inv2, float* db, const uint32_t* rowmax,
+                                 int64_t M, float* s1, float* inv1, cudaStream_t s);
 cudaError_t launch_rowfinalize(const uint32_t* rowmax, int64_t M, float* s1, float* inv1,
                                cudaStream_t s);
 

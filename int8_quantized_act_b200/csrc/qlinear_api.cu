@@ -385,9 +385,7 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   float* s2 = at<float>(ws, L.s2);
   float* inv2 = at<float>(ws, L.inv2);
   int8_t* dyq = at<int8_t>(ws, L.dyq);
-  if (cudaMemsetAsync(colmax, 0, static_cast<size_t>(N) * 4, s) != cudaSuccess ||
-      cudaMemsetAsync(colsum, 0, static_cast<size_t>(N) * 8, s) != cudaSuccess)
-    return QL_ERR_CUDA;
+  if (ql::launch_zero_stats(colmax, colsum, N, nullptr, 0, s) != cudaSuccess) return QL_ERR_CUDA;
   cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, nullptr, nullptr,
                                       d_status, s);
   if (e == cudaSuccess) e = ql::launch_colfinalize(colmax, colsum, N, s2, inv2, db, s);
@@ -449,13 +447,10 @@ int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
   float* inv2 = at<float>(ws, L.inv2);
   // Pass 1 over dY: column maxima of |dY*s_x| and column sums, row maxima of
   // |dY*s_w|; pass 2: both code sets, elementwise.
-  if (cudaMemsetAsync(colmax, 0, static_cast<size_t>(N) * 4, s) != cudaSuccess ||
-      cudaMemsetAsync(colsum, 0, static_cast<size_t>(N) * 8, s) != cudaSuccess ||
-      cudaMemsetAsync(rowmax, 0, static_cast<size_t>(M) * 4, s) != cudaSuccess)
-    return QL_ERR_CUDA;
+  if (ql::launch_zero_stats(colmax, colsum, N, rowmax, M, s) != cudaSuccess) return QL_ERR_CUDA;
   cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, sw, rowmax, d_status, s);
-  if (e == cudaSuccess) e = ql::launch_colfinalize(colmax, colsum, N, s2, inv2, db, s);
-  if (e == cudaSuccess) e = ql::launch_rowfinalize(rowmax, M, s1, inv1, s);
+  if (e == cudaSuccess)
+    e = ql::launch_finalize_both(colmax, colsum, N, s2, inv2, db, rowmax, M, s1, inv1, s);
   if (e == cudaSuccess)
     e = ql::launch_dualquant(dy, dyt, M, N, sw, inv1, sx, inv2, dyq_r, dyq_c, d_status, s);
   if (e != cudaSuccess) return QL_ERR_CUDA;

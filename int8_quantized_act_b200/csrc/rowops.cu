@@ -500,6 +500,40 @@ __global__ void colfinalize_kernel(const uint32_t* __restrict__ colmax,
   if (db) db[n] = static_cast<float>(colsum[n]);
 }
 
+// Zero the column maxima and sums and (if given) the row maxima before the
+// column statistics pass accumulates into them: one launch for all three.
+__global__ void zero_stats_kernel(uint32_t* __restrict__ colmax, double* __restrict__ colsum,
+                                  int64_t N, uint32_t* __restrict__ rowmax, int64_t M) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N + M; i += stride) {
+    if (i < N) {
+      colmax[i] = 0u;
+      colsum[i] = 0.0;
+    } else if (rowmax) {
+      rowmax[i - N] = 0u;
+    }
+  }
+}
+
+// Both finalizations in one launch: threads [0, N) do colfinalize's work,
+// threads [N, N + M) rowfinalize's.
+__global__ void finalize_both_kernel(const uint32_t* __restrict__ colmax,
+                                     const double* __restrict__ colsum, int64_t N, float* s2,
+                                     float* inv2, float* db, const uint32_t* __restrict__ rowmax,
+                                     int64_t M, float* s1, float* inv1) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < N) {
+    const float amax = __uint_as_float(colmax[i]);
+    s2[i] = amax == 0.0f ? 0.0f : amax / 127.0f;
+    inv2[i] = amax == 0.0f ? 0.0f : 127.0f / amax;
+    if (db) db[i] = static_cast<float>(colsum[i]);
+  } else if (i < N + M) {
+    const float amax = __uint_as_float(rowmax[i - N]);
+    s1[i - N] = amax == 0.0f ? 0.0f : amax / 127.0f;
+    inv1[i - N] = amax == 0.0f ? 0.0f : 127.0f / amax;
+  }
+}
+
 // s1[m] = amax/127 and inv1[m] = 127/amax of the row maxima (0 for a zero row).
 __global__ void rowfinalize_kernel(const uint32_t* __restrict__ rowmax, int64_t M, float* s1,
                                    float* inv1) {
@@ -689,6 +723,24 @@ cudaError_t launch_dequant_rows(const int8_t* q, int64_t ldq, const float* s, vo
 cudaError_t launch_rowfinalize(const uint32_t* rowmax, int64_t M, float* s1, float* inv1,
                                cudaStream_t s) {
   rowfinalize_kernel<<<static_cast<unsigned>((M + 255) / 256), 256, 0, s>>>(rowmax, M, s1, inv1);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_stats(uint32_t* colmax, double* colsum, int64_t N, uint32_t* rowmax,
+                              int64_t M, cudaStream_t s) {
+  const int64_t n = N + (rowmax ? M : 0);
+  zero_stats_kernel<<<grid_cap((n + 255) / 256, 4), 256, 0, s>>>(colmax, colsum, N, rowmax,
+                                                                 rowmax ? M : 0);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_both(const uint32_t* colmax, const double* colsum, int64_t N,
+                                 float* s2, float* inv2, float* db, const uint32_t* rowmax,
+                                 int64_t M, float* s1, float* inv1, cudaStream_t s) {
+  finalize_both_kernel<<<static_cast<unsigned>((N + M + 255) / 256), 256, 0, s>>>(
+      colmax, colsum, N, s2, inv2, db, rowmax, M, s1, inv1);
   count_launches(1);
   return cudaGetLastError();
 }
