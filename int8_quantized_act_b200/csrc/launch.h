@@ -59,12 +59,13 @@ cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const
 // Zero colmax [N], colsum [N] and (if rowmax != NULL) rowmax [M] in one launch.
 cudaError_t launch_zero_stats(uint32_t* colmax, double* colsum, int64_t N, uint32_t* rowmax,
                               int64_t M, cudaStream_t s);
-// launch_colfinalize and launch_rowfinalize in one launch.
+// s2 = colmax/127, inv2 = 127/colmax, db = colsum (if db) for the N columns and
+// s1 = rowmax/127, inv1 = 127/rowmax for the M rows (M = 0: columns only), in one
+// launch; a zero maximum gives 0 for both.
 cudaError_t launch_finalize_both(const uint32_t* colmax, const double* colsum, int64_t N,
                                  float* s2, float* inv2, float* db, const uint32_t* rowmax,
                                  int64_t M, float* s1, float* inv1, cudaStream_t s);
-cudaError_t launch_rowfinalize(const uint32_t* rowmax, int64_t M, float* s1, float* inv1,
-                               cudaStream_t s);
+
 
 // q2 = rne((dY*rs2[m])*cinv2[n]) and, if q1 != NULL, q1 = rne((dY*cs1[n])*rinv1[m]),
 // both [M,N] (dY streamed through shared memory by TMA).
@@ -73,8 +74,7 @@ cudaError_t launch_dualquant(const void* dy, int dyt, int64_t M, int64_t N, cons
                              int8_t* q1, int8_t* q2, int32_t* status, cudaStream_t s);
 
 // s2[n] = amax/127, inv2[n] = 127/amax (0 for a zero column), db[n] = colsum.
-cudaError_t launch_colfinalize(const uint32_t* colmax, const double* colsum, int64_t N,
-                               float* s2, float* inv2, float* db, cudaStream_t s);
+
 
 // out[r, :] = bias (or 0), dtype ot; used when the contraction is empty.
 cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, const float* bias,

@@ -388,7 +388,8 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   if (ql::launch_zero_stats(colmax, colsum, N, nullptr, 0, s) != cudaSuccess) return QL_ERR_CUDA;
   cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, nullptr, nullptr,
                                       d_status, s);
-  if (e == cudaSuccess) e = ql::launch_colfinalize(colmax, colsum, N, s2, inv2, db, s);
+  if (e == cudaSuccess)
+    e = ql::launch_finalize_both(colmax, colsum, N, s2, inv2, db, nullptr, 0, nullptr, nullptr, s);
   if (e == cudaSuccess)
     e = ql::launch_dualquant(dy, dyt, M, N, nullptr, nullptr, sx, inv2, nullptr, dyq, d_status, s);
   if (e != cudaSuccess || K == 0) return cuda_status(e);

@@ -489,16 +489,6 @@ __global__ void __launch_bounds__(256) dequant_rows_kernel(const int8_t* __restr
   }
 }
 
-__global__ void colfinalize_kernel(const uint32_t* __restrict__ colmax,
-                                   const double* __restrict__ colsum, int N, float* s2,
-                                   float* inv2, float* db) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  const float amax = __uint_as_float(colmax[n]);
-  s2[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
-  inv2[n] = amax == 0.0f ? 0.0f : 127.0f / amax;
-  if (db) db[n] = static_cast<float>(colsum[n]);
-}
 
 // Zero the column maxima and sums and (if given) the row maxima before the
 // column statistics pass accumulates into them: one launch for all three.
@@ -515,8 +505,8 @@ __global__ void zero_stats_kernel(uint32_t* __restrict__ colmax, double* __restr
   }
 }
 
-// Both finalizations in one launch: threads [0, N) do colfinalize's work,
-// threads [N, N + M) rowfinalize's.
+// Scales from the statistics: threads [0, N) turn the column maxima and sums
+// into s2, 127/amax and db; threads [N, N + M) the row maxima into s1, 127/amax.
 __global__ void finalize_both_kernel(const uint32_t* __restrict__ colmax,
                                      const double* __restrict__ colsum, int64_t N, float* s2,
                                      float* inv2, float* db, const uint32_t* __restrict__ rowmax,
@@ -534,15 +524,6 @@ __global__ void finalize_both_kernel(const uint32_t* __restrict__ colmax,
   }
 }
 
-// s1[m] = amax/127 and inv1[m] = 127/amax of the row maxima (0 for a zero row).
-__global__ void rowfinalize_kernel(const uint32_t* __restrict__ rowmax, int64_t M, float* s1,
-                                   float* inv1) {
-  const int64_t m = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (m >= M) return;
-  const float amax = __uint_as_float(rowmax[m]);
-  s1[m] = amax == 0.0f ? 0.0f : amax / 127.0f;
-  inv1[m] = amax == 0.0f ? 0.0f : 127.0f / amax;
-}
 
 template <typename OutT>
 __global__ void fill_rows_kernel(OutT* out, int64_t rows, int cols, const float* bias) {
@@ -720,12 +701,6 @@ cudaError_t launch_dequant_rows(const int8_t* q, int64_t ldq, const float* s, vo
   return cudaGetLastError();
 }
 
-cudaError_t launch_rowfinalize(const uint32_t* rowmax, int64_t M, float* s1, float* inv1,
-                               cudaStream_t s) {
-  rowfinalize_kernel<<<static_cast<unsigned>((M + 255) / 256), 256, 0, s>>>(rowmax, M, s1, inv1);
-  count_launches(1);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_zero_stats(uint32_t* colmax, double* colsum, int64_t N, uint32_t* rowmax,
                               int64_t M, cudaStream_t s) {
@@ -745,13 +720,6 @@ cudaError_t launch_finalize_both(const uint32_t* colmax, const double* colsum, i
   return cudaGetLastError();
 }
 
-cudaError_t launch_colfinalize(const uint32_t* colmax, const double* colsum, int64_t N,
-                               float* s2, float* inv2, float* db, cudaStream_t s) {
-  colfinalize_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, s>>>(
-      colmax, colsum, static_cast<int>(N), s2, inv2, db);
-  count_launches(1);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, const float* bias,
                              cudaStream_t s) {
