@@ -167,11 +167,21 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
           smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
           const float f = fcur[j];
           uint32_t rb = 0;
+          // Two columns per step: the products (only their magnitudes are
+          // used, no sum follows them) and the column sums as packed pairs.
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            mx[i] = max(mx[i], abs_bits(__fmul_rn(d[i], f)));
-            sm[i] += d[i];
-            if (ROWMAX) rb = max(rb, abs_bits(__fmul_rn(d[i], w8[i])));
+          for (int i = 0; i < 8; i += 2) {
+            const float2 dd = make_float2(d[i], d[i + 1]);
+            const float2 p = mul2(dd, make_float2(f, f));
+            mx[i] = max(mx[i], abs_bits(p.x));
+            mx[i + 1] = max(mx[i + 1], abs_bits(p.y));
+            const float2 ss = add2(make_float2(sm[i], sm[i + 1]), dd);
+            sm[i] = ss.x;
+            sm[i + 1] = ss.y;
+            if (ROWMAX) {
+              const float2 r2 = mul2(dd, make_float2(w8[i], w8[i + 1]));
+              rb = __vimax3_u32(rb, abs_bits(r2.x), abs_bits(r2.y));
+            }
           }
           if (ROWMAX) {
             rb = __reduce_max_sync(0xFFFFFFFFu, rb);

@@ -226,30 +226,35 @@ __global__ void __launch_bounds__(256) quant_rows_tma_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// The block-128 rotation + quantization of bf16 rows (the forward's input):
-// a warp owns 1024 columns, 32 per lane, so five of the seven butterfly
-// stages stay inside a lane and two use shuffles (the 256-column layout
-// above needs four).  Pairs of rows arrive by one TMA load per stage from a
-// [rows][cols/64][64] view with the 128-byte swizzle, which puts each lane's
-// four 16-byte pieces in distinct banks; the rows of a pair are handled by
-// two groups of wpr = cols/1024 (rounded up) warps.
 constexpr int kWideStagesMax = 4;
 
-template <int WPR>
-__global__ void __launch_bounds__(64 * WPR, WPR <= 6 ? 3 : 2) quant_b128_wide_kernel(
+// The block-128 rotation + quantization of bf16 rows (the forward's input).
+// A row's cols/128 blocks are spread over 4 lanes each, 32 columns per lane,
+// so five of the seven butterfly stages stay inside a lane and two use
+// shuffles (the 256-column layout above needs four).  The two rows of a pair
+// are laid end to end over the CTA's lanes (a warp may hold the end of one
+// row and the start of the next; a 4-lane block never straddles a warp), so
+// few lanes idle.  Pairs of rows arrive by one TMA load per stage from a
+// [rows][cols/64][64] view with the 128-byte swizzle, which puts each lane's
+// four 16-byte pieces in distinct banks.
+__global__ void __launch_bounds__(512, 2) quant_b128_wide_kernel(
     const __grid_constant__ CUtensorMap tm, int64_t rows, int cols, float hc, unsigned flags,
     int8_t* __restrict__ q, int64_t ldq, float* __restrict__ row_scale,
     int32_t* __restrict__ status, int stages, int stage_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ uint32_t s_max[2][2 * WPR];  // double-buffered by pair parity
+  __shared__ uint32_t s_max[2][16][2];  // [pair parity][warp][row of the pair]
   __shared__ __align__(8) uint64_t s_full[kWideStagesMax];
   __shared__ volatile int s_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int wpr = WPR;  // warps per row
-  const int sub = warp >= wpr ? 1 : 0, cw = warp - sub * wpr;
+  const int nwarps = blockDim.x >> 5;
   const int lines = cols >> 6;      // 128-byte lines per row
+  const int row_lanes = cols >> 5;  // 4 lanes per 128-column block
+  const int sub = static_cast<int>(threadIdx.x) / row_lanes;  // row of the pair; 2: idle lane
+  const int j = static_cast<int>(threadIdx.x) - sub * row_lanes;
+  const int col0 = (j >> 2) * 128 + (j & 3) * 32;
+  const bool active = sub < 2;
   const int64_t pairs = (rows + 1) >> 1;
   const int64_t mine = pairs > blockIdx.x ? (pairs - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   if (threadIdx.x == 0) {
@@ -267,30 +272,29 @@ __global__ void __launch_bounds__(64 * WPR, WPR <= 6 ? 3 : 2) quant_b128_wide_ke
                   static_cast<int>(2 * p));
     }
   }
-  const int col0 = cw * 1024 + lane * 32;
-  const bool col_ok = col0 < cols;  // cols % 128 == 0: whole blocks are in or out
   int64_t done = 0;
   for (int64_t i = 0; i < mine; ++i) {
     const int st = static_cast<int>(i % stages);
     const uint32_t parity = static_cast<uint32_t>((i / stages) & 1);
     const int64_t r = 2 * (blockIdx.x + i * gridDim.x) + sub;
     // A thread that gives up (mbar_wait raises s_abort) still takes part in
-    // both barriers below; the CTA leaves the loop together after the second.
+    // the barrier below; the CTA leaves the loop together after it.
     const bool ok = mbar_wait(smem_u32(&s_full[st]), parity, &s_abort);
     float v[32];
-    if (ok && col_ok) {
-      // Lane l's 64 bytes are half of line gl = sub*lines + col0/64; piece j
-      // (16 bytes) sits at 16-byte slot (4*(l&1) + j) ^ (gl & 7) of the line.
+    if (ok && active) {
+      // Lane's 64 bytes are half of line gl = sub*lines + col0/64; piece p
+      // (16 bytes) sits at 16-byte slot (4*half + p) ^ (gl & 7) of the line.
       const int gl = sub * lines + (col0 >> 6);
+      const int half = (col0 >> 5) & 1;
       const uint8_t* line = smem + st * stage_bytes + gl * 128;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 u = *reinterpret_cast<const uint4*>(line + ((((lane & 1) << 2) + j) ^ (gl & 7)) * 16);
+      for (int pc = 0; pc < 4; ++pc) {
+        const uint4 u = *reinterpret_cast<const uint4*>(line + (((half << 2) + pc) ^ (gl & 7)) * 16);
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          v[8 * j + 2 * e] = __uint_as_float(w4[e] << 16);
-          v[8 * j + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+          v[8 * pc + 2 * e] = __uint_as_float(w4[e] << 16);
+          v[8 * pc + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
         }
       }
     } else {
@@ -301,9 +305,13 @@ __global__ void __launch_bounds__(64 * WPR, WPR <= 6 ? 3 : 2) quant_b128_wide_ke
     uint32_t mbits = 0;
 #pragma unroll
     for (int e = 0; e < 32; ++e) mbits = max(mbits, abs_bits(v[e]));
-    mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
-    uint32_t* smax = s_max[i & 1];
-    if (lane == 0) smax[warp] = mbits;
+    const uint32_t m0 = __reduce_max_sync(0xFFFFFFFFu, sub == 0 ? mbits : 0u);
+    const uint32_t m1 = __reduce_max_sync(0xFFFFFFFFu, sub == 1 ? mbits : 0u);
+    uint32_t(*smax)[2] = s_max[i & 1];
+    if (lane == 0) {
+      smax[warp][0] = m0;
+      smax[warp][1] = m1;
+    }
     // Every thread is done reading stage st (and, one pair back, the other
     // half of s_max, which the next pair rewrites).
     __syncthreads();
@@ -314,24 +322,21 @@ __global__ void __launch_bounds__(64 * WPR, WPR <= 6 ? 3 : 2) quant_b128_wide_ke
       tma_load_3d(smem_u32(smem + st * stage_bytes), &tm, smem_u32(&s_full[st]), 0, 0,
                   static_cast<int>(2 * pn));
     }
-    mbits = 0;
-#pragma unroll
-    for (int w = 0; w < wpr; ++w) mbits = max(mbits, smax[sub * wpr + w]);
     if (s_abort) break;
-    if (r < rows) {
+    if (active && r < rows) {
+      mbits = 0;
+      for (int w = 0; w < nwarps; ++w) mbits = max(mbits, smax[w][sub]);
       const float amax = __uint_as_float(mbits);
       const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
-      if (col_ok) {
-        uint32_t b[32];
+      uint32_t b[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) b[e] = rne_bits_prod(v[e], inv);
-        uint4* dst = reinterpret_cast<uint4*>(q + r * ldq + col0);
-        dst[0] = make_uint4(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]),
-                            pack_codes(b[8], b[9], b[10], b[11]), pack_codes(b[12], b[13], b[14], b[15]));
-        dst[1] = make_uint4(pack_codes(b[16], b[17], b[18], b[19]), pack_codes(b[20], b[21], b[22], b[23]),
-                            pack_codes(b[24], b[25], b[26], b[27]), pack_codes(b[28], b[29], b[30], b[31]));
-      }
-      if (cw == 0 && lane == 0) {
+      for (int e = 0; e < 32; ++e) b[e] = rne_bits_prod(v[e], inv);
+      uint4* dst = reinterpret_cast<uint4*>(q + r * ldq + col0);
+      dst[0] = make_uint4(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]),
+                          pack_codes(b[8], b[9], b[10], b[11]), pack_codes(b[12], b[13], b[14], b[15]));
+      dst[1] = make_uint4(pack_codes(b[16], b[17], b[18], b[19]), pack_codes(b[20], b[21], b[22], b[23]),
+                          pack_codes(b[24], b[25], b[26], b[27]), pack_codes(b[28], b[29], b[30], b[31]));
+      if (j == 0) {
         row_scale[r] = mbits == 0 ? 0.0f : amax / 127.0f;
         if (mbits == 0 && (flags & QL_REJECT_ZERO_ROWS)) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
         if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
@@ -559,39 +564,30 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
     if (!encode_rows_128b(&tm, 2, x, static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
                           static_cast<uint64_t>(ldx) * 2, 2))
       return cudaErrorInvalidValue;
-    const int wpr = static_cast<int>((cols + 1023) / 1024);
+    // Two rows' blocks (4 lanes each) over whole warps; CTAs per SM from the
+    // kernel's actual occupancy, three stages each.
+    const int threads = static_cast<int>((2 * (cols / 128) * 4 + 31) / 32 * 32);
     const int stage_bytes = static_cast<int>((2 * row_bytes + 1023) / 1024 * 1024);
-    // Three CTAs per SM up to 6 warps per row (two above), three stages each.
-    const int per_sm = wpr <= 6 ? 3 : 2;
+    static int occ[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && occ[dev] == 0) {
+      cudaFuncSetAttribute(quant_b128_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 110000);
+      occ[dev] = -1;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_b128_wide_kernel, threads,
+                                                      3 * stage_bytes + 1024) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    per_sm = std::min(per_sm, 3);
     int stages = (220000 / per_sm - 2048) / stage_bytes;
     stages = stages < 2 ? 2 : stages > kWideStagesMax ? kWideStagesMax : stages;
     const int smem = stages * stage_bytes + 1024;
     const int64_t pairs = (rows + 1) / 2;
     const int grid = static_cast<int>(std::min<int64_t>(pairs, static_cast<int64_t>(device_info().sms) * per_sm));
-#define QL_WIDE(W)                                                                              \
-  do {                                                                                          \
-    static bool attr_set[64] = {false};                                                         \
-    int dev = 0;                                                                                \
-    cudaGetDevice(&dev);                                                                        \
-    if (dev < 64 && !attr_set[dev]) {                                                           \
-      cudaFuncSetAttribute(quant_b128_wide_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                           110000);                                                             \
-      attr_set[dev] = true;                                                                     \
-    }                                                                                           \
-    quant_b128_wide_kernel<W><<<grid, 64 * W, smem, s>>>(tm, rows, c, hc, flags, q, ldq, rs, st, \
-                                                         stages, stage_bytes);                  \
-  } while (0)
-    switch (wpr) {
-      case 1: QL_WIDE(1); break;
-      case 2: QL_WIDE(2); break;
-      case 3: QL_WIDE(3); break;
-      case 4: QL_WIDE(4); break;
-      case 5: QL_WIDE(5); break;
-      case 6: QL_WIDE(6); break;
-      case 7: QL_WIDE(7); break;
-      default: QL_WIDE(8); break;
-    }
-#undef QL_WIDE
+    quant_b128_wide_kernel<<<grid, threads, smem, s>>>(tm, rows, c, hc, flags, q, ldq, rs, st,
+                                                        stages, stage_bytes);
     count_launches(1);
     return cudaGetLastError();
   }
