@@ -50,7 +50,12 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;      // 512: the whole TMEM of the SM
 constexpr int NUM_BARS = 2 * STAGES + 5;
-constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16;
+// Float32 epilogues stage each warp's 32 x 32 chunk in shared memory (rows
+// padded to 33 words) so that the stores go out as whole 128-byte row pieces.
+constexpr int kEpiStageFloats = 32 * 33;
+constexpr int kEpiStageBytes = 4 * 4 * kEpiStageFloats;  // 4 epilogue warps
+constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16 +
+                           kEpiStageBytes;
 
 // The single-CTA kernel's tile width: 256 columns, or 64 for outputs of one
 // 128-row slab whose 256-wide tiles would leave most SMs idle (the forward at
@@ -64,7 +69,7 @@ struct Single {
   static constexpr int kStageBytes = A_BYTES + kBBytes;
   static constexpr int kTmemCols = 2 * TBN;  // two accumulators, a power of two >= 32
   static constexpr int kNumBars = 2 * kStages + 5;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 8 * kNumBars + 16;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 8 * kNumBars + 16 + kEpiStageBytes;
 };
 
 struct Epi {
@@ -146,7 +151,7 @@ __device__ __forceinline__ void store16(__nv_bfloat16* p, const float* v) {
 // are computed but not stored.
 template <typename OutT, int HB, bool F16, int TW = BN>
 __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, int quarter,
-                                              int lane, int row0, int col0) {
+                                              int lane, int row0, int col0, float* stage) {
   constexpr int CH = HB > 32 ? HB : 32;  // columns per register chunk
   OutT* out = reinterpret_cast<OutT*>(ep.out);
   const int gr = row0 + quarter * 32 + lane;
@@ -160,8 +165,8 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
     tmem_ld_cols<CH>(taddr + c0, r);
     tmem_wait_ld();
     const int gc0 = col0 + c0;
+    float v[CH];
     if (row_ok && gc0 < ep.cols) {
-      float v[CH];
 #pragma unroll
       for (int i = 0; i < CH; ++i)
         v[i] = (F16 ? __uint_as_float(r[i]) : __int2float_rn(static_cast<int>(r[i]))) * rs;
@@ -193,10 +198,36 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
         }
       }
       if constexpr (HB > 0) fwht_regs<CH, HB>(v, ep.hc);
-      OutT* orow = out + static_cast<int64_t>(gr) * ep.ldo + gc0;
+      if constexpr (std::is_same<OutT, float>::value && HB == 0) {
+        (void)0;
+      } else {
+        OutT* orow = out + static_cast<int64_t>(gr) * ep.ldo + gc0;
 #pragma unroll
-      for (int g = 0; g < CH / 16; ++g)
-        if (gc0 + 16 * g < ep.cols) store16(orow + 16 * g, v + 16 * g);
+        for (int g = 0; g < CH / 16; ++g)
+          if (gc0 + 16 * g < ep.cols) store16(orow + 16 * g, v + 16 * g);
+      }
+    }
+    if constexpr (std::is_same<OutT, float>::value && HB == 0) {
+      // Lane l holds row l of the warp's 32 rows; through the padded stage,
+      // lane l then writes columns 4(l%8)..+3 of rows l/8, l/8+4, ...: each
+      // store instruction covers four whole 128-byte row pieces.  (Every
+      // lane takes part, whatever its row or column range.)
+      if (gc0 < ep.cols) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) stage[lane * 33 + e] = row_ok ? v[e] : 0.0f;
+        __syncwarp();
+        const int cc = (lane & 7) * 4;
+        const int rbase = row0 + quarter * 32;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + (lane >> 3);
+          const float4 val = make_float4(stage[rr * 33 + cc], stage[rr * 33 + cc + 1],
+                                         stage[rr * 33 + cc + 2], stage[rr * 33 + cc + 3]);
+          if (rbase + rr < ep.rows && gc0 + cc < ep.cols)
+            *reinterpret_cast<float4*>(out + static_cast<int64_t>(rbase + rr) * ep.ldo + gc0 + cc) = val;
+        }
+        __syncwarp();
+      }
     }
   }
 }
@@ -247,6 +278,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_stage = reinterpret_cast<float*>(tmem_slot + 4);  // scalar accesses only
 
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
@@ -394,7 +426,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if constexpr (std::is_same<OutT, int32_t>::value)
         epilogue_tile_raw<BN>(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
       else
-        epilogue_tile<OutT, HB, F16, BN>(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN);
+        epilogue_tile<OutT, HB, F16, BN>(eps, tmem_base + acc * BN, quarter, lane, tm * BM, tn * BN,
+                                         epi_stage + quarter * kEpiStageFloats);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -425,7 +458,7 @@ constexpr int PA_BYTES = 128 * BK;                 // 16 KiB: this CTA's A rows
 constexpr int PB_BYTES = 128 * BK;                 // 16 KiB: this CTA's B columns
 constexpr int PSTAGE_BYTES = PA_BYTES + PB_BYTES;  // 32 KiB
 constexpr int PNUM_BARS = 2 * PSTAGES + 5;
-constexpr int PSMEM_BYTES = 1024 + PSTAGES * PSTAGE_BYTES + 8 * PNUM_BARS + 16;
+constexpr int PSMEM_BYTES = 1024 + PSTAGES * PSTAGE_BYTES + 8 * PNUM_BARS + 16 + kEpiStageBytes;
 
 template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
@@ -440,6 +473,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + PSTAGES * PB_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + PNUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_stage = reinterpret_cast<float*>(tmem_slot + 4);  // scalar accesses only
 
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + PSTAGES);
@@ -591,7 +625,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                           tm * 256 + static_cast<int>(rank) * 128, tn * BN);
       else
         epilogue_tile<OutT, HB, F16>(eps, tmem_base + acc * BN, quarter, lane,
-                                     tm * 256 + static_cast<int>(rank) * 128, tn * BN);
+                                     tm * 256 + static_cast<int>(rank) * 128, tn * BN,
+                                     epi_stage + quarter * kEpiStageFloats);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead_tempty0 + 8 * acc);
