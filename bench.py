@@ -44,12 +44,12 @@ NOMINAL_INT8_OVER_BF16 = 2.0   # dense int8 4.5 POPS / dense bf16 2.25 PFLOPS
 # DRAM bytes (read + write) per GEMM launch from the ncu capture summarised in
 # profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
-GEMM_TRAFFIC_BYTES = 364.9e6
-GEMM_TRAFFIC_SOURCE_SHA = "e474c75de67993c5"
+GEMM_TRAFFIC_BYTES = 372.6e6
+GEMM_TRAFFIC_SOURCE_SHA = "0c9711c96999451d"
 # The same for the update kernel (profiles/update_sr_staged_N7168_K5376.md);
 # DRAM writes still held in L2 when the kernel ends are not counted.
-UPDATE_TRAFFIC_BYTES = 790.3e6
-UPDATE_TRAFFIC_SOURCE_SHA = "698dbcc8523edb2b"
+UPDATE_TRAFFIC_BYTES = 790.9e6
+UPDATE_TRAFFIC_SOURCE_SHA = "149c2ee7695fe67e"
 
 
 def source_sha(files=("gemm_i8.cu", "sm100.cuh")):
