@@ -1,8 +1,8 @@
 // gemm_i8.cu - int8 x int8 -> int32 GEMM on the sm_100a tensor cores
 // (tcgen05.mma.kind::i8) with the layer's scale/bias epilogues.
 //
-// One kernel serves the three products of the layer (the north-star
-// formulas; OneTrainer PR #1681 uses torch._int_mm for the forward one):
+// One kernel serves the three products of the layer (OneTrainer PR #1681
+// uses torch._int_mm for the forward one):
 //   forward  y  = X_q W_q^T      A = X_q   [M,K] K-major,  B = W_q [N,K] K-major
 //   input    dX = dYq_r W_q      A = dYq_r [M,N] K-major,  B = W_q [N,K] MN-major
 //   weight   dW = dYq_c^T X_q    A = dYq_c [M,N] MN-major, B = X_q [M,K] MN-major

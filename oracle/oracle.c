@@ -363,7 +363,7 @@ uint32_t ref_fwd_bf16(const float *x, int64_t M, int64_t K, const int8_t *wq, co
 }
 
 /* ------------------------------------------------------------------ */
-/* Backward preparation (the spec formulas for dX and dW)         */
+/* Backward preparation (the layer's formulas for dX and dW)           */
 /* ------------------------------------------------------------------ */
 
 /* Row part: t'[m,n] = dY[m,n] * s_w[n], quantized per row -> dYq_r, s1[m]. */

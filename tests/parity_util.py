@@ -5,7 +5,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-# North-star float bound: max relative error 1e-3 against the oracle's fp32
+# Float bound: max relative error 1e-3 against the oracle's fp32
 # dequant epilogue.
 REL_TOL = 1e-3
 

@@ -44,7 +44,7 @@ def _rotation_fp32(B: int) -> np.ndarray:
 
 def test_orthogonality_matches_page_value():
     """OneTrainer PR #1681 item 3 prints 5.96e-08 for the fp32 buffer; the
-    spec bound is 1e-7 for every block size."""
+    required bound is 1e-7 for every block size."""
     page = float(golden()["hadamard_orthogonality_fp32_B128"])
     R = torch.from_numpy(_rotation_fp32(128))
     err = (R @ R.T - torch.eye(128)).abs().max().item()
