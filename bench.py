@@ -40,6 +40,7 @@ METRIC = "INT8 qlinear fwd+bwd TOPS (3 int8 GEMMs per train step of the 5376->71
 WORKLOAD = ("qlinear train step: M=12000 K=5376 N=7168, Hadamard block 128, bf16 X/dY/y/dX, "
             "fwd + dX + dW + AdamW stochastic requant")
 NOMINAL_INT8_OVER_BF16 = 2.0   # dense int8 4.5 POPS / dense bf16 2.25 PFLOPS
+NOMINAL_INT8_TOPS = 4500.0     # B200 dense int8 spec, for context next to the measured proxy
 
 # DRAM bytes (read + write) per GEMM launch from the ncu capture summarised in
 # profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
@@ -392,7 +393,8 @@ def run_ours(args, rank, world, local):
                      "ms_per_launch": {k: round(v, 4) for k, v in per_kind.items()},
                      "traffic": (GEMM_TRAFFIC_BYTES if gemm_source_sha() == GEMM_TRAFFIC_SOURCE_SHA
                                  else None),
-                     "traffic_unit": "bytes per launch"},
+                     "traffic_unit": "bytes per launch",
+                     "frac_of_nominal_int8": round(gemm_tops / NOMINAL_INT8_TOPS, 4)},
         "row_kernel": {"kernel": "update_sr (AdamW + stochastic requant)", "bound": "hbm",
                        "achieved": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9, 1),
                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -401,6 +403,15 @@ def run_ours(args, rank, world, local):
                        "traffic": (UPDATE_TRAFFIC_BYTES if source_sha(UPDATE_SOURCES) == UPDATE_TRAFFIC_SOURCE_SHA
                                    else None),
                        "traffic_unit": "bytes per launch"},
+        "row_kernels_gbs": {
+            "note": "algorithmic bytes / call time minus its GEMM launches (so including launch "
+                    "gaps): X quantization 3 B/elem; gradient preparation 2 reads of bf16 dY + "
+                    "2 int8 code writes = 6 B/elem; update 22 B/elem",
+            "quantize_x": round(3 * M_TOK * K_IN / ((fwd_call_ms - per_kind["fwd"]) * 1e-3) / 1e9, 1),
+            "gradient_prep": round(6 * M_TOK * N_OUT / ((bwd_call_ms - per_kind["dx"] - per_kind["dw"]) * 1e-3) / 1e9, 1),
+            "update": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9, 1),
+            "peak": peaks["hbm_gbs"],
+        },
         "breakdown_ms": {
             "fwd_call": round(fwd_call_ms, 4),
             "fwd_quantize_x": round(fwd_call_ms - per_kind["fwd"], 4),
