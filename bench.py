@@ -83,6 +83,9 @@ def parse_args():
     p.add_argument("--swiglu", action="store_true",
                    help="instead of the train step: one SwiGLU MLP training step (d_model 4096, "
                         "d_ff 14336, 8192 tokens; one JSON line)")
+    p.add_argument("--sweep", action="store_true",
+                   help="instead of the train step: the AdamW stochastic-requant update (plain and "
+                        "row-wise weight norm) on [n, n] weights, n = 1024 .. 16384 (one JSON line)")
     p.add_argument("--edge", action="store_true",
                    help="instead of the train step: time the layer's calls at 1..128 tokens, "
                         "where the weight stream bounds the forward (one JSON line)")
@@ -800,8 +803,73 @@ def run_swiglu(args):
     }
 
 
+def run_sweep(args):
+    """The update on square weights n x n, n = 1024, 2048, 4096, 8192, 16384:
+    AdamW (lr 1e-3, wd 0.01) with stochastic requantization, plain and with
+    the row-wise weight norm (float32 magnitude per row and its moments).
+    Bytes per call: 22 per element (codes 1 + gradient 4 + moments 8 in; codes
+    1 + moments 8 out) plus, for the weight norm, 24 per row (magnitude and its
+    two moments read and written).  Device time per call (CUDA events, median)."""
+    import torch
+    import int8_quantized_act_b200 as ql
+    torch.cuda.set_device(0)
+    peaks = load_peaks()
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    out = {"metric": "AdamW stochastic-requant update bandwidth (GB/s)", "unit": "GB/s",
+           "higher_is_better": True, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+           "data": "synthetic", "peak_gbs": peaks["hbm_gbs"],
+           "config": {"workload": "update of int8 [n, n] weights, grads ~N(0, 1e-3), AdamW "
+                                  "lr 1e-3 wd 0.01, fp32 moments; weight norm: g ~U(0.5, 2)"},
+           "sizes": {}}
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    opt = ql.Optim(kind=ql.QL_ADAMW, lr=1e-3, weight_decay=0.01)
+    for n in (1024, 2048, 4096, 8192, 16384):
+        w = torch.randn((n, n), generator=gen, device="cuda") * 0.02
+        q = torch.empty((n, n), dtype=torch.int8, device="cuda")
+        sw = torch.empty(n, device="cuda")
+        ql.qlinear_quantize_rows(w, q, sw, st, flags=ql.QL_REJECT_ZERO_ROWS)
+        del w
+        g = torch.randn((n, n), generator=gen, device="cuda") * 1e-3
+        m = torch.zeros((n, n), device="cuda")
+        v = torch.zeros((n, n), device="cuda")
+        gm = torch.rand(n, generator=gen, device="cuda") * 1.5 + 0.5
+        gmm, gmv = torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
+        row = {}
+        for name, kw in (("adamw", {}), ("adamw_weight_norm", {"g": gm, "g_m": gmm, "g_v": gmv})):
+            t = [0]
+
+            def call():
+                t[0] += 1
+                ql.qweight_update_sr(q, sw, g, opt, m, v, 3, t[0], st, **kw)
+
+            for _ in range(args.warmup):
+                call()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            torch.cuda.synchronize()
+            for a, b in ev:
+                a.record()
+                call()
+                b.record()
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+            nbytes = 22 * n * n + (24 * n if kw else 0)
+            row[f"{name}_us"] = round(ms * 1e3, 1)
+            row[f"{name}_gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+            row[f"{name}_frac"] = round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+        out["sizes"][str(n)] = row
+        del q, g, m, v
+        torch.cuda.empty_cache()
+    if int(st.item()):
+        raise RuntimeError(f"device status {ql.status_flags(int(st.item()))}")
+    return out
+
+
 def main():
     args = parse_args()
+    if args.sweep:
+        print(json.dumps(run_sweep(args)), flush=True)
+        return
     if args.swiglu:
         print(json.dumps(run_swiglu(args)), flush=True)
         return

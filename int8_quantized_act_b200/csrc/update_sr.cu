@@ -128,6 +128,8 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
   const bool adam = c.kind == QL_ADAMW;
 
   const float s = sw[n];
+  // The magnitude is read before thread 0 may overwrite it (after the update).
+  const float gmag_n = WN ? gmag[n] : 0.0f;
   uint4 qv[GPT];
   float w[GPT][16];
 #pragma unroll
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
       }
     }
     dg = p;
-    coef = gmag[n] / (s * nq);
+    coef = gmag_n / (s * nq);
   }
 
   // Optimizer step of every element; moments written back immediately.
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
   }
   if constexpr (WN) {
     if (t == 0) {
-      float gm = gmag[n];
+      float gm = gmag_n;
       if (adam) {
         float a1 = g_m[n], a2 = g_v[n];
         gm = adamw(c, gm, dg, a1, a2);
@@ -265,6 +267,184 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
       *reinterpret_cast<uint4*>(wq + row + 16 * j) =
           sr_group(w[i], inv, amax == 0.0f, static_cast<uint64_t>(row + 16 * j), seed_lo, seed_hi,
                    step_lo, step_hi);
+  }
+}
+
+// The row-wise weight-norm update with the row staged in shared memory by
+// four bulk copies (codes, gradient, moments), so the gradient is read from
+// HBM once although both the direction-gradient reduction and the update use
+// it.  The arithmetic, the thread-to-group mapping (thread t takes the
+// 16-element groups t, t+T, ...; T a power of two <= 256, the pinned
+// 256-lane reduction order) and the stochastic rounding are those of
+// update_sr_kernel<GPT, true>, so the results are the same bits.
+__global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
+    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
+    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, uint32_t seed_lo,
+    uint32_t seed_hi, uint32_t step_lo, uint32_t step_hi, float* __restrict__ gmag,
+    float* __restrict__ g_m, float* __restrict__ g_v, int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float s_red[256];
+  __shared__ float s_qhat[256];  // q / ||q|| for the 255 codes -127 .. 127
+  __shared__ int s_ired[8];
+  __shared__ __align__(8) uint64_t s_full;
+  __shared__ volatile int s_abort;
+  const int n = blockIdx.x;
+  const int t = threadIdx.x;
+  const int T = blockDim.x;  // power of two, 32 .. 256
+  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
+  const int ngroups = K >> 4;
+  const int64_t row = static_cast<int64_t>(n) * K;
+  const bool adam = c.kind == QL_ADAMW;
+  const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
+  const uint32_t bar = smem_u32(&s_full);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    s_abort = 0;
+    fence_mbar_init();
+    const uint32_t dst = smem_u32(smem);
+    mbar_arrive_expect_tx(bar, qbytes + fbytes * (adam ? 3u : 1u));
+    bulk_load(dst, wq + row, qbytes, bar);
+    bulk_load(dst + qbytes, grad + row, fbytes, bar);
+    if (adam) {
+      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar);
+      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar);
+    }
+  }
+  const float s = sw[n];
+  const float gmag_n = gmag[n];  // read before thread 0 overwrites it
+  __syncthreads();
+  mbar_wait(bar, 0, &s_abort);
+  __syncthreads();
+  if (s_abort) {  // uniform: every thread reads the flag after the barrier
+    if (t == 0) {
+      atomicOr(status, 1 << QL_ERR_TIMEOUT);
+      mbar_wait_drain(bar, 0);
+    }
+    return;
+  }
+  const uint4* q_s = reinterpret_cast<const uint4*>(smem);
+  float* g_s = reinterpret_cast<float*>(smem + qbytes);  // then the updated direction
+  const float* m_s = reinterpret_cast<const float*>(smem + qbytes + fbytes);
+  const float* v_s = reinterpret_cast<const float*>(smem + qbytes + 2 * fbytes);
+
+  // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31).
+  int ss = 0;
+  for (int j = t; j < ngroups; j += T) {
+    const uint4 q4 = q_s[j];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int qc = code_at(q4, e);
+      ss += qc * qc;
+    }
+  }
+  ss = warp_sum_i(ss);
+  if (lane == 0) s_ired[warp] = ss;
+  __syncthreads();
+  ss = 0;
+  for (int k = 0; k < nwarps; ++k) ss += s_ired[k];
+  if (ss == 0) {  // a zero direction cannot be normalized: reject the row (uniform)
+    if (t == 0) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+    return;
+  }
+  const float nq = static_cast<float>(sqrt(static_cast<double>(ss)));
+  // A code takes one of 255 values, so q / ||q|| is a 255-entry table: the
+  // same IEEE quotients, computed once per row instead of twice per element.
+  for (int cidx = t; cidx < 255; cidx += T) s_qhat[cidx] = static_cast<float>(cidx - 127) / nq;
+  __syncthreads();
+  // dg in the fixed order: thread t is lane t of 256 virtual lanes, adding
+  // its groups' products in increasing k; lanes >= T hold +0.
+  float p = 0.0f;
+  for (int j = t; j < ngroups; j += T) {
+    const uint4 q4 = q_s[j];
+    float gr[16];
+    load16f(g_s + 16 * j, gr);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) p = p + gr[e] * s_qhat[code_at(q4, e) + 127];
+  }
+  for (int off = 128; off >= 1; off >>= 1) {
+    if (off >= T) {
+      p = p + 0.0f;
+    } else if (off >= 32) {
+      s_red[t] = p;
+      __syncthreads();
+      const float o = s_red[t ^ off];
+      __syncthreads();
+      p = p + o;
+    } else {
+      p = p + __shfl_xor_sync(0xFFFFFFFFu, p, off);
+    }
+  }
+  const float dg = p;
+  const float coef = gmag_n / (s * nq);
+
+  // Optimizer step of every element; moments written back as they are done,
+  // the updated direction parked over the gradient.
+  float amax = 0.0f;
+  int bad = 0;
+  for (int j = t; j < ngroups; j += T) {
+    const int64_t off = row + 16 * j;
+    const uint4 q4 = q_s[j];
+    float gr[16], m1[16], m2[16];
+    load16f(g_s + 16 * j, gr);
+    if (adam) {
+      load16f(m_s + 16 * j, m1);
+      load16f(v_s + 16 * j, m2);
+    }
+    float w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float qf = code_f(q4, e);
+      const float gg = coef * (gr[e] - dg * s_qhat[code_at(q4, e) + 127]);
+      const float wv = s * qf;
+      w[e] = adam ? adamw(c, wv, gg, m1[e], m2[e]) : wv - c.lr * gg;
+      bad |= !finite(w[e]);
+      amax = fmaxf(amax, fabsf(w[e]));
+    }
+    if (adam) {
+      store16f(mom1 + off, m1);
+      store16f(mom2 + off, m2);
+    }
+    store16f(g_s + 16 * j, w);
+  }
+  if (t == 0) {
+    float gm = gmag_n;
+    if (adam) {
+      float a1 = g_m[n], a2 = g_v[n];
+      gm = adamw(c, gm, dg, a1, a2);
+      g_m[n] = a1;
+      g_v[n] = a2;
+    } else {
+      gm = gm - c.lr * dg;
+    }
+    gmag[n] = gm;
+  }
+
+  // Row max (also the barrier before the scale is overwritten).
+  amax = warp_max(amax);
+  bad = warp_or(bad);
+  __syncthreads();
+  if (lane == 0) {
+    s_red[warp] = amax;
+    s_ired[warp] = bad;
+  }
+  __syncthreads();
+  amax = 0.0f;
+  bad = 0;
+  for (int k = 0; k < nwarps; ++k) {
+    amax = fmaxf(amax, s_red[k]);
+    bad |= s_ired[k];
+  }
+  const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
+  if (t == 0) {
+    sw[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
+    if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  }
+  for (int j = t; j < ngroups; j += T) {
+    float w[16];
+    load16f(g_s + 16 * j, w);
+    *reinterpret_cast<uint4*>(wq + row + 16 * j) =
+        sr_group(w, inv, amax == 0.0f, static_cast<uint64_t>(row + 16 * j), seed_lo, seed_hi,
+                 step_lo, step_hi);
   }
 }
 
@@ -507,6 +687,33 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
   update_sr_kernel<G, W><<<grid, T, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, g, g_m, \
                                             g_v, status)
   if (g != nullptr) {  // weight norm: power-of-two thread count for the pinned reduction
+    const int64_t row_bytes = K * (c.kind == QL_ADAMW ? 13 : 5);
+    // Dynamic budget: the opt-in limit less the kernel's own static arrays.
+    static int64_t wn_budget[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && wn_budget[dev] == 0) {
+      cudaFuncAttributes fa{};
+      cudaError_t e = cudaFuncGetAttributes(&fa, update_sr_wn_staged_kernel);
+      int64_t b = -1;
+      if (e == cudaSuccess) {
+        b = device_info().smem_optin - static_cast<int64_t>(fa.sharedSizeBytes);
+        e = cudaFuncSetAttribute(update_sr_wn_staged_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(b));
+      }
+      if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // returned here; not left for a later check
+        return e;
+      }
+      wn_budget[dev] = b;
+    }
+    const int64_t budget = dev < 64 ? wn_budget[dev] : 0;
+    if (row_bytes <= budget) {
+      update_sr_wn_staged_kernel<<<grid, T, static_cast<size_t>(row_bytes), s>>>(
+          wq, sw, grad, k, c, m, v, sl, sh, tl, th, g, g_m, g_v, status);
+      count_launches(1);
+      return cudaGetLastError();
+    }
     if (gpt <= 1) QL_UPD(1, true);
     else if (gpt <= 2) QL_UPD(2, true);
     else if (gpt <= 4) QL_UPD(4, true);
