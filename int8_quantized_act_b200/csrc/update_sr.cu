@@ -10,10 +10,11 @@
 // reduction; then every 4-element chunk draws one Philox4x32-10 block and
 // writes 4 stochastically rounded codes.  Rows up to ~8K elements are staged
 // whole by the bulk-copy engine (update_sr_staged_kernel); longer rows are
-// loaded through registers (update_sr_rows_kernel); the row-wise weight-norm
-// variant (update_sr_kernel) keeps 16-element groups for its pinned
-// reduction order.  Bytes per element: AdamW 22 (1+4+4+4 in, 1+4+4 out),
-// SGD 6.
+// loaded through registers (update_sr_rows_kernel).  The row-wise weight-norm
+// variant stages its row the same way (update_sr_wn_staged_kernel; beyond
+// shared memory, update_sr_kernel) and keeps 16-element groups only for the
+// pinned order of its direction-gradient reduction.  Bytes per element:
+// AdamW 22 (1+4+4+4 in, 1+4+4 out), SGD 6.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -270,184 +271,6 @@ __global__ void __launch_bounds__(256) update_sr_kernel(
   }
 }
 
-// The row-wise weight-norm update with the row staged in shared memory by
-// four bulk copies (codes, gradient, moments), so the gradient is read from
-// HBM once although both the direction-gradient reduction and the update use
-// it.  The arithmetic, the thread-to-group mapping (thread t takes the
-// 16-element groups t, t+T, ...; T a power of two <= 256, the pinned
-// 256-lane reduction order) and the stochastic rounding are those of
-// update_sr_kernel<GPT, true>, so the results are the same bits.
-__global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
-    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
-    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, uint32_t seed_lo,
-    uint32_t seed_hi, uint32_t step_lo, uint32_t step_hi, float* __restrict__ gmag,
-    float* __restrict__ g_m, float* __restrict__ g_v, int32_t* __restrict__ status) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float s_red[256];
-  __shared__ float s_qhat[256];  // q / ||q|| for the 255 codes -127 .. 127
-  __shared__ int s_ired[8];
-  __shared__ __align__(8) uint64_t s_full;
-  __shared__ volatile int s_abort;
-  const int n = blockIdx.x;
-  const int t = threadIdx.x;
-  const int T = blockDim.x;  // power of two, 32 .. 256
-  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
-  const int ngroups = K >> 4;
-  const int64_t row = static_cast<int64_t>(n) * K;
-  const bool adam = c.kind == QL_ADAMW;
-  const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
-  const uint32_t bar = smem_u32(&s_full);
-  if (t == 0) {
-    mbar_init(bar, 1);
-    s_abort = 0;
-    fence_mbar_init();
-    const uint32_t dst = smem_u32(smem);
-    mbar_arrive_expect_tx(bar, qbytes + fbytes * (adam ? 3u : 1u));
-    bulk_load(dst, wq + row, qbytes, bar);
-    bulk_load(dst + qbytes, grad + row, fbytes, bar);
-    if (adam) {
-      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar);
-      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar);
-    }
-  }
-  const float s = sw[n];
-  const float gmag_n = gmag[n];  // read before thread 0 overwrites it
-  __syncthreads();
-  mbar_wait(bar, 0, &s_abort);
-  __syncthreads();
-  if (s_abort) {  // uniform: every thread reads the flag after the barrier
-    if (t == 0) {
-      atomicOr(status, 1 << QL_ERR_TIMEOUT);
-      mbar_wait_drain(bar, 0);
-    }
-    return;
-  }
-  const uint4* q_s = reinterpret_cast<const uint4*>(smem);
-  float* g_s = reinterpret_cast<float*>(smem + qbytes);  // then the updated direction
-  const float* m_s = reinterpret_cast<const float*>(smem + qbytes + fbytes);
-  const float* v_s = reinterpret_cast<const float*>(smem + qbytes + 2 * fbytes);
-
-  // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31).
-  int ss = 0;
-  for (int j = t; j < ngroups; j += T) {
-    const uint4 q4 = q_s[j];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int qc = code_at(q4, e);
-      ss += qc * qc;
-    }
-  }
-  ss = warp_sum_i(ss);
-  if (lane == 0) s_ired[warp] = ss;
-  __syncthreads();
-  ss = 0;
-  for (int k = 0; k < nwarps; ++k) ss += s_ired[k];
-  if (ss == 0) {  // a zero direction cannot be normalized: reject the row (uniform)
-    if (t == 0) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
-    return;
-  }
-  const float nq = static_cast<float>(sqrt(static_cast<double>(ss)));
-  // A code takes one of 255 values, so q / ||q|| is a 255-entry table: the
-  // same IEEE quotients, computed once per row instead of twice per element.
-  for (int cidx = t; cidx < 255; cidx += T) s_qhat[cidx] = static_cast<float>(cidx - 127) / nq;
-  __syncthreads();
-  // dg in the fixed order: thread t is lane t of 256 virtual lanes, adding
-  // its groups' products in increasing k; lanes >= T hold +0.
-  float p = 0.0f;
-  for (int j = t; j < ngroups; j += T) {
-    const uint4 q4 = q_s[j];
-    float gr[16];
-    load16f(g_s + 16 * j, gr);
-#pragma unroll
-    for (int e = 0; e < 16; ++e) p = p + gr[e] * s_qhat[code_at(q4, e) + 127];
-  }
-  for (int off = 128; off >= 1; off >>= 1) {
-    if (off >= T) {
-      p = p + 0.0f;
-    } else if (off >= 32) {
-      s_red[t] = p;
-      __syncthreads();
-      const float o = s_red[t ^ off];
-      __syncthreads();
-      p = p + o;
-    } else {
-      p = p + __shfl_xor_sync(0xFFFFFFFFu, p, off);
-    }
-  }
-  const float dg = p;
-  const float coef = gmag_n / (s * nq);
-
-  // Optimizer step of every element; moments written back as they are done,
-  // the updated direction parked over the gradient.
-  float amax = 0.0f;
-  int bad = 0;
-  for (int j = t; j < ngroups; j += T) {
-    const int64_t off = row + 16 * j;
-    const uint4 q4 = q_s[j];
-    float gr[16], m1[16], m2[16];
-    load16f(g_s + 16 * j, gr);
-    if (adam) {
-      load16f(m_s + 16 * j, m1);
-      load16f(v_s + 16 * j, m2);
-    }
-    float w[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float qf = code_f(q4, e);
-      const float gg = coef * (gr[e] - dg * s_qhat[code_at(q4, e) + 127]);
-      const float wv = s * qf;
-      w[e] = adam ? adamw(c, wv, gg, m1[e], m2[e]) : wv - c.lr * gg;
-      bad |= !finite(w[e]);
-      amax = fmaxf(amax, fabsf(w[e]));
-    }
-    if (adam) {
-      store16f(mom1 + off, m1);
-      store16f(mom2 + off, m2);
-    }
-    store16f(g_s + 16 * j, w);
-  }
-  if (t == 0) {
-    float gm = gmag_n;
-    if (adam) {
-      float a1 = g_m[n], a2 = g_v[n];
-      gm = adamw(c, gm, dg, a1, a2);
-      g_m[n] = a1;
-      g_v[n] = a2;
-    } else {
-      gm = gm - c.lr * dg;
-    }
-    gmag[n] = gm;
-  }
-
-  // Row max (also the barrier before the scale is overwritten).
-  amax = warp_max(amax);
-  bad = warp_or(bad);
-  __syncthreads();
-  if (lane == 0) {
-    s_red[warp] = amax;
-    s_ired[warp] = bad;
-  }
-  __syncthreads();
-  amax = 0.0f;
-  bad = 0;
-  for (int k = 0; k < nwarps; ++k) {
-    amax = fmaxf(amax, s_red[k]);
-    bad |= s_ired[k];
-  }
-  const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
-  if (t == 0) {
-    sw[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
-    if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
-  }
-  for (int j = t; j < ngroups; j += T) {
-    float w[16];
-    load16f(g_s + 16 * j, w);
-    *reinterpret_cast<uint4*>(wq + row + 16 * j) =
-        sr_group(w, inv, amax == 0.0f, static_cast<uint64_t>(row + 16 * j), seed_lo, seed_hi,
-                 step_lo, step_hi);
-  }
-}
-
 // Philox round keys k_r = seed + r * (0x9E3779B9, 0xBB67AE85) mod 2^32,
 // computed once on the host so each round xors a kernel-parameter constant.
 struct PhiloxKeys {
@@ -661,6 +484,207 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
   }
 }
 
+// The row-wise weight-norm update with the row staged in shared memory by
+// four bulk copies (codes, gradient, moments), so the gradient is read from
+// HBM once although both the direction-gradient reduction and the update use
+// it.  Only the reduction for dg keeps the 16-element groups: the first L
+// threads (L a power of two <= 256) are the virtual lanes of the pinned
+// 256-lane order, lane l adding the groups l, l+L, ... (L = 256, or every
+// group has its own lane).  ||q||^2 (an integer sum), the elementwise step,
+// the row max and the stochastic rounding are free of order and run on all
+// threads over 4-element chunks, as in update_sr_staged_kernel: consecutive
+// threads touch consecutive 16-byte pieces of shared and global memory.  The
+// arithmetic per element and the random words are those of
+// update_sr_kernel<GPT, true>, so the results are the same bits.
+__global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
+    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
+    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
+    uint32_t step_lo, uint32_t step_hi, float* __restrict__ gmag, float* __restrict__ g_m,
+    float* __restrict__ g_v, int L, int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float s_red[256];
+  __shared__ float s_qhat[256];  // q / ||q|| for every byte value q = -128 .. 127
+  __shared__ int s_ired[16];
+  __shared__ float s_dg;
+  __shared__ __align__(8) uint64_t s_full;
+  __shared__ volatile int s_abort;
+  const int n = blockIdx.x;
+  const int t = threadIdx.x;
+  const int T = blockDim.x;  // multiple of 32, L .. 512
+  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
+  const int ngroups = K >> 4, nch = K >> 2;
+  const int64_t row = static_cast<int64_t>(n) * K;
+  const bool adam = c.kind == QL_ADAMW;
+  const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
+  const uint32_t bar = smem_u32(&s_full);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    s_abort = 0;
+    fence_mbar_init();
+    const uint32_t dst = smem_u32(smem);
+    mbar_arrive_expect_tx(bar, qbytes + fbytes * (adam ? 3u : 1u));
+    bulk_load(dst, wq + row, qbytes, bar);
+    bulk_load(dst + qbytes, grad + row, fbytes, bar);
+    if (adam) {
+      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar);
+      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar);
+    }
+  }
+  const float s = sw[n];
+  const float gmag_n = gmag[n];  // read before thread 0 overwrites it
+  __syncthreads();
+  mbar_wait(bar, 0, &s_abort);
+  __syncthreads();
+  if (s_abort) {  // uniform: every thread reads the flag after the barrier
+    if (t == 0) {
+      atomicOr(status, 1 << QL_ERR_TIMEOUT);
+      mbar_wait_drain(bar, 0);
+    }
+    return;
+  }
+  const uint32_t* q_s = reinterpret_cast<const uint32_t*>(smem);
+  float4* g_s = reinterpret_cast<float4*>(smem + qbytes);  // then the updated direction
+  const float4* m_s = reinterpret_cast<const float4*>(smem + qbytes + fbytes);
+  const float4* v_s = reinterpret_cast<const float4*>(smem + qbytes + 2 * fbytes);
+
+  // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31).
+  int ss = 0;
+  for (int ch = t; ch < nch; ch += T) {
+    const uint32_t q4 = q_s[ch];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int qc = static_cast<int8_t>(q4 >> (8 * e));
+      ss += qc * qc;
+    }
+  }
+  ss = warp_sum_i(ss);
+  if (lane == 0) s_ired[warp] = ss;
+  __syncthreads();
+  ss = 0;
+  for (int k = 0; k < nwarps; ++k) ss += s_ired[k];
+  if (ss == 0) {  // a zero direction cannot be normalized: reject the row (uniform)
+    if (t == 0) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+    return;
+  }
+  const float nq = static_cast<float>(sqrt(static_cast<double>(ss)));
+  // A code is one byte, so q / ||q|| is a 256-entry table: the same IEEE
+  // quotients, computed once per row instead of twice per element.
+  for (int cidx = t; cidx < 256; cidx += T) s_qhat[cidx] = static_cast<float>(cidx - 128) / nq;
+  __syncthreads();
+  // dg in the fixed order: virtual lane t < L adds its groups' products in
+  // increasing k; lanes >= L hold +0.
+  float p = 0.0f;
+  if (t < L) {
+    const uint4* q16 = reinterpret_cast<const uint4*>(smem);
+    const float* gf = reinterpret_cast<const float*>(smem + qbytes);
+    for (int j = t; j < ngroups; j += L) {
+      const uint4 q4 = q16[j];
+      float gr[16];
+      load16f(gf + 16 * j, gr);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) p = p + gr[e] * s_qhat[code_at(q4, e) + 128];
+    }
+  }
+  for (int off = 128; off >= 1; off >>= 1) {
+    if (off >= L) {
+      p = p + 0.0f;
+    } else if (off >= 32) {
+      if (t < L) s_red[t] = p;
+      __syncthreads();
+      const float o = t < L ? s_red[t ^ off] : 0.0f;
+      __syncthreads();
+      p = p + o;
+    } else {
+      p = p + __shfl_xor_sync(0xFFFFFFFFu, p, off);
+    }
+  }
+  if (t == 0) s_dg = p;  // every lane < L holds the same sum
+  __syncthreads();
+  const float dg = s_dg;
+  const float coef = gmag_n / (s * nq);
+
+  // Optimizer step of every element; moments written back as they are done,
+  // the updated direction parked over the gradient.
+  float4* m_out = reinterpret_cast<float4*>(mom1 + row);
+  float4* v_out = reinterpret_cast<float4*>(mom2 + row);
+  float amax = 0.0f;
+  int bad = 0;
+  for (int ch = t; ch < nch; ch += T) {
+    const uint32_t q4 = q_s[ch];
+    const float4 g4 = g_s[ch];
+    const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
+    float m1[4], m2[4];
+    if (adam) {
+      const float4 a = m_s[ch], b = v_s[ch];
+      m1[0] = a.x; m1[1] = a.y; m1[2] = a.z; m1[3] = a.w;
+      m2[0] = b.x; m2[1] = b.y; m2[2] = b.z; m2[3] = b.w;
+    }
+    float w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float qhat = s_qhat[static_cast<int>(static_cast<int8_t>(q4 >> (8 * e))) + 128];
+      const float gg = coef * (gr[e] - dg * qhat);
+      const float wv = s * code_byte_f(q4, e);
+      w[e] = adam ? adamw(c, wv, gg, m1[e], m2[e]) : wv - c.lr * gg;
+      bad |= !finite(w[e]);
+      amax = fmaxf(amax, fabsf(w[e]));
+    }
+    if (adam) {
+      __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
+      __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
+    }
+    g_s[ch] = make_float4(w[0], w[1], w[2], w[3]);
+  }
+  if (t == 0) {
+    float gm = gmag_n;
+    if (adam) {
+      float a1 = g_m[n], a2 = g_v[n];
+      gm = adamw(c, gm, dg, a1, a2);
+      g_m[n] = a1;
+      g_v[n] = a2;
+    } else {
+      gm = gm - c.lr * dg;
+    }
+    gmag[n] = gm;
+  }
+
+  // Row max (also the barrier before the scale is overwritten).
+  amax = warp_max(amax);
+  bad = warp_or(bad);
+  if (lane == 0) {
+    s_red[warp] = amax;
+    s_ired[warp] = bad;
+  }
+  __syncthreads();
+  amax = 0.0f;
+  bad = 0;
+  for (int k = 0; k < nwarps; ++k) {
+    amax = fmaxf(amax, s_red[k]);
+    bad |= s_ired[k];
+  }
+  const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
+  if (t == 0) {
+    sw[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
+    if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  }
+  // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
+  // step lo, step hi), key = seed); chunk ch of this row is block row/4 + ch.
+  uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
+  const uint64_t blk0 = static_cast<uint64_t>(row) >> 2;
+  for (int ch = t; ch < nch; ch += T) {
+    const uint64_t blk = blk0 + static_cast<uint64_t>(ch);
+    const uint4 rn = philox10_keys(
+        make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32), step_lo, step_hi),
+        keys);
+    const float4 w = g_s[ch];
+    uint32_t out = 0;
+    if (amax != 0.0f)
+      out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
+                       sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+    __stcs(q_out + ch, out);
+  }
+}
+
 // Chunks of 4 elements per thread (sets the thread count of both kernels).
 #ifndef QL_UPDATE_STAGED_CHUNKS
 #define QL_UPDATE_STAGED_CHUNKS 4
@@ -709,8 +733,15 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     }
     const int64_t budget = dev < 64 ? wn_budget[dev] : 0;
     if (row_bytes <= budget) {
-      update_sr_wn_staged_kernel<<<grid, T, static_cast<size_t>(row_bytes), s>>>(
-          wq, sw, grad, k, c, m, v, sl, sh, tl, th, g, g_m, g_v, status);
+      PhiloxKeys keys;
+      for (int r = 0; r < 10; ++r) {
+        keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
+        keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
+      }
+      const int nch = static_cast<int>(K / 4);
+      const int tr = std::max(T, std::min(512, std::max(32, (nch / QL_UPDATE_STAGED_CHUNKS + 31) / 32 * 32)));
+      update_sr_wn_staged_kernel<<<grid, tr, static_cast<size_t>(row_bytes), s>>>(
+          wq, sw, grad, k, c, m, v, keys, tl, th, g, g_m, g_v, T, status);
       count_launches(1);
       return cudaGetLastError();
     }
