@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
 // The row-wise weight-norm update with the row staged in shared memory by
 // four bulk copies (codes, gradient, moments), so the gradient is read from
 // HBM once although both the direction-gradient reduction and the update use
-// it.  Only the reduction for dg keeps the 16-element groups: the first L
+// it; the moments land on a second barrier while the reductions run.  Only the reduction for dg keeps the 16-element groups: the first L
 // threads (L a power of two <= 256) are the virtual lanes of the pinned
 // 256-lane order, lane l adding the groups l, l+L, ... (L = 256, or every
 // group has its own lane).  ||q||^2 (an integer sum), the elementwise step,
@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
   __shared__ float s_qhat[256];  // q / ||q|| for every byte value q = -128 .. 127
   __shared__ int s_ired[16];
   __shared__ float s_dg;
-  __shared__ __align__(8) uint64_t s_full;
+  __shared__ __align__(8) uint64_t s_full[2];  // codes + gradient; moments
   __shared__ volatile int s_abort;
   const int n = blockIdx.x;
   const int t = threadIdx.x;
@@ -516,18 +516,22 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
   const int64_t row = static_cast<int64_t>(n) * K;
   const bool adam = c.kind == QL_ADAMW;
   const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
-  const uint32_t bar = smem_u32(&s_full);
+  // Two barriers: the reductions need only the codes and the gradient, so
+  // they run while the moments are still arriving.
+  const uint32_t bar = smem_u32(&s_full[0]), bar_mv = smem_u32(&s_full[1]);
   if (t == 0) {
     mbar_init(bar, 1);
+    mbar_init(bar_mv, 1);
     s_abort = 0;
     fence_mbar_init();
     const uint32_t dst = smem_u32(smem);
-    mbar_arrive_expect_tx(bar, qbytes + fbytes * (adam ? 3u : 1u));
+    mbar_arrive_expect_tx(bar, qbytes + fbytes);
     bulk_load(dst, wq + row, qbytes, bar);
     bulk_load(dst + qbytes, grad + row, fbytes, bar);
     if (adam) {
-      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar);
-      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar);
+      mbar_arrive_expect_tx(bar_mv, 2 * fbytes);
+      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar_mv);
+      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar_mv);
     }
   }
   const float s = sw[n];
@@ -536,9 +540,10 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
   mbar_wait(bar, 0, &s_abort);
   __syncthreads();
   if (s_abort) {  // uniform: every thread reads the flag after the barrier
-    if (t == 0) {
+    if (t == 0) {  // copies may still be landing: wait for them (bounded)
       atomicOr(status, 1 << QL_ERR_TIMEOUT);
       mbar_wait_drain(bar, 0);
+      if (adam) mbar_wait_drain(bar_mv, 0);
     }
     return;
   }
@@ -563,7 +568,10 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
   ss = 0;
   for (int k = 0; k < nwarps; ++k) ss += s_ired[k];
   if (ss == 0) {  // a zero direction cannot be normalized: reject the row (uniform)
-    if (t == 0) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+    if (t == 0) {
+      atomicOr(status, 1 << QL_ERR_ZERO_ROW);
+      if (adam) mbar_wait_drain(bar_mv, 0);  // the moments' copies end first
+    }
     return;
   }
   const float nq = static_cast<float>(sqrt(static_cast<double>(ss)));
@@ -599,7 +607,15 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
     }
   }
   if (t == 0) s_dg = p;  // every lane < L holds the same sum
+  if (adam) mbar_wait(bar_mv, 0, &s_abort);
   __syncthreads();
+  if (s_abort) {
+    if (t == 0) {
+      atomicOr(status, 1 << QL_ERR_TIMEOUT);
+      mbar_wait_drain(bar_mv, 0);
+    }
+    return;
+  }
   const float dg = s_dg;
   const float coef = gmag_n / (s * nq);
 
