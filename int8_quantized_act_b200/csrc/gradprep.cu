@@ -134,7 +134,12 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   const int t0 = blockIdx.y * tiles_per_cta;
   const int t1 = t0 + tiles_per_cta < tiles ? t0 + tiles_per_cta : tiles;
   const int col = cb * kCols + lane * 8;
-  uint32_t mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  // Maxima as floats: fmaxf with an |x| operand is one instruction where the
+  // bit-pattern max takes two; for finite values both give the same bits.
+  // fmaxf drops NaN, so a NaN input is caught through the column sums: a
+  // lane's float partial sum turns NaN only from a NaN input (or from an
+  // infinite one, which the maxima report).
+  float mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   float sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   uint32_t rbad = 0;
   if (warp == 8) {
@@ -166,25 +171,26 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
           float d[8];
           smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
           const float f = fcur[j];
-          uint32_t rb = 0;
+          float rbf = 0.0f;
           // Two columns per step: the products (only their magnitudes are
           // used, no sum follows them) and the column sums as packed pairs.
 #pragma unroll
           for (int i = 0; i < 8; i += 2) {
             const float2 dd = make_float2(d[i], d[i + 1]);
             const float2 p = mul2(dd, make_float2(f, f));
-            mx[i] = max(mx[i], abs_bits(p.x));
-            mx[i + 1] = max(mx[i + 1], abs_bits(p.y));
+            mx[i] = fmaxf(mx[i], fabsf(p.x));
+            mx[i + 1] = fmaxf(mx[i + 1], fabsf(p.y));
             const float2 ss = add2(make_float2(sm[i], sm[i + 1]), dd);
             sm[i] = ss.x;
             sm[i + 1] = ss.y;
             if (ROWMAX) {
               const float2 r2 = mul2(dd, make_float2(w8[i], w8[i + 1]));
-              rb = __vimax3_u32(rb, abs_bits(r2.x), abs_bits(r2.y));
+              rbf = fmaxf(rbf, fmaxf(fabsf(r2.x), fabsf(r2.y)));
             }
           }
           if (ROWMAX) {
-            rb = __reduce_max_sync(0xFFFFFFFFu, rb);
+            // Non-negative floats order like their bit patterns.
+            uint32_t rb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(rbf));
             if (lane == 0) atomicMax(rowmax + m, rb);
             rbad = max(rbad, rb);
           }
@@ -198,7 +204,7 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   if (warp < 8) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      s_max[warp][i * 32 + lane] = mx[i];  // column lane*8+i at slot i*32+lane
+      s_max[warp][i * 32 + lane] = __float_as_uint(mx[i]);  // column lane*8+i at slot i*32+lane
       s_sum[warp][i * 32 + lane] = sm[i];
     }
   }
@@ -207,14 +213,17 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
     const int slot = (tid % 8) * 32 + tid / 8;
     uint32_t a = 0;
     double t = 0.0;
+    bool nan = false;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       a = max(a, s_max[w][slot]);
-      t += static_cast<double>(s_sum[w][slot]);
+      const float part = s_sum[w][slot];
+      nan |= part != part;
+      t += static_cast<double>(part);
     }
-    // inf/NaN patterns sort above every finite value: report them (the
-    // affected outputs are unspecified).
-    if (a >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    // An infinite maximum or a NaN partial sum means a non-finite input:
+    // report it (the affected outputs are unspecified).
+    if (a >= kInfBits || nan) atomicOr(status, 1 << QL_ERR_NONFINITE);
     atomicMax(colmax + cb * kCols + tid, a);
     atomicAdd(colsum + cb * kCols + tid, t);
   }

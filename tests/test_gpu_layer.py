@@ -289,6 +289,27 @@ def test_bwd_combined_matches_oracle_and_separate_calls(M, N, K, B, dyt, dxt):
     assert_close(host(db), rdb, np.abs(dy32.astype(np.float64)).sum(0), what="db")
 
 
+@pytest.mark.parametrize("dyt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("bad", [float("nan"), float("inf"), float("-inf")])
+def test_bwd_combined_flags_nonfinite(dyt, bad):
+    """One non-finite dY element sets QL_ERR_NONFINITE in the combined
+    backward's gradient preparation (NaN through the column sums, +-inf
+    through the maxima); the outputs are unspecified."""
+    M, N, K, B = 300, 528, 256, 128
+    x_t, w, _, dy_t = layer_inputs(M, K, N, dyt, 77)
+    wq, sw = prep_weight(w, B)
+    xq_np, sx_np, _ = oracle.quantize_rows(x_t.float().numpy(), B=B)
+    dy_t = dy_t.clone()
+    dy_t[123, 301] = bad
+    ws = torch.empty(ql.qlinear_bwd_workspace_bytes(M, N, K, B), dtype=torch.uint8, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    db = torch.empty(N, dtype=torch.float32, device="cuda")
+    st = new_status()
+    ql.qlinear_bwd(dev(dy_t), wq, sw, dev(xq_np), dev(sx_np), B, dx, dw, db, ws, st)
+    assert status_word(st) & (1 << ql.QL_ERR_NONFINITE)
+
+
 # ------------------------------------------------------------------ full size
 def _sample_rows(M, n, seed):
     rng = np.random.Generator(np.random.PCG64(seed))
