@@ -32,6 +32,7 @@ __all__ = [
     "tiny_layer",
     "rotated_layer",
     "swiglu_mlp",
+    "swiglu_stage_inputs",
     "update_state",
 ]
 
