@@ -50,7 +50,7 @@ GEMM_TRAFFIC_SOURCE_SHA = "7bf4b5057333e762"
 # The same for the update kernel (profiles/update_sr_staged_N7168_K5376.md);
 # DRAM writes still held in L2 when the kernel ends are not counted.
 UPDATE_TRAFFIC_BYTES = 789.3e6
-UPDATE_TRAFFIC_SOURCE_SHA = "e012c3a9984e033c"
+UPDATE_TRAFFIC_SOURCE_SHA = "15723c9e11db1e6f"
 
 
 def source_sha(files=("gemm_i8.cu", "sm100.cuh")):

@@ -485,17 +485,17 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
 }
 
 // The row-wise weight-norm update with the row staged in shared memory by
-// four bulk copies (codes, gradient, moments), so the gradient is read from
-// HBM once although both the direction-gradient reduction and the update use
-// it; the moments land on a second barrier while the reductions run.  Only the reduction for dg keeps the 16-element groups: the first L
-// threads (L a power of two <= 256) are the virtual lanes of the pinned
-// 256-lane order, lane l adding the groups l, l+L, ... (L = 256, or every
-// group has its own lane).  ||q||^2 (an integer sum), the elementwise step,
-// the row max and the stochastic rounding are free of order and run on all
-// threads over 4-element chunks, as in update_sr_staged_kernel: consecutive
-// threads touch consecutive 16-byte pieces of shared and global memory.  The
-// arithmetic per element and the random words are those of
-// update_sr_kernel<GPT, true>, so the results are the same bits.
+// four bulk copies, so the gradient is read from HBM once although both the
+// direction-gradient reduction and the update use it; codes and gradient
+// land on one barrier, the moments on a second while the reductions run.
+// Only the dg reduction keeps 16-element groups: the first L threads (L a
+// power of two <= 256) are the virtual lanes of the pinned 256-lane order,
+// lane l adding groups l, l+L, ... (L = 256, or each group has its own lane).
+// ||q||^2 (an integer sum), the elementwise step, the row max and the
+// stochastic rounding are free of order and run on all threads over
+// 4-element chunks as in update_sr_staged_kernel (consecutive threads touch
+// consecutive 16-byte pieces).  Per-element arithmetic and random words are
+// those of update_sr_kernel<GPT, true>, so the results are the same bits.
 __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
     int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
     UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
