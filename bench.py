@@ -46,11 +46,11 @@ NOMINAL_INT8_TOPS = 4500.0     # B200 dense int8 spec, for context next to the m
 # profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
 GEMM_TRAFFIC_BYTES = 372.6e6
-GEMM_TRAFFIC_SOURCE_SHA = "7bf4b5057333e762"
+GEMM_TRAFFIC_SOURCE_SHA = "2522eb5692e879da"
 # The same for the update kernel (profiles/update_sr_staged_N7168_K5376.md);
 # DRAM writes still held in L2 when the kernel ends are not counted.
 UPDATE_TRAFFIC_BYTES = 789.3e6
-UPDATE_TRAFFIC_SOURCE_SHA = "15723c9e11db1e6f"
+UPDATE_TRAFFIC_SOURCE_SHA = "2bf6f7f04bb79f74"
 
 
 def source_sha(files=("gemm_i8.cu", "sm100.cuh")):

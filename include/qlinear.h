@@ -29,9 +29,9 @@
  *     N = out_features.  All pointers are DEVICE pointers unless stated.
  *   - The caller owns every buffer.  The library never allocates device
  *     memory; its only global state is a per-device, one-time set-up on
- *     first use (kernel attributes, occupancy figures).  Make the first call
- *     of each entry point on a device from one host thread; after that,
- *     calls from any number of host threads are safe.
+ *     first use (kernel attributes, occupancy figures), kept in atomics:
+ *     calls from several host threads are safe (two first calls may both
+ *     run the set-up, which writes the same values).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call is asynchronous on `stream` and never
  *     synchronizes.

@@ -756,7 +756,10 @@ int pair_slots(K kern) {
   static int slots[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && slots[dev] > 0) return slots[dev];
+  if (dev < 64) {
+    const int cached = __atomic_load_n(&slots[dev], __ATOMIC_ACQUIRE);
+    if (cached > 0) return cached;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 74, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -771,7 +774,7 @@ int pair_slots(K kern) {
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1)
     n = device_info().sms / 2;
-  if (dev < 64) slots[dev] = n;
+  if (dev < 64) __atomic_store_n(&slots[dev], n, __ATOMIC_RELEASE);
   return n;
 }
 

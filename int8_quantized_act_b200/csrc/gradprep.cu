@@ -341,9 +341,9 @@ void allow_smem() {
   static bool done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !done[dev]) {
+  if (dev < 64 && !__atomic_load_n(&done[dev], __ATOMIC_ACQUIRE)) {
     cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    done[dev] = true;
+    __atomic_store_n(&done[dev], true, __ATOMIC_RELEASE);
   }
 }
 

@@ -571,9 +571,9 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
     static int occ[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && occ[dev] == 0) {
+    if (dev < 64 && __atomic_load_n(&occ[dev], __ATOMIC_ACQUIRE) == 0) {
       cudaFuncSetAttribute(quant_b128_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 110000);
-      occ[dev] = -1;
+      __atomic_store_n(&occ[dev], -1, __ATOMIC_RELEASE);
     }
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_b128_wide_kernel, threads,
@@ -606,10 +606,10 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
     static bool attr_set[64] = {false};                                                        \
     int dev = 0;                                                                               \
     cudaGetDevice(&dev);                                                                       \
-    if (dev < 64 && !attr_set[dev]) {                                                          \
+    if (dev < 64 && !__atomic_load_n(&attr_set[dev], __ATOMIC_ACQUIRE)) {                      \
       cudaFuncSetAttribute(quant_rows_tma_kernel<InT, CPW, BT>,                                \
                            cudaFuncAttributeMaxDynamicSharedMemorySize, 100000);               \
-      attr_set[dev] = true;                                                                    \
+      __atomic_store_n(&attr_set[dev], true, __ATOMIC_RELEASE);                                \
     }                                                                                          \
     quant_rows_tma_kernel<InT, CPW, BT><<<grid, 256, smem, s>>>(                               \
         x, rows, c, ldx, cs, B, hc, flags, q, ldq, rs, st, stages, stage_bytes);               \

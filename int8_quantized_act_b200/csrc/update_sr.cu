@@ -732,7 +732,7 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     static int64_t wn_budget[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && wn_budget[dev] == 0) {
+    if (dev < 64 && __atomic_load_n(&wn_budget[dev], __ATOMIC_ACQUIRE) == 0) {
       cudaFuncAttributes fa{};
       cudaError_t e = cudaFuncGetAttributes(&fa, update_sr_wn_staged_kernel);
       int64_t b = -1;
@@ -745,9 +745,9 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
         (void)cudaGetLastError();  // returned here; not left for a later check
         return e;
       }
-      wn_budget[dev] = b;
+      __atomic_store_n(&wn_budget[dev], b, __ATOMIC_RELEASE);
     }
-    const int64_t budget = dev < 64 ? wn_budget[dev] : 0;
+    const int64_t budget = dev < 64 ? __atomic_load_n(&wn_budget[dev], __ATOMIC_ACQUIRE) : 0;
     if (row_bytes <= budget) {
       PhiloxKeys keys;
       for (int r = 0; r < 10; ++r) {
@@ -779,10 +779,10 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
       static bool staged_set[64] = {false};
       int dev = 0;
       cudaGetDevice(&dev);
-      if (dev < 64 && !staged_set[dev]) {
+      if (dev < 64 && !__atomic_load_n(&staged_set[dev], __ATOMIC_ACQUIRE)) {
         cudaFuncSetAttribute(update_sr_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(budget));
-        staged_set[dev] = true;
+        __atomic_store_n(&staged_set[dev], true, __ATOMIC_RELEASE);
       }
       update_sr_staged_kernel<<<grid, tr, static_cast<size_t>(row_bytes), s>>>(
           wq, sw, grad, k, c, m, v, keys, tl, th, status);
@@ -795,10 +795,10 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     static bool smem_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !smem_set[dev]) {
+    if (dev < 64 && !__atomic_load_n(&smem_set[dev], __ATOMIC_ACQUIRE)) {
       cudaFuncSetAttribute(update_sr_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            4 * 32768);
-      smem_set[dev] = true;
+      __atomic_store_n(&smem_set[dev], true, __ATOMIC_RELEASE);
     }
     update_sr_rows_kernel<<<grid, tr, static_cast<size_t>(4) * K, s>>>(
         wq, sw, grad, k, c, m, v, keys, tl, th, status);
