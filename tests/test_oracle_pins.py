@@ -622,6 +622,39 @@ def test_adamw_step_matches_torch(warm):
     assert np.abs(w - p.detach().numpy()).max() <= 1e-6 * np.abs(w).max()
 
 
+def test_adamw_first_step_closed_form():
+    """At step 1 from zero moments the bias corrections cancel: m_hat = g and
+    v_hat = g^2, so w' = w (1 - lr wd) - lr g / (|g| + eps), independent of
+    the betas.  A dropped correction, swapped betas or a wrong sign move it
+    by orders of magnitude more than float32 rounding."""
+    d = workloads.update_state(8, 96, seed=8)
+    q, s, _ = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    lr, wd, eps = 1e-3, 0.01, 1e-8
+    w, m, v, *_, st = oracle.update_float(q, s, d["grad"], oracle.ADAMW, lr, step=1,
+                                          m=d["m"], v=d["v"], wd=wd)
+    assert st == 0
+    w0 = _dequant(q, s)
+    g = d["grad"].astype(np.float64)
+    want = w0 * (1.0 - lr * wd) - lr * g / (np.abs(g) + eps)
+    assert np.abs(w - want).max() <= 1e-6 * (np.abs(w0).max() + lr)
+    assert np.allclose(m, 0.1 * g, rtol=1e-6) and np.allclose(v, 0.001 * g * g, rtol=1e-5)
+
+
+def test_adamw_zero_gradient_is_pure_decoupled_decay():
+    """With g = 0 and zero moments the Adam term vanishes and only the
+    decoupled decay remains: w' = w (1 - lr wd).  Weight decay folded into
+    the gradient (L2) would instead move every weight by about lr."""
+    d = workloads.update_state(4, 64, seed=9)
+    q, s, _ = oracle.quantize_rows(d["w"], flags=oracle.REJECT_ZERO_ROWS)
+    lr, wd = 1e-3, 0.01
+    zero = np.zeros_like(d["grad"])
+    w, m, v, *_, st = oracle.update_float(q, s, zero, oracle.ADAMW, lr, step=1,
+                                          m=d["m"], v=d["v"], wd=wd)
+    assert st == 0 and not m.any() and not v.any()
+    w0 = _dequant(q, s)
+    assert np.abs(w - w0 * (1.0 - lr * wd)).max() <= 1e-7 * np.abs(w0).max()
+
+
 def test_weight_norm_step_matches_torch_autograd():
     """Row-wise weight norm (dim=0): w = g * v / ||v||.  torch autograd gives
     dL/dg and dL/dv for dL/dw = grad; torch AdamW then steps g and v."""
