@@ -167,6 +167,29 @@ def _contig(t: Optional[torch.Tensor], what: str):
         raise ValueError(f"{what}: expected a contiguous tensor")
 
 
+def _fits(t: Optional[torch.Tensor], rows: int, cols: int, what: str, exact_cols: bool):
+    """A 2-D operand must hold `rows` rows of `cols` columns: at least `rows`
+    rows and exactly `cols` columns (operands the library reads with their
+    row length as the leading dimension) or at least `cols` (operands passed
+    with their own leading dimension).  The C ABI sees only pointers, so this
+    is the one place where a short buffer can be refused before a kernel
+    reads or writes past it.  Absent or empty operands are left to the
+    library."""
+    if t is None or rows == 0 or cols == 0:
+        return
+    ok = t.dim() == 2 and t.size(0) >= rows and (
+        t.size(1) == cols if exact_cols else t.size(1) >= cols)
+    if not ok:
+        want = f"[>={rows}, {cols}]" if exact_cols else f"[>={rows}, >={cols}]"
+        raise ValueError(f"{what}: expected a 2-D tensor of shape {want}, got {list(t.shape)}")
+
+
+def _holds(t: Optional[torch.Tensor], n: int, what: str):
+    """A vector operand must have at least n elements (absent: left to the library)."""
+    if t is not None and n > 0 and t.numel() < n:
+        raise ValueError(f"{what}: expected at least {n} elements, got {t.numel()}")
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -197,6 +220,12 @@ def qlinear_quantize_rows(x, q, row_scale, status, col_scale=None, hadamard_bloc
     """q, row_scale <- per-row int8 quantization of x (optionally x*col_scale,
     rotated by the block-Hadamard of width hadamard_block)."""
     rows, cols = x.shape
+    _fits(q, rows, cols, "q", exact_cols=False)
+    _contig(row_scale, "row_scale")
+    _contig(col_scale, "col_scale")
+    _holds(row_scale, rows, "row_scale")
+    _holds(col_scale, cols, "col_scale")
+    _holds(status, 1, "status")
     code = lib().qlinear_quantize_rows(
         _dev(x, "x"), _dtype_code(x, "x"), rows, cols, _rowmajor(x, "x"),
         _dev(col_scale, "col_scale", torch.float32), hadamard_block, flags,
@@ -222,6 +251,7 @@ def qlinear_dequantize(wq, sw, hadamard_block: int, w, stream=None):
     if tuple(w.shape) != (N, K):
         raise ValueError("qlinear_dequantize: wq and w shapes differ")
     _contig(sw, "sw")
+    _holds(sw, N, "sw")
     code = lib().qlinear_dequantize(
         _dev(wq, "wq", torch.int8), _rowmajor(wq, "wq"), _dev(sw, "sw", torch.float32), N, K,
         hadamard_block, _dev(w, "w"), _dtype_code(w, "w"), _rowmajor(w, "w"), _stream(stream))
@@ -250,6 +280,11 @@ def qlinear_fwd_bf16(x, wq_bf16, sw, bias, hadamard_block: int, y, ws, status, s
     N = wq_bf16.shape[0]
     for t, n in ((x, "x"), (wq_bf16, "wq_bf16"), (sw, "sw"), (bias, "bias"), (y, "y")):
         _contig(t, n)
+    _fits(wq_bf16, N, K, "wq_bf16", exact_cols=True)
+    _fits(y, M, N, "y", exact_cols=True)
+    _holds(sw, N, "sw")
+    _holds(bias, N, "bias")
+    _holds(status, 1, "status")
     code = lib().qlinear_fwd_bf16(
         _dev(x, "x"), _dtype_code(x, "x"), M, K, _dev(wq_bf16, "wq_bf16", torch.bfloat16),
         _dev(sw, "sw", torch.float32), N, _dev(bias, "bias", torch.float32), hadamard_block,
@@ -267,6 +302,13 @@ def qlinear_fwd(x, wq, sw, bias, hadamard_block: int, y, xq_saved, sx_saved, sta
     for t, n in ((x, "x"), (wq, "wq"), (sw, "sw"), (bias, "bias"), (y, "y"),
                  (xq_saved, "xq_saved"), (sx_saved, "sx_saved")):
         _contig(t, n)
+    _fits(wq, N, K, "wq", exact_cols=True)
+    _fits(y, M, N, "y", exact_cols=True)
+    _fits(xq_saved, M, K, "xq_saved", exact_cols=True)
+    _holds(sw, N, "sw")
+    _holds(bias, N, "bias")
+    _holds(sx_saved, M, "sx_saved")
+    _holds(status, 1, "status")
     code = lib().qlinear_fwd(
         _dev(x, "x"), _dtype_code(x, "x"), M, K, _dev(wq, "wq", torch.int8),
         _dev(sw, "sw", torch.float32), N, _dev(bias, "bias", torch.float32), hadamard_block,
@@ -282,6 +324,10 @@ def qlinear_bwd_dx(dy, wq, sw, hadamard_block: int, dx, ws, status, stream=None)
     K = wq.shape[1]
     for t, n in ((dy, "dy"), (wq, "wq"), (sw, "sw"), (dx, "dx")):
         _contig(t, n)
+    _fits(wq, N, K, "wq", exact_cols=True)
+    _fits(dx, M, K, "dx", exact_cols=True)
+    _holds(sw, N, "sw")
+    _holds(status, 1, "status")
     code = lib().qlinear_bwd_dx(
         _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(wq, "wq", torch.int8),
         _dev(sw, "sw", torch.float32), K, hadamard_block, _dev(dx, "dx"), _dtype_code(dx, "dx"),
@@ -302,6 +348,14 @@ def qlinear_bwd(dy, wq, sw, xq, sx, hadamard_block: int, dx, dw, db, ws, status,
     for t, n in ((dy, "dy"), (wq, "wq"), (sw, "sw"), (xq, "xq"), (sx, "sx"), (dx, "dx"),
                  (dw, "dw"), (db, "db")):
         _contig(t, n)
+    _fits(wq, N, K, "wq", exact_cols=True)
+    _fits(xq, M, K, "xq", exact_cols=True)
+    _fits(dx, M, K, "dx", exact_cols=True)
+    _fits(dw, N, K, "dw", exact_cols=True)
+    _holds(sw, N, "sw")
+    _holds(sx, M, "sx")
+    _holds(db, N, "db")
+    _holds(status, 1, "status")
     code = lib().qlinear_bwd(
         _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(wq, "wq", torch.int8),
         _dev(sw, "sw", torch.float32), _dev(xq, "xq", torch.int8), _dev(sx, "sx", torch.float32),
@@ -321,6 +375,10 @@ def qlinear_bwd_dx_noalloc(dy, wq, sw, hadamard_block: int, dx, status, stream=N
     K = wq.shape[1]
     for t, n in ((dy, "dy"), (wq, "wq"), (sw, "sw"), (dx, "dx")):
         _contig(t, n)
+    _fits(wq, N, K, "wq", exact_cols=True)
+    _fits(dx, M, K, "dx", exact_cols=True)
+    _holds(sw, N, "sw")
+    _holds(status, 1, "status")
     code = lib().qlinear_bwd_dx_noalloc(
         _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(wq, "wq", torch.int8),
         _dev(sw, "sw", torch.float32), K, hadamard_block, _dev(dx, "dx"), _dtype_code(dx, "dx"),
@@ -334,6 +392,11 @@ def qlinear_bwd_dw(dy, xq, sx, dw, db, ws, status, stream=None):
     K = xq.shape[1]
     for t, n in ((dy, "dy"), (xq, "xq"), (sx, "sx"), (dw, "dw"), (db, "db")):
         _contig(t, n)
+    _fits(xq, M, K, "xq", exact_cols=True)
+    _fits(dw, N, K, "dw", exact_cols=True)
+    _holds(sx, M, "sx")
+    _holds(db, N, "db")
+    _holds(status, 1, "status")
     code = lib().qlinear_bwd_dw(
         _dev(dy, "dy"), _dtype_code(dy, "dy"), M, N, _dev(xq, "xq", torch.int8),
         _dev(sx, "sx", torch.float32), K, _dev(dw, "dw", torch.float32),
@@ -347,8 +410,14 @@ def qweight_update_sr(wq, sw, grad, opt: Optim, m, v, seed: int, step: int, stat
     """One optimizer step of the int8 weight with stochastic requantization,
     in place (wq, sw, m, v and, for weight norm, g, g_m, g_v)."""
     N, K = wq.shape
-    for t, n in ((wq, "wq"), (sw, "sw"), (grad, "grad"), (m, "m"), (v, "v")):
+    for t, n in ((wq, "wq"), (sw, "sw"), (grad, "grad"), (m, "m"), (v, "v"), (g, "g"),
+                 (g_m, "g_m"), (g_v, "g_v")):
         _contig(t, n)
+    for t, n in ((grad, "grad"), (m, "m"), (v, "v")):
+        _fits(t, N, K, n, exact_cols=True)
+    for t, n in ((sw, "sw"), (g, "g"), (g_m, "g_m"), (g_v, "g_v")):
+        _holds(t, N, n)
+    _holds(status, 1, "status")
     o = _Optim(int(opt.kind), float(opt.lr), float(opt.beta1), float(opt.beta2),
                float(opt.eps), float(opt.weight_decay))
     wn = None
