@@ -14,7 +14,6 @@ NONFINITE 1<<5, UNSUPPORTED 1<<6.
 from __future__ import annotations
 
 import ctypes
-import os
 
 import numpy as np
 
