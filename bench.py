@@ -46,7 +46,7 @@ NOMINAL_INT8_TOPS = 4500.0     # B200 dense int8 spec, for context next to the m
 # profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
 GEMM_TRAFFIC_BYTES = 372.6e6
-GEMM_TRAFFIC_SOURCE_SHA = "2522eb5692e879da"
+GEMM_TRAFFIC_SOURCE_SHA = "422d63c4c93c197d"
 # The same for the update kernel (profiles/update_sr_staged_N7168_K5376.md);
 # DRAM writes still held in L2 when the kernel ends are not counted.
 UPDATE_TRAFFIC_BYTES = 789.3e6

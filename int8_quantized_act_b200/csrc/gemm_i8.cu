@@ -45,17 +45,12 @@ constexpr int64_t kMaxSplitBlocks = 1023;
 // Most contraction splits used to spread a small (<= 128-row) output.
 constexpr int64_t kMaxSmallSplits = QL_SMALL_OUTPUT_SPLITS;
 constexpr int A_BYTES = BM * BK;       // 16 KiB
-constexpr int B_BYTES = BN * BK;       // 32 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 2 * BN;      // 512: the whole TMEM of the SM
-constexpr int NUM_BARS = 2 * STAGES + 5;
 // Float32 epilogues stage each warp's 32 x 32 chunk in shared memory (rows
 // padded to 33 words) so that the stores go out as whole 128-byte row pieces.
 constexpr int kEpiStageFloats = 32 * 33;
 constexpr int kEpiStageBytes = 4 * 4 * kEpiStageFloats;  // 4 epilogue warps
-constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 8 * NUM_BARS + 16 +
-                           kEpiStageBytes;
 
 // The single-CTA kernel's tile width: 256 columns, or 64 for outputs of one
 // 128-row slab whose 256-wide tiles would leave most SMs idle (the forward at
