@@ -42,6 +42,14 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, n), n
 
 
+def test_every_declared_function_has_a_binding_of_the_same_name():
+    """The Python binding mirrors the C ABI name for name, and each binding
+    function is exported by the package."""
+    for n in declared_functions():
+        assert callable(getattr(ql, n, None)), n
+        assert n in ql.__all__, n
+
+
 def test_status_strings(L):
     for code in range(9):
         assert ql.ql_status_string(code).startswith("QL_")
