@@ -209,7 +209,8 @@ QL_API int qlinear_fwd(const void *x, int xt, int64_t M, int64_t K,
                 int hadamard_block, void *y, int yt,
                 int8_t *xq_saved, float *sx_saved, int32_t *d_status, void *stream);
 
-/* Input gradient:
+/* Input gradient ([QT] intro: the backward products are integer GEMMs too;
+ * [CR] item 2 for the rotation):
  *   dYq, s' = quantize_rows(dY, col_scale = s_w)       (row quantization of dY*s_w)
  *   dX[m,k] = (float)(sum_n dYq[m,n] W_q[n,k]) * s'[m], then dX R if B > 0
  * (the layer saw xR, and R is symmetric, so dL/dx = dL/d(xR) R^T = (...) R).
@@ -221,7 +222,9 @@ QL_API int qlinear_bwd_dx(const void *dy, int dyt, int64_t M, int64_t N,
                    void *dx, int dxt, void *ws, size_t ws_bytes,
                    int32_t *d_status, void *stream);
 
-/* Weight (and bias) gradient from the int8-saved input:
+/* Weight (and bias) gradient from the int8-saved input ([QT] intro: the
+ * Linear input is saved as int8 and the weight gradient is an integer GEMM;
+ * biases and gradients stay float):
  *   t''[m,n] = dY[m,n]*s_x[m]; per column n: s''[n] = max_m|t''|/127,
  *   dYq_c[m,n] = clamp(rne(t''*(127/max_m|t''|)), +-127)
  *   dW[n,k] = (float)(sum_m dYq_c[m,n] X_q[m,k]) * s''[n]   (float32 [N,K],
