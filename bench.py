@@ -42,13 +42,13 @@ WORKLOAD = ("qlinear train step: M=12000 K=5376 N=7168, Hadamard block 128, bf16
 NOMINAL_INT8_OVER_BF16 = 2.0   # dense int8 4.5 POPS / dense bf16 2.25 PFLOPS
 NOMINAL_INT8_TOPS = 4500.0     # B200 dense int8 spec, for context next to the measured proxy
 
-# DRAM bytes (read + write) per GEMM launch from the ncu capture summarised in
-# profiles/gemm_i8_qlinear_M12000.md (mean of the forward, input-gradient and
+# DRAM bytes (read + write) per GEMM launch from an ncu capture of the
+# 12000-token layer step (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
 GEMM_TRAFFIC_BYTES = 372.6e6
 GEMM_TRAFFIC_SOURCE_SHA = "422d63c4c93c197d"
-# The same for the update kernel (profiles/update_sr_staged_N7168_K5376.md);
-# DRAM writes still held in L2 when the kernel ends are not counted.
+# The same for the update kernel on the [7168, 5376] weight; DRAM writes
+# still held in L2 when the kernel ends are not counted.
 UPDATE_TRAFFIC_BYTES = 789.3e6
 UPDATE_TRAFFIC_SOURCE_SHA = "2bf6f7f04bb79f74"
 

@@ -30,7 +30,7 @@
  *   [PX]  Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
  *         1, 2, 3", SC'11 - the Philox4x32 counter-based generator.
  *
- * Readings where the pages leave a step open (each is listed in the design doc):
+ * Readings where the pages leave a step open:
  *   - Per-row symmetric scale s = amax/127, codes rne(t * (127/amax)) clamped
  *     to [-127,127]; a zero row gets s = 0 and zero codes (flagged when the
  *     caller rejects zero rows, as [QT] rejects zero directions).
