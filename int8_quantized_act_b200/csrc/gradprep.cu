@@ -136,9 +136,11 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   const int col = cb * kCols + lane * 8;
   // Maxima as floats: fmaxf with an |x| operand is one instruction where the
   // bit-pattern max takes two; for finite values both give the same bits.
-  // fmaxf drops NaN, so a NaN input is caught through the column sums: a
-  // lane's float partial sum turns NaN only from a NaN input (or from an
-  // infinite one, which the maxima report).
+  // fmaxf drops NaN, so non-finite inputs are also caught through the
+  // column sums: a lane's float partial sum stays finite unless an input is
+  // NaN or infinite (an infinite dY in a row whose s_x is 0 makes a NaN
+  // product, which the maximum drops, but an infinite sum) or the float sum
+  // itself overflows, when db is not finite either.
   float mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   float sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   uint32_t rbad = 0;
@@ -213,17 +215,17 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
     const int slot = (tid % 8) * 32 + tid / 8;
     uint32_t a = 0;
     double t = 0.0;
-    bool nan = false;
+    bool bad = false;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       a = max(a, s_max[w][slot]);
       const float part = s_sum[w][slot];
-      nan |= part != part;
+      bad |= !isfinite(part);
       t += static_cast<double>(part);
     }
-    // An infinite maximum or a NaN partial sum means a non-finite input:
-    // report it (the affected outputs are unspecified).
-    if (a >= kInfBits || nan) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    // An infinite maximum or a non-finite partial sum: report it (the
+    // affected outputs are unspecified).
+    if (a >= kInfBits || bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
     atomicMax(colmax + cb * kCols + tid, a);
     atomicAdd(colsum + cb * kCols + tid, t);
   }
