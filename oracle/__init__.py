@@ -69,6 +69,10 @@ def _declare(L):
         "ref_update_float": (_U32, [_P, _P, _P, _I64, _I64, ctypes.c_int, _F, _F, _F, _F, _F,
                                     _P, _P, _U64, _P, _P, _P, _P]),
         "ref_sr_expectation_enum": (ctypes.c_double, [_F]),
+        "ref_exp": (_F, [_F]),
+        "ref_swiglu_h": (None, [_P, _I64, _I64, _I64, _P]),
+        "ref_swiglu_quantize": (_U32, [_P, _I64, _I64, _I64, _P, _P]),
+        "ref_swiglu_bwd": (None, [_P, _I64, _I64, _I64, _P, _P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -287,3 +291,47 @@ def update_float(q, s, grad, kind: int, lr: float, step: int,
     st = lib().ref_update_float(_p(q), _p(s), _p(grad), N, K, kind, lr, b1, b2, eps, wd,
                                 _p(m), _p(v), step, _p(g), _p(g_m), _p(g_v), _p(w))
     return w, m, v, g, g_m, g_v, st
+
+
+# ---------------------------------------------------------------- SwiGLU gate
+def exp(x: float) -> float:
+    """e^x in float32 by the oracle's stated method (see oracle.c)."""
+    return float(lib().ref_exp(float(x)))
+
+
+def exp_array(x: np.ndarray) -> np.ndarray:
+    f = lib().ref_exp
+    x = _f32(x)
+    return np.array([f(float(v)) for v in x.ravel()], np.float32).reshape(x.shape)
+
+
+def swiglu_h(ab: np.ndarray) -> np.ndarray:
+    """h = silu(a) * b for ab = [a | b] of shape [M, 2F]; returns h [M, F]."""
+    ab = _f32(ab)
+    M, F2 = ab.shape
+    F = F2 // 2
+    h = np.empty((M, F), np.float32)
+    lib().ref_swiglu_h(_p(ab), M, F, F2, _p(h))
+    return h
+
+
+def swiglu_quantize(ab: np.ndarray):
+    """The second projection's saved input: (h codes [M, F], s_h [M], status)."""
+    ab = _f32(ab)
+    M, F2 = ab.shape
+    F = F2 // 2
+    q = np.empty((M, F), np.int8)
+    s = np.empty((M,), np.float32)
+    st = lib().ref_swiglu_quantize(_p(ab), M, F, F2, _p(q), _p(s))
+    return q, s, st
+
+
+def swiglu_bwd(ab: np.ndarray, dh: np.ndarray) -> np.ndarray:
+    """[da | db] [M, 2F] from ab [M, 2F] and dh [M, F]."""
+    ab, dh = _f32(ab), _f32(dh)
+    M, F2 = ab.shape
+    F = F2 // 2
+    assert dh.shape == (M, F)
+    dab = np.empty((M, F2), np.float32)
+    lib().ref_swiglu_bwd(_p(ab), M, F, F2, _p(dh), _p(dab))
+    return dab

@@ -695,3 +695,92 @@ double ref_sr_expectation_enum(float v) {
     for (uint32_t u = 0; u < (1u << 24); ++u) total += (double)sr_round(v, u);
     return total / 16777216.0;
 }
+
+/* ------------------------------------------------------------------ */
+/* SwiGLU gate of the three-projection MLP (the MLP training step the   */
+/* layer is measured in: w1 and w3 take the same input, w2 takes h):    */
+/* h = silu(a) * b with silu(a) = a / (1 + e^-a)                        */
+/* ------------------------------------------------------------------ */
+
+/* e^x in float32, the same float32 steps wherever it is evaluated, so a
+ * code that depends on it is reproducible bit for bit (library expf
+ * implementations differ in the last place).  Method: Cody and Waite's
+ * argument reduction (W. J. Cody, W. Waite, "Software Manual for the
+ * Elementary Functions", 1980): n = rint(x * log2(e)), r = x - n*ln2 with
+ * ln2 split into its float32 value C1 and the remainder C2, each step one
+ * correctly rounded fused multiply-add; then e^r from its Taylor series
+ * sum_{k=0..7} r^k / k! by Horner's rule (|r| <= ln2/2 + tiny, so the first
+ * omitted term r^8/8! is below 5.4e-9 relative); then times 2^n as two exact
+ * powers of two (2^n1 * 2^n2, n1 = n/2), so the only rounding in the
+ * subnormal range is the last product.  x is clamped to [-104, 89] first:
+ * e^89 overflows float32 and e^-104 is below half the smallest subnormal. */
+float ref_exp(float x) {
+    if (x != x) return x;
+    const float L2E = 1.44269504088896341f;            /* log2(e) */
+    const float C1 = 0.693147182464599609375f;         /* fl32(ln 2) */
+    const float C2 = -1.904654299957768e-09f;          /* ln 2 - C1 */
+    static const float c[8] = {1.0f, 1.0f, 0.5f, 0.16666666666666666f,
+                               0.041666666666666664f, 0.008333333333333333f,
+                               0.001388888888888889f, 0.0001984126984126984f}; /* 1/k! */
+    float xc = x > 89.0f ? 89.0f : (x < -104.0f ? -104.0f : x);
+    float nf = rintf(xc * L2E);
+    int n = (int)nf;
+    float r = fmaf(-nf, C1, xc);
+    r = fmaf(-nf, C2, r);
+    float p = c[7];
+    for (int k = 6; k >= 0; --k) p = fmaf(p, r, c[k]);
+    int n1 = n / 2, n2 = n - n1;
+    uint32_t b1 = (uint32_t)(n1 + 127) << 23, b2 = (uint32_t)(n2 + 127) << 23;
+    float f1, f2;
+    memcpy(&f1, &b1, 4);
+    memcpy(&f2, &b2, 4);
+    return (p * f1) * f2;
+}
+
+/* silu(a) = a / (1 + e^-a): one float32 addition and one IEEE division. */
+static float ref_silu(float a) { return a / (1.0f + ref_exp(-a)); }
+
+/* h[m, f] = silu(a[m, f]) * b[m, f] for the stacked pre-activations
+ * ab [M, 2F] (a = columns 0..F-1, b = columns F..2F-1, pitch ldab). */
+void ref_swiglu_h(const float *ab, int64_t M, int64_t F, int64_t ldab, float *h) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t f = 0; f < F; ++f) {
+            const float a = ab[m * ldab + f], b = ab[m * ldab + F + f];
+            h[m * F + f] = ref_silu(a) * b;
+        }
+}
+
+/* The input of the MLP's second projection as that layer saves it: h per
+ * row quantized exactly as the layer's forward quantizes its input (no
+ * rotation): s_h[m] = amax/127, hq = clamp(rne(h * (127/amax)), +-127); a
+ * zero row of h gives s_h = 0 and zero codes; a non-finite h sets
+ * ORC_BIT_NONFINITE. */
+uint32_t ref_swiglu_quantize(const float *ab, int64_t M, int64_t F, int64_t ldab,
+                             int8_t *hq, float *sh) {
+    float *h = (float *)malloc((size_t)(M * F > 0 ? M * F : 1) * sizeof(float));
+    ref_swiglu_h(ab, M, F, ldab, h);
+    uint32_t st = ref_quantize_rows(h, M, F, F, NULL, 0, 0u, hq, F, sh);
+    free(h);
+    return st;
+}
+
+/* The gate's backward: given dh [M, F] (the input gradient of the second
+ * projection) and ab, the gradient at the stacked pre-activations
+ * dab [M, 2F]:  with e = e^-a, d = 1 + e, sigma = 1/d, silu = a/d,
+ *   da = (dh * b) * (sigma * (1 + a * (1 - sigma)))    (d silu/da)
+ *   db = dh * silu
+ * each operation one float32 rounding in the order written. */
+void ref_swiglu_bwd(const float *ab, int64_t M, int64_t F, int64_t ldab, const float *dh,
+                    float *dab) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t f = 0; f < F; ++f) {
+            const float a = ab[m * ldab + f], b = ab[m * ldab + F + f];
+            const float g = dh[m * F + f];
+            const float d = 1.0f + ref_exp(-a);
+            const float sigma = 1.0f / d;
+            const float silu = a / d;
+            const float ds = sigma * (1.0f + a * (1.0f - sigma));
+            dab[m * 2 * F + f] = (g * b) * ds;
+            dab[m * 2 * F + F + f] = g * silu;
+        }
+}

@@ -711,3 +711,97 @@ def test_update_argument_checks():
     assert oracle.update_sr(q, s, g, oracle.SGD, 0.1, seed=0, step=0)[-1] == oracle.BIT_ARG
     assert oracle.update_sr(q, s, g, oracle.SGD, 0.1, seed=0, step=1, wd=0.1)[-1] == oracle.BIT_ARG
     assert oracle.update_sr(q, s, g, 7, 0.1, seed=0, step=1)[-1] == oracle.BIT_ARG
+
+
+# ---------------------------------------------------------------- SwiGLU gate
+U32 = 2.0 ** -24  # unit roundoff of float32
+
+
+def test_exp_within_one_ulp_of_float64():
+    """The oracle's exp (Cody-Waite reduction + Taylor series) against numpy's
+    float64 exp on a dense sweep: under 1 ulp of float32 where the result is
+    a normal number, under one subnormal step below that; exact at 0."""
+    xs = np.concatenate([np.linspace(-110, 95, 100001, dtype=np.float32),
+                         np.float32([0.0, -0.0, 1e-30, -1e-30, 1e-7, 88.72, -87.3, -103.9])])
+    e = oracle.exp_array(xs).astype(np.float64)
+    ref = np.exp(xs.astype(np.float64))
+    normal = (ref > 1.1754944e-38) & (ref < 3.4028235e38)
+    ulp = np.spacing(ref[normal].astype(np.float32)).astype(np.float64)
+    assert (np.abs(e[normal] - ref[normal]) / ulp).max() < 1.0
+    low = ref <= 1.1754944e-38
+    assert np.abs(e[low] - ref[low]).max() <= 2.0 ** -149
+    assert oracle.exp(0.0) == 1.0
+    assert oracle.exp(89.0) == math.inf and oracle.exp(math.inf) == math.inf
+    assert oracle.exp(-110.0) == 0.0 and oracle.exp(-math.inf) == 0.0
+    assert math.isnan(oracle.exp(math.nan))
+    # e^x at the float32 nearest k ln 2: 2^k e^(x - k ln 2) to the same bound
+    for k in range(-120, 120, 7):
+        x = float(np.float32(k * math.log(2.0)))
+        ref = 2.0 ** k * math.exp(x - k * math.log(2.0))
+        assert abs(oracle.exp(x) - ref) < float(np.spacing(np.float32(ref)))
+
+
+def _silu64(a):
+    return a / (1.0 + np.exp(-a))
+
+
+def _swiglu_inputs(M, F, seed):
+    ab = workloads.normal((M, 2 * F), 1.28, seed)
+    ab[0, :4] = np.float32([0.0, -0.0, 100.0, -100.0])   # silu = 0, 0, a, -0
+    ab[1, :3] = np.float32([-120.0, 90.0, 1e-30])
+    return ab
+
+
+def test_swiglu_h_against_float64():
+    """h = silu(a) * b within 4 float32 roundings of the float64 value: the
+    exp (< 1 ulp), 1 + e, the division and the product.  Below a = -88.7,
+    e^-a overflows float32 and silu(a) = a/inf = -0, where the true value
+    |a| e^a is under 3e-37: an absolute allowance of that size."""
+    M, F = 64, 512
+    ab = _swiglu_inputs(M, F, 11)
+    h = oracle.swiglu_h(ab).astype(np.float64)
+    a, b = ab[:, :F].astype(np.float64), ab[:, F:].astype(np.float64)
+    ref = _silu64(a) * b
+    tiny = 3e-37 * np.abs(b)
+    assert np.all(np.abs(h - ref) <= 4 * U32 * np.abs(ref) + tiny)
+    assert h[0, 0] == 0.0 and h[0, 2] == np.float32(100.0) * ab[0, F + 2]
+    assert h[0, 3] == 0.0 and np.signbit(h[0, 3]) != np.signbit(ab[0, F + 3])
+    # torch's own silu agrees to the same bound
+    t = torch.nn.functional.silu(torch.from_numpy(a)).numpy() * b
+    assert np.all(np.abs(h - t) <= 4 * U32 * np.abs(t) + tiny)
+
+
+def test_swiglu_quantize_is_the_row_quantization_of_h():
+    """The second projection's saved input: per-row quantization (pinned
+    above) of h, with zero rows and the non-finite flag carried through."""
+    M, F = 48, 384
+    ab = _swiglu_inputs(M, F, 12)
+    ab[5, :F] = 0.0            # a = 0: h row is zero
+    q, s, st = oracle.swiglu_quantize(ab)
+    rq, rs, rst = oracle.quantize_rows(oracle.swiglu_h(ab), B=0)
+    assert st == rst == 0 and s[5] == 0 and not q[5].any()
+    assert np.array_equal(q, rq) and np.array_equal(s, rs)
+    # every code reconstructs h within half a step
+    h = oracle.swiglu_h(ab).astype(np.float64)
+    assert np.all(np.abs(q * s[:, None].astype(np.float64) - h) <= s[:, None] / 2 * (1 + 1e-6))
+    ab[7, F + 3] = np.nan
+    assert oracle.swiglu_quantize(ab)[2] == oracle.BIT_NONFINITE
+
+
+def test_swiglu_bwd_against_torch_autograd():
+    """[da | db] against torch autograd of silu(a) * b in float64, within a
+    few float32 roundings of each term's magnitude."""
+    M, F = 40, 256
+    ab = _swiglu_inputs(M, F, 13)
+    dh = workloads.normal((M, F), 1.0, 14)
+    dab = oracle.swiglu_bwd(ab, dh).astype(np.float64)
+    a = torch.from_numpy(ab[:, :F].astype(np.float64)).requires_grad_()
+    b = torch.from_numpy(ab[:, F:].astype(np.float64)).requires_grad_()
+    (torch.nn.functional.silu(a) * b).backward(torch.from_numpy(dh.astype(np.float64)))
+    a64, b64, g = a.detach().numpy(), b.detach().numpy(), dh.astype(np.float64)
+    sig = 1.0 / (1.0 + np.exp(-a64))
+    mag_a = np.abs(g * b64) * (sig + np.abs(a64) * sig * (1 - sig))
+    tiny = 1e-35 * np.abs(g) * (1 + np.abs(b64))  # e^-a overflow below a = -88.7
+    assert np.all(np.abs(dab[:, :F] - a.grad.numpy()) <= 10 * U32 * mag_a + tiny)
+    mag_b = np.abs(g * _silu64(a64))
+    assert np.all(np.abs(dab[:, F:] - b.grad.numpy()) <= 6 * U32 * mag_b + tiny)
