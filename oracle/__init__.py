@@ -70,6 +70,7 @@ def _declare(L):
                                     _P, _P, _U64, _P, _P, _P, _P]),
         "ref_sr_expectation_enum": (ctypes.c_double, [_F]),
         "ref_exp": (_F, [_F]),
+        "ref_fwd_quantized": (_U32, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P]),
         "ref_swiglu_h": (None, [_P, _I64, _I64, _I64, _P]),
         "ref_swiglu_quantize": (_U32, [_P, _I64, _I64, _I64, _P, _P]),
         "ref_swiglu_bwd": (None, [_P, _I64, _I64, _I64, _P, _P]),
@@ -175,6 +176,17 @@ def fwd(x, wq, sw, bias=None, B: int = 0):
     sx = np.empty((M,), np.float32)
     st = lib().ref_fwd(_p(x), M, K, _p(wq), _p(sw), N, _p(b), B, _p(y), _p(xq), _p(sx))
     return y, xq, sx, st
+
+
+def fwd_quantized(xq, sx, wq, sw, bias=None):
+    """The forward from codes and row scales: returns y (fp32 [M,N]), status."""
+    xq, sx, wq, sw = _i8(xq), _f32(sx), _i8(wq), _f32(sw)
+    M, K = xq.shape
+    N = wq.shape[0]
+    b = None if bias is None else _f32(bias)
+    y = np.empty((M, N), np.float32)
+    st = lib().ref_fwd_quantized(_p(xq), _p(sx), M, K, _p(wq), _p(sw), N, _p(b), _p(y))
+    return y, st
 
 
 def round_bf16(v: float) -> float:

@@ -313,6 +313,24 @@ uint32_t ref_fwd(const float *x, int64_t M, int64_t K, const int8_t *wq, const f
     return st;
 }
 
+/* The same forward from an input that is already quantized (codes xq [M,K]
+ * and row scales sx [M] in the layer's format, e.g. the SwiGLU gate's
+ * quantized h): y[m,n] = ((float)acc[m,n] * sx[m]) * s_w[n] + bias[n]. */
+uint32_t ref_fwd_quantized(const int8_t *xq, const float *sx, int64_t M, int64_t K,
+                           const int8_t *wq, const float *sw, int64_t N, const float *bias,
+                           float *y) {
+    if (K > ORC_MAX_CONTRACTION) return ORC_BIT_UNSUPP;
+    int32_t *acc = (int32_t *)malloc((size_t)(M * N > 0 ? M * N : 1) * sizeof(int32_t));
+    uint32_t st = ref_gemm_nt(xq, K, wq, K, M, N, K, acc, N);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float v = ((float)acc[m * N + n] * sx[m]) * sw[n];
+            y[m * N + n] = bias ? v + bias[n] : v;
+        }
+    free(acc);
+    return st;
+}
+
 /* ------------------------------------------------------------------ */
 /* The forward's bf16 route ([CR] third commit note, items 1 and 2: the  */
 /* activations are rotated instead of the weight being un-rotated, and   */

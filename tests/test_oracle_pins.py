@@ -805,3 +805,21 @@ def test_swiglu_bwd_against_torch_autograd():
     assert np.all(np.abs(dab[:, :F] - a.grad.numpy()) <= 10 * U32 * mag_a + tiny)
     mag_b = np.abs(g * _silu64(a64))
     assert np.all(np.abs(dab[:, F:] - b.grad.numpy()) <= 6 * U32 * mag_b + tiny)
+
+
+def test_fwd_quantized_is_the_forward_after_its_quantization():
+    """The forward from codes equals the whole forward when given the codes
+    and scales that the forward's own quantization produces (bit for bit),
+    and is the exact product for unit scales."""
+    x = workloads.normal((37, 256), 1.0, 31)
+    w = workloads.normal((48, 256), 0.02, 32)
+    b = workloads.normal((48,), 0.01, 33)
+    wq, sw, _ = oracle.quantize_rows(w, flags=oracle.REJECT_ZERO_ROWS)
+    y, xq, sx, st = oracle.fwd(x, wq, sw, b, 0)
+    y2, st2 = oracle.fwd_quantized(xq, sx, wq, sw, b)
+    assert st == st2 == 0 and np.array_equal(y, y2)
+    rng = np.random.Generator(np.random.PCG64(34))
+    xi = rng.integers(-127, 128, (5, 64)).astype(np.int8)
+    wi = rng.integers(-127, 128, (16, 64)).astype(np.int8)
+    y3, _ = oracle.fwd_quantized(xi, np.ones(5, np.float32), wi, np.ones(16, np.float32))
+    assert np.array_equal(y3, (xi.astype(np.int64) @ wi.astype(np.int64).T).astype(np.float32))
