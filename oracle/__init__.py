@@ -71,6 +71,10 @@ def _declare(L):
         "ref_sr_expectation_enum": (ctypes.c_double, [_F]),
         "ref_exp": (_F, [_F]),
         "ref_fwd_quantized": (_U32, [_P, _P, _I64, _I64, _P, _P, _I64, _P, _P]),
+        "ref_muon_momentum": (None, [_P, _P, _I64, _F, _P]),
+        "ref_newton_schulz5": (None, [_P, _I64, _I64, ctypes.c_int, _P]),
+        "ref_update_muon_sr": (_U32, [_P, _P, _P, _I64, _I64, _I64, _F, _F, _U64, _U64, _I64]),
+        "ref_adamw_vector": (_U32, [_P, _P, _P, _P, _I64, _F, _F, _F, _F, _F, _U64]),
         "ref_swiglu_h": (None, [_P, _I64, _I64, _I64, _P]),
         "ref_swiglu_quantize": (_U32, [_P, _I64, _I64, _I64, _P, _P]),
         "ref_swiglu_bwd": (None, [_P, _I64, _I64, _I64, _P, _P]),
@@ -347,3 +351,42 @@ def swiglu_bwd(ab: np.ndarray, dh: np.ndarray) -> np.ndarray:
     dab = np.empty((M, F2), np.float32)
     lib().ref_swiglu_bwd(_p(ab), M, F, F2, _p(dh), _p(dab))
     return dab
+
+
+# ---------------------------------------------------------------- MuonAuxAdamW
+def muon_momentum(G, M, beta: float = 0.95):
+    """Returns (M', U): the new momentum and the Nesterov-blended update."""
+    G = _f32(G)
+    M2 = _f32(M).copy()
+    U = np.empty_like(G)
+    lib().ref_muon_momentum(_p(G), _p(M2), G.size, beta, _p(U))
+    return M2, U
+
+
+def newton_schulz5(U, steps: int = 5) -> np.ndarray:
+    """The orthogonalized update NS5(U) in float64 [R, C]."""
+    U = _f32(U)
+    R, C = U.shape
+    O = np.empty((R, C), np.float64)
+    lib().ref_newton_schulz5(_p(U), R, C, steps, _p(O))
+    return O
+
+
+def update_muon_sr(q, s, O, lr: float, wd: float, seed: int, step: int, n_full=None,
+                   row0: int = 0):
+    """One Muon step with stochastic requantization from the float32 update O;
+    returns the new (q, s, status) as copies.  n_full: rows of the whole weight
+    (for the max(1, N/K)^0.5 factor) when q holds a slice of rows from row0."""
+    q, s, O = _i8(q).copy(), _f32(s).copy(), _f32(O)
+    N, K = q.shape
+    st = lib().ref_update_muon_sr(_p(q), _p(s), _p(O), N, K, N if n_full is None else n_full,
+                                  lr, wd, seed, step, row0)
+    return q, s, st
+
+
+def adamw_vector(p, g, m, v, lr: float, step: int, b1=0.9, b2=0.999, eps=1e-8, wd=0.0):
+    """AdamW on a float32 vector; returns new (p, m, v, status)."""
+    p, g = _f32(p).copy(), _f32(g)
+    m, v = _f32(m).copy(), _f32(v).copy()
+    st = lib().ref_adamw_vector(_p(p), _p(g), _p(m), _p(v), p.size, lr, b1, b2, eps, wd, step)
+    return p, m, v, st

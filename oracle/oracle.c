@@ -802,3 +802,130 @@ void ref_swiglu_bwd(const float *ab, int64_t M, int64_t F, int64_t ldab, const f
             dab[m * 2 * F + F + f] = g * silu;
         }
 }
+
+/* ------------------------------------------------------------------ */
+/* MuonAuxAdamW ([QT] feature table, row "Optimizers": the third update  */
+/* path it names).  The pages give only the name; the definition        */
+/* followed is the published Muon optimizer (K. Jordan, Y. Jin, V. Boza,  */
+/* J. You, F. Cesista, L. Newhouse, J. Bernstein, "Muon: An optimizer for */
+/* hidden layers in neural networks", 2024) for the 2-D weights, with     */
+/* AdamW for the float parameters (biases, magnitudes):                   */
+/*   M' = beta*M + (1-beta)*G,  U = (1-beta)*G + beta*M'   (Nesterov)     */
+/*   O = NS5(U): quintic Newton-Schulz on U/||U||_F, 5 steps              */
+/*   w' = w*(1 - lr*wd) - lr*max(1, N/K)^0.5 * O, then the layer's         */
+/*   stochastic requantization of each row.                               */
+/* ------------------------------------------------------------------ */
+
+/* Momentum and Nesterov blend, float32, one rounding per operation in the
+ * order written; omb = fl32(1 - beta) computed in float64.  M is updated in
+ * place; U receives the blended update. */
+void ref_muon_momentum(const float *G, float *M, int64_t n, float beta, float *U) {
+    const float omb = (float)(1.0 - (double)beta);
+    for (int64_t i = 0; i < n; ++i) {
+        const float m = beta * M[i] + omb * G[i];
+        M[i] = m;
+        U[i] = omb * G[i] + beta * m;
+    }
+}
+
+/* O = NS5(U) in float64.  X = U, or U^T when U has more rows than columns
+ * (so X is r x c with r <= c); X = X / (||X||_F + 1e-7); then `steps` times
+ *   A = X X^T;  B = b*A + c*(A A);  X = a*X + B X
+ * with (a, b, c) = (3.4445, -4.7750, 2.0315); O = X (transposed back).
+ * Acting on the singular values alone, each step maps s -> a s + b s^3 +
+ * c s^5, so O = U_svd p(S/(||U||_F + 1e-7)) V_svd^T with p the step applied
+ * `steps` times.  U [R, C] float row-major, O [R, C] double row-major. */
+void ref_newton_schulz5(const float *U, int64_t R, int64_t C, int steps, double *O) {
+    const double a = 3.4445, b = -4.7750, c = 2.0315;
+    const int tr = R > C;
+    const int64_t r = tr ? C : R, cc = tr ? R : C;
+    double *X = (double *)malloc((size_t)(r * cc > 0 ? r * cc : 1) * sizeof(double));
+    double *Y = (double *)malloc((size_t)(r * cc > 0 ? r * cc : 1) * sizeof(double));
+    double *A = (double *)malloc((size_t)(r * r > 0 ? r * r : 1) * sizeof(double));
+    double *B = (double *)malloc((size_t)(r * r > 0 ? r * r : 1) * sizeof(double));
+    double nrm = 0.0;
+    for (int64_t i = 0; i < r; ++i)
+        for (int64_t j = 0; j < cc; ++j) {
+            const double v = tr ? (double)U[j * C + i] : (double)U[i * C + j];
+            X[i * cc + j] = v;
+            nrm += v * v;
+        }
+    nrm = sqrt(nrm) + 1e-7;
+    for (int64_t i = 0; i < r * cc; ++i) X[i] /= nrm;
+    for (int s = 0; s < steps; ++s) {
+        for (int64_t i = 0; i < r; ++i)           /* A = X X^T */
+            for (int64_t j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < cc; ++k) acc += X[i * cc + k] * X[j * cc + k];
+                A[i * r + j] = acc;
+            }
+        for (int64_t i = 0; i < r; ++i)           /* B = b A + c A A */
+            for (int64_t j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < r; ++k) acc += A[i * r + k] * A[k * r + j];
+                B[i * r + j] = b * A[i * r + j] + c * acc;
+            }
+        for (int64_t i = 0; i < r; ++i)           /* X = a X + B X */
+            for (int64_t j = 0; j < cc; ++j) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < r; ++k) acc += B[i * r + k] * X[k * cc + j];
+                Y[i * cc + j] = a * X[i * cc + j] + acc;
+            }
+        double *t = X;
+        X = Y;
+        Y = t;
+    }
+    for (int64_t i = 0; i < r; ++i)
+        for (int64_t j = 0; j < cc; ++j) {
+            if (tr) O[j * C + i] = X[i * cc + j];
+            else O[i * C + j] = X[i * cc + j];
+        }
+    free(X);
+    free(Y);
+    free(A);
+    free(B);
+}
+
+/* One Muon step of an int8 weight [N, K] with stochastic requantization, in
+ * place, from the orthogonalized update O (float32 [N, K]):
+ *   w = s*q;  w' = w*a - st*O,  a = fl32(1 - lr*wd), st = fl32(lr*max(1, N/K)^0.5)
+ * (constants in float64, rounded once; per element one rounding per
+ * operation), then per row s' = max|w'|/127 and the codes by the same
+ * Philox-keyed stochastic rounding as ref_update_sr (row index n0 + n keys
+ * the stream).  The scale factor uses the whole weight's N and K (Nfull),
+ * which a slice of rows does not change. */
+uint32_t ref_update_muon_sr(int8_t *q, float *s, const float *O, int64_t N, int64_t K,
+                            int64_t Nfull, float lr, float wd, uint64_t seed, uint64_t step,
+                            int64_t n0) {
+    if (step < 1) return ORC_BIT_ARG;
+    const double scale = Nfull > K ? sqrt((double)Nfull / (double)K) : 1.0;
+    const float a = (float)(1.0 - (double)lr * (double)wd);
+    const float st = (float)((double)lr * scale);
+    uint32_t status = 0;
+    float *w = (float *)malloc((size_t)(K > 0 ? K : 1) * sizeof(float));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            const float wv = s[n] * (float)q[n * K + k];
+            w[k] = wv * a - st * O[n * K + k];
+        }
+        status |= sr_requant_row(w, K, n0 + n, seed, step, q + n * K, &s[n]);
+    }
+    free(w);
+    return status;
+}
+
+/* AdamW on a float32 vector (the "aux" optimizer of MuonAuxAdamW for biases
+ * and other float parameters): the same per-element arithmetic and host
+ * constants as the int8 weights' AdamW (ref_update_sr), without
+ * requantization. */
+uint32_t ref_adamw_vector(float *p, const float *g, float *m, float *v, int64_t n, float lr,
+                          float b1, float b2, float eps, float wd, uint64_t step) {
+    if (step < 1) return ORC_BIT_ARG;
+    adamw_consts c = adamw_setup(lr, b1, b2, eps, wd, step);
+    uint32_t st = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        p[i] = adamw_elem(&c, p[i], g[i], &m[i], &v[i]);
+        if (!isfinite(p[i])) st |= ORC_BIT_NONFINITE;
+    }
+    return st;
+}

@@ -823,3 +823,96 @@ def test_fwd_quantized_is_the_forward_after_its_quantization():
     wi = rng.integers(-127, 128, (16, 64)).astype(np.int8)
     y3, _ = oracle.fwd_quantized(xi, np.ones(5, np.float32), wi, np.ones(16, np.float32))
     assert np.array_equal(y3, (xi.astype(np.int64) @ wi.astype(np.int64).T).astype(np.float32))
+
+
+# ---------------------------------------------------------------- MuonAuxAdamW
+NS_COEF = (3.4445, -4.7750, 2.0315)
+
+
+def _ns5_by_svd(U, steps=5):
+    """The quintic Newton-Schulz map acts on singular values only: the same
+    O from numpy's SVD and the scalar iteration s -> a s + b s^3 + c s^5."""
+    a, b, c = NS_COEF
+    U64 = U.astype(np.float64)
+    u, sv, vt = np.linalg.svd(U64, full_matrices=False)
+    x = sv / (np.linalg.norm(U64) + 1e-7)
+    for _ in range(steps):
+        x = a * x + b * x ** 3 + c * x ** 5
+    return (u * x) @ vt
+
+
+@pytest.mark.parametrize("R,C", [(48, 80), (80, 48), (64, 64), (1, 32)])
+def test_newton_schulz_matches_the_svd_closed_form(R, C):
+    U = workloads.normal((R, C), 1e-3, R * 7 + C)
+    O = oracle.newton_schulz5(U)
+    ref = _ns5_by_svd(U)
+    assert np.abs(O - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    # after five steps every singular value sits in the iteration's band
+    sv = np.linalg.svd(O, compute_uv=False)
+    assert sv.min() > 0.6 and sv.max() < 1.25
+
+
+def test_newton_schulz_zero_and_one_step():
+    assert not oracle.newton_schulz5(np.zeros((8, 16), np.float32)).any()
+    U = workloads.normal((16, 24), 1.0, 3)
+    O1 = oracle.newton_schulz5(U, steps=1)
+    assert np.abs(O1 - _ns5_by_svd(U, steps=1)).max() <= 1e-12
+
+
+def test_muon_momentum_against_torch_lerp():
+    """M' and the Nesterov blend against torch's lerp form in float64 (the
+    published implementation's momentum.lerp_(g, 1-beta); g.lerp_(m, beta)),
+    within float32 roundings of each term."""
+    G = workloads.normal((64, 96), 1e-3, 4)
+    M = workloads.normal((64, 96), 1e-3, 5)
+    M2, U = oracle.muon_momentum(G, M, 0.95)
+    g, m = torch.from_numpy(G.astype(np.float64)), torch.from_numpy(M.astype(np.float64))
+    m.lerp_(g, 1 - 0.95)
+    u = g.clone().lerp_(m, 0.95)
+    mag = np.abs(G.astype(np.float64)) + np.abs(M.astype(np.float64))
+    assert np.all(np.abs(M2 - m.numpy()) <= 4 * 2.0 ** -24 * mag)
+    assert np.all(np.abs(U - u.numpy()) <= 8 * 2.0 ** -24 * mag)
+    # beta = 0: plain gradient, exactly
+    M3, U3 = oracle.muon_momentum(G, M, 0.0)
+    assert np.array_equal(M3, G) and np.array_equal(U3, G)
+
+
+def test_muon_update_step_and_requant():
+    """The float step w*(1-lr*wd) - lr*max(1,N/K)^0.5*O against torch's
+    mul_/add_ in float64; a zero update with no decay leaves every code and
+    scale unchanged; the stochastic rounding is that of the other updates."""
+    N, K = 96, 64   # N > K: the step size is scaled by sqrt(N/K)
+    w = workloads.normal((N, K), 0.02, 6)
+    q, s, _ = oracle.quantize_rows(w, flags=oracle.REJECT_ZERO_ROWS)
+    O = workloads.normal((N, K), 0.1, 7)
+    lr, wd = 0.02, 0.01
+    q2, s2, st = oracle.update_muon_sr(q, s, O, lr, wd, seed=9, step=3)
+    assert st == 0
+    p = torch.from_numpy(q.astype(np.float64) * s[:, None].astype(np.float64))
+    p.mul_(1 - lr * wd).add_(torch.from_numpy(O.astype(np.float64)), alpha=-lr * math.sqrt(N / K))
+    ref = p.numpy()
+    # dequantized new codes within one code step of the torch value per row
+    deq = q2.astype(np.float64) * s2[:, None].astype(np.float64)
+    assert np.all(np.abs(deq - ref) <= s2[:, None] * (1 + 1e-5))
+    q3, s3, st = oracle.update_muon_sr(q, s, np.zeros_like(O), lr, 0.0, seed=9, step=3)
+    assert st == 0 and np.array_equal(q3, q) and np.array_equal(s3, s)
+
+
+def test_adamw_vector_matches_torch():
+    n = 300
+    p0 = workloads.normal((n,), 0.01, 8)
+    g = workloads.normal((n,), 1e-3, 9)
+    m = workloads.normal((n,), 1e-4, 10)
+    v = np.square(workloads.normal((n,), 1e-3, 11))
+    p1, m1, v1, st = oracle.adamw_vector(p0, g, m, v, 1e-3, step=10, wd=0.01)
+    assert st == 0
+    t = torch.from_numpy(p0.astype(np.float64)).requires_grad_()
+    opt = torch.optim.AdamW([t], lr=float(np.float32(1e-3)), weight_decay=float(np.float32(0.01)),
+                            betas=(float(np.float32(0.9)), float(np.float32(0.999))),
+                            eps=float(np.float32(1e-8)))
+    opt.state[t]["step"] = torch.tensor(9.0, dtype=torch.float64)
+    opt.state[t]["exp_avg"] = torch.from_numpy(m.astype(np.float64))
+    opt.state[t]["exp_avg_sq"] = torch.from_numpy(v.astype(np.float64))
+    t.grad = torch.from_numpy(g.astype(np.float64))
+    opt.step()
+    assert np.all(np.abs(p1 - t.detach().numpy()) <= 1e-6 * (np.abs(p0) + 1e-3))
