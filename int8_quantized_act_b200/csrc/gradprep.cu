@@ -134,13 +134,11 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   const int t0 = blockIdx.y * tiles_per_cta;
   const int t1 = t0 + tiles_per_cta < tiles ? t0 + tiles_per_cta : tiles;
   const int col = cb * kCols + lane * 8;
-  // Maxima as floats: fmaxf with an |x| operand is one instruction where the
-  // bit-pattern max takes two; for finite values both give the same bits.
-  // fmaxf drops NaN, so non-finite inputs are also caught through the
-  // column sums: a lane's float partial sum stays finite unless an input is
-  // NaN or infinite (an infinite dY in a row whose s_x is 0 makes a NaN
-  // product, which the maximum drops, but an infinite sum) or the float sum
-  // itself overflows, when db is not finite either.
+  // Maxima as floats with NaN-propagating max (max.NaN.f32) over |x|
+  // operands: a NaN or infinite product dY*s_x (an infinite dY in a row whose
+  // s_x is 0 gives NaN) makes its column maximum NaN or +inf, and likewise
+  // dY*s_w for the row maxima, which is exactly when the layer's definition
+  // reports a non-finite value.  The column sums only feed db.
   float mx[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   float sm[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   uint32_t rbad = 0;
@@ -165,37 +163,45 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
     load_scales(t0, fcur);
     ring.consume(t0, t1, lane, [&](int t, const uint8_t* tile) {
       load_scales(t + 1, fnext);
+      // Two rows per step, so one three-operand max covers both.  Rows of
+      // the tile past M were zero-filled by the copy and their factors are
+      // 0: they add nothing to the column maxima and sums.
 #pragma unroll
-      for (int j = 0; j < T::kRowsPerWarp; ++j) {
+      for (int j = 0; j < T::kRowsPerWarp; j += 2) {
         const int r = warp * T::kRowsPerWarp + j;
         const int64_t m = static_cast<int64_t>(t) * T::kRows + r;
-        if (m < M) {  // warp-uniform
-          float d[8];
-          smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
-          const float f = fcur[j];
-          float rbf = 0.0f;
-          // Two columns per step: the products (only their magnitudes are
-          // used, no sum follows them) and the column sums as packed pairs.
+        float d0[8], d1[8];
+        smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d0);
+        smem_load8<InT>(tile + (r + 1) * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d1);
+        const float f0 = fcur[j], f1 = fcur[j + 1];
+        float rb0 = 0.0f, rb1 = 0.0f;
+        // Products (only their magnitudes are used, no sum follows them) and
+        // column sums two columns per instruction.
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) {
-            const float2 dd = make_float2(d[i], d[i + 1]);
-            const float2 p = mul2(dd, make_float2(f, f));
-            mx[i] = fmaxf(mx[i], fabsf(p.x));
-            mx[i + 1] = fmaxf(mx[i + 1], fabsf(p.y));
-            const float2 ss = add2(make_float2(sm[i], sm[i + 1]), dd);
-            sm[i] = ss.x;
-            sm[i + 1] = ss.y;
-            if (ROWMAX) {
-              const float2 r2 = mul2(dd, make_float2(w8[i], w8[i + 1]));
-              rbf = fmaxf(rbf, fmaxf(fabsf(r2.x), fabsf(r2.y)));
-            }
-          }
+        for (int i = 0; i < 8; i += 2) {
+          const float2 a = make_float2(d0[i], d0[i + 1]), b = make_float2(d1[i], d1[i + 1]);
+          const float2 pa = mul2(a, make_float2(f0, f0)), pb = mul2(b, make_float2(f1, f1));
+          mx[i] = fmax3_nan(mx[i], fabsf(pa.x), fabsf(pb.x));
+          mx[i + 1] = fmax3_nan(mx[i + 1], fabsf(pa.y), fabsf(pb.y));
+          const float2 ss = add2(add2(make_float2(sm[i], sm[i + 1]), a), b);
+          sm[i] = ss.x;
+          sm[i + 1] = ss.y;
           if (ROWMAX) {
-            // Non-negative floats order like their bit patterns.
-            uint32_t rb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(rbf));
-            if (lane == 0) atomicMax(rowmax + m, rb);
-            rbad = max(rbad, rb);
+            const float2 wv = make_float2(w8[i], w8[i + 1]);
+            const float2 ra = mul2(a, wv), rv = mul2(b, wv);
+            rb0 = fmax3_nan(rb0, fabsf(ra.x), fabsf(ra.y));
+            rb1 = fmax3_nan(rb1, fabsf(rv.x), fabsf(rv.y));
           }
+        }
+        if (ROWMAX) {
+          // Non-negative floats order like their bit patterns; NaN sorts last.
+          const uint32_t u0 = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(rb0));
+          const uint32_t u1 = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(rb1));
+          if (lane == 0) {
+            if (m < M) atomicMax(rowmax + m, u0);
+            if (m + 1 < M) atomicMax(rowmax + m + 1, u1);
+          }
+          rbad = max(rbad, max(u0, u1));
         }
       }
 #pragma unroll
@@ -215,17 +221,14 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
     const int slot = (tid % 8) * 32 + tid / 8;
     uint32_t a = 0;
     double t = 0.0;
-    bool bad = false;
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       a = max(a, s_max[w][slot]);
-      const float part = s_sum[w][slot];
-      bad |= !isfinite(part);
-      t += static_cast<double>(part);
+      t += static_cast<double>(s_sum[w][slot]);
     }
-    // An infinite maximum or a non-finite partial sum: report it (the
-    // affected outputs are unspecified).
-    if (a >= kInfBits || bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    // A NaN or infinite maximum: report it (the affected outputs are
+    // unspecified).
+    if (a >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
     atomicMax(colmax + cb * kCols + tid, a);
     atomicAdd(colsum + cb * kCols + tid, t);
   }

@@ -283,6 +283,25 @@ __device__ __forceinline__ void fwht128_wide(float (&v)[32], int lane, float c) 
   }
 }
 
+// -------------------------------------------------------------- NaN-aware maxima
+// max(a, b) that is NaN whenever an operand is NaN (max.NaN.f32), where
+// fmaxf would drop the NaN.  With |x| operands the running maximum of a row
+// or column is then NaN as soon as one element is NaN and +inf when one is
+// infinite, so a single compare of its bit pattern against kInfBits tells
+// whether a non-finite value was met.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// The three-operand form (sm_100): max(a, b, c), NaN if any operand is NaN.
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // -------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
