@@ -1,7 +1,7 @@
 // noalloc.cu - qlinear_bwd_dx_noalloc: the input-gradient call for callers
 // that cannot allocate device memory (see include/qlinear.h).  Its scratch is
 // a fixed array in this file's device image instead of a caller workspace.
-#include <mutex>
+#include <atomic>
 
 #include "launch.h"
 #include "../../include/qlinear.h"
@@ -15,25 +15,32 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[QL_NOALLOC_SCRA
 
 constexpr int kMaxDevices = 64;
 
-struct DeviceScratch {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
+// Device address of the array, per device; null until a lookup succeeded.
+std::atomic<void*> g_scratch[kMaxDevices];
 
-DeviceScratch g_scratch[kMaxDevices];
-
-// Device address of the scratch array on the current device, looked up once
-// per device with that device current.
+// Device address of the scratch array on the current device.  The lookup runs
+// with that device current and only a successful one is kept, so a lookup
+// that failed (for example because the library's device code could not be
+// loaded while memory was short) is tried again by the next call.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e;
+  }
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  DeviceScratch& d = g_scratch[dev];
-  std::call_once(d.once, [&d] { d.err = cudaGetSymbolAddress(&d.ptr, g_noalloc_scratch); });
-  if (d.err != cudaSuccess) return d.err;
-  *out = d.ptr;
+  void* p = g_scratch[dev].load(std::memory_order_acquire);
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();  // clear the failed call's error for later calls
+      return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+    }
+    // Two threads may both look it up; they store the same address.
+    g_scratch[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
   return cudaSuccess;
 }
 
@@ -43,8 +50,13 @@ extern "C" int qlinear_bwd_dx_noalloc(const void* dy, int dyt, int64_t M, int64_
                                       const int8_t* wq, const float* sw, int64_t K,
                                       int hadamard_block, void* dx, int dxt, int32_t* d_status,
                                       void* stream) {
-  if (M >= 0 && N >= 0 && K >= 0 &&
-      qlinear_workspace_bytes(M, N, K, hadamard_block) > QL_NOALLOC_SCRATCH_BYTES)
+  // The argument and shape checks of qlinear_bwd_dx first, so both calls
+  // return the same code for the same mistake; then the capacity.
+  bool noop = false;
+  const int pre = ql::check_bwd_dx_args(dy, dyt, M, N, wq, sw, K, hadamard_block, dx, dxt,
+                                        d_status, &noop);
+  if (pre != QL_OK || noop) return pre;
+  if (qlinear_workspace_bytes(M, N, K, hadamard_block) > QL_NOALLOC_SCRATCH_BYTES)
     return QL_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return QL_ERR_CUDA;
