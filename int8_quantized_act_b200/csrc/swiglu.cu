@@ -1,0 +1,244 @@
+// swiglu.cu - the SwiGLU gate of the MLP whose three projections run through
+// this layer (w1 and w3 stacked as one call on the same input, w2 on h):
+// h = silu(a) * b with silu(a) = a / (1 + e^-a).
+//
+// Forward: one kernel reads the stacked pre-activations [a | b] (the stacked
+// projection's output) and writes the second projection's saved input
+// directly, h quantized per row (int8 codes and s_h), so h itself never goes
+// to memory.  Backward: one elementwise kernel turns dh (the second
+// projection's input gradient) into [da | db], the stacked projection's
+// output gradient.
+//
+// e^x is evaluated with fixed float32 steps so that codes decided through it
+// are reproducible bit for bit: Cody and Waite's argument reduction (W. J.
+// Cody, W. Waite, "Software Manual for the Elementary Functions", 1980),
+// n = rint(x log2 e), r = (x - n C1) - n C2 with C1 = fl32(ln 2) and C2 the
+// remainder, each a correctly rounded fused multiply-add; e^r by the Taylor
+// series to degree 7 in Horner form (fused multiply-adds); times 2^n as the
+// product of two exact powers of two.  x is clamped to [-104, 89] first.
+#include <algorithm>
+
+#include "launch.h"
+#include "rowops.cuh"
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+namespace {
+
+// e^x of two values at once: packed f32x2 multiplies and fused multiply-adds,
+// each half one correctly rounded operation, so each result is that of the
+// scalar steps in the file comment; a NaN input gives NaN.
+__device__ __forceinline__ float2 exp_cw2(float2 x) {
+  const float x0 = x.x > 89.0f ? 89.0f : (x.x < -104.0f ? -104.0f : x.x);
+  const float x1 = x.y > 89.0f ? 89.0f : (x.y < -104.0f ? -104.0f : x.y);
+  const float2 y = mul2(make_float2(x0, x1), make_float2(0x1.715476p+0f, 0x1.715476p+0f));
+  const float nf0 = rintf(y.x), nf1 = rintf(y.y);
+  const float2 mn = make_float2(-nf0, -nf1);
+  float2 r = fma2(mn, make_float2(0x1.62e43p-1f, 0x1.62e43p-1f), make_float2(x0, x1));
+  r = fma2(mn, make_float2(-0x1.05c61p-29f, -0x1.05c61p-29f), r);
+  float2 p = make_float2(0x1.a01a02p-13f, 0x1.a01a02p-13f);
+  p = fma2(p, r, make_float2(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
+  p = fma2(p, r, make_float2(0x1.111112p-7f, 0x1.111112p-7f));
+  p = fma2(p, r, make_float2(0x1.555556p-5f, 0x1.555556p-5f));
+  p = fma2(p, r, make_float2(0x1.555556p-3f, 0x1.555556p-3f));
+  p = fma2(p, r, make_float2(0.5f, 0.5f));
+  p = fma2(p, r, make_float2(1.0f, 1.0f));
+  p = fma2(p, r, make_float2(1.0f, 1.0f));
+  const int n0 = static_cast<int>(nf0), n1 = static_cast<int>(nf1);
+  const int a0 = n0 / 2, a1 = n1 / 2;
+  const float2 f1 = make_float2(__int_as_float((a0 + 127) << 23), __int_as_float((a1 + 127) << 23));
+  const float2 f2 = make_float2(__int_as_float((n0 - a0 + 127) << 23),
+                                __int_as_float((n1 - a1 + 127) << 23));
+  float2 e = mul2(mul2(p, f1), f2);
+  if (x.x != x.x) e.x = x.x;
+  if (x.y != x.y) e.y = x.y;
+  return e;
+}
+
+constexpr int kGateThreads = 256;
+constexpr int kGatePiece = 8;                          // columns per thread per piece
+constexpr int kGateSpan = kGateThreads * kGatePiece;   // 2048 columns per piece
+
+// One CTA per row of [a | b] (persistent over rows): thread t owns columns
+// j * 2048 + 8t .. +7 of h for pieces j < P, read with 16-byte loads (a warp
+// reads 512 contiguous bytes of a and of b per piece); the row maximum of |h|
+// is a NaN-propagating max, reduced over the warps through shared memory;
+// the codes are stored 8 at a time.
+template <typename InT, int P>
+__global__ void __launch_bounds__(kGateThreads) swiglu_quant_kernel(
+    const InT* __restrict__ ab, int64_t M, int F, int64_t ldab, int8_t* __restrict__ hq,
+    int64_t ldh, float* __restrict__ sh, int32_t* __restrict__ status) {
+  __shared__ uint32_t s_wmax[2][kGateThreads / 32];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  int par = 0;
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x, par ^= 1) {
+    const InT* ra = ab + m * ldab;
+    const InT* rb = ra + F;
+    float h[P][kGatePiece];
+    float mx0 = 0.0f, mx1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      const int col = j * kGateSpan + t * kGatePiece;
+      if (col < F) {
+        float a8[8], b8[8];
+        load8(ra + col, a8);
+        load8(rb + col, b8);
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const float2 e = exp_cw2(make_float2(-a8[k], -a8[k + 1]));
+          h[j][k] = __fmul_rn(__fdiv_rn(a8[k], __fadd_rn(1.0f, e.x)), b8[k]);
+          h[j][k + 1] = __fmul_rn(__fdiv_rn(a8[k + 1], __fadd_rn(1.0f, e.y)), b8[k + 1]);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) h[j][k] = 0.0f;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; k += 4) {
+        mx0 = fmax3_nan(mx0, fabsf(h[j][k]), fabsf(h[j][k + 1]));
+        mx1 = fmax3_nan(mx1, fabsf(h[j][k + 2]), fabsf(h[j][k + 3]));
+      }
+    }
+    // Non-negative floats order like their bit patterns; NaN sorts last.
+    uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fmax_nan(mx0, mx1)));
+    if (lane == 0) s_wmax[par][warp] = mb;
+    // Rows alternate between the two halves of s_wmax: this half is written
+    // again only after the next row's barrier, which every thread reaches
+    // after reading it here.
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kGateThreads / 32; ++w) mb = max(mb, s_wmax[par][w]);
+    const float amax = __uint_as_float(mb);
+    const float inv = mb == 0 ? 0.0f : 127.0f / amax;
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      const int col = j * kGateSpan + t * kGatePiece;
+      if (col < F) *reinterpret_cast<uint2*>(hq + m * ldh + col) = codes8(h[j], inv);
+    }
+    if (t == 0) {
+      sh[m] = mb == 0 ? 0.0f : amax / 127.0f;
+      if (mb >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    }
+  }
+}
+
+// [da | db] from [a | b] and dh, 8 columns per thread-step:
+//   d = 1 + e^-a, sigma = 1/d, silu = a/d,
+//   da = (dh * b) * (sigma * (1 + a * (1 - sigma))),  db = dh * silu.
+template <typename InT, typename GT, typename OutT>
+__global__ void __launch_bounds__(256) swiglu_bwd_kernel(const InT* __restrict__ ab, int64_t ldab,
+                                                         const GT* __restrict__ dh, int64_t M,
+                                                         int F, OutT* __restrict__ dab) {
+  const int64_t per_row = F / 8;
+  const int64_t total = M * per_row;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += stride) {
+    const int64_t m = i / per_row;
+    const int col = static_cast<int>(i - m * per_row) * 8;
+    float a8[8], b8[8], g8[8], da[8], db[8];
+    load8(ab + m * ldab + col, a8);
+    load8(ab + m * ldab + F + col, b8);
+    load8(dh + m * F + col, g8);
+    float ek[8];
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      const float2 e = exp_cw2(make_float2(-a8[k], -a8[k + 1]));
+      ek[k] = e.x;
+      ek[k + 1] = e.y;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float a = a8[k];
+      const float d = __fadd_rn(1.0f, ek[k]);
+      const float sigma = __fdiv_rn(1.0f, d);
+      const float silu = __fdiv_rn(a, d);
+      const float ds = __fmul_rn(sigma, __fadd_rn(1.0f, __fmul_rn(a, __fsub_rn(1.0f, sigma))));
+      da[k] = __fmul_rn(__fmul_rn(g8[k], b8[k]), ds);
+      db[k] = __fmul_rn(g8[k], silu);
+    }
+    store8(dab + m * 2 * static_cast<int64_t>(F) + col, da);
+    store8(dab + m * 2 * static_cast<int64_t>(F) + F + col, db);
+  }
+}
+
+template <typename InT, int P>
+cudaError_t gate_quant_t(const void* ab, int64_t M, int F, int64_t ldab, int8_t* hq, int64_t ldh,
+                         float* sh, int32_t* st, cudaStream_t s) {
+  auto kern = swiglu_quant_kernel<InT, P>;
+  static int occ[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int per_sm = dev < 64 ? __atomic_load_n(&occ[dev], __ATOMIC_ACQUIRE) : 0;
+  if (per_sm <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGateThreads, 0) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    if (dev < 64) __atomic_store_n(&occ[dev], per_sm, __ATOMIC_RELEASE);
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(M, static_cast<int64_t>(device_info().sms) * per_sm));
+  kern<<<grid, kGateThreads, 0, s>>>(reinterpret_cast<const InT*>(ab), M, F, ldab, hq, ldh, sh, st);
+  return cudaGetLastError();
+}
+
+template <typename InT>
+cudaError_t gate_quant_p(const void* ab, int64_t M, int F, int64_t ldab, int8_t* hq, int64_t ldh,
+                         float* sh, int32_t* st, cudaStream_t s) {
+  switch ((F + kGateSpan - 1) / kGateSpan) {
+    case 1: return gate_quant_t<InT, 1>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    case 2: return gate_quant_t<InT, 2>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    case 3: return gate_quant_t<InT, 3>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    case 4: return gate_quant_t<InT, 4>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    case 5: return gate_quant_t<InT, 5>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    case 6: return gate_quant_t<InT, 6>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    case 7: return gate_quant_t<InT, 7>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    case 8: return gate_quant_t<InT, 8>(ab, M, F, ldab, hq, ldh, sh, st, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename InT, typename GT>
+cudaError_t gate_bwd_o(const void* ab, int64_t ldab, const void* dh, int64_t M, int F, void* dab,
+                       int dabt, cudaStream_t s) {
+  const int64_t total = M * (F / 8);
+  const int grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(device_info().sms) * 8)));
+  const InT* a = reinterpret_cast<const InT*>(ab);
+  const GT* g = reinterpret_cast<const GT*>(dh);
+  if (dabt == QL_BF16)
+    swiglu_bwd_kernel<InT, GT, __nv_bfloat16><<<grid, 256, 0, s>>>(
+        a, ldab, g, M, F, reinterpret_cast<__nv_bfloat16*>(dab));
+  else
+    swiglu_bwd_kernel<InT, GT, float><<<grid, 256, 0, s>>>(a, ldab, g, M, F,
+                                                           reinterpret_cast<float*>(dab));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_swiglu_quant(const void* ab, int abt, int64_t M, int64_t F, int64_t ldab,
+                                int8_t* hq, int64_t ldh, float* sh, int32_t* st, cudaStream_t s) {
+  const cudaError_t e =
+      abt == QL_BF16
+          ? gate_quant_p<__nv_bfloat16>(ab, M, static_cast<int>(F), ldab, hq, ldh, sh, st, s)
+          : gate_quant_p<float>(ab, M, static_cast<int>(F), ldab, hq, ldh, sh, st, s);
+  count_launches(1);
+  return e;
+}
+
+cudaError_t launch_swiglu_bwd(const void* ab, int abt, int64_t ldab, const void* dh, int dht,
+                              int64_t M, int64_t F, void* dab, int dabt, cudaStream_t s) {
+  const int f = static_cast<int>(F);
+  cudaError_t e;
+  if (abt == QL_BF16)
+    e = dht == QL_BF16 ? gate_bwd_o<__nv_bfloat16, __nv_bfloat16>(ab, ldab, dh, M, f, dab, dabt, s)
+                       : gate_bwd_o<__nv_bfloat16, float>(ab, ldab, dh, M, f, dab, dabt, s);
+  else
+    e = dht == QL_BF16 ? gate_bwd_o<float, __nv_bfloat16>(ab, ldab, dh, M, f, dab, dabt, s)
+                       : gate_bwd_o<float, float>(ab, ldab, dh, M, f, dab, dabt, s);
+  count_launches(1);
+  return e;
+}
+
+}  // namespace ql

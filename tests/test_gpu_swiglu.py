@@ -1,13 +1,18 @@
-"""GPU parity of the SwiGLU MLP's projections at full size: 8192 tokens,
-d_model 4096, d_ff 14336, bf16 activations and gradients, no rotation.
+"""GPU parity of the SwiGLU MLP at full size: 8192 tokens, d_model 4096,
+d_ff 14336, bf16 activations and gradients, no rotation.
 
 w1 and w3 act on the same input, so they are stacked into one [2*d_ff,
 d_model] weight and X is quantized once for both; with per-row weight
 scales the stacked call gives exactly the two separate calls' outputs
-(checked below).  Each call is checked against the oracle on its own seeded
-inputs: saved codes and scales in full and bit for bit, float outputs on
-sampled rows (and sampled weight-gradient rows) within the 1e-3 relative
-bound plus half a bf16 ulp."""
+(checked below).  The gate h = silu(a) * b runs fused with the second
+projection's input quantization (qlinear_swiglu_quantize: h codes and
+scales bit for bit against the oracle at full size), the second projection
+takes those codes (qlinear_fwd_quantized), and the gate's backward
+(qlinear_swiglu_bwd: bit for bit) gives the stacked projection's output
+gradient.  Each call is checked against the oracle on seeded inputs: saved
+codes and scales in full and bit for bit, float outputs on sampled rows (and
+sampled weight-gradient rows) within the 1e-3 relative bound plus half a
+bf16 ulp."""
 from __future__ import annotations
 
 import numpy as np
@@ -35,8 +40,8 @@ def mlp():
 
 
 @pytest.fixture(scope="module")
-def stages():
-    return workloads.swiglu_stage_inputs(T=T, d_ff=F, seed=0)
+def gate():
+    return workloads.swiglu_gate_inputs(T=T, d_ff=F, seed=0)
 
 
 def _prep(w):
@@ -96,7 +101,7 @@ def _check_bwd(dy32, dx, dw, db, wq_np, sw_np, xq_np, sx_np, seed):
     assert_close(host(db[ci]), rdb, np.abs(dy32[:, cols].astype(np.float64)).sum(0), what="db")
 
 
-def test_stacked_w13_forward_and_backward(mlp, stages):
+def test_stacked_w13_forward_and_backward(mlp, gate):
     w13 = np.concatenate([mlp["w1"], mlp["w3"]], axis=0)
     wq_np, sw_np = _prep(w13)
     wq, sw = dev(wq_np), dev(sw_np)
@@ -109,15 +114,40 @@ def test_stacked_w13_forward_and_backward(mlp, stages):
     assert torch.equal(y1, y13[:, :F]) and torch.equal(y3, y13[:, F:])
     assert torch.equal(xq1, xq) and torch.equal(sx1, sx)
     del y13, y1, y3
-    dx, dw, db = _bwd(dev(stages["dy13_bf16"]), wq, sw, xq, sx)
-    _check_bwd(stages["dy13"], dx, dw, db, wq_np, sw_np, xq_np, sx_np, 2)
+    # the output gradient [da | db] from the gate's backward (bit for bit
+    # against the oracle, then the stacked projection's backward on it)
+    dab = torch.empty((T, 2 * F), dtype=torch.bfloat16, device="cuda")
+    ql.qlinear_swiglu_bwd(dev(gate["ab_bf16"]), dev(gate["dh_bf16"]), dab)
+    rdab = oracle.swiglu_bwd(gate["ab"], gate["dh"])
+    rdab_bf = torch.from_numpy(rdab).to(torch.bfloat16)
+    assert torch.equal(dab.cpu(), rdab_bf)
+    dy13 = rdab_bf.float().numpy()
+    del rdab, rdab_bf
+    dx, dw, db = _bwd(dab, wq, sw, xq, sx)
+    _check_bwd(dy13, dx, dw, db, wq_np, sw_np, xq_np, sx_np, 2)
 
 
-def test_w2_forward_and_backward(mlp, stages):
+def test_gate_and_w2_forward_and_backward(mlp, gate):
     wq_np, sw_np = _prep(mlp["w2"])
     wq, sw = dev(wq_np), dev(sw_np)
-    y, hq, sh = _fwd(dev(stages["h_bf16"]), wq, sw)
-    hq_np, sh_np = _check_fwd(stages["h"], y, hq, sh, wq_np, sw_np, 3)
+    hq = torch.empty((T, F), dtype=torch.int8, device="cuda")
+    sh = torch.empty(T, dtype=torch.float32, device="cuda")
+    st = new_status()
+    ql.qlinear_swiglu_quantize(dev(gate["ab_bf16"]), hq, sh, st)
+    assert status_word(st) == 0
+    rhq, rsh, rst = oracle.swiglu_quantize(gate["ab"])
+    assert rst == 0
+    hq_np, sh_np = host(hq), host(sh)
+    assert np.array_equal(sh_np, rsh) and np.array_equal(hq_np, rhq)
+    y = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    st = new_status()
+    ql.qlinear_fwd_quantized(hq, sh, wq, sw, None, y, st)
+    assert status_word(st) == 0
+    rows = _rows(T, 10, 3)
+    ry, _ = oracle.fwd_quantized(rhq[rows], rsh[rows], wq_np, sw_np)
+    acc, _ = oracle.gemm_nt(rhq[rows], wq_np)
+    Dm = np.abs(acc.astype(np.float64) * rsh[rows, None].astype(np.float64) * sw_np[None, :])
+    assert_close(host(y[torch.from_numpy(rows).cuda()]), ry, Dm, bf16=True, what="y")
     del y
     dx, dw, db = _bwd(dev(mlp["dy_bf16"]), wq, sw, hq, sh)
     _check_bwd(mlp["dy"], dx, dw, db, wq_np, sw_np, hq_np, sh_np, 4)

@@ -128,28 +128,21 @@ def swiglu_mlp(T: int = 8192, d_model: int = 4096, d_ff: int = 14336,
     }
 
 
-def swiglu_stage_inputs(T: int = 8192, d_ff: int = 14336, seed: int = 0) -> dict:
-    """Inputs of the SwiGLU MLP's second projection and of the stacked
-    first-projection backward, drawn directly (so that each layer call can be
-    checked on its own): pre-activations a, b ~N(0, 1.28^2) (the spread of
-    X W^T for X ~N(0,1), W ~N(0,0.02), d_model 4096); h = silu(a) * b, the w2
-    input; dh ~N(0, 1.28^2), the gradient at h; and the gradient at the
-    stacked [a | b] pre-activations, [dh * b * silu'(a) | dh * silu(a)], with
-    silu(a) = a / (1 + e^-a).  This is the model's gating, not the quantized
-    layer's arithmetic; it is evaluated in float32 and rounded to bf16."""
+def swiglu_gate_inputs(T: int = 8192, d_ff: int = 14336, seed: int = 0) -> dict:
+    """Inputs of the SwiGLU gate and of the calls around it, drawn directly
+    (so that each step can be checked on its own): the stacked
+    pre-activations ab = [a | b] [T, 2 d_ff] ~N(0, 1.28^2) (the spread of
+    X W^T for X ~N(0,1), W ~N(0,0.02), d_model 4096) and the gradient at h,
+    dh [T, d_ff] ~N(0, 1.28^2), each rounded to bf16 (the float32 arrays are
+    the exact upcasts)."""
     sd = 0.02 * 64.0
-    a = normal((T, d_ff), sd, seed + 41)
-    b = normal((T, d_ff), sd, seed + 42)
-    sig = np.float32(1.0) / (np.float32(1.0) + np.exp(-a))
-    silu = a * sig
-    h_bf, h32 = to_bf16(silu * b)
-    dh = normal((T, d_ff), sd, seed + 43)
-    g = np.empty((T, 2 * d_ff), np.float32)
-    g[:, :d_ff] = dh * b * (sig * (np.float32(1.0) + a * (np.float32(1.0) - sig)))
-    g[:, d_ff:] = dh * silu
-    del a, b, dh, sig, silu
-    g_bf, g32 = to_bf16(g)
-    return {"h_bf16": h_bf, "h": h32, "dy13_bf16": g_bf, "dy13": g32}
+    ab = np.empty((T, 2 * d_ff), np.float32)
+    ab[:, :d_ff] = normal((T, d_ff), sd, seed + 41)
+    ab[:, d_ff:] = normal((T, d_ff), sd, seed + 42)
+    ab_bf, ab32 = to_bf16(ab)
+    del ab
+    dh_bf, dh32 = to_bf16(normal((T, d_ff), sd, seed + 43))
+    return {"ab_bf16": ab_bf, "ab": ab32, "dh_bf16": dh_bf, "dh": dh32}
 
 
 def update_state(N: int, K: int, seed: int = 0, warm: bool = False,
