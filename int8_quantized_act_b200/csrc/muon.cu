@@ -1,0 +1,249 @@
+// muon.cu - MuonAuxAdamW for the layer's int8 weights (mini_trainer
+// "docs/quantized-training.md", feature table row "Optimizers", which names
+// it; the method is the published Muon optimizer of Jordan et al., 2024):
+//   M' = beta*M + (1-beta)*G,   U = (1-beta)*G + beta*M'          (Nesterov)
+//   X = U (or U^T when N > K), X /= ||X||_F + 1e-7, then 5 quintic
+//   Newton-Schulz steps  A = X X^T,  B = b A + c A A,  X = a X + B X
+//   w' = w (1 - lr wd) - lr max(1, N/K)^0.5 O  (O = X, back in [N, K]),
+//   then the layer's Philox-keyed stochastic requantization per row.
+// The Newton-Schulz products run on the tcgen05 bf16 GEMM (float32
+// accumulation, bf16 operands as in the published method); X is kept in both
+// layouts so that every product reads K-major operands: A = X X^T from X and
+// X, A A = A A^T (A is symmetric), B X from B and X^T.  The elementwise steps
+// (momentum with ||U||^2, normalization, b A + c A A, a X + B X with its
+// transpose) are the kernels below; the requantization is update_sr.cu's.
+// The float parameters of MuonAuxAdamW (biases, magnitudes) take AdamW:
+// qadamw_vector.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "launch.h"
+#include "rowops.cuh"
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+namespace {
+
+constexpr float kNsA = 3.4445f, kNsB = -4.7750f, kNsC = 2.0315f;
+
+// M' = beta*M + omb*G; U = omb*G + beta*M' (float32, in this order); the sum
+// of U^2 in float64 (one atomic per block).
+__global__ void __launch_bounds__(256) muon_momentum_kernel(const float* __restrict__ G,
+                                                            float* __restrict__ M, int64_t n4,
+                                                            float beta, float omb,
+                                                            double* __restrict__ sumsq) {
+  __shared__ double s_part[8];
+  double acc = 0.0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    const float4 g = __ldcs(reinterpret_cast<const float4*>(G) + i);
+    const float4 m = reinterpret_cast<const float4*>(M)[i];
+    const float gg[4] = {g.x, g.y, g.z, g.w}, mm[4] = {m.x, m.y, m.z, m.w};
+    float mo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      mo[e] = __fadd_rn(__fmul_rn(beta, mm[e]), __fmul_rn(omb, gg[e]));
+      const float u = __fadd_rn(__fmul_rn(omb, gg[e]), __fmul_rn(beta, mo[e]));
+      acc += static_cast<double>(u) * static_cast<double>(u);
+    }
+    reinterpret_cast<float4*>(M)[i] = make_float4(mo[0], mo[1], mo[2], mo[3]);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += s_part[w];
+    atomicAdd(sumsq, t);
+  }
+}
+
+// 32 x 32 tiles through shared memory: out[c][r] = in[r][c] for a row-major
+// in [rows, cols].  `f` maps the input element (float) to the stored value.
+template <typename F>
+__device__ __forceinline__ void transpose_tile(int64_t rows, int64_t cols, int64_t r0, int64_t c0,
+                                               F&& load, __nv_bfloat16* __restrict__ out_t,
+                                               __nv_bfloat16* __restrict__ out,
+                                               __nv_bfloat16 (*tile)[33]) {
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
+#pragma unroll
+  for (int k = 0; k < 32; k += 8) {
+    const int64_t r = r0 + ty + k, c = c0 + tx;
+    if (r < rows && c < cols) {
+      const __nv_bfloat16 v = __float2bfloat16_rn(load(r, c));
+      tile[ty + k][tx] = v;
+      if (out) out[r * cols + c] = v;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 32; k += 8) {
+    const int64_t c = c0 + ty + k, r = r0 + tx;
+    if (r < rows && c < cols) out_t[c * rows + r] = tile[tx][ty + k];
+  }
+  __syncthreads();
+}
+
+// X0 = bf16(U / (||U||_F + 1e-7)) with U recomputed from G and the new M
+// (the same float32 operations as muon_momentum_kernel), written as X [r, c]
+// and X^T [c, r], where X = U when N <= K (r = N) and X = U^T otherwise.
+__global__ void __launch_bounds__(256) ns_init_kernel(const float* __restrict__ G,
+                                                      const float* __restrict__ M, int64_t N,
+                                                      int64_t K, float beta, float omb,
+                                                      const double* __restrict__ sumsq,
+                                                      __nv_bfloat16* __restrict__ X,
+                                                      __nv_bfloat16* __restrict__ Xt) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const float inv = static_cast<float>(1.0 / (sqrt(*sumsq) + 1e-7));
+  const int64_t tiles_c = (K + 31) / 32, tiles = ((N + 31) / 32) * tiles_c;
+  const bool tr = N > K;
+  auto load = [&](int64_t r, int64_t c) {
+    const int64_t i = r * K + c;
+    const float u = __fadd_rn(__fmul_rn(omb, G[i]), __fmul_rn(beta, M[i]));
+    return __fmul_rn(u, inv);
+  };
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+    const int64_t r0 = (t / tiles_c) * 32, c0 = (t % tiles_c) * 32;
+    // U [N, K] row-major; its transpose [K, N].  X is U or U^T.
+    transpose_tile(N, K, r0, c0, load, tr ? X : Xt, tr ? Xt : X, tile);
+  }
+}
+
+// Bm = bf16(b * A + c * A2) elementwise (A bf16, A2 float32, both [r, r]).
+__global__ void __launch_bounds__(256) ns_combine_kernel(const __nv_bfloat16* __restrict__ A,
+                                                         const float* __restrict__ A2, int64_t n,
+                                                         __nv_bfloat16* __restrict__ Bm) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float a = __bfloat162float(A[i]);
+    Bm[i] = __float2bfloat16_rn(__fadd_rn(__fmul_rn(kNsB, a), __fmul_rn(kNsC, A2[i])));
+  }
+}
+
+// X' = bf16(a * X + P) for X [r, c] into Xo (X itself, or the output) and
+// its transpose X'^T [c, r] into Xt.  Each element of X is read by the
+// thread that writes the same element of Xo.
+__global__ void __launch_bounds__(256) ns_step_kernel(const __nv_bfloat16* X,
+                                                      __nv_bfloat16* Xo,
+                                                      const float* __restrict__ P, int64_t r,
+                                                      int64_t c, __nv_bfloat16* __restrict__ Xt) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int64_t tiles_c = (c + 31) / 32, tiles = ((r + 31) / 32) * tiles_c;
+  auto load = [&](int64_t i, int64_t j) {
+    return __fadd_rn(__fmul_rn(kNsA, __bfloat162float(X[i * c + j])), P[i * c + j]);
+  };
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+    const int64_t r0 = (t / tiles_c) * 32, c0 = (t % tiles_c) * 32;
+    transpose_tile(r, c, r0, c0, load, Xt, Xo, tile);
+  }
+}
+
+// AdamW on a float32 vector: the per-element arithmetic of the int8 update.
+__global__ void __launch_bounds__(256) adamw_vector_kernel(float* __restrict__ p,
+                                                           const float* __restrict__ g,
+                                                           float* __restrict__ m,
+                                                           float* __restrict__ v, int64_t n,
+                                                           UpdateConsts c,
+                                                           int32_t* __restrict__ status) {
+  bool bad = false;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    float mm = m[i], vv = v[i];
+    const float gi = g[i];
+    const float w1 = p[i] * c.a;
+    const float mn = c.b1 * mm + c.omb1 * gi;
+    const float vn = c.b2 * vv + c.omb2 * (gi * gi);
+    const float den = sqrtf(vn) * c.rbc2 + c.eps;
+    const float w = w1 - c.st * (mn / den);
+    m[i] = mn;
+    v[i] = vn;
+    p[i] = w;
+    bad |= !isfinite(w);
+  }
+  if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
+}
+
+int grid_for(int64_t items, int per_sm) {
+  const int64_t cap = static_cast<int64_t>(device_info().sms) * per_sm;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((items + 255) / 256, cap)));
+}
+
+}  // namespace
+
+MuonLayout muon_layout(int64_t N, int64_t K) {
+  MuonLayout L;
+  const int64_t r = std::min(N, K), c = std::max(N, K);
+  auto a256 = [](int64_t x) { return (x + 255) / 256 * 256; };
+  int64_t off = 0;
+  L.sumsq = off; off += 256;
+  L.X = off;     off += a256(2 * r * c);
+  L.Xt = off;    off += a256(2 * r * c);
+  L.A = off;     off += a256(2 * r * r);
+  L.A2 = off;    off += a256(4 * r * r);
+  L.Bm = off;    off += a256(2 * r * r);
+  L.P = off;     off += a256(4 * r * c);
+  L.total = off;
+  return L;
+}
+
+cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, int64_t K,
+                                      float beta, int steps, void* O, void* ws, int32_t* status,
+                                      cudaStream_t s) {
+  const MuonLayout L = muon_layout(N, K);
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  double* sumsq = reinterpret_cast<double*>(w + L.sumsq);
+  auto* X = reinterpret_cast<__nv_bfloat16*>(w + L.X);
+  auto* Xt = reinterpret_cast<__nv_bfloat16*>(w + L.Xt);
+  auto* A = reinterpret_cast<__nv_bfloat16*>(w + L.A);
+  auto* A2 = reinterpret_cast<float*>(w + L.A2);
+  auto* Bm = reinterpret_cast<__nv_bfloat16*>(w + L.Bm);
+  auto* P = reinterpret_cast<float*>(w + L.P);
+  const int64_t r = std::min(N, K), c = std::max(N, K);
+  const float omb = static_cast<float>(1.0 - static_cast<double>(beta));
+  cudaError_t e = cudaMemsetAsync(sumsq, 0, sizeof(double), s);
+  if (e != cudaSuccess) return e;
+  muon_momentum_kernel<<<grid_for(N * K / 4, 8), 256, 0, s>>>(grad, mom, N * K / 4, beta, omb, sumsq);
+  ns_init_kernel<<<grid_for(((N + 31) / 32) * ((K + 31) / 32) * 256, 8), 256, 0, s>>>(
+      grad, mom, N, K, beta, omb, sumsq, X, Xt);
+  count_launches(2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (int it = 0; it < steps; ++it) {
+    GemmEpilogue ep;
+    ep.out = A;
+    ep.out_bf16 = 1;
+    ep.ldo = r;
+    if ((e = launch_gemm_bf16(X, c, X, c, r, r, c, ep, status, s)) != cudaSuccess) return e;  // A = X X^T
+    ep.out = A2;
+    ep.out_bf16 = 0;
+    if ((e = launch_gemm_bf16(A, r, A, r, r, r, r, ep, status, s)) != cudaSuccess) return e;  // A A
+    ns_combine_kernel<<<grid_for(r * r, 8), 256, 0, s>>>(A, A2, r * r, Bm);
+    count_launches(1);
+    ep.out = P;
+    ep.ldo = c;
+    if ((e = launch_gemm_bf16(Bm, r, Xt, r, r, c, r, ep, status, s)) != cudaSuccess) return e;  // B X
+    // The last step writes the [N, K]-shaped layout (X^T when N > K) into O.
+    __nv_bfloat16* xo = X;
+    __nv_bfloat16* xto = Xt;
+    if (it == steps - 1) {
+      if (N > K) xto = reinterpret_cast<__nv_bfloat16*>(O);
+      else xo = reinterpret_cast<__nv_bfloat16*>(O);
+    }
+    ns_step_kernel<<<grid_for(((r + 31) / 32) * ((c + 31) / 32) * 256, 8), 256, 0, s>>>(
+        X, xo, P, r, c, xto);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_adamw_vector(float* p, const float* g, float* m, float* v, int64_t n,
+                                const UpdateConsts& c, int32_t* status, cudaStream_t s) {
+  adamw_vector_kernel<<<grid_for(n, 8), 256, 0, s>>>(p, g, m, v, n, c, status);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace ql
