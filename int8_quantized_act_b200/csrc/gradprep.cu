@@ -37,16 +37,18 @@ struct Tile {
   static constexpr int kRowsPerWarp = kRows / 8;
 };
 
-// 8 consecutive elements of a staged row as float32.
+// 8 consecutive elements of a staged row as float32, read with 16-byte
+// shared-memory loads from a shared-space address.
 template <typename InT>
-__device__ __forceinline__ void smem_load8(const uint8_t* p, float (&v)[8]) {
+__device__ __forceinline__ void smem_load8(uint32_t addr, float (&v)[8]) {
   if constexpr (sizeof(InT) == 4) {
-    const float4 a = reinterpret_cast<const float4*>(p)[0];
-    const float4 b = reinterpret_cast<const float4*>(p)[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    const uint4 a = lds128(addr), b = lds128(addr + 16);
+    v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+    v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
+    v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
+    v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
   } else {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint4 u = lds128(addr);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -97,11 +99,12 @@ struct Ring {
   // Consumer warp: wait for tile k, run body, release the stage.
   template <typename F>
   __device__ void consume(int t0, int t1, int lane, F&& body) {
+    const uint32_t base = smem_u32(buf);
     for (int t = t0, k = 0; t < t1; ++t, ++k) {
       const int s = k % kStages;
       const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
       if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) break;
-      body(t, buf + s * kTileBytes);
+      body(t, base + static_cast<uint32_t>(s * kTileBytes));
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
     }
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
       }
     };
     load_scales(t0, fcur);
-    ring.consume(t0, t1, lane, [&](int t, const uint8_t* tile) {
+    ring.consume(t0, t1, lane, [&](int t, uint32_t tile) {
       load_scales(t + 1, fnext);
       // Two rows per step, so one three-operand max covers both.  Rows of
       // the tile past M were zero-filled by the copy and their factors are
@@ -171,8 +174,8 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
         const int r = warp * T::kRowsPerWarp + j;
         const int64_t m = static_cast<int64_t>(t) * T::kRows + r;
         float d0[8], d1[8];
-        smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d0);
-        smem_load8<InT>(tile + (r + 1) * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d1);
+        smem_load8<InT>(tile + (r * kCols + lane * 8) * sizeof(InT), d0);
+        smem_load8<InT>(tile + ((r + 1) * kCols + lane * 8) * sizeof(InT), d1);
         const float f0 = fcur[j], f1 = fcur[j + 1];
         float rb0 = 0.0f, rb1 = 0.0f;
         // Products (only their magnitudes are used, no sum follows them) and
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
       }
     };
     load_rows(t0, f2cur, r1cur);
-    ring.consume(t0, t1, lane, [&](int t, const uint8_t* tile) {
+    ring.consume(t0, t1, lane, [&](int t, uint32_t tile) {
       load_rows(t + 1, f2next, r1next);
 #pragma unroll
       for (int j = 0; j < T::kRowsPerWarp; ++j) {
@@ -293,7 +296,7 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
         const int64_t m = static_cast<int64_t>(t) * T::kRows + r;
         if (m < M && cv) {
           float d[8];
-          smem_load8<InT>(tile + r * kCols * sizeof(InT) + lane * 8 * sizeof(InT), d);
+          smem_load8<InT>(tile + (r * kCols + lane * 8) * sizeof(InT), d);
           const float f2 = f2cur[j];
           uint32_t b[8];
 #pragma unroll

@@ -558,6 +558,8 @@ cudaError_t quant_rows_t(const void* xv, int64_t rows, int64_t cols, int64_t ldx
   const int nch = static_cast<int>((cols + 255) / 256);
   const int c = static_cast<int>(cols);
   const int64_t row_bytes = cols * static_cast<int64_t>(sizeof(InT));
+  if (sizeof(InT) == 2 && quant_blk_eligible(rows, cols, ldx, B, cs != nullptr))
+    return launch_quant_blk(x, rows, cols, ldx, B, hc, flags, q, ldq, rs, st, s);
   if (sizeof(InT) == 2 && B == 128 && !cs && cols % 128 == 0 && cols >= 1024 && cols <= 8192 &&
       (ldx * 2) % 16 == 0 && rows >= 4 * device_info().sms) {
     CUtensorMap tm;
