@@ -4,17 +4,18 @@
 // stochastically in CUDA row kernels, with no floating master weight; feature
 // table rows "Optimizers" and "Row-wise weight normalization").
 //
-// One CTA owns one weight row and reads it from HBM once: codes, gradient
-// and moments in, new moments out, while the updated float row waits in
-// shared memory for the row max; the new scale follows from a CTA max
-// reduction; then every 4-element chunk draws one Philox4x32-10 block and
-// writes 4 stochastically rounded codes.  Rows up to ~8K elements are staged
-// whole by the bulk-copy engine (update_sr_staged_kernel); longer rows are
-// loaded through registers (update_sr_rows_kernel).  The row-wise weight-norm
-// variant stages its row the same way (update_sr_wn_staged_kernel; beyond
-// shared memory, update_sr_kernel) and keeps 16-element groups only for the
-// pinned order of its direction-gradient reduction.  Bytes per element:
-// AdamW 22 (1+4+4+4 in, 1+4+4 out), SGD 6.
+// Each row is read from HBM once: codes, gradient and moments in, new moments
+// out, while the updated float row waits in shared memory for the row max;
+// the new scale follows from a max reduction over the row; then every
+// 4-element chunk draws one Philox4x32-10 block and writes 4 stochastically
+// rounded codes.  Rows up to ~8.8K elements are staged whole by the
+// bulk-copy engine, one row per CTA (update_sr_staged_kernel); longer rows
+// stream through a ring of row pieces in one persistent CTA per SM
+// (update_sr_ring_kernel).  The row-wise weight-norm variant stages its
+// codes and gradient (update_sr_wn_staged_kernel) and keeps 16-element groups
+// only for the pinned order of its direction-gradient reduction.  The Muon
+// step (update_sr_dir_kernel) takes a precomputed update direction.  Bytes
+// per element: AdamW 22 (1+4+4+4 in, 1+4+4 out), SGD 6.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -27,21 +28,6 @@
 namespace ql {
 
 namespace {
-
-// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of two
-// 32x32->64 multiplies, key bumped by the Weyl constants between rounds.
-__device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;  // one 32x32->64 multiply
-    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
-    c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k0, static_cast<uint32_t>(p1),
-                   static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k1, static_cast<uint32_t>(p0));
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
-  }
-  return c;
-}
 
 __device__ __forceinline__ float adamw(const UpdateConsts& c, float w, float g, float& m,
                                        float& v) {
@@ -66,27 +52,6 @@ __device__ __forceinline__ uint32_t sr_code_bits(float val, uint32_t u24) {
   return rne_bits(r);
 }
 
-// Stochastic codes of 16 consecutive elements starting at element e0
-// (a multiple of 16): four Philox blocks, word e & 3 of block e >> 2.
-__device__ __forceinline__ uint4 sr_group(const float (&w)[16], float inv, bool zero_row,
-                                          uint64_t e0, uint32_t sl, uint32_t sh, uint32_t tl,
-                                          uint32_t th) {
-  uint32_t b[16];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint64_t blk = (e0 >> 2) + k;
-    const uint4 r = philox10(make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32),
-                                        tl, th),
-                             sl, sh);
-    const uint32_t words[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      b[4 * k + e] = zero_row ? 0u : sr_code_bits(w[4 * k + e] * inv, words[e] >> 8);
-  }
-  return make_uint4(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]),
-                    pack_codes(b[8], b[9], b[10], b[11]), pack_codes(b[12], b[13], b[14], b[15]));
-}
-
 __device__ __forceinline__ void load16f(const float* p, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -95,184 +60,15 @@ __device__ __forceinline__ void load16f(const float* p, float (&v)[16]) {
   }
 }
 
-__device__ __forceinline__ void store16f(float* p, const float (&v)[16]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    reinterpret_cast<float4*>(p)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-}
-
 __device__ __forceinline__ int code_at(const uint4& q, int i) {
   const uint32_t w = (&q.x)[i >> 2];
   return static_cast<int>(static_cast<int8_t>((w >> (8 * (i & 3))) & 0xFFu));
 }
 
-// The int8 code as a float without the conversion unit: 1.5*2^23 + q is
-// exact in float32 and its bit pattern is that of 1.5*2^23 plus q.
-__device__ __forceinline__ float code_f(const uint4& q, int i) {
-  return __fsub_rn(__int_as_float(0x4B400000 + code_at(q, i)), 12582912.0f);
-}
-
-template <int GPT, bool WN>
-__global__ void __launch_bounds__(256) update_sr_kernel(
-    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
-    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, uint32_t seed_lo,
-    uint32_t seed_hi, uint32_t step_lo, uint32_t step_hi, float* __restrict__ gmag,
-    float* __restrict__ g_m, float* __restrict__ g_v, int32_t* __restrict__ status) {
-  __shared__ float s_red[256];
-  __shared__ int s_ired[8];
-  const int n = blockIdx.x;
-  const int t = threadIdx.x;
-  const int T = blockDim.x;  // power of two, <= 256
-  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
-  const int ngroups = K >> 4;
-  const int64_t row = static_cast<int64_t>(n) * K;
-  const bool adam = c.kind == QL_ADAMW;
-
-  const float s = sw[n];
-  // The magnitude is read before thread 0 may overwrite it (after the update).
-  const float gmag_n = WN ? gmag[n] : 0.0f;
-  uint4 qv[GPT];
-  float w[GPT][16];
-#pragma unroll
-  for (int i = 0; i < GPT; ++i) {
-    const int j = t + T * i;
-    qv[i] = j < ngroups ? *reinterpret_cast<const uint4*>(wq + row + 16 * j) : make_uint4(0, 0, 0, 0);
-  }
-
-  float dg = 0.0f, nq = 0.0f, coef = 0.0f;
-  if constexpr (WN) {
-    // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31).
-    int ss = 0;
-#pragma unroll
-    for (int i = 0; i < GPT; ++i)
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int qc = code_at(qv[i], e);
-        ss += qc * qc;
-      }
-    ss = warp_sum_i(ss);
-    if (lane == 0) s_ired[warp] = ss;
-    __syncthreads();
-    ss = 0;
-    for (int k = 0; k < nwarps; ++k) ss += s_ired[k];
-    if (ss == 0) {  // a zero direction cannot be normalized: reject the row
-      if (t == 0) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
-      return;
-    }
-    nq = static_cast<float>(sqrt(static_cast<double>(ss)));
-    // dg in the fixed order: thread t is lane t of 256 virtual lanes, adding
-    // its groups' products in increasing k; lanes >= T hold +0.
-    float p = 0.0f;
-#pragma unroll
-    for (int i = 0; i < GPT; ++i) {
-      const int j = t + T * i;
-      if (j < ngroups) {
-        float gr[16];
-        load16f(grad + row + 16 * j, gr);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) p = p + gr[e] * (code_f(qv[i], e) / nq);
-      }
-    }
-    for (int off = 128; off >= 1; off >>= 1) {
-      if (off >= T) {
-        p = p + 0.0f;
-      } else if (off >= 32) {
-        s_red[t] = p;
-        __syncthreads();
-        const float o = s_red[t ^ off];
-        __syncthreads();
-        p = p + o;
-      } else {
-        p = p + __shfl_xor_sync(0xFFFFFFFFu, p, off);
-      }
-    }
-    dg = p;
-    coef = gmag_n / (s * nq);
-  }
-
-  // Optimizer step of every element; moments written back immediately.
-  float amax = 0.0f;
-  int bad = 0;
-#pragma unroll
-  for (int i = 0; i < GPT; ++i) {
-    const int j = t + T * i;
-    if (j < ngroups) {
-      const int64_t off = row + 16 * j;
-      float gr[16], m1[16], m2[16];
-      load16f(grad + off, gr);
-      if (adam) {
-        load16f(mom1 + off, m1);
-        load16f(mom2 + off, m2);
-      }
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float qf = code_f(qv[i], e);
-        float gg = gr[e];
-        if constexpr (WN) gg = coef * (gr[e] - dg * (qf / nq));
-        const float wv = s * qf;
-        w[i][e] = adam ? adamw(c, wv, gg, m1[e], m2[e]) : wv - c.lr * gg;
-        bad |= !finite(w[i][e]);
-        amax = fmaxf(amax, fabsf(w[i][e]));
-      }
-      if (adam) {
-        store16f(mom1 + off, m1);
-        store16f(mom2 + off, m2);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) w[i][e] = 0.0f;
-    }
-  }
-  if constexpr (WN) {
-    if (t == 0) {
-      float gm = gmag_n;
-      if (adam) {
-        float a1 = g_m[n], a2 = g_v[n];
-        gm = adamw(c, gm, dg, a1, a2);
-        g_m[n] = a1;
-        g_v[n] = a2;
-      } else {
-        gm = gm - c.lr * dg;
-      }
-      gmag[n] = gm;
-    }
-  }
-
-  // Row max (also the barrier before the scale is overwritten).
-  amax = warp_max(amax);
-  bad = warp_or(bad);
-  __syncthreads();
-  if (lane == 0) {
-    s_red[warp] = amax;
-    s_ired[warp] = bad;
-  }
-  __syncthreads();
-  amax = 0.0f;
-  bad = 0;
-  for (int k = 0; k < nwarps; ++k) {
-    amax = fmaxf(amax, s_red[k]);
-    bad |= s_ired[k];
-  }
-  const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
-  if (t == 0) {
-    sw[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
-    if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
-  }
-
-  // Stochastic requantization: element e = n*K + k uses word e&3 of
-  // Philox(counter = (e>>2 lo, e>>2 hi, step lo, step hi), key = seed).
-#pragma unroll
-  for (int i = 0; i < GPT; ++i) {
-    const int j = t + T * i;
-    if (j < ngroups)
-      *reinterpret_cast<uint4*>(wq + row + 16 * j) =
-          sr_group(w[i], inv, amax == 0.0f, static_cast<uint64_t>(row + 16 * j), seed_lo, seed_hi,
-                   step_lo, step_hi);
-  }
-}
-
-// Philox round keys k_r = seed + r * (0x9E3779B9, 0xBB67AE85) mod 2^32,
-// computed once on the host so each round xors a kernel-parameter constant.
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): ten rounds of two
+// 32x32->64 multiplies; the round keys k_r = seed + r * (0x9E3779B9,
+// 0xBB67AE85) mod 2^32 (the Weyl bumps) are computed once on the host, so
+// each round xors a kernel-parameter constant.
 struct PhiloxKeys {
   uint32_t k0[10], k1[10];
 };
@@ -291,89 +87,6 @@ __device__ __forceinline__ uint4 philox10_keys(uint4 c, const PhiloxKeys& k) {
 __device__ __forceinline__ float code_byte_f(uint32_t q4, int i) {
   return __fsub_rn(__int_as_float(0x4B400000 + static_cast<int>(static_cast<int8_t>(q4 >> (8 * i)))),
                    12582912.0f);
-}
-
-// The plain (not weight-normalized) update.  One CTA per weight row; the row
-// is cut into 4-element chunks (one Philox block each) dealt round-robin to
-// the threads, so every global access of a warp is one contiguous run.
-// Phase 1 streams codes, gradient and moments in, writes the new moments and
-// parks the updated float row in shared memory (4 K bytes) while keeping the
-// running max of |w'|; phase 2, after the CTA max reduction, draws the Philox
-// words and writes the stochastically rounded codes.  Parking the row in
-// shared memory instead of registers keeps the register count low, so
-// several rows are in flight per SM and their loads overlap the arithmetic.
-__global__ void __launch_bounds__(512, 2) update_sr_rows_kernel(
-    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
-    UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
-    uint32_t step_lo, uint32_t step_hi, int32_t* __restrict__ status) {
-  extern __shared__ float4 s_row[];
-  __shared__ uint32_t s_max[16];
-  const int n = blockIdx.x;
-  const int t = threadIdx.x;
-  const int T = blockDim.x;
-  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
-  const int nch = K >> 2;
-  const int64_t row = static_cast<int64_t>(n) * K;
-  const bool adam = c.kind == QL_ADAMW;
-  const float s = sw[n];
-  const uint32_t* q_in = reinterpret_cast<const uint32_t*>(wq + row);
-  const float4* g_in = reinterpret_cast<const float4*>(grad + row);
-  float4* m_io = reinterpret_cast<float4*>(mom1 + row);
-  float4* v_io = reinterpret_cast<float4*>(mom2 + row);
-
-  uint32_t mbits = 0;
-#pragma unroll 2
-  for (int ch = t; ch < nch; ch += T) {
-    const uint32_t q4 = __ldcs(q_in + ch);
-    const float4 g4 = __ldcs(g_in + ch);
-    float gr[4] = {g4.x, g4.y, g4.z, g4.w};
-    float w[4];
-    if (adam) {
-      const float4 m4 = __ldcs(m_io + ch);
-      const float4 v4 = __ldcs(v_io + ch);
-      float m1[4] = {m4.x, m4.y, m4.z, m4.w};
-      float m2[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) w[e] = adamw(c, s * code_byte_f(q4, e), gr[e], m1[e], m2[e]);
-      __stcs(m_io + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
-      __stcs(v_io + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) w[e] = s * code_byte_f(q4, e) - c.lr * gr[e];
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) mbits = max(mbits, abs_bits(w[e]));
-    s_row[ch] = make_float4(w[0], w[1], w[2], w[3]);
-  }
-  mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
-  if (lane == 0) s_max[warp] = mbits;
-  __syncthreads();
-  mbits = 0;
-  for (int k = 0; k < nwarps; ++k) mbits = max(mbits, s_max[k]);
-  const float amax = __uint_as_float(mbits);
-  const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
-  if (t == 0) {
-    sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
-    if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
-  }
-
-  // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
-  // step lo, step hi), key = seed); chunk ch of this row is block row/4 + ch.
-  uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
-  const uint64_t blk0 = static_cast<uint64_t>(row) >> 2;
-#pragma unroll 2
-  for (int ch = t; ch < nch; ch += T) {
-    const uint64_t blk = blk0 + static_cast<uint64_t>(ch);
-    const uint4 r = philox10_keys(
-        make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32), step_lo, step_hi),
-        keys);
-    const float4 w = s_row[ch];
-    uint32_t out = 0;
-    if (mbits != 0)
-      out = pack_codes(sr_code_bits(w.x * inv, r.x >> 8), sr_code_bits(w.y * inv, r.y >> 8),
-                       sr_code_bits(w.z * inv, r.z >> 8), sr_code_bits(w.w * inv, r.w >> 8));
-    __stcs(q_out + ch, out);
-  }
 }
 
 // The same update with the row staged by the bulk-copy engine: one CTA per
@@ -484,19 +197,20 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
   }
 }
 
-// The row-wise weight-norm update with the row staged in shared memory by
-// four bulk copies, so the gradient is read from HBM once although both the
-// direction-gradient reduction and the update use it; codes and gradient
-// land on one barrier, the moments on a second while the reductions run.
-// Only the dg reduction keeps 16-element groups: the first L threads (L a
+// The row-wise weight-norm update with the row's codes and gradient staged
+// in shared memory by two bulk copies, so the gradient is read from HBM once
+// although both the direction-gradient reduction and the update use it; the
+// moments stream through registers in the elementwise step (coalesced
+// 16-byte loads and stores), which keeps a row at 5 bytes of shared memory
+// per element, so several rows share an SM.  Only the dg reduction keeps 16-element groups: the first L threads (L a
 // power of two <= 256) are the virtual lanes of the pinned 256-lane order,
 // lane l adding groups l, l+L, ... (L = 256, or each group has its own lane).
 // ||q||^2 (an integer sum), the elementwise step, the row max and the
 // stochastic rounding are free of order and run on all threads over
 // 4-element chunks as in update_sr_staged_kernel (consecutive threads touch
 // consecutive 16-byte pieces).  Per-element arithmetic and random words are
-// those of update_sr_kernel<GPT, true>, so the results are the same bits.
-__global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
+// the same IEEE operations as the oracle's, so the results are the same bits.
+__global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
     int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
     UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
     uint32_t step_lo, uint32_t step_hi, float* __restrict__ gmag, float* __restrict__ g_m,
@@ -506,33 +220,29 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
   __shared__ float s_qhat[256];  // q / ||q|| for every byte value q = -128 .. 127
   __shared__ int s_ired[16];
   __shared__ float s_dg;
-  __shared__ __align__(8) uint64_t s_full[2];  // codes + gradient; moments
+  __shared__ __align__(8) uint64_t s_full;  // codes + gradient
   __shared__ volatile int s_abort;
   const int n = blockIdx.x;
   const int t = threadIdx.x;
-  const int T = blockDim.x;  // multiple of 32, L .. 512
+  const int T = blockDim.x;  // multiple of 32, L .. 256
   const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
   const int ngroups = K >> 4, nch = K >> 2;
   const int64_t row = static_cast<int64_t>(n) * K;
   const bool adam = c.kind == QL_ADAMW;
   const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
-  // Two barriers: the reductions need only the codes and the gradient, so
-  // they run while the moments are still arriving.
-  const uint32_t bar = smem_u32(&s_full[0]), bar_mv = smem_u32(&s_full[1]);
+  // Only the codes and the gradient are staged (the reductions need them
+  // whole); the moments stream through registers in the elementwise step, so
+  // a row takes 5 bytes of shared memory per element and several rows share
+  // an SM.
+  const uint32_t bar = smem_u32(&s_full);
   if (t == 0) {
     mbar_init(bar, 1);
-    mbar_init(bar_mv, 1);
     s_abort = 0;
     fence_mbar_init();
     const uint32_t dst = smem_u32(smem);
     mbar_arrive_expect_tx(bar, qbytes + fbytes);
     bulk_load(dst, wq + row, qbytes, bar);
     bulk_load(dst + qbytes, grad + row, fbytes, bar);
-    if (adam) {
-      mbar_arrive_expect_tx(bar_mv, 2 * fbytes);
-      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar_mv);
-      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar_mv);
-    }
   }
   const float s = sw[n];
   const float gmag_n = gmag[n];  // read before thread 0 overwrites it
@@ -543,14 +253,11 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
     if (t == 0) {  // copies may still be landing: wait for them (bounded)
       atomicOr(status, 1 << QL_ERR_TIMEOUT);
       mbar_wait_drain(bar, 0);
-      if (adam) mbar_wait_drain(bar_mv, 0);
     }
     return;
   }
   const uint32_t* q_s = reinterpret_cast<const uint32_t*>(smem);
   float4* g_s = reinterpret_cast<float4*>(smem + qbytes);  // then the updated direction
-  const float4* m_s = reinterpret_cast<const float4*>(smem + qbytes + fbytes);
-  const float4* v_s = reinterpret_cast<const float4*>(smem + qbytes + 2 * fbytes);
 
   // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31).
   int ss = 0;
@@ -568,10 +275,7 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
   ss = 0;
   for (int k = 0; k < nwarps; ++k) ss += s_ired[k];
   if (ss == 0) {  // a zero direction cannot be normalized: reject the row (uniform)
-    if (t == 0) {
-      atomicOr(status, 1 << QL_ERR_ZERO_ROW);
-      if (adam) mbar_wait_drain(bar_mv, 0);  // the moments' copies end first
-    }
+    if (t == 0) atomicOr(status, 1 << QL_ERR_ZERO_ROW);
     return;
   }
   const float nq = static_cast<float>(sqrt(static_cast<double>(ss)));
@@ -607,15 +311,7 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
     }
   }
   if (t == 0) s_dg = p;  // every lane < L holds the same sum
-  if (adam) mbar_wait(bar_mv, 0, &s_abort);
   __syncthreads();
-  if (s_abort) {
-    if (t == 0) {
-      atomicOr(status, 1 << QL_ERR_TIMEOUT);
-      mbar_wait_drain(bar_mv, 0);
-    }
-    return;
-  }
   const float dg = s_dg;
   const float coef = gmag_n / (s * nq);
 
@@ -631,7 +327,7 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
     const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
     float m1[4], m2[4];
     if (adam) {
-      const float4 a = m_s[ch], b = v_s[ch];
+      const float4 a = __ldcs(m_out + ch), b = __ldcs(v_out + ch);
       m1[0] = a.x; m1[1] = a.y; m1[2] = a.z; m1[3] = a.w;
       m2[0] = b.x; m2[1] = b.y; m2[2] = b.z; m2[3] = b.w;
     }
@@ -701,12 +397,244 @@ __global__ void __launch_bounds__(512) update_sr_wn_staged_kernel(
   }
 }
 
+// Rows too long to stage whole (more than ~8.8K elements with AdamW): one
+// persistent CTA per SM walks its rows n = blockIdx.x, + gridDim.x, ... while
+// a producer warp streams every row's codes, gradient and moments through a
+// ring of 2048-element pieces by bulk copies, continuing into the next row
+// without a break, so HBM stays busy while the consumers finish a row (its
+// row max and stochastic rounding).  16 consumer warps apply the optimizer
+// step to each piece as it lands (4-element chunks dealt round-robin, moments
+// stored straight back), park the updated row in shared memory (4 K bytes)
+// and then, after the row max, draw the Philox words and write the codes.
+// Per-element arithmetic and random words are those of the other kernels, so
+// the results are the same bits.
+constexpr int kRingPiece = 2048;                    // elements per piece (multiple of 16)
+constexpr int kRingConsumers = 512;                 // 16 consumer warps
+constexpr int kRingThreads = kRingConsumers + 32;   // + the producer warp
+constexpr int kRingStagesMax = 4;
+
+// Named barrier 1 over the consumer warps only, OR-reducing a flag: every
+// consumer gets the same answer, so they leave a loop together.
+__device__ __forceinline__ bool consumers_sync_or(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(flag ? 1u : 0u), "r"(kRingConsumers)
+      : "memory");
+  return r != 0;
+}
+
+template <bool ADAM>
+__global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
+    int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int64_t N,
+    int K, UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
+    uint32_t step_lo, uint32_t step_hi, int stages, int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int EB = ADAM ? 13 : 5;                                // bytes staged per element
+  constexpr uint32_t SB = static_cast<uint32_t>(kRingPiece) * EB;  // bytes per stage
+  float4* parked = reinterpret_cast<float4*>(smem + stages * SB);  // the updated row, 4 K bytes
+  __shared__ uint32_t s_max[kRingConsumers / 32];
+  __shared__ __align__(8) uint64_t s_full[kRingStagesMax], s_empty[kRingStagesMax];
+  __shared__ volatile int s_abort;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int npieces = (K + kRingPiece - 1) / kRingPiece;
+  if (t == 0) {
+    for (int st = 0; st < stages; ++st) {
+      mbar_init(smem_u32(&s_full[st]), 1);
+      mbar_init(smem_u32(&s_empty[st]), kRingConsumers / 32);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == kRingConsumers / 32) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t issued = 0, issued_phase = 0;
+      bool ok = true;
+      int k = 0;
+      for (int64_t n = blockIdx.x; n < N && ok; n += gridDim.x) {
+        const int64_t row = n * K;
+        for (int p = 0; p < npieces; ++p, ++k) {
+          const int st = k % stages;
+          const uint32_t ph = static_cast<uint32_t>(k / stages) & 1u;
+          if (k >= stages && !mbar_wait(smem_u32(&s_empty[st]), ph ^ 1u, &s_abort)) {
+            ok = false;
+            break;
+          }
+          const int e0 = p * kRingPiece;
+          const uint32_t ne = static_cast<uint32_t>(min(kRingPiece, K - e0));
+          const uint32_t dst = smem_u32(smem + st * SB);
+          const uint32_t bar = smem_u32(&s_full[st]);
+          mbar_arrive_expect_tx(bar, ne * EB);
+          bulk_load(dst, wq + row + e0, ne, bar);
+          bulk_load(dst + kRingPiece, grad + row + e0, 4 * ne, bar);
+          if (ADAM) {
+            bulk_load(dst + 5 * kRingPiece, mom1 + row + e0, 4 * ne, bar);
+            bulk_load(dst + 9 * kRingPiece, mom2 + row + e0, 4 * ne, bar);
+          }
+          issued |= 1u << st;
+          issued_phase = (issued_phase & ~(1u << st)) | (ph << st);
+        }
+      }
+      // Every copy issued must land before the CTA may exit.
+      for (int st = 0; st < stages; ++st)
+        if (issued & (1u << st)) mbar_wait_drain(smem_u32(&s_full[st]), (issued_phase >> st) & 1u);
+    }
+    return;
+  }
+  // -------------------------------------------------------------- consumers
+  constexpr int T = kRingConsumers;
+  const int nch_row = K >> 2;
+  int k = 0;
+  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+    const int64_t row = n * K;
+    const float s = sw[n];
+    float4* m_out = reinterpret_cast<float4*>(mom1 + row);
+    float4* v_out = reinterpret_cast<float4*>(mom2 + row);
+    uint32_t mbits = 0;
+    bool ok = true;
+    for (int p = 0; p < npieces; ++p, ++k) {
+      const int st = k % stages;
+      const uint32_t ph = static_cast<uint32_t>(k / stages) & 1u;
+      if (!mbar_wait(smem_u32(&s_full[st]), ph, &s_abort)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* src = smem + st * SB;
+      const uint32_t* q_s = reinterpret_cast<const uint32_t*>(src);
+      const float4* g_s = reinterpret_cast<const float4*>(src + kRingPiece);
+      const float4* m_s = reinterpret_cast<const float4*>(src + 5 * kRingPiece);
+      const float4* v_s = reinterpret_cast<const float4*>(src + 9 * kRingPiece);
+      const int c0 = (p * kRingPiece) >> 2;
+      const int nch = min(kRingPiece, K - p * kRingPiece) >> 2;
+      for (int ch = t; ch < nch; ch += T) {
+        const uint32_t q4 = q_s[ch];
+        const float4 g4 = g_s[ch];
+        const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
+        float w[4];
+        if (ADAM) {
+          const float4 m4 = m_s[ch];
+          const float4 v4 = v_s[ch];
+          float m1[4] = {m4.x, m4.y, m4.z, m4.w};
+          float m2[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[e] = adamw(c, s * code_byte_f(q4, e), gr[e], m1[e], m2[e]);
+          __stcs(m_out + c0 + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
+          __stcs(v_out + c0 + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w[e] = s * code_byte_f(q4, e) - c.lr * gr[e];
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mbits = max(mbits, abs_bits(w[e]));
+        parked[c0 + ch] = make_float4(w[0], w[1], w[2], w[3]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s_empty[st]));
+    }
+    mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+    if (lane == 0) s_max[warp] = mbits;
+    // Row max complete and the parked row written; leave together on abort.
+    if (consumers_sync_or(!ok || s_abort)) break;
+    mbits = 0;
+#pragma unroll
+    for (int w8 = 0; w8 < T / 32; ++w8) mbits = max(mbits, s_max[w8]);
+    const float amax = __uint_as_float(mbits);
+    const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
+    if (t == 0) {
+      sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
+      if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    }
+    // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
+    // step lo, step hi), key = seed); chunk ch of this row is block row/4 + ch.
+    uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
+    const uint64_t blk0 = static_cast<uint64_t>(row) >> 2;
+    for (int ch = t; ch < nch_row; ch += T) {
+      const uint64_t blk = blk0 + static_cast<uint64_t>(ch);
+      const uint4 rn = philox10_keys(
+          make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32), step_lo, step_hi),
+          keys);
+      const float4 w = parked[ch];
+      uint32_t out = 0;
+      if (mbits != 0)
+        out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
+                         sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+      __stcs(q_out + ch, out);
+    }
+    // s_max and the parked row are rewritten by the next row.
+    if (consumers_sync_or(s_abort)) break;
+  }
+  if (t == 0 && s_abort) atomicOr(status, 1 << QL_ERR_TIMEOUT);
+}
+
+// The Muon step of an int8 weight from its orthogonalized update O (bf16
+// [N, K]): w = s*q; w' = (w*a) - st*O, one rounding per operation; then the
+// row max and the Philox-keyed stochastic rounding of the other updates.  One
+// CTA per row, 4-element chunks dealt round-robin (codes 4 bytes, O 8 bytes
+// per chunk), the updated row parked in shared memory (4 K bytes).
+__global__ void __launch_bounds__(512) update_sr_dir_kernel(
+    int8_t* __restrict__ wq, float* __restrict__ sw, const __nv_bfloat16* __restrict__ O, int K,
+    float a, float st, PhiloxKeys keys, uint32_t step_lo, uint32_t step_hi,
+    int32_t* __restrict__ status) {
+  extern __shared__ float4 s_w[];
+  __shared__ uint32_t s_max[16];
+  const int n = blockIdx.x, t = threadIdx.x, T = blockDim.x;
+  const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
+  const int nch = K >> 2;
+  const int64_t row = static_cast<int64_t>(n) * K;
+  const float s = sw[n];
+  const uint32_t* q_in = reinterpret_cast<const uint32_t*>(wq + row);
+  const uint2* o_in = reinterpret_cast<const uint2*>(O + row);
+  uint32_t mbits = 0;
+  for (int ch = t; ch < nch; ch += T) {
+    const uint32_t q4 = __ldcs(q_in + ch);
+    const uint2 o2 = __ldcs(o_in + ch);
+    const float o[4] = {__uint_as_float(o2.x << 16), __uint_as_float(o2.x & 0xFFFF0000u),
+                        __uint_as_float(o2.y << 16), __uint_as_float(o2.y & 0xFFFF0000u)};
+    float w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      w[e] = (s * code_byte_f(q4, e)) * a - st * o[e];
+      mbits = max(mbits, abs_bits(w[e]));
+    }
+    s_w[ch] = make_float4(w[0], w[1], w[2], w[3]);
+  }
+  mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+  if (lane == 0) s_max[warp] = mbits;
+  __syncthreads();
+  mbits = 0;
+  for (int k = 0; k < nwarps; ++k) mbits = max(mbits, s_max[k]);
+  const float amax = __uint_as_float(mbits);
+  const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
+  if (t == 0) {
+    sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
+    if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  }
+  uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
+  const uint64_t blk0 = static_cast<uint64_t>(row) >> 2;
+  for (int ch = t; ch < nch; ch += T) {
+    const uint64_t blk = blk0 + static_cast<uint64_t>(ch);
+    const uint4 rn = philox10_keys(
+        make_uint4(static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32), step_lo, step_hi),
+        keys);
+    const float4 w = s_w[ch];
+    uint32_t out = 0;
+    if (mbits != 0)
+      out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
+                       sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+    __stcs(q_out + ch, out);
+  }
+}
+
+
 // Chunks of 4 elements per thread (sets the thread count of both kernels).
 #ifndef QL_UPDATE_STAGED_CHUNKS
 #define QL_UPDATE_STAGED_CHUNKS 4
-#endif
-#ifndef QL_UPDATE_CHUNKS_PER_THREAD
-#define QL_UPDATE_CHUNKS_PER_THREAD 4
 #endif
 
 }  // namespace
@@ -718,53 +646,42 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
   const int ngroups = static_cast<int>(K / 16);
   int T = 32;
   while (T < ngroups && T < 256) T <<= 1;
-  const int gpt = (ngroups + T - 1) / T;  // 1..8
   const uint32_t sl = static_cast<uint32_t>(seed), sh = static_cast<uint32_t>(seed >> 32);
   const uint32_t tl = static_cast<uint32_t>(step), th = static_cast<uint32_t>(step >> 32);
   const int k = static_cast<int>(K);
   const unsigned grid = static_cast<unsigned>(N);
-#define QL_UPD(G, W)                                                                          \
-  update_sr_kernel<G, W><<<grid, T, 0, s>>>(wq, sw, grad, k, c, m, v, sl, sh, tl, th, g, g_m, \
-                                            g_v, status)
-  if (g != nullptr) {  // weight norm: power-of-two thread count for the pinned reduction
-    const int64_t row_bytes = K * (c.kind == QL_ADAMW ? 13 : 5);
-    // Dynamic budget: the opt-in limit less the kernel's own static arrays.
-    static int64_t wn_budget[64] = {0};
+  if (g != nullptr) {
+    // Weight norm: the row's codes and gradient staged (5 bytes per
+    // element, every K <= 32768 fits), at most 256 threads, of which the
+    // first L are the pinned reduction's virtual lanes.
+    const int64_t row_bytes = 5 * K;
+    static bool wn_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && __atomic_load_n(&wn_budget[dev], __ATOMIC_ACQUIRE) == 0) {
+    if (dev < 64 && !__atomic_load_n(&wn_set[dev], __ATOMIC_ACQUIRE)) {
       cudaFuncAttributes fa{};
       cudaError_t e = cudaFuncGetAttributes(&fa, update_sr_wn_staged_kernel);
-      int64_t b = -1;
-      if (e == cudaSuccess) {
-        b = device_info().smem_optin - static_cast<int64_t>(fa.sharedSizeBytes);
+      if (e == cudaSuccess)
         e = cudaFuncSetAttribute(update_sr_wn_staged_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(b));
-      }
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 device_info().smem_optin - static_cast<int>(fa.sharedSizeBytes));
       if (e != cudaSuccess) {
         (void)cudaGetLastError();  // returned here; not left for a later check
         return e;
       }
-      __atomic_store_n(&wn_budget[dev], b, __ATOMIC_RELEASE);
+      __atomic_store_n(&wn_set[dev], true, __ATOMIC_RELEASE);
     }
-    const int64_t budget = dev < 64 ? __atomic_load_n(&wn_budget[dev], __ATOMIC_ACQUIRE) : 0;
-    if (row_bytes <= budget) {
-      PhiloxKeys keys;
-      for (int r = 0; r < 10; ++r) {
-        keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
-        keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
-      }
-      const int nch = static_cast<int>(K / 4);
-      const int tr = std::max(T, std::min(512, std::max(32, (nch / QL_UPDATE_STAGED_CHUNKS + 31) / 32 * 32)));
-      update_sr_wn_staged_kernel<<<grid, tr, static_cast<size_t>(row_bytes), s>>>(
-          wq, sw, grad, k, c, m, v, keys, tl, th, g, g_m, g_v, T, status);
-      count_launches(1);
-      return cudaGetLastError();
+    PhiloxKeys keys;
+    for (int r = 0; r < 10; ++r) {
+      keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
+      keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
     }
-    if (gpt <= 1) QL_UPD(1, true);
-    else if (gpt <= 2) QL_UPD(2, true);
-    else if (gpt <= 4) QL_UPD(4, true);
-    else QL_UPD(8, true);
+    const int nch = static_cast<int>(K / 4);
+    const int tr = std::max(T, std::min(256, std::max(32, (nch / QL_UPDATE_STAGED_CHUNKS + 31) / 32 * 32)));
+    update_sr_wn_staged_kernel<<<grid, tr, static_cast<size_t>(row_bytes), s>>>(
+        wq, sw, grad, k, c, m, v, keys, tl, th, g, g_m, g_v, T, status);
+    count_launches(1);
+    return cudaGetLastError();
   } else {
     const int nch = static_cast<int>(K / 4);
     PhiloxKeys keys;
@@ -789,21 +706,63 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
       count_launches(1);
       return cudaGetLastError();
     }
-    // Longer rows: registers and a parked row of 4 K bytes.
-    int tr = (nch + QL_UPDATE_CHUNKS_PER_THREAD - 1) / QL_UPDATE_CHUNKS_PER_THREAD;
-    tr = std::min(512, std::max(32, (tr + 31) / 32 * 32));
-    static bool smem_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !__atomic_load_n(&smem_set[dev], __ATOMIC_ACQUIRE)) {
-      cudaFuncSetAttribute(update_sr_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           4 * 32768);
-      __atomic_store_n(&smem_set[dev], true, __ATOMIC_RELEASE);
+    // Longer rows: the piece ring, with as many stages as fit beside the
+    // parked row (4 K bytes).
+    {
+      const int64_t stage_bytes = static_cast<int64_t>(kRingPiece) * (c.kind == QL_ADAMW ? 13 : 5);
+      const int64_t ring_budget = device_info().smem_optin - 1024 - 4 * K;
+      const int stages = static_cast<int>(std::min<int64_t>(kRingStagesMax, ring_budget / stage_bytes));
+      if (stages >= 2) {
+        const size_t smem = static_cast<size_t>(stages * stage_bytes + 4 * K);
+        static bool ring_set[64] = {false};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 64 && !__atomic_load_n(&ring_set[dev], __ATOMIC_ACQUIRE)) {
+          cudaFuncSetAttribute(update_sr_ring_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               device_info().smem_optin - 1024);
+          cudaFuncSetAttribute(update_sr_ring_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               device_info().smem_optin - 1024);
+          __atomic_store_n(&ring_set[dev], true, __ATOMIC_RELEASE);
+        }
+        const unsigned rgrid = static_cast<unsigned>(std::min<int64_t>(N, device_info().sms));
+        if (c.kind == QL_ADAMW)
+          update_sr_ring_kernel<true><<<rgrid, kRingThreads, smem, s>>>(
+              wq, sw, grad, N, k, c, m, v, keys, tl, th, stages, status);
+        else
+          update_sr_ring_kernel<false><<<rgrid, kRingThreads, smem, s>>>(
+              wq, sw, grad, N, k, c, m, v, keys, tl, th, stages, status);
+        count_launches(1);
+        return cudaGetLastError();
+      }
     }
-    update_sr_rows_kernel<<<grid, tr, static_cast<size_t>(4) * K, s>>>(
-        wq, sw, grad, k, c, m, v, keys, tl, th, status);
+    return cudaErrorInvalidConfiguration;  // unreachable for K <= 32768
   }
-#undef QL_UPD
+}
+
+cudaError_t launch_update_dir(int8_t* wq, float* sw, const void* O, int64_t N, int64_t K, float a,
+                              float st, uint64_t seed, uint64_t step, int32_t* status,
+                              cudaStream_t s) {
+  PhiloxKeys keys;
+  const uint32_t sl = static_cast<uint32_t>(seed), sh = static_cast<uint32_t>(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
+    keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
+  }
+  static bool dir_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !__atomic_load_n(&dir_set[dev], __ATOMIC_ACQUIRE)) {
+    cudaFuncSetAttribute(update_sr_dir_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         4 * 32768);
+    __atomic_store_n(&dir_set[dev], true, __ATOMIC_RELEASE);
+  }
+  const int nch = static_cast<int>(K / 4);
+  const int tr = std::min(512, std::max(32, (nch / 4 + 31) / 32 * 32));
+  update_sr_dir_kernel<<<static_cast<unsigned>(N), tr, static_cast<size_t>(4) * K, s>>>(
+      wq, sw, reinterpret_cast<const __nv_bfloat16*>(O), static_cast<int>(K), a, st, keys,
+      static_cast<uint32_t>(step), static_cast<uint32_t>(step >> 32), status);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -62,7 +62,8 @@ def test_sgd_update_bit_exact(N, K):
 
 @pytest.mark.parametrize("warm", [False, True])
 # Rows up to ~8K elements are staged in shared memory; longer ones
-# (14336, 16384, 32768, 14352) take the register path.
+# (14336, 16384, 32768, 14352: a 16-element last piece) stream through the
+# piece ring, each CTA one row here and several rows in the sampled full sizes.
 @pytest.mark.parametrize("N,K", [(64, 1024), (48, 4096), (24, 14336), (16, 16384), (100, 272),
                                  (6, 32768), (5, 14352)])
 def test_adamw_update_bit_exact(N, K, warm):
@@ -78,7 +79,11 @@ def test_adamw_update_bit_exact(N, K, warm):
 
 
 @pytest.mark.parametrize("kind", [ql.QL_ADAMW, ql.QL_SGD])
-@pytest.mark.parametrize("N,K", [(32, 1024), (12, 4096), (6, 16384), (20, 80)])
+# Rows up to K = 16384 (AdamW) are staged whole, one row per CTA; longer
+# rows run the ring kernel: K = 18448 with two resident buffers, a 16-element
+# last moment piece and 160 rows (CTAs walk two rows), K = 32768 with one.
+@pytest.mark.parametrize("N,K", [(32, 1024), (12, 4096), (6, 16384), (20, 80), (160, 18448),
+                                 (4, 32768)])
 def test_weight_norm_update_bit_exact(N, K, kind):
     d = workloads.update_state(N, K, seed=3 * K, weight_norm=True)
     q, s = prepared(d)
@@ -92,14 +97,19 @@ def test_weight_norm_update_bit_exact(N, K, kind):
     check_equal(gpu, ref[:7], NAMES)
 
 
-def test_weight_norm_zero_direction_flagged_and_untouched():
-    d = workloads.update_state(6, 512, seed=5, weight_norm=True)
+# K = 512 and 6160: one staged row per CTA; 18448 (a 16-element last moment
+# piece) and 32768: the ring kernel, with more rows than CTAs so that the
+# rejected rows' moment pieces are drained between other rows
+@pytest.mark.parametrize("N,K,zero", [(6, 512, [2]), (300, 6160, [0, 2, 149, 299]),
+                                      (300, 18448, [0, 2, 149, 299]), (160, 32768, [3, 150])])
+def test_weight_norm_zero_direction_flagged_and_untouched(N, K, zero):
+    d = workloads.update_state(N, K, seed=5, weight_norm=True, warm=True)
     q, s = prepared(d)
-    q[2] = 0
-    s[2] = 0
-    gpu, st = run_gpu(q, s, d["grad"], ql.QL_ADAMW, 1e-3, 1, 1, m=d["m"], v=d["v"], g=d["g"],
-                      g_m=d["g_m"], g_v=d["g_v"])
-    ref = oracle.update_sr(q, s, d["grad"], oracle.ADAMW, 1e-3, 1, 1, m=d["m"], v=d["v"],
+    q[zero] = 0
+    s[zero] = 0
+    gpu, st = run_gpu(q, s, d["grad"], ql.QL_ADAMW, 1e-3, 1, d["step"], m=d["m"], v=d["v"],
+                      g=d["g"], g_m=d["g_m"], g_v=d["g_v"])
+    ref = oracle.update_sr(q, s, d["grad"], oracle.ADAMW, 1e-3, 1, d["step"], m=d["m"], v=d["v"],
                            g=d["g"], g_m=d["g_m"], g_v=d["g_v"])
     assert st == (1 << ql.QL_ERR_ZERO_ROW) and ref[-1] == oracle.BIT_ZERO_ROW
     check_equal(gpu, ref[:7], NAMES)
