@@ -86,6 +86,13 @@ def parse_args():
     p.add_argument("--sweep", action="store_true",
                    help="instead of the train step: the AdamW stochastic-requant update (plain and "
                         "row-wise weight norm) on [n, n] weights, n = 1024 .. 16384 (one JSON line)")
+    p.add_argument("--kernel", default=None,
+                   help="instead of the train step: time one library call of a single kernel "
+                        "family at its full-size shape (quant, quant_dy, bwd, update_staged, "
+                        "update_rows, update_wn, update_wn16, gate, gate_bwd, bf16gemm, muon)")
+    p.add_argument("--muon", action="store_true",
+                   help="instead of the train step: one MuonAuxAdamW step of the 5376->7168 weight "
+                        "(one JSON line)")
     p.add_argument("--edge", action="store_true",
                    help="instead of the train step: time the layer's calls at 1..128 tokens, "
                         "where the weight stream bounds the forward (one JSON line)")
@@ -432,7 +439,7 @@ def run_ours(args, rank, world, local):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(seconds=12.0)
+        out["cpu_baseline"] = cpu_baseline(seconds=10.0)
     return out
 
 
@@ -463,43 +470,159 @@ def cpu_prepare():
     return d, xq, sx, wq, sw
 
 
-def cpu_baseline(seconds=12.0, prepared=None):
-    """The oracle as it stands (single-threaded C) on a bounded sample of the
-    workload, scaled to the metric's unit."""
-    d, xq, sx, wq, sw = prepared or cpu_prepare()
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---- the oracle on every host core: one single-threaded sample per process
+_CPU_ARRAYS = None
+
+
+def _cpu_worker_init(paths):
+    global _CPU_ARRAYS
+    import numpy as np
+    _CPU_ARRAYS = {k: np.load(v, mmap_mode="r") for k, v in paths.items()}
+
+
+def _cpu_worker_sample(args):
+    """Worker i's sample of step t: forward and dX of 4 tokens, dW of 2
+    output rows over all tokens, AdamW requant of 8 weight rows (its own rows
+    and columns of the workload).  Returns the int8 GEMM ops done."""
+    import numpy as np
+    import oracle
+    i, t = args
+    A = _CPU_ARRAYS
+    rows, wcols, urows = 4, 2, 8
+    r0 = (i * rows) % (M_TOK - rows)
+    c0 = (i * wcols) % (N_OUT - wcols)
+    u0 = (i * urows) % (N_OUT - urows)
+    oracle.fwd(A["x"][r0:r0 + rows], A["wq"], A["sw"], A["bias"], BLOCK)
+    oracle.bwd_dx(A["dy"][r0:r0 + rows], A["wq"], A["sw"], BLOCK)
+    dw, *_ = oracle.bwd_dw(np.ascontiguousarray(A["dy"][:, c0:c0 + wcols]), A["xq"], A["sx"])
+    g = np.zeros((urows, K_IN), np.float32)
+    g[:wcols] = dw
+    zeros = np.zeros((urows, K_IN), np.float32)
+    oracle.update_sr(A["wq"][u0:u0 + urows], A["sw"][u0:u0 + urows], g, oracle.ADAMW, 1e-3,
+                     1234, t, m=zeros, v=zeros, wd=0.01)
+    return 2 * rows * N_OUT * K_IN * 2 + 2 * wcols * K_IN * M_TOK
+
+
+class CpuPool:
+    """A process pool (started with spawn, never forked from a process that
+    may hold a GPU context) running the oracle as it stands, one sample per
+    process per step, on every core of the host."""
+
+    def __init__(self, prepared, cores=None):
+        import multiprocessing as mp
+        import tempfile
+        import numpy as np
+        d, xq, sx, wq, sw = prepared
+        self.dir = tempfile.mkdtemp(prefix="qlinear_oracle_")
+        arrays = {"x": d["x"], "dy": d["dy"], "bias": d["bias"], "xq": xq, "sx": sx, "wq": wq,
+                  "sw": sw}
+        paths = {}
+        for k, v in arrays.items():
+            paths[k] = os.path.join(self.dir, k + ".npy")
+            np.save(paths[k], np.ascontiguousarray(v))
+        self.cores = cores or host_cores()
+        self.pool = mp.get_context("spawn").Pool(self.cores, initializer=_cpu_worker_init,
+                                                 initargs=(paths,))
+
+    def step(self, t):
+        return sum(self.pool.map(_cpu_worker_sample, [(i, t) for i in range(self.cores)],
+                                 chunksize=1))
+
+    def close(self):
+        import shutil
+        self.pool.close()
+        self.pool.join()
+        shutil.rmtree(self.dir, ignore_errors=True)
+
+
+def cpu_baseline(seconds=10.0, prepared=None):
+    """The oracle as it stands (single-threaded C) on bounded samples of the
+    workload, scaled to the metric's unit: on one core, and on every core of
+    the host at once (independent samples in a process pool)."""
+    prepared = prepared or cpu_prepare()
+    d, xq, sx, wq, sw = prepared
     rows, wcols, urows = 4, 2, 8
     ops, t0, t = 0, time.perf_counter(), 0
     while time.perf_counter() - t0 < seconds:
         t += 1
         ops += cpu_sample_step(d, xq, sx, wq, sw, rows, wcols, urows, t)
     el = time.perf_counter() - t0
-    return {"value": round(ops / el / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "sample": (f"{t} samples of the step: fwd + dX of {rows} of 12000 tokens, dW of "
-                       f"{wcols} of 7168 output rows over all tokens, AdamW requant of {urows} "
-                       f"weight rows; {el:.1f} s single-threaded; ops = int8 GEMM ops done")}
+    single = {"value": round(ops / el / 1e12, 6), "unit": "TOPS", "cores": 1,
+              "sample": (f"{t} samples of the step: fwd + dX of {rows} of 12000 tokens, dW of "
+                         f"{wcols} of 7168 output rows over all tokens, AdamW requant of {urows} "
+                         f"weight rows; {el:.1f} s on one core; ops = int8 GEMM ops done")}
+    out = {"value": single["value"], "unit": "TOPS", "cores": 1, "kind": "oracle",
+           "cpu_model": cpu_model(), "host_cores": host_cores(), "sample": single["sample"]}
+    try:
+        pool = CpuPool(prepared)
+    except Exception as e:  # no process pool on this host: one core only
+        out["all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"}
+        return out
+    try:
+        pool.step(0)  # warm-up: workers import and map the arrays
+        mops, t0, steps = 0, time.perf_counter(), 0
+        while time.perf_counter() - t0 < seconds:
+            steps += 1
+            mops += pool.step(steps)
+        mel = time.perf_counter() - t0
+    finally:
+        pool.close()
+    out.update({"value": round(mops / mel / 1e12, 6), "cores": pool.cores,
+                "sample": (f"{steps} rounds of {pool.cores} concurrent single-threaded samples "
+                           f"(one per core; each as below, on its own rows and columns) in "
+                           f"{mel:.1f} s"),
+                "single_thread": single})
+    return out
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands on every host core, each
+    step one bounded sample per core (rank 0 only; other ranks exit)."""
     if rank != 0:
         return None
     prepared = cpu_prepare()
-    for _ in range(args.warmup):
-        cpu_sample_step(*prepared, 4, 2, 8, 1)
-    ops, t0 = 0, time.perf_counter()
-    for i in range(args.steps):
-        ops += cpu_sample_step(*prepared, 4, 2, 8, i + 1)
-    el = time.perf_counter() - t0
+    pool = CpuPool(prepared)
+    try:
+        for i in range(max(1, args.warmup)):
+            pool.step(i + 1)
+        ops, t0 = 0, time.perf_counter()
+        for i in range(args.steps):
+            ops += pool.step(i + 1)
+        el = time.perf_counter() - t0
+    finally:
+        pool.close()
     value = ops / el / 1e12
+    sample = (f"each step: one sample per core on {pool.cores} cores, each fwd + dX of 4 of "
+              f"12000 tokens, dW of 2 of 7168 output rows over all tokens, AdamW requant of 8 "
+              f"weight rows")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el * 1e3 / max(1, args.steps), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT,
-                   "hadamard_block": BLOCK, "parallelism": "cpu oracle, rank 0"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-                         "sample": "each step: fwd + dX of 4 of 12000 tokens, dW of 2 of 7168 "
-                                   "output rows over all tokens, AdamW requant of 8 weight rows"},
+                   "hadamard_block": BLOCK, "parallelism": "cpu oracle, rank 0, all host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": pool.cores,
+                         "kind": "oracle", "cpu_model": cpu_model(), "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -688,13 +811,17 @@ def run_edge(args):
 
 
 def run_swiglu(args):
-    """A SwiGLU MLP training step through the layer calls: d_model 4096,
+    """A SwiGLU MLP training step through the library's calls: d_model 4096,
     d_ff 14336, 8192 tokens, bf16 activations and gradients, no rotation,
     AdamW (lr 1e-3, wd 0.01) with stochastic requantization of both weights.
     w1 and w3 run stacked as one [28672, 4096] weight (one quantization of X
-    for both).  The gating silu(a) * b and its derivative are model glue in
-    torch (bf16 elementwise), timed separately.  Metric: the 9 int8 GEMMs' operations
-    (3 x 2 x 8192 x 4096 x 14336 x 3) per second of the whole step."""
+    for both); the gate h = silu(a) * b runs fused with the quantization of
+    the second projection's input (qlinear_swiglu_quantize, h never stored),
+    the second projection takes those codes (qlinear_fwd_quantized), and the
+    gate's backward (qlinear_swiglu_bwd) gives the stacked projection's
+    output gradient.  Every step of it is one of the library's kernels.
+    Metric: the 9 int8 GEMMs' operations (3 x 2 x 8192 x 4096 x 14336 x 3)
+    per second of the whole step."""
     import torch
     import int8_quantized_act_b200 as ql
     torch.cuda.set_device(0)
@@ -724,12 +851,10 @@ def run_swiglu(args):
     h13 = torch.empty((T, 2 * F), dtype=torch.bfloat16, device=dev)
     xq = torch.empty((T, D), dtype=torch.int8, device=dev)
     sx = torch.empty(T, device=dev)
-    h = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
     hq = torch.empty((T, F), dtype=torch.int8, device=dev)
     sh = torch.empty(T, device=dev)
     y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
     dh = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
-    sl, sg, tmp = (torch.empty((T, F), dtype=torch.bfloat16, device=dev) for _ in range(3))
     d13 = torch.empty((T, 2 * F), dtype=torch.bfloat16, device=dev)
     dx = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(max(ql.qlinear_bwd_workspace_bytes(T, D, F, 0),
@@ -744,19 +869,12 @@ def run_swiglu(args):
         rec(0)
         ql.qlinear_fwd(x, w13.q, w13.s, None, 0, h13, xq, sx, st)
         rec(1)
-        a, b = h13[:, :F], h13[:, F:]
-        torch.ops.aten.silu.out(a, out=sl)
-        torch.mul(sl, b, out=h)
+        ql.qlinear_swiglu_quantize(h13, hq, sh, st)
         rec(2)
-        ql.qlinear_fwd(h, w2.q, w2.s, None, 0, y, hq, sh, st)
+        ql.qlinear_fwd_quantized(hq, sh, w2.q, w2.s, None, y, st)
         ql.qlinear_bwd(dy, w2.q, w2.s, hq, sh, 0, dh, w2.dw, w2.db, ws, st)
         rec(3)
-        # d/db = dh * silu(a); d/da = dh * b * silu'(a), silu' = s + silu * (1 - s)
-        torch.mul(dh, sl, out=d13[:, F:])
-        torch.sigmoid(a, out=sg)
-        torch.addcmul(sg, sl, 1 - sg, out=tmp)
-        torch.mul(dh, b, out=d13[:, :F])
-        d13[:, :F].mul_(tmp)
+        ql.qlinear_swiglu_bwd(h13, dh, d13)
         rec(4)
         ql.qlinear_bwd(d13, w13.q, w13.s, xq, sx, 0, dx, w13.dw, w13.db, ws, st)
         rec(5)
@@ -772,18 +890,24 @@ def run_swiglu(args):
     clocks.start()
     time.sleep(0.2)
     torch.cuda.synchronize()
+    launches0 = ql.ql_kernel_launches()
     for i in range(args.steps):
         step(evs[i])
     torch.cuda.synchronize()
+    launches = ql.ql_kernel_launches() - launches0
     clk = clocks.stop()
     if int(st.item()):
         raise RuntimeError(f"device status {ql.status_flags(int(st.item()))}")
     el = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
     step_ms = el(0, 6)
-    glue_ms = el(1, 2) + el(3, 4)
+    gate_ms, gate_bwd_ms = el(1, 2), el(3, 4)
     upd_ms = el(5, 6)
     ops = 9 * 2.0 * T * D * F
     upd_bytes = 22 * (2 * F * D + D * F)
+    # the gate reads bf16 [a | b] and writes int8 h codes; its backward reads
+    # [a | b] and dh and writes [da | db], all bf16
+    gate_bytes = T * F * (4 + 1)
+    gate_bwd_bytes = T * F * (4 + 2 + 4)
     peaks = load_peaks()
     return {
         "metric": "SwiGLU MLP train step TOPS (9 int8 GEMMs per step, d_model 4096, d_ff 14336, 8192 tokens)",
@@ -791,12 +915,15 @@ def run_swiglu(args):
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic",
         "dtype": "i8",
         "config": {"workload": "SwiGLU MLP step: w1|w3 stacked [28672,4096], w2 [4096,14336], "
-                               "8192 tokens, bf16 x/dY, AdamW + stochastic requant of both weights",
+                               "8192 tokens, bf16 x/dY, fused gate + h quantization, AdamW + "
+                               "stochastic requant of both weights",
                    "tokens": T, "d_model": D, "d_ff": F},
         "ms_per_step": round(step_ms, 4),
-        "breakdown_ms": {"layer_calls_and_updates": round(step_ms - glue_ms, 4),
-                         "gating_glue_torch": round(glue_ms, 4), "updates": round(upd_ms, 4)},
-        "tops_excluding_glue": round(ops / ((step_ms - glue_ms) * 1e-3) / 1e12, 2),
+        "gpu_launches": launches,
+        "breakdown_ms": {"gate_fwd_quant": round(gate_ms, 4), "gate_bwd": round(gate_bwd_ms, 4),
+                         "updates": round(upd_ms, 4)},
+        "gate_fwd_gbs": round(gate_bytes / (gate_ms * 1e-3) / 1e9, 1),
+        "gate_bwd_gbs": round(gate_bwd_bytes / (gate_bwd_ms * 1e-3) / 1e9, 1),
         "update_gbs": round(upd_bytes / (upd_ms * 1e-3) / 1e9, 1),
         "update_frac_of_hbm": round(upd_bytes / (upd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "clocks": clk,
@@ -865,6 +992,225 @@ def run_sweep(args):
     return out
 
 
+def run_muon(args):
+    """One MuonAuxAdamW step of the 5376 -> 7168 layer's int8 weight: Muon
+    momentum and five Newton-Schulz steps on the tensor cores (bf16 operands,
+    float32 accumulation), then the Muon requantization step; plus AdamW on
+    the layer's float bias.  Metric: Newton-Schulz tensor operations per
+    second (per step: A = X X^T, A A and B X with X = U^T, r = 5376,
+    c = 7168)."""
+    import torch
+    import int8_quantized_act_b200 as ql
+    torch.cuda.set_device(0)
+    N, K = N_OUT, K_IN
+    r, c = min(N, K), max(N, K)
+    gen = torch.Generator(device="cuda").manual_seed(6)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    wq = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    sw = torch.empty(N, device="cuda")
+    ql.qlinear_quantize_rows(torch.randn((N, K), generator=gen, device="cuda") * 0.02, wq, sw, st,
+                             flags=ql.QL_REJECT_ZERO_ROWS)
+    grad = torch.randn((N, K), generator=gen, device="cuda") * 1e-3
+    mom = torch.zeros((N, K), device="cuda")
+    O = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(ql.qweight_muon_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
+    bias = torch.zeros(N, device="cuda")
+    gb = torch.randn(N, generator=gen, device="cuda") * 1e-3
+    bm, bv = torch.zeros(N, device="cuda"), torch.zeros(N, device="cuda")
+    opt = ql.Optim(kind=ql.QL_ADAMW, lr=1e-3, weight_decay=0.0)
+    t = [0]
+
+    def step(ev=None):
+        t[0] += 1
+        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+        rec(0)
+        ql.qweight_muon_orthogonalize(grad, mom, O, ws, st)
+        rec(1)
+        ql.qweight_update_muon_sr(wq, sw, O, 0.02, 0.01, 13, t[0], st)
+        ql.qvector_adamw(bias, gb, bm, bv, opt, t[0], st)
+        rec(2)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [new_events(3) for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.2)
+    torch.cuda.synchronize()
+    launches0 = ql.ql_kernel_launches()
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    launches = ql.ql_kernel_launches() - launches0
+    clk = clocks.stop()
+    if int(st.item()):
+        raise RuntimeError(f"device status {ql.status_flags(int(st.item()))}")
+    el = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
+    ns_ms, upd_ms = el(0, 1), el(1, 2)
+    ns_ops = 5 * (2.0 * r * r * c + 2.0 * r * r * r + 2.0 * r * c * r)
+    peaks = load_peaks()
+    tflops = ns_ops / (ns_ms * 1e-3) / 1e12
+    upd_bytes = N * K * (1 + 2 + 1)  # codes in, O in (bf16), codes out
+    return {
+        "metric": "MuonAuxAdamW step of the 5376->7168 weight: Newton-Schulz TFLOP/s",
+        "value": round(tflops, 1), "unit": "TFLOP/s", "higher_is_better": True,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic",
+        "dtype": "bf16",
+        "config": {"workload": "Muon momentum + 5 Newton-Schulz steps (bf16 tcgen05) + Muon "
+                               "stochastic requant of the [7168, 5376] int8 weight + AdamW on its "
+                               "bias", "N": N, "K": K},
+        "ms_per_step": round(ns_ms + upd_ms, 4), "gpu_launches": launches,
+        "breakdown_ms": {"orthogonalize": round(ns_ms, 4), "requant_and_bias": round(upd_ms, 4)},
+        "ns_frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
+        "requant_gbs": round(upd_bytes / (upd_ms * 1e-3) / 1e9, 1),
+        "peaks_source": peaks["source"], "clocks": clk,
+    }
+
+
+KERNEL_CASES = {
+    # name: (what one call is, algorithmic bytes moved per call)
+    "quant": ("qlinear_quantize_rows: 12000 x 5376 bf16 rows, Hadamard block 128", 12000 * 5376 * 3),
+    "quant_dy": ("qlinear_quantize_rows: 12000 x 7168 bf16 rows scaled per column (dY * s_w)",
+                 12000 * 7168 * 3),
+    "bwd": ("qlinear_bwd at 12000 tokens (gradient preparation + both GEMMs)", None),
+    "update_staged": ("qweight_update_sr AdamW [7168, 5376]", 22 * 7168 * 5376),
+    "update_rows": ("qweight_update_sr AdamW [4096, 14336]", 22 * 4096 * 14336),
+    "update_wn": ("qweight_update_sr AdamW + weight norm [8192, 8192]", 22 * 8192 * 8192 + 24 * 8192),
+    "update_wn16": ("qweight_update_sr AdamW + weight norm [16384, 16384]",
+                    22 * 16384 * 16384 + 24 * 16384),
+    "gate": ("qlinear_swiglu_quantize [8192, 2 x 14336] bf16 -> h codes", 8192 * 14336 * 5),
+    "gate_bwd": ("qlinear_swiglu_bwd [8192, 2 x 14336] bf16", 8192 * 14336 * 10),
+    "bf16gemm": ("qlinear_fwd_bf16 at 12000 tokens (5376 -> 7168, block 128)", None),
+    "muon": ("qweight_muon_orthogonalize [7168, 5376]", None),
+}
+
+
+def run_kernel(args):
+    """One library call of a single kernel family at its full-size shape,
+    timed alone with CUDA events (the shapes the ncu summaries capture)."""
+    import torch
+    import int8_quantized_act_b200 as ql
+    name = args.kernel
+    torch.cuda.set_device(0)
+    g = torch.Generator(device="cuda").manual_seed(1)
+
+    def randn(shape, std=1.0, dtype=torch.float32):
+        return (torch.randn(shape, generator=g, device="cuda") * std).to(dtype)
+
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def wprep(n, k, B=0):
+        q = torch.empty((n, k), dtype=torch.int8, device="cuda")
+        s = torch.empty(n, device="cuda")
+        ql.qlinear_quantize_rows(randn((n, k), 0.02), q, s, st, hadamard_block=B,
+                                 flags=ql.QL_REJECT_ZERO_ROWS)
+        return q, s
+
+    if name in ("quant", "quant_dy"):
+        M, K = (12000, 5376) if name == "quant" else (12000, 7168)
+        x = randn((M, K), 1.0, torch.bfloat16)
+        q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+        s = torch.empty(M, device="cuda")
+        cs = randn((K,), 1e-3).abs() + 1e-5 if name == "quant_dy" else None
+        B = 128 if name == "quant" else 0
+
+        def run():
+            ql.qlinear_quantize_rows(x, q, s, st, col_scale=cs, hadamard_block=B)
+    elif name == "bwd":
+        M, K, N = M_TOK, K_IN, N_OUT
+        wq, sw = wprep(N, K, BLOCK)
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device="cuda", generator=g)
+        sx = randn((M,), 0.01).abs()
+        dy = randn((M, N), 1.0, torch.bfloat16)
+        ws = torch.empty(ql.qlinear_bwd_workspace_bytes(M, N, K, BLOCK), dtype=torch.uint8,
+                         device="cuda")
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+        dw = torch.empty((N, K), device="cuda")
+        db = torch.empty(N, device="cuda")
+
+        def run():
+            ql.qlinear_bwd(dy, wq, sw, xq, sx, BLOCK, dx, dw, db, ws, st)
+    elif name.startswith("update"):
+        N, K = {"update_rows": (4096, 14336), "update_wn": (8192, 8192),
+                "update_wn16": (16384, 16384), "update_staged": (7168, 5376)}[name]
+        wq, sw = wprep(N, K)
+        grad = randn((N, K), 1e-3)
+        m = torch.zeros((N, K), device="cuda")
+        v = torch.zeros((N, K), device="cuda")
+        wn = None
+        if name.startswith("update_wn"):
+            wn = (torch.rand(N, generator=g, device="cuda") * 1.5 + 0.5,
+                  torch.zeros(N, device="cuda"), torch.zeros(N, device="cuda"))
+        opt = ql.Optim(kind=ql.QL_ADAMW, lr=1e-3, weight_decay=0.01)
+        step = [0]
+
+        def run():
+            step[0] += 1
+            if wn is None:
+                ql.qweight_update_sr(wq, sw, grad, opt, m, v, 7, step[0], st)
+            else:
+                ql.qweight_update_sr(wq, sw, grad, opt, m, v, 7, step[0], st, g=wn[0], g_m=wn[1],
+                                     g_v=wn[2])
+    elif name in ("gate", "gate_bwd"):
+        T, F = 8192, 14336
+        ab = randn((T, 2 * F), 1.28, torch.bfloat16)
+        hq = torch.empty((T, F), dtype=torch.int8, device="cuda")
+        sh = torch.empty(T, device="cuda")
+        dh = randn((T, F), 1.28, torch.bfloat16)
+        dab = torch.empty((T, 2 * F), dtype=torch.bfloat16, device="cuda")
+
+        def run():
+            if name == "gate":
+                ql.qlinear_swiglu_quantize(ab, hq, sh, st)
+            else:
+                ql.qlinear_swiglu_bwd(ab, dh, dab)
+    elif name == "bf16gemm":
+        M, K, N = M_TOK, K_IN, N_OUT
+        wq, sw = wprep(N, K, BLOCK)
+        wb = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+        ql.qlinear_codes_bf16(wq, wb)
+        x = randn((M, K), 1.0, torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(ql.qlinear_fwd_bf16_workspace_bytes(M, K, torch.bfloat16, BLOCK),
+                         dtype=torch.uint8, device="cuda")
+
+        def run():
+            ql.qlinear_fwd_bf16(x, wb, sw, None, BLOCK, y, ws, st)
+    elif name == "muon":
+        N, K = N_OUT, K_IN
+        grad = randn((N, K), 1e-3)
+        mom = torch.zeros((N, K), device="cuda")
+        O = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(ql.qweight_muon_workspace_bytes(N, K), dtype=torch.uint8, device="cuda")
+
+        def run():
+            ql.qweight_muon_orthogonalize(grad, mom, O, ws, st)
+    else:
+        raise SystemExit(f"unknown kernel case {name}; one of {sorted(KERNEL_CASES)}")
+    for _ in range(max(1, args.warmup)):
+        run()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.steps):
+        run()
+    ev[1].record()
+    torch.cuda.synchronize()
+    if int(st.item()):
+        raise RuntimeError(f"device status {ql.status_flags(int(st.item()))}")
+    us = ev[0].elapsed_time(ev[1]) / args.steps * 1e3
+    what, nbytes = KERNEL_CASES[name]
+    out = {"kernel_case": name, "call": what, "us_per_call": round(us, 2), "calls": args.steps,
+           "note": "back-to-back calls, no L2 flush"}
+    if nbytes:
+        peaks = load_peaks()
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out.update({"algorithmic_bytes": nbytes, "gbs": round(gbs, 1),
+                    "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4), "peaks_source": peaks["source"]})
+    return out
+
+
 def main():
     args = parse_args()
     if args.sweep:
@@ -878,6 +1224,12 @@ def main():
         return
     if args.routes:
         print(json.dumps(run_routes(args)), flush=True)
+        return
+    if args.muon:
+        print(json.dumps(run_muon(args)), flush=True)
+        return
+    if args.kernel:
+        print(json.dumps(run_kernel(args)), flush=True)
         return
     world_env = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":

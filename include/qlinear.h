@@ -209,6 +209,50 @@ QL_API int qlinear_fwd(const void *x, int xt, int64_t M, int64_t K,
                 int hadamard_block, void *y, int yt,
                 int8_t *xq_saved, float *sx_saved, int32_t *d_status, void *stream);
 
+/* Forward from an input that is already quantized: the GEMM and epilogue of
+ * qlinear_fwd without its quantization step,
+ *   y[m,n] = ((float)(sum_k xq[m,k] W_q[n,k]) * sx[m]) * s_w[n] + bias[n]
+ * for codes xq [M,K] and row scales sx [M] that a producer kernel wrote in the
+ * layer's own format (per-row symmetric int8, in the weight's basis), such as
+ * qlinear_swiglu_quantize.  Sizes, layouts, requirements and errors as for
+ * qlinear_fwd. */
+QL_API int qlinear_fwd_quantized(const int8_t *xq, const float *sx, int64_t M, int64_t K,
+                                 const int8_t *wq, const float *sw, int64_t N, const float *bias,
+                                 void *y, int yt, int32_t *d_status, void *stream);
+
+/* The SwiGLU gate of an MLP whose three projections are layers of this
+ * library (w1 and w3 stacked as one [2F, d] weight on the same input, w2 on
+ * h), fused with the per-row quantization that the second projection applies
+ * to its input ([CR] item 1: activations quantized per row on every call), so
+ * h never goes to memory:
+ *   h[m,f] = silu(a[m,f]) * b[m,f],  silu(a) = a / (1 + e^-a)
+ *   sh[m] = max_f |h[m,f]| / 127,  hq[m,f] = clamp(rne(h * (127/max|h|)), +-127)
+ * with ab = [a | b] [M, 2F] (dtype abt, pitch ldab elements: a = columns
+ * 0..F-1, b = columns F..2F-1), hq [M, F] int8 (pitch ldh), sh [M] float32.
+ * All float32, one rounding per operation in the order written; e^x by fixed
+ * float32 steps (Cody-Waite reduction with C1 = fl32(ln 2), degree-7 Taylor
+ * series, fused multiply-adds), so codes are reproducible bit for bit.  A zero
+ * row gives sh = 0 and zero codes; a non-finite h sets QL_ERR_NONFINITE.
+ * The result is the input (xq, sx) of qlinear_fwd_quantized and the saved
+ * input of the second projection's backward.  Requirements: F % 16 == 0,
+ * 16 <= F <= 16384 (QL_ERR_UNSUPPORTED above), ldab >= 2F with ldab *
+ * sizeof(abt) % 16 == 0, ldh >= F, ldh % 16 == 0; ab, hq 16-byte aligned. */
+QL_API int qlinear_swiglu_quantize(const void *ab, int abt, int64_t M, int64_t F, int64_t ldab,
+                                   int8_t *hq, int64_t ldh, float *sh, int32_t *d_status,
+                                   void *stream);
+
+/* The gate's backward: from dh [M, F] (dtype dht, contiguous; the input
+ * gradient of the second projection) and ab as above, the gradient at the
+ * stacked pre-activations dab [M, 2F] (dtype dabt, contiguous):
+ *   d = 1 + e^-a, sigma = 1/d, silu = a/d
+ *   da = (dh * b) * (sigma * (1 + a * (1 - sigma))),   db = dh * silu
+ * float32, one rounding per operation in the order written (bf16 output:
+ * the float32 value rounded to nearest even).  dab is the output gradient of
+ * the stacked first projection.  Requirements: F % 16 == 0, F >= 16,
+ * ldab >= 2F with ldab * sizeof(abt) % 16 == 0; ab, dh, dab 16-byte aligned. */
+QL_API int qlinear_swiglu_bwd(const void *ab, int abt, int64_t ldab, const void *dh, int dht,
+                              int64_t M, int64_t F, void *dab, int dabt, void *stream);
+
 /* Input gradient ([QT] intro: the backward products are integer GEMMs too;
  * [CR] item 2 for the rotation):
  *   dYq, s' = quantize_rows(dY, col_scale = s_w)       (row quantization of dY*s_w)
@@ -277,6 +321,52 @@ QL_API int qweight_update_sr(int8_t *wq, float *sw, const float *grad, int64_t N
                       uint64_t seed, uint64_t step, const ql_weightnorm *wn,
                       int32_t *d_status, void *stream);
 
+/* MuonAuxAdamW ([QT] feature table, row "Optimizers", names it among the
+ * update paths).  The pages do not define it; this follows the published
+ * Muon optimizer (K. Jordan et al., "Muon: An optimizer for hidden layers in
+ * neural networks", 2024) for the int8 weights, and AdamW (qvector_adamw)
+ * for the float parameters such as biases.  One Muon step of a weight is
+ * qweight_muon_orthogonalize followed by qweight_update_muon_sr.
+ *
+ * qweight_muon_orthogonalize: from the weight gradient grad [N, K] float32
+ * and the momentum mom [N, K] float32 (updated in place):
+ *   M' = beta*M + (1-beta)*G,  U = (1-beta)*G + beta*M'   (float32, in order)
+ *   X = U, or U^T when N > K; X = X / (||X||_F + 1e-7)      (norm in float64)
+ *   ns_steps times: A = X X^T;  B = b*A + c*(A A);  X = a*X + B X,
+ *   (a, b, c) = (3.4445, -4.7750, 2.0315)
+ * and O [N, K] bf16 = X in the weight's layout.  As in the published method
+ * the products take bf16 operands (X, A and B rounded to bf16; float32
+ * accumulation on the tensor cores), so O matches the float64 iteration of
+ * the same definition to bf16 accuracy, not bit for bit.  ws: at least
+ * qweight_muon_workspace_bytes(N, K) bytes, 256-byte aligned (for N = 7168,
+ * K = 5376 about 0.5 GB).  Requirements: N, K multiples of 16; 0 <= beta < 1;
+ * 1 <= ns_steps <= 16; grad, mom, O 16-byte aligned. */
+QL_API size_t qweight_muon_workspace_bytes(int64_t N, int64_t K);
+QL_API int qweight_muon_orthogonalize(const float *grad, float *mom, int64_t N, int64_t K,
+                                      float momentum, int ns_steps, void *O, void *ws,
+                                      size_t ws_bytes, int32_t *d_status, void *stream);
+
+/* qweight_update_muon_sr: the Muon step of the int8 weight from O (bf16
+ * [N, K]), in place, with the layer's stochastic requantization:
+ *   w = s_w[n]*q;  w' = w*a - st*O,  a = fl32(1 - lr*wd),
+ *   st = fl32(lr * max(1, N/K)^0.5)   (constants in float64, rounded once)
+ * then per row s' = max|w'|/127 and codes by the Philox-keyed stochastic
+ * rounding of qweight_update_sr (same seed/step/element keying).  Bit for
+ * bit reproducible given O.  Requirements: N, K multiples of 16, K <= 32768,
+ * step >= 1; wq, O 16-byte aligned. */
+QL_API int qweight_update_muon_sr(int8_t *wq, float *sw, const void *O, int64_t N, int64_t K,
+                                  float lr, float weight_decay, uint64_t seed, uint64_t step,
+                                  int32_t *d_status, void *stream);
+
+/* qvector_adamw: AdamW on a float32 vector p [n] with gradient g and moments
+ * m, v (updated in place), the same per-element arithmetic and host
+ * constants as qweight_update_sr's AdamW, without requantization (the
+ * "AdamW" part of MuonAuxAdamW: biases and other float parameters).  opt is
+ * a HOST pointer with kind QL_ADAMW; step >= 1.  A non-finite result sets
+ * QL_ERR_NONFINITE. */
+QL_API int qvector_adamw(float *p, const float *g, float *m, float *v, int64_t n,
+                         const ql_optim *opt, uint64_t step, int32_t *d_status, void *stream);
+
 /* Capacity of the library-owned scratch used by qlinear_bwd_dx_noalloc:
  * 32 MiB of device memory. */
 #define QL_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -289,17 +379,23 @@ QL_API int qweight_update_sr(int8_t *wq, float *sw, const float *grad, int64_t N
  * interface convenience; the pages have no counterpart.)
  *
  * Arguments, results and errors are those of qlinear_bwd_dx without ws and
- * ws_bytes.  Instead of a caller buffer it uses a scratch array of
+ * ws_bytes: its argument, shape and null-pointer checks come first and return
+ * the same codes.  Instead of a caller buffer it uses a scratch array of
  * QL_NOALLOC_SCRATCH_BYTES that lives in the library's own device image: it
  * is not allocated by any call, and every GPU that loads the library's
- * device code holds it until the process exits.  Sizes whose workspace,
- * qlinear_workspace_bytes(M, N, K, hadamard_block), exceeds that capacity are
- * rejected with QL_ERR_UNSUPPORTED before anything runs (for example
- * M = 2048, N = 7168 fits; M = 12000, N = 7168 does not).
+ * device code holds it until the process exits.  Sizes with work to do
+ * (M > 0, K > 0) whose workspace, qlinear_workspace_bytes(M, N, K,
+ * hadamard_block), exceeds that capacity are then rejected with
+ * QL_ERR_UNSUPPORTED before anything runs (for example M = 2048, N = 7168
+ * fits; M = 12000, N = 7168 does not).
  *
  * The first call on a device looks up the array's device address on that
- * device (cudaGetSymbolAddress, once per device, thread-safe); make that
- * first call before any stream capture.  All calls in the process share the
+ * device (cudaGetSymbolAddress, thread-safe); make that first call before
+ * any stream capture.  With lazy module loading that lookup can be what
+ * loads the library's device code, and with it the array, onto the device;
+ * if it fails (e.g. the device is out of memory at that moment) the call
+ * returns QL_ERR_CUDA and the next call looks it up again: only a lookup
+ * that succeeded is kept.  All calls in the process share the
  * one array and it keeps whatever the last call left in it; nothing in it
  * needs to start at zero, because every byte this call reads was written
  * earlier in the same call.  Calls that may overlap on the GPU (different

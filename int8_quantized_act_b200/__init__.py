@@ -29,7 +29,9 @@ __all__ = [
     "qlinear_fwd_bf16_workspace_bytes", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
     "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
     "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES", "qlinear_bwd",
-    "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout",
+    "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout", "qlinear_fwd_quantized",
+    "qlinear_swiglu_quantize", "qlinear_swiglu_bwd", "qweight_muon_workspace_bytes",
+    "qweight_muon_orthogonalize", "qweight_update_muon_sr", "qvector_adamw",
 ]
 
 QL_OK, QL_ERR_ARG, QL_ERR_SHAPE, QL_ERR_ALIGN = 0, 1, 2, 3
@@ -120,6 +122,21 @@ def lib() -> ctypes.CDLL:
     L.qlinear_bwd.restype = I
     L.qlinear_bwd.argtypes = [P, I, I64, I64, P, P, P, P, I64, I, P, I, P, P, P,
                               ctypes.c_size_t, P, P]
+    L.qlinear_fwd_quantized.restype = I
+    L.qlinear_fwd_quantized.argtypes = [P, P, I64, I64, P, P, I64, P, P, I, P, P]
+    L.qlinear_swiglu_quantize.restype = I
+    L.qlinear_swiglu_quantize.argtypes = [P, I, I64, I64, I64, P, I64, P, P, P]
+    L.qlinear_swiglu_bwd.restype = I
+    L.qlinear_swiglu_bwd.argtypes = [P, I, I64, P, I, I64, I64, P, I, P]
+    L.qweight_muon_workspace_bytes.restype = ctypes.c_size_t
+    L.qweight_muon_workspace_bytes.argtypes = [I64, I64]
+    L.qweight_muon_orthogonalize.restype = I
+    L.qweight_muon_orthogonalize.argtypes = [P, P, I64, I64, F, I, P, P, ctypes.c_size_t, P, P]
+    L.qweight_update_muon_sr.restype = I
+    L.qweight_update_muon_sr.argtypes = [P, P, P, I64, I64, F, F, ctypes.c_uint64,
+                                         ctypes.c_uint64, P, P]
+    L.qvector_adamw.restype = I
+    L.qvector_adamw.argtypes = [P, P, P, P, I64, ctypes.POINTER(_Optim), ctypes.c_uint64, P, P]
     L.qlinear_bwd_dx_noalloc.restype = I
     L.qlinear_bwd_dx_noalloc.argtypes = [P, I, I64, I64, P, P, I64, I, P, I, P, P]
     L.ql_set_gemm_timing_events.restype = None
@@ -316,6 +333,108 @@ def qlinear_fwd(x, wq, sw, bias, hadamard_block: int, y, xq_saved, sx_saved, sta
         _dev(sx_saved, "sx_saved", torch.float32), _dev(status, "status", torch.int32),
         _stream(stream))
     _check(code, "qlinear_fwd")
+
+
+def qlinear_fwd_quantized(xq, sx, wq, sw, bias, y, status, stream=None):
+    """y <- forward of the layer from an input already quantized (codes xq,
+    row scales sx), e.g. by qlinear_swiglu_quantize."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    for t, n in ((xq, "xq"), (sx, "sx"), (wq, "wq"), (sw, "sw"), (bias, "bias"), (y, "y")):
+        _contig(t, n)
+    _fits(wq, N, K, "wq", exact_cols=True)
+    _fits(y, M, N, "y", exact_cols=True)
+    _holds(sx, M, "sx")
+    _holds(sw, N, "sw")
+    _holds(bias, N, "bias")
+    _holds(status, 1, "status")
+    code = lib().qlinear_fwd_quantized(
+        _dev(xq, "xq", torch.int8), _dev(sx, "sx", torch.float32), M, K,
+        _dev(wq, "wq", torch.int8), _dev(sw, "sw", torch.float32), N,
+        _dev(bias, "bias", torch.float32), _dev(y, "y"), _dtype_code(y, "y"),
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qlinear_fwd_quantized")
+
+
+def qlinear_swiglu_quantize(ab, hq, sh, status, stream=None):
+    """hq, sh <- per-row quantization of h = silu(a) * b, ab = [a | b] [M, 2F]."""
+    M, F2 = ab.shape
+    F = F2 // 2
+    _fits(hq, M, F, "hq", exact_cols=False)
+    _holds(sh, M, "sh")
+    _holds(status, 1, "status")
+    code = lib().qlinear_swiglu_quantize(
+        _dev(ab, "ab"), _dtype_code(ab, "ab"), M, F, _rowmajor(ab, "ab"),
+        _dev(hq, "hq", torch.int8), _rowmajor(hq, "hq"), _dev(sh, "sh", torch.float32),
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qlinear_swiglu_quantize")
+
+
+def qlinear_swiglu_bwd(ab, dh, dab, stream=None):
+    """dab = [da | db] [M, 2F] <- the gate's backward from ab [M, 2F] and dh [M, F]."""
+    M, F2 = ab.shape
+    F = F2 // 2
+    for t, n in ((dh, "dh"), (dab, "dab")):
+        _contig(t, n)
+    _fits(dh, M, F, "dh", exact_cols=True)
+    _fits(dab, M, F2, "dab", exact_cols=True)
+    code = lib().qlinear_swiglu_bwd(
+        _dev(ab, "ab"), _dtype_code(ab, "ab"), _rowmajor(ab, "ab"), _dev(dh, "dh"),
+        _dtype_code(dh, "dh"), M, F, _dev(dab, "dab"), _dtype_code(dab, "dab"),
+        _stream(stream))
+    _check(code, "qlinear_swiglu_bwd")
+
+
+def qweight_muon_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().qweight_muon_workspace_bytes(N, K))
+
+
+def qweight_muon_orthogonalize(grad, mom, O, ws, status, momentum: float = 0.95,
+                               ns_steps: int = 5, stream=None):
+    """mom <- beta*mom + (1-beta)*grad; O (bf16 [N, K]) <- Newton-Schulz of
+    the Nesterov-blended update (the Muon direction)."""
+    N, K = grad.shape
+    for t, n in ((grad, "grad"), (mom, "mom"), (O, "O")):
+        _contig(t, n)
+    _fits(mom, N, K, "mom", exact_cols=True)
+    _fits(O, N, K, "O", exact_cols=True)
+    _holds(ws, qweight_muon_workspace_bytes(N, K), "ws")
+    _holds(status, 1, "status")
+    code = lib().qweight_muon_orthogonalize(
+        _dev(grad, "grad", torch.float32), _dev(mom, "mom", torch.float32), N, K, momentum,
+        ns_steps, _dev(O, "O", torch.bfloat16), _dev(ws, "ws", torch.uint8), ws.numel(),
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qweight_muon_orthogonalize")
+
+
+def qweight_update_muon_sr(wq, sw, O, lr: float, weight_decay: float, seed: int, step: int,
+                           status, stream=None):
+    """The Muon step of the int8 weight from O, with stochastic requantization, in place."""
+    N, K = wq.shape
+    for t, n in ((wq, "wq"), (sw, "sw"), (O, "O")):
+        _contig(t, n)
+    _fits(O, N, K, "O", exact_cols=True)
+    _holds(sw, N, "sw")
+    _holds(status, 1, "status")
+    code = lib().qweight_update_muon_sr(
+        _dev(wq, "wq", torch.int8), _dev(sw, "sw", torch.float32), _dev(O, "O", torch.bfloat16),
+        N, K, lr, weight_decay, seed, step, _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qweight_update_muon_sr")
+
+
+def qvector_adamw(p, g, m, v, opt: Optim, step: int, status, stream=None):
+    """AdamW on a float32 vector (biases and other float parameters), in place."""
+    n = p.numel()
+    for t, nm in ((p, "p"), (g, "g"), (m, "m"), (v, "v")):
+        _contig(t, nm)
+        _holds(t, n, nm)
+    _holds(status, 1, "status")
+    o = _Optim(opt.kind, opt.lr, opt.beta1, opt.beta2, opt.eps, opt.weight_decay)
+    code = lib().qvector_adamw(
+        _dev(p, "p", torch.float32), _dev(g, "g", torch.float32), _dev(m, "m", torch.float32),
+        _dev(v, "v", torch.float32), n, ctypes.byref(o), step,
+        _dev(status, "status", torch.int32), _stream(stream))
+    _check(code, "qvector_adamw")
 
 
 def qlinear_bwd_dx(dy, wq, sw, hadamard_block: int, dx, ws, status, stream=None):

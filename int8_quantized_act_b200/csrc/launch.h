@@ -25,11 +25,22 @@ void gemm_timing_events(cudaEvent_t* before, cudaEvent_t* after);
 // elements, out-of-range elements read as zero; 128-byte swizzle or none.
 // Whole rows as [rows][cols / L][L] (L elements = one 128-byte line; cols a
 // multiple of L, at most 256 lines), boxes of box_rows rows, 128-byte swizzle.
+// Any rank (1..5): dims[0] innermost (elements), strides[i] the byte pitch of
+// dimension i + 1 (rank - 1 of them), box the copied extent per dimension.
+bool encode_tmap(CUtensorMap* m, int elem_bytes, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box, bool swizzle128);
 bool encode_rows_128b(CUtensorMap* m, int elem_bytes, const void* base, uint64_t cols,
                       uint64_t rows, uint64_t pitch, uint32_t box_rows);
 bool encode_tmap_2d(CUtensorMap* m, int elem_bytes, const void* base, uint64_t inner,
                     uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
                     bool swizzle128);
+
+// The host checks of qlinear_bwd_dx that come before its workspace is looked
+// at, in its order (argument, shape, then null pointers): returns the status
+// code, and sets *noop when the call has nothing to compute (M == 0 or K == 0).
+int check_bwd_dx_args(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
+                      const float* sw, int64_t K, int hadamard_block, const void* dx, int dxt,
+                      const int32_t* d_status, bool* noop);
 
 // -------------------------------------------------------------- row kernels
 // Per-row quantization (optionally scaled per column and rotated); see
@@ -38,6 +49,15 @@ cudaError_t launch_quant_rows(const void* x, int xt, int64_t rows, int64_t cols,
                               const float* col_scale, int B, float hc, unsigned flags,
                               int8_t* q, int64_t ldq, float* row_scale, int32_t* status,
                               cudaStream_t s);
+
+// The same quantization for bf16 rows of 128..16384 columns (a multiple of
+// 128) and blocks B <= 128 without a column scale, two threads per
+// 128-column block, rows in and codes out by TMA: eligible when there are
+// enough rows to give every SM a tile.  Launched by launch_quant_rows.
+bool quant_blk_eligible(int64_t rows, int64_t cols, int64_t ldx, int B, bool col_scale);
+cudaError_t launch_quant_blk(const void* x, int64_t rows, int64_t cols, int64_t ldx, int B,
+                             float hc, unsigned flags, int8_t* q, int64_t ldq, float* rs,
+                             int32_t* st, cudaStream_t s);
 
 // y = x R per row (x may equal y).  xt / yt: 0 = float32, 1 = bf16.
 cudaError_t launch_hadamard(const void* x, int xt, int64_t ldx, void* y, int yt, int64_t ldy,
@@ -79,6 +99,36 @@ cudaError_t launch_dualquant(const void* dy, int dyt, int64_t M, int64_t N, cons
 // out[r, :] = bias (or 0), dtype ot; used when the contraction is empty.
 cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, const float* bias,
                              cudaStream_t s);
+
+// -------------------------------------------------------------- MuonAuxAdamW
+// Workspace of the Newton-Schulz iteration for an [N, K] weight (r = min,
+// c = max of N, K): ||U||^2, X [r, c] and X^T bf16, A, B [r, r] bf16, A A
+// [r, r] and B X [r, c] float32; byte offsets, each 256-byte aligned.
+struct MuonLayout {
+  int64_t sumsq, X, Xt, A, A2, Bm, P, total;
+};
+MuonLayout muon_layout(int64_t N, int64_t K);
+// M <- beta*M + (1-beta)*G; O [N, K] bf16 <- NS(U) after `steps` (>= 1) steps.
+cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, int64_t K,
+                                      float beta, int steps, void* O, void* ws, int32_t* status,
+                                      cudaStream_t s);
+// p <- AdamW(p, g) elementwise (m, v in place), the constants of UpdateConsts.
+struct UpdateConsts;
+cudaError_t launch_adamw_vector(float* p, const float* g, float* m, float* v, int64_t n,
+                                const UpdateConsts& c, int32_t* status, cudaStream_t s);
+// w = s*q; w' = w*a - st*O (O bf16 [N, K]); per-row stochastic requantization.
+cudaError_t launch_update_dir(int8_t* wq, float* sw, const void* O, int64_t N, int64_t K, float a,
+                              float st, uint64_t seed, uint64_t step, int32_t* status,
+                              cudaStream_t s);
+
+// -------------------------------------------------------------- SwiGLU gate
+// hq, sh = per-row quantization of h = silu(a) * b for ab = [a | b] [M, 2F]
+// (dtype abt, pitch ldab); F <= 16384.
+cudaError_t launch_swiglu_quant(const void* ab, int abt, int64_t M, int64_t F, int64_t ldab,
+                                int8_t* hq, int64_t ldh, float* sh, int32_t* st, cudaStream_t s);
+// dab [M, 2F] (dtype dabt, contiguous) = [da | db] from ab and dh [M, F] (dht).
+cudaError_t launch_swiglu_bwd(const void* ab, int abt, int64_t ldab, const void* dh, int dht,
+                              int64_t M, int64_t F, void* dab, int dabt, cudaStream_t s);
 
 // -------------------------------------------------------------- GEMM
 // out[r, c] = ((float)acc[r,c] * row_scale[r]) * col_scale[c] + bias[c]

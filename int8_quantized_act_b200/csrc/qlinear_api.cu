@@ -162,6 +162,27 @@ int run_dw_product(const int8_t* dyq_c, const int8_t* xq, const float* s2, int64
 
 }  // namespace
 
+namespace ql {
+
+int check_bwd_dx_args(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
+                      const float* sw, int64_t K, int hadamard_block, const void* dx, int dxt,
+                      const int32_t* d_status, bool* noop) {
+  *noop = false;
+  if (!valid_dtype(dyt) || !valid_dtype(dxt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || M > INT32_MAX ||
+      K > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
+  if (M == 0 || K == 0) {
+    *noop = true;
+    return QL_OK;
+  }
+  if (!dx || !d_status || (N > 0 && (!dy || !wq || !sw))) return QL_ERR_ARG;
+  return QL_OK;
+}
+
+}  // namespace ql
+
 extern "C" {
 
 void ql_set_gemm_timing_events(void* const* before, void* const* after, int n) {
@@ -267,6 +288,56 @@ int qlinear_fwd(const void* x, int xt, int64_t M, int64_t K, const int8_t* wq, c
   return cuda_status(ql::launch_gemm_i8(xq_saved, false, K, wq, false, K, M, N, K, ep, d_status, s));
 }
 
+int qlinear_fwd_quantized(const int8_t* xq, const float* sx, int64_t M, int64_t K,
+                          const int8_t* wq, const float* sw, int64_t N, const float* bias, void* y,
+                          int yt, int32_t* d_status, void* stream) {
+  if (!valid_dtype(yt)) return QL_ERR_ARG;
+  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || M > INT32_MAX || N > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (K > QL_MAX_CONTRACTION) return QL_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return QL_OK;
+  if (!y || !d_status || (K > 0 && (!xq || !sx || !wq || !sw))) return QL_ERR_ARG;
+  if (!aligned16(y) || (bias && !aligned16(bias)) ||
+      (K > 0 && (!aligned16(xq) || !aligned16(wq) || !aligned16(sw))))
+    return QL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  if (K == 0) return cuda_status(ql::launch_fill_rows(y, yt, M, N, bias, s));
+  GemmEpilogue ep;
+  ep.out = y;
+  ep.out_bf16 = yt == QL_BF16;
+  ep.ldo = N;
+  ep.row_scale = sx;
+  ep.col_scale = sw;
+  ep.bias = bias;
+  return cuda_status(ql::launch_gemm_i8(xq, false, K, wq, false, K, M, N, K, ep, d_status, s));
+}
+
+int qlinear_swiglu_quantize(const void* ab, int abt, int64_t M, int64_t F, int64_t ldab,
+                            int8_t* hq, int64_t ldh, float* sh, int32_t* d_status, void* stream) {
+  if (!valid_dtype(abt)) return QL_ERR_ARG;
+  if (M < 0 || F < 16 || F % 16 != 0 || ldab < 2 * F || ldh < F || ldh % 16 != 0 ||
+      M > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (F > 16384) return QL_ERR_UNSUPPORTED;
+  if (M == 0) return QL_OK;
+  if (!ab || !hq || !sh || !d_status) return QL_ERR_ARG;
+  if (!aligned16(ab) || !aligned16(hq) || (ldab * elem_size(abt)) % 16 != 0) return QL_ERR_ALIGN;
+  return cuda_status(ql::launch_swiglu_quant(ab, abt, M, F, ldab, hq, ldh, sh, d_status,
+                                             as_stream(stream)));
+}
+
+int qlinear_swiglu_bwd(const void* ab, int abt, int64_t ldab, const void* dh, int dht, int64_t M,
+                       int64_t F, void* dab, int dabt, void* stream) {
+  if (!valid_dtype(abt) || !valid_dtype(dht) || !valid_dtype(dabt)) return QL_ERR_ARG;
+  if (M < 0 || F < 16 || F % 16 != 0 || ldab < 2 * F || F > INT32_MAX / 2) return QL_ERR_SHAPE;
+  if (M == 0) return QL_OK;
+  if (!ab || !dh || !dab) return QL_ERR_ARG;
+  if (!aligned16(ab) || !aligned16(dh) || !aligned16(dab) || (ldab * elem_size(abt)) % 16 != 0)
+    return QL_ERR_ALIGN;
+  return cuda_status(ql::launch_swiglu_bwd(ab, abt, ldab, dh, dht, M, F, dab, dabt,
+                                           as_stream(stream)));
+}
+
 int qlinear_dequantize(const int8_t* wq, int64_t ldq, const float* sw, int64_t N, int64_t K,
                        int hadamard_block, void* w, int wt, int64_t ldw, void* stream) {
   if (!valid_dtype(wt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
@@ -336,14 +407,12 @@ int qlinear_fwd_bf16(const void* x, int xt, int64_t M, int64_t K, const void* wq
 int qlinear_bwd_dx(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
                    const float* sw, int64_t K, int hadamard_block, void* dx, int dxt, void* ws,
                    size_t ws_bytes, int32_t* d_status, void* stream) {
-  if (!valid_dtype(dyt) || !valid_dtype(dxt) || !valid_block(hadamard_block)) return QL_ERR_ARG;
-  if (M < 0 || K < 0 || N < 0 || K % 16 != 0 || N % 16 != 0 || M > INT32_MAX ||
-      K > INT32_MAX)
-    return QL_ERR_SHAPE;
-  if (hadamard_block > 0 && K % hadamard_block != 0) return QL_ERR_SHAPE;
-  if (M == 0 || K == 0) return QL_OK;
+  bool noop = false;
+  const int pre = ql::check_bwd_dx_args(dy, dyt, M, N, wq, sw, K, hadamard_block, dx, dxt,
+                                        d_status, &noop);
+  if (pre != QL_OK || noop) return pre;
   const WsLayout L = ws_layout(M, N, K, hadamard_block);
-  if (!dx || !d_status || !ws || (N > 0 && (!dy || !wq || !sw))) return QL_ERR_ARG;
+  if (!ws) return QL_ERR_ARG;
   if (ws_bytes < L.total) return QL_ERR_SHAPE;
   if (!aligned16(dx) || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
       (N > 0 && (!aligned16(dy) || !aligned16(wq) || !aligned16(sw))))
@@ -460,6 +529,69 @@ int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
   const int r = run_dx_product(dyq_r, wq, s1, M, N, K, hadamard_block, dx, dxt, ws, L, d_status, s);
   if (r != QL_OK) return r;
   return run_dw_product(dyq_c, xq, s2, M, N, K, dw, ws, L, d_status, s);
+}
+
+size_t qweight_muon_workspace_bytes(int64_t N, int64_t K) {
+  if (N < 0 || K < 0) return 0;
+  return static_cast<size_t>(ql::muon_layout(N, K).total);
+}
+
+int qweight_muon_orthogonalize(const float* grad, float* mom, int64_t N, int64_t K, float momentum,
+                               int ns_steps, void* O, void* ws, size_t ws_bytes,
+                               int32_t* d_status, void* stream) {
+  if (!(momentum >= 0.0f && momentum < 1.0f) || ns_steps < 1 || ns_steps > 16) return QL_ERR_ARG;
+  if (N < 0 || K < 0 || N % 16 != 0 || K % 16 != 0 || N > INT32_MAX || K > INT32_MAX)
+    return QL_ERR_SHAPE;
+  if (N == 0 || K == 0) return QL_OK;
+  if (!grad || !mom || !O || !ws || !d_status) return QL_ERR_ARG;
+  if (ws_bytes < qweight_muon_workspace_bytes(N, K)) return QL_ERR_SHAPE;
+  if (!aligned16(grad) || !aligned16(mom) || !aligned16(O) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return QL_ERR_ALIGN;
+  return cuda_status(ql::launch_muon_orthogonalize(grad, mom, N, K, momentum, ns_steps, O, ws,
+                                                   d_status, as_stream(stream)));
+}
+
+int qweight_update_muon_sr(int8_t* wq, float* sw, const void* O, int64_t N, int64_t K, float lr,
+                           float weight_decay, uint64_t seed, uint64_t step, int32_t* d_status,
+                           void* stream) {
+  if (!std::isfinite(lr) || !std::isfinite(weight_decay) || step < 1) return QL_ERR_ARG;
+  if (N < 0 || K < 0 || N % 16 != 0 || K % 16 != 0 || N > INT32_MAX) return QL_ERR_SHAPE;
+  if (K > 32768) return QL_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return QL_OK;
+  if (!wq || !sw || !O || !d_status) return QL_ERR_ARG;
+  if (!aligned16(wq) || !aligned16(O)) return QL_ERR_ALIGN;
+  // Host constants in float64, each rounded once: the decoupled decay factor
+  // and the step size times max(1, N/K)^0.5.
+  const double scale = N > K ? std::sqrt(static_cast<double>(N) / static_cast<double>(K)) : 1.0;
+  const float a = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(weight_decay));
+  const float st = static_cast<float>(static_cast<double>(lr) * scale);
+  return cuda_status(ql::launch_update_dir(wq, sw, O, N, K, a, st, seed, step, d_status,
+                                           as_stream(stream)));
+}
+
+int qvector_adamw(float* p, const float* g, float* m, float* v, int64_t n, const ql_optim* opt,
+                  uint64_t step, int32_t* d_status, void* stream) {
+  if (!opt || opt->kind != QL_ADAMW || step < 1 || !std::isfinite(opt->lr) ||
+      !(opt->beta1 >= 0.0f && opt->beta1 < 1.0f) || !(opt->beta2 >= 0.0f && opt->beta2 < 1.0f) ||
+      !std::isfinite(opt->eps) || !std::isfinite(opt->weight_decay))
+    return QL_ERR_ARG;
+  if (n < 0) return QL_ERR_SHAPE;
+  if (n == 0) return QL_OK;
+  if (!p || !g || !m || !v || !d_status) return QL_ERR_ARG;
+  ql::UpdateConsts c;
+  c.kind = QL_ADAMW;
+  c.lr = opt->lr;
+  const double t = static_cast<double>(step);
+  c.a = static_cast<float>(1.0 - static_cast<double>(opt->lr) * static_cast<double>(opt->weight_decay));
+  c.st = static_cast<float>(static_cast<double>(opt->lr) / (1.0 - std::pow(static_cast<double>(opt->beta1), t)));
+  c.rbc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(opt->beta2), t)));
+  c.b1 = opt->beta1;
+  c.b2 = opt->beta2;
+  c.omb1 = static_cast<float>(1.0 - static_cast<double>(opt->beta1));
+  c.omb2 = static_cast<float>(1.0 - static_cast<double>(opt->beta2));
+  c.eps = opt->eps;
+  return cuda_status(ql::launch_adamw_vector(p, g, m, v, n, c, d_status, as_stream(stream)));
 }
 
 int qweight_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,

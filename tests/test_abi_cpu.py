@@ -154,6 +154,33 @@ def test_host_validation_returns_before_any_launch(L):
     assert L.qlinear_hadamard(fake(A), 0, 32, fake(A), 0, 32, 4, 32, 0, None) == ql.QL_ERR_ARG
 
 
+def test_noalloc_checks_arguments_before_capacity(L):
+    """qlinear_bwd_dx_noalloc returns qlinear_bwd_dx's code for a bad
+    argument or shape even when the sizes exceed its scratch, treats an empty
+    output as a no-op, and only then reports the capacity; none of these
+    calls reaches the device."""
+    A = 0x10000
+    f, g = L.qlinear_bwd_dx_noalloc, L.qlinear_bwd_dx
+    M, N, K = 12000, 7168, 5376  # workspace far beyond the 32 MiB scratch
+    assert ql.qlinear_workspace_bytes(M, N, K, 0) > ql.QL_NOALLOC_SCRATCH_BYTES
+    ws = fake(0x100000)
+    cases = [
+        ((fake(A), 7, M, N, fake(A), fake(A), K, 0, fake(A), 0), ql.QL_ERR_ARG),      # dtype
+        ((fake(A), 0, M, N, fake(A), fake(A), K, 3, fake(A), 0), ql.QL_ERR_ARG),      # block
+        ((fake(A), 0, M, N, fake(A), fake(A), K + 8, 0, fake(A), 0), ql.QL_ERR_SHAPE),  # K % 16
+        ((fake(A), 0, M, N, fake(A), fake(A), K + 16, 32, fake(A), 0), ql.QL_ERR_SHAPE),  # K % B
+        ((fake(A), 0, M, N, fake(A), fake(A), K, 0, None, 0), ql.QL_ERR_ARG),         # null dx
+    ]
+    for args, code in cases:
+        assert f(*args, fake(A), None) == code
+        assert g(*args, ws, 1 << 40, fake(A), None) == code
+    # nothing to compute: no-op, whatever the other sizes
+    assert f(fake(A), 0, M, N, fake(A), fake(A), 0, 0, fake(A), 0, fake(A), None) == ql.QL_OK
+    assert f(None, 0, 0, 10 ** 9, None, None, 16, 0, None, 0, None, None) == ql.QL_OK
+    # valid arguments, too large for the scratch
+    assert f(fake(A), 0, M, N, fake(A), fake(A), K, 0, fake(A), 0, fake(A), None) == ql.QL_ERR_UNSUPPORTED
+
+
 def test_update_validation(L):
     A = 0x10000
     opt = ql._Optim(ql.QL_SGD, 0.1, 0.9, 0.999, 1e-8, 0.5)

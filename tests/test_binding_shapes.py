@@ -57,6 +57,16 @@ def test_valid_calls_pass(fake):
                    E(M), st())
     ql.qlinear_fwd(E(1, K), E(N, K, dtype=I8), E(N), None, 128, E(1, N), E(1, K, dtype=I8),
                    E(1), st())
+    # the SwiGLU gate, its backward and the forward from codes (the MLP step)
+    ql.qlinear_swiglu_quantize(E(M, 2 * K, dtype=BF), E(M, K, dtype=I8), E(M), st())
+    ql.qlinear_swiglu_bwd(E(M, 2 * K, dtype=BF), E(M, K, dtype=BF), E(M, 2 * K, dtype=BF))
+    ql.qlinear_swiglu_bwd(E(M, 2 * K), E(M, K), E(M, 2 * K))
+    ql.qlinear_fwd_quantized(E(M, K, dtype=I8), E(M), E(N, K, dtype=I8), E(N), E(N), E(M, N), st())
+    # MuonAuxAdamW (the Muon GPU tests and bench)
+    ql.qweight_muon_orthogonalize(E(M, K), E(M, K), E(M, K, dtype=BF),
+                                  E(ql.qweight_muon_workspace_bytes(M, K), dtype=torch.uint8), st())
+    ql.qweight_update_muon_sr(E(M, K, dtype=I8), E(M), E(M, K, dtype=BF), 0.02, 0.01, 1, 1, st())
+    ql.qvector_adamw(E(N), E(N), E(N), E(N), ql.Optim(), 1, st())
     # M = 0 and K = 0 (the degenerate-size GPU test)
     ql.qlinear_fwd(E(0, 64), E(32, 64, dtype=I8), E(32), None, 0, E(0, 32), E(0, 64, dtype=I8),
                    E(0), st())
@@ -80,7 +90,7 @@ def test_valid_calls_pass(fake):
                          g=E(N), g_m=E(N), g_v=E(N))
     ql.qlinear_dequantize(E(N, K, dtype=I8), E(N), 128, E(N, K))
     ql.qlinear_dequantize(E(24, 512, dtype=I8), E(24), 64, E(24, 640)[:, :512])
-    assert len(fake.calls) == 21
+    assert len(fake.calls) == 30
 
 
 # ------------------------------------------------------------------ refused
@@ -152,6 +162,28 @@ BAD = [
                                   E(N, K), 0, 1, st(), g=E(N - 1), g_m=E(N), g_v=E(N))),
     ("dequantize: scales short",
      lambda: ql.qlinear_dequantize(E(N, K, dtype=I8), E(N - 1), 0, E(N, K))),
+    ("fwd from codes: scales short",
+     lambda: ql.qlinear_fwd_quantized(E(M, K, dtype=I8), E(M - 1), E(N, K, dtype=I8), E(N),
+                                      None, E(M, N), st())),
+    ("fwd from codes: y too small",
+     lambda: ql.qlinear_fwd_quantized(E(M, K, dtype=I8), E(M), E(N, K, dtype=I8), E(N), None,
+                                      E(M - 1, N), st())),
+    ("muon: momentum too small",
+     lambda: ql.qweight_muon_orthogonalize(E(M, K), E(M - 1, K), E(M, K, dtype=BF),
+                                           E(1 << 22, dtype=torch.uint8), st())),
+    ("muon step: update of another shape",
+     lambda: ql.qweight_update_muon_sr(E(M, K, dtype=I8), E(M), E(M, K - 16, dtype=BF), 0.02, 0.0,
+                                       1, 1, st())),
+    ("vector adamw: moments short",
+     lambda: ql.qvector_adamw(E(N), E(N), E(N - 1), E(N), ql.Optim(), 1, st())),
+    ("gate: codes too narrow",
+     lambda: ql.qlinear_swiglu_quantize(E(M, 2 * K, dtype=BF), E(M, K - 16, dtype=I8), E(M), st())),
+    ("gate: scales short",
+     lambda: ql.qlinear_swiglu_quantize(E(M, 2 * K, dtype=BF), E(M, K, dtype=I8), E(M - 1), st())),
+    ("gate backward: dh too small",
+     lambda: ql.qlinear_swiglu_bwd(E(M, 2 * K, dtype=BF), E(M - 1, K, dtype=BF), E(M, 2 * K, dtype=BF))),
+    ("gate backward: output too small",
+     lambda: ql.qlinear_swiglu_bwd(E(M, 2 * K, dtype=BF), E(M, K, dtype=BF), E(M, 2 * K - 16, dtype=BF))),
 ]
 
 

@@ -340,15 +340,26 @@ def test_full_layer_sampled(M):
     assert_close(host(y)[rows], ry, D, bf16=True, what="y")
 
     dy_t = dev(d["dy_bf16"])
-    dx, _ = gpu_dx(dy_t, wq, sw, B, torch.bfloat16)
+    dx, ws_dx = gpu_dx(dy_t, wq, sw, B, torch.bfloat16)
+    # every row-quantized gradient code and row scale of the input gradient
+    rq_all, rs1_all, rst = oracle.bwd_prep_rows(d["dy"], sw_np)
+    assert rst == 0
+    s1_off = (M * N + 255) // 256 * 256
+    assert np.array_equal(host(ws_dx[:M * N]).view(np.int8).reshape(M, N), rq_all)
+    assert np.array_equal(host(ws_dx[s1_off: s1_off + 4 * M]).view(np.float32), rs1_all)
+    del ws_dx
     rdx, rq, rs1, _ = oracle.bwd_dx(d["dy"][rows], wq_np, sw_np, B)
     acc, _ = oracle.gemm_nn(rq, wq_np)
     assert_close(host(dx)[rows], rdx, rotated_magnitude(acc * rs1[:, None].astype(np.float64), B),
                  bf16=True, what="dX")
 
     dw, db, ws = gpu_dw(dy_t, xq, sx)
-    dx2, dw2, db2, _ = gpu_bwd(dy_t, wq, sw, xq, sx, B, torch.bfloat16)
+    dx2, dw2, db2, ws2 = gpu_bwd(dy_t, wq, sw, xq, sx, B, torch.bfloat16)
     assert torch.equal(dx2, dx) and torch.equal(dw2, dw) and torch.equal(db2, db)
+    # the combined backward's row-quantized codes and scales, all rows
+    assert np.array_equal(host(ws2[:M * N]).view(np.int8).reshape(M, N), rq_all)
+    assert np.array_equal(host(ws2[s1_off: s1_off + 4 * M]).view(np.float32), rs1_all)
+    del ws2, rq_all
     cols = _sample_rows(N, 12, M + 1)
     rdw, rdb, rqc, rs2, _ = oracle.bwd_dw(d["dy"][:, cols], xq_np, sx_np)
     gq = host(ws[: M * N]).view(np.int8).reshape(M, N)
