@@ -8,12 +8,16 @@
 // sums (the bias gradient) and, optionally, the row maxima; pass 2
 // (dualquant) writes one or both int8 code sets elementwise.
 //
-// Both passes stream dY in tiles of 256 columns x 32 rows (bf16) or 16 rows
-// (float32), 16 KB each, through a 4-stage ring: a producer warp issues one
-// TMA load per tile (rows / columns past the matrix read as zero) while 8
-// consumer warps work on earlier tiles, so ~64 KB per CTA are in flight
-// without tying up registers.  Block (x, y) owns column block x and a
-// contiguous run of row tiles, so per-column state stays in registers.
+// Both passes stream dY in tiles of 1024 columns x 16 rows (bf16) or 8 rows
+// (float32), 32 KB each, through a 3-stage ring: a producer warp issues one
+// TMA load per 256-column quarter of a tile (rows / columns past the matrix
+// read as zero; quarters wholly past the last column are not loaded), so
+// each row of a tile is read as 2 KB in a row, while 8 consumer warps work on
+// earlier tiles: warp w takes quarter w % 4 and half w / 4 of the rows, 8 (4)
+// rows.  Up to 96 KB per CTA and two CTAs per SM are in flight without tying
+// up registers.  Block (x, y) owns column block x and a contiguous run of row
+// tiles, so per-column state stays in registers.  The per-row factors of a
+// warp's rows are loaded one row per lane and broadcast by shuffles.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -26,15 +30,18 @@ namespace ql {
 
 namespace {
 
-constexpr int kCols = 256;        // columns per tile (8 per lane)
-constexpr int kStages = 4;
-constexpr int kTileBytes = 16384;
+constexpr int kCols = 256;        // columns of a quarter (8 per lane)
+constexpr int kSub = 4;           // quarters per tile
+constexpr int kBlockCols = kSub * kCols;
+constexpr int kStages = 3;
+constexpr int kTileBytes = 32768;
 constexpr int kThreads = 288;     // 8 consumer warps + 1 producer warp
 
 template <typename InT>
 struct Tile {
-  static constexpr int kRows = kTileBytes / (kCols * static_cast<int>(sizeof(InT)));  // 32 / 16
-  static constexpr int kRowsPerWarp = kRows / 8;
+  static constexpr int kRows = kTileBytes / (kBlockCols * static_cast<int>(sizeof(InT)));  // 16 / 8
+  static constexpr int kRowsPerWarp = kRows / (8 / kSub);                                    // 8 / 4
+  static_assert(kRowsPerWarp % 2 == 0 && kRowsPerWarp <= 32, "rows of a warp: pairs, one per lane");
 };
 
 // 8 consecutive elements of a staged row as float32, read with 16-byte
@@ -78,16 +85,19 @@ struct Ring {
     }
   }
 
-  // Producer (one thread): load tile t of column block cb into each free stage.
-  __device__ void produce(const CUtensorMap* tm, int cb, int t0, int t1, int rows_per_tile) {
+  // Producer (one thread): load tile t of column block cb into each free
+  // stage, the first nsub quarters (those that start before the last column).
+  __device__ void produce(const CUtensorMap* tm, int cb, int nsub, int t0, int t1,
+                          int rows_per_tile) {
     uint32_t issued = 0, issued_phase = 0;
     for (int t = t0, k = 0; t < t1; ++t, ++k) {
       const int s = k % kStages;
       const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
       if (k >= kStages && !mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag)) break;
-      mbar_arrive_expect_tx(smem_u32(&full[s]), kTileBytes);
-      tma_load_2d(smem_u32(buf + s * kTileBytes), tm, smem_u32(&full[s]), cb * kCols,
-                  t * rows_per_tile);
+      mbar_arrive_expect_tx(smem_u32(&full[s]), static_cast<uint32_t>(nsub * (kTileBytes / kSub)));
+      for (int q = 0; q < nsub; ++q)
+        tma_load_2d(smem_u32(buf + s * kTileBytes + q * (kTileBytes / kSub)), tm,
+                    smem_u32(&full[s]), cb * kBlockCols + q * kCols, t * rows_per_tile);
       issued |= 1u << s;
       issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
     }
@@ -128,6 +138,7 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   // The final per-column reduction reuses the (drained) ring buffer.
   uint32_t(*s_max)[kCols] = reinterpret_cast<uint32_t(*)[kCols]>(buf);
   float(*s_sum)[kCols] = reinterpret_cast<float(*)[kCols]>(buf + 8 * kCols * 4);
+  static_assert(8 * kCols * 8 <= kStages * kTileBytes, "reduction fits in the ring");
   Ring ring{buf, s_full, s_empty, &s_abort};
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   ring.init(tid);
@@ -136,7 +147,10 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   const int tiles = static_cast<int>((M + T::kRows - 1) / T::kRows);
   const int t0 = blockIdx.y * tiles_per_cta;
   const int t1 = t0 + tiles_per_cta < tiles ? t0 + tiles_per_cta : tiles;
-  const int col = cb * kCols + lane * 8;
+  const int nsub = min(kSub, (N - cb * kBlockCols + kCols - 1) / kCols);
+  const int sub = warp % kSub;                      // this warp's quarter
+  const bool live = warp < 8 && sub < nsub;         // it holds columns of the matrix
+  const int col = cb * kBlockCols + sub * kCols + lane * 8;
   // Maxima as floats with NaN-propagating max (max.NaN.f32) over |x|
   // operands: a NaN or infinite product dY*s_x (an infinite dY in a row whose
   // s_x is 0 gives NaN) makes its column maximum NaN or +inf, and likewise
@@ -148,35 +162,39 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   if (warp == 8) {
     if (lane == 0) {
       tma_prefetch_desc(&tm);
-      ring.produce(&tm, cb, t0, t1, T::kRows);
+      ring.produce(&tm, cb, nsub, t0, t1, T::kRows);
     }
     __syncwarp();
   } else {
     float w8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (ROWMAX && col < N) load8(sw + col, w8);
-    // The row scales of the next tile are loaded while this one is worked on.
-    float fcur[T::kRowsPerWarp], fnext[T::kRowsPerWarp];
-    auto load_scales = [&](int t, float (&f)[T::kRowsPerWarp]) {
-#pragma unroll
-      for (int j = 0; j < T::kRowsPerWarp; ++j) {
-        const int64_t m = static_cast<int64_t>(t) * T::kRows + warp * T::kRowsPerWarp + j;
-        f[j] = (t < t1 && m < M) ? __ldg(sx + m) : 0.0f;
-      }
+    const uint32_t qoff = static_cast<uint32_t>(sub * (kTileBytes / kSub));
+    // Lane j < kRowsPerWarp holds the factor s_x of row j of this warp's rows;
+    // the next tile's are loaded while this one is worked on.
+    constexpr int RW = T::kRowsPerWarp;
+    const int rw0 = (warp / kSub) * RW;  // this warp's first row of a tile
+    auto load_scale = [&](int t) {
+      const int64_t m = static_cast<int64_t>(t) * T::kRows + rw0 + lane;
+      return (lane < RW && t < t1 && m < M) ? __ldg(sx + m) : 0.0f;
     };
-    load_scales(t0, fcur);
-    ring.consume(t0, t1, lane, [&](int t, uint32_t tile) {
-      load_scales(t + 1, fnext);
+    float fcur = load_scale(t0);
+    ring.consume(t0, t1, lane, [&](int t, uint32_t stage) {
+      if (!live) return;  // a quarter past the last column: nothing loaded
+      const uint32_t tile = stage + qoff;
+      const float fnext = load_scale(t + 1);
+      const int64_t m0 = static_cast<int64_t>(t) * T::kRows + rw0;
+      uint32_t rmax = 0;  // lane j: the maximum of row j of this warp's rows
       // Two rows per step, so one three-operand max covers both.  Rows of
       // the tile past M were zero-filled by the copy and their factors are
       // 0: they add nothing to the column maxima and sums.
 #pragma unroll
-      for (int j = 0; j < T::kRowsPerWarp; j += 2) {
-        const int r = warp * T::kRowsPerWarp + j;
-        const int64_t m = static_cast<int64_t>(t) * T::kRows + r;
+      for (int j = 0; j < RW; j += 2) {
+        const int r = rw0 + j;
         float d0[8], d1[8];
         smem_load8<InT>(tile + (r * kCols + lane * 8) * sizeof(InT), d0);
         smem_load8<InT>(tile + ((r + 1) * kCols + lane * 8) * sizeof(InT), d1);
-        const float f0 = fcur[j], f1 = fcur[j + 1];
+        const float f0 = __shfl_sync(0xFFFFFFFFu, fcur, j);
+        const float f1 = __shfl_sync(0xFFFFFFFFu, fcur, j + 1);
         float rb0 = 0.0f, rb1 = 0.0f;
         // Products (only their magnitudes are used, no sum follows them) and
         // column sums two columns per instruction.
@@ -200,15 +218,14 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
           // Non-negative floats order like their bit patterns; NaN sorts last.
           const uint32_t u0 = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(rb0));
           const uint32_t u1 = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(rb1));
-          if (lane == 0) {
-            if (m < M) atomicMax(rowmax + m, u0);
-            if (m + 1 < M) atomicMax(rowmax + m + 1, u1);
-          }
-          rbad = max(rbad, max(u0, u1));
+          rmax = lane == j ? u0 : (lane == j + 1 ? u1 : rmax);
         }
       }
-#pragma unroll
-      for (int j = 0; j < T::kRowsPerWarp; ++j) fcur[j] = fnext[j];
+      if (ROWMAX && lane < RW && m0 + lane < M) {
+        atomicMax(rowmax + m0 + lane, rmax);
+        rbad = max(rbad, rmax);
+      }
+      fcur = fnext;
     });
   }
   __syncthreads();  // ring drained (the producer waited for its copies): reuse it
@@ -220,22 +237,24 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
     }
   }
   __syncthreads();
-  if (tid < kCols && cb * kCols + tid < N) {
-    const int slot = (tid % 8) * 32 + tid / 8;
+  for (int c = tid; c < kBlockCols; c += blockDim.x) {
+    if (cb * kBlockCols + c >= N) break;
+    const int q = c / kCols, j = c % kCols;
+    const int slot = (j % 8) * 32 + j / 8;
     uint32_t a = 0;
     double t = 0.0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      a = max(a, s_max[w][slot]);
-      t += static_cast<double>(s_sum[w][slot]);
+    for (int h = 0; h < 8 / kSub; ++h) {  // the warps of quarter q
+      a = max(a, s_max[q + kSub * h][slot]);
+      t += static_cast<double>(s_sum[q + kSub * h][slot]);
     }
     // A NaN or infinite maximum: report it (the affected outputs are
     // unspecified).
     if (a >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
-    atomicMax(colmax + cb * kCols + tid, a);
-    atomicAdd(colsum + cb * kCols + tid, t);
+    atomicMax(colmax + cb * kBlockCols + c, a);
+    atomicAdd(colsum + cb * kBlockCols + c, t);
   }
-  if (ROWMAX && rbad >= kInfBits && lane == 0) atomicOr(status, 1 << QL_ERR_NONFINITE);
+  if (ROWMAX && rbad >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
   if (tid == 0 && s_abort) atomicOr(status, 1 << QL_ERR_TIMEOUT);
 }
 
@@ -261,12 +280,15 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
   const int tiles = static_cast<int>((M + T::kRows - 1) / T::kRows);
   const int t0 = blockIdx.y * tiles_per_cta;
   const int t1 = t0 + tiles_per_cta < tiles ? t0 + tiles_per_cta : tiles;
-  const int col = cb * kCols + lane * 8;
+  const int nsub = min(kSub, (N - cb * kBlockCols + kCols - 1) / kCols);
+  const int sub = warp % kSub;                      // this warp's quarter
+  const bool live = warp < 8 && sub < nsub;         // it holds columns of the matrix
+  const int col = cb * kBlockCols + sub * kCols + lane * 8;
   const bool cv = col < N;
   if (warp == 8) {
     if (lane == 0) {
       tma_prefetch_desc(&tm);
-      ring.produce(&tm, cb, t0, t1, T::kRows);
+      ring.produce(&tm, cb, nsub, t0, t1, T::kRows);
     }
     __syncwarp();
   } else {
@@ -275,48 +297,61 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
       load8(cinv2 + col, iv);
       if (Q1) load8(cs1 + col, w8);
     }
-    // The next tile's row factors are loaded while this one is worked on.
-    float f2cur[T::kRowsPerWarp], f2next[T::kRowsPerWarp];
-    float r1cur[T::kRowsPerWarp], r1next[T::kRowsPerWarp];
-    auto load_rows = [&](int t, float (&f2)[T::kRowsPerWarp], float (&r1)[T::kRowsPerWarp]) {
-#pragma unroll
-      for (int j = 0; j < T::kRowsPerWarp; ++j) {
-        const int64_t m = static_cast<int64_t>(t) * T::kRows + warp * T::kRowsPerWarp + j;
-        const bool in = t < t1 && m < M;
-        f2[j] = in ? __ldg(rs2 + m) : 0.0f;
-        r1[j] = (Q1 && in) ? __ldg(rinv1 + m) : 0.0f;
-      }
+    // Lane j < kRowsPerWarp holds the factors of row j of this warp's rows;
+    // the next tile's are loaded while this one is worked on.
+    constexpr int RW = T::kRowsPerWarp;
+    const int rw0 = (warp / kSub) * RW;  // this warp's first row of a tile
+    const uint32_t qoff = static_cast<uint32_t>(sub * (kTileBytes / kSub));
+    auto load_rows = [&](int t, float& f2, float& r1) {
+      const int64_t m = static_cast<int64_t>(t) * T::kRows + rw0 + lane;
+      const bool in = lane < RW && t < t1 && m < M;
+      f2 = in ? __ldg(rs2 + m) : 0.0f;
+      r1 = (Q1 && in) ? __ldg(rinv1 + m) : 0.0f;
     };
+    float f2cur, r1cur;
     load_rows(t0, f2cur, r1cur);
-    ring.consume(t0, t1, lane, [&](int t, uint32_t tile) {
+    ring.consume(t0, t1, lane, [&](int t, uint32_t stage) {
+      if (!live) return;  // a quarter past the last column: nothing loaded
+      const uint32_t tile = stage + qoff;
+      float f2next, r1next;
       load_rows(t + 1, f2next, r1next);
 #pragma unroll
-      for (int j = 0; j < T::kRowsPerWarp; ++j) {
-        const int r = warp * T::kRowsPerWarp + j;
+      for (int j = 0; j < RW; ++j) {
+        const int r = rw0 + j;
         const int64_t m = static_cast<int64_t>(t) * T::kRows + r;
+        const float f2 = __shfl_sync(0xFFFFFFFFu, f2cur, j);
+        const float r1 = Q1 ? __shfl_sync(0xFFFFFFFFu, r1cur, j) : 0.0f;
         if (m < M && cv) {
           float d[8];
           smem_load8<InT>(tile + (r * kCols + lane * 8) * sizeof(InT), d);
-          const float f2 = f2cur[j];
+          // Products two at a time; the rounding add one at a time (a packed
+          // multiply whose result feeds a packed add is fused into one fma by
+          // the code generator, which would skip the product's rounding).
           uint32_t b[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], f2), iv[i]);
+          for (int i = 0; i < 8; i += 2) {
+            const float2 v = mul2(mul2(make_float2(d[i], d[i + 1]), make_float2(f2, f2)),
+                                  make_float2(iv[i], iv[i + 1]));
+            b[i] = __float_as_uint(__fadd_rn(v.x, kRneMagic));
+            b[i + 1] = __float_as_uint(__fadd_rn(v.y, kRneMagic));
+          }
           *reinterpret_cast<uint2*>(q2 + m * N + col) =
               make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
           if (Q1) {
-            const float r1 = r1cur[j];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) b[i] = rne_bits_prod(__fmul_rn(d[i], w8[i]), r1);
+            for (int i = 0; i < 8; i += 2) {
+              const float2 v = mul2(mul2(make_float2(d[i], d[i + 1]), make_float2(w8[i], w8[i + 1])),
+                                    make_float2(r1, r1));
+              b[i] = __float_as_uint(__fadd_rn(v.x, kRneMagic));
+              b[i + 1] = __float_as_uint(__fadd_rn(v.y, kRneMagic));
+            }
             *reinterpret_cast<uint2*>(q1 + m * N + col) =
                 make_uint2(pack_codes(b[0], b[1], b[2], b[3]), pack_codes(b[4], b[5], b[6], b[7]));
           }
         }
       }
-#pragma unroll
-      for (int j = 0; j < T::kRowsPerWarp; ++j) {
-        f2cur[j] = f2next[j];
-        r1cur[j] = r1next[j];
-      }
+      f2cur = f2next;
+      r1cur = r1next;
     });
   }
   __syncthreads();
@@ -332,7 +367,7 @@ struct Grid {
 
 // Column blocks x row groups, about `per_sm` resident CTAs per SM in total.
 Grid plan(int64_t M, int64_t N, int rows_per_tile, int per_sm) {
-  const int cbs = static_cast<int>((N + kCols - 1) / kCols);
+  const int cbs = static_cast<int>((N + kBlockCols - 1) / kBlockCols);
   const int tiles = static_cast<int>((M + rows_per_tile - 1) / rows_per_tile);
   int groups = device_info().sms * per_sm / cbs;  // round down: one wave of resident CTAs
   if (groups > tiles) groups = tiles;
@@ -367,7 +402,7 @@ cudaError_t colstats_t(const void* dy, int64_t M, int64_t N, const float* sx, ui
                        cudaStream_t s) {
   CUtensorMap tm;
   if (!dy_map<InT>(&tm, dy, M, N)) return cudaErrorInvalidValue;
-  const Grid g = plan(M, N, Tile<InT>::kRows, 3);
+  const Grid g = plan(M, N, Tile<InT>::kRows, 2);
   if (rowmax) {
     allow_smem<colstats_tma_kernel<InT, true>>();
     colstats_tma_kernel<InT, true><<<g.grid, kThreads, kSmemBytes, s>>>(
@@ -387,7 +422,7 @@ cudaError_t dualquant_t(const void* dy, int64_t M, int64_t N, const float* cs1,
                         int8_t* q2, int32_t* status, cudaStream_t s) {
   CUtensorMap tm;
   if (!dy_map<InT>(&tm, dy, M, N)) return cudaErrorInvalidValue;
-  const Grid g = plan(M, N, Tile<InT>::kRows, 3);
+  const Grid g = plan(M, N, Tile<InT>::kRows, 2);
   if (q1) {
     allow_smem<dualquant_tma_kernel<InT, true>>();
     dualquant_tma_kernel<InT, true><<<g.grid, kThreads, kSmemBytes, s>>>(
