@@ -26,15 +26,24 @@ namespace ql {
 
 namespace {
 
-// e^x of two values at once: packed f32x2 multiplies and fused multiply-adds,
-// each half one correctly rounded operation, so each result is that of the
-// scalar steps in the file comment; a NaN input gives NaN.
+// e^x of two values at once, the steps of the file comment with packed
+// f32x2 multiplies and fused multiply-adds (each half one correctly rounded
+// operation).  rint(y) for |y| < 2^22 is (y + 1.5*2^23) - 1.5*2^23, the
+// integer n the low bits of y + 1.5*2^23; the addition is scalar, since a
+// packed add of a packed product's result is fused into one fma by the code
+// generator, which would skip the rounding of y.  For -126 <= n <= 127,
+// 2^n is a normal float and (p * 2^(n/2)) * 2^(n - n/2) = p * 2^n with one
+// rounding either way (p * 2^(n/2) is exact), so one multiply suffices; other
+// n (x beyond about -87.3 or 88) take the two multiplies.  A NaN x gives an
+// unspecified result: the callers' outputs are NaN through x itself.
 __device__ __forceinline__ float2 exp_cw2(float2 x) {
-  const float x0 = x.x > 89.0f ? 89.0f : (x.x < -104.0f ? -104.0f : x.x);
-  const float x1 = x.y > 89.0f ? 89.0f : (x.y < -104.0f ? -104.0f : x.y);
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const float x0 = fminf(fmaxf(x.x, -104.0f), 89.0f);
+  const float x1 = fminf(fmaxf(x.y, -104.0f), 89.0f);
   const float2 y = mul2(make_float2(x0, x1), make_float2(0x1.715476p+0f, 0x1.715476p+0f));
-  const float nf0 = rintf(y.x), nf1 = rintf(y.y);
-  const float2 mn = make_float2(-nf0, -nf1);
+  const float t0 = __fadd_rn(y.x, kMagic), t1 = __fadd_rn(y.y, kMagic);
+  const float2 mn = sub2(make_float2(kMagic, kMagic), make_float2(t0, t1));  // -rint(y)
+  const int n0 = __float_as_int(t0) - 0x4B400000, n1 = __float_as_int(t1) - 0x4B400000;
   float2 r = fma2(mn, make_float2(0x1.62e43p-1f, 0x1.62e43p-1f), make_float2(x0, x1));
   r = fma2(mn, make_float2(-0x1.05c61p-29f, -0x1.05c61p-29f), r);
   float2 p = make_float2(0x1.a01a02p-13f, 0x1.a01a02p-13f);
@@ -45,14 +54,14 @@ __device__ __forceinline__ float2 exp_cw2(float2 x) {
   p = fma2(p, r, make_float2(0.5f, 0.5f));
   p = fma2(p, r, make_float2(1.0f, 1.0f));
   p = fma2(p, r, make_float2(1.0f, 1.0f));
-  const int n0 = static_cast<int>(nf0), n1 = static_cast<int>(nf1);
-  const int a0 = n0 / 2, a1 = n1 / 2;
-  const float2 f1 = make_float2(__int_as_float((a0 + 127) << 23), __int_as_float((a1 + 127) << 23));
-  const float2 f2 = make_float2(__int_as_float((n0 - a0 + 127) << 23),
-                                __int_as_float((n1 - a1 + 127) << 23));
-  float2 e = mul2(mul2(p, f1), f2);
-  if (x.x != x.x) e.x = x.x;
-  if (x.y != x.y) e.y = x.y;
+  float2 e = mul2(p, make_float2(__int_as_float((n0 + 127) << 23), __int_as_float((n1 + 127) << 23)));
+  if (static_cast<unsigned>(n0 + 126) > 253u || static_cast<unsigned>(n1 + 126) > 253u) {
+    const int a0 = n0 / 2, a1 = n1 / 2;
+    const float2 f1 = make_float2(__int_as_float((a0 + 127) << 23), __int_as_float((a1 + 127) << 23));
+    const float2 f2 = make_float2(__int_as_float((n0 - a0 + 127) << 23),
+                                  __int_as_float((n1 - a1 + 127) << 23));
+    e = mul2(mul2(p, f1), f2);
+  }
   return e;
 }
 
@@ -87,8 +96,12 @@ __global__ void __launch_bounds__(kGateThreads) swiglu_quant_kernel(
 #pragma unroll
         for (int k = 0; k < 8; k += 2) {
           const float2 e = exp_cw2(make_float2(-a8[k], -a8[k + 1]));
-          h[j][k] = __fmul_rn(__fdiv_rn(a8[k], __fadd_rn(1.0f, e.x)), b8[k]);
-          h[j][k + 1] = __fmul_rn(__fdiv_rn(a8[k + 1], __fadd_rn(1.0f, e.y)), b8[k + 1]);
+          // 1 + e scalar: e may come from a packed multiply (see exp_cw2)
+          const float2 s = make_float2(__fdiv_rn(a8[k], __fadd_rn(1.0f, e.x)),
+                                       __fdiv_rn(a8[k + 1], __fadd_rn(1.0f, e.y)));
+          const float2 hv = mul2(s, make_float2(b8[k], b8[k + 1]));
+          h[j][k] = hv.x;
+          h[j][k + 1] = hv.y;
         }
       } else {
 #pragma unroll
@@ -114,7 +127,18 @@ __global__ void __launch_bounds__(kGateThreads) swiglu_quant_kernel(
 #pragma unroll
     for (int j = 0; j < P; ++j) {
       const int col = j * kGateSpan + t * kGatePiece;
-      if (col < F) *reinterpret_cast<uint2*>(hq + m * ldh + col) = codes8(h[j], inv);
+      if (col < F) {
+        // products two at a time, the rounding adds one at a time
+        uint32_t c[8];
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const float2 v = mul2(make_float2(h[j][k], h[j][k + 1]), make_float2(inv, inv));
+          c[k] = __float_as_uint(__fadd_rn(v.x, kRneMagic));
+          c[k + 1] = __float_as_uint(__fadd_rn(v.y, kRneMagic));
+        }
+        *reinterpret_cast<uint2*>(hq + m * ldh + col) =
+            make_uint2(pack_codes(c[0], c[1], c[2], c[3]), pack_codes(c[4], c[5], c[6], c[7]));
+      }
     }
     if (t == 0) {
       sh[m] = mb == 0 ? 0.0f : amax / 127.0f;
