@@ -27,6 +27,18 @@ extern "C" {
  * NULL status, QL_ERR_CUDA if the launch fails. */
 QL_API int ql_test_wait_timeout(int32_t *d_status, uint32_t limit_us, void *stream);
 
+/* The float32 reciprocal and quotient steps the SwiGLU gate kernels use for
+ * a / (1 + e^-a) and 1 / (1 + e^-a) (Markstein's correction steps on the
+ * approximate hardware reciprocal), applied elementwise to device arrays of
+ * n values: y[i] = 1/d[i] and q[i] = a[i]/d[i], each meant to equal the
+ * correctly rounded (IEEE round-to-nearest-even) result.  Operands outside
+ * the steps' range (d < 1, d > 2^24, |a| < 2^-90 or > 2^100, zero, inf,
+ * NaN) take the IEEE division, as in the kernels; y[i] is then 1/d[i] by
+ * IEEE division too.  Asynchronous on `stream`; QL_ERR_ARG for n < 0 or a
+ * NULL pointer with n > 0, QL_ERR_CUDA if the launch fails. */
+QL_API int ql_test_divrn(const float *a, const float *d, int64_t n, float *q, float *y,
+                         void *stream);
+
 #ifdef __cplusplus
 }
 #endif

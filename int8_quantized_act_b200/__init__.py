@@ -29,7 +29,7 @@ __all__ = [
     "qlinear_fwd_bf16_workspace_bytes", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
     "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
     "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES", "qlinear_bwd",
-    "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout", "qlinear_fwd_quantized",
+    "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout", "ql_test_divrn", "qlinear_fwd_quantized",
     "qlinear_swiglu_quantize", "qlinear_swiglu_bwd", "qweight_muon_workspace_bytes",
     "qweight_muon_orthogonalize", "qweight_update_muon_sr", "qvector_adamw",
 ]
@@ -117,6 +117,8 @@ def lib() -> ctypes.CDLL:
     L.qlinear_bwd_dw.argtypes = [P, I, I64, I64, P, P, I64, P, P, P, ctypes.c_size_t, P, P]
     L.ql_test_wait_timeout.restype = I
     L.ql_test_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
+    L.ql_test_divrn.restype = I
+    L.ql_test_divrn.argtypes = [P, P, I64, P, P, P]
     L.qlinear_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.qlinear_bwd_workspace_bytes.argtypes = [I64, I64, I64, I]
     L.qlinear_bwd.restype = I
@@ -572,3 +574,15 @@ def ql_test_wait_timeout(status, limit_us: int, stream=None):
     limit_us and sets the QL_ERR_TIMEOUT bit in `status`."""
     _check(lib().ql_test_wait_timeout(_dev(status, "status", torch.int32), int(limit_us),
                                       _stream(stream)), "ql_test_wait_timeout")
+
+
+def ql_test_divrn(a, d, q, y, stream=None):
+    """The SwiGLU gate's float32 division steps (include/qlinear_testing.h)
+    on float32 device vectors: q = a / d and y = 1 / d elementwise."""
+    n = a.numel()
+    for t, what in ((d, "d"), (q, "q"), (y, "y")):
+        if t.numel() != n:
+            raise ValueError(f"ql_test_divrn: {what} has {t.numel()} values, a has {n}")
+    _check(lib().ql_test_divrn(_dev(a, "a", torch.float32), _dev(d, "d", torch.float32), n,
+                               _dev(q, "q", torch.float32), _dev(y, "y", torch.float32),
+                               _stream(stream)), "ql_test_divrn")

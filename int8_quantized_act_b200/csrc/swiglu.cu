@@ -18,6 +18,7 @@
 // product of two exact powers of two.  x is clamped to [-104, 89] first.
 #include <algorithm>
 
+#include "divrn.cuh"
 #include "launch.h"
 #include "rowops.cuh"
 #include "../../include/qlinear.h"
@@ -65,17 +66,19 @@ __device__ __forceinline__ float2 exp_cw2(float2 x) {
   return e;
 }
 
-constexpr int kGateThreads = 256;
+constexpr int kGateThreads = 448;
 constexpr int kGatePiece = 8;                          // columns per thread per piece
-constexpr int kGateSpan = kGateThreads * kGatePiece;   // 2048 columns per piece
+constexpr int kGateSpan = kGateThreads * kGatePiece;   // 3584 columns per piece
 
 // One CTA per row of [a | b] (persistent over rows): thread t owns columns
-// j * 2048 + 8t .. +7 of h for pieces j < P, read with 16-byte loads (a warp
+// j * 3584 + 8t .. +7 of h for pieces j < P, read with 16-byte loads (a warp
 // reads 512 contiguous bytes of a and of b per piece); the row maximum of |h|
 // is a NaN-propagating max, reduced over the warps through shared memory;
-// the codes are stored 8 at a time.
+// the codes are stored 8 at a time.  448 threads (14 warps), two CTAs per SM:
+// d_ff = 14336 is exactly four pieces, and the 8 * P values of h a thread
+// holds across its row fit the register budget of two CTAs per SM.
 template <typename InT, int P>
-__global__ void __launch_bounds__(kGateThreads) swiglu_quant_kernel(
+__global__ void __launch_bounds__(kGateThreads, 2) swiglu_quant_kernel(
     const InT* __restrict__ ab, int64_t M, int F, int64_t ldab, int8_t* __restrict__ hq,
     int64_t ldh, float* __restrict__ sh, int32_t* __restrict__ status) {
   __shared__ uint32_t s_wmax[2][kGateThreads / 32];
@@ -93,13 +96,30 @@ __global__ void __launch_bounds__(kGateThreads) swiglu_quant_kernel(
         float a8[8], b8[8];
         load8(ra + col, a8);
         load8(rb + col, b8);
+        // silu = a / (1 + e^-a), 1 + e scalar (e may come from a packed
+        // multiply, see exp_cw2); the division by the correction steps of
+        // divrn.cuh, the IEEE division for operands outside their range.
+        float d8[8], s8[8];
+        bool ok = true;
 #pragma unroll
         for (int k = 0; k < 8; k += 2) {
           const float2 e = exp_cw2(make_float2(-a8[k], -a8[k + 1]));
-          // 1 + e scalar: e may come from a packed multiply (see exp_cw2)
-          const float2 s = make_float2(__fdiv_rn(a8[k], __fadd_rn(1.0f, e.x)),
-                                       __fdiv_rn(a8[k + 1], __fadd_rn(1.0f, e.y)));
-          const float2 hv = mul2(s, make_float2(b8[k], b8[k + 1]));
+          d8[k] = __fadd_rn(1.0f, e.x);
+          d8[k + 1] = __fadd_rn(1.0f, e.y);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          ok = ok && div_rn_ok(a8[k], d8[k]);
+          s8[k] = div_rn(a8[k], d8[k], recip_rn(d8[k]));
+        }
+        if (!ok) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (!div_rn_ok(a8[k], d8[k])) s8[k] = __fdiv_rn(a8[k], d8[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const float2 hv = mul2(make_float2(s8[k], s8[k + 1]), make_float2(b8[k], b8[k + 1]));
           h[j][k] = hv.x;
           h[j][k + 1] = hv.y;
         }
@@ -172,15 +192,28 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const InT* __restrict__
       ek[k] = e.x;
       ek[k + 1] = e.y;
     }
+    float d8[8], sg8[8], sl8[8];
+    bool ok = true;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float a = a8[k];
-      const float d = __fadd_rn(1.0f, ek[k]);
-      const float sigma = __fdiv_rn(1.0f, d);
-      const float silu = __fdiv_rn(a, d);
+      d8[k] = __fadd_rn(1.0f, ek[k]);
+      ok = ok && div_rn_ok(a8[k], d8[k]);
+      sg8[k] = recip_rn(d8[k]);                 // sigma = 1/d
+      sl8[k] = div_rn(a8[k], d8[k], sg8[k]);    // silu = a/d
+    }
+    if (!ok) {  // operands outside the correction steps' range: IEEE division
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (!(d8[k] >= 1.0f && d8[k] <= 16777216.0f)) sg8[k] = __fdiv_rn(1.0f, d8[k]);
+        if (!div_rn_ok(a8[k], d8[k])) sl8[k] = __fdiv_rn(a8[k], d8[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float a = a8[k], sigma = sg8[k];
       const float ds = __fmul_rn(sigma, __fadd_rn(1.0f, __fmul_rn(a, __fsub_rn(1.0f, sigma))));
       da[k] = __fmul_rn(__fmul_rn(g8[k], b8[k]), ds);
-      db[k] = __fmul_rn(g8[k], silu);
+      db[k] = __fmul_rn(g8[k], sl8[k]);
     }
     store8(dab + m * 2 * static_cast<int64_t>(F) + col, da);
     store8(dab + m * 2 * static_cast<int64_t>(F) + F + col, db);

@@ -210,6 +210,14 @@ def test_timeout_hook_validation(L):
     assert L.ql_test_wait_timeout(fake(0x10000), 10000001, None) == ql.QL_ERR_ARG
 
 
+def test_divrn_hook_validation(L):
+    A = 0x10000
+    assert L.ql_test_divrn(fake(A), fake(A), -1, fake(A), fake(A), None) == ql.QL_ERR_ARG
+    assert L.ql_test_divrn(None, fake(A), 4, fake(A), fake(A), None) == ql.QL_ERR_ARG
+    assert L.ql_test_divrn(fake(A), fake(A), 4, fake(A), None, None) == ql.QL_ERR_ARG
+    assert L.ql_test_divrn(None, None, 0, None, None, None) == ql.QL_OK
+
+
 def test_dequantize_validation(L):
     A = 0x10000
     f = L.qlinear_dequantize
