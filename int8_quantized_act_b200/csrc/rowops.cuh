@@ -302,6 +302,19 @@ __device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
   return d;
 }
 
+// The NaN-propagating minima (min.NaN.f32, two and three operands).
+__device__ __forceinline__ float fmin_nan(float a, float b) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+__device__ __forceinline__ float fmin3_nan(float a, float b, float c) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // -------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll

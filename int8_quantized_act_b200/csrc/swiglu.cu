@@ -16,6 +16,10 @@
 // remainder, each a correctly rounded fused multiply-add; e^r by the Taylor
 // series to degree 7 in Horner form (fused multiply-adds); times 2^n as the
 // product of two exact powers of two.  x is clamped to [-104, 89] first.
+// Groups of eight values whose a lie in [-16, 2^100] (|a| >= 2^-90) take a
+// faster form with the same results (exp_fast2, and the correctly rounded
+// division of divrn.cuh); others take these steps as written and the IEEE
+// division.
 #include <algorithm>
 
 #include "divrn.cuh"
@@ -27,43 +31,108 @@ namespace ql {
 
 namespace {
 
-// e^x of two values at once, the steps of the file comment with packed
-// f32x2 multiplies and fused multiply-adds (each half one correctly rounded
-// operation).  rint(y) for |y| < 2^22 is (y + 1.5*2^23) - 1.5*2^23, the
-// integer n the low bits of y + 1.5*2^23; the addition is scalar, since a
-// packed add of a packed product's result is fused into one fma by the code
-// generator, which would skip the rounding of y.  For -126 <= n <= 127,
-// 2^n is a normal float and (p * 2^(n/2)) * 2^(n - n/2) = p * 2^n with one
-// rounding either way (p * 2^(n/2) is exact), so one multiply suffices; other
-// n (x beyond about -87.3 or 88) take the two multiplies.  A NaN x gives an
-// unspecified result: the callers' outputs are NaN through x itself.
-__device__ __forceinline__ float2 exp_cw2(float2 x) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const float x0 = fminf(fmaxf(x.x, -104.0f), 89.0f);
-  const float x1 = fminf(fmaxf(x.y, -104.0f), 89.0f);
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: x + kMagic rounds x to an integer
+
+// e^x by the steps of the file comment, for every x (a NaN gives NaN).
+// rint(y) for |y| < 2^22 is (y + 1.5*2^23) - 1.5*2^23, the integer n in the
+// low bits of y + 1.5*2^23.
+__device__ __forceinline__ float exp_ref(float x) {
+  if (x != x) return x;
+  const float xc = fminf(fmaxf(x, -104.0f), 89.0f);
+  const float t = __fadd_rn(__fmul_rn(xc, 0x1.715476p+0f), kMagic);
+  const float mn = __fsub_rn(kMagic, t);  // -rint(y)
+  const int n = __float_as_int(t) - 0x4B400000;
+  float r = __fmaf_rn(mn, 0x1.62e43p-1f, xc);
+  r = __fmaf_rn(mn, -0x1.05c61p-29f, r);
+  float p = 0x1.a01a02p-13f;
+  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
+  p = __fmaf_rn(p, r, 0x1.111112p-7f);
+  p = __fmaf_rn(p, r, 0x1.555556p-5f);
+  p = __fmaf_rn(p, r, 0x1.555556p-3f);
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const int a = n / 2;
+  return __fmul_rn(__fmul_rn(p, __int_as_float((a + 127) << 23)), __int_as_float((n - a + 127) << 23));
+}
+
+// e^x of two values at once for x <= 16, with packed f32x2 multiplies and
+// fused multiply-adds (each half one correctly rounded operation): the same
+// result as exp_ref for -86.5 <= x <= 16, and for x < -86.5 the value at
+// -86.5 (below 2^-125, so 1 + e^x is exactly 1 for both, the only use made
+// of it).  Then n lies in [-125, 23]: the Horner steps run on 2p (every
+// coefficient doubled: each step scales exactly), and 2p * 2^(n-1), one
+// multiply by a normal power of two, is p * 2^n with the one rounding of the
+// two exact-then-rounded multiplies of exp_ref.  The rounding addition is
+// scalar: a packed add of a packed product's result is fused into one fma by
+// the code generator, which would skip the rounding of y.
+__device__ __forceinline__ float2 exp_fast2(float2 x) {
+  const float x0 = fmaxf(x.x, -86.5f), x1 = fmaxf(x.y, -86.5f);
   const float2 y = mul2(make_float2(x0, x1), make_float2(0x1.715476p+0f, 0x1.715476p+0f));
   const float t0 = __fadd_rn(y.x, kMagic), t1 = __fadd_rn(y.y, kMagic);
   const float2 mn = sub2(make_float2(kMagic, kMagic), make_float2(t0, t1));  // -rint(y)
-  const int n0 = __float_as_int(t0) - 0x4B400000, n1 = __float_as_int(t1) - 0x4B400000;
   float2 r = fma2(mn, make_float2(0x1.62e43p-1f, 0x1.62e43p-1f), make_float2(x0, x1));
   r = fma2(mn, make_float2(-0x1.05c61p-29f, -0x1.05c61p-29f), r);
-  float2 p = make_float2(0x1.a01a02p-13f, 0x1.a01a02p-13f);
-  p = fma2(p, r, make_float2(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
-  p = fma2(p, r, make_float2(0x1.111112p-7f, 0x1.111112p-7f));
-  p = fma2(p, r, make_float2(0x1.555556p-5f, 0x1.555556p-5f));
-  p = fma2(p, r, make_float2(0x1.555556p-3f, 0x1.555556p-3f));
-  p = fma2(p, r, make_float2(0.5f, 0.5f));
+  float2 p = make_float2(0x1.a01a02p-12f, 0x1.a01a02p-12f);
+  p = fma2(p, r, make_float2(0x1.6c16c2p-9f, 0x1.6c16c2p-9f));
+  p = fma2(p, r, make_float2(0x1.111112p-6f, 0x1.111112p-6f));
+  p = fma2(p, r, make_float2(0x1.555556p-4f, 0x1.555556p-4f));
+  p = fma2(p, r, make_float2(0x1.555556p-2f, 0x1.555556p-2f));
   p = fma2(p, r, make_float2(1.0f, 1.0f));
-  p = fma2(p, r, make_float2(1.0f, 1.0f));
-  float2 e = mul2(p, make_float2(__int_as_float((n0 + 127) << 23), __int_as_float((n1 + 127) << 23)));
-  if (static_cast<unsigned>(n0 + 126) > 253u || static_cast<unsigned>(n1 + 126) > 253u) {
-    const int a0 = n0 / 2, a1 = n1 / 2;
-    const float2 f1 = make_float2(__int_as_float((a0 + 127) << 23), __int_as_float((a1 + 127) << 23));
-    const float2 f2 = make_float2(__int_as_float((n0 - a0 + 127) << 23),
-                                  __int_as_float((n1 - a1 + 127) << 23));
-    e = mul2(mul2(p, f1), f2);
+  p = fma2(p, r, make_float2(2.0f, 2.0f));
+  p = fma2(p, r, make_float2(2.0f, 2.0f));
+  // 2^(n-1) = bits (n + 126) << 23, n = bits(t) - bits(1.5 * 2^23)
+  const float s0 = __int_as_float((__float_as_int(t0) - (0x4B400000 - 126)) << 23);
+  const float s1 = __int_as_float((__float_as_int(t1) - (0x4B400000 - 126)) << 23);
+  return mul2(p, make_float2(s0, s1));
+}
+
+// Whether eight gate values take the fast steps: every a in [-16, 2^100]
+// with |a| >= 2^-90 (no zero, NaN or infinity).  Then x = -a <= 16, so
+// d = 1 + e^-a lies in [1, 2^24], and a / d is a normal float: the range of
+// exp_fast2 and of the division's correction steps (divrn.cuh).
+__device__ __forceinline__ bool fast_ok8(const float (&a)[8]) {
+  float lo = fmin3_nan(a[0], a[1], a[2]), hi = fmax3_nan(a[0], a[1], a[2]);
+  float mg = fmin3_nan(fabsf(a[0]), fabsf(a[1]), fabsf(a[2]));
+  lo = fmin3_nan(lo, a[3], a[4]);
+  hi = fmax3_nan(hi, a[3], a[4]);
+  mg = fmin3_nan(mg, fabsf(a[3]), fabsf(a[4]));
+  lo = fmin3_nan(lo, a[5], a[6]);
+  hi = fmax3_nan(hi, a[5], a[6]);
+  mg = fmin3_nan(mg, fabsf(a[5]), fabsf(a[6]));
+  lo = fmin_nan(lo, a[7]);
+  hi = fmax_nan(hi, a[7]);
+  mg = fmin_nan(mg, fabsf(a[7]));
+  return lo >= -16.0f && hi <= 0x1p+100f && mg >= 0x1p-90f;
+}
+
+// d = 1 + e^-a and (with Q) q = a / d for eight values: the fast steps when
+// fast_ok8 holds, else exp_ref and the IEEE division.  1 + e is a scalar
+// addition (e comes from a packed multiply, see exp_fast2).  With R also
+// y = 1/d.
+template <bool R>
+__device__ __forceinline__ void silu_parts8(const float (&a)[8], float (&q)[8], float (&y)[8]) {
+  if (fast_ok8(a)) {
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      const float2 e = exp_fast2(make_float2(-a[k], -a[k + 1]));
+      const float d0 = __fadd_rn(1.0f, e.x), d1 = __fadd_rn(1.0f, e.y);
+      const float y0 = recip_rn(d0), y1 = recip_rn(d1);
+      q[k] = div_rn(a[k], d0, y0);
+      q[k + 1] = div_rn(a[k + 1], d1, y1);
+      if (R) {
+        y[k] = y0;
+        y[k + 1] = y1;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float d = __fadd_rn(1.0f, exp_ref(-a[k]));
+      q[k] = __fdiv_rn(a[k], d);
+      if (R) y[k] = __fdiv_rn(1.0f, d);
+    }
   }
-  return e;
 }
 
 constexpr int kGateThreads = 448;
@@ -96,27 +165,8 @@ __global__ void __launch_bounds__(kGateThreads, 2) swiglu_quant_kernel(
         float a8[8], b8[8];
         load8(ra + col, a8);
         load8(rb + col, b8);
-        // silu = a / (1 + e^-a), 1 + e scalar (e may come from a packed
-        // multiply, see exp_cw2); the division by the correction steps of
-        // divrn.cuh, the IEEE division for operands outside their range.
-        float d8[8], s8[8];
-        bool ok = true;
-#pragma unroll
-        for (int k = 0; k < 8; k += 2) {
-          const float2 e = exp_cw2(make_float2(-a8[k], -a8[k + 1]));
-          d8[k] = __fadd_rn(1.0f, e.x);
-          d8[k + 1] = __fadd_rn(1.0f, e.y);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          ok = ok && div_rn_ok(a8[k], d8[k]);
-          s8[k] = div_rn(a8[k], d8[k], recip_rn(d8[k]));
-        }
-        if (!ok) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            if (!div_rn_ok(a8[k], d8[k])) s8[k] = __fdiv_rn(a8[k], d8[k]);
-        }
+        float s8[8], unused[8];
+        silu_parts8<false>(a8, s8, unused);
 #pragma unroll
         for (int k = 0; k < 8; k += 2) {
           const float2 hv = mul2(make_float2(s8[k], s8[k + 1]), make_float2(b8[k], b8[k + 1]));
@@ -185,35 +235,23 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const InT* __restrict__
     load8(ab + m * ldab + col, a8);
     load8(ab + m * ldab + F + col, b8);
     load8(dh + m * F + col, g8);
-    float ek[8];
+    float sg8[8], sl8[8];
+    silu_parts8<true>(a8, sl8, sg8);  // silu = a/d, sigma = 1/d
+    // ds = sigma * (1 + a * (1 - sigma)) scalar (its adds follow products);
+    // the products with dh two at a time.
+    float ds[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      ds[k] = __fmul_rn(sg8[k], __fadd_rn(1.0f, __fmul_rn(a8[k], __fsub_rn(1.0f, sg8[k]))));
 #pragma unroll
     for (int k = 0; k < 8; k += 2) {
-      const float2 e = exp_cw2(make_float2(-a8[k], -a8[k + 1]));
-      ek[k] = e.x;
-      ek[k + 1] = e.y;
-    }
-    float d8[8], sg8[8], sl8[8];
-    bool ok = true;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      d8[k] = __fadd_rn(1.0f, ek[k]);
-      ok = ok && div_rn_ok(a8[k], d8[k]);
-      sg8[k] = recip_rn(d8[k]);                 // sigma = 1/d
-      sl8[k] = div_rn(a8[k], d8[k], sg8[k]);    // silu = a/d
-    }
-    if (!ok) {  // operands outside the correction steps' range: IEEE division
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (!(d8[k] >= 1.0f && d8[k] <= 16777216.0f)) sg8[k] = __fdiv_rn(1.0f, d8[k]);
-        if (!div_rn_ok(a8[k], d8[k])) sl8[k] = __fdiv_rn(a8[k], d8[k]);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float a = a8[k], sigma = sg8[k];
-      const float ds = __fmul_rn(sigma, __fadd_rn(1.0f, __fmul_rn(a, __fsub_rn(1.0f, sigma))));
-      da[k] = __fmul_rn(__fmul_rn(g8[k], b8[k]), ds);
-      db[k] = __fmul_rn(g8[k], sl8[k]);
+      const float2 g = make_float2(g8[k], g8[k + 1]);
+      const float2 v = mul2(mul2(g, make_float2(b8[k], b8[k + 1])), make_float2(ds[k], ds[k + 1]));
+      const float2 w = mul2(g, make_float2(sl8[k], sl8[k + 1]));
+      da[k] = v.x;
+      da[k + 1] = v.y;
+      db[k] = w.x;
+      db[k + 1] = w.y;
     }
     store8(dab + m * 2 * static_cast<int64_t>(F) + col, da);
     store8(dab + m * 2 * static_cast<int64_t>(F) + F + col, db);
