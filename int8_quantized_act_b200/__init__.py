@@ -29,7 +29,7 @@ __all__ = [
     "qlinear_fwd_bf16_workspace_bytes", "qlinear_fwd", "qlinear_bwd_dx", "qlinear_bwd_dw",
     "qweight_update_sr", "status_flags", "ql_set_gemm_timing_events", "ql_kernel_launches",
     "qlinear_bwd_dx_noalloc", "QL_NOALLOC_SCRATCH_BYTES", "qlinear_bwd",
-    "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout", "ql_test_divrn", "qlinear_fwd_quantized",
+    "qlinear_bwd_workspace_bytes", "ql_test_wait_timeout", "ql_test_divrn", "ql_test_sqrtrn", "qlinear_fwd_quantized",
     "qlinear_swiglu_quantize", "qlinear_swiglu_bwd", "qweight_muon_workspace_bytes",
     "qweight_muon_orthogonalize", "qweight_update_muon_sr", "qvector_adamw",
 ]
@@ -119,6 +119,8 @@ def lib() -> ctypes.CDLL:
     L.ql_test_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
     L.ql_test_divrn.restype = I
     L.ql_test_divrn.argtypes = [P, P, I64, P, P, P]
+    L.ql_test_sqrtrn.restype = I
+    L.ql_test_sqrtrn.argtypes = [P, I64, P, P, P]
     L.qlinear_bwd_workspace_bytes.restype = ctypes.c_size_t
     L.qlinear_bwd_workspace_bytes.argtypes = [I64, I64, I64, I]
     L.qlinear_bwd.restype = I
@@ -586,3 +588,17 @@ def ql_test_divrn(a, d, q, y, stream=None):
     _check(lib().ql_test_divrn(_dev(a, "a", torch.float32), _dev(d, "d", torch.float32), n,
                                _dev(q, "q", torch.float32), _dev(y, "y", torch.float32),
                                _stream(stream)), "ql_test_divrn")
+
+
+def ql_test_sqrtrn(v, s_plain, s_refined, stream=None):
+    """The optimizer updates' float32 square-root steps
+    (include/qlinear_testing.h) on a float32 device vector: the plain and the
+    refined form of sqrt(v), elementwise."""
+    n = v.numel()
+    for t, what in ((s_plain, "s_plain"), (s_refined, "s_refined")):
+        if t.numel() != n:
+            raise ValueError(f"ql_test_sqrtrn: {what} has {t.numel()} values, v has {n}")
+    _check(lib().ql_test_sqrtrn(_dev(v, "v", torch.float32), n,
+                                _dev(s_plain, "s_plain", torch.float32),
+                                _dev(s_refined, "s_refined", torch.float32), _stream(stream)),
+           "ql_test_sqrtrn")

@@ -180,6 +180,13 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
 struct UpdateConsts {
   int kind = 0;  // 0 SGD, 1 AdamW
   float lr = 0, a = 1, st = 0, rbc2 = 1, b1 = 0, b2 = 0, omb1 = 0, omb2 = 0, eps = 0;
+  // AdamW constants that keep sqrt(v)*rbc2 + eps inside [2^-60, 2^60] for
+  // every v in [2^-100, 2^100]: the range of the fast square-root and
+  // division steps (set by finish()).
+  int fast = 0;
+  void finish() {
+    fast = eps >= 0x1p-60f && eps <= 1.0f && rbc2 >= 1.0f && rbc2 <= 512.0f;
+  }
 };
 
 cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64_t K,

@@ -591,6 +591,7 @@ int qvector_adamw(float* p, const float* g, float* m, float* v, int64_t n, const
   c.omb1 = static_cast<float>(1.0 - static_cast<double>(opt->beta1));
   c.omb2 = static_cast<float>(1.0 - static_cast<double>(opt->beta2));
   c.eps = opt->eps;
+  c.finish();
   return cuda_status(ql::launch_adamw_vector(p, g, m, v, n, c, d_status, as_stream(stream)));
 }
 
@@ -626,6 +627,7 @@ int qweight_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N, int64
     c.omb1 = static_cast<float>(1.0 - static_cast<double>(opt->beta1));
     c.omb2 = static_cast<float>(1.0 - static_cast<double>(opt->beta2));
     c.eps = opt->eps;
+    c.finish();
   }
   return cuda_status(ql::launch_update_sr(wq, sw, grad, N, K, c, m, v, seed, step,
                                           wn ? wn->g : nullptr, wn ? wn->g_m : nullptr,

@@ -20,6 +20,7 @@
 
 #include <algorithm>
 
+#include "divrn.cuh"
 #include "launch.h"
 #include "rowops.cuh"
 #include "sm100.cuh"
@@ -38,6 +39,42 @@ __device__ __forceinline__ float adamw(const UpdateConsts& c, float w, float g, 
   m = mn;
   v = vn;
   return w1 - c.st * (mn / den);
+}
+
+// The same step on four elements.  The square root and the division are the
+// correctly rounded steps of divrn.cuh when the constants allow it (c.fast)
+// and every v' lies in [2^-100, 2^100] and every m' in +-[2^-66, 2^60]: then
+// den = sqrt(v')*rbc2 + eps lies in [2^-60, 2^60] and m'/den is a normal
+// float.  Otherwise the IEEE operations; the results are the same bits.
+__device__ __forceinline__ void adamw4(const UpdateConsts& c, const float (&w)[4],
+                                      const float (&g)[4], float (&m)[4], float (&v)[4],
+                                      float (&out)[4]) {
+  float mn[4], vn[4], q[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    mn[e] = c.b1 * m[e] + c.omb1 * g[e];
+    vn[e] = c.b2 * v[e] + c.omb2 * (g[e] * g[e]);
+  }
+  const float vlo = fmin_nan(fmin3_nan(vn[0], vn[1], vn[2]), vn[3]);
+  const float vhi = fmax_nan(fmax3_nan(vn[0], vn[1], vn[2]), vn[3]);
+  const float mlo = fmin_nan(fmin3_nan(fabsf(mn[0]), fabsf(mn[1]), fabsf(mn[2])), fabsf(mn[3]));
+  const float mhi = fmax_nan(fmax3_nan(fabsf(mn[0]), fabsf(mn[1]), fabsf(mn[2])), fabsf(mn[3]));
+  if (c.fast && vlo >= 0x1p-100f && vhi <= 0x1p+100f && mlo >= 0x1p-66f && mhi <= 0x1p+60f) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float den = sqrt_rn_t<false>(vn[e]) * c.rbc2 + c.eps;
+      q[e] = div_rn(mn[e], den, recip_rn(den));
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[e] = mn[e] / (sqrtf(vn[e]) * c.rbc2 + c.eps);
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    out[e] = w[e] * c.a - c.st * q[e];
+    m[e] = mn[e];
+    v[e] = vn[e];
+  }
 }
 
 // floor(v) + 1 with probability frac(v), decided by u24 < frac * 2^24;
@@ -146,8 +183,10 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
         const float4 v4 = v_s[ch];
         float m1[4] = {m4.x, m4.y, m4.z, m4.w};
         float m2[4] = {v4.x, v4.y, v4.z, v4.w};
+        float wv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = adamw(c, s * code_byte_f(q4, e), gr[e], m1[e], m2[e]);
+        for (int e = 0; e < 4; ++e) wv[e] = s * code_byte_f(q4, e);
+        adamw4(c, wv, gr, m1, m2, w);
         __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
         __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
       } else {
@@ -321,31 +360,56 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
   float4* v_out = reinterpret_cast<float4*>(mom2 + row);
   float amax = 0.0f;
   int bad = 0;
-  for (int ch = t; ch < nch; ch += T) {
-    const uint32_t q4 = q_s[ch];
-    const float4 g4 = g_s[ch];
-    const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
-    float m1[4], m2[4];
+  // Four chunks per pass, their moment loads issued together.
+  constexpr int U = 4;
+  for (int ch0 = t; ch0 < nch; ch0 += U * T) {
+    float4 ma[U], va[U];
     if (adam) {
-      const float4 a = __ldcs(m_out + ch), b = __ldcs(v_out + ch);
-      m1[0] = a.x; m1[1] = a.y; m1[2] = a.z; m1[3] = a.w;
-      m2[0] = b.x; m2[1] = b.y; m2[2] = b.z; m2[3] = b.w;
-    }
-    float w[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float qhat = s_qhat[static_cast<int>(static_cast<int8_t>(q4 >> (8 * e))) + 128];
-      const float gg = coef * (gr[e] - dg * qhat);
-      const float wv = s * code_byte_f(q4, e);
-      w[e] = adam ? adamw(c, wv, gg, m1[e], m2[e]) : wv - c.lr * gg;
-      bad |= !finite(w[e]);
-      amax = fmaxf(amax, fabsf(w[e]));
+      for (int u = 0; u < U; ++u) {
+        const int ch = ch0 + u * T;
+        if (ch < nch) {
+          ma[u] = __ldcs(m_out + ch);
+          va[u] = __ldcs(v_out + ch);
+        }
+      }
     }
-    if (adam) {
-      __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
-      __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int ch = ch0 + u * T;
+      if (ch >= nch) break;
+      const uint32_t q4 = q_s[ch];
+      const float4 g4 = g_s[ch];
+      const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
+      float m1[4], m2[4];
+      if (adam) {
+        m1[0] = ma[u].x; m1[1] = ma[u].y; m1[2] = ma[u].z; m1[3] = ma[u].w;
+        m2[0] = va[u].x; m2[1] = va[u].y; m2[2] = va[u].z; m2[3] = va[u].w;
+      }
+      float w[4], gg[4], wv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float qhat = s_qhat[static_cast<int>(static_cast<int8_t>(q4 >> (8 * e))) + 128];
+        gg[e] = coef * (gr[e] - dg * qhat);
+        wv[e] = s * code_byte_f(q4, e);
+      }
+      if (adam) {
+        adamw4(c, wv, gg, m1, m2, w);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = wv[e] - c.lr * gg[e];
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bad |= !finite(w[e]);
+        amax = fmaxf(amax, fabsf(w[e]));
+      }
+      if (adam) {
+        __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
+        __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
+      }
+      g_s[ch] = make_float4(w[0], w[1], w[2], w[3]);
     }
-    g_s[ch] = make_float4(w[0], w[1], w[2], w[3]);
   }
   if (t == 0) {
     float gm = gmag_n;
@@ -522,8 +586,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
           const float4 v4 = v_s[ch];
           float m1[4] = {m4.x, m4.y, m4.z, m4.w};
           float m2[4] = {v4.x, v4.y, v4.z, v4.w};
+          float wv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) w[e] = adamw(c, s * code_byte_f(q4, e), gr[e], m1[e], m2[e]);
+          for (int e = 0; e < 4; ++e) wv[e] = s * code_byte_f(q4, e);
+          adamw4(c, wv, gr, m1, m2, w);
           __stcs(m_out + c0 + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
           __stcs(v_out + c0 + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
         } else {

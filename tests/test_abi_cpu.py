@@ -216,6 +216,9 @@ def test_divrn_hook_validation(L):
     assert L.ql_test_divrn(None, fake(A), 4, fake(A), fake(A), None) == ql.QL_ERR_ARG
     assert L.ql_test_divrn(fake(A), fake(A), 4, fake(A), None, None) == ql.QL_ERR_ARG
     assert L.ql_test_divrn(None, None, 0, None, None, None) == ql.QL_OK
+    assert L.ql_test_sqrtrn(fake(A), -1, fake(A), fake(A), None) == ql.QL_ERR_ARG
+    assert L.ql_test_sqrtrn(fake(A), 4, None, fake(A), None) == ql.QL_ERR_ARG
+    assert L.ql_test_sqrtrn(None, 0, None, None, None) == ql.QL_OK
 
 
 def test_dequantize_validation(L):

@@ -146,50 +146,3 @@ def test_gate_validation():
     assert e.value.code == ql.QL_ERR_UNSUPPORTED
     assert status_word(st) == 0
 
-
-def _divrn(a, d):
-    ta, td = dev(a), dev(d)
-    q, y = torch.empty_like(ta), torch.empty_like(ta)
-    ql.ql_test_divrn(ta, td, q, y)
-    return host(q), host(y)
-
-
-def _bits_equal(x, ref):
-    """Bit for bit, every NaN counting as equal to every NaN."""
-    xb, rb = x.view(np.uint32), ref.view(np.uint32)
-    both_nan = np.isnan(x) & np.isnan(ref)
-    return np.array_equal(np.where(both_nan, 0, xb), np.where(both_nan, 0, rb))
-
-
-@pytest.mark.parametrize("exponent", [0, 1, 7, 12, 23])
-def test_reciprocal_steps_every_significand(exponent):
-    """y = 1/d by the gate's correction steps equals the IEEE quotient for
-    every float32 significand of d = 2^exponent * [1, 2)."""
-    sig = np.arange(1 << 23, dtype=np.uint32)
-    d = ((np.uint32(127 + exponent) << np.uint32(23)) | sig).view(np.float32)
-    a = np.ones_like(d)
-    q, y = _divrn(a, d)
-    ref = np.float32(1.0) / d
-    assert _bits_equal(y, ref) and _bits_equal(q, ref)
-
-
-def test_quotient_steps_random_and_edge_operands():
-    """q = a/d against the IEEE quotient: random a over the steps' whole
-    exponent range and d in [1, 2^24] (as 1 + e^-a is), then the edges:
-    all-ones significands, d at the range ends and past them, a = +-0,
-    subnormal, huge, infinite and NaN (the IEEE fallback)."""
-    rng = np.random.Generator(np.random.PCG64(11))
-    n = 1 << 24
-    a = (rng.uniform(1, 2, n) * np.exp2(rng.integers(-90, 101, n))).astype(np.float32)
-    a *= np.where(rng.random(n) < 0.5, -1, 1).astype(np.float32)
-    d = (1.0 + np.exp2(rng.uniform(-30, 24, n))).astype(np.float32)
-    d = np.minimum(d, np.float32(2.0 ** 24))
-    q, _ = _divrn(a, d)
-    assert _bits_equal(q, a / d)
-    ones = np.float32(np.nextafter(np.float32(2), np.float32(0)))  # 1.111...1 (binary)
-    edge_a = np.float32([1, -1, ones, -ones, 3, 0.0, -0.0, 1e-40, -1e-40, 2.0 ** -90, 2.0 ** -91,
-                         2.0 ** 100, 2.0 ** 101, 3e38, np.inf, -np.inf, np.nan, 7, 7, 7, 7, 7])
-    edge_d = np.float32([ones, ones, ones, 1, 3, 1.5, 1.5, 1.5, 1.5, 2.0 ** 24, 2.0 ** 24,
-                         1, 1, 1, 1, 1, 1, 1, 2.0 ** 24, 2.0 ** 25, 0.5, np.inf])
-    q, y = _divrn(edge_a, edge_d)
-    assert _bits_equal(q, edge_a / edge_d) and _bits_equal(y, np.float32(1) / edge_d)
