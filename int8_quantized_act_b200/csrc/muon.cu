@@ -61,30 +61,60 @@ __global__ void __launch_bounds__(256) muon_momentum_kernel(const float* __restr
   }
 }
 
-// 32 x 32 tiles through shared memory: out[c][r] = in[r][c] for a row-major
-// in [rows, cols].  `f` maps the input element (float) to the stored value.
+// One 64 x 64 tile of a row-major [rows, cols] float-valued matrix (rows,
+// cols multiples of 8) written as bf16 into out [rows, cols] (if given) and
+// transposed into out_t [cols, rows].  load(i, j, v) gives the 8 values at
+// row i, columns j..j+7.  Thread t computes rows t/8 and t/8 + 32, columns
+// 8(t%8)..+7 (16-byte stores; the thread that reads an element is the one
+// that writes it in out), then writes rows t/8 and t/8 + 32 of the
+// transposed tile, 8 values gathered from a column of the shared tile (rows
+// padded to 66 values: conflict-free), 16 bytes a store.
 template <typename F>
-__device__ __forceinline__ void transpose_tile(int64_t rows, int64_t cols, int64_t r0, int64_t c0,
-                                               F&& load, __nv_bfloat16* __restrict__ out_t,
-                                               __nv_bfloat16* __restrict__ out,
-                                               __nv_bfloat16 (*tile)[33]) {
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
+__device__ __forceinline__ void transpose64(int64_t rows, int64_t cols, int64_t r0, int64_t c0,
+                                            F&& load, __nv_bfloat16* __restrict__ out,
+                                            __nv_bfloat16* __restrict__ out_t,
+                                            __nv_bfloat16 (*tile)[66]) {
+  const int t = threadIdx.x, tr = t >> 3, tc = (t & 7) * 8;
 #pragma unroll
-  for (int k = 0; k < 32; k += 8) {
-    const int64_t r = r0 + ty + k, c = c0 + tx;
-    if (r < rows && c < cols) {
-      const __nv_bfloat16 v = __float2bfloat16_rn(load(r, c));
-      tile[ty + k][tx] = v;
-      if (out) out[r * cols + c] = v;
+  for (int h = 0; h < 2; ++h) {
+    const int lr = tr + 32 * h;
+    const int64_t i = r0 + lr, j = c0 + tc;
+    if (i < rows && j < cols) {
+      float v[8];
+      load(i, j, v);
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat16 b0 = __float2bfloat16_rn(v[2 * k]);
+        const __nv_bfloat16 b1 = __float2bfloat16_rn(v[2 * k + 1]);
+        tile[lr][tc + 2 * k] = b0;
+        tile[lr][tc + 2 * k + 1] = b1;
+        o[k] = static_cast<uint32_t>(__bfloat16_as_ushort(b0)) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(b1)) << 16);
+      }
+      if (out) *reinterpret_cast<uint4*>(out + i * cols + j) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
   __syncthreads();
 #pragma unroll
-  for (int k = 0; k < 32; k += 8) {
-    const int64_t c = c0 + ty + k, r = r0 + tx;
-    if (r < rows && c < cols) out_t[c * rows + r] = tile[tx][ty + k];
+  for (int h = 0; h < 2; ++h) {
+    const int lc = tr + 32 * h;                // row of the transposed tile
+    const int64_t ci = c0 + lc, rj = r0 + tc;  // out_t [cols, rows]
+    if (ci < cols && rj < rows) {
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        o[k] = static_cast<uint32_t>(__bfloat16_as_ushort(tile[tc + 2 * k][lc])) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(tile[tc + 2 * k + 1][lc])) << 16);
+      *reinterpret_cast<uint4*>(out_t + ci * rows + rj) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
   __syncthreads();
+}
+
+__device__ __forceinline__ void load8f(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
 // X0 = bf16(U / (||U||_F + 1e-7)) with U recomputed from G and the new M
@@ -96,48 +126,74 @@ __global__ void __launch_bounds__(256) ns_init_kernel(const float* __restrict__ 
                                                       const double* __restrict__ sumsq,
                                                       __nv_bfloat16* __restrict__ X,
                                                       __nv_bfloat16* __restrict__ Xt) {
-  __shared__ __nv_bfloat16 tile[32][33];
+  __shared__ __align__(16) __nv_bfloat16 tile[64][66];
   const float inv = static_cast<float>(1.0 / (sqrt(*sumsq) + 1e-7));
-  const int64_t tiles_c = (K + 31) / 32, tiles = ((N + 31) / 32) * tiles_c;
+  const int64_t tiles_c = (K + 63) / 64, tiles = ((N + 63) / 64) * tiles_c;
   const bool tr = N > K;
-  auto load = [&](int64_t r, int64_t c) {
-    const int64_t i = r * K + c;
-    const float u = __fadd_rn(__fmul_rn(omb, G[i]), __fmul_rn(beta, M[i]));
-    return __fmul_rn(u, inv);
+  auto load = [&](int64_t r, int64_t c, float (&v)[8]) {
+    float g[8], m[8];
+    load8f(G + r * K + c, g);
+    load8f(M + r * K + c, m);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      v[k] = __fmul_rn(__fadd_rn(__fmul_rn(omb, g[k]), __fmul_rn(beta, m[k])), inv);
   };
   for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-    const int64_t r0 = (t / tiles_c) * 32, c0 = (t % tiles_c) * 32;
+    const int64_t r0 = (t / tiles_c) * 64, c0 = (t % tiles_c) * 64;
     // U [N, K] row-major; its transpose [K, N].  X is U or U^T.
-    transpose_tile(N, K, r0, c0, load, tr ? X : Xt, tr ? Xt : X, tile);
+    transpose64(N, K, r0, c0, load, tr ? Xt : X, tr ? X : Xt, tile);
   }
 }
 
-// Bm = bf16(b * A + c * A2) elementwise (A bf16, A2 float32, both [r, r]).
+// Bm = bf16(b * A + c * A2) elementwise (A bf16, A2 float32, both [r, r]),
+// 8 elements a thread-step (16-byte loads and stores; n is a multiple of 8).
 __global__ void __launch_bounds__(256) ns_combine_kernel(const __nv_bfloat16* __restrict__ A,
                                                          const float* __restrict__ A2, int64_t n,
                                                          __nv_bfloat16* __restrict__ Bm) {
+  const int64_t n8 = n / 8;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
-    const float a = __bfloat162float(A[i]);
-    Bm[i] = __float2bfloat16_rn(__fadd_rn(__fmul_rn(kNsB, a), __fmul_rn(kNsC, A2[i])));
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const uint4 a = reinterpret_cast<const uint4*>(A)[i];
+    const float4 p0 = reinterpret_cast<const float4*>(A2)[2 * i];
+    const float4 p1 = reinterpret_cast<const float4*>(A2)[2 * i + 1];
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    const float a2[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float lo = __uint_as_float(aw[k] << 16), hi = __uint_as_float(aw[k] & 0xFFFF0000u);
+      const __nv_bfloat16 b0 = __float2bfloat16_rn(__fadd_rn(__fmul_rn(kNsB, lo), __fmul_rn(kNsC, a2[2 * k])));
+      const __nv_bfloat16 b1 = __float2bfloat16_rn(__fadd_rn(__fmul_rn(kNsB, hi), __fmul_rn(kNsC, a2[2 * k + 1])));
+      o[k] = static_cast<uint32_t>(__bfloat16_as_ushort(b0)) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(b1)) << 16);
+    }
+    reinterpret_cast<uint4*>(Bm)[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
 // X' = bf16(a * X + P) for X [r, c] into Xo (X itself, or the output) and
-// its transpose X'^T [c, r] into Xt.  Each element of X is read by the
-// thread that writes the same element of Xo.
+// its transpose X'^T [c, r] into Xt (transpose64: the thread that reads an
+// element of X writes it in Xo).
 __global__ void __launch_bounds__(256) ns_step_kernel(const __nv_bfloat16* X,
                                                       __nv_bfloat16* Xo,
                                                       const float* __restrict__ P, int64_t r,
                                                       int64_t c, __nv_bfloat16* __restrict__ Xt) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int64_t tiles_c = (c + 31) / 32, tiles = ((r + 31) / 32) * tiles_c;
-  auto load = [&](int64_t i, int64_t j) {
-    return __fadd_rn(__fmul_rn(kNsA, __bfloat162float(X[i * c + j])), P[i * c + j]);
+  __shared__ __align__(16) __nv_bfloat16 tile[64][66];
+  const int64_t tiles_c = (c + 63) / 64, tiles = ((r + 63) / 64) * tiles_c;
+  auto load = [&](int64_t i, int64_t j, float (&v)[8]) {
+    const uint4 xv = *reinterpret_cast<const uint4*>(X + i * c + j);
+    float p[8];
+    load8f(P + i * c + j, p);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __fadd_rn(__fmul_rn(kNsA, __uint_as_float(xw[k] << 16)), p[2 * k]);
+      v[2 * k + 1] = __fadd_rn(__fmul_rn(kNsA, __uint_as_float(xw[k] & 0xFFFF0000u)), p[2 * k + 1]);
+    }
   };
   for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-    const int64_t r0 = (t / tiles_c) * 32, c0 = (t % tiles_c) * 32;
-    transpose_tile(r, c, r0, c0, load, Xt, Xo, tile);
+    const int64_t r0 = (t / tiles_c) * 64, c0 = (t % tiles_c) * 64;
+    transpose64(r, c, r0, c0, load, Xo, Xt, tile);
   }
 }
 
@@ -206,7 +262,7 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
   cudaError_t e = cudaMemsetAsync(sumsq, 0, sizeof(double), s);
   if (e != cudaSuccess) return e;
   muon_momentum_kernel<<<grid_for(N * K / 4, 8), 256, 0, s>>>(grad, mom, N * K / 4, beta, omb, sumsq);
-  ns_init_kernel<<<grid_for(((N + 31) / 32) * ((K + 31) / 32) * 256, 8), 256, 0, s>>>(
+  ns_init_kernel<<<grid_for(((N + 63) / 64) * ((K + 63) / 64) * 256, 8), 256, 0, s>>>(
       grad, mom, N, K, beta, omb, sumsq, X, Xt);
   count_launches(2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -219,7 +275,7 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
     ep.out = A2;
     ep.out_bf16 = 0;
     if ((e = launch_gemm_bf16(A, r, A, r, r, r, r, ep, status, s)) != cudaSuccess) return e;  // A A
-    ns_combine_kernel<<<grid_for(r * r, 8), 256, 0, s>>>(A, A2, r * r, Bm);
+    ns_combine_kernel<<<grid_for(r * r / 8, 8), 256, 0, s>>>(A, A2, r * r, Bm);
     count_launches(1);
     ep.out = P;
     ep.ldo = c;
@@ -231,7 +287,7 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
       if (N > K) xto = reinterpret_cast<__nv_bfloat16*>(O);
       else xo = reinterpret_cast<__nv_bfloat16*>(O);
     }
-    ns_step_kernel<<<grid_for(((r + 31) / 32) * ((c + 31) / 32) * 256, 8), 256, 0, s>>>(
+    ns_step_kernel<<<grid_for(((r + 63) / 64) * ((c + 63) / 64) * 256, 8), 256, 0, s>>>(
         X, xo, P, r, c, xto);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
