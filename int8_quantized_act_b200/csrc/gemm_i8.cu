@@ -310,6 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the previous kernel's outputs (operands) are visible from here
   const uint32_t tmem_base = *tmem_slot;
   // Contraction splits of kps k-blocks each (one split unless the
   // contraction exceeds the int32-safe length); tile t is split t / per_split.
@@ -431,6 +432,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -506,6 +508,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
+  griddep_wait();  // the previous kernel's outputs (operands) are visible from here
   const uint32_t tmem_base = *tmem_slot;
   // Contraction splits of kps k-blocks each (one split unless the
   // contraction exceeds the int32-safe length); tile t is split t / per_split.
@@ -630,6 +633,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  griddep_launch_dependents();
   __syncwarp();
   tc_fence_before();
   cluster_sync();  // neither CTA leaves while the pair may still touch it
@@ -791,9 +795,9 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
-  kern<<<2 * pairs, NUM_THREADS, PSMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1,
-                                                    ep, status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(NUM_THREADS), PSMEM_BYTES, s, ta, tb,
+                             tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1, ep, status);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
   count_launches(1);
   return e;
@@ -819,10 +823,10 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1,
-                                              A_MN ? BM : a_box_rows(ep.rows), ep,
-                                              status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s, ta, tb, tiles_m,
+                             tiles_n, kblocks, kps, A_MN ? 8 : 1,
+                             A_MN ? BM : a_box_rows(ep.rows), ep, status);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
   count_launches(1);
   return e;

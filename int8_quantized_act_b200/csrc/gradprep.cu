@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   ring.init(tid);
   __syncthreads();
+  griddep_wait();  // dY and the factors (earlier kernels' outputs) are visible from here
   const int cb = blockIdx.x;
   const int tiles = static_cast<int>((M + T::kRows - 1) / T::kRows);
   const int t0 = blockIdx.y * tiles_per_cta;
@@ -228,6 +229,7 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
       fcur = fnext;
     });
   }
+  griddep_launch_dependents();
   __syncthreads();  // ring drained (the producer waited for its copies): reuse it
   if (warp < 8) {
 #pragma unroll
@@ -276,6 +278,7 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   ring.init(tid);
   __syncthreads();
+  griddep_wait();  // dY and the factors (earlier kernels' outputs) are visible from here
   const int cb = blockIdx.x;
   const int tiles = static_cast<int>((M + T::kRows - 1) / T::kRows);
   const int t0 = blockIdx.y * tiles_per_cta;
@@ -354,6 +357,7 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
       r1cur = r1next;
     });
   }
+  griddep_launch_dependents();
   __syncthreads();
   if (tid == 0 && s_abort) atomicOr(status, 1 << QL_ERR_TIMEOUT);
 }
@@ -403,17 +407,18 @@ cudaError_t colstats_t(const void* dy, int64_t M, int64_t N, const float* sx, ui
   CUtensorMap tm;
   if (!dy_map<InT>(&tm, dy, M, N)) return cudaErrorInvalidValue;
   const Grid g = plan(M, N, Tile<InT>::kRows, 2);
+  cudaError_t e = cudaSuccess;
   if (rowmax) {
     allow_smem<colstats_tma_kernel<InT, true>>();
-    colstats_tma_kernel<InT, true><<<g.grid, kThreads, kSmemBytes, s>>>(
-        tm, M, static_cast<int>(N), sx, colmax, colsum, sw, rowmax, status, g.tiles_per_cta);
+    e = launch_pdl(colstats_tma_kernel<InT, true>, g.grid, dim3(kThreads), kSmemBytes, s, tm, M,
+                   static_cast<int>(N), sx, colmax, colsum, sw, rowmax, status, g.tiles_per_cta);
   } else {
     allow_smem<colstats_tma_kernel<InT, false>>();
-    colstats_tma_kernel<InT, false><<<g.grid, kThreads, kSmemBytes, s>>>(
-        tm, M, static_cast<int>(N), sx, colmax, colsum, sw, rowmax, status, g.tiles_per_cta);
+    e = launch_pdl(colstats_tma_kernel<InT, false>, g.grid, dim3(kThreads), kSmemBytes, s, tm, M,
+                   static_cast<int>(N), sx, colmax, colsum, sw, rowmax, status, g.tiles_per_cta);
   }
   count_launches(1);
-  return cudaGetLastError();
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template <typename InT>
@@ -423,17 +428,18 @@ cudaError_t dualquant_t(const void* dy, int64_t M, int64_t N, const float* cs1,
   CUtensorMap tm;
   if (!dy_map<InT>(&tm, dy, M, N)) return cudaErrorInvalidValue;
   const Grid g = plan(M, N, Tile<InT>::kRows, 2);
+  cudaError_t e = cudaSuccess;
   if (q1) {
     allow_smem<dualquant_tma_kernel<InT, true>>();
-    dualquant_tma_kernel<InT, true><<<g.grid, kThreads, kSmemBytes, s>>>(
-        tm, M, static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
+    e = launch_pdl(dualquant_tma_kernel<InT, true>, g.grid, dim3(kThreads), kSmemBytes, s, tm, M,
+                   static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
   } else {
     allow_smem<dualquant_tma_kernel<InT, false>>();
-    dualquant_tma_kernel<InT, false><<<g.grid, kThreads, kSmemBytes, s>>>(
-        tm, M, static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
+    e = launch_pdl(dualquant_tma_kernel<InT, false>, g.grid, dim3(kThreads), kSmemBytes, s, tm, M,
+                   static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
   }
   count_launches(1);
-  return cudaGetLastError();
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 }  // namespace

@@ -18,6 +18,26 @@ const DeviceInfo& device_info();  // current device, cached
 // Launch accounting (ql_kernel_launches) and the GEMM timing events
 // (ql_set_gemm_timing_events) of the calling thread.
 void count_launches(int n);
+
+// Launch kern<<<grid, block, smem, s>>>(args...) with programmatic stream
+// serialization: it may start while the previous kernel on the stream
+// finishes (its prologue overlaps that kernel's tail) and calls
+// griddep_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 void gemm_timing_events(cudaEvent_t* before, cudaEvent_t* after);
 
 // 2-D tensor map over a row-major [outer][inner] array of elem_bytes-byte

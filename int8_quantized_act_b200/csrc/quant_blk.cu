@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kBlkThreads, 2) quant_blk_kernel(
   }
   if (t < 2 * kBlkMaxRows) s_rmax[t / kBlkMaxRows][t % kBlkMaxRows] = 0u;
   __syncthreads();
+  griddep_wait();  // the rows (a previous kernel's output) are visible from here
   if (t == 0) {
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_q);
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(kBlkThreads, 2) quant_blk_kernel(
     fence_proxy_async_smem();  // the codes, before a store reads them
     done = i + 1;
   }
+  griddep_launch_dependents();
   __syncthreads();
   if (t == 0 && !s_abort && mine > 0) {
     const int64_t last = blockIdx.x + (mine - 1) * gridDim.x;
@@ -298,8 +300,9 @@ cudaError_t launch_blk_t(const CUtensorMap& tx, const CUtensorMap& tq, int64_t r
   const int smem = 1024 + stages * stage_bytes + 2 * out_bytes;
   const int64_t tiles = (rows + R - 1) / R;
   const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(device_info().sms) * per_sm));
-  kern<<<grid, threads, smem, s>>>(tx, tq, rows, nb, R, hc, flags, rs, st, stages, stage_bytes);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(threads), static_cast<size_t>(smem), s, tx,
+                                   tq, rows, nb, R, hc, flags, rs, st, stages, stage_bytes);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 }  // namespace

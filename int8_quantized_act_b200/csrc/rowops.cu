@@ -499,6 +499,8 @@ __global__ void __launch_bounds__(256) dequant_rows_kernel(const int8_t* __restr
 // column statistics pass accumulates into them: one launch for all three.
 __global__ void zero_stats_kernel(uint32_t* __restrict__ colmax, double* __restrict__ colsum,
                                   int64_t N, uint32_t* __restrict__ rowmax, int64_t M) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N + M; i += stride) {
     if (i < N) {
@@ -516,6 +518,8 @@ __global__ void finalize_both_kernel(const uint32_t* __restrict__ colmax,
                                      const double* __restrict__ colsum, int64_t N, float* s2,
                                      float* inv2, float* db, const uint32_t* __restrict__ rowmax,
                                      int64_t M, float* s1, float* inv1) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < N) {
     const float amax = __uint_as_float(colmax[i]);
@@ -703,19 +707,20 @@ cudaError_t launch_dequant_rows(const int8_t* q, int64_t ldq, const float* s, vo
 cudaError_t launch_zero_stats(uint32_t* colmax, double* colsum, int64_t N, uint32_t* rowmax,
                               int64_t M, cudaStream_t s) {
   const int64_t n = N + (rowmax ? M : 0);
-  zero_stats_kernel<<<grid_cap((n + 255) / 256, 4), 256, 0, s>>>(colmax, colsum, N, rowmax,
-                                                                 rowmax ? M : 0);
+  const cudaError_t e = launch_pdl(zero_stats_kernel, dim3(grid_cap((n + 255) / 256, 4)), dim3(256),
+                                   0, s, colmax, colsum, N, rowmax, rowmax ? M : 0);
   count_launches(1);
-  return cudaGetLastError();
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 cudaError_t launch_finalize_both(const uint32_t* colmax, const double* colsum, int64_t N,
                                  float* s2, float* inv2, float* db, const uint32_t* rowmax,
                                  int64_t M, float* s1, float* inv1, cudaStream_t s) {
-  finalize_both_kernel<<<static_cast<unsigned>((N + M + 255) / 256), 256, 0, s>>>(
-      colmax, colsum, N, s2, inv2, db, rowmax, M, s1, inv1);
+  const cudaError_t e = launch_pdl(finalize_both_kernel, dim3(static_cast<unsigned>((N + M + 255) / 256)),
+                                   dim3(256), 0, s, colmax, colsum, N, s2, inv2, db, rowmax, M, s1,
+                                   inv1);
   count_launches(1);
-  return cudaGetLastError();
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 

@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
   const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
   const int64_t row = static_cast<int64_t>(n) * K;
   const uint32_t bar = smem_u32(&s_full);
+  griddep_wait();  // the gradient (an earlier kernel's output) is visible from here
   if (t == 0) {
     mbar_init(bar, 1);
     s_abort = 0;
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
     sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
     if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
   }
+  griddep_launch_dependents();
   // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
   // step lo, step hi), key = seed); chunk ch of this row is block row/4 + ch.
   uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
@@ -274,6 +276,7 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
   // a row takes 5 bytes of shared memory per element and several rows share
   // an SM.
   const uint32_t bar = smem_u32(&s_full);
+  griddep_wait();  // the gradient (an earlier kernel's output) is visible from here
   if (t == 0) {
     mbar_init(bar, 1);
     s_abort = 0;
@@ -443,6 +446,7 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
     sw[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
     if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
   }
+  griddep_launch_dependents();
   // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
   // step lo, step hi), key = seed); chunk ch of this row is block row/4 + ch.
   uint32_t* q_out = reinterpret_cast<uint32_t*>(wq + row);
@@ -515,6 +519,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
     fence_mbar_init();
   }
   __syncthreads();
+  griddep_wait();  // the gradient (an earlier kernel's output) is visible from here
   if (warp == kRingConsumers / 32) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -635,6 +640,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
     // s_max and the parked row are rewritten by the next row.
     if (consumers_sync_or(s_abort)) break;
   }
+  griddep_launch_dependents();
   if (t == 0 && s_abort) atomicOr(status, 1 << QL_ERR_TIMEOUT);
 }
 
@@ -709,6 +715,7 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
                              const UpdateConsts& c, float* m, float* v, uint64_t seed,
                              uint64_t step, float* g, float* g_m, float* g_v, int32_t* status,
                              cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
   const int ngroups = static_cast<int>(K / 16);
   int T = 32;
   while (T < ngroups && T < 256) T <<= 1;
@@ -726,7 +733,7 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     cudaGetDevice(&dev);
     if (dev < 64 && !__atomic_load_n(&wn_set[dev], __ATOMIC_ACQUIRE)) {
       cudaFuncAttributes fa{};
-      cudaError_t e = cudaFuncGetAttributes(&fa, update_sr_wn_staged_kernel);
+      e = cudaFuncGetAttributes(&fa, update_sr_wn_staged_kernel);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(update_sr_wn_staged_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -744,10 +751,10 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     }
     const int nch = static_cast<int>(K / 4);
     const int tr = std::max(T, std::min(256, std::max(32, (nch / QL_UPDATE_STAGED_CHUNKS + 31) / 32 * 32)));
-    update_sr_wn_staged_kernel<<<grid, tr, static_cast<size_t>(row_bytes), s>>>(
-        wq, sw, grad, k, c, m, v, keys, tl, th, g, g_m, g_v, T, status);
+    e = launch_pdl(update_sr_wn_staged_kernel, dim3(grid), dim3(tr), static_cast<size_t>(row_bytes),
+                   s, wq, sw, grad, k, c, m, v, keys, tl, th, g, g_m, g_v, T, status);
     count_launches(1);
-    return cudaGetLastError();
+    return e == cudaSuccess ? cudaGetLastError() : e;
   } else {
     const int nch = static_cast<int>(K / 4);
     PhiloxKeys keys;
@@ -767,10 +774,10 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
                              static_cast<int>(budget));
         __atomic_store_n(&staged_set[dev], true, __ATOMIC_RELEASE);
       }
-      update_sr_staged_kernel<<<grid, tr, static_cast<size_t>(row_bytes), s>>>(
-          wq, sw, grad, k, c, m, v, keys, tl, th, status);
+      e = launch_pdl(update_sr_staged_kernel, dim3(grid), dim3(tr), static_cast<size_t>(row_bytes),
+                     s, wq, sw, grad, k, c, m, v, keys, tl, th, status);
       count_launches(1);
-      return cudaGetLastError();
+      return e == cudaSuccess ? cudaGetLastError() : e;
     }
     // Longer rows: the piece ring, with as many stages as fit beside the
     // parked row (4 K bytes).
@@ -794,13 +801,13 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
         }
         const unsigned rgrid = static_cast<unsigned>(std::min<int64_t>(N, device_info().sms));
         if (c.kind == QL_ADAMW)
-          update_sr_ring_kernel<true><<<rgrid, kRingThreads, smem, s>>>(
-              wq, sw, grad, N, k, c, m, v, keys, tl, th, stages, status);
+          e = launch_pdl(update_sr_ring_kernel<true>, dim3(rgrid), dim3(kRingThreads), smem, s, wq,
+                         sw, grad, N, k, c, m, v, keys, tl, th, stages, status);
         else
-          update_sr_ring_kernel<false><<<rgrid, kRingThreads, smem, s>>>(
-              wq, sw, grad, N, k, c, m, v, keys, tl, th, stages, status);
+          e = launch_pdl(update_sr_ring_kernel<false>, dim3(rgrid), dim3(kRingThreads), smem, s, wq,
+                         sw, grad, N, k, c, m, v, keys, tl, th, stages, status);
         count_launches(1);
-        return cudaGetLastError();
+        return e == cudaSuccess ? cudaGetLastError() : e;
       }
     }
     return cudaErrorInvalidConfiguration;  // unreachable for K <= 32768
