@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
     float* __restrict__ g_v, int L, int32_t* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_red[256];
+  __shared__ float s_amax[16];  // row maximum per warp (s_red may still be read)
   __shared__ float s_qhat[256];  // q / ||q|| for every byte value q = -128 .. 127
   __shared__ int s_ired[16];
   __shared__ float s_dg;
@@ -301,15 +302,12 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
   const uint32_t* q_s = reinterpret_cast<const uint32_t*>(smem);
   float4* g_s = reinterpret_cast<float4*>(smem + qbytes);  // then the updated direction
 
-  // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31).
+  // ||q||^2 as an exact integer sum (<= 127^2 * 32768 < 2^31), four codes
+  // a dot-product instruction.
   int ss = 0;
   for (int ch = t; ch < nch; ch += T) {
-    const uint32_t q4 = q_s[ch];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int qc = static_cast<int8_t>(q4 >> (8 * e));
-      ss += qc * qc;
-    }
+    const int q4 = static_cast<int>(q_s[ch]);
+    ss = __dp4a(q4, q4, ss);
   }
   ss = warp_sum_i(ss);
   if (lane == 0) s_ired[warp] = ss;
@@ -339,22 +337,48 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
       for (int e = 0; e < 16; ++e) p = p + gr[e] * s_qhat[code_at(q4, e) + 128];
     }
   }
-  for (int off = 128; off >= 1; off >>= 1) {
-    if (off >= L) {
-      p = p + 0.0f;
-    } else if (off >= 32) {
-      if (t < L) s_red[t] = p;
-      __syncthreads();
-      const float o = t < L ? s_red[t ^ off] : 0.0f;
-      __syncthreads();
-      p = p + o;
-    } else {
-      p = p + __shfl_xor_sync(0xFFFFFFFFu, p, off);
+  // The butterfly p += p[lane ^ off], off = 128 .. 1, over the 256 virtual
+  // lanes.  Levels with off >= L add a partner that holds +0 (once is the
+  // same as repeatedly).  The levels 32 <= off < L cross warps: every lane's
+  // column of values goes through shared memory once and each thread repeats
+  // the levels for all L/32 warps of its column (own + partner, the same
+  // additions the partners make), keeping its own warp's result.  The levels
+  // below 32 are shuffles.
+  if (L < 256) p = p + 0.0f;
+  if (L > 32) {
+    if (t < L) s_red[t] = p;
+    __syncthreads();
+    if (t < L) {
+      const int W = L >> 5;
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = u < W ? s_red[u * 32 + lane] : 0.0f;
+#pragma unroll
+      for (int k = 4; k >= 1; k >>= 1) {
+        if (k < W) {
+          float nv[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) nv[u] = v[u] + v[u ^ k];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = nv[u];
+        }
+      }
+      float mine = v[0];
+#pragma unroll
+      for (int u = 1; u < 8; ++u) mine = warp == u ? v[u] : mine;
+      p = mine;
     }
   }
-  if (t == 0) s_dg = p;  // every lane < L holds the same sum
-  __syncthreads();
-  const float dg = s_dg;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1)
+    if (off < L) p = p + __shfl_xor_sync(0xFFFFFFFFu, p, off);
+  // Every lane < L holds the same sum; lanes >= L (T > L) take it from lane 0.
+  float dg = p;
+  if (L < T) {
+    if (t == 0) s_dg = p;
+    __syncthreads();
+    dg = s_dg;
+  }
   const float coef = gmag_n / (s * nq);
 
   // Optimizer step of every element; moments written back as they are done,
@@ -431,14 +455,14 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
   amax = warp_max(amax);
   bad = warp_or(bad);
   if (lane == 0) {
-    s_red[warp] = amax;
+    s_amax[warp] = amax;
     s_ired[warp] = bad;
   }
   __syncthreads();
   amax = 0.0f;
   bad = 0;
   for (int k = 0; k < nwarps; ++k) {
-    amax = fmaxf(amax, s_red[k]);
+    amax = fmaxf(amax, s_amax[k]);
     bad |= s_ired[k];
   }
   const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
