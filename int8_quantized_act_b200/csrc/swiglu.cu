@@ -25,6 +25,7 @@
 #include "divrn.cuh"
 #include "launch.h"
 #include "rowops.cuh"
+#include "sm100.cuh"
 #include "../../include/qlinear.h"
 
 namespace ql {
@@ -140,31 +141,86 @@ constexpr int kGatePiece = 8;                          // columns per thread per
 constexpr int kGateSpan = kGateThreads * kGatePiece;   // 3584 columns per piece
 
 // One CTA per row of [a | b] (persistent over rows): thread t owns columns
-// j * 3584 + 8t .. +7 of h for pieces j < P, read with 16-byte loads (a warp
-// reads 512 contiguous bytes of a and of b per piece); the row maximum of |h|
-// is a NaN-propagating max, reduced over the warps through shared memory;
-// the codes are stored 8 at a time.  448 threads (14 warps), two CTAs per SM:
-// d_ff = 14336 is exactly four pieces, and the 8 * P values of h a thread
-// holds across its row fit the register budget of two CTAs per SM.
+// j * 3584 + 8t .. +7 of h for pieces j < P.  Each thread streams its own
+// slots of the next row into shared memory with 16-byte asynchronous copies
+// (cp.async, one commit group per piece): piece j of the next row is issued as
+// soon as piece j of this row has been used, so the loads run under the rest
+// of the row's arithmetic, and since a thread reads only what it copied, no
+// barrier guards the slots.  The row maximum of |h| is a NaN-propagating max,
+// reduced over the warps through shared memory; the codes are stored 8 at a
+// time.  448 threads (14 warps), two CTAs per SM: d_ff = 14336 is exactly four
+// pieces, and the 8 * P values of h a thread holds across its row fit the
+// register budget of two CTAs per SM.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// 8 values of a staged slot as float32.
+__device__ __forceinline__ void slot8(uint32_t addr, const __nv_bfloat16*, float (&v)[8]) {
+  const uint4 u = lds128(addr);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = __uint_as_float(w[e] << 16);
+    v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void slot8(uint32_t addr, const float*, float (&v)[8]) {
+  const uint4 u = lds128(addr), w = lds128(addr + 16);
+  v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+  v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+  v[4] = __uint_as_float(w.x); v[5] = __uint_as_float(w.y);
+  v[6] = __uint_as_float(w.z); v[7] = __uint_as_float(w.w);
+}
+
 template <typename InT, int P>
 __global__ void __launch_bounds__(kGateThreads, 2) swiglu_quant_kernel(
     const InT* __restrict__ ab, int64_t M, int F, int64_t ldab, int8_t* __restrict__ hq,
     int64_t ldh, float* __restrict__ sh, int32_t* __restrict__ status) {
+  constexpr int E = kGatePiece * static_cast<int>(sizeof(InT));  // bytes of 8 values
+  extern __shared__ __align__(16) uint8_t stage[];  // [P][a, b][kGateThreads][E]
   __shared__ uint32_t s_wmax[2][kGateThreads / 32];
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const uint32_t base = smem_u32(stage);
+  auto slot = [&](int j, int half) {
+    return base + static_cast<uint32_t>(((j * 2 + half) * kGateThreads + t) * E);
+  };
+  // Piece j of row m into this thread's slots (nothing past the last row or
+  // column), then one commit group either way.
+  auto issue = [&](int64_t m, int j) {
+    const int col = j * kGateSpan + t * kGatePiece;
+    if (m < M && col < F) {
+      const char* ra = reinterpret_cast<const char*>(ab + m * ldab + col);
+      const char* rb = reinterpret_cast<const char*>(ab + m * ldab + F + col);
+#pragma unroll
+      for (int c = 0; c < E; c += 16) {
+        cp_async16(slot(j, 0) + c, ra + c);
+        cp_async16(slot(j, 1) + c, rb + c);
+      }
+    }
+    cp_async_commit();
+  };
+  griddep_wait();  // [a | b] (a previous kernel's output) is visible from here
+#pragma unroll
+  for (int j = 0; j < P; ++j) issue(blockIdx.x, j);
   int par = 0;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x, par ^= 1) {
-    const InT* ra = ab + m * ldab;
-    const InT* rb = ra + F;
+    const int64_t mn = m + gridDim.x;
     float h[P][kGatePiece];
     float mx0 = 0.0f, mx1 = 0.0f;
 #pragma unroll
     for (int j = 0; j < P; ++j) {
+      // P groups are pending (this row's pieces j.., the next row's ..j-1):
+      // the oldest, this row's piece j, has landed once at most P-1 remain.
+      cp_async_wait<P - 1>();
       const int col = j * kGateSpan + t * kGatePiece;
       if (col < F) {
         float a8[8], b8[8];
-        load8(ra + col, a8);
-        load8(rb + col, b8);
+        slot8(slot(j, 0), ab, a8);
+        slot8(slot(j, 1), ab, b8);
         float s8[8], unused[8];
         silu_parts8<false>(a8, s8, unused);
 #pragma unroll
@@ -177,6 +233,7 @@ __global__ void __launch_bounds__(kGateThreads, 2) swiglu_quant_kernel(
 #pragma unroll
         for (int k = 0; k < 8; ++k) h[j][k] = 0.0f;
       }
+      issue(mn, j);  // the slots are free: their values are in h[j]
 #pragma unroll
       for (int k = 0; k < 8; k += 4) {
         mx0 = fmax3_nan(mx0, fabsf(h[j][k]), fabsf(h[j][k + 1]));
@@ -215,6 +272,8 @@ __global__ void __launch_bounds__(kGateThreads, 2) swiglu_quant_kernel(
       if (mb >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
     }
   }
+  griddep_launch_dependents();
+  cp_async_wait<0>();  // the groups issued past the last row are empty
 }
 
 // [da | db] from [a | b] and dh, 8 columns per thread-step:
@@ -262,19 +321,27 @@ template <typename InT, int P>
 cudaError_t gate_quant_t(const void* ab, int64_t M, int F, int64_t ldab, int8_t* hq, int64_t ldh,
                          float* sh, int32_t* st, cudaStream_t s) {
   auto kern = swiglu_quant_kernel<InT, P>;
+  const size_t smem = static_cast<size_t>(P) * 2 * kGateThreads * kGatePiece * sizeof(InT);
   static int occ[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   int per_sm = dev < 64 ? __atomic_load_n(&occ[dev], __ATOMIC_ACQUIRE) : 0;
   if (per_sm <= 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGateThreads, 0) != cudaSuccess ||
-        per_sm < 1)
-      per_sm = 1;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGateThreads, smem);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return e;
+    }
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
     if (dev < 64) __atomic_store_n(&occ[dev], per_sm, __ATOMIC_RELEASE);
   }
   const int grid = static_cast<int>(std::min<int64_t>(M, static_cast<int64_t>(device_info().sms) * per_sm));
-  kern<<<grid, kGateThreads, 0, s>>>(reinterpret_cast<const InT*>(ab), M, F, ldab, hq, ldh, sh, st);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kGateThreads), smem, s,
+                                   reinterpret_cast<const InT*>(ab), M, F, ldab, hq, ldh, sh, st);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 template <typename InT>
