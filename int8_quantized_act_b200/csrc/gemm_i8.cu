@@ -528,8 +528,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         tile_coords(t - sp * per_split, tiles_m, tiles_n, group, tm, tn);
         const int a_row = tm * 256 + static_cast<int>(rank) * 128;
         const int b_col = tn * 256 + static_cast<int>(rank) * 128;
-        const int kb1 = min(kblocks, (sp + 1) * kps);
-        for (int kb = sp * kps; kb < kb1; ++kb) {
+        const int kb0 = sp * kps, kb1 = min(kblocks, (sp + 1) * kps);
+        // Integer products: every other tile of this pair walks its
+        // contraction backwards, so it starts on the k-slices the tiles just
+        // finished (same operand rows for the next tiles of a group) while
+        // they are still in L2; int32 sums are exact in any order.  The MMA
+        // issuer takes the stages as they come (its first stage initialises).
+        const bool back = !F16 && (((t - pair) / npairs) & 1);
+        for (int i = 0; i < kb1 - kb0; ++i) {
+          const int kb = back ? kb1 - 1 - i : kb0 + i;
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -796,7 +803,7 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
   cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(NUM_THREADS), PSMEM_BYTES, s, ta, tb,
-                             tiles_m, tiles_n, kblocks, kps, A_MN ? 8 : 1, ep, status);
+                             tiles_m, tiles_n, kblocks, kps, A_MN ? 16 : 1, ep, status);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
   count_launches(1);
@@ -824,7 +831,7 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
   cudaError_t e = launch_pdl(kern, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s, ta, tb, tiles_m,
-                             tiles_n, kblocks, kps, A_MN ? 8 : 1,
+                             tiles_n, kblocks, kps, A_MN ? 16 : 1,
                              A_MN ? BM : a_box_rows(ep.rows), ep, status);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
