@@ -404,7 +404,16 @@ def run_ours(args, rank, world, local):
                      "traffic": (GEMM_TRAFFIC_BYTES if gemm_source_sha() == GEMM_TRAFFIC_SOURCE_SHA
                                  else None),
                      "traffic_unit": "bytes per launch",
-                     "frac_of_nominal_int8": round(gemm_tops / NOMINAL_INT8_TOPS, 4)},
+                     "frac_of_nominal_int8": round(gemm_tops / NOMINAL_INT8_TOPS, 4),
+                     # the same against the sustained (power-capped, seconds-long) bf16 figure,
+                     # and against the burst peak scaled to the median SM clock sampled in the
+                     # timed region
+                     "frac_of_sustained": round(gemm_tops / (peaks["bf16_tflops_sustained"]
+                                                              * NOMINAL_INT8_OVER_BF16), 4),
+                     "frac_at_sampled_clock": (round(gemm_tops / (int8_peak * clk["sm_mhz"]
+                                                                  / clk["sm_max_mhz"]), 4)
+                                               if clk.get("sm_mhz") and clk.get("sm_max_mhz")
+                                               else None)},
         "row_kernel": {"kernel": "update_sr (AdamW + stochastic requant)", "bound": "hbm",
                        "achieved": round(UPDATE_BYTES / (upd_ms * 1e-3) / 1e9, 1),
                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
