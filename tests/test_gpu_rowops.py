@@ -65,6 +65,33 @@ def test_quantize_rows_bit_exact(rows, cols, B, dtype):
     assert np.array_equal(q, rq)
 
 
+# bf16 rows that take the two-threads-per-block quantizer (at least one
+# tile of R = min(32, 128 / blocks) rows per SM): every block width it
+# instantiates, one 128-column block per row (R = 32) up to 128 blocks per row
+# (R = 1), and row counts that leave a ragged last tile.
+BLK_CASES = [
+    # rows, cols, B
+    (2400, 1024, 0), (2401, 1024, 2), (2400, 1024, 4), (2401, 1024, 8),
+    (2400, 1024, 16), (2401, 1024, 32), (2400, 1024, 64), (2401, 1024, 128),
+    (4801, 128, 128), (4801, 128, 64),
+    (300, 16384, 128), (301, 16384, 32),
+    (1337, 3456, 128),
+]
+
+
+@pytest.mark.parametrize("rows,cols,B", BLK_CASES)
+def test_quantize_rows_block_quantizer_bit_exact(rows, cols, B):
+    x = workloads.normal((rows, cols), 1.0, rows * 13 + cols + B)
+    x[:, : max(1, cols // 64)] *= np.float32(25.0)
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    x32 = xt.float().numpy()
+    q, s, st = _quant_gpu(dev(xt), B)
+    rq, rs, rst = oracle.quantize_rows(x32, B=B)
+    assert st == 0 and rst == 0
+    assert np.array_equal(s, rs)
+    assert np.array_equal(q, rq)
+
+
 @pytest.mark.parametrize("rows", [96, 700])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_quantize_rows_with_col_scale(dtype, rows):
