@@ -86,11 +86,13 @@ struct Ring {
   }
 
   // Producer (one thread): load tile t of column block cb into each free
-  // stage, the first nsub quarters (those that start before the last column).
+  // stage, the first nsub quarters (those that start before the last column);
+  // tiles t0 .. t1-1 in increasing order, or decreasing with rev.
   __device__ void produce(const CUtensorMap* tm, int cb, int nsub, int t0, int t1,
-                          int rows_per_tile) {
+                          int rows_per_tile, bool rev = false) {
     uint32_t issued = 0, issued_phase = 0;
-    for (int t = t0, k = 0; t < t1; ++t, ++k) {
+    for (int k = 0; k < t1 - t0; ++k) {
+      const int t = rev ? t1 - 1 - k : t0 + k;
       const int s = k % kStages;
       const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
       if (k >= kStages && !mbar_wait(smem_u32(&empty[s]), ph ^ 1u, abort_flag)) break;
@@ -106,11 +108,13 @@ struct Ring {
       if (issued & (1u << s)) mbar_wait_drain(smem_u32(&full[s]), (issued_phase >> s) & 1u);
   }
 
-  // Consumer warp: wait for tile k, run body, release the stage.
+  // Consumer warp: wait for tile k, run body, release the stage (the
+  // producer's tile order).
   template <typename F>
-  __device__ void consume(int t0, int t1, int lane, F&& body) {
+  __device__ void consume(int t0, int t1, int lane, F&& body, bool rev = false) {
     const uint32_t base = smem_u32(buf);
-    for (int t = t0, k = 0; t < t1; ++t, ++k) {
+    for (int k = 0; k < t1 - t0; ++k) {
+      const int t = rev ? t1 - 1 - k : t0 + k;
       const int s = k % kStages;
       const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
       if (!mbar_wait(smem_u32(&full[s]), ph, abort_flag)) break;
@@ -261,7 +265,9 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
 }
 
 // Pass 2: q2[m,n] = rne((dY*rs2[m]) * cinv2[n]) and, with Q1,
-// q1[m,n] = rne((dY*cs1[n]) * rinv1[m]).
+// q1[m,n] = rne((dY*cs1[n]) * rinv1[m]).  Each CTA walks its tiles in the
+// reverse of pass 1's order, so it starts on the tiles pass 1 read last,
+// which are the likeliest to be still in L2.
 template <typename InT, bool Q1>
 __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
     const __grid_constant__ CUtensorMap tm, int64_t M, int N, const float* __restrict__ cs1,
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
   if (warp == 8) {
     if (lane == 0) {
       tma_prefetch_desc(&tm);
-      ring.produce(&tm, cb, nsub, t0, t1, T::kRows);
+      ring.produce(&tm, cb, nsub, t0, t1, T::kRows, true);
     }
     __syncwarp();
   } else {
@@ -307,17 +313,17 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
     const uint32_t qoff = static_cast<uint32_t>(sub * (kTileBytes / kSub));
     auto load_rows = [&](int t, float& f2, float& r1) {
       const int64_t m = static_cast<int64_t>(t) * T::kRows + rw0 + lane;
-      const bool in = lane < RW && t < t1 && m < M;
+      const bool in = lane < RW && t >= t0 && t < t1 && m < M;
       f2 = in ? __ldg(rs2 + m) : 0.0f;
       r1 = (Q1 && in) ? __ldg(rinv1 + m) : 0.0f;
     };
     float f2cur, r1cur;
-    load_rows(t0, f2cur, r1cur);
+    load_rows(t1 - 1, f2cur, r1cur);
     ring.consume(t0, t1, lane, [&](int t, uint32_t stage) {
       if (!live) return;  // a quarter past the last column: nothing loaded
       const uint32_t tile = stage + qoff;
       float f2next, r1next;
-      load_rows(t + 1, f2next, r1next);
+      load_rows(t - 1, f2next, r1next);
 #pragma unroll
       for (int j = 0; j < RW; ++j) {
         const int r = rw0 + j;
@@ -355,7 +361,7 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
       }
       f2cur = f2next;
       r1cur = r1next;
-    });
+    }, true);
   }
   griddep_launch_dependents();
   __syncthreads();

@@ -140,7 +140,9 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
   __shared__ uint32_t s_max[16];
   __shared__ __align__(8) uint64_t s_full;
   __shared__ volatile int s_abort;
-  const int n = blockIdx.x;
+  // Rows from the last: the gradient rows a preceding GEMM wrote last are the
+  // likeliest to be still in L2 (the result does not depend on the order).
+  const int n = gridDim.x - 1 - blockIdx.x;
   const int t = threadIdx.x;
   const int T = blockDim.x;
   const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
   __shared__ float s_dg;
   __shared__ __align__(8) uint64_t s_full;  // codes + gradient
   __shared__ volatile int s_abort;
-  const int n = blockIdx.x;
+  const int n = gridDim.x - 1 - blockIdx.x;  // rows from the last, as the staged kernel
   const int t = threadIdx.x;
   const int T = blockDim.x;  // multiple of 32, L .. 256
   const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
@@ -490,7 +492,7 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
 }
 
 // Rows too long to stage whole (more than ~8.8K elements with AdamW): one
-// persistent CTA per SM walks its rows n = blockIdx.x, + gridDim.x, ... while
+// persistent CTA per SM walks its rows N-1-i for i = blockIdx.x, + gridDim.x, ... while
 // a producer warp streams every row's codes, gradient and moments through a
 // ring of 2048-element pieces by bulk copies, continuing into the next row
 // without a break, so HBM stays busy while the consumers finish a row (its
@@ -550,7 +552,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
       uint32_t issued = 0, issued_phase = 0;
       bool ok = true;
       int k = 0;
-      for (int64_t n = blockIdx.x; n < N && ok; n += gridDim.x) {
+      for (int64_t i = blockIdx.x; i < N && ok; i += gridDim.x) {
+        const int64_t n = N - 1 - i;  // rows from the last (see the consumers)
         const int64_t row = n * K;
         for (int p = 0; p < npieces; ++p, ++k) {
           const int st = k % stages;
@@ -584,7 +587,10 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
   constexpr int T = kRingConsumers;
   const int nch_row = K >> 2;
   int k = 0;
-  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+  for (int64_t i = blockIdx.x; i < N; i += gridDim.x) {
+    // Rows from the last: the gradient rows a preceding GEMM wrote last are
+    // the likeliest to be still in L2 (the result does not depend on the order).
+    const int64_t n = N - 1 - i;
     const int64_t row = n * K;
     const float s = sw[n];
     float4* m_out = reinterpret_cast<float4*>(mom1 + row);
