@@ -16,7 +16,7 @@
 // remainder, each a correctly rounded fused multiply-add; e^r by the Taylor
 // series to degree 7 in Horner form (fused multiply-adds); times 2^n as the
 // product of two exact powers of two.  x is clamped to [-104, 89] first.
-// Groups of eight values whose a lie in [-16, 2^100] (|a| >= 2^-90) take a
+// Groups of eight values whose a lie in [-16, 86] (|a| >= 2^-90) take a
 // faster form with the same results (exp_fast2, and the correctly rounded
 // division of divrn.cuh); others take these steps as written and the IEEE
 // division.
@@ -57,18 +57,16 @@ __device__ __forceinline__ float exp_ref(float x) {
   return __fmul_rn(__fmul_rn(p, __int_as_float((a + 127) << 23)), __int_as_float((n - a + 127) << 23));
 }
 
-// e^x of two values at once for x <= 16, with packed f32x2 multiplies and
-// fused multiply-adds (each half one correctly rounded operation): the same
-// result as exp_ref for -86.5 <= x <= 16, and for x < -86.5 the value at
-// -86.5 (below 2^-125, so 1 + e^x is exactly 1 for both, the only use made
-// of it).  Then n lies in [-125, 23]: the Horner steps run on 2p (every
-// coefficient doubled: each step scales exactly), and 2p * 2^(n-1), one
-// multiply by a normal power of two, is p * 2^n with the one rounding of the
-// two exact-then-rounded multiplies of exp_ref.  The rounding addition is
+// e^x of two values at once for -86 <= x <= 16, with packed f32x2
+// multiplies and fused multiply-adds (each half one correctly rounded
+// operation): the same result as exp_ref.  n lies in [-125, 23]: the Horner
+// steps run on 2p (every coefficient doubled: each step scales exactly), and
+// 2p * 2^(n-1), one multiply by a normal power of two, is p * 2^n with the
+// one rounding of the two exact-then-rounded multiplies of exp_ref.  The rounding addition is
 // scalar: a packed add of a packed product's result is fused into one fma by
 // the code generator, which would skip the rounding of y.
 __device__ __forceinline__ float2 exp_fast2(float2 x) {
-  const float x0 = fmaxf(x.x, -86.5f), x1 = fmaxf(x.y, -86.5f);
+  const float x0 = x.x, x1 = x.y;
   const float2 y = mul2(make_float2(x0, x1), make_float2(0x1.715476p+0f, 0x1.715476p+0f));
   const float t0 = __fadd_rn(y.x, kMagic), t1 = __fadd_rn(y.y, kMagic);
   const float2 mn = sub2(make_float2(kMagic, kMagic), make_float2(t0, t1));  // -rint(y)
@@ -88,9 +86,9 @@ __device__ __forceinline__ float2 exp_fast2(float2 x) {
   return mul2(p, make_float2(s0, s1));
 }
 
-// Whether eight gate values take the fast steps: every a in [-16, 2^100]
-// with |a| >= 2^-90 (no zero, NaN or infinity).  Then x = -a <= 16, so
-// d = 1 + e^-a lies in [1, 2^24], and a / d is a normal float: the range of
+// Whether eight gate values take the fast steps: every a in [-16, 86] with
+// |a| >= 2^-90 (no zero, NaN or infinity).  Then x = -a lies in [-86, 16],
+// d = 1 + e^-a in [1, 2^24], and a / d is a normal float: the range of
 // exp_fast2 and of the division's correction steps (divrn.cuh).
 __device__ __forceinline__ bool fast_ok8(const float (&a)[8]) {
   float lo = fmin3_nan(a[0], a[1], a[2]), hi = fmax3_nan(a[0], a[1], a[2]);
@@ -104,7 +102,7 @@ __device__ __forceinline__ bool fast_ok8(const float (&a)[8]) {
   lo = fmin_nan(lo, a[7]);
   hi = fmax_nan(hi, a[7]);
   mg = fmin_nan(mg, fabsf(a[7]));
-  return lo >= -16.0f && hi <= 0x1p+100f && mg >= 0x1p-90f;
+  return lo >= -16.0f && hi <= 86.0f && mg >= 0x1p-90f;
 }
 
 // d = 1 + e^-a and (with Q) q = a / d for eight values: the fast steps when
