@@ -83,9 +83,25 @@ struct Epi {
 // moment form a compact block and share their operand stripes in L2.
 // group = 1 is plain row-major order (best when the B operand fits in L2 and
 // every tile-row reuses it); the weight gradient, whose operands are both
-// long stripes of the whole contraction, uses groups of 8.
+// long stripes of the whole contraction, uses groups of 16.  group = 0 walks
+// only the upper triangle (tm <= tn) of a square grid, row by row: the
+// symmetric products X X^T and A A, whose lower tiles are the transposes.
+__device__ __forceinline__ int tiles_per_split(int tiles_m, int tiles_n, int group) {
+  return group == 0 ? tiles_m * (tiles_m + 1) / 2 : tiles_m * tiles_n;
+}
+
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int group, int& tm,
                                             int& tn) {
+  if (group == 0) {
+    int r = t, m = 0;
+    while (r >= tiles_m - m) {
+      r -= tiles_m - m;
+      ++m;
+    }
+    tm = m;
+    tn = m + r;
+    return;
+  }
   const int per_group = group * tiles_n;
   const int g = t / per_group;
   const int first = g * group;
@@ -314,7 +330,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   // Contraction splits of kps k-blocks each (one split unless the
   // contraction exceeds the int32-safe length); tile t is split t / per_split.
-  const int per_split = tiles_m * tiles_n;
+  const int per_split = tiles_per_split(tiles_m, tiles_n, group);
   const int num_tiles = per_split * ((kblocks + kps - 1) / kps);
 
   if (warp == 0) {
@@ -512,7 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   // Contraction splits of kps k-blocks each (one split unless the
   // contraction exceeds the int32-safe length); tile t is split t / per_split.
-  const int per_split = tiles_m * tiles_n;
+  const int per_split = tiles_per_split(tiles_m, tiles_n, group);
   const int num_tiles = per_split * ((kblocks + kps - 1) / kps);
   const uint32_t lead_full0 = mapa_shared(full0, 0);
   const uint32_t lead_tempty0 = mapa_shared(tempty0, 0);
@@ -786,7 +802,8 @@ int pair_slots(K kern) {
 
 template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
-                     int kblocks, int kps, const Epi& ep, int32_t* status, cudaStream_t s) {
+                     int kblocks, int kps, const Epi& ep, int32_t* status, cudaStream_t s,
+                     bool upper = false) {
   auto kern = gemm_i8_pair_kernel<A_MN, B_MN, OutT, HB, F16>;
   static int configured[64] = {0};
   int dev = 0;
@@ -796,14 +813,16 @@ cudaError_t run_pair(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, 
     if (e != cudaSuccess) return e;
     __atomic_store_n(&configured[dev], 1, __ATOMIC_RELEASE);
   }
-  const int tiles = tiles_m * tiles_n * ((kblocks + kps - 1) / kps);
+  const int per_split = upper ? tiles_m * (tiles_m + 1) / 2 : tiles_m * tiles_n;
+  const int tiles = per_split * ((kblocks + kps - 1) / kps);
   const int slots = pair_slots(kern);
   const int pairs = tiles < slots ? tiles : slots;
   cudaEvent_t before = nullptr, after = nullptr;
   gemm_timing_events(&before, &after);
   if (before) cudaEventRecord(before, s);
   cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(NUM_THREADS), PSMEM_BYTES, s, ta, tb,
-                             tiles_m, tiles_n, kblocks, kps, A_MN ? 16 : 1, ep, status);
+                             tiles_m, tiles_n, kblocks, kps, upper ? 0 : (A_MN ? 16 : 1), ep,
+                             status);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (after) cudaEventRecord(after, s);
   count_launches(1);
@@ -841,9 +860,12 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int t
 
 template <bool A_MN, bool B_MN, typename OutT, int HB, bool F16 = false>
 cudaError_t go(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, int tiles_m, int tiles_n,
-               int kblocks, const Epi& ep, int32_t* status, cudaStream_t s, int kps = 0) {
+               int kblocks, const Epi& ep, int32_t* status, cudaStream_t s, int kps = 0,
+               bool upper = false) {
   if (kps <= 0) kps = kblocks;
-  if (pair) return run_pair<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, kps, ep, status, s);
+  if (pair)
+    return run_pair<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, kps, ep, status,
+                                               s, upper);
   return run<A_MN, B_MN, OutT, HB, F16>(ta, tb, tiles_m, tiles_n, kblocks, kps, ep, status, s);
 }
 
@@ -998,7 +1020,7 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
 
 cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t rows,
                              int64_t cols, int64_t kc, const GemmEpilogue& e, int32_t* status,
-                             cudaStream_t s) {
+                             cudaStream_t s, bool* upper_only) {
   // Both operands K-major bf16: a 128-byte stage row holds 64 elements and
   // each kind::f16 MMA consumes K = 16 (32 bytes), the same byte layout as
   // the int8 path.
@@ -1033,9 +1055,16 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
       return run<false, false, __nv_bfloat16, 0, true, 64>(ta, tb, tiles_m, tn64, kblocks, kblocks, ep, status, s);
     return run<false, false, float, 0, true, 64>(ta, tb, tiles_m, tn64, kblocks, kblocks, ep, status, s);
   }
+  // A symmetric product (the caller passes upper_only set): with CTA-pair
+  // tiles on a square grid only the upper tiles are computed, and
+  // *upper_only stays true to tell the caller to fill the lower ones.
+  const bool upper = upper_only && *upper_only && pair && rows == cols;
+  if (upper_only) *upper_only = upper;
   if (e.out_bf16)
-    return go<false, false, __nv_bfloat16, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
-  return go<false, false, float, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s);
+    return go<false, false, __nv_bfloat16, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep,
+                                                   status, s, 0, upper);
+  return go<false, false, float, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep, status, s,
+                                          0, upper);
 }
 
 // ------------------------------------------------------------------ long contractions

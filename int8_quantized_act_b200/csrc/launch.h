@@ -192,9 +192,12 @@ cudaError_t launch_gemm_i8_long(const int8_t* A, bool a_mn, int64_t lda, const i
 // The same GEMM on bf16 operands (tcgen05 kind::f16, float32 accumulator):
 // A [rows][kc] and B [cols][kc] both K-major bf16 with pitches lda, ldb
 // elements; out = acc * row_scale * col_scale + bias as above, hb must be 0.
+// upper_only (optional, in/out): for a product known to be symmetric, set
+// it to ask for the upper 256 x 256 tiles only; it comes back true when only
+// those were written (CTA-pair tiles on a square grid), false when all were.
 cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t rows,
                              int64_t cols, int64_t kc, const GemmEpilogue& ep, int32_t* status,
-                             cudaStream_t s);
+                             cudaStream_t s, bool* upper_only = nullptr);
 
 // -------------------------------------------------------------- update
 struct UpdateConsts {

@@ -197,6 +197,75 @@ __global__ void __launch_bounds__(256) ns_step_kernel(const __nv_bfloat16* X,
   }
 }
 
+// 8 consecutive values as float32 and back (exact for bf16).
+__device__ __forceinline__ void load8v(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void load8v(const float* p, float (&v)[8]) { load8f(p, v); }
+__device__ __forceinline__ void store8v(__nv_bfloat16* p, const float (&v)[8]) {
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    o[k] = (__float_as_uint(v[2 * k]) >> 16) | (__float_as_uint(v[2 * k + 1]) & 0xFFFF0000u);
+  *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+__device__ __forceinline__ void store8v(float* p, const float (&v)[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// The lower 256 x 256 tiles of a symmetric r x r matrix (r a multiple of 8)
+// from the upper ones (the symmetric GEMMs write only tiles with tile-row <=
+// tile-column): a[i][j] = a[j][i] where i / 256 > j / 256, by 64 x 64 blocks
+// of the lower tiles only: 16-byte loads of the source block's rows into a
+// shared tile (rows padded to 65 floats), 16-byte stores of the destination's
+// rows gathered from its columns.
+template <typename T>
+__global__ void __launch_bounds__(256) ns_mirror_kernel(T* __restrict__ a, int64_t r) {
+  __shared__ float tile[64][65];
+  const int t = threadIdx.x, tr = t >> 3, tc = (t & 7) * 8;
+  const int64_t nt = (r + 255) / 256;  // 256-tiles a side
+  const int64_t blocks = nt * (nt - 1) / 2 * 16;
+  for (int64_t b = blockIdx.x; b < blocks; b += gridDim.x) {
+    int64_t ti = 1, rem = b / 16;  // lower tile (ti, tj), tj < ti, row by row
+    while (rem >= ti) {
+      rem -= ti;
+      ++ti;
+    }
+    const int64_t I = ti * 4 + (b % 16) / 4, J = rem * 4 + (b % 4);  // destination 64-block
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lr = tr + 32 * h;
+      const int64_t i = J * 64 + lr, j = I * 64 + tc;  // source: rows of block (J, I)
+      if (i < r && j < r) {
+        float v[8];
+        load8v(a + i * r + j, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) tile[lr][tc + k] = v[k];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lc = tr + 32 * h;
+      const int64_t i = I * 64 + lc, j = J * 64 + tc;  // destination row i, columns j..j+7
+      if (i < r && j < r) {
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = tile[tc + k][lc];
+        store8v(a + i * r + j, v);
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // AdamW on a float32 vector: the per-element arithmetic of the int8 update.
 __global__ void __launch_bounds__(256) adamw_vector_kernel(float* __restrict__ p,
                                                            const float* __restrict__ g,
@@ -267,14 +336,29 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
   count_launches(2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   for (int it = 0; it < steps; ++it) {
+    // A = X X^T and A A are symmetric: the GEMM computes the upper tiles and
+    // the lower ones are copied from them (exactly symmetric results).
+    const int64_t nt = (r + 255) / 256;
+    const int mgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(
+        nt * (nt - 1) / 2 * 16, static_cast<int64_t>(device_info().sms) * 8)));
     GemmEpilogue ep;
     ep.out = A;
     ep.out_bf16 = 1;
     ep.ldo = r;
-    if ((e = launch_gemm_bf16(X, c, X, c, r, r, c, ep, status, s)) != cudaSuccess) return e;  // A = X X^T
+    bool upper = true;
+    if ((e = launch_gemm_bf16(X, c, X, c, r, r, c, ep, status, s, &upper)) != cudaSuccess) return e;  // A = X X^T
+    if (upper) {
+      ns_mirror_kernel<__nv_bfloat16><<<mgrid, 256, 0, s>>>(A, r);
+      count_launches(1);
+    }
     ep.out = A2;
     ep.out_bf16 = 0;
-    if ((e = launch_gemm_bf16(A, r, A, r, r, r, r, ep, status, s)) != cudaSuccess) return e;  // A A
+    upper = true;
+    if ((e = launch_gemm_bf16(A, r, A, r, r, r, r, ep, status, s, &upper)) != cudaSuccess) return e;  // A A
+    if (upper) {
+      ns_mirror_kernel<float><<<mgrid, 256, 0, s>>>(A2, r);
+      count_launches(1);
+    }
     ns_combine_kernel<<<grid_for(r * r / 8, 8), 256, 0, s>>>(A, A2, r * r, Bm);
     count_launches(1);
     ep.out = P;
