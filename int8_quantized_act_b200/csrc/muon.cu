@@ -117,6 +117,25 @@ __device__ __forceinline__ void load8f(const float* p, float (&v)[8]) {
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+// 8 consecutive bf16 values as float32 and back (exact).
+__device__ __forceinline__ void load8v(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void store8v(__nv_bfloat16* p, const float (&v)[8]) {
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    o[k] = (__float_as_uint(v[2 * k]) >> 16) | (__float_as_uint(v[2 * k + 1]) & 0xFFFF0000u);
+  *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+
 // X0 = bf16(U / (||U||_F + 1e-7)) with U recomputed from G and the new M
 // (the same float32 operations as muon_momentum_kernel), written as X [r, c]
 // and X^T [c, r], where X = U when N <= K (r = N) and X = U^T otherwise.
@@ -171,6 +190,62 @@ __global__ void __launch_bounds__(256) ns_combine_kernel(const __nv_bfloat16* __
   }
 }
 
+// The same combination for a symmetric A whose square A2 holds only its
+// upper 256 x 256 tiles (tile-row <= tile-column): Bm is symmetric, so each
+// 64 x 64 block of the upper tiles is computed from A and A2 and written
+// both in place and, in a strictly upper tile, transposed into the lower
+// one (through a shared tile, rows padded to 65 floats); the same values as
+// combining the whole of a mirrored A2.
+__global__ void __launch_bounds__(256) ns_combine_sym_kernel(const __nv_bfloat16* __restrict__ A,
+                                                             const float* __restrict__ A2,
+                                                             int64_t r,
+                                                             __nv_bfloat16* __restrict__ Bm) {
+  __shared__ float tile[64][65];
+  const int t = threadIdx.x, tr = t >> 3, tc = (t & 7) * 8;
+  const int64_t nt = (r + 255) / 256;
+  const int64_t blocks = nt * (nt + 1) / 2 * 16;
+  for (int64_t b = blockIdx.x; b < blocks; b += gridDim.x) {
+    int64_t ti = 0, rem = b / 16;  // upper tile (ti, tj), tj >= ti, row by row
+    while (rem >= nt - ti) {
+      rem -= nt - ti;
+      ++ti;
+    }
+    const int64_t tj = ti + rem;
+    const int64_t I = ti * 4 + (b % 16) / 4, J = tj * 4 + (b % 4);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lr = tr + 32 * h;
+      const int64_t i = I * 64 + lr, j = J * 64 + tc;
+      if (i < r && j < r) {
+        float a[8], a2[8], v[8];
+        load8v(A + i * r + j, a);
+        load8f(A2 + i * r + j, a2);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          v[k] = __bfloat162float(__float2bfloat16_rn(
+              __fadd_rn(__fmul_rn(kNsB, a[k]), __fmul_rn(kNsC, a2[k]))));
+          tile[lr][tc + k] = v[k];
+        }
+        store8v(Bm + i * r + j, v);
+      }
+    }
+    if (ti == tj) continue;  // uniform per CTA: a diagonal tile has no mirror image
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lc = tr + 32 * h;
+      const int64_t i = J * 64 + lc, j = I * 64 + tc;  // the transposed block (J, I)
+      if (i < r && j < r) {
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = tile[tc + k][lc];
+        store8v(Bm + i * r + j, v);
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // X' = bf16(a * X + P) for X [r, c] into Xo (X itself, or the output) and
 // its transpose X'^T [c, r] into Xt (transpose64: the thread that reads an
 // element of X writes it in Xo).
@@ -197,37 +272,13 @@ __global__ void __launch_bounds__(256) ns_step_kernel(const __nv_bfloat16* X,
   }
 }
 
-// 8 consecutive values as float32 and back (exact for bf16).
-__device__ __forceinline__ void load8v(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    v[2 * k] = __uint_as_float(w[k] << 16);
-    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-  }
-}
-__device__ __forceinline__ void load8v(const float* p, float (&v)[8]) { load8f(p, v); }
-__device__ __forceinline__ void store8v(__nv_bfloat16* p, const float (&v)[8]) {
-  uint32_t o[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    o[k] = (__float_as_uint(v[2 * k]) >> 16) | (__float_as_uint(v[2 * k + 1]) & 0xFFFF0000u);
-  *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
-}
-__device__ __forceinline__ void store8v(float* p, const float (&v)[8]) {
-  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
-  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
-}
-
-// The lower 256 x 256 tiles of a symmetric r x r matrix (r a multiple of 8)
+// The lower 256 x 256 tiles of a symmetric bf16 r x r matrix (r a multiple of 8)
 // from the upper ones (the symmetric GEMMs write only tiles with tile-row <=
 // tile-column): a[i][j] = a[j][i] where i / 256 > j / 256, by 64 x 64 blocks
 // of the lower tiles only: 16-byte loads of the source block's rows into a
 // shared tile (rows padded to 65 floats), 16-byte stores of the destination's
 // rows gathered from its columns.
-template <typename T>
-__global__ void __launch_bounds__(256) ns_mirror_kernel(T* __restrict__ a, int64_t r) {
+__global__ void __launch_bounds__(256) ns_mirror_kernel(__nv_bfloat16* __restrict__ a, int64_t r) {
   __shared__ float tile[64][65];
   const int t = threadIdx.x, tr = t >> 3, tc = (t & 7) * 8;
   const int64_t nt = (r + 255) / 256;  // 256-tiles a side
@@ -348,18 +399,20 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
     bool upper = true;
     if ((e = launch_gemm_bf16(X, c, X, c, r, r, c, ep, status, s, &upper)) != cudaSuccess) return e;  // A = X X^T
     if (upper) {
-      ns_mirror_kernel<__nv_bfloat16><<<mgrid, 256, 0, s>>>(A, r);
+      ns_mirror_kernel<<<mgrid, 256, 0, s>>>(A, r);
       count_launches(1);
     }
     ep.out = A2;
     ep.out_bf16 = 0;
     upper = true;
     if ((e = launch_gemm_bf16(A, r, A, r, r, r, r, ep, status, s, &upper)) != cudaSuccess) return e;  // A A
-    if (upper) {
-      ns_mirror_kernel<float><<<mgrid, 256, 0, s>>>(A2, r);
-      count_launches(1);
+    if (upper) {  // Bm from A and the upper tiles of A2, mirrored as it is written
+      ns_combine_sym_kernel<<<static_cast<int>(std::min<int64_t>(nt * (nt + 1) / 2 * 16,
+                                                                  static_cast<int64_t>(device_info().sms) * 8)),
+                              256, 0, s>>>(A, A2, r, Bm);
+    } else {
+      ns_combine_kernel<<<grid_for(r * r / 8, 8), 256, 0, s>>>(A, A2, r * r, Bm);
     }
-    ns_combine_kernel<<<grid_for(r * r / 8, 8), 256, 0, s>>>(A, A2, r * r, Bm);
     count_launches(1);
     ep.out = P;
     ep.ldo = c;
