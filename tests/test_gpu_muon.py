@@ -39,7 +39,10 @@ def _orthogonalize(G, M, beta=0.95, steps=5):
     return host(m), O
 
 
-@pytest.mark.parametrize("N,K", [(256, 384), (384, 256), (128, 128), (16, 1040)])
+@pytest.mark.parametrize("N,K", [(256, 384), (384, 256), (128, 128), (16, 1040),
+                                 # two 256-tiles a side with a ragged second one: the
+                                 # symmetric products' upper-tile path and its mirror
+                                 (400, 640), (640, 400), (784, 784)])
 def test_momentum_bit_exact_and_newton_schulz_close(N, K):
     G = workloads.normal((N, K), 1e-3, N + K)
     M = workloads.normal((N, K), 1e-3, N + K + 1)
