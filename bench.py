@@ -45,12 +45,12 @@ NOMINAL_INT8_TOPS = 4500.0     # B200 dense int8 spec, for context next to the m
 # DRAM bytes (read + write) per GEMM launch from an ncu capture of the
 # 12000-token layer step (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
-GEMM_TRAFFIC_BYTES = 372.6e6
-GEMM_TRAFFIC_SOURCE_SHA = "422d63c4c93c197d"
+GEMM_TRAFFIC_BYTES = 336.4e6
+GEMM_TRAFFIC_SOURCE_SHA = "c7ab7c66c3ffc89c"
 # The same for the update kernel on the [7168, 5376] weight; DRAM writes
 # still held in L2 when the kernel ends are not counted.
-UPDATE_TRAFFIC_BYTES = 789.3e6
-UPDATE_TRAFFIC_SOURCE_SHA = "2bf6f7f04bb79f74"
+UPDATE_TRAFFIC_BYTES = 790.5e6
+UPDATE_TRAFFIC_SOURCE_SHA = "cf0218e1b40ac5f0"
 
 
 def source_sha(files=("gemm_i8.cu", "sm100.cuh")):
@@ -66,7 +66,7 @@ def gemm_source_sha():
     return source_sha()
 
 
-UPDATE_SOURCES = ("update_sr.cu", "rowops.cuh", "sm100.cuh")
+UPDATE_SOURCES = ("update_sr.cu", "rowops.cuh", "divrn.cuh", "sm100.cuh")
 
 
 def parse_args():
