@@ -46,14 +46,23 @@ __device__ __forceinline__ float adamw(const UpdateConsts& c, float w, float g, 
 // and every v' lies in [2^-100, 2^100] and every m' in +-[2^-66, 2^60]: then
 // den = sqrt(v')*rbc2 + eps lies in [2^-60, 2^60] and m'/den is a normal
 // float.  Otherwise the IEEE operations; the results are the same bits.
+// Those steps run on pairs of elements (f32x2 multiplies and fused
+// multiply-adds; each half is the scalar IEEE operation).  A product that
+// is added to something stays a scalar multiply: a packed multiply feeding
+// a packed add can be compiled into one fused multiply-add.
 __device__ __forceinline__ void adamw4(const UpdateConsts& c, const float (&w)[4],
                                       const float (&g)[4], float (&m)[4], float (&v)[4],
                                       float (&out)[4]) {
   float mn[4], vn[4], q[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    mn[e] = c.b1 * m[e] + c.omb1 * g[e];
-    vn[e] = c.b2 * v[e] + c.omb2 * (g[e] * g[e]);
+  for (int h = 0; h < 4; h += 2) {
+    const float2 gg = mul2(make_float2(g[h], g[h + 1]), make_float2(g[h], g[h + 1]));
+    const float gs[2] = {gg.x, gg.y};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      mn[h + e] = __fadd_rn(__fmul_rn(c.b1, m[h + e]), __fmul_rn(c.omb1, g[h + e]));
+      vn[h + e] = __fadd_rn(__fmul_rn(c.b2, v[h + e]), __fmul_rn(c.omb2, gs[e]));
+    }
   }
   const float vlo = fmin_nan(fmin3_nan(vn[0], vn[1], vn[2]), vn[3]);
   const float vhi = fmax_nan(fmax3_nan(vn[0], vn[1], vn[2]), vn[3]);
@@ -61,9 +70,26 @@ __device__ __forceinline__ void adamw4(const UpdateConsts& c, const float (&w)[4
   const float mhi = fmax_nan(fmax3_nan(fabsf(mn[0]), fabsf(mn[1]), fabsf(mn[2])), fabsf(mn[3]));
   if (c.fast && vlo >= 0x1p-100f && vhi <= 0x1p+100f && mlo >= 0x1p-66f && mhi <= 0x1p+60f) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float den = sqrt_rn_t<false>(vn[e]) * c.rbc2 + c.eps;
-      q[e] = div_rn(mn[e], den, recip_rn(den));
+    for (int h = 0; h < 4; h += 2) {
+      // sqrt_rn_t<false> (v' > 0 here), then recip_rn and div_rn, two at a time
+      const float2 vv = make_float2(vn[h], vn[h + 1]);
+      const float2 z = make_float2(rsqrt_approx(vv.x), rsqrt_approx(vv.y));
+      const float2 g0 = mul2(vv, z);
+      const float2 hz = mul2(make_float2(0.5f, 0.5f), z);
+      const float2 rs = fma2(make_float2(-g0.x, -g0.y), g0, vv);
+      const float2 sq = fma2(rs, hz, g0);
+      const float d0 = __fadd_rn(__fmul_rn(sq.x, c.rbc2), c.eps);
+      const float d1 = __fadd_rn(__fmul_rn(sq.y, c.rbc2), c.eps);
+      const float2 nd = make_float2(-d0, -d1);
+      const float2 y0 = make_float2(rcp_approx(d0), rcp_approx(d1));
+      const float2 ey = fma2(nd, y0, make_float2(1.0f, 1.0f));
+      const float2 y = fma2(y0, ey, y0);
+      const float2 mm = make_float2(mn[h], mn[h + 1]);
+      const float2 q0 = mul2(mm, y);
+      const float2 rq = fma2(nd, q0, mm);
+      const float2 qq = fma2(rq, y, q0);
+      q[h] = qq.x;
+      q[h + 1] = qq.y;
     }
   } else {
 #pragma unroll
@@ -71,22 +97,44 @@ __device__ __forceinline__ void adamw4(const UpdateConsts& c, const float (&w)[4
   }
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    out[e] = w[e] * c.a - c.st * q[e];
+    out[e] = __fsub_rn(__fmul_rn(w[e], c.a), __fmul_rn(c.st, q[e]));
     m[e] = mn[e];
     v[e] = vn[e];
   }
 }
 
-// floor(v) + 1 with probability frac(v), decided by u24 < frac * 2^24;
-// clamped to [-127, 127].  Returns rne_bits of the (integer-valued) result, so
-// its low byte is the int8 code (exact: adding 1.5*2^23 to an integer-valued
-// float below 2^22 in magnitude is exact).
-__device__ __forceinline__ uint32_t sr_code_bits(float val, uint32_t u24) {
-  const float f = floorf(val);
-  const float frac = val - f;
-  float r = (__uint2float_rn(u24) < frac * 16777216.0f) ? f + 1.0f : f;
-  r = fminf(fmaxf(r, -127.0f), 127.0f);
-  return rne_bits(r);
+// The codes of a 4-element chunk w under the scale inverse inv with the
+// chunk's Philox words rn: for v = w[e] * inv and u24 = rn[e] >> 8, floor(v)
+// + 1 with probability frac(v), decided by u24 < frac * 2^24, clamped to
+// [-127, 127]; the integer-valued result plus 1.5 * 2^23 (exact below 2^22
+// in magnitude) holds the int8 code in its low byte, and the four low bytes
+// are packed.  The products w * inv stay scalar (their difference with the
+// floor is taken next); frac * 2^24, f + 1 and the rounding add run two at
+// a time.
+__device__ __forceinline__ uint32_t sr_codes4(float4 w, float inv, uint4 rn) {
+  const float v[4] = {__fmul_rn(w.x, inv), __fmul_rn(w.y, inv), __fmul_rn(w.z, inv),
+                      __fmul_rn(w.w, inv)};
+  const uint32_t u[4] = {rn.x >> 8, rn.y >> 8, rn.z >> 8, rn.w >> 8};
+  float f[4], fr[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[e] = floorf(v[e]);
+    fr[e] = __fsub_rn(v[e], f[e]);
+  }
+  const float2 s24 = make_float2(16777216.0f, 16777216.0f), one = make_float2(1.0f, 1.0f);
+  const float2 t01 = mul2(make_float2(fr[0], fr[1]), s24), t23 = mul2(make_float2(fr[2], fr[3]), s24);
+  const float2 u01 = add2(make_float2(f[0], f[1]), one), u23 = add2(make_float2(f[2], f[3]), one);
+  const float t[4] = {t01.x, t01.y, t23.x, t23.y}, f1[4] = {u01.x, u01.y, u23.x, u23.y};
+  float r[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    r[e] = (__uint2float_rn(u[e]) < t[e]) ? f1[e] : f[e];
+    r[e] = fminf(fmaxf(r[e], -127.0f), 127.0f);
+  }
+  const float2 mg = make_float2(kRneMagic, kRneMagic);
+  const float2 c01 = add2(make_float2(r[0], r[1]), mg), c23 = add2(make_float2(r[2], r[3]), mg);
+  return pack_codes(__float_as_uint(c01.x), __float_as_uint(c01.y), __float_as_uint(c23.x),
+                    __float_as_uint(c23.y));
 }
 
 __device__ __forceinline__ void load16f(const float* p, float (&v)[16]) {
@@ -124,6 +172,21 @@ __device__ __forceinline__ uint4 philox10_keys(uint4 c, const PhiloxKeys& k) {
 __device__ __forceinline__ float code_byte_f(uint32_t q4, int i) {
   return __fsub_rn(__int_as_float(0x4B400000 + static_cast<int>(static_cast<int8_t>(q4 >> (8 * i)))),
                    12582912.0f);
+}
+
+// wv[e] = s * code_byte_f(q4, e), two at a time (for products that are
+// multiplied next, not added to).
+__device__ __forceinline__ void dequant4(uint32_t q4, float s, float (&wv)[4]) {
+  const float2 mg = make_float2(12582912.0f, 12582912.0f), ss = make_float2(s, s);
+#pragma unroll
+  for (int h = 0; h < 4; h += 2) {
+    const float2 b = make_float2(
+        __int_as_float(0x4B400000 + static_cast<int>(static_cast<int8_t>(q4 >> (8 * h)))),
+        __int_as_float(0x4B400000 + static_cast<int>(static_cast<int8_t>(q4 >> (8 * h + 8)))));
+    const float2 p = mul2(ss, sub2(b, mg));
+    wv[h] = p.x;
+    wv[h + 1] = p.y;
+  }
 }
 
 // The same update with the row staged by the bulk-copy engine: one CTA per
@@ -187,8 +250,7 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
         float m1[4] = {m4.x, m4.y, m4.z, m4.w};
         float m2[4] = {v4.x, v4.y, v4.z, v4.w};
         float wv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) wv[e] = s * code_byte_f(q4, e);
+        dequant4(q4, s, wv);
         adamw4(c, wv, gr, m1, m2, w);
         __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
         __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
@@ -234,26 +296,37 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
     const float4 w = g_s[ch];
     uint32_t out = 0;
     if (mbits != 0)
-      out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
-                       sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+      out = sr_codes4(w, inv, rn);
     __stcs(q_out + ch, out);
   }
 }
 
 // The row-wise weight-norm update with the row's codes and gradient staged
 // in shared memory by two bulk copies, so the gradient is read from HBM once
-// although both the direction-gradient reduction and the update use it; the
-// moments stream through registers in the elementwise step (coalesced
-// 16-byte loads and stores), which keeps a row at 5 bytes of shared memory
-// per element, so several rows share an SM.  Only the dg reduction keeps 16-element groups: the first L threads (L a
-// power of two <= 256) are the virtual lanes of the pinned 256-lane order,
+// although both the direction-gradient reduction and the update use it.
+// With MS (AdamW rows that fit three times in an SM's shared memory at 13
+// bytes per element, K up to ~5.6K) the two moments are staged by two more
+// bulk copies on the same barrier, so every load of the row is in flight at
+// once and the elementwise step reads shared memory only (up to 384
+// threads, three or more CTAs per SM; with two, as at K = 8192, an SM's
+// loads stall while both rows compute, which measured slower than streaming
+// the moments).  Otherwise the moments stream through registers in the
+// elementwise step (coalesced 16-byte loads issued U chunks ahead), which
+// keeps a row at 5 bytes of shared memory per element, so several rows share
+// an SM: U = 1 with four CTAs of up to 64 registers while four rows fit an
+// SM (K up to ~10.8K), U = 4 with three CTAs of 80 registers for longer
+// rows, where shared memory leaves fewer CTAs to hide the loads (512-thread
+// CTAs with U = 1 measured slower there).  Only the dg reduction
+// keeps 16-element groups: the first L threads (L a power of two <= 256) are
+// the virtual lanes of the pinned 256-lane order,
 // lane l adding groups l, l+L, ... (L = 256, or each group has its own lane).
 // ||q||^2 (an integer sum), the elementwise step, the row max and the
 // stochastic rounding are free of order and run on all threads over
 // 4-element chunks as in update_sr_staged_kernel (consecutive threads touch
 // consecutive 16-byte pieces).  Per-element arithmetic and random words are
 // the same IEEE operations as the oracle's, so the results are the same bits.
-__global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
+template <bool MS, int U>
+__global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) update_sr_wn_staged_kernel(
     int8_t* __restrict__ wq, float* __restrict__ sw, const float* __restrict__ grad, int K,
     UpdateConsts c, float* __restrict__ mom1, float* __restrict__ mom2, PhiloxKeys keys,
     uint32_t step_lo, uint32_t step_hi, float* __restrict__ gmag, float* __restrict__ g_m,
@@ -268,16 +341,14 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
   __shared__ volatile int s_abort;
   const int n = gridDim.x - 1 - blockIdx.x;  // rows from the last, as the staged kernel
   const int t = threadIdx.x;
-  const int T = blockDim.x;  // multiple of 32, L .. 256
+  const int T = blockDim.x;  // multiple of 32, L .. 256 (.. 384 with MS)
   const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
   const int ngroups = K >> 4, nch = K >> 2;
   const int64_t row = static_cast<int64_t>(n) * K;
   const bool adam = c.kind == QL_ADAMW;
   const uint32_t qbytes = static_cast<uint32_t>(K), fbytes = 4u * static_cast<uint32_t>(K);
-  // Only the codes and the gradient are staged (the reductions need them
-  // whole); the moments stream through registers in the elementwise step, so
-  // a row takes 5 bytes of shared memory per element and several rows share
-  // an SM.
+  // The codes and the gradient are staged (the reductions need them whole),
+  // with MS the moments too.
   const uint32_t bar = smem_u32(&s_full);
   griddep_wait();  // the gradient (an earlier kernel's output) is visible from here
   if (t == 0) {
@@ -285,9 +356,13 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
     s_abort = 0;
     fence_mbar_init();
     const uint32_t dst = smem_u32(smem);
-    mbar_arrive_expect_tx(bar, qbytes + fbytes);
+    mbar_arrive_expect_tx(bar, qbytes + fbytes * (MS ? 3u : 1u));
     bulk_load(dst, wq + row, qbytes, bar);
     bulk_load(dst + qbytes, grad + row, fbytes, bar);
+    if (MS) {
+      bulk_load(dst + qbytes + fbytes, mom1 + row, fbytes, bar);
+      bulk_load(dst + qbytes + 2 * fbytes, mom2 + row, fbytes, bar);
+    }
   }
   const float s = sw[n];
   const float gmag_n = gmag[n];  // read before thread 0 overwrites it
@@ -389,55 +464,73 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
   float4* v_out = reinterpret_cast<float4*>(mom2 + row);
   float amax = 0.0f;
   int bad = 0;
-  // Four chunks per pass, their moment loads issued together.
-  constexpr int U = 4;
-  for (int ch0 = t; ch0 < nch; ch0 += U * T) {
-    float4 ma[U], va[U];
+  auto update_chunk = [&](int ch, float (&m1)[4], float (&m2)[4]) {
+    const uint32_t q4 = q_s[ch];
+    const float4 g4 = g_s[ch];
+    const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
+    float w[4], gg[4], wv[4], dd[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float qhat = s_qhat[static_cast<int>(static_cast<int8_t>(q4 >> (8 * e))) + 128];
+      dd[e] = __fsub_rn(gr[e], __fmul_rn(dg, qhat));
+    }
+    // coef * (g - dg * qhat) and s * q, two at a time (both are multiplied next)
+    const float2 cc = make_float2(coef, coef);
+    const float2 g01 = mul2(cc, make_float2(dd[0], dd[1])), g23 = mul2(cc, make_float2(dd[2], dd[3]));
+    gg[0] = g01.x; gg[1] = g01.y; gg[2] = g23.x; gg[3] = g23.y;
     if (adam) {
+      dequant4(q4, s, wv);
+      adamw4(c, wv, gg, m1, m2, w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = __fsub_rn(__fmul_rn(s, code_byte_f(q4, e)), __fmul_rn(c.lr, gg[e]));
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      bad |= !finite(w[e]);
+      amax = fmaxf(amax, fabsf(w[e]));
+    }
+    if (adam) {
+      __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
+      __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
+    }
+    g_s[ch] = make_float4(w[0], w[1], w[2], w[3]);
+  };
+  if (MS) {
+    const float4* m_s = reinterpret_cast<const float4*>(smem + qbytes + fbytes);
+    const float4* v_s = reinterpret_cast<const float4*>(smem + qbytes + 2 * fbytes);
+    for (int ch = t; ch < nch; ch += T) {
+      const float4 m4 = m_s[ch], v4 = v_s[ch];
+      float m1[4] = {m4.x, m4.y, m4.z, m4.w};
+      float m2[4] = {v4.x, v4.y, v4.z, v4.w};
+      update_chunk(ch, m1, m2);
+    }
+  } else {
+    // U chunks per pass, their moment loads issued together.
+    for (int ch0 = t; ch0 < nch; ch0 += U * T) {
+      float4 ma[U], va[U];
+      if (adam) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int ch = ch0 + u * T;
+          if (ch < nch) {
+            ma[u] = __ldcs(m_out + ch);
+            va[u] = __ldcs(v_out + ch);
+          }
+        }
+      }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int ch = ch0 + u * T;
-        if (ch < nch) {
-          ma[u] = __ldcs(m_out + ch);
-          va[u] = __ldcs(v_out + ch);
+        if (ch >= nch) break;
+        float m1[4], m2[4];
+        if (adam) {
+          m1[0] = ma[u].x; m1[1] = ma[u].y; m1[2] = ma[u].z; m1[3] = ma[u].w;
+          m2[0] = va[u].x; m2[1] = va[u].y; m2[2] = va[u].z; m2[3] = va[u].w;
         }
+        update_chunk(ch, m1, m2);
       }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int ch = ch0 + u * T;
-      if (ch >= nch) break;
-      const uint32_t q4 = q_s[ch];
-      const float4 g4 = g_s[ch];
-      const float gr[4] = {g4.x, g4.y, g4.z, g4.w};
-      float m1[4], m2[4];
-      if (adam) {
-        m1[0] = ma[u].x; m1[1] = ma[u].y; m1[2] = ma[u].z; m1[3] = ma[u].w;
-        m2[0] = va[u].x; m2[1] = va[u].y; m2[2] = va[u].z; m2[3] = va[u].w;
-      }
-      float w[4], gg[4], wv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float qhat = s_qhat[static_cast<int>(static_cast<int8_t>(q4 >> (8 * e))) + 128];
-        gg[e] = coef * (gr[e] - dg * qhat);
-        wv[e] = s * code_byte_f(q4, e);
-      }
-      if (adam) {
-        adamw4(c, wv, gg, m1, m2, w);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = wv[e] - c.lr * gg[e];
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        bad |= !finite(w[e]);
-        amax = fmaxf(amax, fabsf(w[e]));
-      }
-      if (adam) {
-        __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
-        __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
-      }
-      g_s[ch] = make_float4(w[0], w[1], w[2], w[3]);
     }
   }
   if (t == 0) {
@@ -485,8 +578,7 @@ __global__ void __launch_bounds__(256) update_sr_wn_staged_kernel(
     const float4 w = g_s[ch];
     uint32_t out = 0;
     if (amax != 0.0f)
-      out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
-                       sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+      out = sr_codes4(w, inv, rn);
     __stcs(q_out + ch, out);
   }
 }
@@ -622,8 +714,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
           float m1[4] = {m4.x, m4.y, m4.z, m4.w};
           float m2[4] = {v4.x, v4.y, v4.z, v4.w};
           float wv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) wv[e] = s * code_byte_f(q4, e);
+          dequant4(q4, s, wv);
           adamw4(c, wv, gr, m1, m2, w);
           __stcs(m_out + c0 + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
           __stcs(v_out + c0 + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
@@ -663,8 +754,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
       const float4 w = parked[ch];
       uint32_t out = 0;
       if (mbits != 0)
-        out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
-                         sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+        out = sr_codes4(w, inv, rn);
       __stcs(q_out + ch, out);
     }
     // s_max and the parked row are rewritten by the next row.
@@ -727,8 +817,7 @@ __global__ void __launch_bounds__(512) update_sr_dir_kernel(
     const float4 w = s_w[ch];
     uint32_t out = 0;
     if (mbits != 0)
-      out = pack_codes(sr_code_bits(w.x * inv, rn.x >> 8), sr_code_bits(w.y * inv, rn.y >> 8),
-                       sr_code_bits(w.z * inv, rn.z >> 8), sr_code_bits(w.w * inv, rn.w >> 8));
+      out = sr_codes4(w, inv, rn);
     __stcs(q_out + ch, out);
   }
 }
@@ -755,34 +844,48 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
   const unsigned grid = static_cast<unsigned>(N);
   if (g != nullptr) {
     // Weight norm: the row's codes and gradient staged (5 bytes per
-    // element, every K <= 32768 fits), at most 256 threads, of which the
-    // first L are the pinned reduction's virtual lanes.
-    const int64_t row_bytes = 5 * K;
-    static bool wn_set[64] = {false};
+    // element, every K <= 32768 fits), and with AdamW the moments too when
+    // three such rows fit an SM (13 bytes per element, K up to ~5.6K); at
+    // most 256 threads (384 with the moments staged), of which the first L
+    // are the pinned reduction's virtual lanes.
+    const int nch = static_cast<int>(K / 4);
+    const int64_t full_bytes = 13 * K;
+    // (an SM has 1 KB more shared memory than one CTA may take; 4 KB covers
+    // the kernel's static arrays and the per-CTA reserve)
+    const bool ms = c.kind == QL_ADAMW &&
+                    3 * (full_bytes + 4096) <= device_info().smem_optin + 1024;
+    // Streamed moments: one chunk ahead while four rows fit an SM, four
+    // chunks ahead otherwise.
+    const bool u1 = 4 * (5 * K + 4096) <= device_info().smem_optin + 1024;
+    const int variant = ms ? 0 : (u1 ? 1 : 2);
+    const int64_t row_bytes = ms ? full_bytes : 5 * K;
+    static bool wn_set[3][64] = {{false}};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !__atomic_load_n(&wn_set[dev], __ATOMIC_ACQUIRE)) {
+    auto kern = variant == 0 ? update_sr_wn_staged_kernel<true, 1>
+                : variant == 1 ? update_sr_wn_staged_kernel<false, 1>
+                               : update_sr_wn_staged_kernel<false, 4>;
+    if (dev < 64 && !__atomic_load_n(&wn_set[variant][dev], __ATOMIC_ACQUIRE)) {
       cudaFuncAttributes fa{};
-      e = cudaFuncGetAttributes(&fa, update_sr_wn_staged_kernel);
+      e = cudaFuncGetAttributes(&fa, kern);
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(update_sr_wn_staged_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  device_info().smem_optin - static_cast<int>(fa.sharedSizeBytes));
       if (e != cudaSuccess) {
         (void)cudaGetLastError();  // returned here; not left for a later check
         return e;
       }
-      __atomic_store_n(&wn_set[dev], true, __ATOMIC_RELEASE);
+      __atomic_store_n(&wn_set[variant][dev], true, __ATOMIC_RELEASE);
     }
     PhiloxKeys keys;
     for (int r = 0; r < 10; ++r) {
       keys.k0[r] = sl + static_cast<uint32_t>(r) * 0x9E3779B9u;
       keys.k1[r] = sh + static_cast<uint32_t>(r) * 0xBB67AE85u;
     }
-    const int nch = static_cast<int>(K / 4);
-    const int tr = std::max(T, std::min(256, std::max(32, (nch / QL_UPDATE_STAGED_CHUNKS + 31) / 32 * 32)));
-    e = launch_pdl(update_sr_wn_staged_kernel, dim3(grid), dim3(tr), static_cast<size_t>(row_bytes),
-                   s, wq, sw, grad, k, c, m, v, keys, tl, th, g, g_m, g_v, T, status);
+    const int tmax = ms ? 384 : 256;
+    const int tr = std::max(T, std::min(tmax, std::max(32, (nch / QL_UPDATE_STAGED_CHUNKS + 31) / 32 * 32)));
+    e = launch_pdl(kern, dim3(grid), dim3(tr), static_cast<size_t>(row_bytes), s, wq, sw, grad, k,
+                   c, m, v, keys, tl, th, g, g_m, g_v, T, status);
     count_launches(1);
     return e == cudaSuccess ? cudaGetLastError() : e;
   } else {
