@@ -75,7 +75,7 @@ def parse_args():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--e2e-steps", type=int, default=60)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--routes", action="store_true",
                    help="instead of the train step: time the forward's int8 and bf16 routes "
@@ -263,6 +263,36 @@ class Layer:
         if update_events:
             update_events[1].record()
 
+    def copy_floor(self, reps=5):
+        """Device time of one step's copies alone: X and dY in and y and dX out
+        at once, on two streams, from and to the same pinned buffers (the
+        PCIe bound of run_e2e)."""
+        torch = self.torch
+        s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def once():
+            cur = torch.cuda.current_stream()
+            s1.wait_stream(cur)
+            s2.wait_stream(cur)
+            with torch.cuda.stream(s1):
+                self.x.copy_(self.x_host, non_blocking=True)
+                self.dy.copy_(self.dy_host, non_blocking=True)
+            with torch.cuda.stream(s2):
+                self.y_host.copy_(self.y, non_blocking=True)
+                self.dx_host.copy_(self.dx, non_blocking=True)
+            cur.wait_stream(s1)
+            cur.wait_stream(s2)
+
+        once()
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            once()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
     def run_e2e(self, steps):
         """`steps` layer steps through the public API with host buffers: each
         step copies its X and dY in from pinned host memory and its y and dX
@@ -366,6 +396,7 @@ def run_ours(args, rank, world, local):
     layer.run_e2e(2)
     barrier(world)
     e2e_ms = max_over_ranks(layer.run_e2e(e2e_steps), world) / e2e_steps
+    copy_ms = layer.copy_floor()
     word = int(layer.status.item())
     if word:
         raise RuntimeError(f"device status {ql.status_flags(word)}")
@@ -443,7 +474,8 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": round(job_tops(world, 1, e2e_ms), 2), "unit": "TOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,
-                "overlap": "copies in, step, copies out on three streams, two buffer sets"},
+                "overlap": "copies in, step, copies out on three streams, two buffer sets",
+                "copies_alone_ms": round(copy_ms, 4)},
         "gpu_launches": int(launches),
         "clocks": clk,
     }
