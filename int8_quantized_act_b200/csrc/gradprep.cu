@@ -264,16 +264,32 @@ __global__ void __launch_bounds__(kThreads) colstats_tma_kernel(
   if (tid == 0 && s_abort) atomicOr(status, 1 << QL_ERR_TIMEOUT);
 }
 
+// 127/amax and amax/127 of a maximum kept as float bits (0 for a zero maximum).
+__device__ __forceinline__ float inv_of(uint32_t bits) {
+  const float amax = __uint_as_float(bits);
+  return amax == 0.0f ? 0.0f : 127.0f / amax;
+}
+__device__ __forceinline__ float scale_of(uint32_t bits) {
+  const float amax = __uint_as_float(bits);
+  return amax == 0.0f ? 0.0f : amax / 127.0f;
+}
+
 // Pass 2: q2[m,n] = rne((dY*rs2[m]) * cinv2[n]) and, with Q1,
-// q1[m,n] = rne((dY*cs1[n]) * rinv1[m]).  Each CTA walks its tiles in the
-// reverse of pass 1's order, so it starts on the tiles pass 1 read last,
-// which are the likeliest to be still in L2.
+// q1[m,n] = rne((dY*cs1[n]) * rinv1[m]), where cinv2 = 127/colmax and
+// rinv1 = 127/rowmax come straight from pass 1's maxima (IEEE divisions, a
+// few per CTA and tile).  The scales the GEMM epilogues need are written
+// here too, each by one CTA: s2 = colmax/127 and db (the column sums) by
+// the first row group, s1 = rowmax/127 by the first column block.  Each CTA
+// walks its tiles in the reverse of pass 1's order, so it starts on the
+// tiles pass 1 read last, which are the likeliest to be still in L2.
 template <typename InT, bool Q1>
 __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
     const __grid_constant__ CUtensorMap tm, int64_t M, int N, const float* __restrict__ cs1,
-    const float* __restrict__ rinv1, const float* __restrict__ rs2,
-    const float* __restrict__ cinv2, int8_t* __restrict__ q1, int8_t* __restrict__ q2,
-    int32_t* __restrict__ status, int tiles_per_cta) {
+    const float* __restrict__ rs2, const uint32_t* __restrict__ colmax,
+    const double* __restrict__ colsum, const uint32_t* __restrict__ rowmax,
+    float* __restrict__ s1, float* __restrict__ s2, float* __restrict__ db,
+    int8_t* __restrict__ q1, int8_t* __restrict__ q2, int32_t* __restrict__ status,
+    int tiles_per_cta) {
   using T = Tile<InT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* buf = reinterpret_cast<uint8_t*>(
@@ -284,7 +300,7 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   ring.init(tid);
   __syncthreads();
-  griddep_wait();  // dY and the factors (earlier kernels' outputs) are visible from here
+  griddep_wait();  // dY and the maxima (earlier kernels' outputs) are visible from here
   const int cb = blockIdx.x;
   const int tiles = static_cast<int>((M + T::kRows - 1) / T::kRows);
   const int t0 = blockIdx.y * tiles_per_cta;
@@ -303,7 +319,24 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
   } else {
     float w8[8] = {0, 0, 0, 0, 0, 0, 0, 0}, iv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (cv) {
-      load8(cinv2 + col, iv);
+      const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(colmax + col));
+      const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(colmax + col + 4));
+      const uint32_t cm[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) iv[i] = inv_of(cm[i]);
+      if (blockIdx.y == 0 && warp < kSub) {  // one writer per column
+        float sc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sc[i] = scale_of(cm[i]);
+        reinterpret_cast<float4*>(s2 + col)[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+        reinterpret_cast<float4*>(s2 + col)[1] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+        if (db) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sc[i] = static_cast<float>(colsum[col + i]);
+          reinterpret_cast<float4*>(db + col)[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+          reinterpret_cast<float4*>(db + col)[1] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+        }
+      }
       if (Q1) load8(cs1 + col, w8);
     }
     // Lane j < kRowsPerWarp holds the factors of row j of this warp's rows;
@@ -315,7 +348,12 @@ __global__ void __launch_bounds__(kThreads) dualquant_tma_kernel(
       const int64_t m = static_cast<int64_t>(t) * T::kRows + rw0 + lane;
       const bool in = lane < RW && t >= t0 && t < t1 && m < M;
       f2 = in ? __ldg(rs2 + m) : 0.0f;
-      r1 = (Q1 && in) ? __ldg(rinv1 + m) : 0.0f;
+      r1 = 0.0f;
+      if (Q1 && in) {
+        const uint32_t rb = __ldg(rowmax + m);
+        r1 = inv_of(rb);
+        if (cb == 0 && sub == 0) s1[m] = scale_of(rb);  // one writer per row
+      }
     };
     float f2cur, r1cur;
     load_rows(t1 - 1, f2cur, r1cur);
@@ -428,9 +466,10 @@ cudaError_t colstats_t(const void* dy, int64_t M, int64_t N, const float* sx, ui
 }
 
 template <typename InT>
-cudaError_t dualquant_t(const void* dy, int64_t M, int64_t N, const float* cs1,
-                        const float* rinv1, const float* rs2, const float* cinv2, int8_t* q1,
-                        int8_t* q2, int32_t* status, cudaStream_t s) {
+cudaError_t dualquant_t(const void* dy, int64_t M, int64_t N, const float* cs1, const float* rs2,
+                        const uint32_t* colmax, const double* colsum, const uint32_t* rowmax,
+                        float* s1, float* s2, float* db, int8_t* q1, int8_t* q2,
+                        int32_t* status, cudaStream_t s) {
   CUtensorMap tm;
   if (!dy_map<InT>(&tm, dy, M, N)) return cudaErrorInvalidValue;
   const Grid g = plan(M, N, Tile<InT>::kRows, 2);
@@ -438,11 +477,13 @@ cudaError_t dualquant_t(const void* dy, int64_t M, int64_t N, const float* cs1,
   if (q1) {
     allow_smem<dualquant_tma_kernel<InT, true>>();
     e = launch_pdl(dualquant_tma_kernel<InT, true>, g.grid, dim3(kThreads), kSmemBytes, s, tm, M,
-                   static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
+                   static_cast<int>(N), cs1, rs2, colmax, colsum, rowmax, s1, s2, db, q1, q2,
+                   status, g.tiles_per_cta);
   } else {
     allow_smem<dualquant_tma_kernel<InT, false>>();
     e = launch_pdl(dualquant_tma_kernel<InT, false>, g.grid, dim3(kThreads), kSmemBytes, s, tm, M,
-                   static_cast<int>(N), cs1, rinv1, rs2, cinv2, q1, q2, status, g.tiles_per_cta);
+                   static_cast<int>(N), cs1, rs2, colmax, colsum, rowmax, s1, s2, db, q1, q2,
+                   status, g.tiles_per_cta);
   }
   count_launches(1);
   return e == cudaSuccess ? cudaGetLastError() : e;
@@ -459,11 +500,14 @@ cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const
 }
 
 cudaError_t launch_dualquant(const void* dy, int dyt, int64_t M, int64_t N, const float* cs1,
-                             const float* rinv1, const float* rs2, const float* cinv2,
-                             int8_t* q1, int8_t* q2, int32_t* status, cudaStream_t s) {
+                             const float* rs2, const uint32_t* colmax, const double* colsum,
+                             const uint32_t* rowmax, float* s1, float* s2, float* db, int8_t* q1,
+                             int8_t* q2, int32_t* status, cudaStream_t s) {
   if (dyt == QL_BF16)
-    return dualquant_t<__nv_bfloat16>(dy, M, N, cs1, rinv1, rs2, cinv2, q1, q2, status, s);
-  return dualquant_t<float>(dy, M, N, cs1, rinv1, rs2, cinv2, q1, q2, status, s);
+    return dualquant_t<__nv_bfloat16>(dy, M, N, cs1, rs2, colmax, colsum, rowmax, s1, s2, db, q1,
+                                      q2, status, s);
+  return dualquant_t<float>(dy, M, N, cs1, rs2, colmax, colsum, rowmax, s1, s2, db, q1, q2,
+                            status, s);
 }
 
 }  // namespace ql

@@ -95,26 +95,19 @@ cudaError_t launch_colstats(const void* dy, int dyt, int64_t M, int64_t N, const
                             uint32_t* colmax, double* colsum, const float* sw, uint32_t* rowmax,
                             int32_t* status, cudaStream_t s);
 
-// s1[m] = amax/127, inv1[m] = 127/amax of the row maxima (0 for a zero row).
 // Zero colmax [N], colsum [N] and (if rowmax != NULL) rowmax [M] in one launch.
 cudaError_t launch_zero_stats(uint32_t* colmax, double* colsum, int64_t N, uint32_t* rowmax,
                               int64_t M, cudaStream_t s);
-// s2 = colmax/127, inv2 = 127/colmax, db = colsum (if db) for the N columns and
-// s1 = rowmax/127, inv1 = 127/rowmax for the M rows (M = 0: columns only), in one
-// launch; a zero maximum gives 0 for both.
-cudaError_t launch_finalize_both(const uint32_t* colmax, const double* colsum, int64_t N,
-                                 float* s2, float* inv2, float* db, const uint32_t* rowmax,
-                                 int64_t M, float* s1, float* inv1, cudaStream_t s);
 
-
-// q2 = rne((dY*rs2[m])*cinv2[n]) and, if q1 != NULL, q1 = rne((dY*cs1[n])*rinv1[m]),
-// both [M,N] (dY streamed through shared memory by TMA).
+// From the statistics pass's maxima (float bits; a zero maximum gives zero
+// factors and scales): q2 = rne((dY*rs2[m]) * (127/colmax[n])) and, if
+// q1 != NULL, q1 = rne((dY*cs1[n]) * (127/rowmax[m])), both [M,N] (dY streamed
+// through shared memory by TMA); also s2 = colmax/127, db = colsum (if db)
+// and, with q1, s1 = rowmax/127.
 cudaError_t launch_dualquant(const void* dy, int dyt, int64_t M, int64_t N, const float* cs1,
-                             const float* rinv1, const float* rs2, const float* cinv2,
-                             int8_t* q1, int8_t* q2, int32_t* status, cudaStream_t s);
-
-// s2[n] = amax/127, inv2[n] = 127/amax (0 for a zero column), db[n] = colsum.
-
+                             const float* rs2, const uint32_t* colmax, const double* colsum,
+                             const uint32_t* rowmax, float* s1, float* s2, float* db, int8_t* q1,
+                             int8_t* q2, int32_t* status, cudaStream_t s);
 
 // out[r, :] = bias (or 0), dtype ot; used when the contraction is empty.
 cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, const float* bias,

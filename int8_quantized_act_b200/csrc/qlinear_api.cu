@@ -78,7 +78,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 // Workspace carve-up shared by the two backward calls.
 struct WsLayout {
-  size_t dyq, s1, colmax, s2, inv2, colsum, dxtmp, parts, parts_elems, total;
+  size_t dyq, s1, colmax, s2, colsum, dxtmp, parts, parts_elems, total;
 };
 
 // Contractions longer than the int32-safe 131,071 (the input gradient's over
@@ -98,7 +98,6 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int B) {
   L.s1 = off;     off += align256(4 * (M > 0 ? m : 1));
   L.colmax = off; off += align256(4 * (N > 0 ? n : 1));
   L.s2 = off;     off += align256(4 * (N > 0 ? n : 1));
-  L.inv2 = off;   off += align256(4 * (N > 0 ? n : 1));
   L.colsum = off; off += align256(8 * (N > 0 ? n : 1));
   L.dxtmp = off;
   if (B > 128 || (dx_splits > 0 && B > 0)) off += align256(4 * m * k);
@@ -452,24 +451,22 @@ int qlinear_bwd_dw(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* 
   uint32_t* colmax = at<uint32_t>(ws, L.colmax);
   double* colsum = at<double>(ws, L.colsum);
   float* s2 = at<float>(ws, L.s2);
-  float* inv2 = at<float>(ws, L.inv2);
   int8_t* dyq = at<int8_t>(ws, L.dyq);
   if (ql::launch_zero_stats(colmax, colsum, N, nullptr, 0, s) != cudaSuccess) return QL_ERR_CUDA;
   cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, nullptr, nullptr,
                                       d_status, s);
   if (e == cudaSuccess)
-    e = ql::launch_finalize_both(colmax, colsum, N, s2, inv2, db, nullptr, 0, nullptr, nullptr, s);
-  if (e == cudaSuccess)
-    e = ql::launch_dualquant(dy, dyt, M, N, nullptr, nullptr, sx, inv2, nullptr, dyq, d_status, s);
+    e = ql::launch_dualquant(dy, dyt, M, N, nullptr, sx, colmax, colsum, nullptr, nullptr, s2, db,
+                             nullptr, dyq, d_status, s);
   if (e != cudaSuccess || K == 0) return cuda_status(e);
   return run_dw_product(dyq, xq, s2, M, N, K, dw, ws, L, d_status, s);
 }
 
 // qlinear_bwd's workspace: the common layout, then the column-quantized
-// codes [M*N], the row maxima [M] and 127/row max [M].
+// codes [M*N] and the row maxima [M].
 size_t bwd_extra(int64_t M, int64_t N) {
   return align256(static_cast<size_t>(M) * static_cast<size_t>(N)) +
-         2 * align256(4 * static_cast<size_t>(M > 0 ? M : 1));
+         align256(4 * static_cast<size_t>(M > 0 ? M : 1));
 }
 
 size_t qlinear_bwd_workspace_bytes(int64_t M, int64_t N, int64_t K, int hadamard_block) {
@@ -509,20 +506,17 @@ int qlinear_bwd(const void* dy, int dyt, int64_t M, int64_t N, const int8_t* wq,
   int8_t* dyq_c = at<int8_t>(ws, L.total);
   const size_t rm_off = L.total + align256(static_cast<size_t>(M) * static_cast<size_t>(N));
   uint32_t* rowmax = at<uint32_t>(ws, rm_off);
-  float* inv1 = at<float>(ws, rm_off + align256(4 * static_cast<size_t>(M)));
   float* s1 = at<float>(ws, L.s1);
   uint32_t* colmax = at<uint32_t>(ws, L.colmax);
   double* colsum = at<double>(ws, L.colsum);
   float* s2 = at<float>(ws, L.s2);
-  float* inv2 = at<float>(ws, L.inv2);
   // Pass 1 over dY: column maxima of |dY*s_x| and column sums, row maxima of
-  // |dY*s_w|; pass 2: both code sets, elementwise.
+  // |dY*s_w|; pass 2: the scales and both code sets, elementwise.
   if (ql::launch_zero_stats(colmax, colsum, N, rowmax, M, s) != cudaSuccess) return QL_ERR_CUDA;
   cudaError_t e = ql::launch_colstats(dy, dyt, M, N, sx, colmax, colsum, sw, rowmax, d_status, s);
   if (e == cudaSuccess)
-    e = ql::launch_finalize_both(colmax, colsum, N, s2, inv2, db, rowmax, M, s1, inv1, s);
-  if (e == cudaSuccess)
-    e = ql::launch_dualquant(dy, dyt, M, N, sw, inv1, sx, inv2, dyq_r, dyq_c, d_status, s);
+    e = ql::launch_dualquant(dy, dyt, M, N, sw, sx, colmax, colsum, rowmax, s1, s2, db, dyq_r,
+                             dyq_c, d_status, s);
   if (e != cudaSuccess) return QL_ERR_CUDA;
   // Input gradient (as qlinear_bwd_dx after its quantization), then weight
   // gradient (as qlinear_bwd_dw after its quantization).

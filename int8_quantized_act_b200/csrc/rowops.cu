@@ -512,28 +512,6 @@ __global__ void zero_stats_kernel(uint32_t* __restrict__ colmax, double* __restr
   }
 }
 
-// Scales from the statistics: threads [0, N) turn the column maxima and sums
-// into s2, 127/amax and db; threads [N, N + M) the row maxima into s1, 127/amax.
-__global__ void finalize_both_kernel(const uint32_t* __restrict__ colmax,
-                                     const double* __restrict__ colsum, int64_t N, float* s2,
-                                     float* inv2, float* db, const uint32_t* __restrict__ rowmax,
-                                     int64_t M, float* s1, float* inv1) {
-  griddep_wait();
-  griddep_launch_dependents();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < N) {
-    const float amax = __uint_as_float(colmax[i]);
-    s2[i] = amax == 0.0f ? 0.0f : amax / 127.0f;
-    inv2[i] = amax == 0.0f ? 0.0f : 127.0f / amax;
-    if (db) db[i] = static_cast<float>(colsum[i]);
-  } else if (i < N + M) {
-    const float amax = __uint_as_float(rowmax[i - N]);
-    s1[i - N] = amax == 0.0f ? 0.0f : amax / 127.0f;
-    inv1[i - N] = amax == 0.0f ? 0.0f : 127.0f / amax;
-  }
-}
-
-
 template <typename OutT>
 __global__ void fill_rows_kernel(OutT* out, int64_t rows, int cols, const float* bias) {
   const int64_t total = rows * cols;
@@ -713,15 +691,6 @@ cudaError_t launch_zero_stats(uint32_t* colmax, double* colsum, int64_t N, uint3
   return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
-cudaError_t launch_finalize_both(const uint32_t* colmax, const double* colsum, int64_t N,
-                                 float* s2, float* inv2, float* db, const uint32_t* rowmax,
-                                 int64_t M, float* s1, float* inv1, cudaStream_t s) {
-  const cudaError_t e = launch_pdl(finalize_both_kernel, dim3(static_cast<unsigned>((N + M + 255) / 256)),
-                                   dim3(256), 0, s, colmax, colsum, N, s2, inv2, db, rowmax, M, s1,
-                                   inv1);
-  count_launches(1);
-  return e == cudaSuccess ? cudaGetLastError() : e;
-}
 
 
 cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, const float* bias,

@@ -60,7 +60,7 @@ def test_workspace_formula(L):
     def a(x):
         return (x + 255) // 256 * 256
     M, N, K = 12000, 7168, 5376
-    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    base = a(M * N) + a(4 * M) + 2 * a(4 * N) + a(8 * N)
     assert ql.qlinear_workspace_bytes(M, N, K, 128) == base
     assert ql.qlinear_workspace_bytes(M, N, K, 256) == base + a(4 * M * K)
     assert ql.qlinear_workspace_bytes(-1, N, K, 0) == 0
@@ -82,19 +82,19 @@ def test_workspace_grows_by_the_int32_partials_of_long_contractions(L):
     # (200 tokens: more than one 128-row slab, so no extra small-output splits)
     M, K = 200, 256
     for N, splits in ((limit + 1, 2), (400000, 4)):
-        base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+        base = a(M * N) + a(4 * M) + 2 * a(4 * N) + a(8 * N)
         assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * splits * M * K)
         # rotated: the float32 product waits for its second pass
         assert ql.qlinear_workspace_bytes(M, N, K, 128) == base + a(4 * M * K) + a(4 * splits * M * K)
     M, N = 262144, 144         # 2048 blocks -> 3 splits over the tokens
-    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    base = a(M * N) + a(4 * M) + 2 * a(4 * N) + a(8 * N)
     assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 3 * N * K)
     # a small output takes the larger of the two split counts
     M, N = 262144, 48
-    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    base = a(M * N) + a(4 * M) + 2 * a(4 * N) + a(8 * N)
     assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 8 * N * K)
     M, N = 8, 1100000          # 8594 blocks -> 9 splits > 8
-    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    base = a(M * N) + a(4 * M) + 2 * a(4 * N) + a(8 * N)
     assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 9 * M * K)
 
 
@@ -104,11 +104,11 @@ def test_workspace_small_outputs_reserve_split_partials(L):
     def a(x):
         return (x + 255) // 256 * 256
     M, N, K = 17, 7168, 5376
-    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    base = a(M * N) + a(4 * M) + 2 * a(4 * N) + a(8 * N)
     assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 8 * M * K)
     assert ql.qlinear_workspace_bytes(M, N, K, 128) == base + a(4 * M * K) + a(4 * 8 * M * K)
     M, N = 4096, 64
-    base = a(M * N) + a(4 * M) + 3 * a(4 * N) + a(8 * N)
+    base = a(M * N) + a(4 * M) + 2 * a(4 * N) + a(8 * N)
     assert ql.qlinear_workspace_bytes(M, N, K, 0) == base + a(4 * 8 * N * K)
 
 
@@ -117,7 +117,7 @@ def test_bwd_workspace_formula(L):
         return (x + 255) // 256 * 256
     for (M, N, K, B) in ((12000, 7168, 5376, 128), (17, 144, 512, 256)):
         assert (ql.qlinear_bwd_workspace_bytes(M, N, K, B)
-                == ql.qlinear_workspace_bytes(M, N, K, B) + a(M * N) + 2 * a(4 * M))
+                == ql.qlinear_workspace_bytes(M, N, K, B) + a(M * N) + a(4 * M))
 
 
 def test_host_validation_returns_before_any_launch(L):
