@@ -76,6 +76,12 @@ struct Epi {
   const float* col_scale;
   const float* bias;
   float hc;
+  // The Newton-Schulz step in a bf16 kind::f16 epilogue (GemmEpilogue::ns_x);
+  // null: none.
+  const __nv_bfloat16* ns_x;
+  __nv_bfloat16* ns_xt;
+  int64_t ns_ldt;
+  float ns_a;
 };
 
 // Tile t of a tiles_m x tiles_n grid in grouped order: runs of `group`
@@ -209,6 +215,28 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
         }
       }
       if constexpr (HB > 0) fwht_regs<CH, HB>(v, ep.hc);
+      if constexpr (F16 && HB == 0 && !std::is_same<OutT, float>::value) {
+        // Newton-Schulz: x' = bf16(a*x + acc), x from the same position of X.
+        if (ep.ns_x) {
+          const __nv_bfloat16* xrow = ep.ns_x + static_cast<int64_t>(gr) * ep.ldo + gc0;
+#pragma unroll
+          for (int g = 0; g < CH / 16; ++g) {
+            if (gc0 + 16 * g < ep.cols) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const uint4 u = *reinterpret_cast<const uint4*>(xrow + 16 * g + 8 * h);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  float* d = v + 16 * g + 8 * h + 2 * k;
+                  d[0] = __fadd_rn(__fmul_rn(ep.ns_a, __uint_as_float(w[k] << 16)), d[0]);
+                  d[1] = __fadd_rn(__fmul_rn(ep.ns_a, __uint_as_float(w[k] & 0xFFFF0000u)), d[1]);
+                }
+              }
+            }
+          }
+        }
+      }
       if constexpr (std::is_same<OutT, float>::value && HB == 0) {
         (void)0;
       } else {
@@ -236,6 +264,34 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
                                          stage[rr * 33 + cc + 2], stage[rr * 33 + cc + 3]);
           if (rbase + rr < ep.rows && gc0 + cc < ep.cols)
             *reinterpret_cast<float4*>(out + static_cast<int64_t>(rbase + rr) * ep.ldo + gc0 + cc) = val;
+        }
+        __syncwarp();
+      }
+    }
+    if constexpr (F16 && HB == 0 && !std::is_same<OutT, float>::value) {
+      // The transposed copy of the Newton-Schulz step's x': through the
+      // padded stage, lane l writes column gc0 + l of the chunk as a 64-byte
+      // piece of row gc0 + l of ns_xt (the chunk's valid rows only, a
+      // multiple of 16).  Every lane takes part.
+      if (ep.ns_x && gc0 < ep.cols) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          stage[lane * 33 + e] = row_ok ? __bfloat162float(__float2bfloat16_rn(v[e])) : 0.0f;
+        __syncwarp();
+        const int rbase = row0 + quarter * 32;
+        const int nrows = min(32, ep.rows - rbase);
+        if (gc0 + lane < ep.cols && nrows > 0) {
+          __nv_bfloat16* trow = ep.ns_xt + static_cast<int64_t>(gc0 + lane) * ep.ns_ldt + rbase;
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            if (8 * q8 < nrows) {
+              uint32_t o[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                o[k] = bf16x2(stage[(8 * q8 + 2 * k) * 33 + lane], stage[(8 * q8 + 2 * k + 1) * 33 + lane]);
+              *reinterpret_cast<uint4*>(trow + 8 * q8) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
         }
         __syncwarp();
       }
@@ -985,7 +1041,7 @@ cudaError_t launch_gemm_i8(const int8_t* A, bool a_mn, int64_t lda, const int8_t
   const bool ok_b = b_mn ? make_tmap(&tb, B, cols, kc, ldb, 128, BK)
                          : make_tmap(&tb, B, kc, cols, ldb, BK, pair ? 128 : narrow ? 64 : BN);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
-  Epi ep;
+  Epi ep{};
   ep.out = e.out;
   ep.ldo = e.ldo;
   ep.split_stride = 0;
@@ -1034,7 +1090,7 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
                                    static_cast<uint64_t>(ldb) * 2, BK / 2,
                                    pair ? 128 : narrow ? 64 : BN, true);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
-  Epi ep;
+  Epi ep{};
   ep.out = e.out;
   ep.ldo = e.ldo;
   ep.split_stride = 0;
@@ -1049,6 +1105,19 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
   const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
   const int kblocks = static_cast<int>((kc + BK / 2 - 1) / (BK / 2));
   if (e.hb != 0) return cudaErrorInvalidValue;
+  if (e.ns_x) {
+    // The Newton-Schulz epilogue: bf16 output, 16-byte pieces of ns_x, out
+    // and ns_xt rows (pitches multiples of 8 elements, rows a multiple of 16).
+    if (!e.out_bf16 || !e.ns_xt || e.row_scale || e.col_scale || e.bias || (e.ldo % 8) != 0 ||
+        (e.ns_ldt % 8) != 0 || (rows % 16) != 0 || (cols % 16) != 0 ||
+        (reinterpret_cast<uintptr_t>(e.ns_x) & 15) || (reinterpret_cast<uintptr_t>(e.ns_xt) & 15) ||
+        (reinterpret_cast<uintptr_t>(e.out) & 15) || (upper_only && *upper_only))
+      return cudaErrorInvalidValue;
+    ep.ns_x = reinterpret_cast<const __nv_bfloat16*>(e.ns_x);
+    ep.ns_xt = reinterpret_cast<__nv_bfloat16*>(e.ns_xt);
+    ep.ns_ldt = e.ns_ldt;
+    ep.ns_a = e.ns_a;
+  }
   if (narrow) {
     const int tn64 = static_cast<int>((cols + 63) / 64);
     if (e.out_bf16)

@@ -9,9 +9,11 @@
 // The Newton-Schulz products run on the tcgen05 bf16 GEMM (float32
 // accumulation, bf16 operands as in the published method); X is kept in both
 // layouts so that every product reads K-major operands: A = X X^T from X and
-// X, A A = A A^T (A is symmetric), B X from B and X^T.  The elementwise steps
-// (momentum with ||U||^2, normalization, b A + c A A, a X + B X with its
-// transpose) are the kernels below; the requantization is update_sr.cu's.
+// X, A A = A A^T (A is symmetric), B X from B and X^T.  The step
+// X' = a X + B X and its transpose are written by the B X product's epilogue
+// (GemmEpilogue::ns_x); the other elementwise steps (momentum with ||U||^2,
+// normalization, b A + c A A) are the kernels below; the requantization is
+// update_sr.cu's.
 // The float parameters of MuonAuxAdamW (biases, magnitudes) take AdamW:
 // qadamw_vector.
 #include <cuda_bf16.h>
@@ -246,32 +248,6 @@ __global__ void __launch_bounds__(256) ns_combine_sym_kernel(const __nv_bfloat16
   }
 }
 
-// X' = bf16(a * X + P) for X [r, c] into Xo (X itself, or the output) and
-// its transpose X'^T [c, r] into Xt (transpose64: the thread that reads an
-// element of X writes it in Xo).
-__global__ void __launch_bounds__(256) ns_step_kernel(const __nv_bfloat16* X,
-                                                      __nv_bfloat16* Xo,
-                                                      const float* __restrict__ P, int64_t r,
-                                                      int64_t c, __nv_bfloat16* __restrict__ Xt) {
-  __shared__ __align__(16) __nv_bfloat16 tile[64][66];
-  const int64_t tiles_c = (c + 63) / 64, tiles = ((r + 63) / 64) * tiles_c;
-  auto load = [&](int64_t i, int64_t j, float (&v)[8]) {
-    const uint4 xv = *reinterpret_cast<const uint4*>(X + i * c + j);
-    float p[8];
-    load8f(P + i * c + j, p);
-    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[2 * k] = __fadd_rn(__fmul_rn(kNsA, __uint_as_float(xw[k] << 16)), p[2 * k]);
-      v[2 * k + 1] = __fadd_rn(__fmul_rn(kNsA, __uint_as_float(xw[k] & 0xFFFF0000u)), p[2 * k + 1]);
-    }
-  };
-  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-    const int64_t r0 = (t / tiles_c) * 64, c0 = (t % tiles_c) * 64;
-    transpose64(r, c, r0, c0, load, Xo, Xt, tile);
-  }
-}
-
 // The lower 256 x 256 tiles of a symmetric bf16 r x r matrix (r a multiple of 8)
 // from the upper ones (the symmetric GEMMs write only tiles with tile-row <=
 // tile-column): a[i][j] = a[j][i] where i / 256 > j / 256, by 64 x 64 blocks
@@ -357,10 +333,10 @@ MuonLayout muon_layout(int64_t N, int64_t K) {
   L.sumsq = off; off += 256;
   L.X = off;     off += a256(2 * r * c);
   L.Xt = off;    off += a256(2 * r * c);
+  L.Xt2 = off;   off += a256(2 * r * c);
   L.A = off;     off += a256(2 * r * r);
   L.A2 = off;    off += a256(4 * r * r);
   L.Bm = off;    off += a256(2 * r * r);
-  L.P = off;     off += a256(4 * r * c);
   L.total = off;
   return L;
 }
@@ -376,7 +352,8 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
   auto* A = reinterpret_cast<__nv_bfloat16*>(w + L.A);
   auto* A2 = reinterpret_cast<float*>(w + L.A2);
   auto* Bm = reinterpret_cast<__nv_bfloat16*>(w + L.Bm);
-  auto* P = reinterpret_cast<float*>(w + L.P);
+  __nv_bfloat16* xt_in = Xt;  // X^T as the B X product reads it
+  __nv_bfloat16* xt_out = reinterpret_cast<__nv_bfloat16*>(w + L.Xt2);
   const int64_t r = std::min(N, K), c = std::max(N, K);
   const float omb = static_cast<float>(1.0 - static_cast<double>(beta));
   cudaError_t e = cudaMemsetAsync(sumsq, 0, sizeof(double), s);
@@ -414,20 +391,26 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
       ns_combine_kernel<<<grid_for(r * r / 8, 8), 256, 0, s>>>(A, A2, r * r, Bm);
     }
     count_launches(1);
-    ep.out = P;
-    ep.ldo = c;
-    if ((e = launch_gemm_bf16(Bm, r, Xt, r, r, c, r, ep, status, s)) != cudaSuccess) return e;  // B X
-    // The last step writes the [N, K]-shaped layout (X^T when N > K) into O.
+    // X' = a X + B X in the product's epilogue: X' over X (in place: each
+    // element is read and written by the same thread, and X is not an
+    // operand of this product) and X'^T into the other X^T buffer (the one
+    // read here is the product's B operand).  The last step writes the
+    // [N, K]-shaped layout (X'^T when N > K) into O.
     __nv_bfloat16* xo = X;
-    __nv_bfloat16* xto = Xt;
+    __nv_bfloat16* xto = xt_out;
     if (it == steps - 1) {
       if (N > K) xto = reinterpret_cast<__nv_bfloat16*>(O);
       else xo = reinterpret_cast<__nv_bfloat16*>(O);
     }
-    ns_step_kernel<<<grid_for(((r + 63) / 64) * ((c + 63) / 64) * 256, 8), 256, 0, s>>>(
-        X, xo, P, r, c, xto);
-    count_launches(1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ep.out = xo;
+    ep.out_bf16 = 1;
+    ep.ldo = c;
+    ep.ns_x = X;
+    ep.ns_xt = xto;
+    ep.ns_ldt = r;
+    ep.ns_a = kNsA;
+    if ((e = launch_gemm_bf16(Bm, r, xt_in, r, r, c, r, ep, status, s)) != cudaSuccess) return e;  // B X
+    std::swap(xt_in, xt_out);
   }
   return cudaSuccess;
 }
