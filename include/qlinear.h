@@ -339,7 +339,7 @@ QL_API int qweight_update_sr(int8_t *wq, float *sw, const float *grad, int64_t N
  * accumulation on the tensor cores), so O matches the float64 iteration of
  * the same definition to bf16 accuracy, not bit for bit.  ws: at least
  * qweight_muon_workspace_bytes(N, K) bytes, 256-byte aligned (for N = 7168,
- * K = 5376 about 0.46 GB).  Requirements: N, K multiples of 16; 0 <= beta < 1;
+ * K = 5376 about 0.35 GB).  Requirements: N, K multiples of 16; 0 <= beta < 1;
  * 1 <= ns_steps <= 16; grad, mom, O 16-byte aligned. */
 QL_API size_t qweight_muon_workspace_bytes(int64_t N, int64_t K);
 QL_API int qweight_muon_orthogonalize(const float *grad, float *mom, int64_t N, int64_t K,

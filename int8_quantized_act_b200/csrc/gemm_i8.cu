@@ -76,12 +76,13 @@ struct Epi {
   const float* col_scale;
   const float* bias;
   float hc;
-  // The Newton-Schulz step in a bf16 kind::f16 epilogue (GemmEpilogue::ns_x);
-  // null: none.
+  // The Newton-Schulz steps in a bf16 kind::f16 epilogue (GemmEpilogue::ns_x,
+  // ns_mirror); null / 0: none.
   const __nv_bfloat16* ns_x;
   __nv_bfloat16* ns_xt;
   int64_t ns_ldt;
-  float ns_a;
+  float ns_a, ns_c;
+  int ns_mirror;
 };
 
 // Tile t of a tiles_m x tiles_n grid in grouped order: runs of `group`
@@ -216,7 +217,7 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
       }
       if constexpr (HB > 0) fwht_regs<CH, HB>(v, ep.hc);
       if constexpr (F16 && HB == 0 && !std::is_same<OutT, float>::value) {
-        // Newton-Schulz: x' = bf16(a*x + acc), x from the same position of X.
+        // Newton-Schulz: x' = bf16(a*x + c*acc), x from the same position of X.
         if (ep.ns_x) {
           const __nv_bfloat16* xrow = ep.ns_x + static_cast<int64_t>(gr) * ep.ldo + gc0;
 #pragma unroll
@@ -229,8 +230,10 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                   float* d = v + 16 * g + 8 * h + 2 * k;
-                  d[0] = __fadd_rn(__fmul_rn(ep.ns_a, __uint_as_float(w[k] << 16)), d[0]);
-                  d[1] = __fadd_rn(__fmul_rn(ep.ns_a, __uint_as_float(w[k] & 0xFFFF0000u)), d[1]);
+                  d[0] = __fadd_rn(__fmul_rn(ep.ns_a, __uint_as_float(w[k] << 16)),
+                                   __fmul_rn(ep.ns_c, d[0]));
+                  d[1] = __fadd_rn(__fmul_rn(ep.ns_a, __uint_as_float(w[k] & 0xFFFF0000u)),
+                                   __fmul_rn(ep.ns_c, d[1]));
                 }
               }
             }
@@ -269,11 +272,16 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
       }
     }
     if constexpr (F16 && HB == 0 && !std::is_same<OutT, float>::value) {
-      // The transposed copy of the Newton-Schulz step's x': through the
-      // padded stage, lane l writes column gc0 + l of the chunk as a 64-byte
-      // piece of row gc0 + l of ns_xt (the chunk's valid rows only, a
-      // multiple of 16).  Every lane takes part.
-      if (ep.ns_x && gc0 < ep.cols) {
+      // The transposed copy of the stored values: into ns_xt, or with
+      // ns_mirror (a symmetric product on its upper 256 x 256 tiles) into the
+      // output's lower tile, for a strictly upper tile.  Through the padded
+      // stage, lane l writes column gc0 + l of the chunk as a 64-byte piece of
+      // row gc0 + l of the target (the chunk's valid rows only, a multiple of
+      // 16).  Every lane takes part.
+      const bool mirror = ep.ns_mirror && row0 / 256 < col0 / 256;
+      __nv_bfloat16* tgt = mirror ? reinterpret_cast<__nv_bfloat16*>(ep.out) : ep.ns_xt;
+      const int64_t ldt = mirror ? ep.ldo : ep.ns_ldt;
+      if ((mirror || (ep.ns_x && ep.ns_xt)) && gc0 < ep.cols) {
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           stage[lane * 33 + e] = row_ok ? __bfloat162float(__float2bfloat16_rn(v[e])) : 0.0f;
@@ -281,7 +289,7 @@ __device__ __forceinline__ void epilogue_tile(const Epi& ep, uint32_t acc_tmem, 
         const int rbase = row0 + quarter * 32;
         const int nrows = min(32, ep.rows - rbase);
         if (gc0 + lane < ep.cols && nrows > 0) {
-          __nv_bfloat16* trow = ep.ns_xt + static_cast<int64_t>(gc0 + lane) * ep.ns_ldt + rbase;
+          __nv_bfloat16* trow = tgt + static_cast<int64_t>(gc0 + lane) * ldt + rbase;
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             if (8 * q8 < nrows) {
@@ -1105,20 +1113,25 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
   const int tiles_n = static_cast<int>((cols + BN - 1) / BN);
   const int kblocks = static_cast<int>((kc + BK / 2 - 1) / (BK / 2));
   if (e.hb != 0) return cudaErrorInvalidValue;
-  if (e.ns_x) {
+  if (e.ns_x || e.ns_xt || e.ns_mirror) {
     // The Newton-Schulz epilogue: bf16 output, 16-byte pieces of ns_x, out
-    // and ns_xt rows (pitches multiples of 8 elements, rows a multiple of 16).
-    if (!e.out_bf16 || !e.ns_xt || e.row_scale || e.col_scale || e.bias || (e.ldo % 8) != 0 ||
-        (e.ns_ldt % 8) != 0 || (rows % 16) != 0 || (cols % 16) != 0 ||
-        (reinterpret_cast<uintptr_t>(e.ns_x) & 15) || (reinterpret_cast<uintptr_t>(e.ns_xt) & 15) ||
-        (reinterpret_cast<uintptr_t>(e.out) & 15) || (upper_only && *upper_only))
+    // and ns_xt rows (pitches multiples of 8 elements, rows a multiple of 16);
+    // a transposed copy into ns_xt needs ns_x, ns_mirror a symmetric product.
+    if (!e.out_bf16 || e.row_scale || e.col_scale || e.bias || (e.ldo % 8) != 0 ||
+        (rows % 16) != 0 || (cols % 16) != 0 || (reinterpret_cast<uintptr_t>(e.out) & 15) ||
+        (e.ns_x && (reinterpret_cast<uintptr_t>(e.ns_x) & 15)) ||
+        (e.ns_xt && (!e.ns_x || e.ns_mirror || (e.ns_ldt % 8) != 0 ||
+                     (reinterpret_cast<uintptr_t>(e.ns_xt) & 15))) ||
+        (e.ns_mirror && !(upper_only && *upper_only)))
       return cudaErrorInvalidValue;
     ep.ns_x = reinterpret_cast<const __nv_bfloat16*>(e.ns_x);
     ep.ns_xt = reinterpret_cast<__nv_bfloat16*>(e.ns_xt);
     ep.ns_ldt = e.ns_ldt;
     ep.ns_a = e.ns_a;
+    ep.ns_c = e.ns_c;
   }
   if (narrow) {
+    if (upper_only) *upper_only = false;  // every tile is computed
     const int tn64 = static_cast<int>((cols + 63) / 64);
     if (e.out_bf16)
       return run<false, false, __nv_bfloat16, 0, true, 64>(ta, tb, tiles_m, tn64, kblocks, kblocks, ep, status, s);
@@ -1129,6 +1142,9 @@ cudaError_t launch_gemm_bf16(const void* A, int64_t lda, const void* B, int64_t 
   // *upper_only stays true to tell the caller to fill the lower ones.
   const bool upper = upper_only && *upper_only && pair && rows == cols;
   if (upper_only) *upper_only = upper;
+  // The lower tiles are mirrored only when the product runs on its upper
+  // tiles (otherwise every tile is computed).
+  ep.ns_mirror = e.ns_mirror && upper ? 1 : 0;
   if (e.out_bf16)
     return go<false, false, __nv_bfloat16, 0, true>(pair, ta, tb, tiles_m, tiles_n, kblocks, ep,
                                                    status, s, 0, upper);

@@ -116,10 +116,10 @@ cudaError_t launch_fill_rows(void* out, int ot, int64_t rows, int64_t cols, cons
 // -------------------------------------------------------------- MuonAuxAdamW
 // Workspace of the Newton-Schulz iteration for an [N, K] weight (r = min,
 // c = max of N, K): ||U||^2, X [r, c] bf16 and two buffers of X^T [c, r] bf16
-// (each step reads one and writes the other), A, B [r, r] bf16, A A [r, r]
-// float32; byte offsets, each 256-byte aligned.
+// (each step reads one and writes the other), A and B [r, r] bf16; byte
+// offsets, each 256-byte aligned.
 struct MuonLayout {
-  int64_t sumsq, X, Xt, Xt2, A, A2, Bm, total;
+  int64_t sumsq, X, Xt, Xt2, A, Bm, total;
 };
 MuonLayout muon_layout(int64_t N, int64_t K);
 // M <- beta*M + (1-beta)*G; O [N, K] bf16 <- NS(U) after `steps` (>= 1) steps.
@@ -157,16 +157,21 @@ struct GemmEpilogue {
   const float* bias = nullptr;
   int hb = 0;
   float hc = 1.0f;
-  // launch_gemm_bf16 only: the Newton-Schulz step X' = a*X + acc in the
-  // epilogue.  With ns_x set (bf16 [rows, cols], pitch ldo, the same as out;
-  // out may be ns_x itself), out = bf16(ns_a * x + acc), each operation
-  // rounded once, and the same values are written transposed into ns_xt
-  // ([cols, rows] bf16, pitch ns_ldt elements), which must not be an operand
-  // of the product.  No scales or bias; rows and cols multiples of 16.
+  // launch_gemm_bf16 only, bf16 output, no scales or bias, rows and cols
+  // multiples of 16: the elementwise Newton-Schulz steps in the epilogue.
+  // With ns_x set (bf16 [rows, cols], pitch ldo, the same as out; out may be
+  // ns_x itself): out = bf16(ns_a * x + ns_c * acc), each operation rounded
+  // once (ns_c = 1 multiplies exactly).  With ns_xt also set, the stored
+  // values are written transposed into ns_xt ([cols, rows] bf16, pitch
+  // ns_ldt elements), which must not be an operand of the product.  With
+  // ns_mirror (a symmetric product run with upper_only): each strictly upper
+  // tile's stored values are written transposed into its lower mirror tile
+  // of out, so out comes back complete.
   const void* ns_x = nullptr;
   void* ns_xt = nullptr;
   int64_t ns_ldt = 0;
-  float ns_a = 0.0f;
+  float ns_a = 0.0f, ns_c = 1.0f;
+  int ns_mirror = 0;
 };
 
 // A: rows x contraction, K-major ([rows][kc], pitch lda bytes) or MN-major

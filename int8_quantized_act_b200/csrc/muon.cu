@@ -119,24 +119,6 @@ __device__ __forceinline__ void load8f(const float* p, float (&v)[8]) {
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// 8 consecutive bf16 values as float32 and back (exact).
-__device__ __forceinline__ void load8v(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    v[2 * k] = __uint_as_float(w[k] << 16);
-    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-  }
-}
-__device__ __forceinline__ void store8v(__nv_bfloat16* p, const float (&v)[8]) {
-  uint32_t o[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    o[k] = (__float_as_uint(v[2 * k]) >> 16) | (__float_as_uint(v[2 * k + 1]) & 0xFFFF0000u);
-  *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
-}
-
 
 // X0 = bf16(U / (||U||_F + 1e-7)) with U recomputed from G and the new M
 // (the same float32 operations as muon_momentum_kernel), written as X [r, c]
@@ -163,133 +145,6 @@ __global__ void __launch_bounds__(256) ns_init_kernel(const float* __restrict__ 
     const int64_t r0 = (t / tiles_c) * 64, c0 = (t % tiles_c) * 64;
     // U [N, K] row-major; its transpose [K, N].  X is U or U^T.
     transpose64(N, K, r0, c0, load, tr ? Xt : X, tr ? X : Xt, tile);
-  }
-}
-
-// Bm = bf16(b * A + c * A2) elementwise (A bf16, A2 float32, both [r, r]),
-// 8 elements a thread-step (16-byte loads and stores; n is a multiple of 8).
-__global__ void __launch_bounds__(256) ns_combine_kernel(const __nv_bfloat16* __restrict__ A,
-                                                         const float* __restrict__ A2, int64_t n,
-                                                         __nv_bfloat16* __restrict__ Bm) {
-  const int64_t n8 = n / 8;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += stride) {
-    const uint4 a = reinterpret_cast<const uint4*>(A)[i];
-    const float4 p0 = reinterpret_cast<const float4*>(A2)[2 * i];
-    const float4 p1 = reinterpret_cast<const float4*>(A2)[2 * i + 1];
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-    const float a2[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float lo = __uint_as_float(aw[k] << 16), hi = __uint_as_float(aw[k] & 0xFFFF0000u);
-      const __nv_bfloat16 b0 = __float2bfloat16_rn(__fadd_rn(__fmul_rn(kNsB, lo), __fmul_rn(kNsC, a2[2 * k])));
-      const __nv_bfloat16 b1 = __float2bfloat16_rn(__fadd_rn(__fmul_rn(kNsB, hi), __fmul_rn(kNsC, a2[2 * k + 1])));
-      o[k] = static_cast<uint32_t>(__bfloat16_as_ushort(b0)) |
-             (static_cast<uint32_t>(__bfloat16_as_ushort(b1)) << 16);
-    }
-    reinterpret_cast<uint4*>(Bm)[i] = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-}
-
-// The same combination for a symmetric A whose square A2 holds only its
-// upper 256 x 256 tiles (tile-row <= tile-column): Bm is symmetric, so each
-// 64 x 64 block of the upper tiles is computed from A and A2 and written
-// both in place and, in a strictly upper tile, transposed into the lower
-// one (through a shared tile, rows padded to 65 floats); the same values as
-// combining the whole of a mirrored A2.
-__global__ void __launch_bounds__(256) ns_combine_sym_kernel(const __nv_bfloat16* __restrict__ A,
-                                                             const float* __restrict__ A2,
-                                                             int64_t r,
-                                                             __nv_bfloat16* __restrict__ Bm) {
-  __shared__ float tile[64][65];
-  const int t = threadIdx.x, tr = t >> 3, tc = (t & 7) * 8;
-  const int64_t nt = (r + 255) / 256;
-  const int64_t blocks = nt * (nt + 1) / 2 * 16;
-  for (int64_t b = blockIdx.x; b < blocks; b += gridDim.x) {
-    int64_t ti = 0, rem = b / 16;  // upper tile (ti, tj), tj >= ti, row by row
-    while (rem >= nt - ti) {
-      rem -= nt - ti;
-      ++ti;
-    }
-    const int64_t tj = ti + rem;
-    const int64_t I = ti * 4 + (b % 16) / 4, J = tj * 4 + (b % 4);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int lr = tr + 32 * h;
-      const int64_t i = I * 64 + lr, j = J * 64 + tc;
-      if (i < r && j < r) {
-        float a[8], a2[8], v[8];
-        load8v(A + i * r + j, a);
-        load8f(A2 + i * r + j, a2);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          v[k] = __bfloat162float(__float2bfloat16_rn(
-              __fadd_rn(__fmul_rn(kNsB, a[k]), __fmul_rn(kNsC, a2[k]))));
-          tile[lr][tc + k] = v[k];
-        }
-        store8v(Bm + i * r + j, v);
-      }
-    }
-    if (ti == tj) continue;  // uniform per CTA: a diagonal tile has no mirror image
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int lc = tr + 32 * h;
-      const int64_t i = J * 64 + lc, j = I * 64 + tc;  // the transposed block (J, I)
-      if (i < r && j < r) {
-        float v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = tile[tc + k][lc];
-        store8v(Bm + i * r + j, v);
-      }
-    }
-    __syncthreads();
-  }
-}
-
-// The lower 256 x 256 tiles of a symmetric bf16 r x r matrix (r a multiple of 8)
-// from the upper ones (the symmetric GEMMs write only tiles with tile-row <=
-// tile-column): a[i][j] = a[j][i] where i / 256 > j / 256, by 64 x 64 blocks
-// of the lower tiles only: 16-byte loads of the source block's rows into a
-// shared tile (rows padded to 65 floats), 16-byte stores of the destination's
-// rows gathered from its columns.
-__global__ void __launch_bounds__(256) ns_mirror_kernel(__nv_bfloat16* __restrict__ a, int64_t r) {
-  __shared__ float tile[64][65];
-  const int t = threadIdx.x, tr = t >> 3, tc = (t & 7) * 8;
-  const int64_t nt = (r + 255) / 256;  // 256-tiles a side
-  const int64_t blocks = nt * (nt - 1) / 2 * 16;
-  for (int64_t b = blockIdx.x; b < blocks; b += gridDim.x) {
-    int64_t ti = 1, rem = b / 16;  // lower tile (ti, tj), tj < ti, row by row
-    while (rem >= ti) {
-      rem -= ti;
-      ++ti;
-    }
-    const int64_t I = ti * 4 + (b % 16) / 4, J = rem * 4 + (b % 4);  // destination 64-block
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int lr = tr + 32 * h;
-      const int64_t i = J * 64 + lr, j = I * 64 + tc;  // source: rows of block (J, I)
-      if (i < r && j < r) {
-        float v[8];
-        load8v(a + i * r + j, v);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) tile[lr][tc + k] = v[k];
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int lc = tr + 32 * h;
-      const int64_t i = I * 64 + lc, j = J * 64 + tc;  // destination row i, columns j..j+7
-      if (i < r && j < r) {
-        float v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = tile[tc + k][lc];
-        store8v(a + i * r + j, v);
-      }
-    }
-    __syncthreads();
   }
 }
 
@@ -335,7 +190,6 @@ MuonLayout muon_layout(int64_t N, int64_t K) {
   L.Xt = off;    off += a256(2 * r * c);
   L.Xt2 = off;   off += a256(2 * r * c);
   L.A = off;     off += a256(2 * r * r);
-  L.A2 = off;    off += a256(4 * r * r);
   L.Bm = off;    off += a256(2 * r * r);
   L.total = off;
   return L;
@@ -350,7 +204,6 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
   auto* X = reinterpret_cast<__nv_bfloat16*>(w + L.X);
   auto* Xt = reinterpret_cast<__nv_bfloat16*>(w + L.Xt);
   auto* A = reinterpret_cast<__nv_bfloat16*>(w + L.A);
-  auto* A2 = reinterpret_cast<float*>(w + L.A2);
   auto* Bm = reinterpret_cast<__nv_bfloat16*>(w + L.Bm);
   __nv_bfloat16* xt_in = Xt;  // X^T as the B X product reads it
   __nv_bfloat16* xt_out = reinterpret_cast<__nv_bfloat16*>(w + L.Xt2);
@@ -364,33 +217,24 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
   count_launches(2);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   for (int it = 0; it < steps; ++it) {
-    // A = X X^T and A A are symmetric: the GEMM computes the upper tiles and
-    // the lower ones are copied from them (exactly symmetric results).
-    const int64_t nt = (r + 255) / 256;
-    const int mgrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(
-        nt * (nt - 1) / 2 * 16, static_cast<int64_t>(device_info().sms) * 8)));
+    // A = X X^T and B = b A + c (A A) are symmetric: the GEMM computes their
+    // upper 256 x 256 tiles and its epilogue also writes each strictly upper
+    // tile transposed into the lower one (exactly symmetric results); B is
+    // formed in the A A product's epilogue from A and the float32
+    // accumulator.
     GemmEpilogue ep;
     ep.out = A;
     ep.out_bf16 = 1;
     ep.ldo = r;
+    ep.ns_mirror = 1;
     bool upper = true;
     if ((e = launch_gemm_bf16(X, c, X, c, r, r, c, ep, status, s, &upper)) != cudaSuccess) return e;  // A = X X^T
-    if (upper) {
-      ns_mirror_kernel<<<mgrid, 256, 0, s>>>(A, r);
-      count_launches(1);
-    }
-    ep.out = A2;
-    ep.out_bf16 = 0;
+    ep.out = Bm;
+    ep.ns_x = A;
+    ep.ns_a = kNsB;
+    ep.ns_c = kNsC;
     upper = true;
-    if ((e = launch_gemm_bf16(A, r, A, r, r, r, r, ep, status, s, &upper)) != cudaSuccess) return e;  // A A
-    if (upper) {  // Bm from A and the upper tiles of A2, mirrored as it is written
-      ns_combine_sym_kernel<<<static_cast<int>(std::min<int64_t>(nt * (nt + 1) / 2 * 16,
-                                                                  static_cast<int64_t>(device_info().sms) * 8)),
-                              256, 0, s>>>(A, A2, r, Bm);
-    } else {
-      ns_combine_kernel<<<grid_for(r * r / 8, 8), 256, 0, s>>>(A, A2, r * r, Bm);
-    }
-    count_launches(1);
+    if ((e = launch_gemm_bf16(A, r, A, r, r, r, r, ep, status, s, &upper)) != cudaSuccess) return e;  // b A + c A A
     // X' = a X + B X in the product's epilogue: X' over X (in place: each
     // element is read and written by the same thread, and X is not an
     // operand of this product) and X'^T into the other X^T buffer (the one
@@ -403,12 +247,13 @@ cudaError_t launch_muon_orthogonalize(const float* grad, float* mom, int64_t N, 
       else xo = reinterpret_cast<__nv_bfloat16*>(O);
     }
     ep.out = xo;
-    ep.out_bf16 = 1;
     ep.ldo = c;
+    ep.ns_mirror = 0;
     ep.ns_x = X;
     ep.ns_xt = xto;
     ep.ns_ldt = r;
     ep.ns_a = kNsA;
+    ep.ns_c = 1.0f;
     if ((e = launch_gemm_bf16(Bm, r, xt_in, r, r, c, r, ep, status, s)) != cudaSuccess) return e;  // B X
     std::swap(xt_in, xt_out);
   }
