@@ -767,25 +767,42 @@ __global__ void __launch_bounds__(kRingThreads, 1) update_sr_ring_kernel(
 // The Muon step of an int8 weight from its orthogonalized update O (bf16
 // [N, K]): w = s*q; w' = (w*a) - st*O, one rounding per operation; then the
 // row max and the Philox-keyed stochastic rounding of the other updates.  One
-// CTA per row, 4-element chunks dealt round-robin (codes 4 bytes, O 8 bytes
-// per chunk), the updated row parked in shared memory (4 K bytes).
+// CTA per row stages the row's codes and O by two bulk copies on one mbarrier
+// (3 bytes per element, so every load of the row is in flight at once),
+// 4-element chunks dealt round-robin, the updated row parked in shared
+// memory (4 K bytes).
 __global__ void __launch_bounds__(512) update_sr_dir_kernel(
     int8_t* __restrict__ wq, float* __restrict__ sw, const __nv_bfloat16* __restrict__ O, int K,
     float a, float st, PhiloxKeys keys, uint32_t step_lo, uint32_t step_hi,
     int32_t* __restrict__ status) {
-  extern __shared__ float4 s_w[];
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t s_max[16];
+  __shared__ __align__(8) uint64_t s_full;
+  __shared__ volatile int s_abort;
   const int n = blockIdx.x, t = threadIdx.x, T = blockDim.x;
   const int warp = t >> 5, lane = t & 31, nwarps = T >> 5;
   const int nch = K >> 2;
   const int64_t row = static_cast<int64_t>(n) * K;
+  const uint32_t qbytes = static_cast<uint32_t>(K), obytes = 2u * static_cast<uint32_t>(K);
+  float4* s_w = reinterpret_cast<float4*>(smem);  // the updated row (4 K bytes)
+  const uint32_t bar = smem_u32(&s_full);
+  if (t == 0) {
+    mbar_init(bar, 1);
+    s_abort = 0;
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, qbytes + obytes);
+    bulk_load(smem_u32(smem) + 4u * K, wq + row, qbytes, bar);
+    bulk_load(smem_u32(smem) + 5u * K, O + row, obytes, bar);
+  }
   const float s = sw[n];
-  const uint32_t* q_in = reinterpret_cast<const uint32_t*>(wq + row);
-  const uint2* o_in = reinterpret_cast<const uint2*>(O + row);
+  __syncthreads();  // barrier initialised before anyone waits on it
+  const bool ok = mbar_wait(bar, 0, &s_abort);
+  const uint32_t* q_in = reinterpret_cast<const uint32_t*>(smem + 4 * K);
+  const uint2* o_in = reinterpret_cast<const uint2*>(smem + 5 * K);
   uint32_t mbits = 0;
-  for (int ch = t; ch < nch; ch += T) {
-    const uint32_t q4 = __ldcs(q_in + ch);
-    const uint2 o2 = __ldcs(o_in + ch);
+  for (int ch = t; ok && ch < nch; ch += T) {
+    const uint32_t q4 = q_in[ch];
+    const uint2 o2 = o_in[ch];
     const float o[4] = {__uint_as_float(o2.x << 16), __uint_as_float(o2.x & 0xFFFF0000u),
                         __uint_as_float(o2.y << 16), __uint_as_float(o2.y & 0xFFFF0000u)};
     float w[4];
@@ -799,6 +816,13 @@ __global__ void __launch_bounds__(512) update_sr_dir_kernel(
   mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
   if (lane == 0) s_max[warp] = mbits;
   __syncthreads();
+  if (s_abort) {
+    if (t == 0) {  // timed out: wait (bounded) for the copies before the CTA exits
+      atomicOr(status, 1 << QL_ERR_TIMEOUT);
+      mbar_wait_drain(bar, 0);
+    }
+    return;
+  }
   mbits = 0;
   for (int k = 0; k < nwarps; ++k) mbits = max(mbits, s_max[k]);
   const float amax = __uint_as_float(mbits);
@@ -961,12 +985,13 @@ cudaError_t launch_update_dir(int8_t* wq, float* sw, const void* O, int64_t N, i
   cudaGetDevice(&dev);
   if (dev < 64 && !__atomic_load_n(&dir_set[dev], __ATOMIC_ACQUIRE)) {
     cudaFuncSetAttribute(update_sr_dir_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         4 * 32768);
+                         7 * 32768);
     __atomic_store_n(&dir_set[dev], true, __ATOMIC_RELEASE);
   }
   const int nch = static_cast<int>(K / 4);
   const int tr = std::min(512, std::max(32, (nch / 4 + 31) / 32 * 32));
-  update_sr_dir_kernel<<<static_cast<unsigned>(N), tr, static_cast<size_t>(4) * K, s>>>(
+  // the updated row (4 bytes per element), then the staged codes (1) and O (2)
+  update_sr_dir_kernel<<<static_cast<unsigned>(N), tr, static_cast<size_t>(7) * K, s>>>(
       wq, sw, reinterpret_cast<const __nv_bfloat16*>(O), static_cast<int>(K), a, st, keys,
       static_cast<uint32_t>(step), static_cast<uint32_t>(step >> 32), status);
   count_launches(1);
