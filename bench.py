@@ -45,12 +45,12 @@ NOMINAL_INT8_TOPS = 4500.0     # B200 dense int8 spec, for context next to the m
 # DRAM bytes (read + write) per GEMM launch from an ncu capture of the
 # 12000-token layer step (mean of the forward, input-gradient and
 # weight-gradient launches), valid only for the GEMM source it was taken on.
-GEMM_TRAFFIC_BYTES = 336.4e6
-GEMM_TRAFFIC_SOURCE_SHA = "c7ab7c66c3ffc89c"
+GEMM_TRAFFIC_BYTES = 336.2e6
+GEMM_TRAFFIC_SOURCE_SHA = "99e20f7e2ee73977"
 # The same for the update kernel on the [7168, 5376] weight; DRAM writes
 # still held in L2 when the kernel ends are not counted.
-UPDATE_TRAFFIC_BYTES = 790.8e6
-UPDATE_TRAFFIC_SOURCE_SHA = "1868160c819b3e9c"
+UPDATE_TRAFFIC_BYTES = 790.6e6
+UPDATE_TRAFFIC_SOURCE_SHA = "bc45bf15ea5b9260"
 
 
 def source_sha(files=("gemm_i8.cu", "sm100.cuh")):
