@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(512, 1) update_sr_staged_kernel(
 // elementwise step (coalesced 16-byte loads issued U chunks ahead), which
 // keeps a row at 5 bytes of shared memory per element, so several rows share
 // an SM: U = 1 with four CTAs of up to 64 registers while four rows fit an
-// SM (K up to ~10.8K), U = 4 with three CTAs of 80 registers for longer
+// SM (K up to ~10.6K), U = 4 with three CTAs of 80 registers for longer
 // rows, where shared memory leaves fewer CTAs to hide the loads (512-thread
 // CTAs with U = 1 measured slower there).  Only the dg reduction
 // keeps 16-element groups: the first L threads (L a power of two <= 256) are
@@ -333,8 +333,9 @@ __global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) upd
     float* __restrict__ g_v, int L, int32_t* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float s_red[256];
-  __shared__ float s_amax[16];  // row maximum per warp (s_red may still be read)
+  __shared__ uint32_t s_amax[16];  // row maximum (bits) per warp (s_red may still be read)
   __shared__ float s_qhat[256];  // q / ||q|| for every byte value q = -128 .. 127
+  __shared__ float s_dgq[256];   // dg * (q / ||q||), the same table times dg
   __shared__ int s_ired[16];
   __shared__ float s_dg;
   __shared__ __align__(8) uint64_t s_full;  // codes + gradient
@@ -411,7 +412,14 @@ __global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) upd
       float gr[16];
       load16f(gf + 16 * j, gr);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) p = p + gr[e] * s_qhat[code_at(q4, e) + 128];
+      for (int e = 0; e < 16; e += 2) {
+        // products two at a time, added one at a time in increasing k
+        const float2 pr = mul2(make_float2(gr[e], gr[e + 1]),
+                               make_float2(s_qhat[code_at(q4, e) + 128],
+                                           s_qhat[code_at(q4, e + 1) + 128]));
+        p = __fadd_rn(p, pr.x);
+        p = __fadd_rn(p, pr.y);
+      }
     }
   }
   // The butterfly p += p[lane ^ off], off = 128 .. 1, over the 256 virtual
@@ -457,13 +465,15 @@ __global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) upd
     dg = s_dg;
   }
   const float coef = gmag_n / (s * nq);
+  // dg * qhat for every code value, once per row instead of once per element
+  for (int cidx = t; cidx < 256; cidx += T) s_dgq[cidx] = __fmul_rn(dg, s_qhat[cidx]);
+  __syncthreads();
 
   // Optimizer step of every element; moments written back as they are done,
   // the updated direction parked over the gradient.
   float4* m_out = reinterpret_cast<float4*>(mom1 + row);
   float4* v_out = reinterpret_cast<float4*>(mom2 + row);
-  float amax = 0.0f;
-  int bad = 0;
+  uint32_t mbits = 0;  // max |w'| as float bits (NaN above inf)
   auto update_chunk = [&](int ch, float (&m1)[4], float (&m2)[4]) {
     const uint32_t q4 = q_s[ch];
     const float4 g4 = g_s[ch];
@@ -471,8 +481,7 @@ __global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) upd
     float w[4], gg[4], wv[4], dd[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float qhat = s_qhat[static_cast<int>(static_cast<int8_t>(q4 >> (8 * e))) + 128];
-      dd[e] = __fsub_rn(gr[e], __fmul_rn(dg, qhat));
+      dd[e] = __fsub_rn(gr[e], s_dgq[static_cast<int>(static_cast<int8_t>(q4 >> (8 * e))) + 128]);
     }
     // coef * (g - dg * qhat) and s * q, two at a time (both are multiplied next)
     const float2 cc = make_float2(coef, coef);
@@ -487,10 +496,7 @@ __global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) upd
         w[e] = __fsub_rn(__fmul_rn(s, code_byte_f(q4, e)), __fmul_rn(c.lr, gg[e]));
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      bad |= !finite(w[e]);
-      amax = fmaxf(amax, fabsf(w[e]));
-    }
+    for (int e = 0; e < 4; ++e) mbits = max(mbits, abs_bits(w[e]));
     if (adam) {
       __stcs(m_out + ch, make_float4(m1[0], m1[1], m1[2], m1[3]));
       __stcs(v_out + ch, make_float4(m2[0], m2[1], m2[2], m2[3]));
@@ -547,23 +553,16 @@ __global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) upd
   }
 
   // Row max (also the barrier before the scale is overwritten).
-  amax = warp_max(amax);
-  bad = warp_or(bad);
-  if (lane == 0) {
-    s_amax[warp] = amax;
-    s_ired[warp] = bad;
-  }
+  mbits = __reduce_max_sync(0xFFFFFFFFu, mbits);
+  if (lane == 0) s_amax[warp] = mbits;
   __syncthreads();
-  amax = 0.0f;
-  bad = 0;
-  for (int k = 0; k < nwarps; ++k) {
-    amax = fmaxf(amax, s_amax[k]);
-    bad |= s_ired[k];
-  }
-  const float inv = amax == 0.0f ? 0.0f : 127.0f / amax;
+  mbits = 0;
+  for (int k = 0; k < nwarps; ++k) mbits = max(mbits, s_amax[k]);
+  const float amax = __uint_as_float(mbits);
+  const float inv = mbits == 0 ? 0.0f : 127.0f / amax;
   if (t == 0) {
-    sw[n] = amax == 0.0f ? 0.0f : amax / 127.0f;
-    if (bad) atomicOr(status, 1 << QL_ERR_NONFINITE);
+    sw[n] = mbits == 0 ? 0.0f : amax / 127.0f;
+    if (mbits >= kInfBits) atomicOr(status, 1 << QL_ERR_NONFINITE);
   }
   griddep_launch_dependents();
   // Element e = n*K + k uses word e&3 of Philox(counter = (e>>2 lo, e>>2 hi,
@@ -577,7 +576,7 @@ __global__ void __launch_bounds__(MS ? 384 : 256, MS ? 3 : (U == 1 ? 4 : 3)) upd
         keys);
     const float4 w = g_s[ch];
     uint32_t out = 0;
-    if (amax != 0.0f)
+    if (mbits != 0)
       out = sr_codes4(w, inv, rn);
     __stcs(q_out + ch, out);
   }
@@ -874,13 +873,13 @@ cudaError_t launch_update_sr(int8_t* wq, float* sw, const float* grad, int64_t N
     // are the pinned reduction's virtual lanes.
     const int nch = static_cast<int>(K / 4);
     const int64_t full_bytes = 13 * K;
-    // (an SM has 1 KB more shared memory than one CTA may take; 4 KB covers
+    // (an SM has 1 KB more shared memory than one CTA may take; 5 KB covers
     // the kernel's static arrays and the per-CTA reserve)
     const bool ms = c.kind == QL_ADAMW &&
-                    3 * (full_bytes + 4096) <= device_info().smem_optin + 1024;
+                    3 * (full_bytes + 5120) <= device_info().smem_optin + 1024;
     // Streamed moments: one chunk ahead while four rows fit an SM, four
     // chunks ahead otherwise.
-    const bool u1 = 4 * (5 * K + 4096) <= device_info().smem_optin + 1024;
+    const bool u1 = 4 * (5 * K + 5120) <= device_info().smem_optin + 1024;
     const int variant = ms ? 0 : (u1 ? 1 : 2);
     const int64_t row_bytes = ms ? full_bytes : 5 * K;
     static bool wn_set[3][64] = {{false}};

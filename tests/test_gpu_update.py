@@ -82,12 +82,12 @@ def test_adamw_update_bit_exact(N, K, warm):
 # Rows up to K = 16384 (AdamW) are staged whole, one row per CTA; longer
 # rows run the ring kernel: K = 18448 with two resident buffers, a 16-element
 # last moment piece and 160 rows (CTAs walk two rows), K = 32768 with one.
-# AdamW rows up to K = 5632 stage their moments too (352 threads there,
-# more than the 256 virtual lanes); K = 5760 is the first that does not.
-# Streamed moments are loaded one chunk ahead up to K = 10848, four chunks
-# ahead from K = 10864 on.
+# AdamW rows up to K = 5584 stage their moments too (352 threads there,
+# more than the 256 virtual lanes); K = 5600 is the first that does not.
+# Streamed moments are loaded one chunk ahead up to K = 10640, four chunks
+# ahead from K = 10656 on.
 @pytest.mark.parametrize("N,K", [(32, 1024), (12, 4096), (6, 16384), (20, 80), (160, 18448),
-                                 (4, 32768), (10, 5632), (10, 5760), (6, 10848), (6, 10864)])
+                                 (4, 32768), (10, 5584), (10, 5600), (6, 10640), (6, 10656)])
 def test_weight_norm_update_bit_exact(N, K, kind):
     d = workloads.update_state(N, K, seed=3 * K, weight_norm=True)
     q, s = prepared(d)
