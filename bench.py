@@ -50,7 +50,7 @@ GEMM_TRAFFIC_SOURCE_SHA = "99e20f7e2ee73977"
 # The same for the update kernel on the [7168, 5376] weight; DRAM writes
 # still held in L2 when the kernel ends are not counted.
 UPDATE_TRAFFIC_BYTES = 790.6e6
-UPDATE_TRAFFIC_SOURCE_SHA = "bc45bf15ea5b9260"
+UPDATE_TRAFFIC_SOURCE_SHA = "af301d8b5fe11a46"
 
 
 def source_sha(files=("gemm_i8.cu", "sm100.cuh")):
