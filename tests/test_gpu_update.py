@@ -79,9 +79,9 @@ def test_adamw_update_bit_exact(N, K, warm):
 
 
 @pytest.mark.parametrize("kind", [ql.QL_ADAMW, ql.QL_SGD])
-# Rows up to K = 16384 (AdamW) are staged whole, one row per CTA; longer
-# rows run the ring kernel: K = 18448 with two resident buffers, a 16-element
-# last moment piece and 160 rows (CTAs walk two rows), K = 32768 with one.
+# Weight-norm rows of every length stage their codes and gradient, one row
+# per CTA: K = 80 with fewer groups than lanes, K = 18448 and 32768 with
+# two and one rows per SM.
 # AdamW rows up to K = 5584 stage their moments too (352 threads there,
 # more than the 256 virtual lanes); K = 5600 is the first that does not.
 # Streamed moments are loaded one chunk ahead up to K = 10640, four chunks
@@ -101,9 +101,9 @@ def test_weight_norm_update_bit_exact(N, K, kind):
     check_equal(gpu, ref[:7], NAMES)
 
 
-# K = 512 and 6160: one staged row per CTA; 18448 (a 16-element last moment
-# piece) and 32768: the ring kernel, with more rows than CTAs so that the
-# rejected rows' moment pieces are drained between other rows
+# Zero directions among other rows, in each form of the weight-norm kernel:
+# K = 512 (moments staged), 6160 (one chunk of moments ahead), 18448 and
+# 32768 (four chunks ahead; two and one rows per SM)
 @pytest.mark.parametrize("N,K,zero", [(6, 512, [2]), (300, 6160, [0, 2, 149, 299]),
                                       (300, 18448, [0, 2, 149, 299]), (160, 32768, [3, 150])])
 def test_weight_norm_zero_direction_flagged_and_untouched(N, K, zero):
